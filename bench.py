@@ -1,0 +1,540 @@
+#!/usr/bin/env python
+"""Benchmark of the H3 transport hot path on B200: effective HBM GB/s.
+
+One step is one pass of the whole path on the ragged 32k-token workload
+(T = 32768 packed tokens, W = 6 virtual ranks, heads 10,10,9,9,9,9, 8 packed
+segments):
+
+  1. h3_partition            token/head ranges, segments clipped and rebased (host)
+  2. h3_seq_to_head          packed QKV [32768, 3, 56, 128] -> 6 x [32768, 3, H_j, 128]
+  3. h3_head_to_seq          back to [32768, 3, 56, 128], chunked one plane per
+                             launch under the 896,000,000-byte window
+  4. h3_ragged_reduce_scatter 6 BF16 partials [32768, 7168] + bias -> 6 x [T_r, 7168]
+
+value = algorithmic bytes of all steps (each input read once + each output
+written once) / device time, summed over GPUs.  Every kernel's inputs are
+1.4-2.8 GB, far larger than the 126 MB L2, so no flush is needed between
+steps.  With --gpus N (torchrun) every GPU runs an independent replica of the
+step: the path has no exchange between GPUs when all virtual ranks share one
+GPU's memory.
+
+--impl reference times the plain CPU oracle (oracle/) on the host cores on a
+bounded sample of the same workload; it is the slow reference, not a target.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import workloads as wl  # noqa: E402
+
+METRIC = "relayout + reduce-scatter effective HBM GB/s and % of B200 HBM peak"
+UNIT = "GB/s"
+FALLBACK_HBM_GBS = 6650.0
+STEP_T, STEP_W, STEP_P, STEP_SEGS, STEP_SEED = 32768, 6, 3, 8, 2
+WINDOW = 896_000_000
+
+
+# ---------------------------------------------------------------------------
+# host-side helpers (no GPU needed; covered by the gloo tests)
+# ---------------------------------------------------------------------------
+
+def dist_env():
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return rank, world, local
+
+
+def max_over_ranks(x: float, device) -> float:
+    """Largest value of x over all ranks (x itself without a process group)."""
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return float(x)
+    t = torch.tensor([float(x)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def sum_over_ranks(x: float, device) -> float:
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return float(x)
+    t = torch.tensor([float(x)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.SUM)
+    return float(t.item())
+
+
+def throughput_gbs(bytes_per_step_per_gpu: float, steps: int, n_gpus: int, seconds: float) -> float:
+    """Whole-job GB/s: every GPU's bytes over the slowest GPU's time."""
+    return bytes_per_step_per_gpu * steps * n_gpus / seconds / 1e9
+
+
+def load_peak():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            v = float(json.load(f)["hbm_gbs"])
+        return v, "measured"
+    except (OSError, KeyError, ValueError):
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+def kernel_source_digest() -> str:
+    h = hashlib.sha256()
+    for name in ("relayout.cu", "reduce_scatter.cu"):
+        with open(os.path.join(ROOT, "ragged_reduce_b200", "csrc", name), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def load_traffic(kernel: str):
+    """DRAM bytes per launch from the committed ncu summary, or None when the
+    kernels changed since it was taken."""
+    try:
+        with open(os.path.join(ROOT, "profiles", "dram_traffic.json")) as f:
+            table = json.load(f)
+    except (OSError, ValueError):
+        return None
+    entry = table.get(kernel)
+    if not entry or entry.get("source_digest") != kernel_source_digest():
+        return None
+    return entry.get("bytes_per_launch")
+
+
+class ClockSampler:
+    """nvidia-smi clock / throttle samples while the timed region runs."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_id: str | None):
+        self.gpu_id = gpu_id
+        self.proc = None
+        self.lines: list[str] = []
+
+    def __enter__(self):
+        cmd = ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+               "-lms", "100"]
+        if self.gpu_id:
+            cmd += ["-i", self.gpu_id]
+        try:
+            self.proc = subprocess.Popen(cmd, stdout=subprocess.PIPE, stderr=subprocess.DEVNULL,
+                                         text=True)
+        except OSError:
+            self.proc = None
+        time.sleep(0.3)
+        return self
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            time.sleep(0.15)
+            self.proc.terminate()
+            try:
+                out, _ = self.proc.communicate(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+                out, _ = self.proc.communicate()
+            self.lines = [ln for ln in out.splitlines() if ln.strip()]
+        return False
+
+    def summary(self) -> dict:
+        sm, mx, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            parts = [p.strip() for p in ln.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                mx.append(float(parts[2]))
+            except ValueError:
+                continue
+            for name, val in zip(names, parts[5:9]):
+                if val.lower() == "active":
+                    reasons.add(name)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(mx),
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ---------------------------------------------------------------------------
+# the step on the GPU
+# ---------------------------------------------------------------------------
+
+class Step:
+    """Device buffers and calls of one step of the path (inputs resident)."""
+
+    def __init__(self, device, T=STEP_T, W=STEP_W, P=STEP_P, n_segs=STEP_SEGS, seed=STEP_SEED,
+                 relayout=True, reduce=True):
+        import ragged_reduce_b200 as rr
+        self.rr = rr
+        self.device = device
+        self.T, self.W, self.P, self.H, self.D = T, W, P, wl.H3_HEADS, wl.H3_HEAD_DIM
+        self.C = wl.H3_HIDDEN
+        self.bounds = wl.segment_bounds(T, n_segs, seed)
+        self.part = rr.partition(T, self.H, W, self.bounds)
+        if relayout:
+            self.qkv = wl.normal_bf16((T, P, self.H, self.D), seed, 1.0, device)
+            self.send = rr.split_rows(self.qkv, self.part.token_starts)
+            self.heads = rr.alloc_head_side(T, P, self.H, self.D, W, device)
+            self.back_full, self.back = rr.alloc_seq_side(T, P, self.H, self.D, W, device)
+        if reduce:
+            rw = wl.ReduceWorkload("step", T=T, C=self.C, W=W, seed=seed + 100)
+            self.partials, self.bias = wl.partials_and_bias(rw, device)
+            self.partial_list = list(self.partials.unbind(0))
+            self.red_full, self.red_out = rr.alloc_reduce_outputs(T, self.C, W, device)
+        relayout_bytes = T * P * self.H * self.D * 2 * 2
+        reduce_bytes = (W + 1) * T * self.C * 2 + self.C * 2
+        self.kernel_bytes = {"seq_to_head": relayout_bytes, "head_to_seq": relayout_bytes,
+                             "ragged_reduce_scatter": reduce_bytes}
+        self.bytes_per_step = sum(self.kernel_bytes.values())
+        self.launches = {}
+
+    def run(self, events=None, stream=None):
+        rr = self.rr
+        if events is not None:
+            events[0].record(stream)
+        rr.partition(self.T, self.H, self.W, self.bounds)
+        i1 = rr.seq_to_head(self.send, self.heads, stream=stream)
+        if events is not None:
+            events[1].record(stream)
+        i2 = rr.head_to_seq(self.heads, self.back, window_bytes=WINDOW, stream=stream)
+        if events is not None:
+            events[2].record(stream)
+        i3 = rr.ragged_reduce_scatter(self.partial_list, self.bias, self.red_out, stream=stream)
+        if events is not None:
+            events[3].record(stream)
+        self.launches = {"seq_to_head": i1["launches"], "head_to_seq": i2["launches"],
+                         "ragged_reduce_scatter": i3["launches"]}
+        return i1["launches"] + i2["launches"] + i3["launches"]
+
+    def verify(self) -> bool:
+        """Round trip and reduce spot check (not timed)."""
+        ok = torch.equal(self.back_full.view(torch.int16), self.qkv.view(torch.int16))
+        acc = self.partials[0].float()
+        for k in range(1, self.W):
+            acc += self.partials[k].float()
+        acc += self.bias.float()
+        ok = ok and torch.equal(self.red_full.view(torch.int16), acc.to(torch.bfloat16).view(torch.int16))
+        return bool(ok)
+
+    def host_io(self):
+        """Pinned host copies of the step's inputs and room for its results."""
+        return {
+            "qkv": self.qkv.cpu().pin_memory(),
+            "partials": self.partials.cpu().pin_memory(),
+            "bias": self.bias.cpu().pin_memory(),
+            "back": torch.empty(self.back_full.shape, dtype=torch.bfloat16).pin_memory(),
+            "red": torch.empty(self.red_full.shape, dtype=torch.bfloat16).pin_memory(),
+        }
+
+    def run_e2e(self, io, stream):
+        self.qkv.copy_(io["qkv"], non_blocking=True)
+        self.partials.copy_(io["partials"], non_blocking=True)
+        self.bias.copy_(io["bias"], non_blocking=True)
+        n = self.run(stream=stream)
+        io["back"].copy_(self.back_full, non_blocking=True)
+        io["red"].copy_(self.red_full, non_blocking=True)
+        return n
+
+    @staticmethod
+    def io_bytes(io):
+        h2d = sum(io[k].numel() * 2 for k in ("qkv", "partials", "bias"))
+        d2h = sum(io[k].numel() * 2 for k in ("back", "red"))
+        return h2d, d2h
+
+
+def gpu_uuid(device) -> str | None:
+    try:
+        u = str(torch.cuda.get_device_properties(device).uuid)
+        return u if u.startswith("GPU-") else "GPU-" + u
+    except Exception:
+        return None
+
+
+def barrier(local):
+    import torch.distributed as dist
+    if dist.is_available() and dist.is_initialized():
+        dist.barrier(device_ids=[local])
+    torch.cuda.synchronize()
+
+
+def run_gpu(args):
+    import torch.distributed as dist
+    rank, world, local = dist_env()
+    if args.gpus != world:
+        raise SystemExit(f"--gpus {args.gpus} but WORLD_SIZE={world}")
+    torch.cuda.set_device(local)
+    device = torch.device("cuda", local)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+                                device_id=device)
+    step = Step(device)
+    stream = torch.cuda.current_stream(device)
+
+    # warm-up (untimed) and a correctness check of the buffers the bench times
+    for _ in range(args.warmup):
+        step.run(stream=stream)
+    torch.cuda.synchronize()
+    if not step.verify():
+        raise SystemExit("bench step produced wrong results")
+
+    K = args.steps
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(K)]
+    start = torch.cuda.Event(enable_timing=True)
+    end = torch.cuda.Event(enable_timing=True)
+    launches = 0
+    with ClockSampler(gpu_uuid(device)) as clocks:
+        barrier(local)
+        start.record(stream)
+        for k in range(K):
+            launches += step.run(events=evs[k], stream=stream)
+        end.record(stream)
+        barrier(local)
+    elapsed = start.elapsed_time(end) / 1e3
+    per_kernel_s = {"seq_to_head": 0.0, "head_to_seq": 0.0, "ragged_reduce_scatter": 0.0}
+    for e in evs:
+        per_kernel_s["seq_to_head"] += e[0].elapsed_time(e[1]) / 1e3
+        per_kernel_s["head_to_seq"] += e[1].elapsed_time(e[2]) / 1e3
+        per_kernel_s["ragged_reduce_scatter"] += e[2].elapsed_time(e[3]) / 1e3
+    t_max = max_over_ranks(elapsed, device)
+    launches_total = int(sum_over_ranks(launches, device))
+    value = throughput_gbs(step.bytes_per_step, K, world, t_max)
+    peak, peak_kind = load_peak()
+
+    kernels = {}
+    for name, secs in per_kernel_s.items():
+        n_launch = step.launches[name] * K
+        per_launch_s = secs / n_launch
+        bytes_per_launch = step.kernel_bytes[name] / step.launches[name]
+        kernels[name] = {"gbs": round(bytes_per_launch / per_launch_s / 1e9, 1),
+                         "us_per_launch": round(per_launch_s * 1e6, 2),
+                         "launches_per_step": step.launches[name],
+                         "bytes_per_launch": int(bytes_per_launch),
+                         "share": round(secs / sum(per_kernel_s.values()), 3)}
+    dom = max(kernels, key=lambda k: kernels[k]["share"])
+    achieved = kernels[dom]["gbs"]
+    roofline = {"bound": "hbm", "kernel": dom, "achieved": achieved, "peak": peak,
+                "unit": "GB/s", "frac": round(achieved / peak, 4),
+                "peak_source": f"{peak_kind}: MEASURED_PEAKS.json hbm_gbs" if peak_kind == "measured"
+                else "fallback 6650 GB/s",
+                "traffic": load_traffic(dom), "algorithmic_bytes_per_launch": kernels[dom]["bytes_per_launch"]}
+
+    # end to end through the public API with pinned host buffers
+    e2e = None
+    if args.e2e_steps > 0:
+        io = step.host_io()
+        h2d, d2h = Step.io_bytes(io)
+        step.run_e2e(io, stream)
+        torch.cuda.synchronize()
+        barrier(local)
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(args.e2e_steps):
+            step.run_e2e(io, stream)
+        e1.record(stream)
+        barrier(local)
+        t_e2e = max_over_ranks(e0.elapsed_time(e1) / 1e3, device)
+        ok = torch.equal(io["back"].view(torch.int16), io["qkv"].view(torch.int16))
+        e2e = {"value": round(throughput_gbs(step.bytes_per_step, args.e2e_steps, world, t_e2e), 2),
+               "unit": UNIT, "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
+               "steps": args.e2e_steps, "ms_per_step": round(t_e2e / args.e2e_steps * 1e3, 3),
+               "round_trip_ok": bool(ok)}
+        del io
+
+    result = None
+    if rank == 0:
+        result = {
+            "metric": METRIC, "value": round(value, 1), "unit": UNIT, "n_gpus": world,
+            "steps": K, "warmup": args.warmup, "ms_per_step": round(t_max / K * 1e3, 4),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": "bf16", "data": "synthetic",
+            "config": {"workload": "h3_transport_step_T32768_W6", "tokens": STEP_T,
+                       "planes": STEP_P, "heads": wl.H3_HEADS, "head_dim": wl.H3_HEAD_DIM,
+                       "world": STEP_W, "segments": STEP_SEGS, "reduce_cols": wl.H3_HIDDEN,
+                       "window_bytes": WINDOW, "parallelism": f"replicas x{world}",
+                       "l2": "no flush: every kernel's inputs (1.4-2.8 GB) exceed the 126 MB L2",
+                       "bytes_per_step": step.bytes_per_step},
+            "pct_of_peak": round(100.0 * value / world / peak, 2),
+            "roofline": roofline,
+            "kernels": kernels,
+            "gpu_launches": launches_total,
+            "clocks": clocks.summary(),
+            "e2e": e2e,
+            "library": os.path.relpath(step.rr.library_path, ROOT),
+        }
+    del step
+    torch.cuda.empty_cache()
+    if world > 1:
+        dist.barrier(device_ids=[local])
+        dist.destroy_process_group()
+    return result
+
+
+# ---------------------------------------------------------------------------
+# the oracle on the host cores
+# ---------------------------------------------------------------------------
+
+class OracleStep:
+    """The same step through the CPU oracle on a token sample of the workload."""
+
+    def __init__(self, tokens: int, W=STEP_W, P=STEP_P, seed=STEP_SEED):
+        import oracle
+        self.o = oracle.load()
+        self.T, self.W, self.P, self.H, self.D, self.C = tokens, W, P, wl.H3_HEADS, wl.H3_HEAD_DIM, wl.H3_HIDDEN
+        self.bounds = wl.segment_bounds(tokens, min(STEP_SEGS, tokens), seed)
+        full = wl.bf16_bits(wl.normal_bf16((tokens, P, self.H, self.D), seed))
+        ts = self.o.partition_range(tokens, W)
+        self.send = [full[ts[r]:ts[r + 1]] for r in range(W)]
+        rw = wl.ReduceWorkload("sample", T=tokens, C=self.C, W=W, seed=seed + 100)
+        partials, bias = wl.partials_and_bias(rw, "cpu")
+        self.partials = [wl.bf16_bits(p) for p in partials.unbind(0)]
+        self.bias = wl.bf16_bits(bias)
+        self.bytes = tokens * P * self.H * self.D * 2 * 2 * 2 + (W + 1) * tokens * self.C * 2 + self.C * 2
+
+    def run(self):
+        o = self.o
+        ts = o.partition_range(self.T, self.W)
+        for r in range(self.W):
+            o.clip_segments(self.bounds, int(ts[r]), int(ts[r + 1]))
+        heads = o.seq_to_head(self.send, self.T, self.P, self.H, self.D, self.W)
+        o.head_to_seq(heads, self.T, self.P, self.H, self.D, self.W)
+        o.ragged_reduce_scatter(self.partials, self.bias, self.W)
+
+
+def oracle_seconds_per_token() -> float:
+    s = OracleStep(256)
+    t0 = time.perf_counter()
+    s.run()
+    return (time.perf_counter() - t0) / 256
+
+
+def cpu_baseline(budget_s: float = 12.0) -> dict:
+    per_tok = oracle_seconds_per_token()
+    tokens = int(min(STEP_T, max(STEP_W, budget_s / 2 / per_tok)))
+    s = OracleStep(tokens)
+    times = []
+    for _ in range(2):
+        t0 = time.perf_counter()
+        s.run()
+        times.append(time.perf_counter() - t0)
+    t = min(times)
+    return {"value": round(s.bytes / t / 1e9, 3), "unit": UNIT, "cores": 1, "kind": "oracle",
+            "sample": f"the step on {tokens} of {STEP_T} tokens (W={STEP_W}, same shapes otherwise), "
+                      f"best of 2, {t:.2f} s each, single-threaded C oracle"}
+
+
+def run_reference(args):
+    rank, world, _ = dist_env()
+    if rank != 0:
+        return None
+    budget = float(args.reference_budget)  # seconds for warm-up + timed steps
+    per_tok = oracle_seconds_per_token()
+    per_step = budget / max(1, args.steps + args.warmup)
+    tokens = int(min(STEP_T, max(STEP_W, per_step / per_tok)))
+    s = OracleStep(tokens)
+    for _ in range(args.warmup):
+        s.run()
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        s.run()
+    t = time.perf_counter() - t0
+    value = s.bytes * args.steps / t / 1e9
+    sample = (f"each step: the path on {tokens} of {STEP_T} tokens (W={STEP_W}, same shapes "
+              f"otherwise), single-threaded C oracle")
+    return {
+        "impl": "reference", "metric": METRIC, "value": round(value, 3), "unit": UNIT,
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": round(t / args.steps * 1e3, 3), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": "h3_transport_step_T32768_W6", "tokens": STEP_T, "world": STEP_W,
+                   "sample_tokens": tokens},
+        "cpu_baseline": {"value": round(value, 3), "unit": UNIT, "cores": 1, "kind": "oracle",
+                         "sample": sample},
+        "e2e": {"value": round(value, 3), "unit": UNIT, "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+        "gpu_launches": 0,
+    }
+
+
+def run_profile(args):
+    """Run one kernel of the step --steps times (for ncu captures); no timing."""
+    torch.cuda.set_device(0)
+    device = torch.device("cuda", 0)
+    T = args.profile_tokens
+    relayout = args.profile in ("seq_to_head", "head_to_seq")
+    step = Step(device, T=T, relayout=relayout, reduce=not relayout)
+    rr = step.rr
+    if args.profile == "head_to_seq":
+        rr.seq_to_head(step.send, step.heads)
+    launches = 0
+    for _ in range(args.steps):
+        if args.profile == "seq_to_head":
+            launches += rr.seq_to_head(step.send, step.heads)["launches"]
+        elif args.profile == "head_to_seq":
+            launches += rr.head_to_seq(step.heads, step.back, window_bytes=WINDOW)["launches"]
+        else:
+            launches += rr.ragged_reduce_scatter(step.partial_list, step.bias, step.red_out)["launches"]
+    torch.cuda.synchronize()
+    print(json.dumps({"profile": args.profile, "tokens": T, "launches": launches}), flush=True)
+    return 0
+
+
+def parse_args(argv=None):
+    p = argparse.ArgumentParser(description=__doc__.split("\n")[0])
+    p.add_argument("--gpus", type=int, default=1)
+    p.add_argument("--steps", type=int, default=1000)
+    p.add_argument("--warmup", type=int, default=20)
+    p.add_argument("--impl", choices=["native", "reference"], default="native")
+    p.add_argument("--e2e-steps", type=int, default=5)
+    p.add_argument("--no-cpu-baseline", action="store_true")
+    p.add_argument("--profile", choices=["seq_to_head", "head_to_seq", "reduce_scatter"],
+                   help="run only this kernel of the step --steps times (ncu captures); no timing")
+    p.add_argument("--profile-tokens", type=int, default=STEP_T)
+    p.add_argument("--reference-budget", type=float, default=90.0,
+                   help="seconds of oracle work for --impl reference (warm-up + timed)")
+    return p.parse_args(argv)
+
+
+def main(argv=None):
+    args = parse_args(argv)
+    if args.profile:
+        return run_profile(args)
+    if args.warmup < 3:
+        raise SystemExit("--warmup must be at least 3")
+    if args.impl == "reference":
+        result = run_reference(args)
+        if result is not None:
+            print(json.dumps(result), flush=True)
+        return 0
+    result = run_gpu(args)
+    if result is not None:
+        rank, world, _ = dist_env()
+        if world == 1 and not args.no_cpu_baseline:
+            result["cpu_baseline"] = cpu_baseline()
+        else:
+            result["cpu_baseline"] = None
+        print(json.dumps(result), flush=True)
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

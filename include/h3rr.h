@@ -1,0 +1,219 @@
+/*
+ * h3rr.h - C ABI of the B200 (sm_100a) library for the data-parallel hot path
+ * of the distributed H3 denoiser: the Ulysses sequence->head relayout of
+ * packed BF16 QKV/QKVG, its inverse head->sequence relayout, and the
+ * tensor-mode ragged reduce-scatter.
+ *
+ * All W "virtual ranks" live in one GPU's memory: rank r's send and receive
+ * buffers are ordinary device buffers, and the library moves bytes between
+ * them with its own kernels.  No collective library is involved.
+ *
+ * Sources (page title, section):
+ *   "Distributed H3 Execution" (h3-blackwell-runtime DISTRIBUTED.md)
+ *      - intro: the "ulysses" mode's sequence-to-head all-to-all on QKV and
+ *        the inverse head-to-sequence all-to-all around attention; the packed
+ *        sequence is kept, empty token or head partitions are rejected, no
+ *        padding is added.
+ *      - "Partition Contract": 56 heads of width 128, balanced and possibly
+ *        ragged (table: W=6 -> 10,10,9,9,9,9); tokens split the same way;
+ *        segment boundaries clipped to each rank's interval and rebased;
+ *        tensor mode's ragged reduce-scatter sums the rank partials and
+ *        assigns token rows; the bias is added exactly once after reduction.
+ *   FastVideo PR #1807 "[perf] Harden Ulysses agreement and tune bounded H3
+ *        transfers", "Problem and behavior": one batch plane transferred at a
+ *        time under an 896,000,000-byte window; outputs keep storage of their
+ *        own.
+ *
+ * Conventions shared by every call
+ *   - Partition of n items over W ranks: q = n / W, m = n % W; rank i owns
+ *     q + (i < m) items starting at i*q + min(i, m).
+ *   - BF16 buffers are dense row-major arrays of 16-bit patterns.
+ *     Sequence side, rank r:  [T_r, P, H, D]  (tokens ts_r .. te_r-1, all heads)
+ *     Head side, rank j:      [T, P, H_j, D]  (all tokens, heads hs_j .. he_j-1)
+ *     Sequence-side buffers may be views into one [T, P, H, D] tensor at
+ *     token offsets ts_r; head-side buffers may be views into one tensor.
+ *   - Pointer arrays (send[], recv[], partials[], out[]) are HOST arrays of
+ *     `world` DEVICE pointers; they are read during the call only.  The
+ *     library allocates no device memory and keeps no pointer after return.
+ *   - The caller owns every buffer.  Outputs must not overlap any input or
+ *     any other output (outputs keep storage of their own); overlap is
+ *     detected and rejected.
+ *   - Every device pointer must be 16-byte aligned and every contiguous run
+ *     a multiple of 16 bytes (head_dim*2 % 16 == 0, cols % 8 == 0).
+ *   - `stream` is a cudaStream_t (NULL = the legacy default stream).  Work
+ *     is enqueued on it and the call returns without synchronising; results
+ *     are visible to later work on that stream.
+ *   - Arguments are checked before anything is launched; on any error
+ *     nothing is launched and the returned status says why.
+ *   - `info` (nullable) receives what actually ran: launches, chunks, grid,
+ *     block and kernel variant.
+ *   - Stateless and thread-safe: no environment variables are read and no
+ *     state outlives a call, apart from a per-device cache of the SM count.
+ */
+#ifndef H3RR_H
+#define H3RR_H
+
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#if defined(__GNUC__)
+#define H3RR_API __attribute__((visibility("default")))
+#else
+#define H3RR_API
+#endif
+
+#define H3RR_ABI_VERSION 1
+#define H3RR_MAX_WORLD 64
+
+typedef enum h3_status {
+    H3_OK = 0,
+    H3_ERR_INVALID_ARG = 1,      /* NULL pointer, negative size, overlapping outputs, bad segments */
+    H3_ERR_EMPTY_PARTITION = 2,  /* world > tokens or world > heads: some rank would own nothing */
+    H3_ERR_MISALIGNED = 3,       /* a pointer or a contiguous run is not 16-byte aligned */
+    H3_ERR_WINDOW = 4,           /* one plane of one rank does not fit in window_bytes */
+    H3_ERR_UNSUPPORTED = 5,      /* world > H3RR_MAX_WORLD, or a size beyond the kernels' index range */
+    H3_ERR_CUDA = 6              /* the CUDA runtime reported an error while launching */
+} h3_status;
+
+/* Kernel variants reported in h3_exec_info.variant. */
+#define H3_VARIANT_NONE 0
+#define H3_VARIANT_VECTOR 1      /* 16-byte vector loads/stores through registers */
+#define H3_VARIANT_BULK 2        /* bulk async copies through shared memory */
+#define H3_VARIANT_REDUCE 3      /* warp-level fp32 reduce-scatter */
+
+typedef struct h3_exec_info {
+    int32_t launches;            /* kernel launches enqueued by the call */
+    int32_t chunks;              /* plane chunks: 1 unchunked, P in chunked mode */
+    int32_t grid;                /* CTAs per launch */
+    int32_t block;               /* threads per CTA */
+    int32_t variant;             /* H3_VARIANT_* */
+    int32_t planes_per_launch;   /* planes moved by one launch */
+} h3_exec_info;
+
+/* Optional launch overrides for h3_*_ex; zero fields mean "library default". */
+typedef struct h3_launch_config {
+    int32_t variant;             /* 0 = default, H3_VARIANT_VECTOR or H3_VARIANT_BULK */
+    int32_t ctas_per_sm;         /* 0 = default (occupancy-derived) */
+    int32_t reserved0;
+    int32_t reserved1;
+} h3_launch_config;
+
+/* ABI version of the loaded library (H3RR_ABI_VERSION it was built with). */
+H3RR_API int32_t h3_abi_version(void);
+
+/* Short static English description of a status code. */
+H3RR_API const char* h3_status_string(h3_status status);
+
+/*
+ * h3_partition - the partition contract, host only ("Distributed H3
+ * Execution", "Partition Contract").
+ *
+ *   n_tokens, n_heads, world : T, H, W.  W >= 1; W <= T and W <= H, else
+ *                              H3_ERR_EMPTY_PARTITION.
+ *   seg_bounds  [n_segs+1]   : packed segment boundaries, 0 = b_0 < b_1 <
+ *                              ... < b_S = T (strictly increasing, else
+ *                              H3_ERR_INVALID_ARG).  May be NULL iff n_segs == 0,
+ *                              in which case the segment outputs below are
+ *                              not touched and may be NULL.
+ *   token_starts [world+1]   : out, ts_0 .. ts_W (int64).
+ *   head_starts  [world+1]   : out, hs_0 .. hs_W (int32).
+ *   piece_offsets [world+1]  : out.  Rank r's clipped pieces are
+ *                              k = piece_offsets[r] .. piece_offsets[r+1]-1.
+ *   local_seg_ids [n_segs+world-1] : out, global segment index of piece k.
+ *   local_bounds [n_segs+2*world-1] : out.  Rank r's rebased bounds are
+ *                              local_bounds[piece_offsets[r] + r ...
+ *                              piece_offsets[r+1] + r] (pieces + 1 values,
+ *                              first 0, last T_r).
+ * A segment whose intersection with [ts_r, te_r) is empty gives no piece.
+ * All arrays are caller-allocated host memory.
+ */
+H3RR_API h3_status h3_partition(int64_t n_tokens, int32_t n_heads, int32_t world,
+                       const int64_t* seg_bounds, int32_t n_segs,
+                       int64_t* token_starts, int32_t* head_starts,
+                       int64_t* local_bounds, int32_t* local_seg_ids,
+                       int32_t* piece_offsets);
+
+/*
+ * h3_seq_to_head - Ulysses sequence->head relayout ("Distributed H3
+ * Execution", intro: QKV sequence-to-head all-to-all).
+ *
+ *   send[world] : device, rank r's [T_r, P, H, D] BF16 (T_r tokens, all heads).
+ *   recv[world] : device, rank j's [T, P, H_j, D] BF16, written.
+ *   out_j[t, p, h, d] = send_{r(t)}[t - ts_{r(t)}, p, hs_j + h, d]   (bit copy)
+ *   n_tokens T, planes P (3 = QKV, 4 = QKVG, 1 = a single operand),
+ *   n_heads H, head_dim D, world W.
+ *   window_bytes : 0 = one launch over all planes.  > 0 = chunked mode (FastVideo
+ *                  PR #1807, "Problem and behavior"): one launch per plane p,
+ *                  and both the largest per-rank send slice of one plane
+ *                  (max_r T_r*H*D*2) and the largest per-rank receive slice
+ *                  (max_j T*H_j*D*2) must be <= window_bytes, else
+ *                  H3_ERR_WINDOW.  The result is identical either way.
+ */
+H3RR_API h3_status h3_seq_to_head(const void* const* send, void* const* recv,
+                         int64_t n_tokens, int32_t planes, int32_t n_heads,
+                         int32_t head_dim, int32_t world, int64_t window_bytes,
+                         void* stream, h3_exec_info* info);
+
+/*
+ * h3_head_to_seq - inverse head->sequence relayout ("Distributed H3
+ * Execution", intro: inverse head-to-sequence all-to-all around attention).
+ *
+ *   send[world] : device, rank j's [T, P, H_j, D] BF16.
+ *   recv[world] : device, rank r's [T_r, P, H, D] BF16, written.
+ *   out_r[t', p, hs_j + h, d] = send_j[ts_r + t', p, h, d]   (bit copy)
+ *   Other arguments as h3_seq_to_head (the window bounds the per-rank head-
+ *   side slice of one plane and the per-rank sequence-side slice).
+ */
+H3RR_API h3_status h3_head_to_seq(const void* const* send, void* const* recv,
+                         int64_t n_tokens, int32_t planes, int32_t n_heads,
+                         int32_t head_dim, int32_t world, int64_t window_bytes,
+                         void* stream, h3_exec_info* info);
+
+/*
+ * h3_ragged_reduce_scatter - tensor-mode ragged reduce-scatter ("Distributed
+ * H3 Execution", "Partition Contract": rank partials summed, token rows
+ * assigned, projection bias added exactly once after the reduction).
+ *
+ *   partials[world] : device, rank w's partial output [T, C] BF16 (no bias).
+ *   bias            : device [C] BF16, or NULL for no bias.
+ *   out[world]      : device, rank r's rows [T_r, C] BF16, written.
+ *   out_r[t', c] = bf16_rne( ((p_0 + p_1) + ... + p_{W-1}) + bias[c] ),
+ *     t = ts_r + t', every term widened exactly to binary32, the sum taken
+ *     in binary32 in rank order 0..W-1 starting from p_0, the bias added
+ *     once after the sum, rounded to BF16 to nearest, ties to even.  No
+ *     flush-to-zero; Inf and NaN propagate (a NaN result may be any NaN).
+ *   n_tokens T, cols C (C % 8 == 0), world W.
+ */
+H3RR_API h3_status h3_ragged_reduce_scatter(const void* const* partials, const void* bias,
+                                   void* const* out, int64_t n_tokens, int64_t cols,
+                                   int32_t world, void* stream, h3_exec_info* info);
+
+/*
+ * Same as h3_seq_to_head / h3_head_to_seq / h3_ragged_reduce_scatter with
+ * explicit launch overrides (cfg may be NULL).  Every variant computes the
+ * same bytes; the overrides exist for tuning and for testing each variant.
+ * An unknown variant returns H3_ERR_INVALID_ARG.
+ */
+H3RR_API h3_status h3_seq_to_head_ex(const void* const* send, void* const* recv,
+                            int64_t n_tokens, int32_t planes, int32_t n_heads,
+                            int32_t head_dim, int32_t world, int64_t window_bytes,
+                            void* stream, const h3_launch_config* cfg,
+                            h3_exec_info* info);
+H3RR_API h3_status h3_head_to_seq_ex(const void* const* send, void* const* recv,
+                            int64_t n_tokens, int32_t planes, int32_t n_heads,
+                            int32_t head_dim, int32_t world, int64_t window_bytes,
+                            void* stream, const h3_launch_config* cfg,
+                            h3_exec_info* info);
+H3RR_API h3_status h3_ragged_reduce_scatter_ex(const void* const* partials, const void* bias,
+                                      void* const* out, int64_t n_tokens, int64_t cols,
+                                      int32_t world, void* stream,
+                                      const h3_launch_config* cfg, h3_exec_info* info);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* H3RR_H */

@@ -1,0 +1,254 @@
+"""B200-native (sm_100a) H3 Ulysses relayouts and tensor-mode ragged reduce-scatter.
+
+Python binding of ``include/h3rr.h``: argument marshalling only.  Every byte
+the calls produce is computed by the library's own CUDA kernels; there is no
+CPU or PyTorch fallback, and importing this package fails if ``libh3rr.so``
+is missing.
+
+Terms ("Distributed H3 Execution", sections intro and "Partition Contract"):
+W virtual ranks; T packed tokens split by quotient/remainder into token ranges
+[ts_r, te_r); H heads (56 for H3) split the same way into head ranges
+[hs_j, he_j); P planes of a packed operand (3 for QKV, 4 for QKVG, 1 for the
+attention output); D = 128 values per head.
+
+* ``partition``                - host: token/head ranges and clipped, rebased segments
+* ``seq_to_head``              - sequence side [T_r, P, H, D] -> head side [T, P, H_j, D]
+* ``head_to_seq``              - head side -> sequence side
+* ``ragged_reduce_scatter``    - W partials [T, C] -> rank rows [T_r, C], bias once
+"""
+from __future__ import annotations
+
+import ctypes as C
+from dataclasses import dataclass
+
+import numpy as np
+import torch
+
+from . import _abi
+from ._abi import (ExecInfo, H3Error, LaunchConfig, H3_VARIANT_BULK, H3_VARIANT_REDUCE,
+                   H3_VARIANT_VECTOR, MAX_WORLD)
+
+__all__ = [
+    "H3Error", "Partition", "partition", "seq_to_head", "head_to_seq",
+    "ragged_reduce_scatter", "alloc_head_side", "alloc_seq_side", "split_rows",
+    "H3_VARIANT_VECTOR", "H3_VARIANT_BULK", "H3_VARIANT_REDUCE", "MAX_WORLD", "library_path",
+]
+
+library_path = _abi.LIB_PATH
+
+
+@dataclass
+class Partition:
+    """Result of ``partition``: ranges per rank and each rank's rebased segments."""
+
+    token_starts: np.ndarray          # int64 [W+1]
+    head_starts: np.ndarray           # int32 [W+1]
+    local_bounds: list                # per rank: int64 [pieces+1], 0 .. T_r
+    seg_ids: list                     # per rank: int32 [pieces], global segment index
+
+    @property
+    def world(self) -> int:
+        return len(self.token_starts) - 1
+
+    def tokens(self, r: int) -> int:
+        return int(self.token_starts[r + 1] - self.token_starts[r])
+
+    def heads(self, j: int) -> int:
+        return int(self.head_starts[j + 1] - self.head_starts[j])
+
+
+def partition(n_tokens: int, n_heads: int, world: int, seg_bounds=None) -> Partition:
+    """Token and head ranges of every rank, and the packed segments clipped to
+    each rank's token range and rebased to it (``h3_partition``)."""
+    W = int(world)
+    ts = np.zeros(max(W, 0) + 1, dtype=np.int64)
+    hs = np.zeros(max(W, 0) + 1, dtype=np.int32)
+    if seg_bounds is None:
+        st = _abi.lib.h3_partition(int(n_tokens), int(n_heads), W, None, 0,
+                                   ts.ctypes.data_as(_abi._i64p), hs.ctypes.data_as(_abi._i32p),
+                                   None, None, None)
+        _abi.check(st, "h3_partition")
+        return Partition(ts, hs, [], [])
+    b = np.ascontiguousarray(seg_bounds, dtype=np.int64)
+    S = len(b) - 1
+    if S < 1:
+        raise ValueError("seg_bounds needs at least two boundaries")
+    lb = np.zeros(S + 2 * W - 1, dtype=np.int64)
+    ids = np.zeros(S + W - 1, dtype=np.int32)
+    off = np.zeros(W + 1, dtype=np.int32)
+    st = _abi.lib.h3_partition(int(n_tokens), int(n_heads), W, b.ctypes.data_as(_abi._i64p), S,
+                               ts.ctypes.data_as(_abi._i64p), hs.ctypes.data_as(_abi._i32p),
+                               lb.ctypes.data_as(_abi._i64p), ids.ctypes.data_as(_abi._i32p),
+                               off.ctypes.data_as(_abi._i32p))
+    _abi.check(st, "h3_partition")
+    bounds = [lb[off[r] + r: off[r + 1] + r + 1].copy() for r in range(W)]
+    seg = [ids[off[r]: off[r + 1]].copy() for r in range(W)]
+    return Partition(ts, hs, bounds, seg)
+
+
+# ---------------------------------------------------------------------------
+# buffer helpers (allocation is the caller's; these use torch's allocator)
+# ---------------------------------------------------------------------------
+
+def split_rows(x: torch.Tensor, starts) -> list:
+    """Views of x's leading dimension at the given rank starts."""
+    return [x[int(starts[r]):int(starts[r + 1])] for r in range(len(starts) - 1)]
+
+
+def alloc_head_side(T: int, P: int, H: int, D: int, W: int, device, dtype=torch.bfloat16):
+    """One [T, P, H_j, D] buffer per head-side rank."""
+    part = partition(T, H, W)
+    return [torch.empty((T, P, part.heads(j), D), dtype=dtype, device=device) for j in range(W)]
+
+
+def alloc_seq_side(T: int, P: int, H: int, D: int, W: int, device, dtype=torch.bfloat16):
+    """One [T, P, H, D] tensor and its per-rank [T_r, P, H, D] views."""
+    part = partition(T, H, W)
+    full = torch.empty((T, P, H, D), dtype=dtype, device=device)
+    return full, split_rows(full, part.token_starts)
+
+
+# ---------------------------------------------------------------------------
+# marshalling
+# ---------------------------------------------------------------------------
+
+def _as_list(x):
+    if isinstance(x, torch.Tensor):
+        return list(x.unbind(0))
+    return list(x)
+
+
+def _check_tensors(ts, what: str, itemsize: int = 2):
+    dev = None
+    for t in ts:
+        if not isinstance(t, torch.Tensor):
+            raise TypeError(f"{what}: expected torch tensors")
+        if t.device.type != "cuda":
+            raise ValueError(f"{what}: tensors must be on a CUDA device (got {t.device})")
+        if t.element_size() != itemsize:
+            raise ValueError(f"{what}: expected {itemsize}-byte elements (got {t.dtype})")
+        if not t.is_contiguous():
+            raise ValueError(f"{what}: tensors must be contiguous")
+        if dev is None:
+            dev = t.device
+        elif t.device != dev:
+            raise ValueError(f"{what}: all tensors must be on one device")
+    return dev
+
+
+def _stream_handle(stream, device) -> int:
+    if stream is None:
+        stream = torch.cuda.current_stream(device)
+    return int(stream.cuda_stream) if hasattr(stream, "cuda_stream") else int(stream)
+
+
+def _config(variant: int, ctas_per_sm: int):
+    if not variant and not ctas_per_sm:
+        return None
+    return C.byref(LaunchConfig(int(variant), int(ctas_per_sm), 0, 0))
+
+
+def _relayout(seq_to_head_dir: bool, send, recv, window_bytes, stream, variant, ctas_per_sm):
+    send = _as_list(send)
+    recv = _as_list(recv)
+    W = len(send)
+    if W < 1 or len(recv) != W:
+        raise ValueError("send and recv need one tensor per rank (same count)")
+    dev = _check_tensors(send + recv, "relayout")
+    seq_side = send if seq_to_head_dir else recv
+    head_side = recv if seq_to_head_dir else send
+    if any(t.dim() != 4 for t in send + recv):
+        raise ValueError("relayout buffers are 4-D: [tokens, planes, heads, head_dim]")
+    _, P, H, D = seq_side[0].shape
+    T = sum(int(t.shape[0]) for t in seq_side)
+    part = partition(T, H, W)
+    for r, t in enumerate(seq_side):
+        if tuple(t.shape) != (part.tokens(r), P, H, D):
+            raise ValueError(f"sequence-side rank {r}: shape {tuple(t.shape)}, "
+                             f"expected {(part.tokens(r), P, H, D)}")
+    for j, t in enumerate(head_side):
+        if tuple(t.shape) != (T, P, part.heads(j), D):
+            raise ValueError(f"head-side rank {j}: shape {tuple(t.shape)}, "
+                             f"expected {(T, P, part.heads(j), D)}")
+    info = ExecInfo()
+    name = "h3_seq_to_head" if seq_to_head_dir else "h3_head_to_seq"
+    cfg = _config(variant, ctas_per_sm)
+    args = [_abi.pointer_array([t.data_ptr() for t in send]),
+            _abi.pointer_array([t.data_ptr() for t in recv]),
+            T, int(P), int(H), int(D), W, int(window_bytes),
+            C.c_void_p(_stream_handle(stream, dev))]
+    with torch.cuda.device(dev):
+        if cfg is None:
+            st = getattr(_abi.lib, name)(*args, C.byref(info))
+        else:
+            st = getattr(_abi.lib, name + "_ex")(*args, cfg, C.byref(info))
+    _abi.check(st, name)
+    return info.as_dict()
+
+
+def seq_to_head(send, recv, *, window_bytes: int = 0, stream=None, variant: int = 0,
+                ctas_per_sm: int = 0) -> dict:
+    """Ulysses sequence->head relayout.
+
+    send: W tensors [T_r, P, H, D] (or views of one [T, P, H, D] tensor, see
+    ``split_rows``); recv: W tensors [T, P, H_j, D], written.  window_bytes > 0
+    moves one plane per launch under that byte bound.  Returns what ran
+    (launches, chunks, grid, block, variant)."""
+    return _relayout(True, send, recv, window_bytes, stream, variant, ctas_per_sm)
+
+
+def head_to_seq(send, recv, *, window_bytes: int = 0, stream=None, variant: int = 0,
+                ctas_per_sm: int = 0) -> dict:
+    """Inverse head->sequence relayout: send W tensors [T, P, H_j, D] -> recv W
+    tensors [T_r, P, H, D]."""
+    return _relayout(False, send, recv, window_bytes, stream, variant, ctas_per_sm)
+
+
+def ragged_reduce_scatter(partials, bias, out, *, stream=None, ctas_per_sm: int = 0) -> dict:
+    """Tensor-mode ragged reduce-scatter.
+
+    partials: W BF16 tensors [T, C] (or one [W, T, C] tensor); bias: BF16 [C]
+    or None; out: W BF16 tensors [T_r, C], written with
+    bf16_rne(((p_0 + p_1) + ... + p_{W-1}) + bias) summed in binary32."""
+    partials = _as_list(partials)
+    out = _as_list(out)
+    W = len(partials)
+    if W < 1 or len(out) != W:
+        raise ValueError("partials and out need one tensor per rank (same count)")
+    tensors = partials + out + ([bias] if bias is not None else [])
+    dev = _check_tensors(tensors, "ragged_reduce_scatter")
+    if any(t.dtype != torch.bfloat16 for t in tensors):
+        raise ValueError("ragged_reduce_scatter works on BF16 tensors")
+    if any(t.dim() != 2 for t in partials + out):
+        raise ValueError("partials and outputs are 2-D: [tokens, cols]")
+    T, Cc = partials[0].shape
+    if any(tuple(p.shape) != (T, Cc) for p in partials):
+        raise ValueError("all partials must have the same [T, C] shape")
+    if bias is not None and tuple(bias.shape) != (Cc,):
+        raise ValueError(f"bias must be [C] = [{Cc}]")
+    part = partition(T, W, W) if T >= W else None
+    if part is not None:
+        for r, o in enumerate(out):
+            if tuple(o.shape) != (part.tokens(r), Cc):
+                raise ValueError(f"out rank {r}: shape {tuple(o.shape)}, expected "
+                                 f"{(part.tokens(r), Cc)}")
+    info = ExecInfo()
+    cfg = _config(0, ctas_per_sm)
+    args = [_abi.pointer_array([p.data_ptr() for p in partials]),
+            C.c_void_p(bias.data_ptr() if bias is not None else 0),
+            _abi.pointer_array([o.data_ptr() for o in out]),
+            int(T), int(Cc), W, C.c_void_p(_stream_handle(stream, dev))]
+    with torch.cuda.device(dev):
+        if cfg is None:
+            st = _abi.lib.h3_ragged_reduce_scatter(*args, C.byref(info))
+        else:
+            st = _abi.lib.h3_ragged_reduce_scatter_ex(*args, cfg, C.byref(info))
+    _abi.check(st, "h3_ragged_reduce_scatter")
+    return info.as_dict()
+
+
+def alloc_reduce_outputs(T: int, C_: int, W: int, device, dtype=torch.bfloat16):
+    """One [T, C] tensor and its per-rank [T_r, C] row views."""
+    part = partition(T, W, W)
+    full = torch.empty((T, C_), dtype=dtype, device=device)
+    return full, split_rows(full, part.token_starts)

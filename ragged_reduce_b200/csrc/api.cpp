@@ -1,0 +1,338 @@
+// C ABI entry points (include/h3rr.h): argument checks, the launch plan and
+// the kernel launches.  Every check runs before anything is enqueued; on an
+// error nothing is launched.
+#include <climits>
+#include <cstring>
+
+#include "h3rr_internal.h"
+
+using namespace h3rr;
+
+namespace {
+
+constexpr int64_t kMaxInt32 = INT32_MAX;
+// Column loops step by up to 1024 vectors past the row end; keep that in int32.
+constexpr int64_t kMaxRowVecs = int64_t(1) << 30;
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+void clear_info(h3_exec_info* info)
+{
+    if (info)
+        std::memset(info, 0, sizeof(*info));
+}
+
+// Partition checks shared by the relayouts and the reduce-scatter
+// ("Distributed H3 Execution", intro: empty token or head partitions are
+// rejected).
+h3_status check_world(int64_t n_tokens, int64_t n_heads, int32_t world)
+{
+    if (world < 1 || n_tokens < 0 || n_heads < 0)
+        return H3_ERR_INVALID_ARG;
+    if (world > kMaxWorld)
+        return H3_ERR_UNSUPPORTED;
+    if (n_tokens < world || n_heads < world)
+        return H3_ERR_EMPTY_PARTITION;
+    return H3_OK;
+}
+
+// Outputs may not overlap inputs or each other (FastVideo PR #1807, "Problem
+// and behavior": outputs keep storage of their own).
+h3_status check_no_overlap(const void* const* in, const uint64_t* in_bytes, int n_in,
+                           void* const* out, const uint64_t* out_bytes, int n_out)
+{
+    for (int i = 0; i < n_out; ++i) {
+        const uintptr_t o = reinterpret_cast<uintptr_t>(out[i]);
+        for (int k = 0; k < n_in; ++k)
+            if (ranges_overlap(o, out_bytes[i], reinterpret_cast<uintptr_t>(in[k]), in_bytes[k]))
+                return H3_ERR_INVALID_ARG;
+        for (int k = i + 1; k < n_out; ++k)
+            if (ranges_overlap(o, out_bytes[i], reinterpret_cast<uintptr_t>(out[k]), out_bytes[k]))
+                return H3_ERR_INVALID_ARG;
+    }
+    return H3_OK;
+}
+
+h3_status relayout(bool seq_to_head, const void* const* send, void* const* recv,
+                   int64_t n_tokens, int32_t planes, int32_t n_heads, int32_t head_dim,
+                   int32_t world, int64_t window_bytes, void* stream,
+                   const h3_launch_config* cfg, h3_exec_info* info)
+{
+    clear_info(info);
+    h3_status st = check_world(n_tokens, n_heads, world);
+    if (st != H3_OK)
+        return st;
+    if (planes < 1 || head_dim < 1 || window_bytes < 0 || !send || !recv)
+        return H3_ERR_INVALID_ARG;
+    if (cfg && cfg->variant != 0 && cfg->variant != H3_VARIANT_VECTOR)
+        return H3_ERR_INVALID_ARG;
+    if (cfg && cfg->ctas_per_sm < 0)
+        return H3_ERR_INVALID_ARG;
+    if ((int64_t(head_dim) * 2) % kVecBytes != 0)
+        return H3_ERR_MISALIGNED;
+    // Index ranges of the kernels: rows (token, plane) and row vectors in int32.
+    if (n_tokens > kMaxInt32 || n_tokens * planes > kMaxInt32 ||
+        int64_t(n_heads) * head_dim * 2 / kVecBytes > kMaxRowVecs)
+        return H3_ERR_UNSUPPORTED;
+
+    const Split ts = make_split(n_tokens, world);
+    const Split hs = make_split(n_heads, world);
+    const uint64_t row_bytes = uint64_t(n_heads) * head_dim * 2;  // one (token, plane) row
+    const uint64_t head_bytes = uint64_t(head_dim) * 2;
+
+    // Sequence-side and head-side byte sizes per rank.
+    uint64_t seq_bytes[kMaxWorld];
+    uint64_t head_side_bytes[kMaxWorld];
+    for (int r = 0; r < world; ++r) {
+        seq_bytes[r] = uint64_t(ts.size(r)) * planes * row_bytes;
+        head_side_bytes[r] = uint64_t(n_tokens) * planes * uint64_t(hs.size(r)) * head_bytes;
+    }
+    for (int r = 0; r < world; ++r) {
+        if (!send[r] || !recv[r])
+            return H3_ERR_INVALID_ARG;
+        if (!aligned16(send[r]) || !aligned16(recv[r]))
+            return H3_ERR_MISALIGNED;
+    }
+    const uint64_t* in_bytes = seq_to_head ? seq_bytes : head_side_bytes;
+    const uint64_t* out_bytes = seq_to_head ? head_side_bytes : seq_bytes;
+    st = check_no_overlap(send, in_bytes, world, recv, out_bytes, world);
+    if (st != H3_OK)
+        return st;
+
+    // Chunked mode (FastVideo PR #1807, "Problem and behavior"): one batch
+    // plane per launch; one plane's per-rank send and receive slices must
+    // both fit in the window.
+    const bool chunked = window_bytes > 0;
+    if (chunked) {
+        const uint64_t seq_plane = uint64_t(ts.largest()) * row_bytes;
+        const uint64_t head_plane = uint64_t(n_tokens) * uint64_t(hs.largest()) * head_bytes;
+        if (seq_plane > uint64_t(window_bytes) || head_plane > uint64_t(window_bytes))
+            return H3_ERR_WINDOW;
+    }
+
+    RelayoutArgs a;
+    std::memset(&a, 0, sizeof(a));
+    for (int r = 0; r < world; ++r) {
+        char* s = const_cast<char*>(static_cast<const char*>(send[r]));
+        char* d = static_cast<char*>(recv[r]);
+        a.seq[r] = seq_to_head ? s : d;
+        a.head[r] = seq_to_head ? d : s;
+    }
+    a.T = int32_t(n_tokens);
+    a.P = planes;
+    a.tq = int32_t(ts.q);
+    a.tm = int32_t(ts.m);
+    a.hq = int32_t(hs.q);
+    a.hm = int32_t(hs.m);
+    a.row_vecs = int32_t(row_bytes / kVecBytes);
+    a.head_vecs = int32_t(head_bytes / kVecBytes);
+
+    const int variant = cfg ? cfg->variant : 0;
+    const int ctas_per_sm = cfg ? cfg->ctas_per_sm : 0;
+    const int chunks = chunked ? planes : 1;
+    const int per_launch = chunked ? 1 : planes;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    LaunchShape shape;
+    int launched = 0;
+    for (int c = 0; c < chunks; ++c) {
+        a.plane0 = c * per_launch;
+        a.nplanes = per_launch;
+        a.rows = int32_t(n_tokens * per_launch);
+        const cudaError_t err = launch_relayout(seq_to_head, a, variant, ctas_per_sm, s, &shape);
+        if (err != cudaSuccess) {
+            cudaGetLastError();
+            if (info) {
+                info->launches = launched;
+                info->chunks = chunks;
+            }
+            return H3_ERR_CUDA;
+        }
+        ++launched;
+    }
+    if (info) {
+        info->launches = launched;
+        info->chunks = chunks;
+        info->grid = shape.grid;
+        info->block = shape.block;
+        info->variant = shape.variant;
+        info->planes_per_launch = per_launch;
+    }
+    return H3_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+int32_t h3_abi_version(void) { return H3RR_ABI_VERSION; }
+
+const char* h3_status_string(h3_status status)
+{
+    switch (status) {
+        case H3_OK: return "ok";
+        case H3_ERR_INVALID_ARG: return "invalid argument";
+        case H3_ERR_EMPTY_PARTITION: return "empty token or head partition";
+        case H3_ERR_MISALIGNED: return "pointer or run not 16-byte aligned";
+        case H3_ERR_WINDOW: return "one plane does not fit in the byte window";
+        case H3_ERR_UNSUPPORTED: return "unsupported size or world";
+        case H3_ERR_CUDA: return "CUDA launch error";
+    }
+    return "unknown status";
+}
+
+h3_status h3_partition(int64_t n_tokens, int32_t n_heads, int32_t world,
+                       const int64_t* seg_bounds, int32_t n_segs, int64_t* token_starts,
+                       int32_t* head_starts, int64_t* local_bounds, int32_t* local_seg_ids,
+                       int32_t* piece_offsets)
+{
+    h3_status st = check_world(n_tokens, n_heads, world);
+    if (st != H3_OK)
+        return st;
+    if (!token_starts || !head_starts || n_segs < 0)
+        return H3_ERR_INVALID_ARG;
+    if (n_segs > 0) {
+        if (!seg_bounds || !local_bounds || !local_seg_ids || !piece_offsets)
+            return H3_ERR_INVALID_ARG;
+        if (seg_bounds[0] != 0 || seg_bounds[n_segs] != n_tokens)
+            return H3_ERR_INVALID_ARG;
+        for (int32_t k = 0; k < n_segs; ++k)
+            if (seg_bounds[k + 1] <= seg_bounds[k])
+                return H3_ERR_INVALID_ARG;
+    }
+    const Split ts = make_split(n_tokens, world);
+    const Split hs = make_split(n_heads, world);
+    for (int32_t r = 0; r <= world; ++r) {
+        token_starts[r] = ts.start(r);
+        head_starts[r] = int32_t(hs.start(r));
+    }
+    if (n_segs == 0)
+        return H3_OK;
+    int32_t pieces = 0;
+    for (int32_t r = 0; r < world; ++r) {
+        piece_offsets[r] = pieces;
+        pieces += clip_segments(seg_bounds, n_segs, token_starts[r], token_starts[r + 1],
+                                local_bounds + pieces + r, local_seg_ids + pieces);
+    }
+    piece_offsets[world] = pieces;
+    return H3_OK;
+}
+
+h3_status h3_seq_to_head_ex(const void* const* send, void* const* recv, int64_t n_tokens,
+                            int32_t planes, int32_t n_heads, int32_t head_dim, int32_t world,
+                            int64_t window_bytes, void* stream, const h3_launch_config* cfg,
+                            h3_exec_info* info)
+{
+    return relayout(true, send, recv, n_tokens, planes, n_heads, head_dim, world, window_bytes,
+                    stream, cfg, info);
+}
+
+h3_status h3_head_to_seq_ex(const void* const* send, void* const* recv, int64_t n_tokens,
+                            int32_t planes, int32_t n_heads, int32_t head_dim, int32_t world,
+                            int64_t window_bytes, void* stream, const h3_launch_config* cfg,
+                            h3_exec_info* info)
+{
+    return relayout(false, send, recv, n_tokens, planes, n_heads, head_dim, world, window_bytes,
+                    stream, cfg, info);
+}
+
+h3_status h3_seq_to_head(const void* const* send, void* const* recv, int64_t n_tokens,
+                         int32_t planes, int32_t n_heads, int32_t head_dim, int32_t world,
+                         int64_t window_bytes, void* stream, h3_exec_info* info)
+{
+    return relayout(true, send, recv, n_tokens, planes, n_heads, head_dim, world, window_bytes,
+                    stream, nullptr, info);
+}
+
+h3_status h3_head_to_seq(const void* const* send, void* const* recv, int64_t n_tokens,
+                         int32_t planes, int32_t n_heads, int32_t head_dim, int32_t world,
+                         int64_t window_bytes, void* stream, h3_exec_info* info)
+{
+    return relayout(false, send, recv, n_tokens, planes, n_heads, head_dim, world, window_bytes,
+                    stream, nullptr, info);
+}
+
+h3_status h3_ragged_reduce_scatter_ex(const void* const* partials, const void* bias,
+                                      void* const* out, int64_t n_tokens, int64_t cols,
+                                      int32_t world, void* stream, const h3_launch_config* cfg,
+                                      h3_exec_info* info)
+{
+    clear_info(info);
+    h3_status st = check_world(n_tokens, world, world);
+    if (st != H3_OK)
+        return st;
+    if (cols < 1 || !partials || !out)
+        return H3_ERR_INVALID_ARG;
+    if (cfg && (cfg->variant != 0 && cfg->variant != H3_VARIANT_REDUCE))
+        return H3_ERR_INVALID_ARG;
+    if (cfg && cfg->ctas_per_sm < 0)
+        return H3_ERR_INVALID_ARG;
+    if (cols % 8 != 0)
+        return H3_ERR_MISALIGNED;
+    if (n_tokens > kMaxInt32 || cols / 8 > kMaxRowVecs)
+        return H3_ERR_UNSUPPORTED;
+    const Split ts = make_split(n_tokens, world);
+    const uint64_t row_bytes = uint64_t(cols) * 2;
+    uint64_t in_bytes[kMaxWorld + 1];
+    uint64_t out_bytes[kMaxWorld];
+    const void* inputs[kMaxWorld + 1];
+    for (int r = 0; r < world; ++r) {
+        if (!partials[r] || !out[r])
+            return H3_ERR_INVALID_ARG;
+        if (!aligned16(partials[r]) || !aligned16(out[r]))
+            return H3_ERR_MISALIGNED;
+        inputs[r] = partials[r];
+        in_bytes[r] = uint64_t(n_tokens) * row_bytes;
+        out_bytes[r] = uint64_t(ts.size(r)) * row_bytes;
+    }
+    int n_in = world;
+    if (bias) {
+        if (!aligned16(bias))
+            return H3_ERR_MISALIGNED;
+        inputs[n_in] = bias;
+        in_bytes[n_in] = row_bytes;
+        ++n_in;
+    }
+    st = check_no_overlap(inputs, in_bytes, n_in, out, out_bytes, world);
+    if (st != H3_OK)
+        return st;
+
+    ReduceArgs a;
+    std::memset(&a, 0, sizeof(a));
+    for (int r = 0; r < world; ++r) {
+        a.part[r] = static_cast<const char*>(partials[r]);
+        a.out[r] = static_cast<char*>(out[r]);
+    }
+    a.bias = static_cast<const char*>(bias);
+    a.T = int32_t(n_tokens);
+    a.W = world;
+    a.tq = int32_t(ts.q);
+    a.tm = int32_t(ts.m);
+    a.row_vecs = int32_t(cols / 8);
+    a.row_bytes = int64_t(row_bytes);
+    LaunchShape shape;
+    const cudaError_t err = launch_reduce_scatter(a, cfg ? cfg->ctas_per_sm : 0,
+                                                  static_cast<cudaStream_t>(stream), &shape);
+    if (err != cudaSuccess) {
+        cudaGetLastError();
+        return H3_ERR_CUDA;
+    }
+    if (info) {
+        info->launches = 1;
+        info->chunks = 1;
+        info->grid = shape.grid;
+        info->block = shape.block;
+        info->variant = shape.variant;
+        info->planes_per_launch = 1;
+    }
+    return H3_OK;
+}
+
+h3_status h3_ragged_reduce_scatter(const void* const* partials, const void* bias, void* const* out,
+                                   int64_t n_tokens, int64_t cols, int32_t world, void* stream,
+                                   h3_exec_info* info)
+{
+    return h3_ragged_reduce_scatter_ex(partials, bias, out, n_tokens, cols, world, stream, nullptr,
+                                       info);
+}
+
+}  // extern "C"

@@ -1,0 +1,91 @@
+// Internal declarations shared by the host plan, the kernels and the C ABI.
+#pragma once
+
+#include <cstdint>
+
+#include <cuda_runtime.h>
+
+#include "h3rr.h"
+
+namespace h3rr {
+
+constexpr int kMaxWorld = H3RR_MAX_WORLD;
+constexpr int kVecBytes = 16;  // one 16-byte vector = 8 BF16 values
+
+// ---------------------------------------------------------------------------
+// Quotient/remainder partition ("Distributed H3 Execution", "Partition
+// Contract"): n items over w ranks, q = n / w, m = n % w; rank i owns q + (i < m)
+// items starting at i*q + min(i, m).  Host side; the kernels carry (q, m).
+// ---------------------------------------------------------------------------
+struct Split {
+    int64_t q = 0;
+    int64_t m = 0;
+    int32_t w = 0;
+    int64_t start(int32_t i) const { return i * q + (i < m ? i : m); }
+    int64_t size(int32_t i) const { return q + (i < m ? 1 : 0); }
+    int64_t largest() const { return q + (m > 0 ? 1 : 0); }
+};
+
+Split make_split(int64_t n, int32_t w);
+
+// Clip packed segments to [ts, te) and rebase; returns the piece count.
+int32_t clip_segments(const int64_t* bounds, int32_t n_segs, int64_t ts, int64_t te,
+                      int64_t* local_bounds, int32_t* seg_ids);
+
+// [a, a+na) and [b, b+nb) share a byte.
+bool ranges_overlap(uintptr_t a, uint64_t na, uintptr_t b, uint64_t nb);
+
+// ---------------------------------------------------------------------------
+// Kernel arguments (passed by value as __grid_constant__ parameters).
+// ---------------------------------------------------------------------------
+
+// One relayout launch moves planes [plane0, plane0 + nplanes) of every token.
+// A "row" is one (token, plane) pair: row_vecs vectors on the sequence side,
+// split into W runs of H_j * head_vecs vectors on the head side.
+struct RelayoutArgs {
+    char* seq[kMaxWorld];    // sequence-side rank buffers [T_r, P, H, D]
+    char* head[kMaxWorld];   // head-side rank buffers [T, P, H_j, D]
+    int32_t T;
+    int32_t P;
+    int32_t plane0;
+    int32_t nplanes;
+    int32_t rows;            // T * nplanes
+    int32_t tq, tm;          // token split
+    int32_t hq, hm;          // head split
+    int32_t row_vecs;        // H * D * 2 / 16
+    int32_t head_vecs;       // D * 2 / 16
+};
+
+struct ReduceArgs {
+    const char* part[kMaxWorld];  // partials [T, C]
+    char* out[kMaxWorld];         // outputs [T_r, C]
+    const char* bias;             // [C] or nullptr
+    int32_t T;
+    int32_t W;
+    int32_t tq, tm;
+    int32_t row_vecs;             // C / 8
+    int64_t row_bytes;            // C * 2
+};
+
+struct LaunchShape {
+    int grid = 0;
+    int block = 0;
+    int variant = H3_VARIANT_NONE;
+};
+
+// Enqueue one relayout launch.  seq_to_head selects the direction.
+cudaError_t launch_relayout(bool seq_to_head, const RelayoutArgs& a, int variant,
+                            int ctas_per_sm, cudaStream_t stream, LaunchShape* shape);
+
+// Enqueue the reduce-scatter launch.
+cudaError_t launch_reduce_scatter(const ReduceArgs& a, int ctas_per_sm, cudaStream_t stream,
+                                  LaunchShape* shape);
+
+// SM count of the current device (cached per device).
+int current_sm_count(int* device);
+
+// Resident CTAs per SM of a kernel at the given block size and dynamic shared
+// memory (cached per kernel and device).
+int resident_ctas(const void* kernel, int block, size_t smem, int device);
+
+}  // namespace h3rr

@@ -1,0 +1,109 @@
+// Host-side partition plan: quotient/remainder splits, segment clipping,
+// overlap checks and the per-device launch caches.
+//
+// "Distributed H3 Execution", "Partition Contract": head ownership is
+// balanced and may be ragged (W=6 -> 10,10,9,9,9,9: the first ranks take the
+// remainder); token ranges use the same split; segment boundaries are clipped
+// to each rank's token interval and rebased before AdaLN modulation and
+// residual gating.
+#include <mutex>
+#include <unordered_map>
+
+#include "h3rr_internal.h"
+
+namespace h3rr {
+
+Split make_split(int64_t n, int32_t w)
+{
+    Split s;
+    s.w = w;
+    s.q = n / w;
+    s.m = n % w;
+    return s;
+}
+
+int32_t clip_segments(const int64_t* bounds, int32_t n_segs, int64_t ts, int64_t te,
+                      int64_t* local_bounds, int32_t* seg_ids)
+{
+    // Segments tile [0, T) in order, so the pieces inside [ts, te) are the
+    // segments from the one holding ts up to the one holding te-1.
+    int32_t pieces = 0;
+    for (int32_t k = 0; k < n_segs; ++k) {
+        const int64_t lo = bounds[k] < ts ? ts : bounds[k];
+        const int64_t hi = bounds[k + 1] > te ? te : bounds[k + 1];
+        if (hi <= lo)
+            continue;
+        local_bounds[pieces] = lo - ts;
+        seg_ids[pieces] = k;
+        ++pieces;
+    }
+    local_bounds[pieces] = te - ts;
+    return pieces;
+}
+
+bool ranges_overlap(uintptr_t a, uint64_t na, uintptr_t b, uint64_t nb)
+{
+    if (na == 0 || nb == 0)
+        return false;
+    return a < b + nb && b < a + na;
+}
+
+int current_sm_count(int* device)
+{
+    static std::mutex mu;
+    static std::unordered_map<int, int> cache;
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess)
+        return 0;
+    if (device)
+        *device = dev;
+    std::lock_guard<std::mutex> lock(mu);
+    auto it = cache.find(dev);
+    if (it != cache.end())
+        return it->second;
+    int n = 0;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+        return 0;
+    cache.emplace(dev, n);
+    return n;
+}
+
+int resident_ctas(const void* kernel, int block, size_t smem, int device)
+{
+    struct Key {
+        const void* k;
+        int block;
+        size_t smem;
+        int dev;
+        bool operator==(const Key& o) const
+        {
+            return k == o.k && block == o.block && smem == o.smem && dev == o.dev;
+        }
+    };
+    struct Hash {
+        size_t operator()(const Key& x) const
+        {
+            return std::hash<const void*>()(x.k) ^ (size_t(x.block) << 20) ^ (x.smem << 3) ^
+                   size_t(x.dev);
+        }
+    };
+    static std::mutex mu;
+    static std::unordered_map<Key, int, Hash> cache;
+    const Key key{kernel, block, smem, device};
+    {
+        std::lock_guard<std::mutex> lock(mu);
+        auto it = cache.find(key);
+        if (it != cache.end())
+            return it->second;
+    }
+    int n = 0;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, kernel, block, smem) != cudaSuccess)
+        n = 1;
+    if (n < 1)
+        n = 1;
+    std::lock_guard<std::mutex> lock(mu);
+    cache.emplace(key, n);
+    return n;
+}
+
+}  // namespace h3rr

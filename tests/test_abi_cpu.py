@@ -1,0 +1,245 @@
+"""The C-ABI library on the host: exports, the partition plan, argument checks.
+
+No compute call reaches a GPU here.  Tests that pass made-up device pointers
+run only when no CUDA device is visible, and each of them is built to fail a
+host-side check, so nothing is ever launched.
+"""
+import ctypes as C
+import re
+
+import numpy as np
+import pytest
+import torch
+
+import ragged_reduce_b200 as rr
+from ragged_reduce_b200 import _abi
+
+NO_GPU = not torch.cuda.is_available()
+
+
+def _declared_functions():
+    text = open(_abi.HEADER_PATH).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"H3RR_API\s+[\w\s\*]+?\b(h3_\w+)\s*\(", text)))
+
+
+def test_header_declares_the_four_calls():
+    names = _declared_functions()
+    for n in ("h3_partition", "h3_seq_to_head", "h3_head_to_seq", "h3_ragged_reduce_scatter"):
+        assert n in names
+    assert len(names) >= 9
+
+
+def test_library_exports_every_declared_symbol():
+    lib = C.CDLL(_abi.LIB_PATH)
+    missing = [n for n in _declared_functions() if not hasattr(lib, n)]
+    assert not missing, missing
+    assert _abi.lib.h3_abi_version() == _abi.ABI_VERSION
+
+
+def test_status_strings():
+    for code in range(7):
+        assert _abi.describe(code) != "unknown status"
+    assert _abi.describe(99) == "unknown status"
+
+
+# ---------------------------------------------------------------------------
+# the host plan against the oracle
+# ---------------------------------------------------------------------------
+
+def test_partition_head_table(oracle_lib):
+    for W, sizes in {2: [28] * 2, 4: [14] * 4, 6: [10, 10, 9, 9, 9, 9], 8: [7] * 8}.items():
+        p = rr.partition(1024, 56, W)
+        assert list(np.diff(p.head_starts)) == sizes
+        assert np.array_equal(p.head_starts, oracle_lib.partition_range(56, W))
+
+
+def test_partition_matches_oracle_random(oracle_lib):
+    rng = np.random.default_rng(21)
+    for _ in range(300):
+        T = int(rng.integers(1, 300_000))
+        W = int(rng.integers(1, 65))
+        H = int(rng.integers(W, 200))
+        if T < W:
+            continue
+        S = int(rng.integers(1, min(T, 40) + 1))
+        cuts = np.sort(rng.choice(np.arange(1, T), size=S - 1, replace=False)) if S > 1 else []
+        bounds = np.concatenate([[0], cuts, [T]]).astype(np.int64)
+        p = rr.partition(T, H, W, bounds)
+        assert np.array_equal(p.token_starts, oracle_lib.partition_range(T, W))
+        assert np.array_equal(p.head_starts.astype(np.int64), oracle_lib.partition_range(H, W))
+        for r in range(W):
+            lb, ids = oracle_lib.clip_segments(bounds, int(p.token_starts[r]),
+                                               int(p.token_starts[r + 1]))
+            assert np.array_equal(p.local_bounds[r], lb), (T, W, r)
+            assert np.array_equal(p.seg_ids[r], ids), (T, W, r)
+
+
+def test_partition_tiny_workload_worked_example():
+    p = rr.partition(1024, 56, 2, [0, 400, 737, 1024])
+    assert list(p.token_starts) == [0, 512, 1024]
+    assert [list(b) for b in p.local_bounds] == [[0, 400, 512], [0, 225, 512]]
+    assert [list(s) for s in p.seg_ids] == [[0, 1], [1, 2]]
+
+
+def test_partition_workload_token_starts():
+    # quotient/remainder token ranges of the full-size workloads
+    assert list(rr.partition(32768, 56, 6).token_starts) == [0, 5462, 10924, 16385, 21846, 27307, 32768]
+    assert list(rr.partition(131072, 56, 4).token_starts) == [0, 32768, 65536, 98304, 131072]
+    assert list(rr.partition(65536, 56, 8).token_starts) == list(range(0, 65537, 8192))
+    assert list(rr.partition(250000, 56, 4).token_starts) == [0, 62500, 125000, 187500, 250000]
+
+
+@pytest.mark.parametrize("T,H,W,status", [
+    (10, 56, 0, _abi.H3_ERR_INVALID_ARG),
+    (10, 56, -1, _abi.H3_ERR_INVALID_ARG),
+    (10, 5, 6, _abi.H3_ERR_EMPTY_PARTITION),
+    (5, 56, 6, _abi.H3_ERR_EMPTY_PARTITION),
+    (0, 56, 1, _abi.H3_ERR_EMPTY_PARTITION),
+    (1000, 100, 65, _abi.H3_ERR_UNSUPPORTED),
+])
+def test_partition_rejects(T, H, W, status):
+    with pytest.raises(rr.H3Error) as e:
+        rr.partition(T, H, W)
+    assert e.value.status == status
+
+
+@pytest.mark.parametrize("bounds", [[0, 5, 5, 10], [1, 5, 10], [0, 5, 9], [0, 7, 3, 10]])
+def test_partition_rejects_bad_segments(bounds):
+    with pytest.raises(rr.H3Error) as e:
+        rr.partition(10, 56, 2, bounds)
+    assert e.value.status == _abi.H3_ERR_INVALID_ARG
+
+
+# ---------------------------------------------------------------------------
+# argument checks of the device calls (host only; nothing may launch)
+# ---------------------------------------------------------------------------
+
+BASE = 1 << 40  # made-up, never dereferenced
+
+
+def _ptrs(addrs):
+    return _abi.pointer_array(addrs)
+
+
+def _relayout_status(send, recv, T, P, H, D, W, window=0, fn="h3_seq_to_head"):
+    info = _abi.ExecInfo()
+    st = getattr(_abi.lib, fn)(_ptrs(send), _ptrs(recv), T, P, H, D, W, window, None,
+                               C.byref(info))
+    return st, info
+
+
+def _layout(T, P, H, D, W):
+    """Disjoint made-up addresses for send (seq side) and recv (head side)."""
+    ts = np.array([r * (T // W) + min(r, T % W) for r in range(W + 1)])
+    hs = np.array([j * (H // W) + min(j, H % W) for j in range(W + 1)])
+    addr = BASE
+    send, recv = [], []
+    for r in range(W):
+        send.append(addr)
+        addr += int(ts[r + 1] - ts[r]) * P * H * D * 2 + 4096
+    for j in range(W):
+        recv.append(addr)
+        addr += T * P * int(hs[j + 1] - hs[j]) * D * 2 + 4096
+    return send, recv
+
+
+needs_no_gpu = pytest.mark.skipif(not NO_GPU, reason="made-up pointers are only passed with no GPU visible")
+
+
+@needs_no_gpu
+@pytest.mark.parametrize("fn", ["h3_seq_to_head", "h3_head_to_seq"])
+def test_relayout_argument_checks(fn):
+    T, P, H, D, W = 1000, 3, 56, 128, 6
+    send, recv = _layout(T, P, H, D, W)
+    if fn == "h3_head_to_seq":
+        send, recv = recv, send
+    E = _abi
+    assert _relayout_status(send, recv, T, P, H, D, 0, fn=fn)[0] == E.H3_ERR_INVALID_ARG
+    assert _relayout_status(send, recv, T, P, H, D, 65, fn=fn)[0] == E.H3_ERR_UNSUPPORTED
+    assert _relayout_status(send[:5] + [send[5]], recv, 5, P, H, D, 6, fn=fn)[0] == E.H3_ERR_EMPTY_PARTITION
+    assert _relayout_status(send, recv, T, P, 5, D, 6, fn=fn)[0] == E.H3_ERR_EMPTY_PARTITION
+    assert _relayout_status(send, recv, T, 0, H, D, W, fn=fn)[0] == E.H3_ERR_INVALID_ARG
+    assert _relayout_status(send, recv, T, P, H, 0, W, fn=fn)[0] == E.H3_ERR_INVALID_ARG
+    assert _relayout_status(send, recv, T, P, H, 100, W, fn=fn)[0] == E.H3_ERR_MISALIGNED
+    assert _relayout_status(send, recv, T, P, H, D, W, window=-1, fn=fn)[0] == E.H3_ERR_INVALID_ARG
+    bad = list(send)
+    bad[3] += 8
+    assert _relayout_status(bad, recv, T, P, H, D, W, fn=fn)[0] == E.H3_ERR_MISALIGNED
+    bad = list(recv)
+    bad[5] += 2
+    assert _relayout_status(send, bad, T, P, H, D, W, fn=fn)[0] == E.H3_ERR_MISALIGNED
+    bad = list(send)
+    bad[2] = 0
+    assert _relayout_status(bad, recv, T, P, H, D, W, fn=fn)[0] == E.H3_ERR_INVALID_ARG
+    # an output overlapping an input, and two outputs overlapping each other
+    bad = list(recv)
+    bad[1] = send[4] + 1024
+    assert _relayout_status(send, bad, T, P, H, D, W, fn=fn)[0] == E.H3_ERR_INVALID_ARG
+    bad = list(recv)
+    bad[2] = recv[1] + 512
+    assert _relayout_status(send, bad, T, P, H, D, W, fn=fn)[0] == E.H3_ERR_INVALID_ARG
+    # window smaller than one plane of one rank (largest slice: 167 tokens x 14,336 B)
+    assert _relayout_status(send, recv, T, P, H, D, W, window=167 * 14336 - 1, fn=fn)[0] == E.H3_ERR_WINDOW
+    # sizes beyond the kernels' 32-bit row index
+    assert _relayout_status(send, recv, 2**31, P, H, D, W, fn=fn)[0] == E.H3_ERR_UNSUPPORTED
+    # a NULL pointer array
+    info = _abi.ExecInfo()
+    assert getattr(_abi.lib, fn)(None, _ptrs(recv), T, P, H, D, W, 0, None, C.byref(info)) == E.H3_ERR_INVALID_ARG
+    assert info.launches == 0
+
+
+@needs_no_gpu
+def test_relayout_window_check_long_workload():
+    # 250k tokens over 4 ranks: one plane of one rank is exactly 896,000,000 bytes
+    T, P, H, D, W = 250000, 4, 56, 128, 4
+    send, recv = _layout(T, P, H, D, W)
+    assert 62500 * 56 * 128 * 2 == 896_000_000
+    assert 250000 * 14 * 128 * 2 == 896_000_000
+    st, info = _relayout_status(send, recv, T, P, H, D, W, window=896_000_000 - 16)
+    assert st == _abi.H3_ERR_WINDOW and info.launches == 0
+
+
+@needs_no_gpu
+def test_reduce_argument_checks():
+    T, Cc, W = 1000, 7168, 6
+    addr = BASE
+    parts, outs = [], []
+    for _ in range(W):
+        parts.append(addr)
+        addr += T * Cc * 2 + 4096
+    bias = addr
+    addr += Cc * 2 + 4096
+    for r in range(W):
+        outs.append(addr)
+        addr += (T // W + 1) * Cc * 2 + 4096
+
+    def st(parts=parts, bias=bias, outs=outs, T=T, Cc=Cc, W=W):
+        info = _abi.ExecInfo()
+        s = _abi.lib.h3_ragged_reduce_scatter(_ptrs(parts), C.c_void_p(bias), _ptrs(outs), T, Cc,
+                                              W, None, C.byref(info))
+        assert info.launches == 0
+        return s
+
+    E = _abi
+    assert st(W=0) == E.H3_ERR_INVALID_ARG
+    assert st(W=65) == E.H3_ERR_UNSUPPORTED
+    assert st(T=5) == E.H3_ERR_EMPTY_PARTITION
+    assert st(Cc=7164) == E.H3_ERR_MISALIGNED
+    assert st(Cc=0) == E.H3_ERR_INVALID_ARG
+    assert st(bias=bias + 2) == E.H3_ERR_MISALIGNED
+    assert st(parts=[p + (8 if i == 2 else 0) for i, p in enumerate(parts)]) == E.H3_ERR_MISALIGNED
+    assert st(outs=[0] + outs[1:]) == E.H3_ERR_INVALID_ARG
+    assert st(outs=[parts[3]] + outs[1:]) == E.H3_ERR_INVALID_ARG      # output over a partial
+    assert st(outs=[bias - 64] + outs[1:]) == E.H3_ERR_INVALID_ARG     # output over the bias
+    assert st(outs=[outs[0], outs[0] + 256] + outs[2:]) == E.H3_ERR_INVALID_ARG
+    assert st(T=2**31) == E.H3_ERR_UNSUPPORTED
+
+
+def test_binding_rejects_host_tensors():
+    x = torch.zeros(4, 3, 8, 8, dtype=torch.bfloat16)
+    with pytest.raises(ValueError):
+        rr.seq_to_head([x], [x.clone()])
+    with pytest.raises(ValueError):
+        rr.ragged_reduce_scatter([torch.zeros(4, 8, dtype=torch.bfloat16)], None,
+                                 [torch.zeros(4, 8, dtype=torch.bfloat16)])

@@ -1,0 +1,238 @@
+"""GPU parity of the Ulysses relayouts against the CPU oracle (bit-exact).
+
+Small shapes are compared element by element with the oracle's full loops;
+full-size workloads are compared on sampled elements through the oracle's
+gather map, plus properties that hold at any size (round trip, torch slicing).
+"""
+import numpy as np
+import pytest
+import torch
+
+import ragged_reduce_b200 as rr
+import workloads as wl
+from tests import gpu_util as gu
+
+pytestmark = pytest.mark.gpu
+
+DEV = "cuda"
+
+
+def _seq_inputs(T, P, H, D, W, seed, kind="bits"):
+    if kind == "bits":
+        full = wl.random_bits((T, P, H, D), seed, DEV)
+    else:
+        full = wl.normal_bf16((T, P, H, D), seed, 1.0, DEV)
+    part = rr.partition(T, H, W)
+    return full, rr.split_rows(full, part.token_starts), part
+
+
+# T, P, H, D, W: ragged tokens and heads, several CTAs' worth of rows, every
+# kernel template (1..8 vectors per thread, two-row and one-row), the generic
+# kernel (rows wider than 1024 vectors), narrow 16-byte heads, one head per
+# rank, one token per rank.
+SMALL = [
+    (1024, 3, 56, 128, 2),
+    (1000, 3, 56, 128, 6),
+    (777, 4, 56, 128, 8),
+    (513, 1, 56, 128, 4),
+    (100, 3, 56, 128, 1),
+    (64, 3, 56, 128, 56),
+    (9, 3, 56, 128, 9),
+    (130, 2, 7, 64, 3),
+    (50, 3, 5, 8, 5),
+    (301, 2, 16, 64, 5),
+    (40, 3, 24, 128, 7),
+    (20, 2, 300, 128, 7),
+    (33, 3, 56, 256, 4),
+    (7, 4, 56, 128, 7),
+]
+
+
+@pytest.mark.parametrize("T,P,H,D,W", SMALL)
+@pytest.mark.parametrize("window", [0, "plane"])
+def test_relayout_matches_oracle(oracle_lib, T, P, H, D, W, window):
+    full, send, part = _seq_inputs(T, P, H, D, W, seed=T * 31 + W)
+    if window == "plane":
+        window = max(part.tokens(0) * H * D * 2, T * part.heads(0) * D * 2)
+    recv = rr.alloc_head_side(T, P, H, D, W, DEV)
+    info = rr.seq_to_head(send, recv, window_bytes=window)
+    assert info["launches"] == (P if window else 1)
+    want = oracle_lib.seq_to_head([gu.bits(s) for s in send], T, P, H, D, W)
+    for j in range(W):
+        assert np.array_equal(gu.bits(recv[j]), want[j]), f"seq->head rank {j}"
+    back_full, back = rr.alloc_seq_side(T, P, H, D, W, DEV)
+    info = rr.head_to_seq(recv, back, window_bytes=window)
+    assert info["launches"] == (P if window else 1)
+    want_back = oracle_lib.head_to_seq(want, T, P, H, D, W)
+    for r in range(W):
+        assert np.array_equal(gu.bits(back[r]), want_back[r]), f"head->seq rank {r}"
+    assert gu.same_bits(back_full, full)  # round trip
+
+
+def test_world_one_identity():
+    T, P, H, D = 257, 3, 56, 128
+    full = wl.random_bits((T, P, H, D), 5, DEV)
+    (recv,) = rr.alloc_head_side(T, P, H, D, 1, DEV)
+    rr.seq_to_head([full], [recv])
+    assert gu.same_bits(recv, full)
+    back = torch.empty_like(full)
+    rr.head_to_seq([recv], [back])
+    assert gu.same_bits(back, full)
+
+
+def test_tiny_workload_round_trip(oracle_lib):
+    w = wl.TINY_QKV_W2
+    full = wl.packed_operand(w, device=DEV)
+    bounds = wl.segment_bounds(w.T, w.n_segs, w.seed, w.seg_lengths)
+    part = rr.partition(w.T, w.H, w.W, bounds)
+    assert [list(b) for b in part.local_bounds] == [[0, 400, 512], [0, 225, 512]]
+    send = rr.split_rows(full, part.token_starts)
+    recv = rr.alloc_head_side(w.T, w.P, w.H, w.D, w.W, DEV)
+    rr.seq_to_head(send, recv)
+    want = oracle_lib.seq_to_head([gu.bits(s) for s in send], w.T, w.P, w.H, w.D, w.W)
+    for j in range(w.W):
+        assert np.array_equal(gu.bits(recv[j]), want[j])
+    back_full, back = rr.alloc_seq_side(w.T, w.P, w.H, w.D, w.W, DEV)
+    rr.head_to_seq(recv, back)
+    assert gu.same_bits(back_full, full)
+
+
+def test_guard_bands_untouched():
+    T, P, H, D, W = 1000, 3, 56, 128, 6
+    full, send, part = _seq_inputs(T, P, H, D, W, seed=9)
+    bufs, recv = [], []
+    for j in range(W):
+        b, o = gu.guarded((T, P, part.heads(j), D), DEV)
+        bufs.append(b)
+        recv.append(o)
+    rr.seq_to_head(send, recv)
+    assert all(gu.guards_intact(b) for b in bufs)
+    sbufs, back = [], []
+    for r in range(W):
+        b, o = gu.guarded((part.tokens(r), P, H, D), DEV)
+        sbufs.append(b)
+        back.append(o)
+    rr.head_to_seq(recv, back)
+    assert all(gu.guards_intact(b) for b in sbufs)
+    assert gu.same_bits(torch.cat(back), full)
+
+
+def test_separate_send_buffers_and_side_stream(oracle_lib):
+    """Send buffers in separate allocations, work on a non-default stream."""
+    T, P, H, D, W = 600, 4, 56, 128, 4
+    part = rr.partition(T, H, W)
+    send = [wl.random_bits((part.tokens(r), P, H, D), 100 + r, DEV) for r in range(W)]
+    recv = rr.alloc_head_side(T, P, H, D, W, DEV)
+    s = torch.cuda.Stream()
+    s.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(s):
+        rr.seq_to_head(send, recv, stream=s)
+    s.synchronize()
+    want = oracle_lib.seq_to_head([gu.bits(x) for x in send], T, P, H, D, W)
+    for j in range(W):
+        assert np.array_equal(gu.bits(recv[j]), want[j])
+
+
+def test_chunked_plan_actually_ran():
+    """The chunked plan reports one launch per plane; an unchunked control
+    reports one launch and fails the chunked assertion."""
+    T, P, H, D, W = 1000, 4, 56, 128, 4
+    full, send, part = _seq_inputs(T, P, H, D, W, seed=3)
+    plane = max(part.tokens(0) * H * D * 2, T * part.heads(0) * D * 2)
+    recv = rr.alloc_head_side(T, P, H, D, W, DEV)
+    info = rr.seq_to_head(send, recv, window_bytes=plane)
+    assert info["chunks"] == P and info["launches"] == P and info["planes_per_launch"] == 1
+    control = rr.seq_to_head(send, recv, window_bytes=0)
+    assert control["chunks"] == 1 and control["launches"] == 1
+    with pytest.raises(AssertionError):
+        assert control["launches"] == P
+    with pytest.raises(rr.H3Error) as e:
+        rr.seq_to_head(send, recv, window_bytes=plane - 16)
+    assert e.value.status == 4  # H3_ERR_WINDOW
+
+
+def test_overlapping_output_rejected_on_device():
+    """An output over an input is refused before launch (all bytes in bounds)."""
+    T, P, H, D, W = 64, 3, 56, 128, 2
+    full, send, part = _seq_inputs(T, P, H, D, W, seed=4)
+    recv = rr.alloc_head_side(T, P, H, D, W, DEV)
+    alias = full.view(-1)[: recv[1].numel()].view(recv[1].shape)
+    with pytest.raises(rr.H3Error) as e:
+        rr.seq_to_head(send, [recv[0], alias])
+    assert e.value.status == 1
+
+
+def test_stress_alternating(oracle_lib):
+    """100 rounds alternating direction and world size on one stream."""
+    T, P, H, D = 999, 3, 56, 128
+    x = wl.random_bits((T, P, H, D), 77, DEV)
+    cur = x.clone()
+    worlds = [2, 4, 6, 8, 3, 7, 1, 5]
+    for it in range(100):
+        W = worlds[it % len(worlds)]
+        part = rr.partition(T, H, W)
+        recv = rr.alloc_head_side(T, P, H, D, W, DEV)
+        rr.seq_to_head(rr.split_rows(cur, part.token_starts), recv,
+                       window_bytes=(0 if it % 3 else T * part.heads(0) * D * 2 + part.tokens(0) * H * D * 2))
+        nxt = torch.empty_like(cur)
+        rr.head_to_seq(recv, rr.split_rows(nxt, part.token_starts))
+        cur = nxt
+    torch.cuda.synchronize()
+    assert gu.same_bits(cur, x)
+
+
+# ---------------------------------------------------------------------------
+# full-size workloads: sampled oracle elements + properties at any size
+# ---------------------------------------------------------------------------
+
+def _full_size_round_trip(o, w, planes=None, window=0, seed_offset=0):
+    P = w.P if planes is None else planes
+    full = wl.packed_operand(w, planes=P, device=DEV, seed_offset=seed_offset)
+    bounds = wl.segment_bounds(w.T, w.n_segs, w.seed, w.seg_lengths)
+    part = rr.partition(w.T, w.H, w.W, bounds)
+    send = rr.split_rows(full, part.token_starts)
+    recv = rr.alloc_head_side(w.T, P, w.H, w.D, w.W, DEV)
+    info = rr.seq_to_head(send, recv, window_bytes=window)
+    # torch slicing as a third opinion on every element
+    for j in range(w.W):
+        hs, he = int(part.head_starts[j]), int(part.head_starts[j + 1])
+        assert gu.same_bits(recv[j], full[:, :, hs:he, :]), f"rank {j} differs from slicing"
+    gu.sampled_check_seq_to_head(o, send, recv, w.T, P, w.H, w.D, w.W, seed=w.seed)
+    back_full, back = rr.alloc_seq_side(w.T, P, w.H, w.D, w.W, DEV)
+    info_back = rr.head_to_seq(recv, back, window_bytes=window)
+    gu.sampled_check_head_to_seq(o, recv, back, w.T, P, w.H, w.D, w.W, seed=w.seed + 1)
+    assert gu.same_bits(back_full, full)
+    return info, info_back
+
+
+def test_full_qkv_32k_w6(oracle_lib):
+    w = wl.QKV_32K_W6
+    info, _ = _full_size_round_trip(oracle_lib, w)
+    assert info["launches"] == 1
+
+
+def test_full_qkvg_128k_w4(oracle_lib):
+    w = wl.QKVG_128K_W4
+    _full_size_round_trip(oracle_lib, w)
+    torch.cuda.empty_cache()
+
+
+def test_full_attention_output_128k_w4(oracle_lib):
+    """head->seq on the attention output [131072, 56, 128] (one plane)."""
+    w = wl.QKVG_128K_W4
+    part = rr.partition(w.T, w.H, w.W)
+    heads = [wl.normal_bf16((w.T, 1, part.heads(j), w.D), w.seed + 10 + j, 1.0, DEV)
+             for j in range(w.W)]
+    out_full, out = rr.alloc_seq_side(w.T, 1, w.H, w.D, w.W, DEV)
+    rr.head_to_seq(heads, out)
+    gu.sampled_check_head_to_seq(oracle_lib, heads, out, w.T, 1, w.H, w.D, w.W, seed=5)
+    assert gu.same_bits(out_full, torch.cat(heads, dim=2))
+    torch.cuda.empty_cache()
+
+
+def test_full_qkvg_250k_w4_chunked(oracle_lib):
+    w = wl.QKVG_250K_W4_CHUNKED
+    info, info_back = _full_size_round_trip(oracle_lib, w, window=w.window_bytes)
+    for i in (info, info_back):
+        assert i["chunks"] == 4 and i["launches"] == 4 and i["planes_per_launch"] == 1
+    torch.cuda.empty_cache()
