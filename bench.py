@@ -498,6 +498,92 @@ def run_profile(args):
     return 0
 
 
+def _time_calls(fn, iters: int, warmup: int = 3) -> float:
+    """Average device seconds per call of fn() (back-to-back on one stream)."""
+    for _ in range(warmup):
+        fn()
+    torch.cuda.synchronize()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(iters):
+        fn()
+    e1.record()
+    e1.synchronize()
+    return e0.elapsed_time(e1) / 1e3 / iters
+
+
+def run_workload_report(args):
+    """Every kernel of the path on every workload, each variant: one JSON line
+    per (workload, call, variant) with GB/s and the fraction of the peak."""
+    import ragged_reduce_b200 as rr
+    torch.cuda.set_device(0)
+    dev = torch.device("cuda", 0)
+    peak, peak_kind = load_peak()
+    iters = max(3, args.steps)
+    lines = []
+
+    def emit(workload, call, variant, nbytes, secs, info):
+        rec = {"workload": workload, "call": call, "variant": variant,
+               "gbs": round(nbytes / secs / 1e9, 1), "us": round(secs * 1e6, 1),
+               "frac_of_" + peak_kind: round(nbytes / secs / 1e9 / peak, 4),
+               "bytes": nbytes, "launches": info["launches"], "grid": info["grid"],
+               "block": info["block"]}
+        lines.append(rec)
+        print(json.dumps(rec), flush=True)
+
+    variants = [("default", 0), ("vector", rr.H3_VARIANT_VECTOR), ("bulk", rr.H3_VARIANT_BULK)]
+    for w in (wl.TINY_QKV_W2, wl.QKV_32K_W6, wl.QKVG_128K_W4, wl.QKVG_250K_W4_CHUNKED):
+        x = wl.packed_operand(w, device=dev)
+        part = rr.partition(w.T, w.H, w.W)
+        send = rr.split_rows(x, part.token_starts)
+        heads = rr.alloc_head_side(w.T, w.P, w.H, w.D, w.W, dev)
+        back_full, back = rr.alloc_seq_side(w.T, w.P, w.H, w.D, w.W, dev)
+        nbytes = 2 * x.numel() * 2
+        for vname, v in variants:
+            info = rr.seq_to_head(send, heads, window_bytes=w.window_bytes, variant=v)
+            secs = _time_calls(lambda: rr.seq_to_head(send, heads, window_bytes=w.window_bytes,
+                                                      variant=v), iters)
+            emit(w.name, "seq_to_head", vname, nbytes, secs, info)
+            info = rr.head_to_seq(heads, back, window_bytes=w.window_bytes, variant=v)
+            secs = _time_calls(lambda: rr.head_to_seq(heads, back, window_bytes=w.window_bytes,
+                                                      variant=v), iters)
+            emit(w.name, "head_to_seq", vname, nbytes, secs, info)
+            if not torch.equal(back_full.view(torch.int16), x.view(torch.int16)):
+                raise SystemExit(f"{w.name} {vname}: round trip differs")
+        if w.inverse_planes:
+            # head->seq on the attention output [T, 1, H, D]
+            del heads, back_full, back
+            torch.cuda.empty_cache()
+            heads1 = [wl.normal_bf16((w.T, 1, part.heads(j), w.D), w.seed + 10 + j, 1.0, dev)
+                      for j in range(w.W)]
+            out_full, out = rr.alloc_seq_side(w.T, 1, w.H, w.D, w.W, dev)
+            nb1 = 2 * out_full.numel() * 2
+            for vname, v in variants:
+                info = rr.head_to_seq(heads1, out, variant=v)
+                secs = _time_calls(lambda: rr.head_to_seq(heads1, out, variant=v), iters)
+                emit(w.name + "_attn_out", "head_to_seq", vname, nb1, secs, info)
+            del heads1, out_full, out
+        else:
+            del heads, back_full, back
+        del x, send
+        torch.cuda.empty_cache()
+    for rw in (wl.RS_64K_W8, wl.ReduceWorkload("reduce_scatter_T32768_C7168_W6", T=32768,
+                                               C=wl.H3_HIDDEN, W=6, seed=102)):
+        partials, bias = wl.partials_and_bias(rw, dev)
+        plist = list(partials.unbind(0))
+        out_full, out = rr.alloc_reduce_outputs(rw.T, rw.C, rw.W, dev)
+        nbytes = (rw.W + 1) * rw.T * rw.C * 2 + rw.C * 2
+        info = rr.ragged_reduce_scatter(plist, bias, out)
+        secs = _time_calls(lambda: rr.ragged_reduce_scatter(plist, bias, out), iters)
+        emit(rw.name, "ragged_reduce_scatter", "default", nbytes, secs, info)
+        del partials, bias, plist, out_full, out
+        torch.cuda.empty_cache()
+    if rr.bulk_wait_timeouts() != 0:
+        raise SystemExit("bulk kernel reported expired waits")
+    return 0
+
+
 def parse_args(argv=None):
     p = argparse.ArgumentParser(description=__doc__.split("\n")[0])
     p.add_argument("--gpus", type=int, default=1)
@@ -509,6 +595,8 @@ def parse_args(argv=None):
     p.add_argument("--profile", choices=["seq_to_head", "head_to_seq", "reduce_scatter"],
                    help="run only this kernel of the step --steps times (ncu captures); no timing")
     p.add_argument("--profile-tokens", type=int, default=STEP_T)
+    p.add_argument("--report-workloads", action="store_true",
+                   help="time every kernel and variant on every workload (one JSON line each)")
     p.add_argument("--reference-budget", type=float, default=90.0,
                    help="seconds of oracle work for --impl reference (warm-up + timed)")
     return p.parse_args(argv)
@@ -518,6 +606,8 @@ def main(argv=None):
     args = parse_args(argv)
     if args.profile:
         return run_profile(args)
+    if args.report_workloads:
+        return run_workload_report(args)
     if args.warmup < 3:
         raise SystemExit("--warmup must be at least 3")
     if args.impl == "reference":

@@ -95,7 +95,7 @@ typedef struct h3_exec_info {
 
 /* Optional launch overrides for h3_*_ex; zero fields mean "library default". */
 typedef struct h3_launch_config {
-    int32_t variant;             /* 0 = default, H3_VARIANT_VECTOR or H3_VARIANT_BULK */
+    int32_t variant;             /* 0 = default, H3_VARIANT_VECTOR or H3_VARIANT_BULK (relayouts) */
     int32_t ctas_per_sm;         /* 0 = default (occupancy-derived) */
     int32_t reserved0;
     int32_t reserved1;
@@ -211,6 +211,16 @@ H3RR_API h3_status h3_ragged_reduce_scatter_ex(const void* const* partials, cons
                                       void* const* out, int64_t n_tokens, int64_t cols,
                                       int32_t world, void* stream,
                                       const h3_launch_config* cfg, h3_exec_info* info);
+
+/*
+ * h3_bulk_wait_timeouts - how many bounded waits of the bulk relayout kernel
+ * (H3_VARIANT_BULK) expired on the current device since the count was last
+ * cleared.  Each wait on a shared-memory barrier gives up after a fixed
+ * number of polls instead of spinning forever; an expiry means that launch's
+ * output is incomplete.  Synchronises `stream`; reset != 0 clears the count.
+ * count: host out-param.  Returns H3_ERR_CUDA if the copy fails.
+ */
+H3RR_API h3_status h3_bulk_wait_timeouts(void* stream, uint32_t* count, int32_t reset);
 
 #ifdef __cplusplus
 }

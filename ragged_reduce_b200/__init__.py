@@ -32,6 +32,7 @@ __all__ = [
     "H3Error", "Partition", "partition", "seq_to_head", "head_to_seq",
     "ragged_reduce_scatter", "alloc_head_side", "alloc_seq_side", "split_rows",
     "H3_VARIANT_VECTOR", "H3_VARIANT_BULK", "H3_VARIANT_REDUCE", "MAX_WORLD", "library_path",
+    "bulk_wait_timeouts", "alloc_reduce_outputs",
 ]
 
 library_path = _abi.LIB_PATH
@@ -245,6 +246,19 @@ def ragged_reduce_scatter(partials, bias, out, *, stream=None, ctas_per_sm: int 
             st = _abi.lib.h3_ragged_reduce_scatter_ex(*args, cfg, C.byref(info))
     _abi.check(st, "h3_ragged_reduce_scatter")
     return info.as_dict()
+
+
+def bulk_wait_timeouts(stream=None, reset: bool = False, device=None) -> int:
+    """Expired bounded waits of the bulk relayout kernel on this device
+    (``h3_bulk_wait_timeouts``; synchronises the stream).  Non-zero means a
+    bulk launch gave up and its output is incomplete."""
+    dev = torch.device("cuda", torch.cuda.current_device()) if device is None else torch.device(device)
+    count = C.c_uint32(0)
+    with torch.cuda.device(dev):
+        st = _abi.lib.h3_bulk_wait_timeouts(C.c_void_p(_stream_handle(stream, dev)), C.byref(count),
+                                            1 if reset else 0)
+    _abi.check(st, "h3_bulk_wait_timeouts")
+    return int(count.value)
 
 
 def alloc_reduce_outputs(T: int, C_: int, W: int, device, dtype=torch.bfloat16):

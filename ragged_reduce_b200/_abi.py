@@ -107,6 +107,8 @@ def _load() -> C.CDLL:
     lib.h3_ragged_reduce_scatter_ex.restype = C.c_int
     lib.h3_ragged_reduce_scatter_ex.argtypes = _REDUCE_ARGS + [C.POINTER(LaunchConfig),
                                                                C.POINTER(ExecInfo)]
+    lib.h3_bulk_wait_timeouts.restype = C.c_int
+    lib.h3_bulk_wait_timeouts.argtypes = [C.c_void_p, C.POINTER(C.c_uint32), C.c_int32]
     version = lib.h3_abi_version()
     if version != ABI_VERSION:
         raise ImportError(f"libh3rr ABI version {version}, binding expects {ABI_VERSION}")

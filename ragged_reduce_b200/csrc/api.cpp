@@ -64,7 +64,7 @@ h3_status relayout(bool seq_to_head, const void* const* send, void* const* recv,
         return st;
     if (planes < 1 || head_dim < 1 || window_bytes < 0 || !send || !recv)
         return H3_ERR_INVALID_ARG;
-    if (cfg && cfg->variant != 0 && cfg->variant != H3_VARIANT_VECTOR)
+    if (cfg && cfg->variant != 0 && cfg->variant != H3_VARIANT_VECTOR && cfg->variant != H3_VARIANT_BULK)
         return H3_ERR_INVALID_ARG;
     if (cfg && cfg->ctas_per_sm < 0)
         return H3_ERR_INVALID_ARG;
@@ -120,6 +120,7 @@ h3_status relayout(bool seq_to_head, const void* const* send, void* const* recv,
     }
     a.T = int32_t(n_tokens);
     a.P = planes;
+    a.W = world;
     a.tq = int32_t(ts.q);
     a.tm = int32_t(ts.m);
     a.hq = int32_t(hs.q);
@@ -129,6 +130,13 @@ h3_status relayout(bool seq_to_head, const void* const* send, void* const* recv,
 
     const int variant = cfg ? cfg->variant : 0;
     const int ctas_per_sm = cfg ? cfg->ctas_per_sm : 0;
+    if (variant == H3_VARIANT_BULK) {
+        int device = 0;
+        if (cudaGetDevice(&device) != cudaSuccess)
+            return H3_ERR_CUDA;
+        if (!relayout_bulk_fits(a, device))
+            return H3_ERR_UNSUPPORTED;  // a row does not fit the shared-memory ring
+    }
     const int chunks = chunked ? planes : 1;
     const int per_launch = chunked ? 1 : planes;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
@@ -324,6 +332,19 @@ h3_status h3_ragged_reduce_scatter_ex(const void* const* partials, const void* b
         info->variant = shape.variant;
         info->planes_per_launch = 1;
     }
+    return H3_OK;
+}
+
+h3_status h3_bulk_wait_timeouts(void* stream, uint32_t* count, int32_t reset)
+{
+    if (!count)
+        return H3_ERR_INVALID_ARG;
+    unsigned int v = 0;
+    if (read_bulk_wait_timeouts(&v, reset != 0, static_cast<cudaStream_t>(stream)) != cudaSuccess) {
+        cudaGetLastError();
+        return H3_ERR_CUDA;
+    }
+    *count = v;
     return H3_OK;
 }
 

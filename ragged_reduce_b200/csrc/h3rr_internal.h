@@ -47,6 +47,7 @@ struct RelayoutArgs {
     char* head[kMaxWorld];   // head-side rank buffers [T, P, H_j, D]
     int32_t T;
     int32_t P;
+    int32_t W;
     int32_t plane0;
     int32_t nplanes;
     int32_t rows;            // T * nplanes
@@ -77,6 +78,12 @@ struct LaunchShape {
 cudaError_t launch_relayout(bool seq_to_head, const RelayoutArgs& a, int variant,
                             int ctas_per_sm, cudaStream_t stream, LaunchShape* shape);
 
+// Whether the bulk kernel's shared-memory ring fits one row of these args.
+bool relayout_bulk_fits(const RelayoutArgs& a, int device);
+
+// Copy (and optionally clear) the per-device count of expired bulk waits.
+cudaError_t read_bulk_wait_timeouts(unsigned int* count, bool reset, cudaStream_t stream);
+
 // Enqueue the reduce-scatter launch.
 cudaError_t launch_reduce_scatter(const ReduceArgs& a, int ctas_per_sm, cudaStream_t stream,
                                   LaunchShape* shape);
@@ -87,5 +94,9 @@ int current_sm_count(int* device);
 // Resident CTAs per SM of a kernel at the given block size and dynamic shared
 // memory (cached per kernel and device).
 int resident_ctas(const void* kernel, int block, size_t smem, int device);
+
+// Opt a kernel in to `smem` bytes of dynamic shared memory on the current
+// device (once per kernel, device and size).
+cudaError_t allow_dynamic_smem(const void* kernel, size_t smem, int device);
 
 }  // namespace h3rr

@@ -106,4 +106,33 @@ int resident_ctas(const void* kernel, int block, size_t smem, int device)
     return n;
 }
 
+cudaError_t allow_dynamic_smem(const void* kernel, size_t smem, int device)
+{
+    if (smem <= 48 * 1024)
+        return cudaSuccess;
+    struct Key {
+        const void* k;
+        size_t smem;
+        int dev;
+        bool operator==(const Key& o) const { return k == o.k && smem == o.smem && dev == o.dev; }
+    };
+    struct Hash {
+        size_t operator()(const Key& x) const
+        {
+            return std::hash<const void*>()(x.k) ^ (x.smem << 7) ^ size_t(x.dev);
+        }
+    };
+    static std::mutex mu;
+    static std::unordered_map<Key, bool, Hash> done;
+    std::lock_guard<std::mutex> lock(mu);
+    const Key key{kernel, smem, device};
+    if (done.count(key))
+        return cudaSuccess;
+    const cudaError_t err =
+        cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
+    if (err == cudaSuccess)
+        done.emplace(key, true);
+    return err;
+}
+
 }  // namespace h3rr

@@ -10,33 +10,69 @@
 // contiguously in that rank's [T, P, H_j, D] buffer.  Every byte is read once
 // and written once; nothing is padded.
 //
-// The vector variant gives each 128-thread CTA one row at a time (or two):
-// thread i owns the row's 16-byte vectors i, i+128, i+256, ..., so a warp
-// touches 512 contiguous bytes on both sides.  The head-side rank, its base
-// pointer and its row stride for each of a thread's vectors depend only on
-// the column, so they are computed once per thread before the row loop.
-// Sources are read with non-coherent streaming loads (inputs never overlap
-// outputs; the host checks this), outputs are written with streaming stores.
+// Two kernel families move the same bytes:
+//
+// * Vector kernels: a CTA of NT threads takes ROWS rows at a time; thread i
+//   owns the row's vectors i, i+NT, i+2NT, ... (VW = 16 or 32 bytes, 32 when
+//   every pointer and run allows it), so a warp touches 512 or 1024
+//   contiguous bytes on both sides.  The head-side rank, base pointer and
+//   row stride of each of a thread's vectors depend only on the column, so
+//   they are computed once per thread before the row loop.  All loads of an
+//   iteration are issued before its first store.  Sources use non-coherent
+//   streaming loads (inputs never overlap outputs; the host checks this),
+//   outputs streaming stores.
+//
+// * Bulk kernel: one thread per CTA drives the tensor memory accelerator's
+//   1-D bulk copies through a ring of S shared-memory stages, one row per
+//   stage.  Loads run L rows ahead of stores; an mbarrier per stage tracks
+//   load completion and bulk-group waits keep a stage from being refilled
+//   before its stores have read it.  No multicast is used.  Every mbarrier
+//   wait is bounded: on expiry the kernel counts the event in a device word
+//   (read with h3_bulk_wait_timeouts), drains what it issued and returns.
 #include "h3rr_internal.h"
 
 namespace h3rr {
+
+// Count of bounded waits that expired in the bulk kernel (per device).
+__device__ unsigned int g_bulk_wait_timeouts = 0;
+
 namespace {
 
-constexpr int kThreads = 128;
+// ---------------------------------------------------------------------------
+// memory access helpers
+// ---------------------------------------------------------------------------
+template <int VW>
+struct Vec {
+    uint32_t r[VW / 4];
+};
 
-__device__ __forceinline__ uint4 ld_stream(const char* p)
+__device__ __forceinline__ void ld_stream(Vec<16>& v, const char* p)
 {
-    uint4 v;
     asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0, %1, %2, %3}, [%4];"
-                 : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+                 : "=r"(v.r[0]), "=r"(v.r[1]), "=r"(v.r[2]), "=r"(v.r[3])
                  : "l"(p));
-    return v;
 }
 
-__device__ __forceinline__ void st_stream(char* p, const uint4& v)
+__device__ __forceinline__ void ld_stream(Vec<32>& v, const char* p)
 {
-    asm volatile("st.global.cs.v4.u32 [%0], {%1, %2, %3, %4};" ::"l"(p), "r"(v.x), "r"(v.y),
-                 "r"(v.z), "r"(v.w)
+    asm volatile("ld.global.nc.L1::no_allocate.v8.u32 {%0, %1, %2, %3, %4, %5, %6, %7}, [%8];"
+                 : "=r"(v.r[0]), "=r"(v.r[1]), "=r"(v.r[2]), "=r"(v.r[3]), "=r"(v.r[4]),
+                   "=r"(v.r[5]), "=r"(v.r[6]), "=r"(v.r[7])
+                 : "l"(p));
+}
+
+__device__ __forceinline__ void st_stream(char* p, const Vec<16>& v)
+{
+    asm volatile("st.global.cs.v4.u32 [%0], {%1, %2, %3, %4};" ::"l"(p), "r"(v.r[0]), "r"(v.r[1]),
+                 "r"(v.r[2]), "r"(v.r[3])
+                 : "memory");
+}
+
+__device__ __forceinline__ void st_stream(char* p, const Vec<32>& v)
+{
+    asm volatile("st.global.cs.v8.u32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};" ::"l"(p),
+                 "r"(v.r[0]), "r"(v.r[1]), "r"(v.r[2]), "r"(v.r[3]), "r"(v.r[4]), "r"(v.r[5]),
+                 "r"(v.r[6]), "r"(v.r[7])
                  : "memory");
 }
 
@@ -52,27 +88,33 @@ __device__ __forceinline__ int32_t split_start(int32_t i, int32_t q, int32_t m)
     return i * q + (i < m ? i : m);
 }
 
-template <bool kSeqToHead, int VPT, int ROWS>
-__global__ void __launch_bounds__(kThreads) relayout_vec_kernel(const __grid_constant__ RelayoutArgs a)
+// ---------------------------------------------------------------------------
+// vector kernels
+// ---------------------------------------------------------------------------
+template <bool kSeqToHead, int VW, int NT, int VPT, int ROWS>
+__global__ void __launch_bounds__(NT) relayout_vec_kernel(const __grid_constant__ RelayoutArgs a)
 {
+    constexpr int kUnits = VW / kVecBytes;  // 16-byte units per vector
+    const int32_t row_v = a.row_vecs / kUnits;
+    const int32_t head_v = a.head_vecs / kUnits;
     // Head-side placement of this thread's columns (same for every row).
     char* hbase[VPT];
-    int64_t hstride[VPT];
+    int32_t hstride[VPT];
     bool live[VPT];
 #pragma unroll
     for (int k = 0; k < VPT; ++k) {
-        const int32_t c = threadIdx.x + k * kThreads;
-        live[k] = c < a.row_vecs;
+        const int32_t c = threadIdx.x + k * NT;
+        live[k] = c < row_v;
         const int32_t cc = live[k] ? c : 0;
-        const int32_t h = cc / a.head_vecs;
-        const int32_t within = cc - h * a.head_vecs;
+        const int32_t h = cc / head_v;
+        const int32_t within = cc - h * head_v;
         const int32_t j = split_owner(h, a.hq, a.hm);
         const int32_t hj = a.hq + (j < a.hm ? 1 : 0);
         const int32_t hl = h - split_start(j, a.hq, a.hm);
-        hbase[k] = a.head[j] + (int64_t(hl) * a.head_vecs + within) * kVecBytes;
-        hstride[k] = int64_t(hj) * a.head_vecs * kVecBytes;
+        hbase[k] = a.head[j] + (int64_t(hl) * head_v + within) * VW;
+        hstride[k] = hj * head_v * VW;
     }
-    const int64_t seq_row_bytes = int64_t(a.row_vecs) * kVecBytes;
+    const int64_t seq_row_bytes = int64_t(row_v) * VW;
 
     for (int64_t i0 = int64_t(blockIdx.x) * ROWS; i0 < a.rows; i0 += int64_t(gridDim.x) * ROWS) {
         char* sptr[ROWS];
@@ -87,18 +129,16 @@ __global__ void __launch_bounds__(kThreads) relayout_vec_kernel(const __grid_con
             const int32_t s = split_owner(t, a.tq, a.tm);
             const int32_t tl = t - split_start(s, a.tq, a.tm);
             g[r] = int64_t(t) * a.P + p;
-            sptr[r] = a.seq[s] + (int64_t(tl) * a.P + p) * seq_row_bytes +
-                      int64_t(threadIdx.x) * kVecBytes;
+            sptr[r] = a.seq[s] + (int64_t(tl) * a.P + p) * seq_row_bytes + int64_t(threadIdx.x) * VW;
         }
-        uint4 v[ROWS][VPT];
+        Vec<VW> v[ROWS][VPT];
 #pragma unroll
         for (int r = 0; r < ROWS; ++r) {
 #pragma unroll
             for (int k = 0; k < VPT; ++k) {
                 if (rv[r] && live[k]) {
-                    const char* src = kSeqToHead ? sptr[r] + k * kThreads * kVecBytes
-                                                 : hbase[k] + g[r] * hstride[k];
-                    v[r][k] = ld_stream(src);
+                    const char* src = kSeqToHead ? sptr[r] + k * NT * VW : hbase[k] + g[r] * hstride[k];
+                    ld_stream(v[r][k], src);
                 }
             }
         }
@@ -107,8 +147,7 @@ __global__ void __launch_bounds__(kThreads) relayout_vec_kernel(const __grid_con
 #pragma unroll
             for (int k = 0; k < VPT; ++k) {
                 if (rv[r] && live[k]) {
-                    char* dst = kSeqToHead ? hbase[k] + g[r] * hstride[k]
-                                           : sptr[r] + k * kThreads * kVecBytes;
+                    char* dst = kSeqToHead ? hbase[k] + g[r] * hstride[k] : sptr[r] + k * NT * VW;
                     st_stream(dst, v[r][k]);
                 }
             }
@@ -117,8 +156,10 @@ __global__ void __launch_bounds__(kThreads) relayout_vec_kernel(const __grid_con
 }
 
 // Any row width: one row per CTA iteration, head-side placement per vector.
+constexpr int kGenericThreads = 128;
+
 template <bool kSeqToHead>
-__global__ void __launch_bounds__(kThreads) relayout_generic_kernel(const __grid_constant__ RelayoutArgs a)
+__global__ void __launch_bounds__(kGenericThreads) relayout_generic_kernel(const __grid_constant__ RelayoutArgs a)
 {
     const int64_t seq_row_bytes = int64_t(a.row_vecs) * kVecBytes;
     for (int64_t i64 = blockIdx.x; i64 < a.rows; i64 += gridDim.x) {
@@ -129,7 +170,7 @@ __global__ void __launch_bounds__(kThreads) relayout_generic_kernel(const __grid
         const int32_t tl = t - split_start(s, a.tq, a.tm);
         const int64_t g = int64_t(t) * a.P + p;
         char* srow = a.seq[s] + (int64_t(tl) * a.P + p) * seq_row_bytes;
-        for (int32_t c = threadIdx.x; c < a.row_vecs; c += kThreads) {
+        for (int32_t c = threadIdx.x; c < a.row_vecs; c += kGenericThreads) {
             const int32_t h = c / a.head_vecs;
             const int32_t within = c - h * a.head_vecs;
             const int32_t j = split_owner(h, a.hq, a.hm);
@@ -137,56 +178,304 @@ __global__ void __launch_bounds__(kThreads) relayout_generic_kernel(const __grid
             const int32_t hl = h - split_start(j, a.hq, a.hm);
             char* hp = a.head[j] + ((g * hj + hl) * a.head_vecs + within) * kVecBytes;
             char* sp = srow + int64_t(c) * kVecBytes;
-            if (kSeqToHead)
-                st_stream(hp, ld_stream(sp));
-            else
-                st_stream(sp, ld_stream(hp));
+            Vec<16> v;
+            if (kSeqToHead) {
+                ld_stream(v, sp);
+                st_stream(hp, v);
+            } else {
+                ld_stream(v, hp);
+                st_stream(sp, v);
+            }
         }
     }
 }
 
-template <bool kSeqToHead>
-const void* pick_vec_kernel(int vpt, int* rows_per_iter)
+// ---------------------------------------------------------------------------
+// bulk kernel (tensor memory accelerator, 1-D bulk copies, no multicast)
+// ---------------------------------------------------------------------------
+constexpr int kBulkStages = 14;
+constexpr int kBulkLookahead = 11;
+constexpr int kBulkBarrierBytes = 128;          // room for 16 mbarriers
+constexpr uint32_t kBulkWaitLimit = 1u << 24;   // try_wait polls before giving up
+
+__device__ __forceinline__ uint32_t smem_addr(const void* p)
 {
-    // Two rows per iteration keeps at least 8 vectors per thread in flight
-    // when a row is narrow.
-#define H3RR_VEC_CASE(V, R)                                             \
-    case V:                                                             \
-        *rows_per_iter = R;                                             \
-        return (const void*)relayout_vec_kernel<kSeqToHead, V, R>;
-    switch (vpt) {
-        H3RR_VEC_CASE(1, 2)
-        H3RR_VEC_CASE(2, 2)
-        H3RR_VEC_CASE(3, 2)
-        H3RR_VEC_CASE(4, 2)
-        H3RR_VEC_CASE(5, 1)
-        H3RR_VEC_CASE(6, 1)
-        H3RR_VEC_CASE(7, 1)
-        H3RR_VEC_CASE(8, 1)
-        default:
-            break;
+    return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+__device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count)
+{
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_addr(bar)), "r"(count) : "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t* bar, uint32_t bytes)
+{
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_addr(bar)),
+                 "r"(bytes)
+                 : "memory");
+}
+
+// Bounded wait for the phase with the given parity; false if it expired.
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity)
+{
+    for (uint32_t it = 0; it < kBulkWaitLimit; ++it) {
+        uint32_t done;
+        asm volatile(
+            "{\n\t.reg .pred p;\n\t"
+            "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+            "selp.u32 %0, 1, 0, p;\n\t}"
+            : "=r"(done)
+            : "r"(smem_addr(bar)), "r"(parity)
+            : "memory");
+        if (done)
+            return true;
     }
-#undef H3RR_VEC_CASE
-    *rows_per_iter = 1;
-    return (const void*)relayout_generic_kernel<kSeqToHead>;
+    return false;
+}
+
+__device__ __forceinline__ uint64_t evict_first_policy()
+{
+    uint64_t pol;
+    asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(pol));
+    return pol;
+}
+
+__device__ __forceinline__ void bulk_load(void* smem_dst, const void* src, uint32_t bytes, uint64_t* bar,
+                                          uint64_t pol)
+{
+    asm volatile(
+        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint "
+        "[%0], [%1], %2, [%3], %4;" ::"r"(smem_addr(smem_dst)),
+        "l"(src), "r"(bytes), "r"(smem_addr(bar)), "l"(pol)
+        : "memory");
+}
+
+__device__ __forceinline__ void bulk_store(void* dst, const void* smem_src, uint32_t bytes, uint64_t pol)
+{
+    asm volatile("cp.async.bulk.global.shared::cta.bulk_group.L2::cache_hint [%0], [%1], %2, %3;" ::"l"(dst),
+                 "r"(smem_addr(smem_src)), "r"(bytes), "l"(pol)
+                 : "memory");
+}
+
+__device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
+
+template <int N>
+__device__ __forceinline__ void bulk_wait_read()
+{
+    asm volatile("cp.async.bulk.wait_group.read %0;" ::"n"(N) : "memory");
+}
+
+__device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
+
+template <bool kSeqToHead, int S, int L>
+__global__ void __launch_bounds__(32) relayout_bulk_kernel(const __grid_constant__ RelayoutArgs a)
+{
+    static_assert(S <= kBulkBarrierBytes / 8 && L >= 1 && L < S, "bulk ring shape");
+    extern __shared__ __align__(128) unsigned char smem[];
+    uint64_t* bars = reinterpret_cast<uint64_t*>(smem);
+    unsigned char* ring = smem + kBulkBarrierBytes;
+    if (threadIdx.x != 0)
+        return;
+    const uint32_t row_bytes = uint32_t(a.row_vecs) * kVecBytes;
+    const uint32_t head_bytes = uint32_t(a.head_vecs) * kVecBytes;
+    const uint64_t pol = evict_first_policy();
+    for (int s = 0; s < S; ++s)
+        mbar_init(&bars[s], 1);
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+
+    const int64_t n_rows =
+        a.rows > int32_t(blockIdx.x) ? (int64_t(a.rows) - blockIdx.x + gridDim.x - 1) / gridDim.x : 0;
+
+    // Row n of this CTA -> (sequence-side row address, head-side row index g).
+    auto locate = [&](int64_t n, char** seq_row, int64_t* g) {
+        const int32_t i = int32_t(blockIdx.x + n * gridDim.x);
+        const int32_t t = i / a.nplanes;
+        const int32_t p = a.plane0 + (i - t * a.nplanes);
+        const int32_t s = split_owner(t, a.tq, a.tm);
+        const int32_t tl = t - split_start(s, a.tq, a.tm);
+        *seq_row = a.seq[s] + (int64_t(tl) * a.P + p) * row_bytes;
+        *g = int64_t(t) * a.P + p;
+    };
+    auto issue_load = [&](int64_t n) {
+        char* seq_row;
+        int64_t g;
+        locate(n, &seq_row, &g);
+        unsigned char* stage = ring + size_t(n % S) * row_bytes;
+        uint64_t* bar = &bars[n % S];
+        mbar_arrive_expect_tx(bar, row_bytes);
+        if (kSeqToHead) {
+            bulk_load(stage, seq_row, row_bytes, bar, pol);
+        } else {
+            uint32_t off = 0;
+            for (int j = 0; j < a.W; ++j) {
+                const uint32_t run = uint32_t(a.hq + (j < a.hm ? 1 : 0)) * head_bytes;
+                bulk_load(stage + off, a.head[j] + g * run, run, bar, pol);
+                off += run;
+            }
+        }
+    };
+    auto issue_store = [&](int64_t n) {
+        char* seq_row;
+        int64_t g;
+        locate(n, &seq_row, &g);
+        const unsigned char* stage = ring + size_t(n % S) * row_bytes;
+        if (kSeqToHead) {
+            uint32_t off = 0;
+            for (int j = 0; j < a.W; ++j) {
+                const uint32_t run = uint32_t(a.hq + (j < a.hm ? 1 : 0)) * head_bytes;
+                bulk_store(a.head[j] + g * run, stage + off, run, pol);
+                off += run;
+            }
+        } else {
+            bulk_store(seq_row, stage, row_bytes, pol);
+        }
+        bulk_commit();
+    };
+
+    const int64_t prologue = n_rows < L ? n_rows : L;
+    for (int64_t n = 0; n < prologue; ++n)
+        issue_load(n);
+    for (int64_t n = 0; n < n_rows; ++n) {
+        if (n + L < n_rows) {
+            // Stage (n+L)%S last served row n+L-S, whose store group must have
+            // finished reading it: at most S-L-1 newer groups may be pending.
+            bulk_wait_read<S - L - 1>();
+            issue_load(n + L);
+        }
+        if (!mbar_wait(&bars[n % S], uint32_t((n / S) & 1))) {
+            atomicAdd(&g_bulk_wait_timeouts, 1u);
+            // Drain the loads already in flight (bounded) before leaving.
+            for (int64_t m = n + 1; m < n_rows && m <= n + L; ++m)
+                mbar_wait(&bars[m % S], uint32_t((m / S) & 1));
+            break;
+        }
+        issue_store(n);
+    }
+    bulk_wait_all();
+}
+
+// ---------------------------------------------------------------------------
+// dispatch
+// ---------------------------------------------------------------------------
+struct KernelChoice {
+    const void* fn = nullptr;
+    int threads = 0;
+    int rows_per_cta_iter = 1;
+    size_t smem = 0;
+    int variant = H3_VARIANT_NONE;
+};
+
+// Smallest instantiated vectors-per-thread count (at most MAXV) covering `need`.
+template <bool S2H, int VW, int NT, int ROWS, int MAXV>
+bool pick_vec(int need, KernelChoice* kc)
+{
+#define H3RR_VPT(V)                                                              \
+    if constexpr (V <= MAXV) {                                                   \
+        if (need <= V) {                                                         \
+            kc->fn = (const void*)relayout_vec_kernel<S2H, VW, NT, V, ROWS>;     \
+            kc->threads = NT;                                                    \
+            kc->rows_per_cta_iter = ROWS;                                        \
+            kc->variant = H3_VARIANT_VECTOR;                                     \
+            return true;                                                         \
+        }                                                                        \
+    }
+    H3RR_VPT(1)
+    H3RR_VPT(2)
+    H3RR_VPT(4)
+    H3RR_VPT(7)
+    H3RR_VPT(8)
+    H3RR_VPT(14)
+    H3RR_VPT(16)
+#undef H3RR_VPT
+    return false;
+}
+
+// Vector kernel shapes measured fastest on B200 for H3 rows (14,336 bytes):
+// sequence->head with 32-byte vectors, 64 threads and two rows in flight;
+// head->sequence with 32-byte vectors and one warp per CTA.  Wider rows fall
+// back to 16-byte vectors with 128 threads, then to the generic kernel.
+template <bool S2H>
+void choose_vec(const RelayoutArgs& a, bool wide_ok, KernelChoice* kc)
+{
+    if (wide_ok) {
+        const int row32 = a.row_vecs / 2;
+        const bool ok = S2H ? pick_vec<true, 32, 64, 2, 8>((row32 + 63) / 64, kc)
+                            : pick_vec<false, 32, 32, 1, 16>((row32 + 31) / 32, kc);
+        if (ok)
+            return;
+    }
+    if (pick_vec<S2H, 16, 128, 1, 16>((a.row_vecs + 127) / 128, kc))
+        return;
+    kc->fn = (const void*)relayout_generic_kernel<S2H>;
+    kc->threads = kGenericThreads;
+    kc->rows_per_cta_iter = 1;
+    kc->variant = H3_VARIANT_VECTOR;
+}
+
+bool choose_bulk(bool s2h, const RelayoutArgs& a, int device, KernelChoice* kc)
+{
+    const size_t row_bytes = size_t(a.row_vecs) * kVecBytes;
+    const size_t smem = kBulkBarrierBytes + kBulkStages * row_bytes;
+    int max_smem = 0;
+    if (cudaDeviceGetAttribute(&max_smem, cudaDevAttrMaxSharedMemoryPerBlockOptin, device) != cudaSuccess)
+        return false;
+    if (smem > size_t(max_smem))
+        return false;
+    kc->fn = s2h ? (const void*)relayout_bulk_kernel<true, kBulkStages, kBulkLookahead>
+                 : (const void*)relayout_bulk_kernel<false, kBulkStages, kBulkLookahead>;
+    kc->threads = 32;
+    kc->rows_per_cta_iter = 1;
+    kc->smem = smem;
+    kc->variant = H3_VARIANT_BULK;
+    return true;
+}
+
+bool wide_vectors_ok(const RelayoutArgs& a)
+{
+    if ((a.head_vecs % 2) != 0)
+        return false;
+    for (int r = 0; r < a.W; ++r)
+        if ((reinterpret_cast<uintptr_t>(a.seq[r]) & 31u) || (reinterpret_cast<uintptr_t>(a.head[r]) & 31u))
+            return false;
+    return true;
 }
 
 }  // namespace
 
-cudaError_t launch_relayout(bool seq_to_head, const RelayoutArgs& a, int variant,
-                            int ctas_per_sm, cudaStream_t stream, LaunchShape* shape)
+bool relayout_bulk_fits(const RelayoutArgs& a, int device)
 {
-    (void)variant;  // only the vector variant exists so far
-    const int vpt = (a.row_vecs + kThreads - 1) / kThreads;
-    int rows_per_iter = 1;
-    const void* kernel = seq_to_head ? pick_vec_kernel<true>(vpt, &rows_per_iter)
-                                     : pick_vec_kernel<false>(vpt, &rows_per_iter);
+    KernelChoice kc;
+    return choose_bulk(true, a, device, &kc);
+}
+
+cudaError_t launch_relayout(bool seq_to_head, const RelayoutArgs& a, int variant, int ctas_per_sm,
+                            cudaStream_t stream, LaunchShape* shape)
+{
     int device = 0;
     const int sms = current_sm_count(&device);
     if (sms <= 0)
         return cudaErrorNoDevice;
-    const int per_sm = ctas_per_sm > 0 ? ctas_per_sm : resident_ctas(kernel, kThreads, 0, device);
-    const int64_t needed = (int64_t(a.rows) + rows_per_iter - 1) / rows_per_iter;
+    KernelChoice kc;
+    // Default: the bulk kernel for head->sequence with at most four ranks
+    // (fastest measured there), the vector kernels otherwise.
+    const bool want_bulk = variant == H3_VARIANT_BULK || (variant == 0 && !seq_to_head && a.W <= 4);
+    bool bulk = false;
+    if (want_bulk)
+        bulk = choose_bulk(seq_to_head, a, device, &kc);
+    if (variant == H3_VARIANT_BULK && !bulk)
+        return cudaErrorInvalidConfiguration;
+    if (!bulk) {
+        if (seq_to_head)
+            choose_vec<true>(a, wide_vectors_ok(a), &kc);
+        else
+            choose_vec<false>(a, wide_vectors_ok(a), &kc);
+    } else {
+        const cudaError_t err = allow_dynamic_smem(kc.fn, kc.smem, device);
+        if (err != cudaSuccess)
+            return err;
+    }
+    const int per_sm = ctas_per_sm > 0 ? ctas_per_sm : resident_ctas(kc.fn, kc.threads, kc.smem, device);
+    const int64_t needed = (int64_t(a.rows) + kc.rows_per_cta_iter - 1) / kc.rows_per_cta_iter;
     int64_t grid = int64_t(sms) * per_sm;
     if (grid > needed)
         grid = needed;
@@ -194,11 +483,27 @@ cudaError_t launch_relayout(bool seq_to_head, const RelayoutArgs& a, int variant
         grid = 1;
     if (shape) {
         shape->grid = int(grid);
-        shape->block = kThreads;
-        shape->variant = H3_VARIANT_VECTOR;
+        shape->block = kc.threads;
+        shape->variant = kc.variant;
     }
     void* params[] = {const_cast<RelayoutArgs*>(&a)};
-    return cudaLaunchKernel(kernel, dim3(unsigned(grid)), dim3(kThreads), params, 0, stream);
+    return cudaLaunchKernel(kc.fn, dim3(unsigned(grid)), dim3(kc.threads), params, kc.smem, stream);
+}
+
+cudaError_t read_bulk_wait_timeouts(unsigned int* count, bool reset, cudaStream_t stream)
+{
+    cudaError_t err = cudaMemcpyFromSymbolAsync(count, g_bulk_wait_timeouts, sizeof(unsigned int), 0,
+                                                cudaMemcpyDeviceToHost, stream);
+    if (err == cudaSuccess)
+        err = cudaStreamSynchronize(stream);
+    if (err == cudaSuccess && reset) {
+        static const unsigned int zero = 0;
+        err = cudaMemcpyToSymbolAsync(g_bulk_wait_timeouts, &zero, sizeof(zero), 0, cudaMemcpyHostToDevice,
+                                      stream);
+        if (err == cudaSuccess)
+            err = cudaStreamSynchronize(stream);
+    }
+    return err;
 }
 
 }  // namespace h3rr

@@ -190,6 +190,26 @@ def test_relayout_argument_checks(fn):
 
 
 @needs_no_gpu
+def test_relayout_rejects_unknown_variant():
+    T, P, H, D, W = 100, 3, 56, 128, 2
+    send, recv = _layout(T, P, H, D, W)
+    for variant in (3, 4, 99, -1):
+        cfg = _abi.LaunchConfig(variant, 0, 0, 0)
+        info = _abi.ExecInfo()
+        st = _abi.lib.h3_seq_to_head_ex(_ptrs(send), _ptrs(recv), T, P, H, D, W, 0, None,
+                                        C.byref(cfg), C.byref(info))
+        assert st == _abi.H3_ERR_INVALID_ARG and info.launches == 0
+    cfg = _abi.LaunchConfig(0, -2, 0, 0)
+    st = _abi.lib.h3_head_to_seq_ex(_ptrs(recv), _ptrs(send), T, P, H, D, W, 0, None,
+                                    C.byref(cfg), C.byref(_abi.ExecInfo()))
+    assert st == _abi.H3_ERR_INVALID_ARG
+
+
+def test_bulk_timeout_query_needs_count():
+    assert _abi.lib.h3_bulk_wait_timeouts(None, None, 0) == _abi.H3_ERR_INVALID_ARG
+
+
+@needs_no_gpu
 def test_relayout_window_check_long_workload():
     # 250k tokens over 4 ranks: one plane of one rank is exactly 896,000,000 bytes
     T, P, H, D, W = 250000, 4, 56, 128, 4

@@ -69,6 +69,63 @@ def test_relayout_matches_oracle(oracle_lib, T, P, H, D, W, window):
     assert gu.same_bits(back_full, full)  # round trip
 
 
+# every kernel family forced through the _ex entry points, both directions
+VARIANT_SHAPES = [
+    (1000, 3, 56, 128, 6),
+    (777, 4, 56, 128, 8),
+    (513, 2, 56, 128, 4),
+    (64, 3, 56, 128, 2),
+    (100, 3, 56, 128, 1),
+    (9, 3, 56, 128, 9),
+    (130, 2, 7, 64, 3),
+    (50, 3, 5, 8, 5),
+    (40, 3, 24, 128, 7),
+]
+
+
+@pytest.mark.parametrize("T,P,H,D,W", VARIANT_SHAPES)
+@pytest.mark.parametrize("variant", [rr.H3_VARIANT_VECTOR, rr.H3_VARIANT_BULK])
+def test_forced_variant_matches_oracle(oracle_lib, T, P, H, D, W, variant):
+    full, send, part = _seq_inputs(T, P, H, D, W, seed=T * 7 + W + variant)
+    recv = rr.alloc_head_side(T, P, H, D, W, DEV)
+    rr.bulk_wait_timeouts(reset=True)
+    info = rr.seq_to_head(send, recv, variant=variant)
+    assert info["variant"] == variant
+    want = oracle_lib.seq_to_head([gu.bits(s) for s in send], T, P, H, D, W)
+    for j in range(W):
+        assert np.array_equal(gu.bits(recv[j]), want[j]), f"seq->head rank {j}"
+    back_full, back = rr.alloc_seq_side(T, P, H, D, W, DEV)
+    plane = max(part.tokens(0) * H * D * 2, T * part.heads(0) * D * 2)
+    info = rr.head_to_seq(recv, back, variant=variant, window_bytes=plane)
+    assert info["variant"] == variant and info["launches"] == P
+    assert gu.same_bits(back_full, full)
+    assert rr.bulk_wait_timeouts() == 0
+
+
+def test_bulk_rejects_rows_too_wide_for_its_ring():
+    # D=256: a 28,672-byte row, 14 stages do not fit in shared memory
+    T, P, H, D, W = 33, 3, 56, 256, 4
+    full, send, part = _seq_inputs(T, P, H, D, W, seed=1)
+    recv = rr.alloc_head_side(T, P, H, D, W, DEV)
+    with pytest.raises(rr.H3Error) as e:
+        rr.seq_to_head(send, recv, variant=rr.H3_VARIANT_BULK)
+    assert e.value.status == 5  # H3_ERR_UNSUPPORTED
+    info = rr.seq_to_head(send, recv)  # the default falls back to vectors
+    assert info["variant"] == rr.H3_VARIANT_VECTOR
+
+
+def test_default_variants():
+    """Defaults: vectors for seq->head, the bulk ring for head->seq at W <= 4."""
+    for W, want_back in [(2, rr.H3_VARIANT_BULK), (4, rr.H3_VARIANT_BULK), (6, rr.H3_VARIANT_VECTOR)]:
+        T, P, H, D = 300, 3, 56, 128
+        full, send, part = _seq_inputs(T, P, H, D, W, seed=W)
+        recv = rr.alloc_head_side(T, P, H, D, W, DEV)
+        assert rr.seq_to_head(send, recv)["variant"] == rr.H3_VARIANT_VECTOR
+        back_full, back = rr.alloc_seq_side(T, P, H, D, W, DEV)
+        assert rr.head_to_seq(recv, back)["variant"] == want_back
+        assert gu.same_bits(back_full, full)
+
+
 def test_world_one_identity():
     T, P, H, D = 257, 3, 56, 128
     full = wl.random_bits((T, P, H, D), 5, DEV)
