@@ -107,6 +107,11 @@ H3RR_API int32_t h3_abi_version(void);
 /* Short static English description of a status code. */
 H3RR_API const char* h3_status_string(h3_status status);
 
+/* The cudaError_t value behind the calling thread's most recent H3_ERR_CUDA
+ * (0 if none), and, if message is not NULL, the CUDA runtime's static text
+ * for it.  Kept per thread; a later H3_ERR_CUDA on the thread replaces it. */
+H3RR_API int32_t h3_last_cuda_error(const char** message);
+
 /*
  * h3_partition - the partition contract, host only ("Distributed H3
  * Execution", "Partition Contract").

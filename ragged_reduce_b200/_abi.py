@@ -70,7 +70,13 @@ class H3Error(RuntimeError):
         self.status = int(status)
         self.call = call
         name = STATUS_NAMES.get(self.status, str(self.status))
-        super().__init__(f"{call}: {name} ({describe(self.status)})")
+        detail = ""
+        self.cuda_error = 0
+        if self.status == H3_ERR_CUDA:
+            msg = C.c_char_p()
+            self.cuda_error = int(lib.h3_last_cuda_error(C.byref(msg)))
+            detail = f"; cudaError {self.cuda_error}: {msg.value.decode() if msg.value else ''}"
+        super().__init__(f"{call}: {name} ({describe(self.status)}{detail})")
 
 
 _i64p = C.POINTER(C.c_int64)
@@ -107,6 +113,8 @@ def _load() -> C.CDLL:
     lib.h3_ragged_reduce_scatter_ex.restype = C.c_int
     lib.h3_ragged_reduce_scatter_ex.argtypes = _REDUCE_ARGS + [C.POINTER(LaunchConfig),
                                                                C.POINTER(ExecInfo)]
+    lib.h3_last_cuda_error.restype = C.c_int32
+    lib.h3_last_cuda_error.argtypes = [C.POINTER(C.c_char_p)]
     lib.h3_bulk_wait_timeouts.restype = C.c_int
     lib.h3_bulk_wait_timeouts.argtypes = [C.c_void_p, C.POINTER(C.c_uint32), C.c_int32]
     version = lib.h3_abi_version()

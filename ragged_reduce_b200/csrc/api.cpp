@@ -10,6 +10,16 @@ using namespace h3rr;
 
 namespace {
 
+// CUDA error behind the calling thread's most recent H3_ERR_CUDA.
+thread_local int t_last_cuda_error = 0;
+
+h3_status cuda_failure(cudaError_t err)
+{
+    t_last_cuda_error = int(err);
+    cudaGetLastError();  // clear a non-sticky launch error
+    return H3_ERR_CUDA;
+}
+
 constexpr int64_t kMaxInt32 = INT32_MAX;
 // Column loops step by up to 1024 vectors past the row end; keep that in int32.
 constexpr int64_t kMaxRowVecs = int64_t(1) << 30;
@@ -132,8 +142,9 @@ h3_status relayout(bool seq_to_head, const void* const* send, void* const* recv,
     const int ctas_per_sm = cfg ? cfg->ctas_per_sm : 0;
     if (variant == H3_VARIANT_BULK) {
         int device = 0;
-        if (cudaGetDevice(&device) != cudaSuccess)
-            return H3_ERR_CUDA;
+        const cudaError_t err = cudaGetDevice(&device);
+        if (err != cudaSuccess)
+            return cuda_failure(err);
         if (!relayout_bulk_fits(a, device))
             return H3_ERR_UNSUPPORTED;  // a row does not fit the shared-memory ring
     }
@@ -148,12 +159,11 @@ h3_status relayout(bool seq_to_head, const void* const* send, void* const* recv,
         a.rows = int32_t(n_tokens * per_launch);
         const cudaError_t err = launch_relayout(seq_to_head, a, variant, ctas_per_sm, s, &shape);
         if (err != cudaSuccess) {
-            cudaGetLastError();
             if (info) {
                 info->launches = launched;
                 info->chunks = chunks;
             }
-            return H3_ERR_CUDA;
+            return cuda_failure(err);
         }
         ++launched;
     }
@@ -173,6 +183,13 @@ h3_status relayout(bool seq_to_head, const void* const* send, void* const* recv,
 extern "C" {
 
 int32_t h3_abi_version(void) { return H3RR_ABI_VERSION; }
+
+int32_t h3_last_cuda_error(const char** message)
+{
+    if (message)
+        *message = t_last_cuda_error ? cudaGetErrorString(cudaError_t(t_last_cuda_error)) : "no error";
+    return t_last_cuda_error;
+}
 
 const char* h3_status_string(h3_status status)
 {
@@ -320,10 +337,8 @@ h3_status h3_ragged_reduce_scatter_ex(const void* const* partials, const void* b
     LaunchShape shape;
     const cudaError_t err = launch_reduce_scatter(a, cfg ? cfg->ctas_per_sm : 0,
                                                   static_cast<cudaStream_t>(stream), &shape);
-    if (err != cudaSuccess) {
-        cudaGetLastError();
-        return H3_ERR_CUDA;
-    }
+    if (err != cudaSuccess)
+        return cuda_failure(err);
     if (info) {
         info->launches = 1;
         info->chunks = 1;
@@ -340,10 +355,9 @@ h3_status h3_bulk_wait_timeouts(void* stream, uint32_t* count, int32_t reset)
     if (!count)
         return H3_ERR_INVALID_ARG;
     unsigned int v = 0;
-    if (read_bulk_wait_timeouts(&v, reset != 0, static_cast<cudaStream_t>(stream)) != cudaSuccess) {
-        cudaGetLastError();
-        return H3_ERR_CUDA;
-    }
+    const cudaError_t err = read_bulk_wait_timeouts(&v, reset != 0, static_cast<cudaStream_t>(stream));
+    if (err != cudaSuccess)
+        return cuda_failure(err);
     *count = v;
     return H3_OK;
 }

@@ -108,30 +108,36 @@ int resident_ctas(const void* kernel, int block, size_t smem, int device)
 
 cudaError_t allow_dynamic_smem(const void* kernel, size_t smem, int device)
 {
+    // The opt-in is one value per kernel, so it is raised once per kernel and
+    // device to the device's whole opt-in limit; any later launch with a
+    // smaller ring then stays within it.  (Setting it to each launch's own
+    // size would lower it under a later, larger launch.)
     if (smem <= 48 * 1024)
         return cudaSuccess;
     struct Key {
         const void* k;
-        size_t smem;
         int dev;
-        bool operator==(const Key& o) const { return k == o.k && smem == o.smem && dev == o.dev; }
+        bool operator==(const Key& o) const { return k == o.k && dev == o.dev; }
     };
     struct Hash {
-        size_t operator()(const Key& x) const
-        {
-            return std::hash<const void*>()(x.k) ^ (x.smem << 7) ^ size_t(x.dev);
-        }
+        size_t operator()(const Key& x) const { return std::hash<const void*>()(x.k) ^ size_t(x.dev); }
     };
     static std::mutex mu;
-    static std::unordered_map<Key, bool, Hash> done;
+    static std::unordered_map<Key, int, Hash> limit;
     std::lock_guard<std::mutex> lock(mu);
-    const Key key{kernel, smem, device};
-    if (done.count(key))
-        return cudaSuccess;
-    const cudaError_t err =
-        cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
+    const Key key{kernel, device};
+    auto it = limit.find(key);
+    if (it != limit.end())
+        return smem <= size_t(it->second) ? cudaSuccess : cudaErrorInvalidValue;
+    int optin = 0;
+    cudaError_t err = cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, device);
+    if (err != cudaSuccess)
+        return err;
+    if (smem > size_t(optin))
+        return cudaErrorInvalidValue;
+    err = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, optin);
     if (err == cudaSuccess)
-        done.emplace(key, true);
+        limit.emplace(key, optin);
     return err;
 }
 

@@ -363,7 +363,13 @@ struct KernelChoice {
     int rows_per_cta_iter = 1;
     size_t smem = 0;
     int variant = H3_VARIANT_NONE;
+    int per_sm = 0;  // default resident CTAs per SM (0: as many as fit)
 };
+
+// The 32-byte vector kernels keep 4 CTAs per SM by default: on B200 that
+// measured faster than full occupancy in both directions on the 32k-, 128k-
+// and 250k-token H3 workloads (more CTAs in flight lowered DRAM efficiency).
+constexpr int kWideCtasPerSm = 4;
 
 // Smallest instantiated vectors-per-thread count (at most MAXV) covering `need`.
 template <bool S2H, int VW, int NT, int ROWS, int MAXV>
@@ -401,8 +407,10 @@ void choose_vec(const RelayoutArgs& a, bool wide_ok, KernelChoice* kc)
         const int row32 = a.row_vecs / 2;
         const bool ok = S2H ? pick_vec<true, 32, 64, 2, 8>((row32 + 63) / 64, kc)
                             : pick_vec<false, 32, 32, 1, 16>((row32 + 31) / 32, kc);
-        if (ok)
+        if (ok) {
+            kc->per_sm = kWideCtasPerSm;
             return;
+        }
     }
     if (pick_vec<S2H, 16, 128, 1, 16>((a.row_vecs + 127) / 128, kc))
         return;
@@ -456,9 +464,8 @@ cudaError_t launch_relayout(bool seq_to_head, const RelayoutArgs& a, int variant
     if (sms <= 0)
         return cudaErrorNoDevice;
     KernelChoice kc;
-    // Default: the bulk kernel for head->sequence with at most four ranks
-    // (fastest measured there), the vector kernels otherwise.
-    const bool want_bulk = variant == H3_VARIANT_BULK || (variant == 0 && !seq_to_head && a.W <= 4);
+    // Default: the vector kernels; the bulk kernel only when asked for.
+    const bool want_bulk = variant == H3_VARIANT_BULK;
     bool bulk = false;
     if (want_bulk)
         bulk = choose_bulk(seq_to_head, a, device, &kc);
@@ -474,7 +481,8 @@ cudaError_t launch_relayout(bool seq_to_head, const RelayoutArgs& a, int variant
         if (err != cudaSuccess)
             return err;
     }
-    const int per_sm = ctas_per_sm > 0 ? ctas_per_sm : resident_ctas(kc.fn, kc.threads, kc.smem, device);
+    const int fit = resident_ctas(kc.fn, kc.threads, kc.smem, device);
+    int per_sm = ctas_per_sm > 0 ? ctas_per_sm : (kc.per_sm > 0 && kc.per_sm < fit ? kc.per_sm : fit);
     const int64_t needed = (int64_t(a.rows) + kc.rows_per_cta_iter - 1) / kc.rows_per_cta_iter;
     int64_t grid = int64_t(sms) * per_sm;
     if (grid > needed)

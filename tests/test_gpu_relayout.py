@@ -114,15 +114,36 @@ def test_bulk_rejects_rows_too_wide_for_its_ring():
     assert info["variant"] == rr.H3_VARIANT_VECTOR
 
 
+def test_bulk_ring_sizes_alternate(oracle_lib):
+    """Bulk launches whose shared-memory rings differ in size, in both orders
+    (a smaller ring must not shrink what a later, larger one may use)."""
+    for T, P, H, D, W in [(40, 3, 24, 128, 3), (64, 3, 56, 128, 2), (40, 3, 24, 128, 3),
+                          (64, 3, 56, 128, 4), (130, 2, 7, 64, 3), (64, 3, 56, 128, 2)]:
+        full, send, part = _seq_inputs(T, P, H, D, W, seed=T + H + W)
+        recv = rr.alloc_head_side(T, P, H, D, W, DEV)
+        rr.seq_to_head(send, recv, variant=rr.H3_VARIANT_BULK)
+        back_full, back = rr.alloc_seq_side(T, P, H, D, W, DEV)
+        rr.head_to_seq(recv, back, variant=rr.H3_VARIANT_BULK)
+        assert gu.same_bits(back_full, full)
+        want = oracle_lib.seq_to_head([gu.bits(s) for s in send], T, P, H, D, W)
+        for j in range(W):
+            assert np.array_equal(gu.bits(recv[j]), want[j])
+
+
 def test_default_variants():
-    """Defaults: vectors for seq->head, the bulk ring for head->seq at W <= 4."""
-    for W, want_back in [(2, rr.H3_VARIANT_BULK), (4, rr.H3_VARIANT_BULK), (6, rr.H3_VARIANT_VECTOR)]:
+    """Defaults: the vector kernels in both directions, 4 CTAs per SM for the
+    32-byte H3 shapes; the bulk ring only when asked for."""
+    for W, want_back in [(2, rr.H3_VARIANT_VECTOR), (4, rr.H3_VARIANT_VECTOR), (6, rr.H3_VARIANT_VECTOR)]:
         T, P, H, D = 300, 3, 56, 128
         full, send, part = _seq_inputs(T, P, H, D, W, seed=W)
         recv = rr.alloc_head_side(T, P, H, D, W, DEV)
-        assert rr.seq_to_head(send, recv)["variant"] == rr.H3_VARIANT_VECTOR
+        info = rr.seq_to_head(send, recv)
+        assert info["variant"] == rr.H3_VARIANT_VECTOR
+        sms = torch.cuda.get_device_properties(0).multi_processor_count
+        assert info["grid"] == min(4 * sms, (T * P + 1) // 2)
         back_full, back = rr.alloc_seq_side(T, P, H, D, W, DEV)
-        assert rr.head_to_seq(recv, back)["variant"] == want_back
+        info = rr.head_to_seq(recv, back)
+        assert info["variant"] == want_back and info["grid"] == min(4 * sms, T * P)
         assert gu.same_bits(back_full, full)
 
 
