@@ -551,6 +551,19 @@ def run_workload_report(args):
             emit(w.name, "head_to_seq", vname, nbytes, secs, info)
             if not torch.equal(back_full.view(torch.int16), x.view(torch.int16)):
                 raise SystemExit(f"{w.name} {vname}: round trip differs")
+        if w.T >= 32768:
+            # staged through the pages' 896,000,000-byte window: every byte
+            # crosses HBM twice, GB/s still counts the algorithmic bytes once
+            win = torch.empty(min(WINDOW, 2 * x.numel()), dtype=torch.uint8, device=dev)
+            info = rr.seq_to_head_staged(send, heads, win)
+            secs = _time_calls(lambda: rr.seq_to_head_staged(send, heads, win), max(3, iters // 4))
+            emit(w.name, "seq_to_head", "staged_896MB", nbytes, secs, info)
+            info = rr.head_to_seq_staged(heads, back, win)
+            secs = _time_calls(lambda: rr.head_to_seq_staged(heads, back, win), max(3, iters // 4))
+            emit(w.name, "head_to_seq", "staged_896MB", nbytes, secs, info)
+            if not torch.equal(back_full.view(torch.int16), x.view(torch.int16)):
+                raise SystemExit(f"{w.name} staged: round trip differs")
+            del win
         if w.inverse_planes:
             # head->seq on the attention output [T, 1, H, D]
             del heads, back_full, back

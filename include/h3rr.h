@@ -83,6 +83,7 @@ typedef enum h3_status {
 #define H3_VARIANT_VECTOR 1      /* 16-byte vector loads/stores through registers */
 #define H3_VARIANT_BULK 2        /* bulk async copies through shared memory */
 #define H3_VARIANT_REDUCE 3      /* warp-level fp32 reduce-scatter */
+#define H3_VARIANT_STAGED 4      /* pack into a window buffer, then unpack */
 
 typedef struct h3_exec_info {
     int32_t launches;            /* kernel launches enqueued by the call */
@@ -216,6 +217,47 @@ H3RR_API h3_status h3_ragged_reduce_scatter_ex(const void* const* partials, cons
                                       void* const* out, int64_t n_tokens, int64_t cols,
                                       int32_t world, void* stream,
                                       const h3_launch_config* cfg, h3_exec_info* info);
+
+/*
+ * h3_seq_to_head_staged / h3_head_to_seq_staged - the same relayouts staged
+ * through a caller-provided window buffer, the way a registered-window
+ * transport moves them (FastVideo PR #1807, "Problem and behavior": one
+ * batch plane at a time through a window of at most 896,000,000 bytes).
+ *
+ * Work is cut into chunks of one plane and at most
+ * floor(window_bytes / (H*D*2)) tokens; each chunk is packed into `window`
+ * (head-side rank j's block [n, H_j, D] at byte offset n*hs_j*D*2) and then
+ * unpacked into the outputs: two launches per chunk, every byte read and
+ * written twice.  Planes larger than the window are therefore split by
+ * tokens.  The results equal h3_seq_to_head / h3_head_to_seq bit for bit.
+ *
+ *   window       : device scratch, caller-owned, 16-byte aligned, at least
+ *                  one token row (H*D*2 bytes); must not overlap any input or
+ *                  output; its contents on return are unspecified.  Calls that
+ *                  share one window must not overlap in time.
+ *   window_bytes : usable bytes of window (>= H*D*2, else H3_ERR_WINDOW).
+ *   Other arguments, layouts and errors as h3_seq_to_head / h3_head_to_seq.
+ */
+H3RR_API h3_status h3_seq_to_head_staged(const void* const* send, void* const* recv,
+                                         int64_t n_tokens, int32_t planes, int32_t n_heads,
+                                         int32_t head_dim, int32_t world, void* window,
+                                         int64_t window_bytes, void* stream, h3_exec_info* info);
+H3RR_API h3_status h3_head_to_seq_staged(const void* const* send, void* const* recv,
+                                         int64_t n_tokens, int32_t planes, int32_t n_heads,
+                                         int32_t head_dim, int32_t world, void* window,
+                                         int64_t window_bytes, void* stream, h3_exec_info* info);
+
+/*
+ * h3_staged_plan - host only: the chunking the staged calls use.
+ *   chunk_tokens : out, tokens per chunk (the last chunk of a plane may hold fewer).
+ *   chunks       : out, chunks in all (planes * ceil(T / chunk_tokens)); the
+ *                  staged calls enqueue 2 * chunks launches.
+ * Returns H3_ERR_WINDOW if window_bytes < H*D*2, H3_ERR_INVALID_ARG on
+ * non-positive sizes or NULL outputs.
+ */
+H3RR_API h3_status h3_staged_plan(int64_t n_tokens, int32_t planes, int32_t n_heads,
+                                  int32_t head_dim, int64_t window_bytes,
+                                  int64_t* chunk_tokens, int64_t* chunks);
 
 /*
  * h3_bulk_wait_timeouts - how many bounded waits of the bulk relayout kernel

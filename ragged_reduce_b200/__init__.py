@@ -26,13 +26,14 @@ import torch
 
 from . import _abi
 from ._abi import (ExecInfo, H3Error, LaunchConfig, H3_VARIANT_BULK, H3_VARIANT_REDUCE,
-                   H3_VARIANT_VECTOR, MAX_WORLD)
+                   H3_VARIANT_STAGED, H3_VARIANT_VECTOR, MAX_WORLD)
 
 __all__ = [
     "H3Error", "Partition", "partition", "seq_to_head", "head_to_seq",
     "ragged_reduce_scatter", "alloc_head_side", "alloc_seq_side", "split_rows",
     "H3_VARIANT_VECTOR", "H3_VARIANT_BULK", "H3_VARIANT_REDUCE", "MAX_WORLD", "library_path",
-    "bulk_wait_timeouts", "alloc_reduce_outputs",
+    "bulk_wait_timeouts", "alloc_reduce_outputs", "seq_to_head_staged", "head_to_seq_staged",
+    "staged_plan", "H3_VARIANT_STAGED",
 ]
 
 library_path = _abi.LIB_PATH
@@ -147,6 +148,72 @@ def _config(variant: int, ctas_per_sm: int):
     if not variant and not ctas_per_sm:
         return None
     return C.byref(LaunchConfig(int(variant), int(ctas_per_sm), 0, 0))
+
+
+def _relayout_shapes(seq_to_head_dir: bool, send, recv):
+    """Check the per-rank shapes; return (T, P, H, D, W, device)."""
+    W = len(send)
+    if W < 1 or len(recv) != W:
+        raise ValueError("send and recv need one tensor per rank (same count)")
+    dev = _check_tensors(send + recv, "relayout")
+    seq_side = send if seq_to_head_dir else recv
+    head_side = recv if seq_to_head_dir else send
+    if any(t.dim() != 4 for t in send + recv):
+        raise ValueError("relayout buffers are 4-D: [tokens, planes, heads, head_dim]")
+    _, P, H, D = seq_side[0].shape
+    T = sum(int(t.shape[0]) for t in seq_side)
+    part = partition(T, H, W)
+    for r, t in enumerate(seq_side):
+        if tuple(t.shape) != (part.tokens(r), P, H, D):
+            raise ValueError(f"sequence-side rank {r}: shape {tuple(t.shape)}, "
+                             f"expected {(part.tokens(r), P, H, D)}")
+    for j, t in enumerate(head_side):
+        if tuple(t.shape) != (T, P, part.heads(j), D):
+            raise ValueError(f"head-side rank {j}: shape {tuple(t.shape)}, "
+                             f"expected {(T, P, part.heads(j), D)}")
+    return T, int(P), int(H), int(D), W, dev
+
+
+def _relayout_staged(seq_to_head_dir: bool, send, recv, window, stream):
+    send = _as_list(send)
+    recv = _as_list(recv)
+    T, P, H, D, W, dev = _relayout_shapes(seq_to_head_dir, send, recv)
+    _check_tensors([window], "window", itemsize=window.element_size())
+    if window.device != dev:
+        raise ValueError("window must be on the buffers' device")
+    nbytes = window.numel() * window.element_size()
+    info = ExecInfo()
+    name = "h3_seq_to_head_staged" if seq_to_head_dir else "h3_head_to_seq_staged"
+    with torch.cuda.device(dev):
+        st = getattr(_abi.lib, name)(
+            _abi.pointer_array([t.data_ptr() for t in send]),
+            _abi.pointer_array([t.data_ptr() for t in recv]),
+            T, P, H, D, W, C.c_void_p(window.data_ptr()), int(nbytes),
+            C.c_void_p(_stream_handle(stream, dev)), C.byref(info))
+    _abi.check(st, name)
+    return info.as_dict()
+
+
+def seq_to_head_staged(send, recv, window: torch.Tensor, *, stream=None) -> dict:
+    """seq->head staged through a window buffer (any contiguous CUDA tensor;
+    its byte size is the window): chunks of one plane and as many tokens as
+    fit, packed into the window and unpacked.  Same result as ``seq_to_head``."""
+    return _relayout_staged(True, send, recv, window, stream)
+
+
+def head_to_seq_staged(send, recv, window: torch.Tensor, *, stream=None) -> dict:
+    """head->seq staged through a window buffer (see ``seq_to_head_staged``)."""
+    return _relayout_staged(False, send, recv, window, stream)
+
+
+def staged_plan(n_tokens: int, planes: int, n_heads: int, head_dim: int, window_bytes: int):
+    """(tokens per chunk, chunks) of a staged call (``h3_staged_plan``, host only)."""
+    n = C.c_int64(0)
+    k = C.c_int64(0)
+    st = _abi.lib.h3_staged_plan(int(n_tokens), int(planes), int(n_heads), int(head_dim),
+                                 int(window_bytes), C.byref(n), C.byref(k))
+    _abi.check(st, "h3_staged_plan")
+    return int(n.value), int(k.value)
 
 
 def _relayout(seq_to_head_dir: bool, send, recv, window_bytes, stream, variant, ctas_per_sm):

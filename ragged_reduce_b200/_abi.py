@@ -35,6 +35,7 @@ H3_VARIANT_NONE = 0
 H3_VARIANT_VECTOR = 1
 H3_VARIANT_BULK = 2
 H3_VARIANT_REDUCE = 3
+H3_VARIANT_STAGED = 4
 
 MAX_WORLD = 64
 ABI_VERSION = 1
@@ -113,6 +114,14 @@ def _load() -> C.CDLL:
     lib.h3_ragged_reduce_scatter_ex.restype = C.c_int
     lib.h3_ragged_reduce_scatter_ex.argtypes = _REDUCE_ARGS + [C.POINTER(LaunchConfig),
                                                                C.POINTER(ExecInfo)]
+    for name in ("h3_seq_to_head_staged", "h3_head_to_seq_staged"):
+        f = getattr(lib, name)
+        f.restype = C.c_int
+        f.argtypes = [_vpp, _vpp, C.c_int64, C.c_int32, C.c_int32, C.c_int32, C.c_int32,
+                      C.c_void_p, C.c_int64, C.c_void_p, C.POINTER(ExecInfo)]
+    lib.h3_staged_plan.restype = C.c_int
+    lib.h3_staged_plan.argtypes = [C.c_int64, C.c_int32, C.c_int32, C.c_int32, C.c_int64,
+                                   _i64p, _i64p]
     lib.h3_last_cuda_error.restype = C.c_int32
     lib.h3_last_cuda_error.argtypes = [C.POINTER(C.c_char_p)]
     lib.h3_bulk_wait_timeouts.restype = C.c_int

@@ -178,9 +178,170 @@ h3_status relayout(bool seq_to_head, const void* const* send, void* const* recv,
     return H3_OK;
 }
 
+// Shared checks of the relayout calls: world, shapes, pointers, alignment,
+// overlap.  `extra_out` (nullable) is one more output range (the window).
+h3_status check_relayout_args(bool seq_to_head, const void* const* send, void* const* recv,
+                              int64_t n_tokens, int32_t planes, int32_t n_heads, int32_t head_dim,
+                              int32_t world, void* extra_out, uint64_t extra_bytes)
+{
+    h3_status st = check_world(n_tokens, n_heads, world);
+    if (st != H3_OK)
+        return st;
+    if (planes < 1 || head_dim < 1 || !send || !recv)
+        return H3_ERR_INVALID_ARG;
+    if ((int64_t(head_dim) * 2) % kVecBytes != 0)
+        return H3_ERR_MISALIGNED;
+    if (n_tokens > kMaxInt32 || n_tokens * planes > kMaxInt32 ||
+        int64_t(n_heads) * head_dim * 2 / kVecBytes > kMaxRowVecs)
+        return H3_ERR_UNSUPPORTED;
+    const Split ts = make_split(n_tokens, world);
+    const Split hs = make_split(n_heads, world);
+    const uint64_t row_bytes = uint64_t(n_heads) * head_dim * 2;
+    const uint64_t head_bytes = uint64_t(head_dim) * 2;
+    uint64_t seq_bytes[kMaxWorld];
+    uint64_t head_side_bytes[kMaxWorld + 1];
+    void* outs[kMaxWorld + 1];
+    for (int r = 0; r < world; ++r) {
+        if (!send[r] || !recv[r])
+            return H3_ERR_INVALID_ARG;
+        if (!aligned16(send[r]) || !aligned16(recv[r]))
+            return H3_ERR_MISALIGNED;
+        seq_bytes[r] = uint64_t(ts.size(r)) * planes * row_bytes;
+        head_side_bytes[r] = uint64_t(n_tokens) * planes * uint64_t(hs.size(r)) * head_bytes;
+    }
+    const uint64_t* in_bytes = seq_to_head ? seq_bytes : head_side_bytes;
+    uint64_t out_bytes[kMaxWorld + 1];
+    for (int r = 0; r < world; ++r) {
+        outs[r] = recv[r];
+        out_bytes[r] = seq_to_head ? head_side_bytes[r] : seq_bytes[r];
+    }
+    int n_out = world;
+    if (extra_out) {
+        outs[n_out] = extra_out;
+        out_bytes[n_out] = extra_bytes;
+        ++n_out;
+    }
+    return check_no_overlap(send, in_bytes, world, outs, out_bytes, n_out);
+}
+
+h3_status staged_plan(int64_t n_tokens, int32_t n_heads, int32_t head_dim, int64_t window_bytes,
+                      int64_t* chunk_tokens)
+{
+    const int64_t row_bytes = int64_t(n_heads) * head_dim * 2;
+    if (row_bytes <= 0)
+        return H3_ERR_INVALID_ARG;
+    if (window_bytes < row_bytes)
+        return H3_ERR_WINDOW;
+    int64_t n = window_bytes / row_bytes;
+    if (n > n_tokens)
+        n = n_tokens;
+    *chunk_tokens = n;
+    return H3_OK;
+}
+
+h3_status relayout_staged(bool seq_to_head, const void* const* send, void* const* recv,
+                          int64_t n_tokens, int32_t planes, int32_t n_heads, int32_t head_dim,
+                          int32_t world, void* window, int64_t window_bytes, void* stream,
+                          h3_exec_info* info)
+{
+    clear_info(info);
+    if (!window || window_bytes < 0)
+        return H3_ERR_INVALID_ARG;
+    if (!aligned16(window))
+        return H3_ERR_MISALIGNED;
+    h3_status st = check_relayout_args(seq_to_head, send, recv, n_tokens, planes, n_heads, head_dim,
+                                       world, window, uint64_t(window_bytes));
+    if (st != H3_OK)
+        return st;
+    int64_t chunk_tokens = 0;
+    st = staged_plan(n_tokens, n_heads, head_dim, window_bytes, &chunk_tokens);
+    if (st != H3_OK)
+        return st;
+    const Split ts = make_split(n_tokens, world);
+    const Split hs = make_split(n_heads, world);
+    StagedArgs a;
+    std::memset(&a, 0, sizeof(a));
+    for (int r = 0; r < world; ++r) {
+        char* s = const_cast<char*>(static_cast<const char*>(send[r]));
+        char* d = static_cast<char*>(recv[r]);
+        a.seq[r] = seq_to_head ? s : d;
+        a.head[r] = seq_to_head ? d : s;
+    }
+    a.window = static_cast<char*>(window);
+    a.T = int32_t(n_tokens);
+    a.P = planes;
+    a.W = world;
+    a.tq = int32_t(ts.q);
+    a.tm = int32_t(ts.m);
+    a.hq = int32_t(hs.q);
+    a.hm = int32_t(hs.m);
+    a.row_vecs = int32_t(int64_t(n_heads) * head_dim * 2 / kVecBytes);
+    a.head_vecs = int32_t(int64_t(head_dim) * 2 / kVecBytes);
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    LaunchShape shape;
+    int chunks = 0;
+    for (int32_t p = 0; p < planes; ++p) {
+        for (int64_t t0 = 0; t0 < n_tokens; t0 += chunk_tokens) {
+            a.p = p;
+            a.t0 = int32_t(t0);
+            a.n = int32_t(n_tokens - t0 < chunk_tokens ? n_tokens - t0 : chunk_tokens);
+            const cudaError_t err = launch_staged_chunk(seq_to_head, a, s, &shape);
+            if (err != cudaSuccess) {
+                if (info) {
+                    info->launches = 2 * chunks;
+                    info->chunks = chunks;
+                }
+                return cuda_failure(err);
+            }
+            ++chunks;
+        }
+    }
+    if (info) {
+        info->launches = 2 * chunks;
+        info->chunks = chunks;
+        info->grid = shape.grid;
+        info->block = shape.block;
+        info->variant = shape.variant;
+        info->planes_per_launch = 1;
+    }
+    return H3_OK;
+}
+
 }  // namespace
 
 extern "C" {
+
+h3_status h3_seq_to_head_staged(const void* const* send, void* const* recv, int64_t n_tokens,
+                                int32_t planes, int32_t n_heads, int32_t head_dim, int32_t world,
+                                void* window, int64_t window_bytes, void* stream, h3_exec_info* info)
+{
+    return relayout_staged(true, send, recv, n_tokens, planes, n_heads, head_dim, world, window,
+                           window_bytes, stream, info);
+}
+
+h3_status h3_head_to_seq_staged(const void* const* send, void* const* recv, int64_t n_tokens,
+                                int32_t planes, int32_t n_heads, int32_t head_dim, int32_t world,
+                                void* window, int64_t window_bytes, void* stream, h3_exec_info* info)
+{
+    return relayout_staged(false, send, recv, n_tokens, planes, n_heads, head_dim, world, window,
+                           window_bytes, stream, info);
+}
+
+h3_status h3_staged_plan(int64_t n_tokens, int32_t planes, int32_t n_heads, int32_t head_dim,
+                         int64_t window_bytes, int64_t* chunk_tokens, int64_t* chunks)
+{
+    if (!chunk_tokens || !chunks || n_tokens < 1 || planes < 1 || n_heads < 1 || head_dim < 1 ||
+        window_bytes < 0)
+        return H3_ERR_INVALID_ARG;
+    int64_t n = 0;
+    const h3_status st = staged_plan(n_tokens, n_heads, head_dim, window_bytes, &n);
+    if (st != H3_OK)
+        return st;
+    *chunk_tokens = n;
+    *chunks = int64_t(planes) * ((n_tokens + n - 1) / n);
+    return H3_OK;
+}
+
 
 int32_t h3_abi_version(void) { return H3RR_ABI_VERSION; }
 
@@ -198,7 +359,7 @@ const char* h3_status_string(h3_status status)
         case H3_ERR_INVALID_ARG: return "invalid argument";
         case H3_ERR_EMPTY_PARTITION: return "empty token or head partition";
         case H3_ERR_MISALIGNED: return "pointer or run not 16-byte aligned";
-        case H3_ERR_WINDOW: return "one plane does not fit in the byte window";
+        case H3_ERR_WINDOW: return "the data of one launch does not fit in the byte window";
         case H3_ERR_UNSUPPORTED: return "unsupported size or world";
         case H3_ERR_CUDA: return "CUDA launch error";
     }

@@ -68,6 +68,24 @@ struct ReduceArgs {
     int64_t row_bytes;            // C * 2
 };
 
+// One chunk of a staged relayout: tokens [t0, t0 + n) of plane p, packed into
+// `window` head-rank-major (rank j's block [n, H_j, D] at n * hs_j heads).
+struct StagedArgs {
+    char* seq[kMaxWorld];
+    char* head[kMaxWorld];
+    char* window;
+    int32_t T;
+    int32_t P;
+    int32_t W;
+    int32_t p;
+    int32_t t0;
+    int32_t n;
+    int32_t tq, tm;
+    int32_t hq, hm;
+    int32_t row_vecs;
+    int32_t head_vecs;
+};
+
 struct LaunchShape {
     int grid = 0;
     int block = 0;
@@ -83,6 +101,10 @@ bool relayout_bulk_fits(const RelayoutArgs& a, int device);
 
 // Copy (and optionally clear) the per-device count of expired bulk waits.
 cudaError_t read_bulk_wait_timeouts(unsigned int* count, bool reset, cudaStream_t stream);
+
+// Enqueue the two launches (pack, unpack) of one staged chunk.
+cudaError_t launch_staged_chunk(bool seq_to_head, const StagedArgs& a, cudaStream_t stream,
+                                LaunchShape* shape);
 
 // Enqueue the reduce-scatter launch.
 cudaError_t launch_reduce_scatter(const ReduceArgs& a, int ctas_per_sm, cudaStream_t stream,

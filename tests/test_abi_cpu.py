@@ -263,3 +263,49 @@ def test_binding_rejects_host_tensors():
     with pytest.raises(ValueError):
         rr.ragged_reduce_scatter([torch.zeros(4, 8, dtype=torch.bfloat16)], None,
                                  [torch.zeros(4, 8, dtype=torch.bfloat16)])
+
+
+# ---------------------------------------------------------------------------
+# staged relayouts: plan and argument checks
+# ---------------------------------------------------------------------------
+
+def test_staged_plan_values():
+    row = 56 * 128 * 2
+    assert rr.staged_plan(32768, 3, 56, 128, 896_000_000) == (32768, 3)
+    assert rr.staged_plan(250000, 4, 56, 128, 896_000_000) == (62500, 16)
+    assert rr.staged_plan(1000, 3, 56, 128, 7 * row + 100) == (7, 3 * 143)
+    assert rr.staged_plan(5, 2, 56, 128, 10 * row) == (5, 2)
+    with pytest.raises(rr.H3Error) as e:
+        rr.staged_plan(10, 3, 56, 128, row - 16)
+    assert e.value.status == _abi.H3_ERR_WINDOW
+    with pytest.raises(rr.H3Error) as e:
+        rr.staged_plan(0, 3, 56, 128, row)
+    assert e.value.status == _abi.H3_ERR_INVALID_ARG
+
+
+@needs_no_gpu
+@pytest.mark.parametrize("fn", ["h3_seq_to_head_staged", "h3_head_to_seq_staged"])
+def test_staged_argument_checks(fn):
+    T, P, H, D, W = 1000, 3, 56, 128, 6
+    send, recv = _layout(T, P, H, D, W)
+    if fn == "h3_head_to_seq_staged":
+        send, recv = recv, send
+    window = BASE - (1 << 30)
+    row = H * D * 2
+    E = _abi
+
+    def st(window=window, wbytes=64 * row, send=send, recv=recv, W=W, T=T):
+        info = _abi.ExecInfo()
+        s = getattr(_abi.lib, fn)(_ptrs(send), _ptrs(recv), T, P, H, D, W, C.c_void_p(window),
+                                  wbytes, None, C.byref(info))
+        assert info.launches == 0
+        return s
+
+    assert st(window=0) == E.H3_ERR_INVALID_ARG
+    assert st(window=window + 8) == E.H3_ERR_MISALIGNED
+    assert st(wbytes=row - 16) == E.H3_ERR_WINDOW
+    assert st(wbytes=-1) == E.H3_ERR_INVALID_ARG
+    assert st(window=send[2] + 4096) == E.H3_ERR_INVALID_ARG       # window over an input
+    assert st(window=recv[0] - 1024, wbytes=4096) == E.H3_ERR_INVALID_ARG  # over an output
+    assert st(W=0) == E.H3_ERR_INVALID_ARG
+    assert st(T=5) == E.H3_ERR_EMPTY_PARTITION
