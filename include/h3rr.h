@@ -248,6 +248,44 @@ H3RR_API h3_status h3_head_to_seq_staged(const void* const* send, void* const* r
                                          int64_t window_bytes, void* stream, h3_exec_info* info);
 
 /*
+ * h3_seq_to_head_staged_noalloc - h3_seq_to_head_staged with a window that
+ * lives inside the library, so the call allocates no device memory at all.
+ * The pages have no counterpart to this entry point; it exists for callers
+ * that cannot allocate device memory themselves: for example a plugin that
+ * only receives tensors from a host framework whose caching allocator owns
+ * the whole memory budget, or a latency-critical loop in which cudaMalloc
+ * or cudaFree would synchronise the device.  Such callers still pass their
+ * inputs and outputs; only the staging window is provided here.
+ *
+ * The window is a file-scope device array of H3RR_STATIC_WINDOW_BYTES
+ * (16 MiB).  Every GPU that loads the library holds that array until the
+ * process exits.  The call neither allocates nor frees device memory, and
+ * calls no allocating library routine.
+ *
+ *   window_bytes : how much of the array to use, 0 = all of it.  Values
+ *                  above H3RR_STATIC_WINDOW_BYTES (or negative) are rejected
+ *                  with H3_ERR_UNSUPPORTED before anything is launched; a
+ *                  window smaller than one token row (H*D*2 bytes) is
+ *                  H3_ERR_WINDOW.
+ *   Other arguments, layouts, results and errors as h3_seq_to_head_staged.
+ *
+ * The first call on a device looks up the array's device address (one
+ * cudaGetSymbolAddress with that device current, kept for later calls); make
+ * that first call before any stream capture.  Every call on a device shares
+ * the one array and leaves its last chunk in it: nothing in it needs to
+ * start at zero, because each chunk is written in full before it is read.
+ * Calls that overlap on the GPU (for example on two streams without ordering
+ * between them) race on the array and corrupt each other's output; order
+ * them on one stream or with events.
+ */
+#define H3RR_STATIC_WINDOW_BYTES (16ll << 20)
+H3RR_API h3_status h3_seq_to_head_staged_noalloc(const void* const* send, void* const* recv,
+                                                 int64_t n_tokens, int32_t planes,
+                                                 int32_t n_heads, int32_t head_dim, int32_t world,
+                                                 int64_t window_bytes, void* stream,
+                                                 h3_exec_info* info);
+
+/*
  * h3_staged_plan - host only: the chunking the staged calls use.
  *   chunk_tokens : out, tokens per chunk (the last chunk of a plane may hold fewer).
  *   chunks       : out, chunks in all (planes * ceil(T / chunk_tokens)); the

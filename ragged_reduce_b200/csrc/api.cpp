@@ -309,6 +309,21 @@ h3_status relayout_staged(bool seq_to_head, const void* const* send, void* const
 
 }  // namespace
 
+namespace h3rr {
+
+h3_status staged_relayout_with_window(bool seq_to_head, const void* const* send, void* const* recv,
+                                      int64_t n_tokens, int32_t planes, int32_t n_heads,
+                                      int32_t head_dim, int32_t world, void* window,
+                                      int64_t window_bytes, void* stream, h3_exec_info* info)
+{
+    return relayout_staged(seq_to_head, send, recv, n_tokens, planes, n_heads, head_dim, world,
+                           window, window_bytes, stream, info);
+}
+
+h3_status record_cuda_failure(cudaError_t err) { return cuda_failure(err); }
+
+}  // namespace h3rr
+
 extern "C" {
 
 h3_status h3_seq_to_head_staged(const void* const* send, void* const* recv, int64_t n_tokens,

@@ -106,6 +106,15 @@ cudaError_t read_bulk_wait_timeouts(unsigned int* count, bool reset, cudaStream_
 cudaError_t launch_staged_chunk(bool seq_to_head, const StagedArgs& a, cudaStream_t stream,
                                 LaunchShape* shape);
 
+// The staged relayout on a given window (checks, plan and launches).
+h3_status staged_relayout_with_window(bool seq_to_head, const void* const* send, void* const* recv,
+                                      int64_t n_tokens, int32_t planes, int32_t n_heads,
+                                      int32_t head_dim, int32_t world, void* window,
+                                      int64_t window_bytes, void* stream, h3_exec_info* info);
+
+// Record `err` as the calling thread's last CUDA error; returns H3_ERR_CUDA.
+h3_status record_cuda_failure(cudaError_t err);
+
 // Enqueue the reduce-scatter launch.
 cudaError_t launch_reduce_scatter(const ReduceArgs& a, int ctas_per_sm, cudaStream_t stream,
                                   LaunchShape* shape);
