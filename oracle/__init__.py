@@ -62,6 +62,9 @@ class Oracle:
             f.restype = C.c_int32
             f.argtypes = [C.c_int64, C.c_int32, C.c_int32, C.c_int32, C.c_int32,
                           C.c_int32, C.c_int64, _i64p, _i32p, _i64p]
+        lib.h3o_ragged_all_gather.restype = C.c_int32
+        lib.h3o_ragged_all_gather.argtypes = [C.c_void_p, C.c_void_p, C.c_int64, C.c_int64,
+                                              C.c_int32]
         lib.h3o_reduce_rows.restype = None
         lib.h3o_reduce_rows.argtypes = [C.c_void_p, C.c_void_p, _u16p, C.c_int64,
                                         C.c_int64, C.c_int32]
@@ -174,6 +177,20 @@ class Oracle:
         rc = self.lib.h3o_ragged_reduce_scatter(_ptr_array(src),
                                                 None if b is None else b.ctypes.data,
                                                 _ptr_array(out), T, Cc, W)
+        assert rc == 0
+        return out
+
+    def ragged_all_gather(self, blocks, W: int):
+        """blocks: W uint16 arrays [T_r, C] -> W arrays [T, C] (every rank gets all rows)."""
+        src = [np.ascontiguousarray(b, dtype=np.uint16) for b in blocks]
+        assert len(src) == W
+        Cc = src[0].shape[1]
+        T = sum(b.shape[0] for b in src)
+        ts = self.partition_range(T, W)
+        for r, b in enumerate(src):
+            assert b.shape == (ts[r + 1] - ts[r], Cc)
+        out = [np.zeros((T, Cc), dtype=np.uint16) for _ in range(W)]
+        rc = self.lib.h3o_ragged_all_gather(_ptr_array(src), _ptr_array(out), T, Cc, W)
         assert rc == 0
         return out
 

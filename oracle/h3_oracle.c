@@ -379,3 +379,35 @@ done:
     free(vals);
     return rc;
 }
+
+/* ------------------------------------------------------------------------ */
+/* Ragged all-gather of token rows ["Distributed H3 Execution", intro: ragged */
+/* row gathering; "Validation": ragged gather and reduce-scatter behaviour]   */
+/* ------------------------------------------------------------------------ */
+
+/* Every rank receives all T rows: out[j] is [T, C], and its row t is row
+ * t - ts_r of in[r], r the rank that owns token t.  in[r] is [T_r, C].
+ * Element = one 16-bit pattern, copied as is.  Returns -1 on an empty
+ * partition. */
+int32_t h3o_ragged_all_gather(const uint16_t* const* in, uint16_t* const* out,
+                              int64_t T, int64_t C, int32_t W)
+{
+    int64_t* ts = (int64_t*)malloc(sizeof(int64_t) * (size_t)(W + 1));
+    int32_t rc = -1;
+    if (!ts)
+        goto done;
+    if (h3o_partition_range(T, W, ts))
+        goto done;
+    for (int32_t j = 0; j < W; ++j) {
+        for (int64_t t = 0; t < T; ++t) {
+            int32_t r = owner_of(ts, W, t);
+            for (int64_t c = 0; c < C; ++c)
+                out[j][t * C + c] = in[r][(t - ts[r]) * C + c];
+        }
+    }
+    rc = 0;
+done:
+    free(ts);
+    return rc;
+}
+

@@ -386,6 +386,40 @@ def check_reduce_identities(o):
     assert np.array_equal(np.concatenate(outs), x)
 
 
+def check_all_gather(o):
+    """Every rank holds all rows: numpy concatenation of the rank blocks,
+    row-number coded rows, W=1 identity, and reduce-scatter followed by
+    all-gather reproducing the unsharded integer GEMM plus bias."""
+    rng = np.random.default_rng(17)
+    for T, Cc, W in [(10, 8, 3), (97, 16, 8), (5, 8, 5), (33, 24, 1), (64, 8, 6)]:
+        full = rng.integers(0, 1 << 16, size=(T, Cc), dtype=np.uint16)
+        ts = o.partition_range(T, W)
+        blocks = [full[ts[r]:ts[r + 1]] for r in range(W)]
+        outs = o.ragged_all_gather(blocks, W)
+        for j in range(W):
+            assert np.array_equal(outs[j], np.concatenate(blocks, axis=0)), (T, W, j)
+        coded = [np.array([[_bf16_bits_of_exact(float(t))] * Cc for t in range(ts[r], ts[r + 1])],
+                          dtype=np.uint16).reshape(-1, Cc) for r in range(W)]
+        for out in o.ragged_all_gather(coded, W):
+            for t in range(T):
+                assert np.all(out[t] == _bf16_bits_of_exact(float(t)))
+    # reduce-scatter then all-gather: every rank ends with X W^T + b
+    T, K, Cc, W = 40, 12, 8, 6
+    X = rng.integers(-4, 5, size=(T, K))
+    Wt = rng.integers(-4, 5, size=(Cc, K))
+    b = rng.integers(-8, 9, size=Cc)
+    ks = o.partition_range(K, W)
+    partials = [np.array([[_bf16_bits_of_exact(float(v)) for v in row]
+                          for row in X[:, ks[w]:ks[w + 1]] @ Wt[:, ks[w]:ks[w + 1]].T], dtype=np.uint16)
+                for w in range(W)]
+    bias = np.array([_bf16_bits_of_exact(float(v)) for v in b], dtype=np.uint16)
+    gathered = o.ragged_all_gather(o.ragged_reduce_scatter(partials, bias, W), W)
+    want = np.array([[_bf16_bits_of_exact(float(v)) for v in row] for row in X @ Wt.T + b[None, :]],
+                    dtype=np.uint16)
+    for g in gathered:
+        assert np.array_equal(g, want)
+
+
 ALL_CHECKS = [
     check_head_table,
     check_partition_invariants,
@@ -401,6 +435,7 @@ ALL_CHECKS = [
     check_split_gemm,
     check_reduce_row_assignment,
     check_reduce_identities,
+    check_all_gather,
 ]
 
 

@@ -59,6 +59,10 @@ MUTANTS = [
     ("rne_ties_away", "else if (dropped == 0x8000u && (kept & 1u))", "else if (dropped == 0x8000u)"),
     ("rne_truncates", "if (dropped > 0x8000u)\n        kept", "if (dropped > 0xFFFFu)\n        kept"),
     ("nan_becomes_inf", "if (exponent == 0xFFu && mantissa != 0u)", "if (0)"),
+    ("gather_wrong_local_row", "out[j][t * C + c] = in[r][(t - ts[r]) * C + c];",
+     "out[j][t * C + c] = in[r][(t % (ts[r + 1] - ts[r])) * C + c];"),
+    ("gather_from_own_rank", "out[j][t * C + c] = in[r][(t - ts[r]) * C + c];",
+     "out[j][t * C + c] = in[j][((t - ts[r]) % (ts[j + 1] - ts[j])) * C + c];"),
     ("widen_drops_sign", "uint32_t u = ((uint32_t)b) << 16;", "uint32_t u = ((uint32_t)(b & 0x7FFFu)) << 16;"),
 ]
 
