@@ -592,6 +592,18 @@ def run_workload_report(args):
         emit(rw.name, "ragged_reduce_scatter", "default", nbytes, secs, info)
         del partials, bias, plist, out_full, out
         torch.cuda.empty_cache()
+    for (T, C_, W) in ((65536, wl.H3_HIDDEN, 8), (32768, wl.H3_HIDDEN, 6)):
+        full = wl.normal_bf16((T, C_), 9, 1.0, dev)
+        blocks = rr.split_rows(full, rr.partition(T, W, W).token_starts)
+        outs = [torch.empty((T, C_), dtype=torch.bfloat16, device=dev) for _ in range(W)]
+        nbytes = (1 + W) * T * C_ * 2
+        info = rr.ragged_all_gather(blocks, outs)
+        secs = _time_calls(lambda: rr.ragged_all_gather(blocks, outs), iters)
+        emit(f"all_gather_T{T}_C{C_}_W{W}", "ragged_all_gather", "default", nbytes, secs, info)
+        if not all(torch.equal(o.view(torch.int16), full.view(torch.int16)) for o in outs):
+            raise SystemExit("all-gather output differs")
+        del full, blocks, outs
+        torch.cuda.empty_cache()
     if rr.bulk_wait_timeouts() != 0:
         raise SystemExit("bulk kernel reported expired waits")
     return 0

@@ -84,6 +84,7 @@ typedef enum h3_status {
 #define H3_VARIANT_BULK 2        /* bulk async copies through shared memory */
 #define H3_VARIANT_REDUCE 3      /* warp-level fp32 reduce-scatter */
 #define H3_VARIANT_STAGED 4      /* pack into a window buffer, then unpack */
+#define H3_VARIANT_GATHER 5      /* ragged all-gather */
 
 typedef struct h3_exec_info {
     int32_t launches;            /* kernel launches enqueued by the call */
@@ -196,6 +197,23 @@ H3RR_API h3_status h3_head_to_seq(const void* const* send, void* const* recv,
 H3RR_API h3_status h3_ragged_reduce_scatter(const void* const* partials, const void* bias,
                                    void* const* out, int64_t n_tokens, int64_t cols,
                                    int32_t world, void* stream, h3_exec_info* info);
+
+/*
+ * h3_ragged_all_gather - ragged all-gather of token rows ("Distributed H3
+ * Execution", intro: ragged row gathering, whose temporary collective padding
+ * is removed before model operations; "Validation": ragged gather and
+ * reduce-scatter behaviour).  The companion of h3_ragged_reduce_scatter: rank
+ * r holds rows ts_r .. te_r-1, afterwards every rank holds all T rows.
+ *
+ *   in[world]  : device, rank r's rows [T_r, C], 16-bit elements (BF16).
+ *   out[world] : device, rank j's [T, C], written.
+ *   out_j[t, c] = in_{r(t)}[t - ts_{r(t)}, c]   (bit copy; nothing padded)
+ *   n_tokens T, cols C (C % 8 == 0), world W.  Errors as
+ *   h3_ragged_reduce_scatter.
+ */
+H3RR_API h3_status h3_ragged_all_gather(const void* const* in, void* const* out,
+                                        int64_t n_tokens, int64_t cols, int32_t world,
+                                        void* stream, h3_exec_info* info);
 
 /*
  * Same as h3_seq_to_head / h3_head_to_seq / h3_ragged_reduce_scatter with

@@ -25,15 +25,15 @@ import numpy as np
 import torch
 
 from . import _abi
-from ._abi import (ExecInfo, H3Error, LaunchConfig, H3_VARIANT_BULK, H3_VARIANT_REDUCE,
-                   H3_VARIANT_STAGED, H3_VARIANT_VECTOR, MAX_WORLD)
+from ._abi import (ExecInfo, H3Error, LaunchConfig, H3_VARIANT_BULK, H3_VARIANT_GATHER,
+                   H3_VARIANT_REDUCE, H3_VARIANT_STAGED, H3_VARIANT_VECTOR, MAX_WORLD)
 
 __all__ = [
     "H3Error", "Partition", "partition", "seq_to_head", "head_to_seq",
     "ragged_reduce_scatter", "alloc_head_side", "alloc_seq_side", "split_rows",
     "H3_VARIANT_VECTOR", "H3_VARIANT_BULK", "H3_VARIANT_REDUCE", "MAX_WORLD", "library_path",
     "bulk_wait_timeouts", "alloc_reduce_outputs", "seq_to_head_staged", "head_to_seq_staged",
-    "staged_plan", "H3_VARIANT_STAGED",
+    "staged_plan", "H3_VARIANT_STAGED", "ragged_all_gather", "H3_VARIANT_GATHER",
 ]
 
 library_path = _abi.LIB_PATH
@@ -326,6 +326,38 @@ def bulk_wait_timeouts(stream=None, reset: bool = False, device=None) -> int:
                                             1 if reset else 0)
     _abi.check(st, "h3_bulk_wait_timeouts")
     return int(count.value)
+
+
+def ragged_all_gather(blocks, out, *, stream=None) -> dict:
+    """Ragged all-gather of token rows: blocks are W tensors [T_r, C] (rank
+    r's rows; 2-byte elements), out W tensors [T, C], each written with all T
+    rows in token order (``h3_ragged_all_gather``)."""
+    blocks = _as_list(blocks)
+    out = _as_list(out)
+    W = len(blocks)
+    if W < 1 or len(out) != W:
+        raise ValueError("blocks and out need one tensor per rank (same count)")
+    dev = _check_tensors(blocks + out, "ragged_all_gather")
+    if any(t.dim() != 2 for t in blocks + out):
+        raise ValueError("blocks and outputs are 2-D: [tokens, cols]")
+    Cc = int(blocks[0].shape[1])
+    T = sum(int(b.shape[0]) for b in blocks)
+    if T >= W:
+        part = partition(T, W, W)
+        for r, b in enumerate(blocks):
+            if tuple(b.shape) != (part.tokens(r), Cc):
+                raise ValueError(f"block {r}: shape {tuple(b.shape)}, expected {(part.tokens(r), Cc)}")
+    for j, o in enumerate(out):
+        if tuple(o.shape) != (T, Cc):
+            raise ValueError(f"out {j}: shape {tuple(o.shape)}, expected {(T, Cc)}")
+    info = ExecInfo()
+    with torch.cuda.device(dev):
+        st = _abi.lib.h3_ragged_all_gather(_abi.pointer_array([b.data_ptr() for b in blocks]),
+                                           _abi.pointer_array([o.data_ptr() for o in out]),
+                                           T, Cc, W, C.c_void_p(_stream_handle(stream, dev)),
+                                           C.byref(info))
+    _abi.check(st, "h3_ragged_all_gather")
+    return info.as_dict()
 
 
 def alloc_reduce_outputs(T: int, C_: int, W: int, device, dtype=torch.bfloat16):

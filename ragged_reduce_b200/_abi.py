@@ -36,6 +36,7 @@ H3_VARIANT_VECTOR = 1
 H3_VARIANT_BULK = 2
 H3_VARIANT_REDUCE = 3
 H3_VARIANT_STAGED = 4
+H3_VARIANT_GATHER = 5
 
 MAX_WORLD = 64
 ABI_VERSION = 1
@@ -119,6 +120,9 @@ def _load() -> C.CDLL:
         f.restype = C.c_int
         f.argtypes = [_vpp, _vpp, C.c_int64, C.c_int32, C.c_int32, C.c_int32, C.c_int32,
                       C.c_void_p, C.c_int64, C.c_void_p, C.POINTER(ExecInfo)]
+    lib.h3_ragged_all_gather.restype = C.c_int
+    lib.h3_ragged_all_gather.argtypes = [_vpp, _vpp, C.c_int64, C.c_int64, C.c_int32, C.c_void_p,
+                                         C.POINTER(ExecInfo)]
     lib.h3_staged_plan.restype = C.c_int
     lib.h3_staged_plan.argtypes = [C.c_int64, C.c_int32, C.c_int32, C.c_int32, C.c_int64,
                                    _i64p, _i64p]

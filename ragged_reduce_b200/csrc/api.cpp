@@ -538,6 +538,61 @@ h3_status h3_bulk_wait_timeouts(void* stream, uint32_t* count, int32_t reset)
     return H3_OK;
 }
 
+h3_status h3_ragged_all_gather(const void* const* in, void* const* out, int64_t n_tokens,
+                               int64_t cols, int32_t world, void* stream, h3_exec_info* info)
+{
+    clear_info(info);
+    h3_status st = check_world(n_tokens, world, world);
+    if (st != H3_OK)
+        return st;
+    if (cols < 1 || !in || !out)
+        return H3_ERR_INVALID_ARG;
+    if (cols % 8 != 0)
+        return H3_ERR_MISALIGNED;
+    if (n_tokens > kMaxInt32 || cols / 8 > kMaxRowVecs)
+        return H3_ERR_UNSUPPORTED;
+    const Split ts = make_split(n_tokens, world);
+    const uint64_t row_bytes = uint64_t(cols) * 2;
+    uint64_t in_bytes[kMaxWorld];
+    uint64_t out_bytes[kMaxWorld];
+    for (int r = 0; r < world; ++r) {
+        if (!in[r] || !out[r])
+            return H3_ERR_INVALID_ARG;
+        if (!aligned16(in[r]) || !aligned16(out[r]))
+            return H3_ERR_MISALIGNED;
+        in_bytes[r] = uint64_t(ts.size(r)) * row_bytes;
+        out_bytes[r] = uint64_t(n_tokens) * row_bytes;
+    }
+    st = check_no_overlap(in, in_bytes, world, out, out_bytes, world);
+    if (st != H3_OK)
+        return st;
+    GatherArgs a;
+    std::memset(&a, 0, sizeof(a));
+    for (int r = 0; r < world; ++r) {
+        a.in[r] = static_cast<const char*>(in[r]);
+        a.out[r] = static_cast<char*>(out[r]);
+    }
+    a.T = int32_t(n_tokens);
+    a.W = world;
+    a.tq = int32_t(ts.q);
+    a.tm = int32_t(ts.m);
+    a.row_vecs = int32_t(cols / 8);
+    a.row_bytes = int64_t(row_bytes);
+    LaunchShape shape;
+    const cudaError_t err = launch_all_gather(a, 0, static_cast<cudaStream_t>(stream), &shape);
+    if (err != cudaSuccess)
+        return cuda_failure(err);
+    if (info) {
+        info->launches = 1;
+        info->chunks = 1;
+        info->grid = shape.grid;
+        info->block = shape.block;
+        info->variant = shape.variant;
+        info->planes_per_launch = 1;
+    }
+    return H3_OK;
+}
+
 h3_status h3_ragged_reduce_scatter(const void* const* partials, const void* bias, void* const* out,
                                    int64_t n_tokens, int64_t cols, int32_t world, void* stream,
                                    h3_exec_info* info)

@@ -86,6 +86,17 @@ struct StagedArgs {
     int32_t head_vecs;
 };
 
+// Ragged all-gather: rank r's rows [T_r, C] -> every rank's [T, C].
+struct GatherArgs {
+    const char* in[kMaxWorld];
+    char* out[kMaxWorld];
+    int32_t T;
+    int32_t W;
+    int32_t tq, tm;
+    int32_t row_vecs;   // C / 8
+    int64_t row_bytes;  // C * 2
+};
+
 struct LaunchShape {
     int grid = 0;
     int block = 0;
@@ -114,6 +125,10 @@ h3_status staged_relayout_with_window(bool seq_to_head, const void* const* send,
 
 // Record `err` as the calling thread's last CUDA error; returns H3_ERR_CUDA.
 h3_status record_cuda_failure(cudaError_t err);
+
+// Enqueue the all-gather launch.
+cudaError_t launch_all_gather(const GatherArgs& a, int ctas_per_sm, cudaStream_t stream,
+                              LaunchShape* shape);
 
 // Enqueue the reduce-scatter launch.
 cudaError_t launch_reduce_scatter(const ReduceArgs& a, int ctas_per_sm, cudaStream_t stream,

@@ -309,3 +309,32 @@ def test_staged_argument_checks(fn):
     assert st(window=recv[0] - 1024, wbytes=4096) == E.H3_ERR_INVALID_ARG  # over an output
     assert st(W=0) == E.H3_ERR_INVALID_ARG
     assert st(T=5) == E.H3_ERR_EMPTY_PARTITION
+
+
+@needs_no_gpu
+def test_all_gather_argument_checks():
+    T, Cc, W = 1000, 7168, 6
+    addr = BASE
+    ins, outs = [], []
+    for r in range(W):
+        ins.append(addr)
+        addr += (T // W + 1) * Cc * 2 + 4096
+    for r in range(W):
+        outs.append(addr)
+        addr += T * Cc * 2 + 4096
+
+    def st(ins=ins, outs=outs, T=T, Cc=Cc, W=W):
+        info = _abi.ExecInfo()
+        s = _abi.lib.h3_ragged_all_gather(_ptrs(ins), _ptrs(outs), T, Cc, W, None, C.byref(info))
+        assert info.launches == 0
+        return s
+
+    E = _abi
+    assert st(W=0) == E.H3_ERR_INVALID_ARG
+    assert st(W=65) == E.H3_ERR_UNSUPPORTED
+    assert st(T=5) == E.H3_ERR_EMPTY_PARTITION
+    assert st(Cc=7164) == E.H3_ERR_MISALIGNED
+    assert st(ins=[ins[0] + 8] + ins[1:]) == E.H3_ERR_MISALIGNED
+    assert st(outs=[0] + outs[1:]) == E.H3_ERR_INVALID_ARG
+    assert st(outs=[ins[2]] + outs[1:]) == E.H3_ERR_INVALID_ARG
+    assert st(outs=[outs[0], outs[0] + 1024] + outs[2:]) == E.H3_ERR_INVALID_ARG
