@@ -214,6 +214,13 @@ H3RR_API h3_status h3_ragged_reduce_scatter(const void* const* partials, const v
 H3RR_API h3_status h3_ragged_all_gather(const void* const* in, void* const* out,
                                         int64_t n_tokens, int64_t cols, int32_t world,
                                         void* stream, h3_exec_info* info);
+/* With launch overrides: variant 0 / H3_VARIANT_VECTOR (registers) or
+ * H3_VARIANT_BULK (bulk copies through shared memory; H3_ERR_UNSUPPORTED if
+ * 12 rows of C*2 bytes do not fit in shared memory), and ctas_per_sm. */
+H3RR_API h3_status h3_ragged_all_gather_ex(const void* const* in, void* const* out,
+                                           int64_t n_tokens, int64_t cols, int32_t world,
+                                           void* stream, const h3_launch_config* cfg,
+                                           h3_exec_info* info);
 
 /*
  * Same as h3_seq_to_head / h3_head_to_seq / h3_ragged_reduce_scatter with
@@ -316,9 +323,9 @@ H3RR_API h3_status h3_staged_plan(int64_t n_tokens, int32_t planes, int32_t n_he
                                   int64_t* chunk_tokens, int64_t* chunks);
 
 /*
- * h3_bulk_wait_timeouts - how many bounded waits of the bulk relayout kernel
- * (H3_VARIANT_BULK) expired on the current device since the count was last
- * cleared.  Each wait on a shared-memory barrier gives up after a fixed
+ * h3_bulk_wait_timeouts - how many bounded waits of the bulk kernels
+ * (H3_VARIANT_BULK relayouts and all-gather) expired on the current device
+ * since the count was last cleared.  Each wait on a shared-memory barrier gives up after a fixed
  * number of polls instead of spinning forever; an expiry means that launch's
  * output is incomplete.  Synchronises `stream`; reset != 0 clears the count.
  * count: host out-param.  Returns H3_ERR_CUDA if the copy fails.

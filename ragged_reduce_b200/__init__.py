@@ -328,7 +328,7 @@ def bulk_wait_timeouts(stream=None, reset: bool = False, device=None) -> int:
     return int(count.value)
 
 
-def ragged_all_gather(blocks, out, *, stream=None) -> dict:
+def ragged_all_gather(blocks, out, *, stream=None, variant: int = 0, ctas_per_sm: int = 0) -> dict:
     """Ragged all-gather of token rows: blocks are W tensors [T_r, C] (rank
     r's rows; 2-byte elements), out W tensors [T, C], each written with all T
     rows in token order (``h3_ragged_all_gather``)."""
@@ -351,11 +351,15 @@ def ragged_all_gather(blocks, out, *, stream=None) -> dict:
         if tuple(o.shape) != (T, Cc):
             raise ValueError(f"out {j}: shape {tuple(o.shape)}, expected {(T, Cc)}")
     info = ExecInfo()
+    args = [_abi.pointer_array([b.data_ptr() for b in blocks]),
+            _abi.pointer_array([o.data_ptr() for o in out]),
+            T, Cc, W, C.c_void_p(_stream_handle(stream, dev))]
+    cfg = _config(variant, ctas_per_sm)
     with torch.cuda.device(dev):
-        st = _abi.lib.h3_ragged_all_gather(_abi.pointer_array([b.data_ptr() for b in blocks]),
-                                           _abi.pointer_array([o.data_ptr() for o in out]),
-                                           T, Cc, W, C.c_void_p(_stream_handle(stream, dev)),
-                                           C.byref(info))
+        if cfg is None:
+            st = _abi.lib.h3_ragged_all_gather(*args, C.byref(info))
+        else:
+            st = _abi.lib.h3_ragged_all_gather_ex(*args, cfg, C.byref(info))
     _abi.check(st, "h3_ragged_all_gather")
     return info.as_dict()
 

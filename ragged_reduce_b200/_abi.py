@@ -123,6 +123,10 @@ def _load() -> C.CDLL:
     lib.h3_ragged_all_gather.restype = C.c_int
     lib.h3_ragged_all_gather.argtypes = [_vpp, _vpp, C.c_int64, C.c_int64, C.c_int32, C.c_void_p,
                                          C.POINTER(ExecInfo)]
+    lib.h3_ragged_all_gather_ex.restype = C.c_int
+    lib.h3_ragged_all_gather_ex.argtypes = [_vpp, _vpp, C.c_int64, C.c_int64, C.c_int32,
+                                            C.c_void_p, C.POINTER(LaunchConfig),
+                                            C.POINTER(ExecInfo)]
     lib.h3_staged_plan.restype = C.c_int
     lib.h3_staged_plan.argtypes = [C.c_int64, C.c_int32, C.c_int32, C.c_int32, C.c_int64,
                                    _i64p, _i64p]

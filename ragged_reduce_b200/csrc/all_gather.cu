@@ -6,7 +6,8 @@
 // ts_r .. te_r-1 of a [T, C] activation as a [T_r, C] block; after the gather
 // every rank holds all T rows.  With every virtual rank in one GPU's memory
 // there is nothing to pad: each row is read once from its owner's block and
-// written to each of the W outputs.
+// written to each of the W outputs.  A bulk-copy variant (H3_VARIANT_BULK)
+// moves whole rows through shared memory instead of registers.
 //
 // A CTA of NT threads takes one token row per iteration (grid-stride); thread
 // i owns the row's vectors i, i+NT, ... (32 bytes when every pointer and the
@@ -16,6 +17,10 @@
 #include "h3rr_internal.h"
 
 namespace h3rr {
+
+// Count of bounded waits that expired in the bulk all-gather kernel (per device).
+__device__ unsigned int g_gather_wait_timeouts = 0;
+
 namespace {
 
 template <int VW>
@@ -114,9 +119,100 @@ __global__ void __launch_bounds__(kGenericThreads) all_gather_generic_kernel(con
     }
 }
 
+// ---------------------------------------------------------------------------
+// bulk variant: one thread per CTA; each row is bulk-loaded once into a ring
+// of shared-memory stages and bulk-stored to the W outputs (the copy engine
+// does the fan-out).  No multicast.  Waits are bounded; expiries are counted
+// in g_gather_wait_timeouts and reported with the relayout's count.
+// ---------------------------------------------------------------------------
+constexpr int kBulkStages = 12;
+constexpr int kBulkLookahead = 8;
+constexpr int kBulkBarrierBytes = 128;
+constexpr uint32_t kBulkWaitLimit = 1u << 24;
+
+__device__ __forceinline__ uint32_t smem_addr(const void* p)
+{
+    return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity)
+{
+    for (uint32_t it = 0; it < kBulkWaitLimit; ++it) {
+        uint32_t done;
+        asm volatile(
+            "{\n\t.reg .pred p;\n\t"
+            "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+            "selp.u32 %0, 1, 0, p;\n\t}"
+            : "=r"(done)
+            : "r"(smem_addr(bar)), "r"(parity)
+            : "memory");
+        if (done)
+            return true;
+    }
+    return false;
+}
+
+template <int S, int L>
+__global__ void __launch_bounds__(32) all_gather_bulk_kernel(const __grid_constant__ GatherArgs a)
+{
+    static_assert(S <= kBulkBarrierBytes / 8 && L >= 1 && L < S, "bulk ring shape");
+    extern __shared__ __align__(128) unsigned char smem[];
+    uint64_t* bars = reinterpret_cast<uint64_t*>(smem);
+    unsigned char* ring = smem + kBulkBarrierBytes;
+    if (threadIdx.x != 0)
+        return;
+    const uint32_t row_bytes = uint32_t(a.row_bytes);
+    uint64_t pol;
+    asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(pol));
+    for (int s = 0; s < S; ++s)
+        asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(smem_addr(&bars[s])) : "memory");
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    const int64_t n_rows = a.T > int32_t(blockIdx.x) ? (int64_t(a.T) - blockIdx.x + gridDim.x - 1) / gridDim.x : 0;
+    auto issue_load = [&](int64_t n) {
+        const int32_t t = int32_t(blockIdx.x + n * gridDim.x);
+        const int32_t s = split_owner(t, a.tq, a.tm);
+        const int32_t tl = t - split_start(s, a.tq, a.tm);
+        uint64_t* bar = &bars[n % S];
+        asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_addr(bar)),
+                     "r"(row_bytes)
+                     : "memory");
+        asm volatile(
+            "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint "
+            "[%0], [%1], %2, [%3], %4;" ::"r"(smem_addr(ring + size_t(n % S) * row_bytes)),
+            "l"(a.in[s] + int64_t(tl) * row_bytes), "r"(row_bytes), "r"(smem_addr(bar)), "l"(pol)
+            : "memory");
+    };
+    const int64_t prologue = n_rows < L ? n_rows : L;
+    for (int64_t n = 0; n < prologue; ++n)
+        issue_load(n);
+    for (int64_t n = 0; n < n_rows; ++n) {
+        if (n + L < n_rows) {
+            asm volatile("cp.async.bulk.wait_group.read %0;" ::"n"(S - L - 1) : "memory");
+            issue_load(n + L);
+        }
+        if (!mbar_wait(&bars[n % S], uint32_t((n / S) & 1))) {
+            atomicAdd(&g_gather_wait_timeouts, 1u);
+            for (int64_t m = n + 1; m < n_rows && m <= n + L; ++m)
+                mbar_wait(&bars[m % S], uint32_t((m / S) & 1));
+            break;
+        }
+        const int32_t t = int32_t(blockIdx.x + n * gridDim.x);
+        const unsigned char* stage = ring + size_t(n % S) * row_bytes;
+        for (int j = 0; j < a.W; ++j)
+            asm volatile("cp.async.bulk.global.shared::cta.bulk_group.L2::cache_hint [%0], [%1], %2, %3;" ::"l"(
+                             a.out[j] + int64_t(t) * row_bytes),
+                         "r"(smem_addr(stage)), "r"(row_bytes), "l"(pol)
+                         : "memory");
+        asm volatile("cp.async.bulk.commit_group;" ::: "memory");
+    }
+    asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
+}
+
 struct GatherChoice {
     const void* fn = nullptr;
     int threads = 0;
+    size_t smem = 0;
+    int variant = H3_VARIANT_GATHER;
 };
 
 template <int VW, int NT>
@@ -149,23 +245,49 @@ bool wide_ok(const GatherArgs& a)
 
 }  // namespace
 
-cudaError_t launch_all_gather(const GatherArgs& a, int ctas_per_sm, cudaStream_t stream, LaunchShape* shape)
+bool all_gather_bulk_fits(const GatherArgs& a, int device)
+{
+    int max_smem = 0;
+    if (cudaDeviceGetAttribute(&max_smem, cudaDevAttrMaxSharedMemoryPerBlockOptin, device) != cudaSuccess)
+        return false;
+    return size_t(kBulkBarrierBytes) + size_t(kBulkStages) * size_t(a.row_bytes) <= size_t(max_smem);
+}
+
+cudaError_t launch_all_gather(const GatherArgs& a, int variant, int ctas_per_sm, cudaStream_t stream,
+                              LaunchShape* shape)
 {
     int device = 0;
     const int sms = current_sm_count(&device);
     if (sms <= 0)
         return cudaErrorNoDevice;
     GatherChoice gc;
-    bool ok = false;
-    if (wide_ok(a))
-        ok = pick<32, 64>((a.row_vecs / 2 + 63) / 64, &gc);
-    if (!ok)
-        ok = pick<16, 128>((a.row_vecs + 127) / 128, &gc);
-    if (!ok) {
-        gc.fn = (const void*)all_gather_generic_kernel;
-        gc.threads = kGenericThreads;
+    if (variant == H3_VARIANT_BULK) {
+        if (!all_gather_bulk_fits(a, device))
+            return cudaErrorInvalidConfiguration;
+        gc.fn = (const void*)all_gather_bulk_kernel<kBulkStages, kBulkLookahead>;
+        gc.threads = 32;
+        gc.smem = size_t(kBulkBarrierBytes) + size_t(kBulkStages) * size_t(a.row_bytes);
+        gc.variant = H3_VARIANT_BULK;
+        const cudaError_t err = allow_dynamic_smem(gc.fn, gc.smem, device);
+        if (err != cudaSuccess)
+            return err;
+    } else {
+        bool ok = false;
+        if (wide_ok(a))
+            ok = pick<32, 64>((a.row_vecs / 2 + 63) / 64, &gc);
+        if (!ok)
+            ok = pick<16, 128>((a.row_vecs + 127) / 128, &gc);
+        if (!ok) {
+            gc.fn = (const void*)all_gather_generic_kernel;
+            gc.threads = kGenericThreads;
+        }
     }
-    const int per_sm = ctas_per_sm > 0 ? ctas_per_sm : resident_ctas(gc.fn, gc.threads, 0, device);
+    // The vector kernel launches 16 CTAs per SM by default, more than fit at
+    // once: on B200 that measured fastest for the 32k x 7168 (W=6) and
+    // 64k x 7168 (W=8) gathers (5.9 TB/s against 5.6 TB/s at 2 to 10 CTAs per
+    // SM).  The bulk kernel runs one CTA per SM (its ring fills the SM).
+    const int fit = resident_ctas(gc.fn, gc.threads, gc.smem, device);
+    const int per_sm = ctas_per_sm > 0 ? ctas_per_sm : (gc.variant == H3_VARIANT_BULK ? fit : 16);
     int64_t grid = int64_t(sms) * per_sm;
     if (grid > a.T)
         grid = a.T;
@@ -174,10 +296,26 @@ cudaError_t launch_all_gather(const GatherArgs& a, int ctas_per_sm, cudaStream_t
     if (shape) {
         shape->grid = int(grid);
         shape->block = gc.threads;
-        shape->variant = H3_VARIANT_GATHER;
+        shape->variant = gc.variant;
     }
     void* params[] = {const_cast<GatherArgs*>(&a)};
-    return cudaLaunchKernel(gc.fn, dim3(unsigned(grid)), dim3(gc.threads), params, 0, stream);
+    return cudaLaunchKernel(gc.fn, dim3(unsigned(grid)), dim3(gc.threads), params, gc.smem, stream);
+}
+
+cudaError_t read_gather_wait_timeouts(unsigned int* count, bool reset, cudaStream_t stream)
+{
+    cudaError_t err = cudaMemcpyFromSymbolAsync(count, g_gather_wait_timeouts, sizeof(unsigned int), 0,
+                                                cudaMemcpyDeviceToHost, stream);
+    if (err == cudaSuccess)
+        err = cudaStreamSynchronize(stream);
+    if (err == cudaSuccess && reset) {
+        static const unsigned int zero = 0;
+        err = cudaMemcpyToSymbolAsync(g_gather_wait_timeouts, &zero, sizeof(zero), 0,
+                                      cudaMemcpyHostToDevice, stream);
+        if (err == cudaSuccess)
+            err = cudaStreamSynchronize(stream);
+    }
+    return err;
 }
 
 }  // namespace h3rr

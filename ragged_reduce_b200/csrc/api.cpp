@@ -530,16 +530,25 @@ h3_status h3_bulk_wait_timeouts(void* stream, uint32_t* count, int32_t reset)
 {
     if (!count)
         return H3_ERR_INVALID_ARG;
-    unsigned int v = 0;
-    const cudaError_t err = read_bulk_wait_timeouts(&v, reset != 0, static_cast<cudaStream_t>(stream));
+    unsigned int v = 0, g = 0;
+    cudaError_t err = read_bulk_wait_timeouts(&v, reset != 0, static_cast<cudaStream_t>(stream));
+    if (err == cudaSuccess)
+        err = read_gather_wait_timeouts(&g, reset != 0, static_cast<cudaStream_t>(stream));
     if (err != cudaSuccess)
         return cuda_failure(err);
-    *count = v;
+    *count = v + g;
     return H3_OK;
 }
 
 h3_status h3_ragged_all_gather(const void* const* in, void* const* out, int64_t n_tokens,
                                int64_t cols, int32_t world, void* stream, h3_exec_info* info)
+{
+    return h3_ragged_all_gather_ex(in, out, n_tokens, cols, world, stream, nullptr, info);
+}
+
+h3_status h3_ragged_all_gather_ex(const void* const* in, void* const* out, int64_t n_tokens,
+                                  int64_t cols, int32_t world, void* stream,
+                                  const h3_launch_config* cfg, h3_exec_info* info)
 {
     clear_info(info);
     h3_status st = check_world(n_tokens, world, world);
@@ -547,14 +556,18 @@ h3_status h3_ragged_all_gather(const void* const* in, void* const* out, int64_t 
         return st;
     if (cols < 1 || !in || !out)
         return H3_ERR_INVALID_ARG;
+    if (cfg && cfg->variant != 0 && cfg->variant != H3_VARIANT_VECTOR && cfg->variant != H3_VARIANT_BULK)
+        return H3_ERR_INVALID_ARG;
+    if (cfg && cfg->ctas_per_sm < 0)
+        return H3_ERR_INVALID_ARG;
     if (cols % 8 != 0)
         return H3_ERR_MISALIGNED;
     if (n_tokens > kMaxInt32 || cols / 8 > kMaxRowVecs)
         return H3_ERR_UNSUPPORTED;
     const Split ts = make_split(n_tokens, world);
     const uint64_t row_bytes = uint64_t(cols) * 2;
-    uint64_t in_bytes[kMaxWorld];
-    uint64_t out_bytes[kMaxWorld];
+    uint64_t in_bytes[kMaxWorld] = {};
+    uint64_t out_bytes[kMaxWorld] = {};
     for (int r = 0; r < world; ++r) {
         if (!in[r] || !out[r])
             return H3_ERR_INVALID_ARG;
@@ -578,8 +591,18 @@ h3_status h3_ragged_all_gather(const void* const* in, void* const* out, int64_t 
     a.tm = int32_t(ts.m);
     a.row_vecs = int32_t(cols / 8);
     a.row_bytes = int64_t(row_bytes);
+    const int variant = cfg ? cfg->variant : 0;
+    if (variant == H3_VARIANT_BULK) {
+        int device = 0;
+        const cudaError_t derr = cudaGetDevice(&device);
+        if (derr != cudaSuccess)
+            return cuda_failure(derr);
+        if (!all_gather_bulk_fits(a, device))
+            return H3_ERR_UNSUPPORTED;  // a row does not fit the shared-memory ring
+    }
     LaunchShape shape;
-    const cudaError_t err = launch_all_gather(a, 0, static_cast<cudaStream_t>(stream), &shape);
+    const cudaError_t err = launch_all_gather(a, variant, cfg ? cfg->ctas_per_sm : 0,
+                                              static_cast<cudaStream_t>(stream), &shape);
     if (err != cudaSuccess)
         return cuda_failure(err);
     if (info) {

@@ -126,9 +126,11 @@ h3_status staged_relayout_with_window(bool seq_to_head, const void* const* send,
 // Record `err` as the calling thread's last CUDA error; returns H3_ERR_CUDA.
 h3_status record_cuda_failure(cudaError_t err);
 
-// Enqueue the all-gather launch.
-cudaError_t launch_all_gather(const GatherArgs& a, int ctas_per_sm, cudaStream_t stream,
+// Enqueue the all-gather launch (variant 0 / H3_VARIANT_VECTOR or H3_VARIANT_BULK).
+cudaError_t launch_all_gather(const GatherArgs& a, int variant, int ctas_per_sm, cudaStream_t stream,
                               LaunchShape* shape);
+bool all_gather_bulk_fits(const GatherArgs& a, int device);
+cudaError_t read_gather_wait_timeouts(unsigned int* count, bool reset, cudaStream_t stream);
 
 // Enqueue the reduce-scatter launch.
 cudaError_t launch_reduce_scatter(const ReduceArgs& a, int ctas_per_sm, cudaStream_t stream,

@@ -30,6 +30,34 @@ def test_all_gather_matches_oracle(oracle_lib, T, C, W):
         assert np.array_equal(gu.bits(outs[j]), want[j]), f"rank {j}"
 
 
+@pytest.mark.parametrize("T,C,W", [(1000, 7168, 6), (97, 8, 8), (64, 4104, 4), (33, 24, 1), (7, 7168, 7)])
+@pytest.mark.parametrize("variant", [rr.H3_VARIANT_VECTOR, rr.H3_VARIANT_BULK])
+def test_all_gather_forced_variant(oracle_lib, T, C, W, variant):
+    full, blocks = _blocks(T, C, W, 3 * T + W)
+    bufs, outs = [], []
+    for _ in range(W):
+        b, o = gu.guarded((T, C), DEV)
+        bufs.append(b)
+        outs.append(o)
+    rr.bulk_wait_timeouts(reset=True)
+    info = rr.ragged_all_gather(blocks, outs, variant=variant)
+    assert info["variant"] == (rr.H3_VARIANT_BULK if variant == rr.H3_VARIANT_BULK else rr.H3_VARIANT_GATHER)
+    want = oracle_lib.ragged_all_gather([gu.bits(b) for b in blocks], W)
+    for j in range(W):
+        assert np.array_equal(gu.bits(outs[j]), want[j]), f"rank {j}"
+    assert all(gu.guards_intact(b) for b in bufs)
+    assert rr.bulk_wait_timeouts() == 0
+
+
+def test_all_gather_bulk_rejects_wide_rows():
+    T, C, W = 16, 18000, 2  # 36,000-byte rows: 12 stages do not fit
+    full, blocks = _blocks(T, C, W, 1)
+    outs = [torch.empty((T, C), dtype=torch.bfloat16, device=DEV) for _ in range(W)]
+    with pytest.raises(rr.H3Error) as e:
+        rr.ragged_all_gather(blocks, outs, variant=rr.H3_VARIANT_BULK)
+    assert e.value.status == 5
+
+
 def test_all_gather_guard_bands_and_separate_blocks(oracle_lib):
     T, C, W = 500, 7168, 6
     part = rr.partition(T, W, W)
