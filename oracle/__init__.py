@@ -62,6 +62,10 @@ class Oracle:
             f.restype = C.c_int32
             f.argtypes = [C.c_int64, C.c_int32, C.c_int32, C.c_int32, C.c_int32,
                           C.c_int32, C.c_int64, _i64p, _i32p, _i64p]
+        lib.h3o_relayout_layout.restype = C.c_int32
+        lib.h3o_relayout_layout.argtypes = [C.c_void_p, C.c_void_p, C.c_int64, C.c_int32,
+                                            C.c_int32, C.c_int32, C.c_int32, C.c_int32,
+                                            C.c_int32, C.c_int32]
         lib.h3o_ragged_all_gather.restype = C.c_int32
         lib.h3o_ragged_all_gather.argtypes = [C.c_void_p, C.c_void_p, C.c_int64, C.c_int64,
                                               C.c_int32]
@@ -177,6 +181,37 @@ class Oracle:
         rc = self.lib.h3o_ragged_reduce_scatter(_ptr_array(src),
                                                 None if b is None else b.ctypes.data,
                                                 _ptr_array(out), T, Cc, W)
+        assert rc == 0
+        return out
+
+    def relayout_layout(self, send, T, P, H, D, W, seq_to_head: bool, seq_plane_major: bool,
+                        head_plane_major: bool):
+        """Relayout with plane-major options.  seq_to_head: send are W sequence-side
+        buffers ([T_r, P, H, D] or [P, T_r, H, D]) -> W head-side buffers ([T, P, H_j, D]
+        or [P, T, H_j, D]); otherwise the reverse."""
+        ts = self.partition_range(T, W)
+        hs = self.partition_range(H, W)
+        src = [np.ascontiguousarray(s, dtype=np.uint16) for s in send]
+
+        def seq_shape(r):
+            Tr = int(ts[r + 1] - ts[r])
+            return (P, Tr, H, D) if seq_plane_major else (Tr, P, H, D)
+
+        def head_shape(j):
+            Hj = int(hs[j + 1] - hs[j])
+            return (P, T, Hj, D) if head_plane_major else (T, P, Hj, D)
+
+        if seq_to_head:
+            for r, x in enumerate(src):
+                assert x.size == int(np.prod(seq_shape(r)))
+            out = [np.zeros(head_shape(j), dtype=np.uint16) for j in range(W)]
+        else:
+            for j, x in enumerate(src):
+                assert x.size == int(np.prod(head_shape(j)))
+            out = [np.zeros(seq_shape(r), dtype=np.uint16) for r in range(W)]
+        rc = self.lib.h3o_relayout_layout(_ptr_array(src), _ptr_array(out), T, P, H, D, W,
+                                          1 if seq_to_head else 0, int(seq_plane_major),
+                                          int(head_plane_major))
         assert rc == 0
         return out
 

@@ -411,3 +411,67 @@ done:
     return rc;
 }
 
+/* ------------------------------------------------------------------------ */
+/* Relayouts with plane-major buffers                                          */
+/* Sequence side, rank r: [T_r, P, H, D] (token-major) or [P, T_r, H, D]      */
+/* (plane-major: plane p of rank r is one contiguous [T_r, H, D] block).      */
+/* Head side, rank j: [T, P, H_j, D] or [P, T, H_j, D].  Same element maps as  */
+/* h3o_seq_to_head / h3o_head_to_seq; only the buffer index of (t, p, h, d)    */
+/* changes.                                                                    */
+/* ------------------------------------------------------------------------ */
+
+static int64_t seq_index(int64_t tl, int64_t Tr, int64_t p, int64_t P, int64_t h, int64_t H,
+                         int64_t d, int64_t D, int32_t plane_major)
+{
+    if (plane_major)
+        return ((p * Tr + tl) * H + h) * D + d;
+    return ((tl * P + p) * H + h) * D + d;
+}
+
+static int64_t head_index(int64_t t, int64_t T, int64_t p, int64_t P, int64_t hl, int64_t Hj,
+                          int64_t d, int64_t D, int32_t plane_major)
+{
+    if (plane_major)
+        return ((p * T + t) * Hj + hl) * D + d;
+    return ((t * P + p) * Hj + hl) * D + d;
+}
+
+/* seq -> head (dir = 1) or head -> seq (dir = 0) with the given layouts. */
+int32_t h3o_relayout_layout(const uint16_t* const* send, uint16_t* const* recv, int64_t T,
+                            int32_t P, int32_t H, int32_t D, int32_t W, int32_t dir,
+                            int32_t seq_plane_major, int32_t head_plane_major)
+{
+    int64_t* ts = (int64_t*)malloc(sizeof(int64_t) * (size_t)(W + 1));
+    int64_t* hs = (int64_t*)malloc(sizeof(int64_t) * (size_t)(W + 1));
+    int32_t rc = -1;
+    if (!ts || !hs)
+        goto done;
+    if (h3o_partition_range(T, W, ts) || h3o_partition_range(H, W, hs))
+        goto done;
+    for (int32_t r = 0; r < W; ++r) {
+        int64_t Tr = ts[r + 1] - ts[r];
+        for (int64_t tl = 0; tl < Tr; ++tl) {
+            int64_t t = ts[r] + tl;
+            for (int32_t p = 0; p < P; ++p) {
+                for (int32_t h = 0; h < H; ++h) {
+                    int32_t j = owner_of(hs, W, h);
+                    int64_t Hj = hs[j + 1] - hs[j];
+                    for (int32_t d = 0; d < D; ++d) {
+                        int64_t si = seq_index(tl, Tr, p, P, h, H, d, D, seq_plane_major);
+                        int64_t hi = head_index(t, T, p, P, h - hs[j], Hj, d, D, head_plane_major);
+                        if (dir)
+                            recv[j][hi] = send[r][si];
+                        else
+                            recv[r][si] = send[j][hi];
+                    }
+                }
+            }
+        }
+    }
+    rc = 0;
+done:
+    free(ts);
+    free(hs);
+    return rc;
+}
+

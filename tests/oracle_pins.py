@@ -420,6 +420,28 @@ def check_all_gather(o):
         assert np.array_equal(g, want)
 
 
+def check_plane_major_layouts(o):
+    """Plane-major buffers are numpy transposes of the token-major ones: for
+    every layout pair the relayout equals the token-major result with the
+    (token, plane) axes swapped where a side is plane-major; round trips are
+    the identity."""
+    for T, P, H, D, W in [(10, 3, 56, 1, 6), (7, 3, 5, 4, 3), (9, 4, 56, 1, 8), (13, 2, 9, 8, 1)]:
+        full = _index_coded((T, P, H, D))
+        ts = o.partition_range(T, W)
+        send_tm = _split_rows(full, ts)
+        ref = o.seq_to_head(send_tm, T, P, H, D, W)          # token-major both sides
+        for spm in (False, True):
+            for hpm in (False, True):
+                send = [np.ascontiguousarray(x.transpose(1, 0, 2, 3)) if spm else x for x in send_tm]
+                got = o.relayout_layout(send, T, P, H, D, W, True, spm, hpm)
+                for j in range(W):
+                    want = np.ascontiguousarray(ref[j].transpose(1, 0, 2, 3)) if hpm else ref[j]
+                    assert np.array_equal(got[j], want), ("s2h", spm, hpm, j)
+                back = o.relayout_layout(got, T, P, H, D, W, False, spm, hpm)
+                for r in range(W):
+                    assert np.array_equal(back[r], send[r]), ("h2s", spm, hpm, r)
+
+
 ALL_CHECKS = [
     check_head_table,
     check_partition_invariants,
@@ -436,6 +458,7 @@ ALL_CHECKS = [
     check_reduce_row_assignment,
     check_reduce_identities,
     check_all_gather,
+    check_plane_major_layouts,
 ]
 
 

@@ -63,6 +63,10 @@ MUTANTS = [
      "out[j][t * C + c] = in[r][(t % (ts[r + 1] - ts[r])) * C + c];"),
     ("gather_from_own_rank", "out[j][t * C + c] = in[r][(t - ts[r]) * C + c];",
      "out[j][t * C + c] = in[j][((t - ts[r]) % (ts[j + 1] - ts[j])) * C + c];"),
+    ("plane_major_seq_shifts_channel", "return ((p * Tr + tl) * H + h) * D + d;",
+     "return ((p * Tr + tl) * H + h) * D + (d + p) % D;"),
+    ("plane_major_head_swapped", "return ((p * T + t) * Hj + hl) * D + d;",
+     "return ((t * P + p) * Hj + hl) * D + d;"),
     ("widen_drops_sign", "uint32_t u = ((uint32_t)b) << 16;", "uint32_t u = ((uint32_t)(b & 0x7FFFu)) << 16;"),
 ]
 
