@@ -199,6 +199,35 @@ H3RR_API h3_status h3_ragged_reduce_scatter(const void* const* partials, const v
                                    int32_t world, void* stream, h3_exec_info* info);
 
 /*
+ * h3_seq_to_head_layout / h3_head_to_seq_layout - the relayouts with
+ * plane-major buffers on either side.  layout is a bit set:
+ *   H3_LAYOUT_SEQ_PLANE_MAJOR  sequence-side rank r is [P, T_r, H, D] (plane p
+ *                              a contiguous [T_r, H, D] block: separate Q, K, V
+ *                              projection outputs) instead of [T_r, P, H, D];
+ *   H3_LAYOUT_HEAD_PLANE_MAJOR head-side rank j is [P, T, H_j, D] (plane p a
+ *                              contiguous [T, H_j, D] block: the Q, K and V an
+ *                              attention kernel takes) instead of [T, P, H_j, D].
+ * The element maps are those of h3_seq_to_head / h3_head_to_seq; only where
+ * element (t, p, h, d) sits in each buffer changes.  Buffer sizes are the same,
+ * so every check (alignment, overlap, window) is unchanged.  layout 0 equals the
+ * plain calls.  Unknown bits are H3_ERR_INVALID_ARG; cfg (nullable) as in the
+ * _ex calls, except that H3_VARIANT_BULK with a non-zero layout is
+ * H3_ERR_UNSUPPORTED.
+ */
+#define H3_LAYOUT_SEQ_PLANE_MAJOR 1
+#define H3_LAYOUT_HEAD_PLANE_MAJOR 2
+H3RR_API h3_status h3_seq_to_head_layout(const void* const* send, void* const* recv,
+                                         int64_t n_tokens, int32_t planes, int32_t n_heads,
+                                         int32_t head_dim, int32_t world, int64_t window_bytes,
+                                         int32_t layout, void* stream, const h3_launch_config* cfg,
+                                         h3_exec_info* info);
+H3RR_API h3_status h3_head_to_seq_layout(const void* const* send, void* const* recv,
+                                         int64_t n_tokens, int32_t planes, int32_t n_heads,
+                                         int32_t head_dim, int32_t world, int64_t window_bytes,
+                                         int32_t layout, void* stream, const h3_launch_config* cfg,
+                                         h3_exec_info* info);
+
+/*
  * h3_ragged_all_gather - ragged all-gather of token rows ("Distributed H3
  * Execution", intro: ragged row gathering, whose temporary collective padding
  * is removed before model operations; "Validation": ragged gather and

@@ -25,7 +25,8 @@ import numpy as np
 import torch
 
 from . import _abi
-from ._abi import (ExecInfo, H3Error, LaunchConfig, H3_VARIANT_BULK, H3_VARIANT_GATHER,
+from ._abi import (ExecInfo, H3Error, LaunchConfig, H3_LAYOUT_HEAD_PLANE_MAJOR,
+                   H3_LAYOUT_SEQ_PLANE_MAJOR, H3_VARIANT_BULK, H3_VARIANT_GATHER,
                    H3_VARIANT_REDUCE, H3_VARIANT_STAGED, H3_VARIANT_VECTOR, MAX_WORLD)
 
 __all__ = [
@@ -34,6 +35,8 @@ __all__ = [
     "H3_VARIANT_VECTOR", "H3_VARIANT_BULK", "H3_VARIANT_REDUCE", "MAX_WORLD", "library_path",
     "bulk_wait_timeouts", "alloc_reduce_outputs", "seq_to_head_staged", "head_to_seq_staged",
     "staged_plan", "H3_VARIANT_STAGED", "ragged_all_gather", "H3_VARIANT_GATHER",
+    "seq_to_head_layout", "head_to_seq_layout", "H3_LAYOUT_SEQ_PLANE_MAJOR",
+    "H3_LAYOUT_HEAD_PLANE_MAJOR",
 ]
 
 library_path = _abi.LIB_PATH
@@ -150,7 +153,7 @@ def _config(variant: int, ctas_per_sm: int):
     return C.byref(LaunchConfig(int(variant), int(ctas_per_sm), 0, 0))
 
 
-def _relayout_shapes(seq_to_head_dir: bool, send, recv):
+def _relayout_shapes(seq_to_head_dir: bool, send, recv, layout: int = 0):
     """Check the per-rank shapes; return (T, P, H, D, W, device)."""
     W = len(send)
     if W < 1 or len(recv) != W:
@@ -160,18 +163,57 @@ def _relayout_shapes(seq_to_head_dir: bool, send, recv):
     head_side = recv if seq_to_head_dir else send
     if any(t.dim() != 4 for t in send + recv):
         raise ValueError("relayout buffers are 4-D: [tokens, planes, heads, head_dim]")
-    _, P, H, D = seq_side[0].shape
-    T = sum(int(t.shape[0]) for t in seq_side)
+    seq_pm = bool(layout & _abi.H3_LAYOUT_SEQ_PLANE_MAJOR)
+    head_pm = bool(layout & _abi.H3_LAYOUT_HEAD_PLANE_MAJOR)
+    if seq_pm:
+        P, _, H, D = seq_side[0].shape
+        T = sum(int(t.shape[1]) for t in seq_side)
+    else:
+        _, P, H, D = seq_side[0].shape
+        T = sum(int(t.shape[0]) for t in seq_side)
     part = partition(T, H, W)
     for r, t in enumerate(seq_side):
-        if tuple(t.shape) != (part.tokens(r), P, H, D):
-            raise ValueError(f"sequence-side rank {r}: shape {tuple(t.shape)}, "
-                             f"expected {(part.tokens(r), P, H, D)}")
+        want = (P, part.tokens(r), H, D) if seq_pm else (part.tokens(r), P, H, D)
+        if tuple(t.shape) != want:
+            raise ValueError(f"sequence-side rank {r}: shape {tuple(t.shape)}, expected {want}")
     for j, t in enumerate(head_side):
-        if tuple(t.shape) != (T, P, part.heads(j), D):
-            raise ValueError(f"head-side rank {j}: shape {tuple(t.shape)}, "
-                             f"expected {(T, P, part.heads(j), D)}")
+        want = (P, T, part.heads(j), D) if head_pm else (T, P, part.heads(j), D)
+        if tuple(t.shape) != want:
+            raise ValueError(f"head-side rank {j}: shape {tuple(t.shape)}, expected {want}")
     return T, int(P), int(H), int(D), W, dev
+
+
+def _relayout_layout(seq_to_head_dir: bool, send, recv, layout, window_bytes, stream, variant,
+                     ctas_per_sm):
+    send = _as_list(send)
+    recv = _as_list(recv)
+    T, P, H, D, W, dev = _relayout_shapes(seq_to_head_dir, send, recv, layout)
+    info = ExecInfo()
+    name = "h3_seq_to_head_layout" if seq_to_head_dir else "h3_head_to_seq_layout"
+    cfg = _config(variant, ctas_per_sm)
+    with torch.cuda.device(dev):
+        st = getattr(_abi.lib, name)(
+            _abi.pointer_array([t.data_ptr() for t in send]),
+            _abi.pointer_array([t.data_ptr() for t in recv]),
+            T, P, H, D, W, int(window_bytes), int(layout), C.c_void_p(_stream_handle(stream, dev)),
+            cfg, C.byref(info))
+    _abi.check(st, name)
+    return info.as_dict()
+
+
+def seq_to_head_layout(send, recv, layout: int, *, window_bytes: int = 0, stream=None,
+                       variant: int = 0, ctas_per_sm: int = 0) -> dict:
+    """seq->head with plane-major buffers (``layout``: bit set of
+    H3_LAYOUT_SEQ_PLANE_MAJOR / H3_LAYOUT_HEAD_PLANE_MAJOR).  Plane-major
+    sequence side: W tensors [P, T_r, H, D]; plane-major head side: W tensors
+    [P, T, H_j, D] (out[j][0], [1], [2] are that rank's Q, K, V)."""
+    return _relayout_layout(True, send, recv, layout, window_bytes, stream, variant, ctas_per_sm)
+
+
+def head_to_seq_layout(send, recv, layout: int, *, window_bytes: int = 0, stream=None,
+                       variant: int = 0, ctas_per_sm: int = 0) -> dict:
+    """head->seq with plane-major buffers (see ``seq_to_head_layout``)."""
+    return _relayout_layout(False, send, recv, layout, window_bytes, stream, variant, ctas_per_sm)
 
 
 def _relayout_staged(seq_to_head_dir: bool, send, recv, window, stream):

@@ -39,6 +39,8 @@ H3_VARIANT_STAGED = 4
 H3_VARIANT_GATHER = 5
 
 MAX_WORLD = 64
+H3_LAYOUT_SEQ_PLANE_MAJOR = 1
+H3_LAYOUT_HEAD_PLANE_MAJOR = 2
 ABI_VERSION = 1
 
 
@@ -120,6 +122,12 @@ def _load() -> C.CDLL:
         f.restype = C.c_int
         f.argtypes = [_vpp, _vpp, C.c_int64, C.c_int32, C.c_int32, C.c_int32, C.c_int32,
                       C.c_void_p, C.c_int64, C.c_void_p, C.POINTER(ExecInfo)]
+    for name in ("h3_seq_to_head_layout", "h3_head_to_seq_layout"):
+        f = getattr(lib, name)
+        f.restype = C.c_int
+        f.argtypes = [_vpp, _vpp, C.c_int64, C.c_int32, C.c_int32, C.c_int32, C.c_int32,
+                      C.c_int64, C.c_int32, C.c_void_p, C.POINTER(LaunchConfig),
+                      C.POINTER(ExecInfo)]
     lib.h3_ragged_all_gather.restype = C.c_int
     lib.h3_ragged_all_gather.argtypes = [_vpp, _vpp, C.c_int64, C.c_int64, C.c_int32, C.c_void_p,
                                          C.POINTER(ExecInfo)]

@@ -66,9 +66,13 @@ h3_status check_no_overlap(const void* const* in, const uint64_t* in_bytes, int 
 h3_status relayout(bool seq_to_head, const void* const* send, void* const* recv,
                    int64_t n_tokens, int32_t planes, int32_t n_heads, int32_t head_dim,
                    int32_t world, int64_t window_bytes, void* stream,
-                   const h3_launch_config* cfg, h3_exec_info* info)
+                   const h3_launch_config* cfg, h3_exec_info* info, int32_t layout = 0)
 {
     clear_info(info);
+    if (layout & ~(H3_LAYOUT_SEQ_PLANE_MAJOR | H3_LAYOUT_HEAD_PLANE_MAJOR))
+        return H3_ERR_INVALID_ARG;
+    if (layout != 0 && cfg && cfg->variant == H3_VARIANT_BULK)
+        return H3_ERR_UNSUPPORTED;  // the bulk ring moves token-major rows only
     h3_status st = check_world(n_tokens, n_heads, world);
     if (st != H3_OK)
         return st;
@@ -137,6 +141,8 @@ h3_status relayout(bool seq_to_head, const void* const* send, void* const* recv,
     a.hm = int32_t(hs.m);
     a.row_vecs = int32_t(row_bytes / kVecBytes);
     a.head_vecs = int32_t(head_bytes / kVecBytes);
+    a.seq_pm = (layout & H3_LAYOUT_SEQ_PLANE_MAJOR) ? 1 : 0;
+    a.head_pm = (layout & H3_LAYOUT_HEAD_PLANE_MAJOR) ? 1 : 0;
 
     const int variant = cfg ? cfg->variant : 0;
     const int ctas_per_sm = cfg ? cfg->ctas_per_sm : 0;
@@ -157,7 +163,8 @@ h3_status relayout(bool seq_to_head, const void* const* send, void* const* recv,
         a.plane0 = c * per_launch;
         a.nplanes = per_launch;
         a.rows = int32_t(n_tokens * per_launch);
-        const cudaError_t err = launch_relayout(seq_to_head, a, variant, ctas_per_sm, s, &shape);
+        const cudaError_t err =
+            launch_relayout(seq_to_head, a, variant, ctas_per_sm, s, &shape, layout != 0);
         if (err != cudaSuccess) {
             if (info) {
                 info->launches = launched;
@@ -434,6 +441,24 @@ h3_status h3_head_to_seq_ex(const void* const* send, void* const* recv, int64_t 
 {
     return relayout(false, send, recv, n_tokens, planes, n_heads, head_dim, world, window_bytes,
                     stream, cfg, info);
+}
+
+h3_status h3_seq_to_head_layout(const void* const* send, void* const* recv, int64_t n_tokens,
+                                int32_t planes, int32_t n_heads, int32_t head_dim, int32_t world,
+                                int64_t window_bytes, int32_t layout, void* stream,
+                                const h3_launch_config* cfg, h3_exec_info* info)
+{
+    return relayout(true, send, recv, n_tokens, planes, n_heads, head_dim, world, window_bytes,
+                    stream, cfg, info, layout);
+}
+
+h3_status h3_head_to_seq_layout(const void* const* send, void* const* recv, int64_t n_tokens,
+                                int32_t planes, int32_t n_heads, int32_t head_dim, int32_t world,
+                                int64_t window_bytes, int32_t layout, void* stream,
+                                const h3_launch_config* cfg, h3_exec_info* info)
+{
+    return relayout(false, send, recv, n_tokens, planes, n_heads, head_dim, world, window_bytes,
+                    stream, cfg, info, layout);
 }
 
 h3_status h3_seq_to_head(const void* const* send, void* const* recv, int64_t n_tokens,

@@ -55,6 +55,8 @@ struct RelayoutArgs {
     int32_t hq, hm;          // head split
     int32_t row_vecs;        // H * D * 2 / 16
     int32_t head_vecs;       // D * 2 / 16
+    int32_t seq_pm;          // sequence side plane-major [P, T_r, H, D] (layout kernels only)
+    int32_t head_pm;         // head side plane-major [P, T, H_j, D] (layout kernels only)
 };
 
 struct ReduceArgs {
@@ -103,9 +105,11 @@ struct LaunchShape {
     int variant = H3_VARIANT_NONE;
 };
 
-// Enqueue one relayout launch.  seq_to_head selects the direction.
+// Enqueue one relayout launch.  seq_to_head selects the direction; layout
+// selects the kernels that read a.seq_pm / a.head_pm (plane-major buffers).
 cudaError_t launch_relayout(bool seq_to_head, const RelayoutArgs& a, int variant,
-                            int ctas_per_sm, cudaStream_t stream, LaunchShape* shape);
+                            int ctas_per_sm, cudaStream_t stream, LaunchShape* shape,
+                            bool layout = false);
 
 // Whether the bulk kernel's shared-memory ring fits one row of these args.
 bool relayout_bulk_fits(const RelayoutArgs& a, int device);

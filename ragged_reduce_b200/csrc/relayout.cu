@@ -91,7 +91,7 @@ __device__ __forceinline__ int32_t split_start(int32_t i, int32_t q, int32_t m)
 // ---------------------------------------------------------------------------
 // vector kernels
 // ---------------------------------------------------------------------------
-template <bool kSeqToHead, int VW, int NT, int VPT, int ROWS>
+template <bool kSeqToHead, int VW, int NT, int VPT, int ROWS, bool kLayout = false>
 __global__ void __launch_bounds__(NT) relayout_vec_kernel(const __grid_constant__ RelayoutArgs a)
 {
     constexpr int kUnits = VW / kVecBytes;  // 16-byte units per vector
@@ -128,8 +128,16 @@ __global__ void __launch_bounds__(NT) relayout_vec_kernel(const __grid_constant_
             const int32_t p = a.plane0 + (ii - t * a.nplanes);
             const int32_t s = split_owner(t, a.tq, a.tm);
             const int32_t tl = t - split_start(s, a.tq, a.tm);
-            g[r] = int64_t(t) * a.P + p;
-            sptr[r] = a.seq[s] + (int64_t(tl) * a.P + p) * seq_row_bytes + int64_t(threadIdx.x) * VW;
+            if constexpr (kLayout) {
+                // plane-major sides: plane p is a contiguous block of T (or T_s) rows
+                const int32_t ts_len = a.tq + (s < a.tm ? 1 : 0);
+                g[r] = a.head_pm ? int64_t(p) * a.T + t : int64_t(t) * a.P + p;
+                const int64_t srow = a.seq_pm ? int64_t(p) * ts_len + tl : int64_t(tl) * a.P + p;
+                sptr[r] = a.seq[s] + srow * seq_row_bytes + int64_t(threadIdx.x) * VW;
+            } else {
+                g[r] = int64_t(t) * a.P + p;
+                sptr[r] = a.seq[s] + (int64_t(tl) * a.P + p) * seq_row_bytes + int64_t(threadIdx.x) * VW;
+            }
         }
         Vec<VW> v[ROWS][VPT];
 #pragma unroll
@@ -158,7 +166,7 @@ __global__ void __launch_bounds__(NT) relayout_vec_kernel(const __grid_constant_
 // Any row width: one row per CTA iteration, head-side placement per vector.
 constexpr int kGenericThreads = 128;
 
-template <bool kSeqToHead>
+template <bool kSeqToHead, bool kLayout = false>
 __global__ void __launch_bounds__(kGenericThreads) relayout_generic_kernel(const __grid_constant__ RelayoutArgs a)
 {
     const int64_t seq_row_bytes = int64_t(a.row_vecs) * kVecBytes;
@@ -168,8 +176,16 @@ __global__ void __launch_bounds__(kGenericThreads) relayout_generic_kernel(const
         const int32_t p = a.plane0 + (i - t * a.nplanes);
         const int32_t s = split_owner(t, a.tq, a.tm);
         const int32_t tl = t - split_start(s, a.tq, a.tm);
-        const int64_t g = int64_t(t) * a.P + p;
-        char* srow = a.seq[s] + (int64_t(tl) * a.P + p) * seq_row_bytes;
+        int64_t g = int64_t(t) * a.P + p;
+        int64_t srow_index = int64_t(tl) * a.P + p;
+        if constexpr (kLayout) {
+            const int32_t ts_len = a.tq + (s < a.tm ? 1 : 0);
+            if (a.head_pm)
+                g = int64_t(p) * a.T + t;
+            if (a.seq_pm)
+                srow_index = int64_t(p) * ts_len + tl;
+        }
+        char* srow = a.seq[s] + srow_index * seq_row_bytes;
         for (int32_t c = threadIdx.x; c < a.row_vecs; c += kGenericThreads) {
             const int32_t h = c / a.head_vecs;
             const int32_t within = c - h * a.head_vecs;
@@ -372,13 +388,13 @@ struct KernelChoice {
 constexpr int kWideCtasPerSm = 4;
 
 // Smallest instantiated vectors-per-thread count (at most MAXV) covering `need`.
-template <bool S2H, int VW, int NT, int ROWS, int MAXV>
+template <bool S2H, int VW, int NT, int ROWS, int MAXV, bool LAYOUT = false>
 bool pick_vec(int need, KernelChoice* kc)
 {
 #define H3RR_VPT(V)                                                              \
     if constexpr (V <= MAXV) {                                                   \
         if (need <= V) {                                                         \
-            kc->fn = (const void*)relayout_vec_kernel<S2H, VW, NT, V, ROWS>;     \
+            kc->fn = (const void*)relayout_vec_kernel<S2H, VW, NT, V, ROWS, LAYOUT>; \
             kc->threads = NT;                                                    \
             kc->rows_per_cta_iter = ROWS;                                        \
             kc->variant = H3_VARIANT_VECTOR;                                     \
@@ -400,21 +416,21 @@ bool pick_vec(int need, KernelChoice* kc)
 // sequence->head with 32-byte vectors, 64 threads and two rows in flight;
 // head->sequence with 32-byte vectors and one warp per CTA.  Wider rows fall
 // back to 16-byte vectors with 128 threads, then to the generic kernel.
-template <bool S2H>
+template <bool S2H, bool LAYOUT = false>
 void choose_vec(const RelayoutArgs& a, bool wide_ok, KernelChoice* kc)
 {
     if (wide_ok) {
         const int row32 = a.row_vecs / 2;
-        const bool ok = S2H ? pick_vec<true, 32, 64, 2, 8>((row32 + 63) / 64, kc)
-                            : pick_vec<false, 32, 32, 1, 16>((row32 + 31) / 32, kc);
+        const bool ok = S2H ? pick_vec<true, 32, 64, 2, 8, LAYOUT>((row32 + 63) / 64, kc)
+                            : pick_vec<false, 32, 32, 1, 16, LAYOUT>((row32 + 31) / 32, kc);
         if (ok) {
             kc->per_sm = kWideCtasPerSm;
             return;
         }
     }
-    if (pick_vec<S2H, 16, 128, 1, 16>((a.row_vecs + 127) / 128, kc))
+    if (pick_vec<S2H, 16, 128, 1, 16, LAYOUT>((a.row_vecs + 127) / 128, kc))
         return;
-    kc->fn = (const void*)relayout_generic_kernel<S2H>;
+    kc->fn = (const void*)relayout_generic_kernel<S2H, LAYOUT>;
     kc->threads = kGenericThreads;
     kc->rows_per_cta_iter = 1;
     kc->variant = H3_VARIANT_VECTOR;
@@ -457,7 +473,7 @@ bool relayout_bulk_fits(const RelayoutArgs& a, int device)
 }
 
 cudaError_t launch_relayout(bool seq_to_head, const RelayoutArgs& a, int variant, int ctas_per_sm,
-                            cudaStream_t stream, LaunchShape* shape)
+                            cudaStream_t stream, LaunchShape* shape, bool layout)
 {
     int device = 0;
     const int sms = current_sm_count(&device);
@@ -471,11 +487,19 @@ cudaError_t launch_relayout(bool seq_to_head, const RelayoutArgs& a, int variant
         bulk = choose_bulk(seq_to_head, a, device, &kc);
     if (variant == H3_VARIANT_BULK && !bulk)
         return cudaErrorInvalidConfiguration;
+    if (bulk && layout)
+        return cudaErrorInvalidConfiguration;  // the bulk ring moves token-major rows only
     if (!bulk) {
-        if (seq_to_head)
+        if (layout) {
+            if (seq_to_head)
+                choose_vec<true, true>(a, wide_vectors_ok(a), &kc);
+            else
+                choose_vec<false, true>(a, wide_vectors_ok(a), &kc);
+        } else if (seq_to_head) {
             choose_vec<true>(a, wide_vectors_ok(a), &kc);
-        else
+        } else {
             choose_vec<false>(a, wide_vectors_ok(a), &kc);
+        }
     } else {
         const cudaError_t err = allow_dynamic_smem(kc.fn, kc.smem, device);
         if (err != cudaSuccess)

@@ -338,3 +338,18 @@ def test_all_gather_argument_checks():
     assert st(outs=[0] + outs[1:]) == E.H3_ERR_INVALID_ARG
     assert st(outs=[ins[2]] + outs[1:]) == E.H3_ERR_INVALID_ARG
     assert st(outs=[outs[0], outs[0] + 1024] + outs[2:]) == E.H3_ERR_INVALID_ARG
+
+
+@needs_no_gpu
+def test_layout_rejects_unknown_bits():
+    T, P, H, D, W = 100, 3, 56, 128, 2
+    send, recv = _layout(T, P, H, D, W)
+    for layout in (4, 8, -1, 7):
+        info = _abi.ExecInfo()
+        st = _abi.lib.h3_seq_to_head_layout(_ptrs(send), _ptrs(recv), T, P, H, D, W, 0, layout, None,
+                                            None, C.byref(info))
+        assert st == _abi.H3_ERR_INVALID_ARG and info.launches == 0
+    cfg = _abi.LaunchConfig(_abi.H3_VARIANT_BULK, 0, 0, 0)
+    st = _abi.lib.h3_head_to_seq_layout(_ptrs(recv), _ptrs(send), T, P, H, D, W, 0, 2, None,
+                                        C.byref(cfg), C.byref(_abi.ExecInfo()))
+    assert st == _abi.H3_ERR_UNSUPPORTED
