@@ -62,6 +62,10 @@ class Oracle:
             f.restype = C.c_int32
             f.argtypes = [C.c_int64, C.c_int32, C.c_int32, C.c_int32, C.c_int32,
                           C.c_int32, C.c_int64, _i64p, _i32p, _i64p]
+        lib.h3o_reduce_scatter_gated.restype = C.c_int32
+        lib.h3o_reduce_scatter_gated.argtypes = [C.c_void_p, C.c_void_p, C.c_void_p, _i64p,
+                                                 C.c_int32, C.c_void_p, C.c_void_p, C.c_int64,
+                                                 C.c_int64, C.c_int32]
         lib.h3o_relayout_layout.restype = C.c_int32
         lib.h3o_relayout_layout.argtypes = [C.c_void_p, C.c_void_p, C.c_int64, C.c_int32,
                                             C.c_int32, C.c_int32, C.c_int32, C.c_int32,
@@ -212,6 +216,28 @@ class Oracle:
         rc = self.lib.h3o_relayout_layout(_ptr_array(src), _ptr_array(out), T, P, H, D, W,
                                           1 if seq_to_head else 0, int(seq_plane_major),
                                           int(head_plane_major))
+        assert rc == 0
+        return out
+
+    def reduce_scatter_gated(self, partials, bias, gate, bounds, x, W: int):
+        """partials: W uint16 [T, C]; bias [C] or None; gate [S, C]; bounds int64 [S+1];
+        x: W uint16 [T_r, C] -> W arrays [T_r, C] = bf16(x + gate[seg] * reduce-scatter)."""
+        src = [np.ascontiguousarray(p, dtype=np.uint16) for p in partials]
+        assert len(src) == W
+        T, Cc = src[0].shape
+        ts = self.partition_range(T, W)
+        xs = [np.ascontiguousarray(v, dtype=np.uint16) for v in x]
+        for r, v in enumerate(xs):
+            assert v.shape == (ts[r + 1] - ts[r], Cc)
+        b = None if bias is None else np.ascontiguousarray(bias, dtype=np.uint16)
+        g = np.ascontiguousarray(gate, dtype=np.uint16)
+        bd = np.ascontiguousarray(bounds, dtype=np.int64)
+        S = len(bd) - 1
+        assert g.shape == (S, Cc)
+        out = [np.zeros_like(v) for v in xs]
+        rc = self.lib.h3o_reduce_scatter_gated(_ptr_array(src), None if b is None else b.ctypes.data,
+                                               g.ctypes.data, _ptr(bd, _i64p), S, _ptr_array(xs),
+                                               _ptr_array(out), T, Cc, W)
         assert rc == 0
         return out
 

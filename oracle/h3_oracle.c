@@ -475,3 +475,59 @@ done:
     return rc;
 }
 
+/* ------------------------------------------------------------------------ */
+/* Ragged reduce-scatter followed by residual gating per packed segment       */
+/* ["Distributed H3 Execution", "Partition Contract": segment boundaries are  */
+/* clipped to each rank's token interval and rebased before AdaLN modulation  */
+/* and residual gating; rank partials are summed by the ragged reduce-scatter */
+/* and the bias is added once after the reduction].                           */
+/*                                                                            */
+/* For rank r and its local row t' (global token t = ts_r + t'):              */
+/*   y        = the reduce-scatter output element (BF16, as defined above)    */
+/*   k        = the global segment of the rank's clipped piece holding t'     */
+/*   out[t',c] = bf16_rne( f(x[t',c]) + f(gate[k,c]) * f(y) )                  */
+/* in binary32: the product of two BF16 values is exact in binary32, then one */
+/* binary32 add, then round to BF16.  x and out are [T_r, C]; gate is [S, C]. */
+/* ------------------------------------------------------------------------ */
+int32_t h3o_reduce_scatter_gated(const uint16_t* const* partials, const uint16_t* bias,
+                                 const uint16_t* gate, const int64_t* bounds, int32_t n_segs,
+                                 const uint16_t* const* x, uint16_t* const* out,
+                                 int64_t T, int64_t C, int32_t W)
+{
+    int64_t* ts = (int64_t*)malloc(sizeof(int64_t) * (size_t)(W + 1));
+    uint16_t* vals = (uint16_t*)malloc(sizeof(uint16_t) * (size_t)W);
+    int64_t* local_bounds = (int64_t*)malloc(sizeof(int64_t) * (size_t)(n_segs + 1));
+    int32_t* seg_ids = (int32_t*)malloc(sizeof(int32_t) * (size_t)(n_segs + 1));
+    int32_t rc = -1;
+    if (!ts || !vals || !local_bounds || !seg_ids)
+        goto done;
+    if (h3o_partition_range(T, W, ts))
+        goto done;
+    for (int32_t r = 0; r < W; ++r) {
+        int32_t pieces = h3o_clip_segments(bounds, n_segs, ts[r], ts[r + 1], local_bounds, seg_ids);
+        int32_t piece = 0;
+        for (int64_t tl = 0; tl < ts[r + 1] - ts[r]; ++tl) {
+            while (piece + 1 < pieces && tl >= local_bounds[piece + 1])
+                ++piece;
+            int64_t k = seg_ids[piece];
+            int64_t t = ts[r] + tl;
+            for (int64_t c = 0; c < C; ++c) {
+                for (int32_t w = 0; w < W; ++w)
+                    vals[w] = partials[w][t * C + c];
+                uint16_t y = reduce_one(vals, W, bias ? &bias[c] : NULL);
+                float g = h3o_bf16_to_f32(gate[k * C + c]);
+                float prod = g * h3o_bf16_to_f32(y);
+                float sum = h3o_bf16_to_f32(x[r][tl * C + c]) + prod;
+                out[r][tl * C + c] = h3o_f32_to_bf16_rne(sum);
+            }
+        }
+    }
+    rc = 0;
+done:
+    free(ts);
+    free(vals);
+    free(local_bounds);
+    free(seg_ids);
+    return rc;
+}
+

@@ -442,6 +442,67 @@ def check_plane_major_layouts(o):
                     assert np.array_equal(back[r], send[r]), ("h2s", spm, hpm, r)
 
 
+def _bf16_of(x: np.ndarray) -> np.ndarray:
+    """BF16 patterns of float32 values by torch's CPU round-to-nearest-even cast."""
+    t = torch.from_numpy(np.ascontiguousarray(x, dtype=np.float32))
+    return t.to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
+
+
+def _f32_of(bits: np.ndarray) -> np.ndarray:
+    return (np.asarray(bits, dtype=np.uint32) << 16).view(np.float32)
+
+
+def check_gated_reduce_scatter(o):
+    """Fused reduce-scatter + gating equals the reduce-scatter followed by
+    the gating written with numpy binary32 arithmetic and torch's BF16 cast;
+    gate 0 leaves x; gate 1 on x = 0 gives the reduce-scatter; per-segment
+    gate values k+1 show each row's segment, matching the clip cases."""
+    rng = np.random.default_rng(18)
+    for T, Cc, W, bounds in [(10, 8, 3, [0, 2, 9, 10]), (1024, 16, 2, [0, 400, 737, 1024]),
+                             (97, 8, 8, [0, 5, 6, 50, 97]), (9, 8, 3, [0, 3, 6, 9]), (33, 24, 1, [0, 33])]:
+        S = len(bounds) - 1
+        partials = [o.f32_to_bf16(rng.normal(0, 0.5, (T, Cc)).astype(np.float32)) for _ in range(W)]
+        bias = o.f32_to_bf16(rng.normal(0, 0.1, Cc).astype(np.float32))
+        gate = o.f32_to_bf16(rng.normal(0, 1.0, (S, Cc)).astype(np.float32))
+        ts = o.partition_range(T, W)
+        x = [o.f32_to_bf16(rng.normal(0, 1.0, (ts[r + 1] - ts[r], Cc)).astype(np.float32)) for r in range(W)]
+        got = o.reduce_scatter_gated(partials, bias, gate, bounds, x, W)
+        y = o.ragged_reduce_scatter(partials, bias, W)
+        seg = np.searchsorted(np.asarray(bounds), np.arange(T), side="right") - 1
+        for r in range(W):
+            rows = np.arange(ts[r], ts[r + 1])
+            want = _bf16_of(_f32_of(x[r]) + _f32_of(gate[seg[rows]]) * _f32_of(y[r]))
+            assert np.array_equal(got[r], want), (T, W, r)
+        zero = [np.zeros(S * Cc, np.uint16).reshape(S, Cc)][0]
+        got0 = o.reduce_scatter_gated(partials, bias, zero, bounds, x, W)
+        for r in range(W):
+            # x + (+-0) is x, except that -0 + +0 is +0: compare where x is not -0
+            keep = x[r] != 0x8000
+            assert np.array_equal(got0[r][keep], x[r][keep])
+        one = np.full((S, Cc), 0x3F80, np.uint16)
+        xz = [np.zeros_like(v) for v in x]
+        got1 = o.reduce_scatter_gated(partials, bias, one, bounds, xz, W)
+        for r in range(W):
+            # +0 + y is y except that y = -0 gives +0
+            assert np.array_equal(got1[r], np.where(y[r] == 0x8000, 0, y[r]).astype(np.uint16))
+    # segment of each row through the clip: gate row k holds k+1, y = 1
+    with open(os.path.join(GOLDEN, "segment_clip_cases.json")) as f:
+        cases = json.load(f)["cases"]
+    for c in cases:
+        T, W, bounds = c["T"], c["W"], c["bounds"]
+        S = len(bounds) - 1
+        Cc = 8
+        partials = [np.full((T, Cc), 0x3F80 if w == 0 else 0, np.uint16) for w in range(W)]
+        gate = np.array([[_bf16_bits_of_exact(float(k + 1))] * Cc for k in range(S)], np.uint16)
+        ts = o.partition_range(T, W)
+        x = [np.zeros((ts[r + 1] - ts[r], Cc), np.uint16) for r in range(W)]
+        got = o.reduce_scatter_gated(partials, None, gate, bounds, x, W)
+        for r, want in enumerate(c["ranks"]):
+            lb, ids = want["local_bounds"], want["seg_ids"]
+            for k, a, b in zip(ids, lb[:-1], lb[1:]):
+                assert np.all(got[r][a:b] == _bf16_bits_of_exact(float(k + 1))), (c["note"], r, k)
+
+
 ALL_CHECKS = [
     check_head_table,
     check_partition_invariants,
@@ -459,6 +520,7 @@ ALL_CHECKS = [
     check_reduce_identities,
     check_all_gather,
     check_plane_major_layouts,
+    check_gated_reduce_scatter,
 ]
 
 

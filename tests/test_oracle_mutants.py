@@ -67,6 +67,11 @@ MUTANTS = [
      "return ((p * Tr + tl) * H + h) * D + (d + p) % D;"),
     ("plane_major_head_swapped", "return ((p * T + t) * Hj + hl) * D + d;",
      "return ((t * P + p) * Hj + hl) * D + d;"),
+    ("gated_piece_never_advances", "            while (piece + 1 < pieces && tl >= local_bounds[piece + 1])\n                ++piece;",
+     "            while (0)\n                ++piece;"),
+    ("gated_uses_rank_as_segment", "            int64_t k = seg_ids[piece];", "            int64_t k = r % n_segs;"),
+    ("gated_product_dropped", "float sum = h3o_bf16_to_f32(x[r][tl * C + c]) + prod;",
+     "float sum = h3o_bf16_to_f32(x[r][tl * C + c]) + g;"),
     ("widen_drops_sign", "uint32_t u = ((uint32_t)b) << 16;", "uint32_t u = ((uint32_t)(b & 0x7FFFu)) << 16;"),
 ]
 
