@@ -592,6 +592,23 @@ def run_workload_report(args):
         emit(rw.name, "ragged_reduce_scatter", "default", nbytes, secs, info)
         del partials, bias, plist, out_full, out
         torch.cuda.empty_cache()
+    for rw, S in ((wl.RS_64K_W8, 16), (wl.ReduceWorkload("reduce_scatter_T32768_C7168_W6", T=32768,
+                                                          C=wl.H3_HIDDEN, W=6, seed=102), 8)):
+        partials, bias = wl.partials_and_bias(rw, dev)
+        plist = list(partials.unbind(0))
+        gate = wl.normal_bf16((S, rw.C), rw.seed + 2, 1.0, dev)
+        bounds = wl.segment_bounds(rw.T, S, rw.seed)
+        x_full, x = rr.alloc_reduce_outputs(rw.T, rw.C, rw.W, dev)
+        x_full.copy_(wl.normal_bf16((rw.T, rw.C), rw.seed + 3, 1.0, dev))
+        out_full, out = rr.alloc_reduce_outputs(rw.T, rw.C, rw.W, dev)
+        nbytes = (rw.W + 2) * rw.T * rw.C * 2 + (S + 1) * rw.C * 2
+        info = rr.ragged_reduce_scatter_gated(plist, bias, gate, bounds, x, out)
+        secs = _time_calls(lambda: rr.ragged_reduce_scatter_gated(plist, bias, gate, bounds, x, out),
+                           iters)
+        emit(rw.name.replace("reduce_scatter", "gated_reduce_scatter"), "ragged_reduce_scatter_gated",
+             "default", nbytes, secs, info)
+        del partials, bias, plist, gate, x_full, x, out_full, out
+        torch.cuda.empty_cache()
     for (T, C_, W) in ((65536, wl.H3_HIDDEN, 8), (32768, wl.H3_HIDDEN, 6)):
         full = wl.normal_bf16((T, C_), 9, 1.0, dev)
         blocks = rr.split_rows(full, rr.partition(T, W, W).token_starts)

@@ -85,6 +85,7 @@ typedef enum h3_status {
 #define H3_VARIANT_REDUCE 3      /* warp-level fp32 reduce-scatter */
 #define H3_VARIANT_STAGED 4      /* pack into a window buffer, then unpack */
 #define H3_VARIANT_GATHER 5      /* ragged all-gather */
+#define H3_VARIANT_REDUCE_GATED 6 /* reduce-scatter fused with residual gating */
 
 typedef struct h3_exec_info {
     int32_t launches;            /* kernel launches enqueued by the call */
@@ -197,6 +198,36 @@ H3RR_API h3_status h3_head_to_seq(const void* const* send, void* const* recv,
 H3RR_API h3_status h3_ragged_reduce_scatter(const void* const* partials, const void* bias,
                                    void* const* out, int64_t n_tokens, int64_t cols,
                                    int32_t world, void* stream, h3_exec_info* info);
+
+/*
+ * h3_ragged_reduce_scatter_gated - the ragged reduce-scatter fused with
+ * residual gating per packed segment ("Distributed H3 Execution", "Partition
+ * Contract": segment boundaries clipped to each rank's token interval and
+ * rebased before AdaLN modulation and residual gating).
+ *
+ *   partials, bias, n_tokens T, cols C, world W : as h3_ragged_reduce_scatter.
+ *   gate       : device [S, C] BF16, one gating row per packed segment.
+ *   seg_bounds : host [S+1], 0 = b_0 < b_1 < ... < b_S = T (as h3_partition),
+ *                1 <= S <= H3RR_MAX_GATE_SEGMENTS; read during the call only.
+ *   x[world]   : device, rank r's residual rows [T_r, C] BF16.
+ *   out[world] : device, rank r's [T_r, C] BF16, written; out[r] may be x[r]
+ *                itself (in place) but must not partly overlap it or overlap
+ *                anything else.
+ *   For rank r, local row t' (t = ts_r + t'), k = the segment holding t
+ *   (equivalently, the global index of the rank's clipped piece holding t'):
+ *     y          = the h3_ragged_reduce_scatter output element (BF16)
+ *     out_r[t',c] = bf16_rne( x_r[t',c] + gate[k,c] * y )   in binary32
+ *   (the BF16 x BF16 product is exact in binary32; one rounding in the add,
+ *   then round to nearest even).  Equal, bit for bit, to running
+ *   h3_ragged_reduce_scatter and then the gating; one launch, and y is never
+ *   written to memory.
+ */
+#define H3RR_MAX_GATE_SEGMENTS 256
+H3RR_API h3_status h3_ragged_reduce_scatter_gated(const void* const* partials, const void* bias,
+                                                  const void* gate, const int64_t* seg_bounds,
+                                                  int32_t n_segs, const void* const* x,
+                                                  void* const* out, int64_t n_tokens, int64_t cols,
+                                                  int32_t world, void* stream, h3_exec_info* info);
 
 /*
  * h3_seq_to_head_layout / h3_head_to_seq_layout - the relayouts with

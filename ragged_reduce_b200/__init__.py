@@ -36,7 +36,7 @@ __all__ = [
     "bulk_wait_timeouts", "alloc_reduce_outputs", "seq_to_head_staged", "head_to_seq_staged",
     "staged_plan", "H3_VARIANT_STAGED", "ragged_all_gather", "H3_VARIANT_GATHER",
     "seq_to_head_layout", "head_to_seq_layout", "H3_LAYOUT_SEQ_PLANE_MAJOR",
-    "H3_LAYOUT_HEAD_PLANE_MAJOR",
+    "H3_LAYOUT_HEAD_PLANE_MAJOR", "ragged_reduce_scatter_gated",
 ]
 
 library_path = _abi.LIB_PATH
@@ -403,6 +403,48 @@ def ragged_all_gather(blocks, out, *, stream=None, variant: int = 0, ctas_per_sm
         else:
             st = _abi.lib.h3_ragged_all_gather_ex(*args, cfg, C.byref(info))
     _abi.check(st, "h3_ragged_all_gather")
+    return info.as_dict()
+
+
+def ragged_reduce_scatter_gated(partials, bias, gate, seg_bounds, x, out=None, *,
+                                stream=None) -> dict:
+    """Ragged reduce-scatter fused with residual gating per packed segment
+    (``h3_ragged_reduce_scatter_gated``): out_r = bf16(x_r + gate[seg] * y_r),
+    y_r the reduce-scatter output rows of rank r.  gate: BF16 [S, C];
+    seg_bounds: S+1 packed segment bounds (0 .. T); x: W tensors [T_r, C];
+    out: W tensors [T_r, C], or None to update x in place."""
+    partials = _as_list(partials)
+    x = _as_list(x)
+    out = x if out is None else _as_list(out)
+    W = len(partials)
+    if W < 1 or len(x) != W or len(out) != W:
+        raise ValueError("partials, x and out need one tensor per rank (same count)")
+    tensors = partials + x + out + [gate] + ([bias] if bias is not None else [])
+    dev = _check_tensors(tensors, "ragged_reduce_scatter_gated")
+    if any(t.dtype != torch.bfloat16 for t in tensors):
+        raise ValueError("ragged_reduce_scatter_gated works on BF16 tensors")
+    T, Cc = partials[0].shape
+    b = np.ascontiguousarray(seg_bounds, dtype=np.int64)
+    S = len(b) - 1
+    if tuple(gate.shape) != (S, Cc):
+        raise ValueError(f"gate must be [S, C] = [{S}, {Cc}]")
+    if T >= W:
+        part = partition(T, W, W)
+        for r in range(W):
+            for name, t in (("x", x[r]), ("out", out[r])):
+                if tuple(t.shape) != (part.tokens(r), Cc):
+                    raise ValueError(f"{name} rank {r}: shape {tuple(t.shape)}, expected "
+                                     f"{(part.tokens(r), Cc)}")
+    info = ExecInfo()
+    with torch.cuda.device(dev):
+        st = _abi.lib.h3_ragged_reduce_scatter_gated(
+            _abi.pointer_array([p.data_ptr() for p in partials]),
+            C.c_void_p(bias.data_ptr() if bias is not None else 0), C.c_void_p(gate.data_ptr()),
+            b.ctypes.data_as(_abi._i64p), S,
+            _abi.pointer_array([v.data_ptr() for v in x]),
+            _abi.pointer_array([o.data_ptr() for o in out]),
+            int(T), int(Cc), W, C.c_void_p(_stream_handle(stream, dev)), C.byref(info))
+    _abi.check(st, "h3_ragged_reduce_scatter_gated")
     return info.as_dict()
 
 

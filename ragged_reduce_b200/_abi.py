@@ -37,6 +37,8 @@ H3_VARIANT_BULK = 2
 H3_VARIANT_REDUCE = 3
 H3_VARIANT_STAGED = 4
 H3_VARIANT_GATHER = 5
+H3_VARIANT_REDUCE_GATED = 6
+MAX_GATE_SEGMENTS = 256
 
 MAX_WORLD = 64
 H3_LAYOUT_SEQ_PLANE_MAJOR = 1
@@ -135,6 +137,10 @@ def _load() -> C.CDLL:
     lib.h3_ragged_all_gather_ex.argtypes = [_vpp, _vpp, C.c_int64, C.c_int64, C.c_int32,
                                             C.c_void_p, C.POINTER(LaunchConfig),
                                             C.POINTER(ExecInfo)]
+    lib.h3_ragged_reduce_scatter_gated.restype = C.c_int
+    lib.h3_ragged_reduce_scatter_gated.argtypes = [_vpp, C.c_void_p, C.c_void_p, _i64p, C.c_int32,
+                                                   _vpp, _vpp, C.c_int64, C.c_int64, C.c_int32,
+                                                   C.c_void_p, C.POINTER(ExecInfo)]
     lib.h3_staged_plan.restype = C.c_int
     lib.h3_staged_plan.argtypes = [C.c_int64, C.c_int32, C.c_int32, C.c_int32, C.c_int64,
                                    _i64p, _i64p]

@@ -641,6 +641,91 @@ h3_status h3_ragged_all_gather_ex(const void* const* in, void* const* out, int64
     return H3_OK;
 }
 
+h3_status h3_ragged_reduce_scatter_gated(const void* const* partials, const void* bias,
+                                         const void* gate, const int64_t* seg_bounds,
+                                         int32_t n_segs, const void* const* x, void* const* out,
+                                         int64_t n_tokens, int64_t cols, int32_t world,
+                                         void* stream, h3_exec_info* info)
+{
+    clear_info(info);
+    h3_status st = check_world(n_tokens, world, world);
+    if (st != H3_OK)
+        return st;
+    if (cols < 1 || !partials || !out || !x || !gate || !seg_bounds)
+        return H3_ERR_INVALID_ARG;
+    if (n_segs < 1 || n_segs > H3RR_MAX_GATE_SEGMENTS)
+        return n_segs < 1 ? H3_ERR_INVALID_ARG : H3_ERR_UNSUPPORTED;
+    if (seg_bounds[0] != 0 || seg_bounds[n_segs] != n_tokens)
+        return H3_ERR_INVALID_ARG;
+    for (int32_t k = 0; k < n_segs; ++k)
+        if (seg_bounds[k + 1] <= seg_bounds[k])
+            return H3_ERR_INVALID_ARG;
+    if (cols % 8 != 0)
+        return H3_ERR_MISALIGNED;
+    if (n_tokens > kMaxInt32 || cols / 8 > kMaxRowVecs)
+        return H3_ERR_UNSUPPORTED;
+    if (!aligned16(gate) || (bias && !aligned16(bias)))
+        return H3_ERR_MISALIGNED;
+    const Split ts = make_split(n_tokens, world);
+    const uint64_t row_bytes = uint64_t(cols) * 2;
+    for (int r = 0; r < world; ++r) {
+        if (!partials[r] || !out[r] || !x[r])
+            return H3_ERR_INVALID_ARG;
+        if (!aligned16(partials[r]) || !aligned16(out[r]) || !aligned16(x[r]))
+            return H3_ERR_MISALIGNED;
+    }
+    // Outputs against every input and each other; out[r] may be x[r] exactly.
+    for (int r = 0; r < world; ++r) {
+        const uintptr_t o = reinterpret_cast<uintptr_t>(out[r]);
+        const uint64_t on = uint64_t(ts.size(r)) * row_bytes;
+        const bool in_place = out[r] == x[r];
+        for (int k = 0; k < world; ++k) {
+            if (ranges_overlap(o, on, reinterpret_cast<uintptr_t>(partials[k]), uint64_t(n_tokens) * row_bytes))
+                return H3_ERR_INVALID_ARG;
+            if (!(in_place && k == r) &&
+                ranges_overlap(o, on, reinterpret_cast<uintptr_t>(x[k]), uint64_t(ts.size(k)) * row_bytes))
+                return H3_ERR_INVALID_ARG;
+            if (k > r && ranges_overlap(o, on, reinterpret_cast<uintptr_t>(out[k]),
+                                        uint64_t(ts.size(k)) * row_bytes))
+                return H3_ERR_INVALID_ARG;
+        }
+        if (ranges_overlap(o, on, reinterpret_cast<uintptr_t>(gate), uint64_t(n_segs) * row_bytes) ||
+            (bias && ranges_overlap(o, on, reinterpret_cast<uintptr_t>(bias), row_bytes)))
+            return H3_ERR_INVALID_ARG;
+    }
+    GatedArgs g;
+    std::memset(&g, 0, sizeof(g));
+    for (int r = 0; r < world; ++r) {
+        g.r.part[r] = static_cast<const char*>(partials[r]);
+        g.r.out[r] = static_cast<char*>(out[r]);
+        g.x[r] = static_cast<const char*>(x[r]);
+    }
+    g.r.bias = static_cast<const char*>(bias);
+    g.r.T = int32_t(n_tokens);
+    g.r.W = world;
+    g.r.tq = int32_t(ts.q);
+    g.r.tm = int32_t(ts.m);
+    g.r.row_vecs = int32_t(cols / 8);
+    g.r.row_bytes = int64_t(row_bytes);
+    g.gate = static_cast<const char*>(gate);
+    g.n_segs = n_segs;
+    for (int32_t k = 0; k <= n_segs; ++k)
+        g.seg_bounds[k] = int32_t(seg_bounds[k]);
+    LaunchShape shape;
+    const cudaError_t err = launch_reduce_scatter_gated(g, static_cast<cudaStream_t>(stream), &shape);
+    if (err != cudaSuccess)
+        return cuda_failure(err);
+    if (info) {
+        info->launches = 1;
+        info->chunks = 1;
+        info->grid = shape.grid;
+        info->block = shape.block;
+        info->variant = shape.variant;
+        info->planes_per_launch = 1;
+    }
+    return H3_OK;
+}
+
 h3_status h3_ragged_reduce_scatter(const void* const* partials, const void* bias, void* const* out,
                                    int64_t n_tokens, int64_t cols, int32_t world, void* stream,
                                    h3_exec_info* info)

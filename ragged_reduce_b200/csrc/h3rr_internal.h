@@ -99,6 +99,16 @@ struct GatherArgs {
     int64_t row_bytes;  // C * 2
 };
 
+// Reduce-scatter fused with residual gating per packed segment.
+constexpr int kMaxGateSegs = 256;
+struct GatedArgs {
+    ReduceArgs r;                       // partials, out (written), bias, sizes
+    const char* x[kMaxWorld];           // residual rows [T_r, C] (may equal r.out[.])
+    const char* gate;                   // [S, C]
+    int32_t n_segs;
+    int32_t seg_bounds[kMaxGateSegs + 1];  // 0 = b_0 < ... < b_S = T
+};
+
 struct LaunchShape {
     int grid = 0;
     int block = 0;
@@ -135,6 +145,9 @@ cudaError_t launch_all_gather(const GatherArgs& a, int variant, int ctas_per_sm,
                               LaunchShape* shape);
 bool all_gather_bulk_fits(const GatherArgs& a, int device);
 cudaError_t read_gather_wait_timeouts(unsigned int* count, bool reset, cudaStream_t stream);
+
+// Enqueue the gated reduce-scatter launch.
+cudaError_t launch_reduce_scatter_gated(const GatedArgs& a, cudaStream_t stream, LaunchShape* shape);
 
 // Enqueue the reduce-scatter launch.
 cudaError_t launch_reduce_scatter(const ReduceArgs& a, int ctas_per_sm, cudaStream_t stream,

@@ -169,7 +169,121 @@ const void* pick_reduce_kernel(int W)
     }
 }
 
+// ---------------------------------------------------------------------------
+// Reduce-scatter fused with residual gating ("Distributed H3 Execution",
+// "Partition Contract": segment boundaries clipped to each rank's token
+// interval and rebased before AdaLN modulation and residual gating).  Per
+// element: y = the reduce-scatter output (rounded to BF16, exactly as the
+// plain kernel writes it), then out = bf16_rne(x + gate[seg(t)] * y) in
+// binary32.  The product of two BF16 values is exact in binary32, so only the
+// add rounds; fusing changes no bits against running the two steps in turn and
+// saves writing and re-reading y.  seg(t) is found by binary search over the
+// packed segment bounds (the rank's clipped pieces name the same segments).
+// x may be the output buffer itself (in place): each element is read by the
+// thread that then writes it, with plain (coherent) loads.
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ uint4 ld_plain(const char* p)
+{
+    uint4 v;
+    asm volatile("ld.global.v4.u32 {%0, %1, %2, %3}, [%4];"
+                 : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+                 : "l"(p));
+    return v;
+}
+
+template <int kW>
+__global__ void __launch_bounds__(kThreads) reduce_scatter_gated_kernel(const __grid_constant__ GatedArgs g)
+{
+    const ReduceArgs& a = g.r;
+    constexpr int kBatch = kW > 0 ? kW : 8;
+    for (int64_t t64 = blockIdx.x; t64 < a.T; t64 += gridDim.x) {
+        const int32_t t = int32_t(t64);
+        const int32_t s = split_owner(t, a.tq, a.tm);
+        const int32_t tl = t - split_start(s, a.tq, a.tm);
+        int32_t lo = 0, hi = g.n_segs;  // largest k with bounds[k] <= t
+        while (hi - lo > 1) {
+            const int32_t mid = (lo + hi) >> 1;
+            if (g.seg_bounds[mid] <= t)
+                lo = mid;
+            else
+                hi = mid;
+        }
+        const char* grow = g.gate + int64_t(lo) * a.row_bytes;
+        const char* xrow = g.x[s] + int64_t(tl) * a.row_bytes;
+        char* orow = a.out[s] + int64_t(tl) * a.row_bytes;
+        const int64_t in_off = int64_t(t) * a.row_bytes;
+        for (int32_t c = threadIdx.x; c < a.row_vecs; c += kThreads) {
+            const int64_t off = int64_t(c) * kVecBytes;
+            float acc[8];
+            const int W = kW > 0 ? kW : a.W;
+            for (int w0 = 0; w0 < W; w0 += kBatch) {
+                uint4 xv[kBatch];
+#pragma unroll
+                for (int b = 0; b < kBatch; ++b)
+                    if (w0 + b < W)
+                        xv[b] = ld_stream(a.part[w0 + b] + in_off + off);
+#pragma unroll
+                for (int b = 0; b < kBatch; ++b) {
+                    if (w0 + b >= W)
+                        break;
+                    if (w0 + b == 0)
+                        widen(xv[b], acc);
+                    else
+                        add_widened(xv[b], acc);
+                }
+            }
+            if (a.bias != nullptr)
+                add_widened(ld_cached(a.bias + off), acc);
+            float y[8], gt[8], xr[8];
+            widen(narrow_rne(acc), y);          // the reduce-scatter output, as BF16
+            widen(ld_cached(grow + off), gt);
+            widen(ld_plain(xrow + off), xr);
+#pragma unroll
+            for (int e = 0; e < 8; ++e)
+                acc[e] = __fadd_rn(xr[e], __fmul_rn(gt[e], y[e]));
+            st_stream(orow + off, narrow_rne(acc));
+        }
+    }
+}
+
+const void* pick_gated_kernel(int W)
+{
+    switch (W) {
+        case 1: return (const void*)reduce_scatter_gated_kernel<1>;
+        case 2: return (const void*)reduce_scatter_gated_kernel<2>;
+        case 3: return (const void*)reduce_scatter_gated_kernel<3>;
+        case 4: return (const void*)reduce_scatter_gated_kernel<4>;
+        case 5: return (const void*)reduce_scatter_gated_kernel<5>;
+        case 6: return (const void*)reduce_scatter_gated_kernel<6>;
+        case 7: return (const void*)reduce_scatter_gated_kernel<7>;
+        case 8: return (const void*)reduce_scatter_gated_kernel<8>;
+        default: return (const void*)reduce_scatter_gated_kernel<0>;
+    }
+}
+
 }  // namespace
+
+cudaError_t launch_reduce_scatter_gated(const GatedArgs& a, cudaStream_t stream, LaunchShape* shape)
+{
+    const void* kernel = pick_gated_kernel(a.r.W);
+    int device = 0;
+    const int sms = current_sm_count(&device);
+    if (sms <= 0)
+        return cudaErrorNoDevice;
+    const int per_sm = resident_ctas(kernel, kThreads, 0, device);
+    int64_t grid = int64_t(sms) * per_sm;
+    if (grid > a.r.T)
+        grid = a.r.T;
+    if (grid < 1)
+        grid = 1;
+    if (shape) {
+        shape->grid = int(grid);
+        shape->block = kThreads;
+        shape->variant = H3_VARIANT_REDUCE_GATED;
+    }
+    void* params[] = {const_cast<GatedArgs*>(&a)};
+    return cudaLaunchKernel(kernel, dim3(unsigned(grid)), dim3(kThreads), params, 0, stream);
+}
 
 cudaError_t launch_reduce_scatter(const ReduceArgs& a, int ctas_per_sm, cudaStream_t stream,
                                   LaunchShape* shape)

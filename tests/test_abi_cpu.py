@@ -353,3 +353,45 @@ def test_layout_rejects_unknown_bits():
     st = _abi.lib.h3_head_to_seq_layout(_ptrs(recv), _ptrs(send), T, P, H, D, W, 0, 2, None,
                                         C.byref(cfg), C.byref(_abi.ExecInfo()))
     assert st == _abi.H3_ERR_UNSUPPORTED
+
+
+@needs_no_gpu
+def test_gated_argument_checks():
+    T, Cc, W = 1000, 7168, 6
+    addr = BASE
+    parts, xs, outs = [], [], []
+    for _ in range(W):
+        parts.append(addr)
+        addr += T * Cc * 2 + 4096
+    for r in range(W):
+        xs.append(addr)
+        addr += (T // W + 1) * Cc * 2 + 4096
+    for r in range(W):
+        outs.append(addr)
+        addr += (T // W + 1) * Cc * 2 + 4096
+    gate = addr
+    addr += 300 * Cc * 2
+    bias = addr
+
+    def st(bounds=(0, 400, 1000), outs=outs, xs=xs, gate=gate, W=W, T=T):
+        b = np.asarray(bounds, dtype=np.int64)
+        info = _abi.ExecInfo()
+        s = _abi.lib.h3_ragged_reduce_scatter_gated(
+            _ptrs(parts[:max(W, 0)] + [0] * max(0, W - len(parts))), C.c_void_p(bias), C.c_void_p(gate),
+            b.ctypes.data_as(_abi._i64p), len(b) - 1, _ptrs(xs), _ptrs(outs), T, Cc, W, None,
+            C.byref(info))
+        assert info.launches == 0
+        return s
+
+    E = _abi
+    assert st(bounds=(0, 400, 400, 1000)) == E.H3_ERR_INVALID_ARG
+    assert st(bounds=(1, 400, 1000)) == E.H3_ERR_INVALID_ARG
+    assert st(bounds=(0, 400, 999)) == E.H3_ERR_INVALID_ARG
+    assert st(bounds=tuple(range(0, 1000, 3)) + (1000,)) == E.H3_ERR_UNSUPPORTED  # 334 segments
+    assert st(gate=gate + 8) == E.H3_ERR_MISALIGNED
+    assert st(gate=0) == E.H3_ERR_INVALID_ARG
+    assert st(outs=[xs[0] + 16] + outs[1:]) == E.H3_ERR_INVALID_ARG   # partial overlap with x
+    assert st(outs=[parts[1]] + outs[1:]) == E.H3_ERR_INVALID_ARG
+    assert st(outs=[gate] + outs[1:]) == E.H3_ERR_INVALID_ARG
+    assert st(outs=[xs[1]] + outs[1:]) == E.H3_ERR_INVALID_ARG          # another rank's x
+    assert st(T=5) == E.H3_ERR_EMPTY_PARTITION
