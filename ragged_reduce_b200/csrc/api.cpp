@@ -63,6 +63,50 @@ h3_status check_no_overlap(const void* const* in, const uint64_t* in_bytes, int 
     return H3_OK;
 }
 
+h3_status check_relayout_args(bool seq_to_head, const void* const* send, void* const* recv,
+                              int64_t n_tokens, int32_t planes, int32_t n_heads, int32_t head_dim,
+                              int32_t world, void* extra_out, uint64_t extra_bytes)
+{
+    h3_status st = check_world(n_tokens, n_heads, world);
+    if (st != H3_OK)
+        return st;
+    if (planes < 1 || head_dim < 1 || !send || !recv)
+        return H3_ERR_INVALID_ARG;
+    if ((int64_t(head_dim) * 2) % kVecBytes != 0)
+        return H3_ERR_MISALIGNED;
+    if (n_tokens > kMaxInt32 || n_tokens * planes > kMaxInt32 ||
+        int64_t(n_heads) * head_dim * 2 / kVecBytes > kMaxRowVecs)
+        return H3_ERR_UNSUPPORTED;
+    const Split ts = make_split(n_tokens, world);
+    const Split hs = make_split(n_heads, world);
+    const uint64_t row_bytes = uint64_t(n_heads) * head_dim * 2;
+    const uint64_t head_bytes = uint64_t(head_dim) * 2;
+    uint64_t seq_bytes[kMaxWorld];
+    uint64_t head_side_bytes[kMaxWorld + 1];
+    void* outs[kMaxWorld + 1];
+    for (int r = 0; r < world; ++r) {
+        if (!send[r] || !recv[r])
+            return H3_ERR_INVALID_ARG;
+        if (!aligned16(send[r]) || !aligned16(recv[r]))
+            return H3_ERR_MISALIGNED;
+        seq_bytes[r] = uint64_t(ts.size(r)) * planes * row_bytes;
+        head_side_bytes[r] = uint64_t(n_tokens) * planes * uint64_t(hs.size(r)) * head_bytes;
+    }
+    const uint64_t* in_bytes = seq_to_head ? seq_bytes : head_side_bytes;
+    uint64_t out_bytes[kMaxWorld + 1];
+    for (int r = 0; r < world; ++r) {
+        outs[r] = recv[r];
+        out_bytes[r] = seq_to_head ? head_side_bytes[r] : seq_bytes[r];
+    }
+    int n_out = world;
+    if (extra_out) {
+        outs[n_out] = extra_out;
+        out_bytes[n_out] = extra_bytes;
+        ++n_out;
+    }
+    return check_no_overlap(send, in_bytes, world, outs, out_bytes, n_out);
+}
+
 h3_status relayout(bool seq_to_head, const void* const* send, void* const* recv,
                    int64_t n_tokens, int32_t planes, int32_t n_heads, int32_t head_dim,
                    int32_t world, int64_t window_bytes, void* stream,
@@ -73,45 +117,21 @@ h3_status relayout(bool seq_to_head, const void* const* send, void* const* recv,
         return H3_ERR_INVALID_ARG;
     if (layout != 0 && cfg && cfg->variant == H3_VARIANT_BULK)
         return H3_ERR_UNSUPPORTED;  // the bulk ring moves token-major rows only
-    h3_status st = check_world(n_tokens, n_heads, world);
-    if (st != H3_OK)
-        return st;
-    if (planes < 1 || head_dim < 1 || window_bytes < 0 || !send || !recv)
+    if (window_bytes < 0)
         return H3_ERR_INVALID_ARG;
     if (cfg && cfg->variant != 0 && cfg->variant != H3_VARIANT_VECTOR && cfg->variant != H3_VARIANT_BULK)
         return H3_ERR_INVALID_ARG;
     if (cfg && cfg->ctas_per_sm < 0)
         return H3_ERR_INVALID_ARG;
-    if ((int64_t(head_dim) * 2) % kVecBytes != 0)
-        return H3_ERR_MISALIGNED;
-    // Index ranges of the kernels: rows (token, plane) and row vectors in int32.
-    if (n_tokens > kMaxInt32 || n_tokens * planes > kMaxInt32 ||
-        int64_t(n_heads) * head_dim * 2 / kVecBytes > kMaxRowVecs)
-        return H3_ERR_UNSUPPORTED;
+    h3_status st = check_relayout_args(seq_to_head, send, recv, n_tokens, planes, n_heads, head_dim,
+                                       world, nullptr, 0);
+    if (st != H3_OK)
+        return st;
 
     const Split ts = make_split(n_tokens, world);
     const Split hs = make_split(n_heads, world);
     const uint64_t row_bytes = uint64_t(n_heads) * head_dim * 2;  // one (token, plane) row
     const uint64_t head_bytes = uint64_t(head_dim) * 2;
-
-    // Sequence-side and head-side byte sizes per rank.
-    uint64_t seq_bytes[kMaxWorld];
-    uint64_t head_side_bytes[kMaxWorld];
-    for (int r = 0; r < world; ++r) {
-        seq_bytes[r] = uint64_t(ts.size(r)) * planes * row_bytes;
-        head_side_bytes[r] = uint64_t(n_tokens) * planes * uint64_t(hs.size(r)) * head_bytes;
-    }
-    for (int r = 0; r < world; ++r) {
-        if (!send[r] || !recv[r])
-            return H3_ERR_INVALID_ARG;
-        if (!aligned16(send[r]) || !aligned16(recv[r]))
-            return H3_ERR_MISALIGNED;
-    }
-    const uint64_t* in_bytes = seq_to_head ? seq_bytes : head_side_bytes;
-    const uint64_t* out_bytes = seq_to_head ? head_side_bytes : seq_bytes;
-    st = check_no_overlap(send, in_bytes, world, recv, out_bytes, world);
-    if (st != H3_OK)
-        return st;
 
     // Chunked mode (FastVideo PR #1807, "Problem and behavior"): one batch
     // plane per launch; one plane's per-rank send and receive slices must
@@ -187,50 +207,6 @@ h3_status relayout(bool seq_to_head, const void* const* send, void* const* recv,
 
 // Shared checks of the relayout calls: world, shapes, pointers, alignment,
 // overlap.  `extra_out` (nullable) is one more output range (the window).
-h3_status check_relayout_args(bool seq_to_head, const void* const* send, void* const* recv,
-                              int64_t n_tokens, int32_t planes, int32_t n_heads, int32_t head_dim,
-                              int32_t world, void* extra_out, uint64_t extra_bytes)
-{
-    h3_status st = check_world(n_tokens, n_heads, world);
-    if (st != H3_OK)
-        return st;
-    if (planes < 1 || head_dim < 1 || !send || !recv)
-        return H3_ERR_INVALID_ARG;
-    if ((int64_t(head_dim) * 2) % kVecBytes != 0)
-        return H3_ERR_MISALIGNED;
-    if (n_tokens > kMaxInt32 || n_tokens * planes > kMaxInt32 ||
-        int64_t(n_heads) * head_dim * 2 / kVecBytes > kMaxRowVecs)
-        return H3_ERR_UNSUPPORTED;
-    const Split ts = make_split(n_tokens, world);
-    const Split hs = make_split(n_heads, world);
-    const uint64_t row_bytes = uint64_t(n_heads) * head_dim * 2;
-    const uint64_t head_bytes = uint64_t(head_dim) * 2;
-    uint64_t seq_bytes[kMaxWorld];
-    uint64_t head_side_bytes[kMaxWorld + 1];
-    void* outs[kMaxWorld + 1];
-    for (int r = 0; r < world; ++r) {
-        if (!send[r] || !recv[r])
-            return H3_ERR_INVALID_ARG;
-        if (!aligned16(send[r]) || !aligned16(recv[r]))
-            return H3_ERR_MISALIGNED;
-        seq_bytes[r] = uint64_t(ts.size(r)) * planes * row_bytes;
-        head_side_bytes[r] = uint64_t(n_tokens) * planes * uint64_t(hs.size(r)) * head_bytes;
-    }
-    const uint64_t* in_bytes = seq_to_head ? seq_bytes : head_side_bytes;
-    uint64_t out_bytes[kMaxWorld + 1];
-    for (int r = 0; r < world; ++r) {
-        outs[r] = recv[r];
-        out_bytes[r] = seq_to_head ? head_side_bytes[r] : seq_bytes[r];
-    }
-    int n_out = world;
-    if (extra_out) {
-        outs[n_out] = extra_out;
-        out_bytes[n_out] = extra_bytes;
-        ++n_out;
-    }
-    return check_no_overlap(send, in_bytes, world, outs, out_bytes, n_out);
-}
-
 h3_status staged_plan(int64_t n_tokens, int32_t n_heads, int32_t head_dim, int64_t window_bytes,
                       int64_t* chunk_tokens)
 {
