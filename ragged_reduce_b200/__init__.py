@@ -36,7 +36,9 @@ __all__ = [
     "bulk_wait_timeouts", "alloc_reduce_outputs", "seq_to_head_staged", "head_to_seq_staged",
     "staged_plan", "H3_VARIANT_STAGED", "ragged_all_gather", "H3_VARIANT_GATHER",
     "seq_to_head_layout", "head_to_seq_layout", "H3_LAYOUT_SEQ_PLANE_MAJOR",
-    "H3_LAYOUT_HEAD_PLANE_MAJOR", "ragged_reduce_scatter_gated",
+    "H3_LAYOUT_HEAD_PLANE_MAJOR", "ragged_reduce_scatter_gated", "PreparedRelayout",
+    "PreparedReduceScatter", "prepare_seq_to_head", "prepare_head_to_seq",
+    "prepare_ragged_reduce_scatter",
 ]
 
 library_path = _abi.LIB_PATH
@@ -446,6 +448,110 @@ def ragged_reduce_scatter_gated(partials, bias, gate, seg_bounds, x, out=None, *
             int(T), int(Cc), W, C.c_void_p(_stream_handle(stream, dev)), C.byref(info))
     _abi.check(st, "h3_ragged_reduce_scatter_gated")
     return info.as_dict()
+
+
+# ---------------------------------------------------------------------------
+# prepared calls: validate and marshal once, then one C call per invocation
+# ---------------------------------------------------------------------------
+
+class PreparedRelayout:
+    """A relayout whose shapes, buffers and launch options are checked and
+    marshalled once; calling it issues one C call (``h3_*_layout``) on the
+    given (or current) stream.  The buffers are captured by address: refill
+    them in place between calls, do not replace them.
+
+    ``inverse(send, recv)`` prepares the opposite direction over the same
+    shapes (FastVideo PR #1807, "Problem and behavior": the backward pass
+    reuses the plan saved by its forward)."""
+
+    def __init__(self, seq_to_head_dir: bool, send, recv, *, layout: int = 0,
+                 window_bytes: int = 0, variant: int = 0, ctas_per_sm: int = 0):
+        send = _as_list(send)
+        recv = _as_list(recv)
+        T, P, H, D, W, dev = _relayout_shapes(seq_to_head_dir, send, recv, layout)
+        self.seq_to_head_dir = seq_to_head_dir
+        self.shape = (T, P, H, D, W)
+        self.device = dev
+        self.layout = int(layout)
+        self.window_bytes = int(window_bytes)
+        self.variant = int(variant)
+        self.ctas_per_sm = int(ctas_per_sm)
+        self._keep = (send, recv)  # keep the tensors alive while the call holds their addresses
+        name = "h3_seq_to_head_layout" if seq_to_head_dir else "h3_head_to_seq_layout"
+        self._fn = getattr(_abi.lib, name)
+        self._name = name
+        self._cfg = LaunchConfig(self.variant, self.ctas_per_sm, 0, 0)
+        self._info = ExecInfo()
+        self._head = (_abi.pointer_array([t.data_ptr() for t in send]),
+                      _abi.pointer_array([t.data_ptr() for t in recv]),
+                      T, P, H, D, W, self.window_bytes, self.layout)
+
+    def __call__(self, stream=None) -> ExecInfo:
+        s = self.device_stream(stream)
+        st = self._fn(*self._head, s, C.byref(self._cfg), C.byref(self._info))
+        if st != _abi.H3_OK:
+            raise H3Error(st, self._name)
+        return self._info
+
+    def device_stream(self, stream):
+        if stream is None:
+            return C.c_void_p(torch.cuda.current_stream(self.device).cuda_stream)
+        return C.c_void_p(_stream_handle(stream, self.device))
+
+    def inverse(self, send, recv) -> "PreparedRelayout":
+        """The opposite direction with the same layout, window and launch
+        options; send/recv are that direction's buffers."""
+        return PreparedRelayout(not self.seq_to_head_dir, send, recv, layout=self.layout,
+                                window_bytes=self.window_bytes, variant=self.variant,
+                                ctas_per_sm=self.ctas_per_sm)
+
+
+def prepare_seq_to_head(send, recv, **kw) -> PreparedRelayout:
+    """Prepared ``seq_to_head`` / ``seq_to_head_layout`` (see ``PreparedRelayout``)."""
+    return PreparedRelayout(True, send, recv, **kw)
+
+
+def prepare_head_to_seq(send, recv, **kw) -> PreparedRelayout:
+    """Prepared ``head_to_seq`` / ``head_to_seq_layout`` (see ``PreparedRelayout``)."""
+    return PreparedRelayout(False, send, recv, **kw)
+
+
+class PreparedReduceScatter:
+    """A ragged reduce-scatter checked and marshalled once; each call is one
+    ``h3_ragged_reduce_scatter_ex`` call.  Buffers are captured by address."""
+
+    def __init__(self, partials, bias, out, *, ctas_per_sm: int = 0):
+        partials = _as_list(partials)
+        out = _as_list(out)
+        W = len(partials)
+        tensors = partials + out + ([bias] if bias is not None else [])
+        self.device = _check_tensors(tensors, "ragged_reduce_scatter")
+        if any(t.dtype != torch.bfloat16 for t in tensors):
+            raise ValueError("ragged_reduce_scatter works on BF16 tensors")
+        T, Cc = partials[0].shape
+        if any(tuple(p.shape) != (T, Cc) for p in partials) or len(out) != W:
+            raise ValueError("partials must share one [T, C] shape, one output per rank")
+        part = partition(T, W, W)
+        for r, o in enumerate(out):
+            if tuple(o.shape) != (part.tokens(r), Cc):
+                raise ValueError(f"out rank {r}: shape {tuple(o.shape)}, expected {(part.tokens(r), Cc)}")
+        self._keep = (partials, bias, out)
+        self._cfg = LaunchConfig(0, int(ctas_per_sm), 0, 0)
+        self._info = ExecInfo()
+        self._head = (_abi.pointer_array([p.data_ptr() for p in partials]),
+                      C.c_void_p(bias.data_ptr() if bias is not None else 0),
+                      _abi.pointer_array([o.data_ptr() for o in out]), int(T), int(Cc), W)
+
+    def __call__(self, stream=None) -> ExecInfo:
+        s = C.c_void_p(_stream_handle(stream, self.device))
+        st = _abi.lib.h3_ragged_reduce_scatter_ex(*self._head, s, C.byref(self._cfg), C.byref(self._info))
+        if st != _abi.H3_OK:
+            raise H3Error(st, "h3_ragged_reduce_scatter")
+        return self._info
+
+
+def prepare_ragged_reduce_scatter(partials, bias, out, **kw) -> PreparedReduceScatter:
+    return PreparedReduceScatter(partials, bias, out, **kw)
 
 
 def alloc_reduce_outputs(T: int, C_: int, W: int, device, dtype=torch.bfloat16):

@@ -122,3 +122,18 @@ def test_full_reduce_scatter_64k_w8(oracle_lib):
     # rows land in their rank's buffer
     for r in range(w.W):
         assert out[r].data_ptr() == out_full[int(part.token_starts[r])].data_ptr()
+
+
+def test_prepared_reduce_scatter(oracle_lib):
+    T, C, W = 500, 7168, 6
+    w = wl.ReduceWorkload("p", T=T, C=C, W=W, seed=12)
+    partials, bias = wl.partials_and_bias(w, DEV)
+    out_full, out = rr.alloc_reduce_outputs(T, C, W, DEV)
+    call = rr.prepare_ragged_reduce_scatter(list(partials.unbind(0)), bias, out)
+    for round_ in range(2):
+        partials.copy_(wl.normal_bf16((W, T, C), 40 + round_, 0.5, DEV))
+        call()
+        want = oracle_lib.ragged_reduce_scatter([gu.bits(p) for p in partials.unbind(0)],
+                                                gu.bits(bias), W)
+        for r in range(W):
+            assert np.array_equal(gu.bits(out[r]), want[r])

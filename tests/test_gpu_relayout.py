@@ -314,3 +314,27 @@ def test_full_qkvg_250k_w4_chunked(oracle_lib):
     for i in (info, info_back):
         assert i["chunks"] == 4 and i["launches"] == 4 and i["planes_per_launch"] == 1
     torch.cuda.empty_cache()
+
+
+def test_prepared_calls_and_inverse(oracle_lib):
+    """Prepared calls equal the one-shot calls; the inverse of a prepared
+    seq->head is the matching head->seq (the backward reusing the forward's
+    plan); refilling the buffers in place between calls is picked up."""
+    T, P, H, D, W = 1000, 3, 56, 128, 6
+    full, send, part = _seq_inputs(T, P, H, D, W, seed=21)
+    heads = rr.alloc_head_side(T, P, H, D, W, DEV)
+    fwd = rr.prepare_seq_to_head(send, heads, layout=0)
+    back_full, back = rr.alloc_seq_side(T, P, H, D, W, DEV)
+    bwd = fwd.inverse(heads, back)
+    for round_ in range(3):
+        full.copy_(wl.random_bits((T, P, H, D), 30 + round_, DEV))
+        info = fwd()
+        assert info.launches == 1
+        bwd()
+        torch.cuda.synchronize()
+        want = oracle_lib.seq_to_head([gu.bits(s) for s in send], T, P, H, D, W)
+        for j in range(W):
+            assert np.array_equal(gu.bits(heads[j]), want[j])
+        assert gu.same_bits(back_full, full)
+    with pytest.raises(ValueError):
+        rr.prepare_seq_to_head(send, heads[:-1])
