@@ -282,13 +282,15 @@ cudaError_t launch_all_gather(const GatherArgs& a, int variant, int ctas_per_sm,
             gc.threads = kGenericThreads;
         }
     }
-    // The vector kernel launches 16 CTAs per SM by default, more than fit at
-    // once: on B200 that measured fastest for the 32k x 7168 (W=6) and
-    // 64k x 7168 (W=8) gathers (5.9 TB/s against 5.6 TB/s at 2 to 10 CTAs per
-    // SM).  The bulk kernel runs one CTA per SM (its ring fills the SM).
-    const int fit = resident_ctas(gc.fn, gc.threads, gc.smem, device);
-    const int per_sm = ctas_per_sm > 0 ? ctas_per_sm : (gc.variant == H3_VARIANT_BULK ? fit : 16);
-    int64_t grid = int64_t(sms) * per_sm;
+    // The vector kernel launches one CTA per token row by default, scheduled
+    // by the hardware: on B200 that measured 6.6-6.8 TB/s against 5.6-6.0 TB/s
+    // for persistent grid-stride launches.  The bulk kernel runs one CTA per
+    // SM (its ring fills the SM).  ctas_per_sm > 0 caps the grid.
+    int64_t grid = int64_t(a.T);
+    if (ctas_per_sm > 0)
+        grid = int64_t(sms) * ctas_per_sm;
+    else if (gc.variant == H3_VARIANT_BULK)
+        grid = int64_t(sms) * resident_ctas(gc.fn, gc.threads, gc.smem, device);
     if (grid > a.T)
         grid = a.T;
     if (grid < 1)

@@ -270,10 +270,7 @@ cudaError_t launch_reduce_scatter_gated(const GatedArgs& a, cudaStream_t stream,
     const int sms = current_sm_count(&device);
     if (sms <= 0)
         return cudaErrorNoDevice;
-    const int per_sm = resident_ctas(kernel, kThreads, 0, device);
-    int64_t grid = int64_t(sms) * per_sm;
-    if (grid > a.r.T)
-        grid = a.r.T;
+    int64_t grid = a.r.T;  // one CTA per token row (see launch_reduce_scatter)
     if (grid < 1)
         grid = 1;
     if (shape) {
@@ -293,8 +290,11 @@ cudaError_t launch_reduce_scatter(const ReduceArgs& a, int ctas_per_sm, cudaStre
     const int sms = current_sm_count(&device);
     if (sms <= 0)
         return cudaErrorNoDevice;
-    const int per_sm = ctas_per_sm > 0 ? ctas_per_sm : resident_ctas(kernel, kThreads, 0, device);
-    int64_t grid = int64_t(sms) * per_sm;
+    // One CTA per token row by default, scheduled by the hardware: on B200
+    // that measured 1-11 % faster than persistent grid-stride launches, whose
+    // lockstep sweep over the rows resonated with the DRAM mapping at some
+    // grid sizes.  ctas_per_sm > 0 caps the grid (grid-stride).
+    int64_t grid = ctas_per_sm > 0 ? int64_t(sms) * ctas_per_sm : int64_t(a.T);
     if (grid > a.T)
         grid = a.T;
     if (grid < 1)

@@ -379,13 +379,7 @@ struct KernelChoice {
     int rows_per_cta_iter = 1;
     size_t smem = 0;
     int variant = H3_VARIANT_NONE;
-    int per_sm = 0;  // default resident CTAs per SM (0: as many as fit)
 };
-
-// The 32-byte vector kernels keep 4 CTAs per SM by default: on B200 that
-// measured faster than full occupancy in both directions on the 32k-, 128k-
-// and 250k-token H3 workloads (more CTAs in flight lowered DRAM efficiency).
-constexpr int kWideCtasPerSm = 4;
 
 // Smallest instantiated vectors-per-thread count (at most MAXV) covering `need`.
 template <bool S2H, int VW, int NT, int ROWS, int MAXV, bool LAYOUT = false>
@@ -423,10 +417,8 @@ void choose_vec(const RelayoutArgs& a, bool wide_ok, KernelChoice* kc)
         const int row32 = a.row_vecs / 2;
         const bool ok = S2H ? pick_vec<true, 32, 64, 2, 8, LAYOUT>((row32 + 63) / 64, kc)
                             : pick_vec<false, 32, 32, 1, 16, LAYOUT>((row32 + 31) / 32, kc);
-        if (ok) {
-            kc->per_sm = kWideCtasPerSm;
+        if (ok)
             return;
-        }
     }
     if (pick_vec<S2H, 16, 128, 1, 16, LAYOUT>((a.row_vecs + 127) / 128, kc))
         return;
@@ -505,10 +497,19 @@ cudaError_t launch_relayout(bool seq_to_head, const RelayoutArgs& a, int variant
         if (err != cudaSuccess)
             return err;
     }
-    const int fit = resident_ctas(kc.fn, kc.threads, kc.smem, device);
-    int per_sm = ctas_per_sm > 0 ? ctas_per_sm : (kc.per_sm > 0 && kc.per_sm < fit ? kc.per_sm : fit);
+    // Grid: the vector kernels launch one CTA per row (or row pair) by
+    // default and let the hardware schedule them.  On B200 that measured
+    // 2-8 % faster than any persistent grid-stride launch (a multiple of the
+    // SM count): CTAs marching through the rows in lockstep resonated with the
+    // DRAM mapping at some grid sizes.  The bulk kernel keeps one CTA per SM
+    // (its shared-memory ring).  ctas_per_sm > 0 caps the grid at that many
+    // CTAs per SM (grid-stride).
     const int64_t needed = (int64_t(a.rows) + kc.rows_per_cta_iter - 1) / kc.rows_per_cta_iter;
-    int64_t grid = int64_t(sms) * per_sm;
+    int64_t grid = needed;
+    if (ctas_per_sm > 0)
+        grid = int64_t(sms) * ctas_per_sm;
+    else if (kc.variant == H3_VARIANT_BULK)
+        grid = int64_t(sms) * resident_ctas(kc.fn, kc.threads, kc.smem, device);
     if (grid > needed)
         grid = needed;
     if (grid < 1)

@@ -27,6 +27,7 @@ namespace h3rr {
 namespace {
 
 constexpr int kThreads = 128;
+constexpr int64_t kMaxGrid = (int64_t(1) << 31) - 1;
 
 __device__ __forceinline__ uint4 ld_stream(const char* p)
 {
@@ -123,10 +124,9 @@ cudaError_t launch_one(const void* fn, int64_t work, const StagedArgs& a, cudaSt
     const int sms = current_sm_count(&device);
     if (sms <= 0)
         return cudaErrorNoDevice;
-    const int per_sm = resident_ctas(fn, kThreads, 0, device);
-    int64_t grid = int64_t(sms) * per_sm;
-    if (grid > work)
-        grid = work;
+    // One CTA per row / run, scheduled by the hardware (the kernels stride over
+    // the rest if the work exceeds the grid limit).
+    int64_t grid = work < kMaxGrid ? work : kMaxGrid;
     if (grid < 1)
         grid = 1;
     *grid_out = int(grid);

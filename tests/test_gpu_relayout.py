@@ -131,19 +131,22 @@ def test_bulk_ring_sizes_alternate(oracle_lib):
 
 
 def test_default_variants():
-    """Defaults: the vector kernels in both directions, 4 CTAs per SM for the
-    32-byte H3 shapes; the bulk ring only when asked for."""
+    """Defaults: the vector kernels in both directions, one CTA per row pair
+    (seq->head) or row (head->seq); the bulk ring only when asked for."""
     for W, want_back in [(2, rr.H3_VARIANT_VECTOR), (4, rr.H3_VARIANT_VECTOR), (6, rr.H3_VARIANT_VECTOR)]:
         T, P, H, D = 300, 3, 56, 128
         full, send, part = _seq_inputs(T, P, H, D, W, seed=W)
         recv = rr.alloc_head_side(T, P, H, D, W, DEV)
         info = rr.seq_to_head(send, recv)
         assert info["variant"] == rr.H3_VARIANT_VECTOR
-        sms = torch.cuda.get_device_properties(0).multi_processor_count
-        assert info["grid"] == min(4 * sms, (T * P + 1) // 2)
+        assert info["grid"] == (T * P + 1) // 2
         back_full, back = rr.alloc_seq_side(T, P, H, D, W, DEV)
         info = rr.head_to_seq(recv, back)
-        assert info["variant"] == want_back and info["grid"] == min(4 * sms, T * P)
+        assert info["variant"] == want_back and info["grid"] == T * P
+        sms = torch.cuda.get_device_properties(0).multi_processor_count
+        capped = rr.head_to_seq(recv, back, ctas_per_sm=2)
+        assert capped["grid"] == min(2 * sms, T * P)
+        assert gu.same_bits(back_full, full)
         assert gu.same_bits(back_full, full)
 
 
