@@ -65,7 +65,7 @@ extern "C" {
 #define H3RR_API
 #endif
 
-#define H3RR_ABI_VERSION 1
+#define H3RR_ABI_VERSION 2
 #define H3RR_MAX_WORLD 64
 
 typedef enum h3_status {
@@ -96,12 +96,28 @@ typedef struct h3_exec_info {
     int32_t planes_per_launch;   /* planes moved by one launch */
 } h3_exec_info;
 
+/*
+ * Launch order.  By default the register kernels (relayouts, reduce-scatter,
+ * gated reduce-scatter, all-gather) use programmatic dependent launch (sm_90
+ * and later): a kernel may be scheduled while the previous kernel in the
+ * stream is draining, and it waits for that kernel to complete
+ * (griddepcontrol.wait) before its first global-memory access, so results are
+ * those of plain stream order.  Within one chunked relayout call, the launch
+ * of plane p+1 touches memory disjoint from plane p's and runs alongside
+ * plane p's tail; it waits for plane p at its end instead, so that the call's
+ * completion still implies every plane's.  The bulk (TMA) and staged kernels
+ * launch in plain stream order.  A kernel that follows in the stream and was
+ * itself launched with programmatic serialization must wait
+ * (cudaGridDependencySynchronize) before reading these calls' outputs.
+ */
+#define H3_LAUNCH_SERIAL 1       /* launch every kernel in plain stream order */
+
 /* Optional launch overrides for h3_*_ex; zero fields mean "library default". */
 typedef struct h3_launch_config {
     int32_t variant;             /* 0 = default, H3_VARIANT_VECTOR or H3_VARIANT_BULK (relayouts) */
-    int32_t ctas_per_sm;         /* 0 = default (occupancy-derived) */
-    int32_t reserved0;
-    int32_t reserved1;
+    int32_t ctas_per_sm;         /* 0 = default: one CTA per row; n caps the grid at n per SM */
+    int32_t flags;               /* H3_LAUNCH_* bits; other bits: H3_ERR_INVALID_ARG */
+    int32_t reserved1;           /* must be 0 */
 } h3_launch_config;
 
 /* ABI version of the loaded library (H3RR_ABI_VERSION it was built with). */

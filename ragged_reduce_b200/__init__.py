@@ -27,7 +27,8 @@ import torch
 from . import _abi
 from ._abi import (ExecInfo, H3Error, LaunchConfig, H3_LAYOUT_HEAD_PLANE_MAJOR,
                    H3_LAYOUT_SEQ_PLANE_MAJOR, H3_VARIANT_BULK, H3_VARIANT_GATHER,
-                   H3_VARIANT_REDUCE, H3_VARIANT_STAGED, H3_VARIANT_VECTOR, MAX_WORLD)
+                   H3_VARIANT_REDUCE, H3_VARIANT_STAGED, H3_VARIANT_VECTOR, H3_LAUNCH_SERIAL,
+                   MAX_WORLD)
 
 __all__ = [
     "H3Error", "Partition", "partition", "seq_to_head", "head_to_seq",
@@ -36,7 +37,7 @@ __all__ = [
     "bulk_wait_timeouts", "alloc_reduce_outputs", "seq_to_head_staged", "head_to_seq_staged",
     "staged_plan", "H3_VARIANT_STAGED", "ragged_all_gather", "H3_VARIANT_GATHER",
     "seq_to_head_layout", "head_to_seq_layout", "H3_LAYOUT_SEQ_PLANE_MAJOR",
-    "H3_LAYOUT_HEAD_PLANE_MAJOR", "ragged_reduce_scatter_gated", "PreparedRelayout",
+    "H3_LAYOUT_HEAD_PLANE_MAJOR", "ragged_reduce_scatter_gated", "PreparedRelayout", "H3_LAUNCH_SERIAL",
     "PreparedReduceScatter", "prepare_seq_to_head", "prepare_head_to_seq",
     "prepare_ragged_reduce_scatter",
 ]
@@ -149,10 +150,10 @@ def _stream_handle(stream, device) -> int:
     return int(stream.cuda_stream) if hasattr(stream, "cuda_stream") else int(stream)
 
 
-def _config(variant: int, ctas_per_sm: int):
-    if not variant and not ctas_per_sm:
+def _config(variant: int, ctas_per_sm: int, serial: bool = False):
+    if not variant and not ctas_per_sm and not serial:
         return None
-    return C.byref(LaunchConfig(int(variant), int(ctas_per_sm), 0, 0))
+    return C.byref(LaunchConfig(int(variant), int(ctas_per_sm), H3_LAUNCH_SERIAL if serial else 0, 0))
 
 
 def _relayout_shapes(seq_to_head_dir: bool, send, recv, layout: int = 0):
@@ -186,13 +187,13 @@ def _relayout_shapes(seq_to_head_dir: bool, send, recv, layout: int = 0):
 
 
 def _relayout_layout(seq_to_head_dir: bool, send, recv, layout, window_bytes, stream, variant,
-                     ctas_per_sm):
+                     ctas_per_sm, serial=False):
     send = _as_list(send)
     recv = _as_list(recv)
     T, P, H, D, W, dev = _relayout_shapes(seq_to_head_dir, send, recv, layout)
     info = ExecInfo()
     name = "h3_seq_to_head_layout" if seq_to_head_dir else "h3_head_to_seq_layout"
-    cfg = _config(variant, ctas_per_sm)
+    cfg = _config(variant, ctas_per_sm, serial)
     with torch.cuda.device(dev):
         st = getattr(_abi.lib, name)(
             _abi.pointer_array([t.data_ptr() for t in send]),
@@ -204,18 +205,20 @@ def _relayout_layout(seq_to_head_dir: bool, send, recv, layout, window_bytes, st
 
 
 def seq_to_head_layout(send, recv, layout: int, *, window_bytes: int = 0, stream=None,
-                       variant: int = 0, ctas_per_sm: int = 0) -> dict:
+                       variant: int = 0, ctas_per_sm: int = 0, serial: bool = False) -> dict:
     """seq->head with plane-major buffers (``layout``: bit set of
     H3_LAYOUT_SEQ_PLANE_MAJOR / H3_LAYOUT_HEAD_PLANE_MAJOR).  Plane-major
     sequence side: W tensors [P, T_r, H, D]; plane-major head side: W tensors
     [P, T, H_j, D] (out[j][0], [1], [2] are that rank's Q, K, V)."""
-    return _relayout_layout(True, send, recv, layout, window_bytes, stream, variant, ctas_per_sm)
+    return _relayout_layout(True, send, recv, layout, window_bytes, stream, variant, ctas_per_sm,
+                            serial)
 
 
 def head_to_seq_layout(send, recv, layout: int, *, window_bytes: int = 0, stream=None,
-                       variant: int = 0, ctas_per_sm: int = 0) -> dict:
+                       variant: int = 0, ctas_per_sm: int = 0, serial: bool = False) -> dict:
     """head->seq with plane-major buffers (see ``seq_to_head_layout``)."""
-    return _relayout_layout(False, send, recv, layout, window_bytes, stream, variant, ctas_per_sm)
+    return _relayout_layout(False, send, recv, layout, window_bytes, stream, variant, ctas_per_sm,
+                            serial)
 
 
 def _relayout_staged(seq_to_head_dir: bool, send, recv, window, stream):
@@ -260,7 +263,8 @@ def staged_plan(n_tokens: int, planes: int, n_heads: int, head_dim: int, window_
     return int(n.value), int(k.value)
 
 
-def _relayout(seq_to_head_dir: bool, send, recv, window_bytes, stream, variant, ctas_per_sm):
+def _relayout(seq_to_head_dir: bool, send, recv, window_bytes, stream, variant, ctas_per_sm,
+              serial=False):
     send = _as_list(send)
     recv = _as_list(recv)
     W = len(send)
@@ -284,7 +288,7 @@ def _relayout(seq_to_head_dir: bool, send, recv, window_bytes, stream, variant, 
                              f"expected {(T, P, part.heads(j), D)}")
     info = ExecInfo()
     name = "h3_seq_to_head" if seq_to_head_dir else "h3_head_to_seq"
-    cfg = _config(variant, ctas_per_sm)
+    cfg = _config(variant, ctas_per_sm, serial)
     args = [_abi.pointer_array([t.data_ptr() for t in send]),
             _abi.pointer_array([t.data_ptr() for t in recv]),
             T, int(P), int(H), int(D), W, int(window_bytes),
@@ -299,24 +303,26 @@ def _relayout(seq_to_head_dir: bool, send, recv, window_bytes, stream, variant, 
 
 
 def seq_to_head(send, recv, *, window_bytes: int = 0, stream=None, variant: int = 0,
-                ctas_per_sm: int = 0) -> dict:
+                ctas_per_sm: int = 0, serial: bool = False) -> dict:
     """Ulysses sequence->head relayout.
 
     send: W tensors [T_r, P, H, D] (or views of one [T, P, H, D] tensor, see
     ``split_rows``); recv: W tensors [T, P, H_j, D], written.  window_bytes > 0
-    moves one plane per launch under that byte bound.  Returns what ran
-    (launches, chunks, grid, block, variant)."""
-    return _relayout(True, send, recv, window_bytes, stream, variant, ctas_per_sm)
+    moves one plane per launch under that byte bound.  serial=True launches
+    in plain stream order (H3_LAUNCH_SERIAL) instead of programmatic dependent
+    launch.  Returns what ran (launches, chunks, grid, block, variant)."""
+    return _relayout(True, send, recv, window_bytes, stream, variant, ctas_per_sm, serial)
 
 
 def head_to_seq(send, recv, *, window_bytes: int = 0, stream=None, variant: int = 0,
-                ctas_per_sm: int = 0) -> dict:
+                ctas_per_sm: int = 0, serial: bool = False) -> dict:
     """Inverse head->sequence relayout: send W tensors [T, P, H_j, D] -> recv W
     tensors [T_r, P, H, D]."""
-    return _relayout(False, send, recv, window_bytes, stream, variant, ctas_per_sm)
+    return _relayout(False, send, recv, window_bytes, stream, variant, ctas_per_sm, serial)
 
 
-def ragged_reduce_scatter(partials, bias, out, *, stream=None, ctas_per_sm: int = 0) -> dict:
+def ragged_reduce_scatter(partials, bias, out, *, stream=None, ctas_per_sm: int = 0,
+                          serial: bool = False) -> dict:
     """Tensor-mode ragged reduce-scatter.
 
     partials: W BF16 tensors [T, C] (or one [W, T, C] tensor); bias: BF16 [C]
@@ -345,7 +351,7 @@ def ragged_reduce_scatter(partials, bias, out, *, stream=None, ctas_per_sm: int 
                 raise ValueError(f"out rank {r}: shape {tuple(o.shape)}, expected "
                                  f"{(part.tokens(r), Cc)}")
     info = ExecInfo()
-    cfg = _config(0, ctas_per_sm)
+    cfg = _config(0, ctas_per_sm, serial)
     args = [_abi.pointer_array([p.data_ptr() for p in partials]),
             C.c_void_p(bias.data_ptr() if bias is not None else 0),
             _abi.pointer_array([o.data_ptr() for o in out]),
@@ -372,7 +378,8 @@ def bulk_wait_timeouts(stream=None, reset: bool = False, device=None) -> int:
     return int(count.value)
 
 
-def ragged_all_gather(blocks, out, *, stream=None, variant: int = 0, ctas_per_sm: int = 0) -> dict:
+def ragged_all_gather(blocks, out, *, stream=None, variant: int = 0, ctas_per_sm: int = 0,
+                      serial: bool = False) -> dict:
     """Ragged all-gather of token rows: blocks are W tensors [T_r, C] (rank
     r's rows; 2-byte elements), out W tensors [T, C], each written with all T
     rows in token order (``h3_ragged_all_gather``)."""
@@ -398,7 +405,7 @@ def ragged_all_gather(blocks, out, *, stream=None, variant: int = 0, ctas_per_sm
     args = [_abi.pointer_array([b.data_ptr() for b in blocks]),
             _abi.pointer_array([o.data_ptr() for o in out]),
             T, Cc, W, C.c_void_p(_stream_handle(stream, dev))]
-    cfg = _config(variant, ctas_per_sm)
+    cfg = _config(variant, ctas_per_sm, serial)
     with torch.cuda.device(dev):
         if cfg is None:
             st = _abi.lib.h3_ragged_all_gather(*args, C.byref(info))
@@ -465,7 +472,8 @@ class PreparedRelayout:
     reuses the plan saved by its forward)."""
 
     def __init__(self, seq_to_head_dir: bool, send, recv, *, layout: int = 0,
-                 window_bytes: int = 0, variant: int = 0, ctas_per_sm: int = 0):
+                 window_bytes: int = 0, variant: int = 0, ctas_per_sm: int = 0,
+                 serial: bool = False):
         send = _as_list(send)
         recv = _as_list(recv)
         T, P, H, D, W, dev = _relayout_shapes(seq_to_head_dir, send, recv, layout)
@@ -476,11 +484,13 @@ class PreparedRelayout:
         self.window_bytes = int(window_bytes)
         self.variant = int(variant)
         self.ctas_per_sm = int(ctas_per_sm)
+        self.serial = bool(serial)
         self._keep = (send, recv)  # keep the tensors alive while the call holds their addresses
         name = "h3_seq_to_head_layout" if seq_to_head_dir else "h3_head_to_seq_layout"
         self._fn = getattr(_abi.lib, name)
         self._name = name
-        self._cfg = LaunchConfig(self.variant, self.ctas_per_sm, 0, 0)
+        self._cfg = LaunchConfig(self.variant, self.ctas_per_sm,
+                                 H3_LAUNCH_SERIAL if self.serial else 0, 0)
         self._info = ExecInfo()
         self._head = (_abi.pointer_array([t.data_ptr() for t in send]),
                       _abi.pointer_array([t.data_ptr() for t in recv]),
@@ -503,7 +513,7 @@ class PreparedRelayout:
         options; send/recv are that direction's buffers."""
         return PreparedRelayout(not self.seq_to_head_dir, send, recv, layout=self.layout,
                                 window_bytes=self.window_bytes, variant=self.variant,
-                                ctas_per_sm=self.ctas_per_sm)
+                                ctas_per_sm=self.ctas_per_sm, serial=self.serial)
 
 
 def prepare_seq_to_head(send, recv, **kw) -> PreparedRelayout:
@@ -520,7 +530,7 @@ class PreparedReduceScatter:
     """A ragged reduce-scatter checked and marshalled once; each call is one
     ``h3_ragged_reduce_scatter_ex`` call.  Buffers are captured by address."""
 
-    def __init__(self, partials, bias, out, *, ctas_per_sm: int = 0):
+    def __init__(self, partials, bias, out, *, ctas_per_sm: int = 0, serial: bool = False):
         partials = _as_list(partials)
         out = _as_list(out)
         W = len(partials)
@@ -536,7 +546,7 @@ class PreparedReduceScatter:
             if tuple(o.shape) != (part.tokens(r), Cc):
                 raise ValueError(f"out rank {r}: shape {tuple(o.shape)}, expected {(part.tokens(r), Cc)}")
         self._keep = (partials, bias, out)
-        self._cfg = LaunchConfig(0, int(ctas_per_sm), 0, 0)
+        self._cfg = LaunchConfig(0, int(ctas_per_sm), H3_LAUNCH_SERIAL if serial else 0, 0)
         self._info = ExecInfo()
         self._head = (_abi.pointer_array([p.data_ptr() for p in partials]),
                       C.c_void_p(bias.data_ptr() if bias is not None else 0),

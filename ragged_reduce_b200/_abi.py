@@ -43,7 +43,8 @@ MAX_GATE_SEGMENTS = 256
 MAX_WORLD = 64
 H3_LAYOUT_SEQ_PLANE_MAJOR = 1
 H3_LAYOUT_HEAD_PLANE_MAJOR = 2
-ABI_VERSION = 1
+H3_LAUNCH_SERIAL = 1
+ABI_VERSION = 2
 
 
 class ExecInfo(C.Structure):
@@ -64,7 +65,7 @@ class LaunchConfig(C.Structure):
     _fields_ = [
         ("variant", C.c_int32),
         ("ctas_per_sm", C.c_int32),
-        ("reserved0", C.c_int32),
+        ("flags", C.c_int32),
         ("reserved1", C.c_int32),
     ]
 

@@ -74,6 +74,10 @@ __global__ void __launch_bounds__(NT) all_gather_vec_kernel(const __grid_constan
 {
     constexpr int kUnits = VW / kVecBytes;
     const int32_t row_v = a.row_vecs / kUnits;
+    // Programmatic launch: the previous kernel in the stream completes before
+    // the first memory access.
+    pdl_wait_prerequisites();
+    pdl_allow_dependents();
     for (int64_t t64 = blockIdx.x; t64 < a.T; t64 += gridDim.x) {
         const int32_t t = int32_t(t64);
         const int32_t s = split_owner(t, a.tq, a.tm);
@@ -104,6 +108,10 @@ constexpr int kGenericThreads = 128;
 
 __global__ void __launch_bounds__(kGenericThreads) all_gather_generic_kernel(const __grid_constant__ GatherArgs a)
 {
+    // Programmatic launch: the previous kernel in the stream completes before
+    // the first memory access.
+    pdl_wait_prerequisites();
+    pdl_allow_dependents();
     for (int64_t t64 = blockIdx.x; t64 < a.T; t64 += gridDim.x) {
         const int32_t t = int32_t(t64);
         const int32_t s = split_owner(t, a.tq, a.tm);
@@ -254,7 +262,7 @@ bool all_gather_bulk_fits(const GatherArgs& a, int device)
 }
 
 cudaError_t launch_all_gather(const GatherArgs& a, int variant, int ctas_per_sm, cudaStream_t stream,
-                              LaunchShape* shape)
+                              LaunchShape* shape, bool programmatic)
 {
     int device = 0;
     const int sms = current_sm_count(&device);
@@ -300,8 +308,11 @@ cudaError_t launch_all_gather(const GatherArgs& a, int variant, int ctas_per_sm,
         shape->block = gc.threads;
         shape->variant = gc.variant;
     }
+    // The register kernels follow the griddepcontrol protocol; the bulk
+    // kernel launches in plain stream order.
     void* params[] = {const_cast<GatherArgs*>(&a)};
-    return cudaLaunchKernel(gc.fn, dim3(unsigned(grid)), dim3(gc.threads), params, gc.smem, stream);
+    return launch_kernel(gc.fn, grid, gc.threads, gc.smem, stream, params,
+                         programmatic && gc.variant != H3_VARIANT_BULK);
 }
 
 cudaError_t read_gather_wait_timeouts(unsigned int* count, bool reset, cudaStream_t stream)

@@ -32,6 +32,14 @@ void clear_info(h3_exec_info* info)
         std::memset(info, 0, sizeof(*info));
 }
 
+// Launch-config fields every entry point checks the same way.
+bool config_ok(const h3_launch_config* cfg)
+{
+    return !cfg || (cfg->ctas_per_sm >= 0 && (cfg->flags & ~H3_LAUNCH_SERIAL) == 0 && cfg->reserved1 == 0);
+}
+
+bool programmatic_launch(const h3_launch_config* cfg) { return !(cfg && (cfg->flags & H3_LAUNCH_SERIAL)); }
+
 // Partition checks shared by the relayouts and the reduce-scatter
 // ("Distributed H3 Execution", intro: empty token or head partitions are
 // rejected).
@@ -121,7 +129,7 @@ h3_status relayout(bool seq_to_head, const void* const* send, void* const* recv,
         return H3_ERR_INVALID_ARG;
     if (cfg && cfg->variant != 0 && cfg->variant != H3_VARIANT_VECTOR && cfg->variant != H3_VARIANT_BULK)
         return H3_ERR_INVALID_ARG;
-    if (cfg && cfg->ctas_per_sm < 0)
+    if (!config_ok(cfg))
         return H3_ERR_INVALID_ARG;
     h3_status st = check_relayout_args(seq_to_head, send, recv, n_tokens, planes, n_heads, head_dim,
                                        world, nullptr, 0);
@@ -179,12 +187,16 @@ h3_status relayout(bool seq_to_head, const void* const* send, void* const* recv,
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     LaunchShape shape;
     int launched = 0;
+    const bool programmatic = programmatic_launch(cfg);
     for (int c = 0; c < chunks; ++c) {
         a.plane0 = c * per_launch;
         a.nplanes = per_launch;
         a.rows = int32_t(n_tokens * per_launch);
-        const cudaError_t err =
-            launch_relayout(seq_to_head, a, variant, ctas_per_sm, s, &shape, layout != 0);
+        // Planes are disjoint: a later plane's launch depends on nothing the
+        // previous one does and only has to finish after it.
+        a.wait_late = c > 0 ? 1 : 0;
+        const cudaError_t err = launch_relayout(seq_to_head, a, variant, ctas_per_sm, s, &shape,
+                                                layout != 0, programmatic);
         if (err != cudaSuccess) {
             if (info) {
                 info->launches = launched;
@@ -466,7 +478,7 @@ h3_status h3_ragged_reduce_scatter_ex(const void* const* partials, const void* b
         return H3_ERR_INVALID_ARG;
     if (cfg && (cfg->variant != 0 && cfg->variant != H3_VARIANT_REDUCE))
         return H3_ERR_INVALID_ARG;
-    if (cfg && cfg->ctas_per_sm < 0)
+    if (!config_ok(cfg))
         return H3_ERR_INVALID_ARG;
     if (cols % 8 != 0)
         return H3_ERR_MISALIGNED;
@@ -513,7 +525,8 @@ h3_status h3_ragged_reduce_scatter_ex(const void* const* partials, const void* b
     a.row_bytes = int64_t(row_bytes);
     LaunchShape shape;
     const cudaError_t err = launch_reduce_scatter(a, cfg ? cfg->ctas_per_sm : 0,
-                                                  static_cast<cudaStream_t>(stream), &shape);
+                                                  static_cast<cudaStream_t>(stream), &shape,
+                                                  programmatic_launch(cfg));
     if (err != cudaSuccess)
         return cuda_failure(err);
     if (info) {
@@ -559,7 +572,7 @@ h3_status h3_ragged_all_gather_ex(const void* const* in, void* const* out, int64
         return H3_ERR_INVALID_ARG;
     if (cfg && cfg->variant != 0 && cfg->variant != H3_VARIANT_VECTOR && cfg->variant != H3_VARIANT_BULK)
         return H3_ERR_INVALID_ARG;
-    if (cfg && cfg->ctas_per_sm < 0)
+    if (!config_ok(cfg))
         return H3_ERR_INVALID_ARG;
     if (cols % 8 != 0)
         return H3_ERR_MISALIGNED;
@@ -603,7 +616,8 @@ h3_status h3_ragged_all_gather_ex(const void* const* in, void* const* out, int64
     }
     LaunchShape shape;
     const cudaError_t err = launch_all_gather(a, variant, cfg ? cfg->ctas_per_sm : 0,
-                                              static_cast<cudaStream_t>(stream), &shape);
+                                              static_cast<cudaStream_t>(stream), &shape,
+                                              programmatic_launch(cfg));
     if (err != cudaSuccess)
         return cuda_failure(err);
     if (info) {
@@ -688,7 +702,8 @@ h3_status h3_ragged_reduce_scatter_gated(const void* const* partials, const void
     for (int32_t k = 0; k <= n_segs; ++k)
         g.seg_bounds[k] = int32_t(seg_bounds[k]);
     LaunchShape shape;
-    const cudaError_t err = launch_reduce_scatter_gated(g, static_cast<cudaStream_t>(stream), &shape);
+    const cudaError_t err =
+        launch_reduce_scatter_gated(g, static_cast<cudaStream_t>(stream), &shape, true);
     if (err != cudaSuccess)
         return cuda_failure(err);
     if (info) {

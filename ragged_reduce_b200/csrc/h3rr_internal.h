@@ -57,6 +57,7 @@ struct RelayoutArgs {
     int32_t head_vecs;       // D * 2 / 16
     int32_t seq_pm;          // sequence side plane-major [P, T_r, H, D] (layout kernels only)
     int32_t head_pm;         // head side plane-major [P, T, H_j, D] (layout kernels only)
+    int32_t wait_late;       // 1: independent of the previous launch; wait for it at the end
 };
 
 struct ReduceArgs {
@@ -119,7 +120,7 @@ struct LaunchShape {
 // selects the kernels that read a.seq_pm / a.head_pm (plane-major buffers).
 cudaError_t launch_relayout(bool seq_to_head, const RelayoutArgs& a, int variant,
                             int ctas_per_sm, cudaStream_t stream, LaunchShape* shape,
-                            bool layout = false);
+                            bool layout = false, bool programmatic = false);
 
 // Whether the bulk kernel's shared-memory ring fits one row of these args.
 bool relayout_bulk_fits(const RelayoutArgs& a, int device);
@@ -142,16 +143,17 @@ h3_status record_cuda_failure(cudaError_t err);
 
 // Enqueue the all-gather launch (variant 0 / H3_VARIANT_VECTOR or H3_VARIANT_BULK).
 cudaError_t launch_all_gather(const GatherArgs& a, int variant, int ctas_per_sm, cudaStream_t stream,
-                              LaunchShape* shape);
+                              LaunchShape* shape, bool programmatic);
 bool all_gather_bulk_fits(const GatherArgs& a, int device);
 cudaError_t read_gather_wait_timeouts(unsigned int* count, bool reset, cudaStream_t stream);
 
 // Enqueue the gated reduce-scatter launch.
-cudaError_t launch_reduce_scatter_gated(const GatedArgs& a, cudaStream_t stream, LaunchShape* shape);
+cudaError_t launch_reduce_scatter_gated(const GatedArgs& a, cudaStream_t stream, LaunchShape* shape,
+                                        bool programmatic);
 
 // Enqueue the reduce-scatter launch.
 cudaError_t launch_reduce_scatter(const ReduceArgs& a, int ctas_per_sm, cudaStream_t stream,
-                                  LaunchShape* shape);
+                                  LaunchShape* shape, bool programmatic);
 
 // SM count of the current device (cached per device).
 int current_sm_count(int* device);
@@ -163,5 +165,28 @@ int resident_ctas(const void* kernel, int block, size_t smem, int device);
 // Opt a kernel in to `smem` bytes of dynamic shared memory on the current
 // device (once per kernel, device and size).
 cudaError_t allow_dynamic_smem(const void* kernel, size_t smem, int device);
+
+// Launch `kernel` on a 1-D grid; `programmatic` sets programmatic stream
+// serialization (the kernel must follow the griddepcontrol protocol below).
+cudaError_t launch_kernel(const void* kernel, int64_t grid, int block, size_t smem,
+                          cudaStream_t stream, void** params, bool programmatic);
+
+#ifdef __CUDACC__
+// Programmatic dependent launch, device side.  A kernel launched with
+// programmatic stream serialization may start before the previous kernel in
+// the stream has completed; griddepcontrol.wait blocks the calling thread
+// until every prerequisite grid has completed and its writes are visible (a
+// no-op for a plain launch).  launch_dependents lets the next such kernel be
+// scheduled once every CTA of this grid has issued it (or exited).
+__device__ __forceinline__ void pdl_wait_prerequisites()
+{
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+}
+
+__device__ __forceinline__ void pdl_allow_dependents()
+{
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+#endif
 
 }  // namespace h3rr

@@ -141,4 +141,22 @@ cudaError_t allow_dynamic_smem(const void* kernel, size_t smem, int device)
     return err;
 }
 
+cudaError_t launch_kernel(const void* kernel, int64_t grid, int block, size_t smem,
+                          cudaStream_t stream, void** params, bool programmatic)
+{
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(unsigned(grid));
+    cfg.blockDim = dim3(unsigned(block));
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    if (programmatic) {
+        attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+        attr[0].val.programmaticStreamSerializationAllowed = 1;
+        cfg.attrs = attr;
+        cfg.numAttrs = 1;
+    }
+    return cudaLaunchKernelExC(&cfg, kernel, params);
+}
+
 }  // namespace h3rr

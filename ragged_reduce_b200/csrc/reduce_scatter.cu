@@ -101,6 +101,10 @@ template <int kW, int U>
 __global__ void __launch_bounds__(kThreads) reduce_scatter_kernel(const __grid_constant__ ReduceArgs a)
 {
     constexpr int kBatch = kW > 0 ? kW : 8;
+    // Programmatic launch: the previous kernel in the stream completes before
+    // the first memory access.
+    pdl_wait_prerequisites();
+    pdl_allow_dependents();
     for (int64_t t64 = blockIdx.x; t64 < a.T; t64 += gridDim.x) {
         const int32_t t = int32_t(t64);
         const int32_t s = split_owner(t, a.tq, a.tm);
@@ -196,6 +200,10 @@ __global__ void __launch_bounds__(kThreads) reduce_scatter_gated_kernel(const __
 {
     const ReduceArgs& a = g.r;
     constexpr int kBatch = kW > 0 ? kW : 8;
+    // Programmatic launch: the previous kernel in the stream completes before
+    // the first memory access.
+    pdl_wait_prerequisites();
+    pdl_allow_dependents();
     for (int64_t t64 = blockIdx.x; t64 < a.T; t64 += gridDim.x) {
         const int32_t t = int32_t(t64);
         const int32_t s = split_owner(t, a.tq, a.tm);
@@ -263,7 +271,8 @@ const void* pick_gated_kernel(int W)
 
 }  // namespace
 
-cudaError_t launch_reduce_scatter_gated(const GatedArgs& a, cudaStream_t stream, LaunchShape* shape)
+cudaError_t launch_reduce_scatter_gated(const GatedArgs& a, cudaStream_t stream, LaunchShape* shape,
+                                        bool programmatic)
 {
     const void* kernel = pick_gated_kernel(a.r.W);
     int device = 0;
@@ -279,11 +288,11 @@ cudaError_t launch_reduce_scatter_gated(const GatedArgs& a, cudaStream_t stream,
         shape->variant = H3_VARIANT_REDUCE_GATED;
     }
     void* params[] = {const_cast<GatedArgs*>(&a)};
-    return cudaLaunchKernel(kernel, dim3(unsigned(grid)), dim3(kThreads), params, 0, stream);
+    return launch_kernel(kernel, grid, kThreads, 0, stream, params, programmatic);
 }
 
 cudaError_t launch_reduce_scatter(const ReduceArgs& a, int ctas_per_sm, cudaStream_t stream,
-                                  LaunchShape* shape)
+                                  LaunchShape* shape, bool programmatic)
 {
     const void* kernel = pick_reduce_kernel(a.W);
     int device = 0;
@@ -305,7 +314,7 @@ cudaError_t launch_reduce_scatter(const ReduceArgs& a, int ctas_per_sm, cudaStre
         shape->variant = H3_VARIANT_REDUCE;
     }
     void* params[] = {const_cast<ReduceArgs*>(&a)};
-    return cudaLaunchKernel(kernel, dim3(unsigned(grid)), dim3(kThreads), params, 0, stream);
+    return launch_kernel(kernel, grid, kThreads, 0, stream, params, programmatic);
 }
 
 }  // namespace h3rr

@@ -115,6 +115,12 @@ __global__ void __launch_bounds__(NT) relayout_vec_kernel(const __grid_constant_
         hstride[k] = hj * head_v * VW;
     }
     const int64_t seq_row_bytes = int64_t(row_v) * VW;
+    // Programmatic launch: the previous kernel in the stream must be complete
+    // before the first memory access, unless this launch is independent of
+    // it (a later plane of a chunked call), which waits at its end instead.
+    if (!a.wait_late)
+        pdl_wait_prerequisites();
+    pdl_allow_dependents();
 
     for (int64_t i0 = int64_t(blockIdx.x) * ROWS; i0 < a.rows; i0 += int64_t(gridDim.x) * ROWS) {
         char* sptr[ROWS];
@@ -161,6 +167,8 @@ __global__ void __launch_bounds__(NT) relayout_vec_kernel(const __grid_constant_
             }
         }
     }
+    if (a.wait_late)
+        pdl_wait_prerequisites();
 }
 
 // Any row width: one row per CTA iteration, head-side placement per vector.
@@ -170,6 +178,9 @@ template <bool kSeqToHead, bool kLayout = false>
 __global__ void __launch_bounds__(kGenericThreads) relayout_generic_kernel(const __grid_constant__ RelayoutArgs a)
 {
     const int64_t seq_row_bytes = int64_t(a.row_vecs) * kVecBytes;
+    if (!a.wait_late)
+        pdl_wait_prerequisites();
+    pdl_allow_dependents();
     for (int64_t i64 = blockIdx.x; i64 < a.rows; i64 += gridDim.x) {
         const int32_t i = int32_t(i64);
         const int32_t t = i / a.nplanes;
@@ -204,6 +215,8 @@ __global__ void __launch_bounds__(kGenericThreads) relayout_generic_kernel(const
             }
         }
     }
+    if (a.wait_late)
+        pdl_wait_prerequisites();
 }
 
 // ---------------------------------------------------------------------------
@@ -465,7 +478,7 @@ bool relayout_bulk_fits(const RelayoutArgs& a, int device)
 }
 
 cudaError_t launch_relayout(bool seq_to_head, const RelayoutArgs& a, int variant, int ctas_per_sm,
-                            cudaStream_t stream, LaunchShape* shape, bool layout)
+                            cudaStream_t stream, LaunchShape* shape, bool layout, bool programmatic)
 {
     int device = 0;
     const int sms = current_sm_count(&device);
@@ -519,8 +532,11 @@ cudaError_t launch_relayout(bool seq_to_head, const RelayoutArgs& a, int variant
         shape->block = kc.threads;
         shape->variant = kc.variant;
     }
+    // The vector and generic kernels follow the griddepcontrol protocol; the
+    // bulk kernel launches in plain stream order.
     void* params[] = {const_cast<RelayoutArgs*>(&a)};
-    return cudaLaunchKernel(kc.fn, dim3(unsigned(grid)), dim3(kc.threads), params, kc.smem, stream);
+    return launch_kernel(kc.fn, grid, kc.threads, kc.smem, stream, params,
+                         programmatic && kc.variant != H3_VARIANT_BULK);
 }
 
 cudaError_t read_bulk_wait_timeouts(unsigned int* count, bool reset, cudaStream_t stream)

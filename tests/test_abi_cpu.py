@@ -205,6 +205,34 @@ def test_relayout_rejects_unknown_variant():
     assert st == _abi.H3_ERR_INVALID_ARG
 
 
+@needs_no_gpu
+def test_launch_config_rejects_unknown_flags_and_reserved():
+    """Only H3_LAUNCH_SERIAL is a flag; reserved1 must be 0 (every _ex call)."""
+    T, P, H, D, W = 100, 3, 56, 128, 2
+    send, recv = _layout(T, P, H, D, W)
+    Cc = 64
+    blocks = [BASE + r * (1 << 20) for r in range(W)]
+    full = [BASE + (8 << 20) + r * (1 << 20) for r in range(W)]
+    for flags, reserved in ((2, 0), (4, 0), (-1, 0), (_abi.H3_LAUNCH_SERIAL | 8, 0), (0, 1),
+                            (_abi.H3_LAUNCH_SERIAL, -1)):
+        cfg = C.byref(_abi.LaunchConfig(0, 0, flags, reserved))
+        for fn in ("h3_seq_to_head_ex", "h3_head_to_seq_ex"):
+            info = _abi.ExecInfo()
+            st = getattr(_abi.lib, fn)(_ptrs(send), _ptrs(recv), T, P, H, D, W, 0, None, cfg,
+                                       C.byref(info))
+            assert st == _abi.H3_ERR_INVALID_ARG and info.launches == 0, (fn, flags, reserved)
+        for fn in ("h3_seq_to_head_layout", "h3_head_to_seq_layout"):
+            st = getattr(_abi.lib, fn)(_ptrs(send), _ptrs(recv), T, P, H, D, W, 0, 0, None, cfg,
+                                       C.byref(_abi.ExecInfo()))
+            assert st == _abi.H3_ERR_INVALID_ARG, (fn, flags, reserved)
+        st = _abi.lib.h3_ragged_reduce_scatter_ex(_ptrs(full), None, _ptrs(blocks), T, Cc, W, None,
+                                                  cfg, C.byref(_abi.ExecInfo()))
+        assert st == _abi.H3_ERR_INVALID_ARG, (flags, reserved)
+        st = _abi.lib.h3_ragged_all_gather_ex(_ptrs(blocks), _ptrs(full), T, Cc, W, None, cfg,
+                                              C.byref(_abi.ExecInfo()))
+        assert st == _abi.H3_ERR_INVALID_ARG, (flags, reserved)
+
+
 def test_bulk_timeout_query_needs_count():
     assert _abi.lib.h3_bulk_wait_timeouts(None, None, 0) == _abi.H3_ERR_INVALID_ARG
 
