@@ -408,6 +408,90 @@ H3RR_API h3_status h3_staged_plan(int64_t n_tokens, int32_t planes, int32_t n_he
  */
 H3RR_API h3_status h3_bulk_wait_timeouts(void* stream, uint32_t* count, int32_t reset);
 
+/* ------------------------------------------------------------------------
+ * One rank per GPU.  The calls above keep all W virtual ranks in one GPU's
+ * memory.  With one rank per GPU (each process drives one GPU), rank k's share of
+ * each operation is computed by the calls below, which pull what rank k
+ * needs from every rank's buffer with plain 16- or 32-byte loads (no TMA,
+ * no multicast) and write only rank k's own output.  The W rank calls
+ * together write exactly what the one-GPU call writes, bit for bit
+ * ("Distributed H3 Execution", "Remaining GPU Gates": identity of the real
+ * collective at 2-8 GPUs and distributed-versus-single parity).
+ *
+ * Pointer arrays hold the W ranks' buffers as addresses the current device
+ * can load from: its own buffer and the peers' buffers mapped with
+ * h3_ipc_open (or any other peer mapping).  The peers' buffers must be
+ * complete before the call is enqueued and unchanged until it has finished;
+ * the caller orders this across processes (for example a stream
+ * synchronisation and a host barrier on each side).  Arguments are checked
+ * as in the one-GPU calls, plus 0 <= rank < world (else H3_ERR_INVALID_ARG);
+ * overlap is checked between this rank's output and every input address
+ * range.  The bulk variant is not offered (H3_ERR_UNSUPPORTED); cfg as in
+ * the _ex calls otherwise.  Launch order as above.
+ * ------------------------------------------------------------------------ */
+
+/* Rank k's head-side buffer: recv [T, P, H_k, D] (this GPU) gets
+ * recv[t, p, h, d] = send[r(t)][t - ts_{r(t)}, p, hs_k + h, d]
+ * from send[world], the sequence-side buffers [T_r, P, H, D] of all ranks.
+ * window_bytes as h3_seq_to_head (same check over all ranks' slices). */
+H3RR_API h3_status h3_seq_to_head_rank(const void* const* send, void* recv, int64_t n_tokens,
+                                       int32_t planes, int32_t n_heads, int32_t head_dim,
+                                       int32_t world, int32_t rank, int64_t window_bytes,
+                                       void* stream, const h3_launch_config* cfg,
+                                       h3_exec_info* info);
+
+/* Rank k's sequence-side buffer: recv [T_k, P, H, D] (this GPU) gets
+ * recv[t', p, hs_j + h, d] = send[j][ts_k + t', p, h, d] from send[world],
+ * the head-side buffers [T, P, H_j, D] of all ranks. */
+H3RR_API h3_status h3_head_to_seq_rank(const void* const* send, void* recv, int64_t n_tokens,
+                                       int32_t planes, int32_t n_heads, int32_t head_dim,
+                                       int32_t world, int32_t rank, int64_t window_bytes,
+                                       void* stream, const h3_launch_config* cfg,
+                                       h3_exec_info* info);
+
+/* Rank k's rows of the ragged reduce-scatter: out [T_k, C] (this GPU) gets
+ * out[t', c] = bf16_rne(((p_0 + ... + p_{W-1}) + bias)[ts_k + t', c]) in
+ * binary32, rank order, from partials[world] ([T, C] each, any rank's GPU);
+ * bias [C] or NULL (read from wherever it is). */
+H3RR_API h3_status h3_ragged_reduce_scatter_rank(const void* const* partials, const void* bias,
+                                                 void* out, int64_t n_tokens, int64_t cols,
+                                                 int32_t world, int32_t rank, void* stream,
+                                                 const h3_launch_config* cfg,
+                                                 h3_exec_info* info);
+
+/* Rank k's copy of the ragged all-gather: out [T, C] (this GPU) gets every
+ * rank's rows, out[t, c] = in[r(t)][t - ts_{r(t)}, c], from in[world]
+ * ([T_r, C] each). */
+H3RR_API h3_status h3_ragged_all_gather_rank(const void* const* in, void* out, int64_t n_tokens,
+                                             int64_t cols, int32_t world, int32_t rank,
+                                             void* stream, const h3_launch_config* cfg,
+                                             h3_exec_info* info);
+
+/*
+ * CUDA IPC for the pointer arrays above.  h3_ipc_export describes the
+ * device buffer at `ptr` (any address inside a cudaMalloc allocation of the
+ * current device): the allocation's IPC handle and the buffer's offset in
+ * it.  Send the struct to the peers by any means (it is plain bytes).
+ * h3_ipc_open maps a peer's buffer into this process on the current device
+ * (peer access enabled lazily) and returns its address; h3_ipc_close unmaps
+ * it (same pointer and struct).  Mappings are counted per device and
+ * allocation: buffers that share an allocation share one mapping, which the
+ * last close releases (a close that matches no open: H3_ERR_INVALID_ARG).
+ * A process cannot open its own handles.  Close only after the last kernel
+ * reading the mapping has finished.  Memory from virtual-memory-management
+ * allocators (cuMemCreate, expandable segments) has no IPC handle: export
+ * returns H3_ERR_CUDA.  NULL arguments: H3_ERR_INVALID_ARG.
+ */
+#define H3_IPC_HANDLE_BYTES 64
+typedef struct h3_ipc_handle {
+    unsigned char handle[H3_IPC_HANDLE_BYTES]; /* cudaIpcMemHandle_t of the allocation */
+    int64_t offset;                            /* buffer address - allocation base */
+    int64_t alloc_bytes;                       /* size of the allocation */
+} h3_ipc_handle;
+H3RR_API h3_status h3_ipc_export(const void* ptr, h3_ipc_handle* out);
+H3RR_API h3_status h3_ipc_open(const h3_ipc_handle* handle, void** ptr);
+H3RR_API h3_status h3_ipc_close(void* ptr, const h3_ipc_handle* handle);
+
 #ifdef __cplusplus
 }
 #endif

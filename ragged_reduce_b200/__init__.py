@@ -39,6 +39,7 @@ __all__ = [
     "seq_to_head_layout", "head_to_seq_layout", "H3_LAYOUT_SEQ_PLANE_MAJOR",
     "H3_LAYOUT_HEAD_PLANE_MAJOR", "ragged_reduce_scatter_gated", "PreparedRelayout", "H3_LAUNCH_SERIAL",
     "PreparedReduceScatter", "prepare_seq_to_head", "prepare_head_to_seq",
+    "seq_to_head_rank", "head_to_seq_rank", "ragged_reduce_scatter_rank", "ragged_all_gather_rank",
     "prepare_ragged_reduce_scatter",
 ]
 
@@ -460,6 +461,121 @@ def ragged_reduce_scatter_gated(partials, bias, gate, seg_bounds, x, out=None, *
 # ---------------------------------------------------------------------------
 # prepared calls: validate and marshal once, then one C call per invocation
 # ---------------------------------------------------------------------------
+
+# ---------------------------------------------------------------------------
+# One rank per GPU: rank k's share of each operation, pulled from every rank's
+# buffer (``h3_*_rank``).  Inputs are W tensors or device addresses (for
+# example ``peers.PeerBuffers(...).pointers``); the output is this rank's tensor.
+# ---------------------------------------------------------------------------
+def _addresses(items, what: str) -> list:
+    out = []
+    for x in items:
+        if isinstance(x, torch.Tensor):
+            if not x.is_cuda or not x.is_contiguous() or x.element_size() != 2:
+                raise ValueError(f"{what}: CUDA, contiguous, 2-byte elements")
+            out.append(int(x.data_ptr()))
+        elif x is None:
+            raise ValueError(f"{what}: no buffer")
+        else:
+            out.append(int(x))
+    return out
+
+
+def _local_output(t: torch.Tensor, what: str, dims: int):
+    _check_tensors([t], what)
+    if t.dim() != dims:
+        raise ValueError(f"{what} must be {dims}-D")
+    return t.device
+
+
+def seq_to_head_rank(send, recv, rank: int, *, n_heads: int, window_bytes: int = 0, stream=None,
+                     variant: int = 0, ctas_per_sm: int = 0, serial: bool = False) -> dict:
+    """Rank ``rank``'s head-side buffer with one rank per GPU
+    (``h3_seq_to_head_rank``): send = the W ranks' sequence-side buffers
+    [T_r, P, H, D]; recv = this rank's [T, P, H_k, D]."""
+    send = list(send)
+    W = len(send)
+    dev = _local_output(recv, "recv", 4)
+    T, P, Hk, D = (int(v) for v in recv.shape)
+    if Hk != partition(T, n_heads, W).heads(rank):
+        raise ValueError(f"recv has {Hk} heads; rank {rank} of {W} owns "
+                         f"{partition(T, n_heads, W).heads(rank)}")
+    info = ExecInfo()
+    with torch.cuda.device(dev):
+        st = _abi.lib.h3_seq_to_head_rank(
+            _abi.pointer_array(_addresses(send, "send")), C.c_void_p(recv.data_ptr()), T, P,
+            int(n_heads), D, W, int(rank), int(window_bytes),
+            C.c_void_p(_stream_handle(stream, dev)), _config(variant, ctas_per_sm, serial),
+            C.byref(info))
+    _abi.check(st, "h3_seq_to_head_rank")
+    return info.as_dict()
+
+
+def head_to_seq_rank(send, recv, rank: int, *, n_tokens: int, window_bytes: int = 0, stream=None,
+                     variant: int = 0, ctas_per_sm: int = 0, serial: bool = False) -> dict:
+    """Rank ``rank``'s sequence-side rows with one rank per GPU
+    (``h3_head_to_seq_rank``): send = the W ranks' head-side buffers
+    [T, P, H_j, D]; recv = this rank's [T_k, P, H, D]."""
+    send = list(send)
+    W = len(send)
+    dev = _local_output(recv, "recv", 4)
+    Tk, P, H, D = (int(v) for v in recv.shape)
+    if Tk != partition(n_tokens, H, W).tokens(rank):
+        raise ValueError(f"recv has {Tk} tokens; rank {rank} of {W} owns "
+                         f"{partition(n_tokens, H, W).tokens(rank)}")
+    info = ExecInfo()
+    with torch.cuda.device(dev):
+        st = _abi.lib.h3_head_to_seq_rank(
+            _abi.pointer_array(_addresses(send, "send")), C.c_void_p(recv.data_ptr()),
+            int(n_tokens), P, H, D, W, int(rank), int(window_bytes),
+            C.c_void_p(_stream_handle(stream, dev)), _config(variant, ctas_per_sm, serial),
+            C.byref(info))
+    _abi.check(st, "h3_head_to_seq_rank")
+    return info.as_dict()
+
+
+def ragged_reduce_scatter_rank(partials, bias, out, rank: int, *, n_tokens: int, stream=None,
+                               ctas_per_sm: int = 0, serial: bool = False) -> dict:
+    """Rank ``rank``'s rows of the ragged reduce-scatter with one rank per GPU
+    (``h3_ragged_reduce_scatter_rank``): partials = the W ranks' [T, C];
+    bias = [C] tensor, address or None; out = this rank's [T_k, C]."""
+    partials = list(partials)
+    W = len(partials)
+    dev = _local_output(out, "out", 2)
+    Tk, Cc = (int(v) for v in out.shape)
+    if Tk != partition(n_tokens, W, W).tokens(rank):
+        raise ValueError(f"out has {Tk} rows; rank {rank} of {W} owns "
+                         f"{partition(n_tokens, W, W).tokens(rank)}")
+    b = 0 if bias is None else _addresses([bias], "bias")[0]
+    info = ExecInfo()
+    with torch.cuda.device(dev):
+        st = _abi.lib.h3_ragged_reduce_scatter_rank(
+            _abi.pointer_array(_addresses(partials, "partials")), C.c_void_p(b),
+            C.c_void_p(out.data_ptr()), int(n_tokens), Cc, W, int(rank),
+            C.c_void_p(_stream_handle(stream, dev)), _config(0, ctas_per_sm, serial),
+            C.byref(info))
+    _abi.check(st, "h3_ragged_reduce_scatter_rank")
+    return info.as_dict()
+
+
+def ragged_all_gather_rank(blocks, out, rank: int, *, stream=None, ctas_per_sm: int = 0,
+                           serial: bool = False) -> dict:
+    """Rank ``rank``'s copy of the ragged all-gather with one rank per GPU
+    (``h3_ragged_all_gather_rank``): blocks = the W ranks' [T_r, C]; out =
+    this rank's [T, C]."""
+    blocks = list(blocks)
+    W = len(blocks)
+    dev = _local_output(out, "out", 2)
+    T, Cc = (int(v) for v in out.shape)
+    info = ExecInfo()
+    with torch.cuda.device(dev):
+        st = _abi.lib.h3_ragged_all_gather_rank(
+            _abi.pointer_array(_addresses(blocks, "blocks")), C.c_void_p(out.data_ptr()), T, Cc,
+            W, int(rank), C.c_void_p(_stream_handle(stream, dev)),
+            _config(0, ctas_per_sm, serial), C.byref(info))
+    _abi.check(st, "h3_ragged_all_gather_rank")
+    return info.as_dict()
+
 
 class PreparedRelayout:
     """A relayout whose shapes, buffers and launch options are checked and

@@ -44,6 +44,7 @@ MAX_WORLD = 64
 H3_LAYOUT_SEQ_PLANE_MAJOR = 1
 H3_LAYOUT_HEAD_PLANE_MAJOR = 2
 H3_LAUNCH_SERIAL = 1
+H3_IPC_HANDLE_BYTES = 64
 ABI_VERSION = 2
 
 
@@ -67,6 +68,14 @@ class LaunchConfig(C.Structure):
         ("ctas_per_sm", C.c_int32),
         ("flags", C.c_int32),
         ("reserved1", C.c_int32),
+    ]
+
+
+class IpcHandle(C.Structure):
+    _fields_ = [
+        ("handle", C.c_ubyte * H3_IPC_HANDLE_BYTES),
+        ("offset", C.c_int64),
+        ("alloc_bytes", C.c_int64),
     ]
 
 
@@ -149,6 +158,26 @@ def _load() -> C.CDLL:
     lib.h3_last_cuda_error.argtypes = [C.POINTER(C.c_char_p)]
     lib.h3_bulk_wait_timeouts.restype = C.c_int
     lib.h3_bulk_wait_timeouts.argtypes = [C.c_void_p, C.POINTER(C.c_uint32), C.c_int32]
+    for name in ("h3_seq_to_head_rank", "h3_head_to_seq_rank"):
+        f = getattr(lib, name)
+        f.restype = C.c_int
+        f.argtypes = [_vpp, C.c_void_p, C.c_int64, C.c_int32, C.c_int32, C.c_int32, C.c_int32,
+                      C.c_int32, C.c_int64, C.c_void_p, C.POINTER(LaunchConfig),
+                      C.POINTER(ExecInfo)]
+    lib.h3_ragged_reduce_scatter_rank.restype = C.c_int
+    lib.h3_ragged_reduce_scatter_rank.argtypes = [_vpp, C.c_void_p, C.c_void_p, C.c_int64,
+                                                  C.c_int64, C.c_int32, C.c_int32, C.c_void_p,
+                                                  C.POINTER(LaunchConfig), C.POINTER(ExecInfo)]
+    lib.h3_ragged_all_gather_rank.restype = C.c_int
+    lib.h3_ragged_all_gather_rank.argtypes = [_vpp, C.c_void_p, C.c_int64, C.c_int64, C.c_int32,
+                                              C.c_int32, C.c_void_p, C.POINTER(LaunchConfig),
+                                              C.POINTER(ExecInfo)]
+    lib.h3_ipc_export.restype = C.c_int
+    lib.h3_ipc_export.argtypes = [C.c_void_p, C.POINTER(IpcHandle)]
+    lib.h3_ipc_open.restype = C.c_int
+    lib.h3_ipc_open.argtypes = [C.POINTER(IpcHandle), C.POINTER(C.c_void_p)]
+    lib.h3_ipc_close.restype = C.c_int
+    lib.h3_ipc_close.argtypes = [C.c_void_p, C.POINTER(IpcHandle)]
     version = lib.h3_abi_version()
     if version != ABI_VERSION:
         raise ImportError(f"libh3rr ABI version {version}, binding expects {ABI_VERSION}")

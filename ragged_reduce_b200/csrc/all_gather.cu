@@ -245,8 +245,11 @@ bool wide_ok(const GatherArgs& a)
 {
     if ((a.row_bytes % 32) != 0)
         return false;
-    for (int r = 0; r < a.W; ++r)
-        if ((reinterpret_cast<uintptr_t>(a.in[r]) & 31u) || (reinterpret_cast<uintptr_t>(a.out[r]) & 31u))
+    for (int r = 0; r < a.n_in; ++r)
+        if (reinterpret_cast<uintptr_t>(a.in[r]) & 31u)
+            return false;
+    for (int j = 0; j < a.W; ++j)
+        if (reinterpret_cast<uintptr_t>(a.out[j]) & 31u)
             return false;
     return true;
 }

@@ -20,9 +20,9 @@ h3_status cuda_failure(cudaError_t err)
     return H3_ERR_CUDA;
 }
 
-constexpr int64_t kMaxInt32 = INT32_MAX;
-// Column loops step by up to 1024 vectors past the row end; keep that in int32.
-constexpr int64_t kMaxRowVecs = int64_t(1) << 30;
+}  // namespace
+
+namespace h3rr {
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
@@ -70,6 +70,10 @@ h3_status check_no_overlap(const void* const* in, const uint64_t* in_bytes, int 
     }
     return H3_OK;
 }
+
+}  // namespace h3rr
+
+namespace {
 
 h3_status check_relayout_args(bool seq_to_head, const void* const* send, void* const* recv,
                               int64_t n_tokens, int32_t planes, int32_t n_heads, int32_t head_dim,
@@ -601,6 +605,7 @@ h3_status h3_ragged_all_gather_ex(const void* const* in, void* const* out, int64
     }
     a.T = int32_t(n_tokens);
     a.W = world;
+    a.n_in = world;
     a.tq = int32_t(ts.q);
     a.tm = int32_t(ts.m);
     a.row_vecs = int32_t(cols / 8);

@@ -1,6 +1,7 @@
 // Internal declarations shared by the host plan, the kernels and the C ABI.
 #pragma once
 
+#include <climits>
 #include <cstdint>
 
 #include <cuda_runtime.h>
@@ -11,6 +12,25 @@ namespace h3rr {
 
 constexpr int kMaxWorld = H3RR_MAX_WORLD;
 constexpr int kVecBytes = 16;  // one 16-byte vector = 8 BF16 values
+constexpr int64_t kMaxInt32 = INT32_MAX;
+// Column loops step by up to 1024 vectors past the row end; keep that in int32.
+constexpr int64_t kMaxRowVecs = int64_t(1) << 30;
+
+// ---------------------------------------------------------------------------
+// Argument checks shared by the entry points (api.cpp, rank.cpp).
+// ---------------------------------------------------------------------------
+bool aligned16(const void* p);
+void clear_info(h3_exec_info* info);
+// Launch-config fields every entry point checks the same way.
+bool config_ok(const h3_launch_config* cfg);
+bool programmatic_launch(const h3_launch_config* cfg);
+// Partition checks ("Distributed H3 Execution", intro: empty token or head
+// partitions are rejected).
+h3_status check_world(int64_t n_tokens, int64_t n_heads, int32_t world);
+// Outputs may not overlap inputs or each other (FastVideo PR #1807, "Problem
+// and behavior": outputs keep storage of their own).
+h3_status check_no_overlap(const void* const* in, const uint64_t* in_bytes, int n_in,
+                           void* const* out, const uint64_t* out_bytes, int n_out);
 
 // ---------------------------------------------------------------------------
 // Quotient/remainder partition ("Distributed H3 Execution", "Partition
@@ -94,10 +114,30 @@ struct GatherArgs {
     const char* in[kMaxWorld];
     char* out[kMaxWorld];
     int32_t T;
-    int32_t W;
+    int32_t W;          // outputs written (every row goes to out[0..W-1])
+    int32_t n_in;       // input blocks (the token split's ranks)
     int32_t tq, tm;
     int32_t row_vecs;   // C / 8
     int64_t row_bytes;  // C * 2
+};
+
+// One rank's share of sequence->head (one rank per GPU): for every (t, p) of
+// the launch, the run of heads [hs, hs + H_k) of the sequence-side row held
+// by token t's rank, copied to row (t, p) of this rank's head-side buffer.
+struct PullArgs {
+    const char* src[kMaxWorld];  // sequence-side buffers [T_r, P, H, D], any GPU
+    char* dst;                   // this rank's head-side buffer [T, P, H_k, D]
+    int32_t W;                   // ranks (entries of src)
+    int32_t T;
+    int32_t P;
+    int32_t plane0;
+    int32_t nplanes;
+    int32_t rows;                // T * nplanes
+    int32_t tq, tm;              // token split
+    int32_t row_vecs;            // H * D * 2 / 16
+    int32_t run_vecs;            // H_k * D * 2 / 16
+    int32_t col0_vecs;           // hs * D * 2 / 16
+    int32_t wait_late;           // as RelayoutArgs::wait_late
 };
 
 // Reduce-scatter fused with residual gating per packed segment.
@@ -140,6 +180,10 @@ h3_status staged_relayout_with_window(bool seq_to_head, const void* const* send,
 
 // Record `err` as the calling thread's last CUDA error; returns H3_ERR_CUDA.
 h3_status record_cuda_failure(cudaError_t err);
+
+// Enqueue one launch of a rank's share of sequence->head.
+cudaError_t launch_pull_seq_to_head(const PullArgs& a, int ctas_per_sm, cudaStream_t stream,
+                                    LaunchShape* shape, bool programmatic);
 
 // Enqueue the all-gather launch (variant 0 / H3_VARIANT_VECTOR or H3_VARIANT_BULK).
 cudaError_t launch_all_gather(const GatherArgs& a, int variant, int ctas_per_sm, cudaStream_t stream,

@@ -1,0 +1,342 @@
+// C ABI entry points for one rank per GPU (include/h3rr.h, "One rank per
+// GPU"): rank k's share of each operation, pulled from every rank's buffer.
+//
+// "Distributed H3 Execution", "Remaining GPU Gates": the real collective at
+// 2-8 GPUs must give what the single-GPU path gives.  Each rank call below
+// writes exactly rank k's part of the one-GPU call's output:
+//
+//   seq->head  rank k's [T, P, H_k, D] head-side buffer; a kernel of its own
+//              (one contiguous run of H_k heads per (t, p) row).
+//   head->seq  rank k's [T_k, P, H, D] rows: the one-GPU head->seq kernel run
+//              over a single-rank token split of T_k tokens, with every
+//              head-side pointer advanced to row (ts_k, 0).
+//   reduce     rank k's [T_k, C] rows: the one-GPU reduce-scatter kernel over
+//              a single-rank split, every partial advanced to row ts_k.
+//   all-gather rank k's [T, C]: the one-GPU all-gather kernel writing one
+//              output.
+//
+// Inputs may be on other GPUs (mapped with h3_ipc_open); the kernels read them
+// with plain vector loads.  All checks run before anything is enqueued.
+#include <cstring>
+
+#include "h3rr_internal.h"
+
+using namespace h3rr;
+
+namespace {
+
+h3_status fail(cudaError_t err) { return record_cuda_failure(err); }
+
+void fill_info(h3_exec_info* info, int launches, int chunks, const LaunchShape& shape,
+               int planes_per_launch)
+{
+    if (!info)
+        return;
+    info->launches = launches;
+    info->chunks = chunks;
+    info->grid = shape.grid;
+    info->block = shape.block;
+    info->variant = shape.variant;
+    info->planes_per_launch = planes_per_launch;
+}
+
+// Checks of a relayout rank call; on success *chunked tells whether the
+// window asks for one plane per launch.
+h3_status check_relayout_rank(bool seq_to_head, const void* const* send, const void* recv,
+                              int64_t n_tokens, int32_t planes, int32_t n_heads, int32_t head_dim,
+                              int32_t world, int32_t rank, int64_t window_bytes,
+                              const h3_launch_config* cfg, bool* chunked)
+{
+    if (window_bytes < 0)
+        return H3_ERR_INVALID_ARG;
+    if (cfg && cfg->variant == H3_VARIANT_BULK)
+        return H3_ERR_UNSUPPORTED;
+    if (cfg && cfg->variant != 0 && cfg->variant != H3_VARIANT_VECTOR)
+        return H3_ERR_INVALID_ARG;
+    if (!config_ok(cfg))
+        return H3_ERR_INVALID_ARG;
+    h3_status st = check_world(n_tokens, n_heads, world);
+    if (st != H3_OK)
+        return st;
+    if (rank < 0 || rank >= world || planes < 1 || head_dim < 1 || !send || !recv)
+        return H3_ERR_INVALID_ARG;
+    if ((int64_t(head_dim) * 2) % kVecBytes != 0)
+        return H3_ERR_MISALIGNED;
+    if (n_tokens > kMaxInt32 || n_tokens * planes > kMaxInt32 ||
+        int64_t(n_heads) * head_dim * 2 / kVecBytes > kMaxRowVecs)
+        return H3_ERR_UNSUPPORTED;
+    const Split ts = make_split(n_tokens, world);
+    const Split hs = make_split(n_heads, world);
+    const uint64_t row_bytes = uint64_t(n_heads) * head_dim * 2;
+    const uint64_t head_bytes = uint64_t(head_dim) * 2;
+    uint64_t in_bytes[kMaxWorld];
+    for (int r = 0; r < world; ++r) {
+        if (!send[r])
+            return H3_ERR_INVALID_ARG;
+        if (!aligned16(send[r]))
+            return H3_ERR_MISALIGNED;
+        in_bytes[r] = seq_to_head ? uint64_t(ts.size(r)) * planes * row_bytes
+                                  : uint64_t(n_tokens) * planes * uint64_t(hs.size(r)) * head_bytes;
+    }
+    if (!aligned16(recv))
+        return H3_ERR_MISALIGNED;
+    const uint64_t out_bytes = seq_to_head
+                                   ? uint64_t(n_tokens) * planes * uint64_t(hs.size(rank)) * head_bytes
+                                   : uint64_t(ts.size(rank)) * planes * row_bytes;
+    void* out[1] = {const_cast<void*>(recv)};
+    st = check_no_overlap(send, in_bytes, world, out, &out_bytes, 1);
+    if (st != H3_OK)
+        return st;
+    // The window bounds every rank's per-plane slices, exactly as in the
+    // one-GPU call, so that all ranks chunk alike.
+    *chunked = window_bytes > 0;
+    if (*chunked) {
+        const uint64_t seq_plane = uint64_t(ts.largest()) * row_bytes;
+        const uint64_t head_plane = uint64_t(n_tokens) * uint64_t(hs.largest()) * head_bytes;
+        if (seq_plane > uint64_t(window_bytes) || head_plane > uint64_t(window_bytes))
+            return H3_ERR_WINDOW;
+    }
+    return H3_OK;
+}
+
+// Checks of a reduce-scatter or all-gather rank call (rows of `cols` BF16).
+h3_status check_rows_rank(const void* const* in, const uint64_t* in_rows, const void* extra_in,
+                          const void* out, uint64_t out_rows, int64_t cols, int32_t world)
+{
+    const uint64_t row_bytes = uint64_t(cols) * 2;
+    const void* inputs[kMaxWorld + 1];
+    uint64_t in_bytes[kMaxWorld + 1];
+    for (int r = 0; r < world; ++r) {
+        if (!in[r])
+            return H3_ERR_INVALID_ARG;
+        if (!aligned16(in[r]))
+            return H3_ERR_MISALIGNED;
+        inputs[r] = in[r];
+        in_bytes[r] = in_rows[r] * row_bytes;
+    }
+    int n_in = world;
+    if (extra_in) {
+        if (!aligned16(extra_in))
+            return H3_ERR_MISALIGNED;
+        inputs[n_in] = extra_in;
+        in_bytes[n_in] = row_bytes;
+        ++n_in;
+    }
+    if (!aligned16(out))
+        return H3_ERR_MISALIGNED;
+    void* outs[1] = {const_cast<void*>(out)};
+    const uint64_t out_bytes = out_rows * row_bytes;
+    return check_no_overlap(inputs, in_bytes, n_in, outs, &out_bytes, 1);
+}
+
+h3_status check_cols(int64_t n_tokens, int64_t cols, int32_t world, int32_t rank,
+                     const void* in, const void* out)
+{
+    h3_status st = check_world(n_tokens, world, world);
+    if (st != H3_OK)
+        return st;
+    if (cols < 1 || !in || !out || rank < 0 || rank >= world)
+        return H3_ERR_INVALID_ARG;
+    if (cols % 8 != 0)
+        return H3_ERR_MISALIGNED;
+    if (n_tokens > kMaxInt32 || cols / 8 > kMaxRowVecs)
+        return H3_ERR_UNSUPPORTED;
+    return H3_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+h3_status h3_seq_to_head_rank(const void* const* send, void* recv, int64_t n_tokens,
+                              int32_t planes, int32_t n_heads, int32_t head_dim, int32_t world,
+                              int32_t rank, int64_t window_bytes, void* stream,
+                              const h3_launch_config* cfg, h3_exec_info* info)
+{
+    clear_info(info);
+    bool chunked = false;
+    h3_status st = check_relayout_rank(true, send, recv, n_tokens, planes, n_heads, head_dim, world,
+                                       rank, window_bytes, cfg, &chunked);
+    if (st != H3_OK)
+        return st;
+    const Split ts = make_split(n_tokens, world);
+    const Split hs = make_split(n_heads, world);
+    const int64_t head_vecs = int64_t(head_dim) * 2 / kVecBytes;
+    PullArgs a;
+    std::memset(&a, 0, sizeof(a));
+    for (int r = 0; r < world; ++r)
+        a.src[r] = static_cast<const char*>(send[r]);
+    a.dst = static_cast<char*>(recv);
+    a.W = world;
+    a.T = int32_t(n_tokens);
+    a.P = planes;
+    a.tq = int32_t(ts.q);
+    a.tm = int32_t(ts.m);
+    a.row_vecs = int32_t(int64_t(n_heads) * head_vecs);
+    a.run_vecs = int32_t(hs.size(rank) * head_vecs);
+    a.col0_vecs = int32_t(hs.start(rank) * head_vecs);
+    const int chunks = chunked ? planes : 1;
+    const int per_launch = chunked ? 1 : planes;
+    const bool programmatic = programmatic_launch(cfg);
+    LaunchShape shape;
+    for (int c = 0; c < chunks; ++c) {
+        a.plane0 = c * per_launch;
+        a.nplanes = per_launch;
+        a.rows = int32_t(n_tokens * per_launch);
+        a.wait_late = c > 0 ? 1 : 0;  // planes are disjoint (see h3_launch_config)
+        const cudaError_t err = launch_pull_seq_to_head(a, cfg ? cfg->ctas_per_sm : 0,
+                                                        static_cast<cudaStream_t>(stream), &shape,
+                                                        programmatic);
+        if (err != cudaSuccess) {
+            fill_info(info, c, chunks, shape, per_launch);
+            return fail(err);
+        }
+    }
+    fill_info(info, chunks, chunks, shape, per_launch);
+    return H3_OK;
+}
+
+h3_status h3_head_to_seq_rank(const void* const* send, void* recv, int64_t n_tokens,
+                              int32_t planes, int32_t n_heads, int32_t head_dim, int32_t world,
+                              int32_t rank, int64_t window_bytes, void* stream,
+                              const h3_launch_config* cfg, h3_exec_info* info)
+{
+    clear_info(info);
+    bool chunked = false;
+    h3_status st = check_relayout_rank(false, send, recv, n_tokens, planes, n_heads, head_dim,
+                                       world, rank, window_bytes, cfg, &chunked);
+    if (st != H3_OK)
+        return st;
+    const Split ts = make_split(n_tokens, world);
+    const Split hs = make_split(n_heads, world);
+    const int64_t head_bytes = int64_t(head_dim) * 2;
+    const int64_t t_start = ts.start(rank);
+    const int64_t t_rows = ts.size(rank);
+    // A one-rank token split of T_k tokens: every row belongs to "rank 0",
+    // whose sequence-side buffer is this rank's; head-side row (t', p) of the
+    // advanced pointers is global row (ts_k + t', p).
+    RelayoutArgs a;
+    std::memset(&a, 0, sizeof(a));
+    a.seq[0] = static_cast<char*>(recv);
+    for (int j = 0; j < world; ++j)
+        a.head[j] = const_cast<char*>(static_cast<const char*>(send[j])) +
+                    t_start * planes * hs.size(j) * head_bytes;
+    a.T = int32_t(t_rows);
+    a.P = planes;
+    a.W = world;
+    a.tq = int32_t(t_rows);
+    a.tm = 0;
+    a.hq = int32_t(hs.q);
+    a.hm = int32_t(hs.m);
+    a.row_vecs = int32_t(int64_t(n_heads) * head_bytes / kVecBytes);
+    a.head_vecs = int32_t(head_bytes / kVecBytes);
+    const int chunks = chunked ? planes : 1;
+    const int per_launch = chunked ? 1 : planes;
+    const bool programmatic = programmatic_launch(cfg);
+    const int variant = cfg ? cfg->variant : 0;
+    LaunchShape shape;
+    for (int c = 0; c < chunks; ++c) {
+        a.plane0 = c * per_launch;
+        a.nplanes = per_launch;
+        a.rows = int32_t(t_rows * per_launch);
+        a.wait_late = c > 0 ? 1 : 0;
+        const cudaError_t err =
+            launch_relayout(false, a, variant, cfg ? cfg->ctas_per_sm : 0,
+                            static_cast<cudaStream_t>(stream), &shape, false, programmatic);
+        if (err != cudaSuccess) {
+            fill_info(info, c, chunks, shape, per_launch);
+            return fail(err);
+        }
+    }
+    fill_info(info, chunks, chunks, shape, per_launch);
+    return H3_OK;
+}
+
+h3_status h3_ragged_reduce_scatter_rank(const void* const* partials, const void* bias, void* out,
+                                        int64_t n_tokens, int64_t cols, int32_t world,
+                                        int32_t rank, void* stream, const h3_launch_config* cfg,
+                                        h3_exec_info* info)
+{
+    clear_info(info);
+    h3_status st = check_cols(n_tokens, cols, world, rank, partials, out);
+    if (st != H3_OK)
+        return st;
+    if (cfg && cfg->variant != 0 && cfg->variant != H3_VARIANT_REDUCE)
+        return H3_ERR_INVALID_ARG;
+    if (!config_ok(cfg))
+        return H3_ERR_INVALID_ARG;
+    const Split ts = make_split(n_tokens, world);
+    uint64_t in_rows[kMaxWorld];
+    for (int r = 0; r < world; ++r)
+        in_rows[r] = uint64_t(n_tokens);
+    st = check_rows_rank(partials, in_rows, bias, out, uint64_t(ts.size(rank)), cols, world);
+    if (st != H3_OK)
+        return st;
+    const int64_t row_bytes = cols * 2;
+    const int64_t t_rows = ts.size(rank);
+    ReduceArgs a;
+    std::memset(&a, 0, sizeof(a));
+    for (int r = 0; r < world; ++r)
+        a.part[r] = static_cast<const char*>(partials[r]) + ts.start(rank) * row_bytes;
+    a.out[0] = static_cast<char*>(out);
+    a.bias = static_cast<const char*>(bias);
+    a.T = int32_t(t_rows);
+    a.W = world;
+    a.tq = int32_t(t_rows);  // one-rank split: every row is this rank's
+    a.tm = 0;
+    a.row_vecs = int32_t(cols / 8);
+    a.row_bytes = row_bytes;
+    LaunchShape shape;
+    const cudaError_t err =
+        launch_reduce_scatter(a, cfg ? cfg->ctas_per_sm : 0, static_cast<cudaStream_t>(stream),
+                              &shape, programmatic_launch(cfg));
+    if (err != cudaSuccess)
+        return fail(err);
+    fill_info(info, 1, 1, shape, 1);
+    return H3_OK;
+}
+
+h3_status h3_ragged_all_gather_rank(const void* const* in, void* out, int64_t n_tokens,
+                                    int64_t cols, int32_t world, int32_t rank, void* stream,
+                                    const h3_launch_config* cfg, h3_exec_info* info)
+{
+    clear_info(info);
+    h3_status st = check_cols(n_tokens, cols, world, rank, in, out);
+    if (st != H3_OK)
+        return st;
+    if (cfg && cfg->variant == H3_VARIANT_BULK)
+        return H3_ERR_UNSUPPORTED;
+    if (cfg && cfg->variant != 0 && cfg->variant != H3_VARIANT_VECTOR)
+        return H3_ERR_INVALID_ARG;
+    if (!config_ok(cfg))
+        return H3_ERR_INVALID_ARG;
+    const Split ts = make_split(n_tokens, world);
+    uint64_t in_rows[kMaxWorld];
+    for (int r = 0; r < world; ++r)
+        in_rows[r] = uint64_t(ts.size(r));
+    st = check_rows_rank(in, in_rows, nullptr, out, uint64_t(n_tokens), cols, world);
+    if (st != H3_OK)
+        return st;
+    GatherArgs a;
+    std::memset(&a, 0, sizeof(a));
+    for (int r = 0; r < world; ++r)
+        a.in[r] = static_cast<const char*>(in[r]);
+    a.out[0] = static_cast<char*>(out);
+    a.T = int32_t(n_tokens);
+    a.W = 1;  // one output: this rank's
+    a.n_in = world;
+    a.tq = int32_t(ts.q);
+    a.tm = int32_t(ts.m);
+    a.row_vecs = int32_t(cols / 8);
+    a.row_bytes = cols * 2;
+    LaunchShape shape;
+    const cudaError_t err =
+        launch_all_gather(a, 0, cfg ? cfg->ctas_per_sm : 0, static_cast<cudaStream_t>(stream),
+                          &shape, programmatic_launch(cfg));
+    if (err != cudaSuccess)
+        return fail(err);
+    fill_info(info, 1, 1, shape, 1);
+    return H3_OK;
+}
+
+}  // extern "C"

@@ -384,6 +384,49 @@ __global__ void __launch_bounds__(32) relayout_bulk_kernel(const __grid_constant
 }
 
 // ---------------------------------------------------------------------------
+// one rank's share of sequence->head (one rank per GPU)
+// ---------------------------------------------------------------------------
+// Row (t, p) of this rank's head-side buffer is one contiguous run of H_k
+// heads cut from the sequence-side row (t, p) of token t's rank, which may
+// live on another GPU.  One CTA per row; thread i copies vectors i, i+NT,
+// ... of the run, all loads before the stores, MAXV vectors per pass.
+template <int VW, int NT, int MAXV>
+__global__ void __launch_bounds__(NT) pull_seq_to_head_kernel(const __grid_constant__ PullArgs a)
+{
+    constexpr int kUnits = VW / kVecBytes;
+    const int32_t run_v = a.run_vecs / kUnits;
+    if (!a.wait_late)
+        pdl_wait_prerequisites();
+    pdl_allow_dependents();
+    for (int64_t i64 = blockIdx.x; i64 < a.rows; i64 += gridDim.x) {
+        const int32_t i = int32_t(i64);
+        const int32_t t = i / a.nplanes;
+        const int32_t p = a.plane0 + (i - t * a.nplanes);
+        const int32_t s = split_owner(t, a.tq, a.tm);
+        const int32_t tl = t - split_start(s, a.tq, a.tm);
+        const char* src = a.src[s] + ((int64_t(tl) * a.P + p) * a.row_vecs + a.col0_vecs) * kVecBytes;
+        char* dst = a.dst + (int64_t(t) * a.P + p) * a.run_vecs * kVecBytes;
+        for (int32_t c0 = 0; c0 < run_v; c0 += MAXV * NT) {
+            Vec<VW> v[MAXV];
+#pragma unroll
+            for (int k = 0; k < MAXV; ++k) {
+                const int32_t c = c0 + int32_t(threadIdx.x) + k * NT;
+                if (c < run_v)
+                    ld_stream(v[k], src + int64_t(c) * VW);
+            }
+#pragma unroll
+            for (int k = 0; k < MAXV; ++k) {
+                const int32_t c = c0 + int32_t(threadIdx.x) + k * NT;
+                if (c < run_v)
+                    st_stream(dst + int64_t(c) * VW, v[k]);
+            }
+        }
+    }
+    if (a.wait_late)
+        pdl_wait_prerequisites();
+}
+
+// ---------------------------------------------------------------------------
 // dispatch
 // ---------------------------------------------------------------------------
 struct KernelChoice {
@@ -537,6 +580,35 @@ cudaError_t launch_relayout(bool seq_to_head, const RelayoutArgs& a, int variant
     void* params[] = {const_cast<RelayoutArgs*>(&a)};
     return launch_kernel(kc.fn, grid, kc.threads, kc.smem, stream, params,
                          programmatic && kc.variant != H3_VARIANT_BULK);
+}
+
+cudaError_t launch_pull_seq_to_head(const PullArgs& a, int ctas_per_sm, cudaStream_t stream,
+                                    LaunchShape* shape, bool programmatic)
+{
+    int device = 0;
+    const int sms = current_sm_count(&device);
+    if (sms <= 0)
+        return cudaErrorNoDevice;
+    // 32-byte vectors when the run, its start and every buffer allow them.
+    bool wide = (a.row_vecs % 2) == 0 && (a.run_vecs % 2) == 0 && (a.col0_vecs % 2) == 0 &&
+                (reinterpret_cast<uintptr_t>(a.dst) & 31u) == 0;
+    for (int r = 0; wide && r < a.W; ++r)
+        wide = (reinterpret_cast<uintptr_t>(a.src[r]) & 31u) == 0;
+    const void* fn = wide ? (const void*)pull_seq_to_head_kernel<32, 64, 4>
+                          : (const void*)pull_seq_to_head_kernel<16, 128, 4>;
+    const int threads = wide ? 64 : 128;
+    int64_t grid = a.rows;  // one CTA per row, as the other register kernels
+    if (ctas_per_sm > 0 && int64_t(sms) * ctas_per_sm < grid)
+        grid = int64_t(sms) * ctas_per_sm;
+    if (grid < 1)
+        grid = 1;
+    if (shape) {
+        shape->grid = int(grid);
+        shape->block = threads;
+        shape->variant = H3_VARIANT_VECTOR;
+    }
+    void* params[] = {const_cast<PullArgs*>(&a)};
+    return launch_kernel(fn, grid, threads, 0, stream, params, programmatic);
 }
 
 cudaError_t read_bulk_wait_timeouts(unsigned int* count, bool reset, cudaStream_t stream)
