@@ -580,6 +580,28 @@ def run_workload_report(args):
             emit(w.name, "head_to_seq", vname, nbytes, secs, info)
             if not torch.equal(back_full.view(torch.int16), x.view(torch.int16)):
                 raise SystemExit(f"{w.name} {vname}: round trip differs")
+        if w.T in (32768, 131072):
+            # one rank per GPU, all W ranks' shares on this GPU back to back
+            # (the same bytes as the one-GPU call)
+            def s2h_ranks():
+                for k in range(w.W):
+                    last = rr.seq_to_head_rank(send, heads[k], k, n_heads=w.H,
+                                               window_bytes=w.window_bytes)
+                return last
+
+            def h2s_ranks():
+                for k in range(w.W):
+                    last = rr.head_to_seq_rank(heads, back[k], k, n_tokens=w.T,
+                                               window_bytes=w.window_bytes)
+                return last
+
+            for call, fn in (("seq_to_head", s2h_ranks), ("head_to_seq", h2s_ranks)):
+                info = dict(fn())
+                info["launches"] *= w.W
+                secs = _time_calls(fn, iters)
+                emit(w.name, call, "rank_shares", nbytes, secs, info)
+            if not torch.equal(back_full.view(torch.int16), x.view(torch.int16)):
+                raise SystemExit(f"{w.name} rank shares: round trip differs")
         if w.T < 32768:
             # small case: host overhead per call dominates; a prepared call
             # (checks and marshalling done once) and CUDA-graph replay
@@ -638,7 +660,20 @@ def run_workload_report(args):
         info = rr.ragged_reduce_scatter(plist, bias, out)
         secs = _time_calls(lambda: rr.ragged_reduce_scatter(plist, bias, out), iters)
         emit(rw.name, "ragged_reduce_scatter", "default", nbytes, secs, info)
-        del partials, bias, plist, out_full, out
+        want = out_full.clone()
+
+        def rs_ranks():
+            for k in range(rw.W):
+                last = rr.ragged_reduce_scatter_rank(plist, bias, out[k], k, n_tokens=rw.T)
+            return last
+
+        info = dict(rs_ranks())
+        info["launches"] *= rw.W
+        secs = _time_calls(rs_ranks, iters)
+        emit(rw.name, "ragged_reduce_scatter", "rank_shares", nbytes, secs, info)
+        if not torch.equal(out_full.view(torch.int16), want.view(torch.int16)):
+            raise SystemExit(f"{rw.name}: rank shares differ from the one-GPU call")
+        del partials, bias, plist, out_full, out, want
         torch.cuda.empty_cache()
     for rw, S in ((wl.RS_64K_W8, 16), (wl.ReduceWorkload("reduce_scatter_T32768_C7168_W6", T=32768,
                                                           C=wl.H3_HIDDEN, W=6, seed=102), 8)):
@@ -667,6 +702,20 @@ def run_workload_report(args):
         emit(f"all_gather_T{T}_C{C_}_W{W}", "ragged_all_gather", "default", nbytes, secs, info)
         if not all(torch.equal(o.view(torch.int16), full.view(torch.int16)) for o in outs):
             raise SystemExit("all-gather output differs")
+        for o in outs:
+            o.zero_()
+
+        def ag_ranks():
+            for k in range(W):
+                last = rr.ragged_all_gather_rank(blocks, outs[k], k)
+            return last
+
+        info = dict(ag_ranks())
+        info["launches"] *= W
+        secs = _time_calls(ag_ranks, iters)
+        emit(f"all_gather_T{T}_C{C_}_W{W}", "ragged_all_gather", "rank_shares", nbytes, secs, info)
+        if not all(torch.equal(o.view(torch.int16), full.view(torch.int16)) for o in outs):
+            raise SystemExit("all-gather rank shares differ")
         del full, blocks, outs
         torch.cuda.empty_cache()
     if rr.bulk_wait_timeouts() != 0:

@@ -459,6 +459,23 @@ H3RR_API h3_status h3_ragged_reduce_scatter_rank(const void* const* partials, co
                                                  const h3_launch_config* cfg,
                                                  h3_exec_info* info);
 
+/* Rank k's rows of the gated reduce-scatter (h3_ragged_reduce_scatter_gated
+ * with one rank per GPU): out [T_k, C] = bf16_rne(x + gate[seg(t)] * y) for
+ * t = ts_k + t', y = rank k's reduce-scatter rows; x [T_k, C] this rank's
+ * residual (out == x runs in place); gate [S, C] and seg_bounds [S+1] (host,
+ * global packed bounds, 0 = b_0 < ... < b_S = T, S <= H3RR_MAX_GATE_SEGMENTS)
+ * as in the one-GPU call.  Inside, the segments are clipped to [ts_k, te_k)
+ * and rebased ("Distributed H3 Execution", "Partition Contract"), as
+ * h3_partition reports them for rank k. */
+H3RR_API h3_status h3_ragged_reduce_scatter_gated_rank(const void* const* partials,
+                                                       const void* bias, const void* gate,
+                                                       const int64_t* seg_bounds, int32_t n_segs,
+                                                       const void* x, void* out,
+                                                       int64_t n_tokens, int64_t cols,
+                                                       int32_t world, int32_t rank, void* stream,
+                                                       const h3_launch_config* cfg,
+                                                       h3_exec_info* info);
+
 /* Rank k's copy of the ragged all-gather: out [T, C] (this GPU) gets every
  * rank's rows, out[t, c] = in[r(t)][t - ts_{r(t)}, c], from in[world]
  * ([T_r, C] each). */

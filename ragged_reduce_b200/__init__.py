@@ -40,6 +40,7 @@ __all__ = [
     "H3_LAYOUT_HEAD_PLANE_MAJOR", "ragged_reduce_scatter_gated", "PreparedRelayout", "H3_LAUNCH_SERIAL",
     "PreparedReduceScatter", "prepare_seq_to_head", "prepare_head_to_seq",
     "seq_to_head_rank", "head_to_seq_rank", "ragged_reduce_scatter_rank", "ragged_all_gather_rank",
+    "ragged_reduce_scatter_gated_rank",
     "prepare_ragged_reduce_scatter",
 ]
 
@@ -555,6 +556,39 @@ def ragged_reduce_scatter_rank(partials, bias, out, rank: int, *, n_tokens: int,
             C.c_void_p(_stream_handle(stream, dev)), _config(0, ctas_per_sm, serial),
             C.byref(info))
     _abi.check(st, "h3_ragged_reduce_scatter_rank")
+    return info.as_dict()
+
+
+def ragged_reduce_scatter_gated_rank(partials, bias, gate, seg_bounds, x, rank: int, *,
+                                     n_tokens: int, out=None, stream=None,
+                                     serial: bool = False) -> dict:
+    """Rank ``rank``'s rows of the gated reduce-scatter with one rank per GPU
+    (``h3_ragged_reduce_scatter_gated_rank``): partials = the W ranks' [T, C];
+    gate [S, C] and bias [C] (tensors or addresses); seg_bounds = the S+1
+    global packed bounds; x = this rank's residual [T_k, C]; out = x (in
+    place) unless given."""
+    partials = list(partials)
+    W = len(partials)
+    dev = _local_output(x, "x", 2)
+    out = x if out is None else out
+    _local_output(out, "out", 2)
+    Tk, Cc = (int(v) for v in x.shape)
+    if tuple(out.shape) != (Tk, Cc):
+        raise ValueError("out must have x's shape")
+    if Tk != partition(n_tokens, W, W).tokens(rank):
+        raise ValueError(f"x has {Tk} rows; rank {rank} of {W} owns "
+                         f"{partition(n_tokens, W, W).tokens(rank)}")
+    bounds = np.ascontiguousarray(np.asarray(seg_bounds, dtype=np.int64))
+    b = 0 if bias is None else _addresses([bias], "bias")[0]
+    info = ExecInfo()
+    with torch.cuda.device(dev):
+        st = _abi.lib.h3_ragged_reduce_scatter_gated_rank(
+            _abi.pointer_array(_addresses(partials, "partials")), C.c_void_p(b),
+            C.c_void_p(_addresses([gate], "gate")[0]),
+            bounds.ctypes.data_as(C.POINTER(C.c_int64)), int(bounds.size - 1),
+            C.c_void_p(x.data_ptr()), C.c_void_p(out.data_ptr()), int(n_tokens), Cc, W, int(rank),
+            C.c_void_p(_stream_handle(stream, dev)), _config(0, 0, serial), C.byref(info))
+    _abi.check(st, "h3_ragged_reduce_scatter_gated_rank")
     return info.as_dict()
 
 

@@ -168,6 +168,10 @@ def _load() -> C.CDLL:
     lib.h3_ragged_reduce_scatter_rank.argtypes = [_vpp, C.c_void_p, C.c_void_p, C.c_int64,
                                                   C.c_int64, C.c_int32, C.c_int32, C.c_void_p,
                                                   C.POINTER(LaunchConfig), C.POINTER(ExecInfo)]
+    lib.h3_ragged_reduce_scatter_gated_rank.restype = C.c_int
+    lib.h3_ragged_reduce_scatter_gated_rank.argtypes = [
+        _vpp, C.c_void_p, C.c_void_p, _i64p, C.c_int32, C.c_void_p, C.c_void_p, C.c_int64,
+        C.c_int64, C.c_int32, C.c_int32, C.c_void_p, C.POINTER(LaunchConfig), C.POINTER(ExecInfo)]
     lib.h3_ragged_all_gather_rank.restype = C.c_int
     lib.h3_ragged_all_gather_rank.argtypes = [_vpp, C.c_void_p, C.c_int64, C.c_int64, C.c_int32,
                                               C.c_int32, C.c_void_p, C.POINTER(LaunchConfig),

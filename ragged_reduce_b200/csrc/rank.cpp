@@ -14,6 +14,12 @@
 //              a single-rank split, every partial advanced to row ts_k.
 //   all-gather rank k's [T, C]: the one-GPU all-gather kernel writing one
 //              output.
+//   gated      rank k's [T_k, C]: the one-GPU gated kernel over the one-rank
+//              split, with the segments clipped to [ts_k, te_k) and rebased
+//              (the partition contract's per-rank segments) and the gate
+//              pointer advanced to the first of them: a rank's token range
+//              meets consecutive segments, so local piece i is segment
+//              s_0 + i.
 //
 // Inputs may be on other GPUs (mapped with h3_ipc_open); the kernels read them
 // with plain vector loads.  All checks run before anything is enqueued.
@@ -99,14 +105,21 @@ h3_status check_relayout_rank(bool seq_to_head, const void* const* send, const v
     return H3_OK;
 }
 
-// Checks of a reduce-scatter or all-gather rank call (rows of `cols` BF16).
+// Inputs one rank call may check: W partials, the gate rows, the residual
+// and the bias.
+constexpr int kMaxRankInputs = kMaxWorld + 3;
+
+// Checks of a reduce-scatter or all-gather rank call (rows of `cols` BF16):
+// n_in inputs of in_rows[i] rows each, plus one optional row (extra_in).
 h3_status check_rows_rank(const void* const* in, const uint64_t* in_rows, const void* extra_in,
-                          const void* out, uint64_t out_rows, int64_t cols, int32_t world)
+                          const void* out, uint64_t out_rows, int64_t cols, int32_t n_in_rows)
 {
+    if (n_in_rows < 0 || n_in_rows + (extra_in ? 1 : 0) > kMaxRankInputs)
+        return H3_ERR_INVALID_ARG;
     const uint64_t row_bytes = uint64_t(cols) * 2;
-    const void* inputs[kMaxWorld + 1];
-    uint64_t in_bytes[kMaxWorld + 1];
-    for (int r = 0; r < world; ++r) {
+    const void* inputs[kMaxRankInputs];
+    uint64_t in_bytes[kMaxRankInputs];
+    for (int r = 0; r < n_in_rows; ++r) {
         if (!in[r])
             return H3_ERR_INVALID_ARG;
         if (!aligned16(in[r]))
@@ -114,7 +127,7 @@ h3_status check_rows_rank(const void* const* in, const uint64_t* in_rows, const 
         inputs[r] = in[r];
         in_bytes[r] = in_rows[r] * row_bytes;
     }
-    int n_in = world;
+    int n_in = n_in_rows;
     if (extra_in) {
         if (!aligned16(extra_in))
             return H3_ERR_MISALIGNED;
@@ -266,7 +279,7 @@ h3_status h3_ragged_reduce_scatter_rank(const void* const* partials, const void*
     if (!config_ok(cfg))
         return H3_ERR_INVALID_ARG;
     const Split ts = make_split(n_tokens, world);
-    uint64_t in_rows[kMaxWorld];
+    uint64_t in_rows[kMaxWorld] = {};
     for (int r = 0; r < world; ++r)
         in_rows[r] = uint64_t(n_tokens);
     st = check_rows_rank(partials, in_rows, bias, out, uint64_t(ts.size(rank)), cols, world);
@@ -296,6 +309,82 @@ h3_status h3_ragged_reduce_scatter_rank(const void* const* partials, const void*
     return H3_OK;
 }
 
+h3_status h3_ragged_reduce_scatter_gated_rank(const void* const* partials, const void* bias,
+                                              const void* gate, const int64_t* seg_bounds,
+                                              int32_t n_segs, const void* x, void* out,
+                                              int64_t n_tokens, int64_t cols, int32_t world,
+                                              int32_t rank, void* stream,
+                                              const h3_launch_config* cfg, h3_exec_info* info)
+{
+    clear_info(info);
+    h3_status st = check_cols(n_tokens, cols, world, rank, partials, out);
+    if (st != H3_OK)
+        return st;
+    if (!x || !gate || !seg_bounds)
+        return H3_ERR_INVALID_ARG;
+    if (cfg && cfg->variant != 0 && cfg->variant != H3_VARIANT_REDUCE_GATED)
+        return H3_ERR_INVALID_ARG;
+    if (!config_ok(cfg))
+        return H3_ERR_INVALID_ARG;
+    if (n_segs < 1 || n_segs > H3RR_MAX_GATE_SEGMENTS)
+        return n_segs < 1 ? H3_ERR_INVALID_ARG : H3_ERR_UNSUPPORTED;
+    if (seg_bounds[0] != 0 || seg_bounds[n_segs] != n_tokens)
+        return H3_ERR_INVALID_ARG;
+    for (int32_t k = 0; k < n_segs; ++k)
+        if (seg_bounds[k + 1] <= seg_bounds[k])
+            return H3_ERR_INVALID_ARG;
+    if (!aligned16(gate) || !aligned16(x))
+        return H3_ERR_MISALIGNED;
+    const Split ts = make_split(n_tokens, world);
+    const int64_t row_bytes = cols * 2;
+    const int64_t t0 = ts.start(rank);
+    const int64_t t_rows = ts.size(rank);
+    // Inputs: partials, gate and (unless in place) x; the bias rides along.
+    const void* ins[kMaxRankInputs];
+    uint64_t in_rows[kMaxRankInputs];
+    int n_in = 0;
+    for (int r = 0; r < world; ++r) {
+        ins[n_in] = partials[r];
+        in_rows[n_in++] = uint64_t(n_tokens);
+    }
+    ins[n_in] = gate;
+    in_rows[n_in++] = uint64_t(n_segs);
+    if (x != out) {
+        ins[n_in] = x;
+        in_rows[n_in++] = uint64_t(t_rows);
+    }
+    st = check_rows_rank(ins, in_rows, bias, out, uint64_t(t_rows), cols, n_in);
+    if (st != H3_OK)
+        return st;
+    int64_t local_bounds[kMaxGateSegs + 1];
+    int32_t seg_ids[kMaxGateSegs];
+    const int32_t pieces = clip_segments(seg_bounds, n_segs, t0, t0 + t_rows, local_bounds, seg_ids);
+    GatedArgs g;
+    std::memset(&g, 0, sizeof(g));
+    for (int r = 0; r < world; ++r)
+        g.r.part[r] = static_cast<const char*>(partials[r]) + t0 * row_bytes;
+    g.r.out[0] = static_cast<char*>(out);
+    g.x[0] = static_cast<const char*>(x);
+    g.r.bias = static_cast<const char*>(bias);
+    g.r.T = int32_t(t_rows);
+    g.r.W = world;
+    g.r.tq = int32_t(t_rows);
+    g.r.tm = 0;
+    g.r.row_vecs = int32_t(cols / 8);
+    g.r.row_bytes = row_bytes;
+    g.gate = static_cast<const char*>(gate) + int64_t(seg_ids[0]) * row_bytes;
+    g.n_segs = pieces;
+    for (int32_t i = 0; i <= pieces; ++i)
+        g.seg_bounds[i] = int32_t(local_bounds[i]);
+    LaunchShape shape;
+    const cudaError_t err = launch_reduce_scatter_gated(g, static_cast<cudaStream_t>(stream), &shape,
+                                                        programmatic_launch(cfg));
+    if (err != cudaSuccess)
+        return fail(err);
+    fill_info(info, 1, 1, shape, 1);
+    return H3_OK;
+}
+
 h3_status h3_ragged_all_gather_rank(const void* const* in, void* out, int64_t n_tokens,
                                     int64_t cols, int32_t world, int32_t rank, void* stream,
                                     const h3_launch_config* cfg, h3_exec_info* info)
@@ -311,7 +400,7 @@ h3_status h3_ragged_all_gather_rank(const void* const* in, void* out, int64_t n_
     if (!config_ok(cfg))
         return H3_ERR_INVALID_ARG;
     const Split ts = make_split(n_tokens, world);
-    uint64_t in_rows[kMaxWorld];
+    uint64_t in_rows[kMaxWorld] = {};
     for (int r = 0; r < world; ++r)
         in_rows[r] = uint64_t(ts.size(r));
     st = check_rows_rank(in, in_rows, nullptr, out, uint64_t(n_tokens), cols, world);

@@ -388,10 +388,75 @@ __global__ void __launch_bounds__(32) relayout_bulk_kernel(const __grid_constant
 // ---------------------------------------------------------------------------
 // Row (t, p) of this rank's head-side buffer is one contiguous run of H_k
 // heads cut from the sequence-side row (t, p) of token t's rank, which may
-// live on another GPU.  One CTA per row; thread i copies vectors i, i+NT,
-// ... of the run, all loads before the stores, MAXV vectors per pass.
-template <int VW, int NT, int MAXV>
+// live on another GPU.  A run is short (2.5 KB for 10 heads of 128), and one
+// CTA per run left the kernel bound by the rate at which the GPU starts
+// CTAs, so a CTA takes ROWS consecutive runs laid end to end: thread i owns
+// vectors i, i+NT, ... of the group (a fixed run and column per slot), the
+// group's row addresses sit in shared memory, and all loads precede the
+// stores.  Needs ROWS * run <= NT * MAXV vectors.
+template <int VW, int NT, int ROWS, int MAXV>
 __global__ void __launch_bounds__(NT) pull_seq_to_head_kernel(const __grid_constant__ PullArgs a)
+{
+    constexpr int kUnits = VW / kVecBytes;
+    const int32_t run_v = a.run_vecs / kUnits;
+    __shared__ const char* s_src[ROWS];
+    __shared__ char* s_dst[ROWS];
+    int32_t slot_row[MAXV];
+    int32_t slot_col[MAXV];
+#pragma unroll
+    for (int k = 0; k < MAXV; ++k) {
+        const int32_t c = int32_t(threadIdx.x) + k * NT;
+        slot_row[k] = c / run_v;  // >= ROWS: no vector in this slot
+        slot_col[k] = c - slot_row[k] * run_v;
+    }
+    if (!a.wait_late)
+        pdl_wait_prerequisites();
+    pdl_allow_dependents();
+    for (int64_t i0 = int64_t(blockIdx.x) * ROWS; i0 < a.rows; i0 += int64_t(gridDim.x) * ROWS) {
+        if (threadIdx.x < ROWS) {
+            const int64_t i64 = i0 + threadIdx.x;
+            const char* src = nullptr;
+            char* dst = nullptr;
+            if (i64 < a.rows) {
+                const int32_t i = int32_t(i64);
+                const int32_t t = i / a.nplanes;
+                const int32_t p = a.plane0 + (i - t * a.nplanes);
+                const int32_t s = split_owner(t, a.tq, a.tm);
+                const int32_t tl = t - split_start(s, a.tq, a.tm);
+                src = a.src[s] + ((int64_t(tl) * a.P + p) * a.row_vecs + a.col0_vecs) * kVecBytes;
+                dst = a.dst + (int64_t(t) * a.P + p) * a.run_vecs * kVecBytes;
+            }
+            s_src[threadIdx.x] = src;
+            s_dst[threadIdx.x] = dst;
+        }
+        __syncthreads();
+        Vec<VW> v[MAXV];
+#pragma unroll
+        for (int k = 0; k < MAXV; ++k) {
+            if (slot_row[k] < ROWS) {
+                const char* src = s_src[slot_row[k]];
+                if (src)
+                    ld_stream(v[k], src + int64_t(slot_col[k]) * VW);
+            }
+        }
+#pragma unroll
+        for (int k = 0; k < MAXV; ++k) {
+            if (slot_row[k] < ROWS) {
+                char* dst = s_dst[slot_row[k]];
+                if (dst)
+                    st_stream(dst + int64_t(slot_col[k]) * VW, v[k]);
+            }
+        }
+        __syncthreads();  // the next group overwrites the row table
+    }
+    if (a.wait_late)
+        pdl_wait_prerequisites();
+}
+
+// Runs longer than one CTA's slots (NT * MAXV vectors): one run per CTA
+// iteration, in passes of NT * MAXV vectors.
+template <int VW, int NT, int MAXV>
+__global__ void __launch_bounds__(NT) pull_seq_to_head_long_kernel(const __grid_constant__ PullArgs a)
 {
     constexpr int kUnits = VW / kVecBytes;
     const int32_t run_v = a.run_vecs / kUnits;
@@ -582,6 +647,25 @@ cudaError_t launch_relayout(bool seq_to_head, const RelayoutArgs& a, int variant
                          programmatic && kc.variant != H3_VARIANT_BULK);
 }
 
+namespace {
+
+constexpr int kPullThreads = 128;
+constexpr int kPullSlots = 8;  // vectors per thread per group
+
+// The pull kernel for `rows_per_cta` runs per CTA (2, 4 or 8; one run per
+// CTA goes to the long-run kernel).
+template <int VW>
+const void* pull_kernel(int rows_per_cta)
+{
+    switch (rows_per_cta) {
+        case 8: return (const void*)pull_seq_to_head_kernel<VW, kPullThreads, 8, kPullSlots>;
+        case 4: return (const void*)pull_seq_to_head_kernel<VW, kPullThreads, 4, kPullSlots>;
+        default: return (const void*)pull_seq_to_head_kernel<VW, kPullThreads, 2, kPullSlots>;
+    }
+}
+
+}  // namespace
+
 cudaError_t launch_pull_seq_to_head(const PullArgs& a, int ctas_per_sm, cudaStream_t stream,
                                     LaunchShape* shape, bool programmatic)
 {
@@ -594,21 +678,33 @@ cudaError_t launch_pull_seq_to_head(const PullArgs& a, int ctas_per_sm, cudaStre
                 (reinterpret_cast<uintptr_t>(a.dst) & 31u) == 0;
     for (int r = 0; wide && r < a.W; ++r)
         wide = (reinterpret_cast<uintptr_t>(a.src[r]) & 31u) == 0;
-    const void* fn = wide ? (const void*)pull_seq_to_head_kernel<32, 64, 4>
-                          : (const void*)pull_seq_to_head_kernel<16, 128, 4>;
-    const int threads = wide ? 64 : 128;
-    int64_t grid = a.rows;  // one CTA per row, as the other register kernels
+    const int64_t run_v = wide ? a.run_vecs / 2 : a.run_vecs;
+    const int64_t slots = int64_t(kPullThreads) * kPullSlots;
+    // As many runs per CTA (up to 8) as fill the CTA's slots.
+    int rows_per_cta = 8;
+    while (rows_per_cta > 1 && rows_per_cta * run_v > slots)
+        rows_per_cta /= 2;
+    if (run_v > slots)
+        rows_per_cta = 1;
+    const void* fn;
+    if (rows_per_cta == 1)
+        fn = wide ? (const void*)pull_seq_to_head_long_kernel<32, kPullThreads, kPullSlots>
+                  : (const void*)pull_seq_to_head_long_kernel<16, kPullThreads, kPullSlots>;
+    else
+        fn = wide ? pull_kernel<32>(rows_per_cta) : pull_kernel<16>(rows_per_cta);
+    // One CTA per group of runs, as the other register kernels.
+    int64_t grid = (int64_t(a.rows) + rows_per_cta - 1) / rows_per_cta;
     if (ctas_per_sm > 0 && int64_t(sms) * ctas_per_sm < grid)
         grid = int64_t(sms) * ctas_per_sm;
     if (grid < 1)
         grid = 1;
     if (shape) {
         shape->grid = int(grid);
-        shape->block = threads;
+        shape->block = kPullThreads;
         shape->variant = H3_VARIANT_VECTOR;
     }
     void* params[] = {const_cast<PullArgs*>(&a)};
-    return launch_kernel(fn, grid, threads, 0, stream, params, programmatic);
+    return launch_kernel(fn, grid, kPullThreads, 0, stream, params, programmatic);
 }
 
 cudaError_t read_bulk_wait_timeouts(unsigned int* count, bool reset, cudaStream_t stream)

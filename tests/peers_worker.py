@@ -15,6 +15,7 @@ import sys
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 sys.path.insert(0, ROOT)
 
+import numpy as np  # noqa: E402
 import torch  # noqa: E402
 import torch.distributed as dist  # noqa: E402
 
@@ -81,6 +82,20 @@ def main():
     acc += bias.float()
     expect = acc.to(torch.bfloat16)
     checks["reduce_scatter"] = same(out, expect[rs0:rs1])
+
+    # gated, in place on this rank's residual rows
+    S = 5
+    gate = wl.normal_bf16((S, C), 13, 1.0, dev)
+    bounds = wl.segment_bounds(T, S, 14)
+    x_res = wl.normal_bf16((T, C), 15, 1.0, dev)
+    x_mine = x_res[rs0:rs1].clone()
+    rr.ragged_reduce_scatter_gated_rank(part_tab.pointers, bias, gate, bounds, x_mine, rank,
+                                        n_tokens=T)
+    torch.cuda.synchronize()
+    seg = torch.from_numpy(np.searchsorted(np.asarray(bounds), np.arange(T), side="right") - 1)
+    g_rows = gate.index_select(0, seg.to(dev))
+    gated = (x_res.float() + g_rows.float() * expect.float()).to(torch.bfloat16)
+    checks["gated"] = same(x_mine, gated[rs0:rs1])
 
     out_tab = peers.PeerBuffers(out)
     tables.append(out_tab)

@@ -2,8 +2,8 @@
 sharing one GPU, each holding only its own inputs and mapping the other's
 through CUDA IPC (tests/peers_worker.py).  The processes never wait on each
 other inside a kernel; gloo barriers order reads after writes.  Checks
-seq->head, head->seq, reduce-scatter and all-gather against the one-GPU
-definitions, bit for bit."""
+seq->head, head->seq, reduce-scatter, gated reduce-scatter and all-gather
+against the one-GPU definitions, bit for bit."""
 import json
 import os
 import socket

@@ -116,3 +116,33 @@ def test_rank_calls_serial_and_guard_bands(oracle_lib):
         rr.head_to_seq_rank(heads, mine, k, n_tokens=T)
         assert gu.guards_intact(buf)
         assert gu.same_bits(mine, send[k])
+
+
+@pytest.mark.parametrize("T,C,W,S", [(1000, 7168, 6, 8), (1024, 2048, 8, 3), (97, 1024, 2, 1),
+                                     (300, 256, 5, 40), (64, 64, 64, 64), (777, 512, 4, 256)])
+def test_gated_rank_shares(oracle_lib, T, C, W, S):
+    """Each rank's gated rows, in place on its residual, from the clipped and
+    rebased segments of its own token range."""
+    w = wl.ReduceWorkload("g", T=T, C=C, W=W, seed=T + S)
+    partials, bias = wl.partials_and_bias(w, DEV)
+    gate = wl.normal_bf16((S, C), S, 1.0, DEV)
+    bounds = wl.segment_bounds(T, S, S + 1)
+    part = rr.partition(T, W, W)
+    x_full = wl.normal_bf16((T, C), S + 2, 1.0, DEV)
+    x_bits = [gu.bits(v) for v in rr.split_rows(x_full, part.token_starts)]
+    xs = [v.clone() for v in rr.split_rows(x_full, part.token_starts)]
+    for k in range(W):
+        rr.ragged_reduce_scatter_gated_rank(list(partials.unbind(0)), bias, gate, bounds, xs[k], k,
+                                            n_tokens=T)
+    want = oracle_lib.reduce_scatter_gated([gu.bits(p) for p in partials.unbind(0)], gu.bits(bias),
+                                           gu.bits(gate), bounds, x_bits, W)
+    for k in range(W):
+        assert np.array_equal(gu.bits(xs[k]), want[k]), (T, C, W, S, k)
+    # out of place into a guarded buffer gives the same rows and writes nothing else
+    k = W - 1
+    buf, out = gu.guarded((part.tokens(k), C), DEV)
+    x_k = rr.split_rows(x_full, part.token_starts)[k]
+    rr.ragged_reduce_scatter_gated_rank(list(partials.unbind(0)), bias, gate, bounds, x_k, k,
+                                        n_tokens=T, out=out)
+    assert gu.guards_intact(buf)
+    assert np.array_equal(gu.bits(out), want[k])

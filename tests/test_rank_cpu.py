@@ -136,6 +136,67 @@ def test_rows_rank_argument_checks():
     assert rs(cfg=C.byref(_abi.LaunchConfig(E.H3_VARIANT_VECTOR, 0, 0, 0))) == E.H3_ERR_INVALID_ARG
 
 
+@needs_no_gpu
+def test_gated_rank_argument_checks():
+    T, Cc, W, S = 1000, 1024, 4, 3
+    addr = BASE
+    parts = []
+    for _ in range(W):
+        parts.append(addr)
+        addr += T * Cc * 2 + 4096
+    gate = addr
+    addr += S * Cc * 2 + 4096
+    x = addr
+    addr += T * Cc * 2 + 4096
+    bounds = np.array([0, 100, 700, T], dtype=np.int64)
+
+    def st(bounds=bounds, n=S, gate=gate, x=x, out=x, rank=1, bias=0):
+        info = _abi.ExecInfo()
+        s = _abi.lib.h3_ragged_reduce_scatter_gated_rank(
+            _abi.pointer_array(parts), C.c_void_p(bias), C.c_void_p(gate),
+            bounds.ctypes.data_as(C.POINTER(C.c_int64)), n, C.c_void_p(x), C.c_void_p(out), T, Cc,
+            W, rank, None, None, C.byref(info))
+        assert info.launches == 0
+        return s
+
+    assert st(n=0) == E.H3_ERR_INVALID_ARG
+    assert st(n=257) == E.H3_ERR_UNSUPPORTED
+    assert st(bounds=np.array([0, 100, 100, T], dtype=np.int64)) == E.H3_ERR_INVALID_ARG
+    assert st(bounds=np.array([1, 100, 700, T], dtype=np.int64)) == E.H3_ERR_INVALID_ARG
+    assert st(bounds=np.array([0, 100, 700, T - 1], dtype=np.int64)) == E.H3_ERR_INVALID_ARG
+    assert st(gate=gate + 8) == E.H3_ERR_MISALIGNED
+    assert st(x=x + 8, out=x + 8) == E.H3_ERR_MISALIGNED
+    assert st(out=gate) == E.H3_ERR_INVALID_ARG            # output over the gate rows
+    assert st(out=parts[1] + 4096) == E.H3_ERR_INVALID_ARG  # output inside a partial
+    assert st(out=x + 16) == E.H3_ERR_INVALID_ARG           # overlapping, not identical, residual
+    assert st(rank=W) == E.H3_ERR_INVALID_ARG
+    assert st(gate=0) == E.H3_ERR_INVALID_ARG
+
+
+@needs_no_gpu
+def test_gated_rank_checks_at_the_largest_world():
+    """W = 64 partials plus gate, residual and bias all reach the overlap
+    check (the largest input set a rank call examines)."""
+    T, Cc, W, S = 256, 64, 64, 64
+    addr = BASE
+    parts = []
+    for _ in range(W):
+        parts.append(addr)
+        addr += T * Cc * 2 + 4096
+    gate, bias = addr, addr + S * Cc * 2 + 4096
+    x = bias + Cc * 2 + 4096
+    bounds = np.arange(0, T + 1, T // S, dtype=np.int64)
+    for out, want in ((x + 16, E.H3_ERR_INVALID_ARG),      # overlaps the residual
+                      (bias, E.H3_ERR_INVALID_ARG),        # over the bias
+                      (parts[63] + 64, E.H3_ERR_INVALID_ARG)):
+        info = _abi.ExecInfo()
+        st = _abi.lib.h3_ragged_reduce_scatter_gated_rank(
+            _abi.pointer_array(parts), C.c_void_p(bias), C.c_void_p(gate),
+            bounds.ctypes.data_as(C.POINTER(C.c_int64)), S, C.c_void_p(x), C.c_void_p(out), T, Cc,
+            W, 63, None, None, C.byref(info))
+        assert st == want and info.launches == 0
+
+
 def test_ipc_null_and_bad_records():
     h = _abi.IpcHandle()
     ptr = C.c_void_p()
