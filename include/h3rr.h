@@ -408,6 +408,21 @@ H3RR_API h3_status h3_staged_plan(int64_t n_tokens, int32_t planes, int32_t n_he
  */
 H3RR_API h3_status h3_bulk_wait_timeouts(void* stream, uint32_t* count, int32_t reset);
 
+/*
+ * h3_bounded_wait_selftest - diagnostic with no counterpart on the pages:
+ * runs, in one tiny kernel, the bounded shared-memory-barrier wait the bulk
+ * kernels use, on a barrier that expects one arrival.  arrive_first = 0: no
+ * arrival ever comes, so the wait must give up after `polls` tries and
+ * *expired becomes 1; arrive_first = 1: the arrival completes the phase
+ * first and *expired becomes 0.  polls in [1, 2^24].  Synchronises `stream`.
+ * Shows that an expired wait returns control (and leaves the context usable)
+ * without faulting or trapping.  expired: host out-param (-1 until set).
+ * Errors: H3_ERR_INVALID_ARG on bad arguments, H3_ERR_CUDA on a failed
+ * launch or copy.
+ */
+H3RR_API h3_status h3_bounded_wait_selftest(uint32_t polls, int32_t arrive_first, void* stream,
+                                            int32_t* expired);
+
 /* ------------------------------------------------------------------------
  * One rank per GPU.  The calls above keep all W virtual ranks in one GPU's
  * memory.  With one rank per GPU (each process drives one GPU), rank k's share of

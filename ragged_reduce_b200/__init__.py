@@ -40,7 +40,7 @@ __all__ = [
     "H3_LAYOUT_HEAD_PLANE_MAJOR", "ragged_reduce_scatter_gated", "PreparedRelayout", "H3_LAUNCH_SERIAL",
     "PreparedReduceScatter", "prepare_seq_to_head", "prepare_head_to_seq",
     "seq_to_head_rank", "head_to_seq_rank", "ragged_reduce_scatter_rank", "ragged_all_gather_rank",
-    "ragged_reduce_scatter_gated_rank",
+    "ragged_reduce_scatter_gated_rank", "bounded_wait_selftest",
     "prepare_ragged_reduce_scatter",
 ]
 
@@ -378,6 +378,22 @@ def bulk_wait_timeouts(stream=None, reset: bool = False, device=None) -> int:
                                             1 if reset else 0)
     _abi.check(st, "h3_bulk_wait_timeouts")
     return int(count.value)
+
+
+def bounded_wait_selftest(polls: int, arrive_first: bool, *, stream=None, device=None) -> bool:
+    """Run the bulk kernels' bounded barrier wait on a barrier nothing (or one
+    arrival) completes (``h3_bounded_wait_selftest``); True if the wait
+    expired.  Synchronises the stream."""
+    dev = torch.device("cuda", torch.cuda.current_device()) if device is None else torch.device(device)
+    expired = C.c_int32(-1)
+    with torch.cuda.device(dev):
+        st = _abi.lib.h3_bounded_wait_selftest(int(polls), 1 if arrive_first else 0,
+                                               C.c_void_p(_stream_handle(stream, dev)),
+                                               C.byref(expired))
+    _abi.check(st, "h3_bounded_wait_selftest")
+    if expired.value not in (0, 1):
+        raise RuntimeError("bounded wait self-test did not report")
+    return bool(expired.value)
 
 
 def ragged_all_gather(blocks, out, *, stream=None, variant: int = 0, ctas_per_sm: int = 0,

@@ -176,6 +176,9 @@ def _load() -> C.CDLL:
     lib.h3_ragged_all_gather_rank.argtypes = [_vpp, C.c_void_p, C.c_int64, C.c_int64, C.c_int32,
                                               C.c_int32, C.c_void_p, C.POINTER(LaunchConfig),
                                               C.POINTER(ExecInfo)]
+    lib.h3_bounded_wait_selftest.restype = C.c_int
+    lib.h3_bounded_wait_selftest.argtypes = [C.c_uint32, C.c_int32, C.c_void_p,
+                                             C.POINTER(C.c_int32)]
     lib.h3_ipc_export.restype = C.c_int
     lib.h3_ipc_export.argtypes = [C.c_void_p, C.POINTER(IpcHandle)]
     lib.h3_ipc_open.restype = C.c_int

@@ -14,6 +14,7 @@
 // row allow it, else 16), loads all of them, then stores each to the W
 // outputs.  Non-coherent streaming loads (inputs never overlap outputs; the
 // host checks this), streaming stores.
+#include "bulk_copy.cuh"
 #include "h3rr_internal.h"
 
 namespace h3rr {
@@ -136,29 +137,6 @@ __global__ void __launch_bounds__(kGenericThreads) all_gather_generic_kernel(con
 constexpr int kBulkStages = 12;
 constexpr int kBulkLookahead = 8;
 constexpr int kBulkBarrierBytes = 128;
-constexpr uint32_t kBulkWaitLimit = 1u << 24;
-
-__device__ __forceinline__ uint32_t smem_addr(const void* p)
-{
-    return static_cast<uint32_t>(__cvta_generic_to_shared(p));
-}
-
-__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity)
-{
-    for (uint32_t it = 0; it < kBulkWaitLimit; ++it) {
-        uint32_t done;
-        asm volatile(
-            "{\n\t.reg .pred p;\n\t"
-            "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
-            "selp.u32 %0, 1, 0, p;\n\t}"
-            : "=r"(done)
-            : "r"(smem_addr(bar)), "r"(parity)
-            : "memory");
-        if (done)
-            return true;
-    }
-    return false;
-}
 
 template <int S, int L>
 __global__ void __launch_bounds__(32) all_gather_bulk_kernel(const __grid_constant__ GatherArgs a)
@@ -170,32 +148,26 @@ __global__ void __launch_bounds__(32) all_gather_bulk_kernel(const __grid_consta
     if (threadIdx.x != 0)
         return;
     const uint32_t row_bytes = uint32_t(a.row_bytes);
-    uint64_t pol;
-    asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(pol));
+    const uint64_t pol = evict_first_policy();
     for (int s = 0; s < S; ++s)
-        asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(smem_addr(&bars[s])) : "memory");
-    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+        mbar_init(&bars[s], 1);
+    mbar_fence_init();
     const int64_t n_rows = a.T > int32_t(blockIdx.x) ? (int64_t(a.T) - blockIdx.x + gridDim.x - 1) / gridDim.x : 0;
     auto issue_load = [&](int64_t n) {
         const int32_t t = int32_t(blockIdx.x + n * gridDim.x);
         const int32_t s = split_owner(t, a.tq, a.tm);
         const int32_t tl = t - split_start(s, a.tq, a.tm);
         uint64_t* bar = &bars[n % S];
-        asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_addr(bar)),
-                     "r"(row_bytes)
-                     : "memory");
-        asm volatile(
-            "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint "
-            "[%0], [%1], %2, [%3], %4;" ::"r"(smem_addr(ring + size_t(n % S) * row_bytes)),
-            "l"(a.in[s] + int64_t(tl) * row_bytes), "r"(row_bytes), "r"(smem_addr(bar)), "l"(pol)
-            : "memory");
+        mbar_arrive_expect_tx(bar, row_bytes);
+        bulk_load(ring + size_t(n % S) * row_bytes, a.in[s] + int64_t(tl) * row_bytes, row_bytes, bar,
+                  pol);
     };
     const int64_t prologue = n_rows < L ? n_rows : L;
     for (int64_t n = 0; n < prologue; ++n)
         issue_load(n);
     for (int64_t n = 0; n < n_rows; ++n) {
         if (n + L < n_rows) {
-            asm volatile("cp.async.bulk.wait_group.read %0;" ::"n"(S - L - 1) : "memory");
+            bulk_wait_read<S - L - 1>();
             issue_load(n + L);
         }
         if (!mbar_wait(&bars[n % S], uint32_t((n / S) & 1))) {
@@ -207,13 +179,10 @@ __global__ void __launch_bounds__(32) all_gather_bulk_kernel(const __grid_consta
         const int32_t t = int32_t(blockIdx.x + n * gridDim.x);
         const unsigned char* stage = ring + size_t(n % S) * row_bytes;
         for (int j = 0; j < a.W; ++j)
-            asm volatile("cp.async.bulk.global.shared::cta.bulk_group.L2::cache_hint [%0], [%1], %2, %3;" ::"l"(
-                             a.out[j] + int64_t(t) * row_bytes),
-                         "r"(smem_addr(stage)), "r"(row_bytes), "l"(pol)
-                         : "memory");
-        asm volatile("cp.async.bulk.commit_group;" ::: "memory");
+            bulk_store(a.out[j] + int64_t(t) * row_bytes, stage, row_bytes, pol);
+        bulk_commit();
     }
-    asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
+    bulk_wait_all();
 }
 
 struct GatherChoice {

@@ -29,6 +29,7 @@
 //   before its stores have read it.  No multicast is used.  Every mbarrier
 //   wait is bounded: on expiry the kernel counts the event in a device word
 //   (read with h3_bulk_wait_timeouts), drains what it issued and returns.
+#include "bulk_copy.cuh"
 #include "h3rr_internal.h"
 
 namespace h3rr {
@@ -225,76 +226,6 @@ __global__ void __launch_bounds__(kGenericThreads) relayout_generic_kernel(const
 constexpr int kBulkStages = 14;
 constexpr int kBulkLookahead = 11;
 constexpr int kBulkBarrierBytes = 128;          // room for 16 mbarriers
-constexpr uint32_t kBulkWaitLimit = 1u << 24;   // try_wait polls before giving up
-
-__device__ __forceinline__ uint32_t smem_addr(const void* p)
-{
-    return static_cast<uint32_t>(__cvta_generic_to_shared(p));
-}
-
-__device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count)
-{
-    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_addr(bar)), "r"(count) : "memory");
-}
-
-__device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t* bar, uint32_t bytes)
-{
-    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_addr(bar)),
-                 "r"(bytes)
-                 : "memory");
-}
-
-// Bounded wait for the phase with the given parity; false if it expired.
-__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity)
-{
-    for (uint32_t it = 0; it < kBulkWaitLimit; ++it) {
-        uint32_t done;
-        asm volatile(
-            "{\n\t.reg .pred p;\n\t"
-            "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
-            "selp.u32 %0, 1, 0, p;\n\t}"
-            : "=r"(done)
-            : "r"(smem_addr(bar)), "r"(parity)
-            : "memory");
-        if (done)
-            return true;
-    }
-    return false;
-}
-
-__device__ __forceinline__ uint64_t evict_first_policy()
-{
-    uint64_t pol;
-    asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(pol));
-    return pol;
-}
-
-__device__ __forceinline__ void bulk_load(void* smem_dst, const void* src, uint32_t bytes, uint64_t* bar,
-                                          uint64_t pol)
-{
-    asm volatile(
-        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint "
-        "[%0], [%1], %2, [%3], %4;" ::"r"(smem_addr(smem_dst)),
-        "l"(src), "r"(bytes), "r"(smem_addr(bar)), "l"(pol)
-        : "memory");
-}
-
-__device__ __forceinline__ void bulk_store(void* dst, const void* smem_src, uint32_t bytes, uint64_t pol)
-{
-    asm volatile("cp.async.bulk.global.shared::cta.bulk_group.L2::cache_hint [%0], [%1], %2, %3;" ::"l"(dst),
-                 "r"(smem_addr(smem_src)), "r"(bytes), "l"(pol)
-                 : "memory");
-}
-
-__device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
-
-template <int N>
-__device__ __forceinline__ void bulk_wait_read()
-{
-    asm volatile("cp.async.bulk.wait_group.read %0;" ::"n"(N) : "memory");
-}
-
-__device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
 
 template <bool kSeqToHead, int S, int L>
 __global__ void __launch_bounds__(32) relayout_bulk_kernel(const __grid_constant__ RelayoutArgs a)
@@ -310,7 +241,7 @@ __global__ void __launch_bounds__(32) relayout_bulk_kernel(const __grid_constant
     const uint64_t pol = evict_first_policy();
     for (int s = 0; s < S; ++s)
         mbar_init(&bars[s], 1);
-    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    mbar_fence_init();
 
     const int64_t n_rows =
         a.rows > int32_t(blockIdx.x) ? (int64_t(a.rows) - blockIdx.x + gridDim.x - 1) / gridDim.x : 0;

@@ -59,6 +59,28 @@ int main(void)
                                          H3RR_STATIC_WINDOW_BYTES + 16, NULL, &info) ==
            H3_ERR_UNSUPPORTED, "noalloc window beyond its array");
 
+    /* one rank per GPU: rank out of range, NULL output, misaligned columns */
+    {
+        h3_launch_config cfg;
+        h3_ipc_handle handle;
+        void* mapped = NULL;
+        void* fake_out = (void*)(uintptr_t)4096; /* never dereferenced: checks fail first */
+        memset(&cfg, 0, sizeof(cfg));
+        expect(h3_seq_to_head_rank(NULL, NULL, 1000, 3, 56, 128, 6, 0, 0, NULL, NULL, &info) ==
+                   H3_ERR_INVALID_ARG && info.launches == 0, "rank call, null arrays");
+        expect(h3_ragged_reduce_scatter_rank(null_ptrs, NULL, fake_out, 1000, 7168, 6, 6, NULL,
+                                             NULL, &info) == H3_ERR_INVALID_ARG, "rank out of range");
+        expect(h3_ragged_all_gather_rank(null_ptrs, fake_out, 1000, 7164, 6, 0, NULL, NULL, &info) ==
+               H3_ERR_MISALIGNED, "rank call, cols not a multiple of 8");
+        cfg.flags = H3_LAUNCH_SERIAL | 2;
+        expect(h3_ragged_all_gather_rank(null_ptrs, fake_out, 1000, 7168, 6, 0, NULL, &cfg, &info) ==
+               H3_ERR_INVALID_ARG, "unknown launch flag");
+        expect(sizeof(h3_ipc_handle) == 80, "ipc record size");
+        expect(h3_ipc_export(NULL, &handle) == H3_ERR_INVALID_ARG, "ipc export of NULL");
+        expect(h3_ipc_open(NULL, &mapped) == H3_ERR_INVALID_ARG && mapped == NULL, "ipc open of NULL");
+        expect(h3_ipc_close(NULL, &handle) == H3_ERR_INVALID_ARG, "ipc close of NULL");
+    }
+
     if (failures == 0)
         printf("c abi ok\n");
     return failures == 0 ? 0 : 1;

@@ -36,7 +36,7 @@ def main():
                             timeout=datetime.timedelta(seconds=120))
     dev = torch.device("cuda", 0)
     torch.cuda.set_device(dev)
-    T, P, H, D, C = 3000, 3, 56, 128, 2048
+    T, P, H, D, C = 3001, 3, 56, 128, 2048  # ragged over 2 and 3 ranks
     part = rr.partition(T, H, world)
     ts, te = int(part.token_starts[rank]), int(part.token_starts[rank + 1])
     hs, he = int(part.head_starts[rank]), int(part.head_starts[rank + 1])

@@ -1,5 +1,5 @@
-"""The one-rank-per-GPU path across processes: two ranks as two processes
-sharing one GPU, each holding only its own inputs and mapping the other's
+"""The one-rank-per-GPU path across processes: two or three ranks as
+processes sharing one GPU, each holding only its own inputs and mapping the other's
 through CUDA IPC (tests/peers_worker.py).  The processes never wait on each
 other inside a kernel; gloo barriers order reads after writes.  Checks
 seq->head, head->seq, reduce-scatter, gated reduce-scatter and all-gather
@@ -24,8 +24,8 @@ def _free_port():
         return s.getsockname()[1]
 
 
-def test_two_processes_pull_from_each_other():
-    world = 2
+@pytest.mark.parametrize("world", [2, 3])
+def test_processes_pull_from_each_other(world):
     port = _free_port()
     procs = []
     for rank in range(world):

@@ -197,6 +197,14 @@ def test_gated_rank_checks_at_the_largest_world():
         assert st == want and info.launches == 0
 
 
+def test_bounded_wait_selftest_argument_checks():
+    out = C.c_int32(7)
+    for polls, arrive in ((0, 0), ((1 << 24) + 1, 0), (16, 2), (16, -1)):
+        assert _abi.lib.h3_bounded_wait_selftest(polls, arrive, None, C.byref(out)) == E.H3_ERR_INVALID_ARG
+    assert out.value == 7  # untouched on an argument error
+    assert _abi.lib.h3_bounded_wait_selftest(16, 0, None, None) == E.H3_ERR_INVALID_ARG
+
+
 def test_ipc_null_and_bad_records():
     h = _abi.IpcHandle()
     ptr = C.c_void_p()
