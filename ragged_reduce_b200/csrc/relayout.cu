@@ -458,17 +458,20 @@ bool pick_vec(int need, KernelChoice* kc)
     return false;
 }
 
-// Vector kernel shapes measured fastest on B200 for H3 rows (14,336 bytes):
-// sequence->head with 32-byte vectors, 64 threads and two rows in flight;
-// head->sequence with 32-byte vectors and one warp per CTA.  Wider rows fall
-// back to 16-byte vectors with 128 threads, then to the generic kernel.
+// Vector kernel shapes measured fastest on B200 for H3 rows (14,336 bytes =
+// 448 vectors of 32 bytes) with one CTA per row unit: 128 threads, 32-byte
+// vectors, 4 per thread, two rows per CTA for sequence->head (120 registers)
+// and one for head->sequence (72 registers).  They beat 64 threads x 7 x 2
+// rows (seq->head) and one warp x 14 (head->seq) by 1-2 % on every workload;
+// those had won under persistent grids.  Rows wider than 16 KB fall back to
+// 16-byte vectors with 128 threads, then to the generic kernel.
 template <bool S2H, bool LAYOUT = false>
 void choose_vec(const RelayoutArgs& a, bool wide_ok, KernelChoice* kc)
 {
     if (wide_ok) {
         const int row32 = a.row_vecs / 2;
-        const bool ok = S2H ? pick_vec<true, 32, 64, 2, 8, LAYOUT>((row32 + 63) / 64, kc)
-                            : pick_vec<false, 32, 32, 1, 16, LAYOUT>((row32 + 31) / 32, kc);
+        const bool ok = S2H ? pick_vec<true, 32, 128, 2, 4, LAYOUT>((row32 + 127) / 128, kc)
+                            : pick_vec<false, 32, 128, 1, 4, LAYOUT>((row32 + 127) / 128, kc);
         if (ok)
             return;
     }
