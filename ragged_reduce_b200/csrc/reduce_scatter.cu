@@ -12,12 +12,14 @@
 // flush-to-zero, so the result is the same bit pattern the sequential CPU
 // definition gives.
 //
-// Layout of the work: a CTA of 128 threads takes one token row at a time;
-// each thread owns 16-byte column vectors tid, tid+128, ... of the row and,
-// for U of them at once, issues all W partial loads before the first add, so
-// U*W 16-byte loads per thread are in flight.  The row's owner rank is
-// computed once per row.  (128 threads with one vector per thread measured
-// fastest on B200 at W = 6 and 8.)
+// Layout of the work: one CTA per token row; each thread owns column vectors
+// tid, tid+NT, ... of the row and, for U of them at once, issues all W
+// partial loads before the first add, so U*W vector loads per thread are in
+// flight.  The row's owner rank is computed once per row.  With every row
+// and pointer 32-byte aligned (the H3 case, C = 7168) the kernel moves
+// 32-byte vectors (16 BF16 values), two per thread, 128 threads for W <= 6
+// and 64 for W = 7, 8: 5-7 % faster on B200 than 16-byte vectors.  Otherwise
+// 16-byte vectors with 128 threads; W > 8 loads the partials in batches of 8.
 #include <cuda_bf16.h>
 
 #include "h3rr_internal.h"
@@ -94,6 +96,107 @@ __device__ __forceinline__ uint4 narrow_rne(const float* acc)
     return make_uint4(w[0], w[1], w[2], w[3]);
 }
 
+// 32 bytes = 16 BF16 values.
+struct Vec32 {
+    uint32_t r[8];
+};
+
+__device__ __forceinline__ void ld_stream(Vec32& v, const char* p)
+{
+    asm volatile("ld.global.nc.L1::no_allocate.v8.u32 {%0, %1, %2, %3, %4, %5, %6, %7}, [%8];"
+                 : "=r"(v.r[0]), "=r"(v.r[1]), "=r"(v.r[2]), "=r"(v.r[3]), "=r"(v.r[4]),
+                   "=r"(v.r[5]), "=r"(v.r[6]), "=r"(v.r[7])
+                 : "l"(p));
+}
+
+__device__ __forceinline__ void ld_cached(Vec32& v, const char* p)
+{
+    asm volatile("ld.global.nc.v8.u32 {%0, %1, %2, %3, %4, %5, %6, %7}, [%8];"
+                 : "=r"(v.r[0]), "=r"(v.r[1]), "=r"(v.r[2]), "=r"(v.r[3]), "=r"(v.r[4]),
+                   "=r"(v.r[5]), "=r"(v.r[6]), "=r"(v.r[7])
+                 : "l"(p));
+}
+
+__device__ __forceinline__ void st_stream(char* p, const Vec32& v)
+{
+    asm volatile("st.global.cs.v8.u32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};" ::"l"(p),
+                 "r"(v.r[0]), "r"(v.r[1]), "r"(v.r[2]), "r"(v.r[3]), "r"(v.r[4]), "r"(v.r[5]),
+                 "r"(v.r[6]), "r"(v.r[7])
+                 : "memory");
+}
+
+// Exact widening of 16 BF16 values, and the rank-ordered binary32 add.
+__device__ __forceinline__ void widen(const Vec32& v, float* f)
+{
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+        f[2 * i] = __uint_as_float(v.r[i] << 16);
+        f[2 * i + 1] = __uint_as_float(v.r[i] & 0xFFFF0000u);
+    }
+}
+
+__device__ __forceinline__ void add_widened(const Vec32& v, float* acc)
+{
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+        acc[2 * i] = __fadd_rn(acc[2 * i], __uint_as_float(v.r[i] << 16));
+        acc[2 * i + 1] = __fadd_rn(acc[2 * i + 1], __uint_as_float(v.r[i] & 0xFFFF0000u));
+    }
+}
+
+__device__ __forceinline__ Vec32 narrow_rne16(const float* acc)
+{
+    Vec32 o;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+        const __nv_bfloat162 b = __floats2bfloat162_rn(acc[2 * i], acc[2 * i + 1]);
+        o.r[i] = *reinterpret_cast<const uint32_t*>(&b);
+    }
+    return o;
+}
+
+// 32-byte vectors, W fixed at compile time (1..8), U vectors per thread at
+// once: all U*W partial loads are issued before the first add.
+template <int kW, int U, int NT>
+__global__ void __launch_bounds__(NT) reduce_scatter_wide_kernel(const __grid_constant__ ReduceArgs a)
+{
+    const int32_t row_v = a.row_vecs / 2;  // 32-byte vectors per row
+    pdl_wait_prerequisites();
+    pdl_allow_dependents();
+    for (int64_t t64 = blockIdx.x; t64 < a.T; t64 += gridDim.x) {
+        const int32_t t = int32_t(t64);
+        const int32_t s = split_owner(t, a.tq, a.tm);
+        const int32_t tl = t - split_start(s, a.tq, a.tm);
+        const int64_t in_off = int64_t(t) * a.row_bytes;
+        char* orow = a.out[s] + int64_t(tl) * a.row_bytes;
+        for (int32_t c0 = threadIdx.x; c0 < row_v; c0 += NT * U) {
+            Vec32 x[U][kW];
+#pragma unroll
+            for (int u = 0; u < U; ++u)
+#pragma unroll
+                for (int b = 0; b < kW; ++b)
+                    if (c0 + u * NT < row_v)
+                        ld_stream(x[u][b], a.part[b] + in_off + int64_t(c0 + u * NT) * 32);
+#pragma unroll
+            for (int u = 0; u < U; ++u) {
+                if (c0 + u * NT >= row_v)
+                    continue;
+                float acc[16];
+                widen(x[u][0], acc);
+#pragma unroll
+                for (int b = 1; b < kW; ++b)
+                    add_widened(x[u][b], acc);
+                if (a.bias != nullptr) {
+                    Vec32 bv;
+                    ld_cached(bv, a.bias + int64_t(c0 + u * NT) * 32);
+                    add_widened(bv, acc);
+                }
+                st_stream(orow + int64_t(c0 + u * NT) * 32, narrow_rne16(acc));
+            }
+        }
+    }
+}
+
 // kW > 0: W fixed at compile time, all loads issued before the adds.
 // kW == 0: W from the arguments, loaded in batches of 8 ranks (still summed
 // strictly in rank order).
@@ -156,6 +259,34 @@ __global__ void __launch_bounds__(kThreads) reduce_scatter_kernel(const __grid_c
                     st_stream(orow + int64_t(c0 + u * kThreads) * kVecBytes, narrow_rne(acc[u]));
         }
     }
+}
+
+// The 32-byte kernel for W <= 8 (nullptr otherwise) and its block size.
+const void* pick_wide_reduce_kernel(int W, int* threads)
+{
+    *threads = W <= 6 ? 128 : 64;
+    switch (W) {
+        case 1: return (const void*)reduce_scatter_wide_kernel<1, 2, 128>;
+        case 2: return (const void*)reduce_scatter_wide_kernel<2, 2, 128>;
+        case 3: return (const void*)reduce_scatter_wide_kernel<3, 2, 128>;
+        case 4: return (const void*)reduce_scatter_wide_kernel<4, 2, 128>;
+        case 5: return (const void*)reduce_scatter_wide_kernel<5, 2, 128>;
+        case 6: return (const void*)reduce_scatter_wide_kernel<6, 2, 128>;
+        case 7: return (const void*)reduce_scatter_wide_kernel<7, 2, 64>;
+        case 8: return (const void*)reduce_scatter_wide_kernel<8, 2, 64>;
+        default: return nullptr;
+    }
+}
+
+// Every row start and buffer 32-byte aligned.
+bool wide_rows_ok(const ReduceArgs& a)
+{
+    if ((a.row_bytes % 32) != 0 || (reinterpret_cast<uintptr_t>(a.bias) & 31u))
+        return false;
+    for (int r = 0; r < a.W; ++r)
+        if ((reinterpret_cast<uintptr_t>(a.part[r]) & 31u) || (reinterpret_cast<uintptr_t>(a.out[r]) & 31u))
+            return false;
+    return true;
 }
 
 const void* pick_reduce_kernel(int W)
@@ -254,6 +385,94 @@ __global__ void __launch_bounds__(kThreads) reduce_scatter_gated_kernel(const __
     }
 }
 
+__device__ __forceinline__ void ld_plain(Vec32& v, const char* p)
+{
+    asm volatile("ld.global.v8.u32 {%0, %1, %2, %3, %4, %5, %6, %7}, [%8];"
+                 : "=r"(v.r[0]), "=r"(v.r[1]), "=r"(v.r[2]), "=r"(v.r[3]), "=r"(v.r[4]),
+                   "=r"(v.r[5]), "=r"(v.r[6]), "=r"(v.r[7])
+                 : "l"(p));
+}
+
+// The gated kernel with 32-byte vectors, U per thread at once (as
+// reduce_scatter_wide_kernel); same arithmetic per element.
+template <int kW, int U, int NT>
+__global__ void __launch_bounds__(NT) reduce_scatter_gated_wide_kernel(const __grid_constant__ GatedArgs g)
+{
+    const ReduceArgs& a = g.r;
+    const int32_t row_v = a.row_vecs / 2;
+    pdl_wait_prerequisites();
+    pdl_allow_dependents();
+    for (int64_t t64 = blockIdx.x; t64 < a.T; t64 += gridDim.x) {
+        const int32_t t = int32_t(t64);
+        const int32_t s = split_owner(t, a.tq, a.tm);
+        const int32_t tl = t - split_start(s, a.tq, a.tm);
+        int32_t lo = 0, hi = g.n_segs;  // largest k with bounds[k] <= t
+        while (hi - lo > 1) {
+            const int32_t mid = (lo + hi) >> 1;
+            if (g.seg_bounds[mid] <= t)
+                lo = mid;
+            else
+                hi = mid;
+        }
+        const char* grow = g.gate + int64_t(lo) * a.row_bytes;
+        const char* xrow = g.x[s] + int64_t(tl) * a.row_bytes;
+        char* orow = a.out[s] + int64_t(tl) * a.row_bytes;
+        const int64_t in_off = int64_t(t) * a.row_bytes;
+        for (int32_t c0 = threadIdx.x; c0 < row_v; c0 += NT * U) {
+            Vec32 x[U][kW];
+#pragma unroll
+            for (int u = 0; u < U; ++u)
+#pragma unroll
+                for (int b = 0; b < kW; ++b)
+                    if (c0 + u * NT < row_v)
+                        ld_stream(x[u][b], a.part[b] + in_off + int64_t(c0 + u * NT) * 32);
+#pragma unroll
+            for (int u = 0; u < U; ++u) {
+                if (c0 + u * NT >= row_v)
+                    continue;
+                const int64_t off = int64_t(c0 + u * NT) * 32;
+                float acc[16];
+                widen(x[u][0], acc);
+#pragma unroll
+                for (int b = 1; b < kW; ++b)
+                    add_widened(x[u][b], acc);
+                if (a.bias != nullptr) {
+                    Vec32 bv;
+                    ld_cached(bv, a.bias + off);
+                    add_widened(bv, acc);
+                }
+                float y[16], gt[16], xr[16];
+                widen(narrow_rne16(acc), y);  // the reduce-scatter output, as BF16
+                Vec32 gv, xv;
+                ld_cached(gv, grow + off);
+                ld_plain(xv, xrow + off);
+                widen(gv, gt);
+                widen(xv, xr);
+#pragma unroll
+                for (int e = 0; e < 16; ++e)
+                    acc[e] = __fadd_rn(xr[e], __fmul_rn(gt[e], y[e]));
+                st_stream(orow + off, narrow_rne16(acc));
+            }
+        }
+    }
+}
+
+const void* pick_wide_gated_kernel(int W, int* threads)
+{
+    *threads = W <= 6 ? 128 : 64;
+    switch (W) {
+        case 1: return (const void*)reduce_scatter_gated_wide_kernel<1, 2, 128>;
+        case 2: return (const void*)reduce_scatter_gated_wide_kernel<2, 2, 128>;
+        case 3: return (const void*)reduce_scatter_gated_wide_kernel<3, 2, 128>;
+        case 4: return (const void*)reduce_scatter_gated_wide_kernel<4, 2, 128>;
+        case 5: return (const void*)reduce_scatter_gated_wide_kernel<5, 2, 128>;
+        case 6: return (const void*)reduce_scatter_gated_wide_kernel<6, 2, 128>;
+        case 7: return (const void*)reduce_scatter_gated_wide_kernel<7, 2, 64>;
+        case 8: return (const void*)reduce_scatter_gated_wide_kernel<8, 2, 64>;
+        default: return nullptr;
+    }
+}
+
 const void* pick_gated_kernel(int W)
 {
     switch (W) {
@@ -275,6 +494,17 @@ cudaError_t launch_reduce_scatter_gated(const GatedArgs& a, cudaStream_t stream,
                                         bool programmatic)
 {
     const void* kernel = pick_gated_kernel(a.r.W);
+    int threads = kThreads;
+    bool wide = wide_rows_ok(a.r) && (reinterpret_cast<uintptr_t>(a.gate) & 31u) == 0;
+    for (int r = 0; wide && r < a.r.W; ++r)
+        wide = (reinterpret_cast<uintptr_t>(a.x[r]) & 31u) == 0;
+    if (wide) {
+        int wide_threads = 0;
+        if (const void* k = pick_wide_gated_kernel(a.r.W, &wide_threads)) {
+            kernel = k;
+            threads = wide_threads;
+        }
+    }
     int device = 0;
     const int sms = current_sm_count(&device);
     if (sms <= 0)
@@ -284,17 +514,25 @@ cudaError_t launch_reduce_scatter_gated(const GatedArgs& a, cudaStream_t stream,
         grid = 1;
     if (shape) {
         shape->grid = int(grid);
-        shape->block = kThreads;
+        shape->block = threads;
         shape->variant = H3_VARIANT_REDUCE_GATED;
     }
     void* params[] = {const_cast<GatedArgs*>(&a)};
-    return launch_kernel(kernel, grid, kThreads, 0, stream, params, programmatic);
+    return launch_kernel(kernel, grid, threads, 0, stream, params, programmatic);
 }
 
 cudaError_t launch_reduce_scatter(const ReduceArgs& a, int ctas_per_sm, cudaStream_t stream,
                                   LaunchShape* shape, bool programmatic)
 {
     const void* kernel = pick_reduce_kernel(a.W);
+    int threads = kThreads;
+    if (wide_rows_ok(a)) {
+        int wide_threads = 0;
+        if (const void* wide = pick_wide_reduce_kernel(a.W, &wide_threads)) {
+            kernel = wide;
+            threads = wide_threads;
+        }
+    }
     int device = 0;
     const int sms = current_sm_count(&device);
     if (sms <= 0)
@@ -310,11 +548,11 @@ cudaError_t launch_reduce_scatter(const ReduceArgs& a, int ctas_per_sm, cudaStre
         grid = 1;
     if (shape) {
         shape->grid = int(grid);
-        shape->block = kThreads;
+        shape->block = threads;
         shape->variant = H3_VARIANT_REDUCE;
     }
     void* params[] = {const_cast<ReduceArgs*>(&a)};
-    return launch_kernel(kernel, grid, kThreads, 0, stream, params, programmatic);
+    return launch_kernel(kernel, grid, threads, 0, stream, params, programmatic);
 }
 
 }  // namespace h3rr
