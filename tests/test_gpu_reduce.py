@@ -137,3 +137,30 @@ def test_prepared_reduce_scatter(oracle_lib):
                                                 gu.bits(bias), W)
         for r in range(W):
             assert np.array_equal(gu.bits(out[r]), want[r])
+
+
+@pytest.mark.parametrize("W", range(1, 9))
+@pytest.mark.parametrize("C", [1024, 1040])
+def test_every_compiled_width_matches_oracle(oracle_lib, W, C):
+    """Both vector widths for every compile-time W: C = 1024 gives 32-byte
+    aligned rows (the 32-byte kernels), C = 1040 rows of 2,080 bytes (the
+    16-byte kernels); plain and gated reduce-scatter."""
+    T = 257 + W
+    w = wl.ReduceWorkload("w", T=T, C=C, W=W, seed=W * 31 + C)
+    partials, bias = wl.partials_and_bias(w, DEV)
+    out_full, out, info = _run(partials, bias, T, C, W)
+    want = oracle_lib.ragged_reduce_scatter([gu.bits(p) for p in partials], gu.bits(bias), W)
+    for r in range(W):
+        assert np.array_equal(gu.bits(out[r]), want[r]), (W, C, r)
+    S = 3
+    gate = wl.normal_bf16((S, C), W + 5, 1.0, DEV)
+    bounds = wl.segment_bounds(T, S, W)
+    x_full = wl.normal_bf16((T, C), W + 6, 1.0, DEV)
+    part = rr.partition(T, W, W)
+    x = [v.clone() for v in rr.split_rows(x_full, part.token_starts)]
+    rr.ragged_reduce_scatter_gated(partials, bias, gate, bounds, x)
+    want_g = oracle_lib.reduce_scatter_gated([gu.bits(p) for p in partials], gu.bits(bias),
+                                             gu.bits(gate), bounds,
+                                             [gu.bits(v) for v in rr.split_rows(x_full, part.token_starts)], W)
+    for r in range(W):
+        assert np.array_equal(gu.bits(x[r]), want_g[r]), (W, C, r)
