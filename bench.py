@@ -456,7 +456,40 @@ def oracle_seconds_per_token() -> float:
     return (time.perf_counter() - t0) / 256
 
 
-def cpu_baseline(budget_s: float = 12.0) -> dict:
+def host_cores() -> int:
+    try:
+        return len(os.sched_getaffinity(0))
+    except AttributeError:
+        return os.cpu_count() or 1
+
+
+def oracle_all_cores(seconds: float, sample_tokens: int) -> dict:
+    """The unchanged oracle on every host core at once: one thread per core,
+    each running the step on its own token sample for `seconds` (the C oracle
+    runs without the GIL, so the threads use separate cores)."""
+    from concurrent.futures import ThreadPoolExecutor
+    cores = host_cores()
+    tokens = max(STEP_W, min(1024, sample_tokens // cores))
+    steps = [OracleStep(tokens) for _ in range(cores)]
+    deadline = time.perf_counter() + seconds
+
+    def work(s):
+        n = 0
+        while time.perf_counter() < deadline or n == 0:
+            s.run()
+            n += 1
+        return n * s.bytes
+
+    t0 = time.perf_counter()
+    with ThreadPoolExecutor(max_workers=cores) as pool:
+        total = sum(pool.map(work, steps))
+    t = time.perf_counter() - t0
+    return {"value": round(total / t / 1e9, 3), "unit": UNIT, "cores": cores, "kind": "oracle",
+            "sample": f"{cores} threads, each the step on {tokens} tokens repeatedly for "
+                      f"{t:.1f} s, C oracle unchanged"}
+
+
+def cpu_baseline(budget_s: float = 12.0, all_cores_s: float = 4.0) -> dict:
     per_tok = oracle_seconds_per_token()
     tokens = int(min(STEP_T, max(STEP_W, budget_s / 2 / per_tok)))
     s = OracleStep(tokens)
@@ -466,9 +499,14 @@ def cpu_baseline(budget_s: float = 12.0) -> dict:
         s.run()
         times.append(time.perf_counter() - t0)
     t = min(times)
-    return {"value": round(s.bytes / t / 1e9, 3), "unit": UNIT, "cores": 1, "kind": "oracle",
-            "sample": f"the step on {tokens} of {STEP_T} tokens (W={STEP_W}, same shapes otherwise), "
-                      f"best of 2, {t:.2f} s each, single-threaded C oracle"}
+    nbytes = s.bytes
+    del s  # free the sample before the all-cores run allocates its own
+    out = {"value": round(nbytes / t / 1e9, 3), "unit": UNIT, "cores": 1, "kind": "oracle",
+           "sample": f"the step on {tokens} of {STEP_T} tokens (W={STEP_W}, same shapes otherwise), "
+                     f"best of 2, {t:.2f} s each, single-threaded C oracle"}
+    if all_cores_s > 0 and host_cores() > 1:
+        out["all_cores"] = oracle_all_cores(all_cores_s, tokens)
+    return out
 
 
 def run_reference(args):
