@@ -34,7 +34,9 @@
  *     token offsets ts_r; head-side buffers may be views into one tensor.
  *   - Pointer arrays (send[], recv[], partials[], out[]) are HOST arrays of
  *     `world` DEVICE pointers; they are read during the call only.  The
- *     library allocates no device memory and keeps no pointer after return.
+ *     library allocates no device memory (one file-scope 16 MiB window, see
+ *     h3_seq_to_head_staged_noalloc, aside) and keeps no caller pointer after
+ *     return.
  *   - The caller owns every buffer.  Outputs must not overlap any input or
  *     any other output (outputs keep storage of their own); overlap is
  *     detected and rejected.
@@ -47,8 +49,11 @@
  *     nothing is launched and the returned status says why.
  *   - `info` (nullable) receives what actually ran: launches, chunks, grid,
  *     block and kernel variant.
- *   - Stateless and thread-safe: no environment variables are read and no
- *     state outlives a call, apart from a per-device cache of the SM count.
+ *   - Thread-safe, and no environment variables are read.  State kept across
+ *     calls: per-device caches (SM count, resident CTAs per kernel, the
+ *     shared-memory opt-in, the static window's address), each thread's last
+ *     CUDA error, the device-side counters of expired bounded waits, and the
+ *     peer mappings h3_ipc_open holds until h3_ipc_close.
  */
 #ifndef H3RR_H
 #define H3RR_H
@@ -80,9 +85,9 @@ typedef enum h3_status {
 
 /* Kernel variants reported in h3_exec_info.variant. */
 #define H3_VARIANT_NONE 0
-#define H3_VARIANT_VECTOR 1      /* 16-byte vector loads/stores through registers */
+#define H3_VARIANT_VECTOR 1      /* 16- or 32-byte vector loads/stores through registers */
 #define H3_VARIANT_BULK 2        /* bulk async copies through shared memory */
-#define H3_VARIANT_REDUCE 3      /* warp-level fp32 reduce-scatter */
+#define H3_VARIANT_REDUCE 3      /* binary32 reduce-scatter through registers */
 #define H3_VARIANT_STAGED 4      /* pack into a window buffer, then unpack */
 #define H3_VARIANT_GATHER 5      /* ragged all-gather */
 #define H3_VARIANT_REDUCE_GATED 6 /* reduce-scatter fused with residual gating */
