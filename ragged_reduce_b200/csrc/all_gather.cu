@@ -15,6 +15,7 @@
 // outputs.  Non-coherent streaming loads (inputs never overlap outputs; the
 // host checks this), streaming stores.
 #include "bulk_copy.cuh"
+#include "device_access.cuh"
 #include "h3rr_internal.h"
 
 namespace h3rr {
@@ -23,52 +24,6 @@ namespace h3rr {
 __device__ unsigned int g_gather_wait_timeouts = 0;
 
 namespace {
-
-template <int VW>
-struct Vec {
-    uint32_t r[VW / 4];
-};
-
-__device__ __forceinline__ void ld_stream(Vec<16>& v, const char* p)
-{
-    asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0, %1, %2, %3}, [%4];"
-                 : "=r"(v.r[0]), "=r"(v.r[1]), "=r"(v.r[2]), "=r"(v.r[3])
-                 : "l"(p));
-}
-
-__device__ __forceinline__ void ld_stream(Vec<32>& v, const char* p)
-{
-    asm volatile("ld.global.nc.L1::no_allocate.v8.u32 {%0, %1, %2, %3, %4, %5, %6, %7}, [%8];"
-                 : "=r"(v.r[0]), "=r"(v.r[1]), "=r"(v.r[2]), "=r"(v.r[3]), "=r"(v.r[4]),
-                   "=r"(v.r[5]), "=r"(v.r[6]), "=r"(v.r[7])
-                 : "l"(p));
-}
-
-__device__ __forceinline__ void st_stream(char* p, const Vec<16>& v)
-{
-    asm volatile("st.global.cs.v4.u32 [%0], {%1, %2, %3, %4};" ::"l"(p), "r"(v.r[0]), "r"(v.r[1]),
-                 "r"(v.r[2]), "r"(v.r[3])
-                 : "memory");
-}
-
-__device__ __forceinline__ void st_stream(char* p, const Vec<32>& v)
-{
-    asm volatile("st.global.cs.v8.u32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};" ::"l"(p),
-                 "r"(v.r[0]), "r"(v.r[1]), "r"(v.r[2]), "r"(v.r[3]), "r"(v.r[4]), "r"(v.r[5]),
-                 "r"(v.r[6]), "r"(v.r[7])
-                 : "memory");
-}
-
-__device__ __forceinline__ int32_t split_owner(int32_t x, int32_t q, int32_t m)
-{
-    const int32_t big = m * (q + 1);
-    return x < big ? x / (q + 1) : m + (x - big) / q;
-}
-
-__device__ __forceinline__ int32_t split_start(int32_t i, int32_t q, int32_t m)
-{
-    return i * q + (i < m ? i : m);
-}
 
 template <int VW, int NT, int VPT>
 __global__ void __launch_bounds__(NT) all_gather_vec_kernel(const __grid_constant__ GatherArgs a)

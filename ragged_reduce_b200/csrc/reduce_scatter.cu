@@ -22,6 +22,7 @@
 // 16-byte vectors with 128 threads; W > 8 loads the partials in batches of 8.
 #include <cuda_bf16.h>
 
+#include "device_access.cuh"
 #include "h3rr_internal.h"
 
 namespace h3rr {
@@ -29,126 +30,35 @@ namespace {
 
 constexpr int kThreads = 128;
 
-__device__ __forceinline__ uint4 ld_stream(const char* p)
-{
-    uint4 v;
-    asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0, %1, %2, %3}, [%4];"
-                 : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
-                 : "l"(p));
-    return v;
-}
-
-__device__ __forceinline__ uint4 ld_cached(const char* p)
-{
-    uint4 v;
-    asm volatile("ld.global.nc.v4.u32 {%0, %1, %2, %3}, [%4];"
-                 : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
-                 : "l"(p));
-    return v;
-}
-
-__device__ __forceinline__ void st_stream(char* p, const uint4& v)
-{
-    asm volatile("st.global.cs.v4.u32 [%0], {%1, %2, %3, %4};" ::"l"(p), "r"(v.x), "r"(v.y),
-                 "r"(v.z), "r"(v.w)
-                 : "memory");
-}
-
-__device__ __forceinline__ int32_t split_owner(int32_t x, int32_t q, int32_t m)
-{
-    const int32_t big = m * (q + 1);
-    return x < big ? x / (q + 1) : m + (x - big) / q;
-}
-
-__device__ __forceinline__ int32_t split_start(int32_t i, int32_t q, int32_t m)
-{
-    return i * q + (i < m ? i : m);
-}
-
-// BF16 -> binary32 is exact: the 16 bits become the top half of the word.
-__device__ __forceinline__ void widen(const uint4& v, float* f)
-{
-    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-        f[2 * i] = __uint_as_float(w[i] << 16);
-        f[2 * i + 1] = __uint_as_float(w[i] & 0xFFFF0000u);
-    }
-}
-
-__device__ __forceinline__ void add_widened(const uint4& v, float* acc)
-{
-    float f[8];
-    widen(v, f);
-#pragma unroll
-    for (int e = 0; e < 8; ++e)
-        acc[e] = __fadd_rn(acc[e], f[e]);
-}
-
-__device__ __forceinline__ uint4 narrow_rne(const float* acc)
-{
-    uint32_t w[4];
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-        const __nv_bfloat162 b = __floats2bfloat162_rn(acc[2 * i], acc[2 * i + 1]);
-        w[i] = *reinterpret_cast<const uint32_t*>(&b);
-    }
-    return make_uint4(w[0], w[1], w[2], w[3]);
-}
-
-// 32 bytes = 16 BF16 values.
-struct Vec32 {
-    uint32_t r[8];
-};
-
-__device__ __forceinline__ void ld_stream(Vec32& v, const char* p)
-{
-    asm volatile("ld.global.nc.L1::no_allocate.v8.u32 {%0, %1, %2, %3, %4, %5, %6, %7}, [%8];"
-                 : "=r"(v.r[0]), "=r"(v.r[1]), "=r"(v.r[2]), "=r"(v.r[3]), "=r"(v.r[4]),
-                   "=r"(v.r[5]), "=r"(v.r[6]), "=r"(v.r[7])
-                 : "l"(p));
-}
-
-__device__ __forceinline__ void ld_cached(Vec32& v, const char* p)
-{
-    asm volatile("ld.global.nc.v8.u32 {%0, %1, %2, %3, %4, %5, %6, %7}, [%8];"
-                 : "=r"(v.r[0]), "=r"(v.r[1]), "=r"(v.r[2]), "=r"(v.r[3]), "=r"(v.r[4]),
-                   "=r"(v.r[5]), "=r"(v.r[6]), "=r"(v.r[7])
-                 : "l"(p));
-}
-
-__device__ __forceinline__ void st_stream(char* p, const Vec32& v)
-{
-    asm volatile("st.global.cs.v8.u32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};" ::"l"(p),
-                 "r"(v.r[0]), "r"(v.r[1]), "r"(v.r[2]), "r"(v.r[3]), "r"(v.r[4]), "r"(v.r[5]),
-                 "r"(v.r[6]), "r"(v.r[7])
-                 : "memory");
-}
-
-// Exact widening of 16 BF16 values, and the rank-ordered binary32 add.
-__device__ __forceinline__ void widen(const Vec32& v, float* f)
+// Exact widening of a vector of BF16 values to binary32 (the 16 bits become
+// the top half of the word), the rank-ordered binary32 add, and rounding
+// back to BF16 to nearest even.
+template <int VW>
+__device__ __forceinline__ void widen(const Vec<VW>& v, float* f)
 {
 #pragma unroll
-    for (int i = 0; i < 8; ++i) {
+    for (int i = 0; i < VW / 4; ++i) {
         f[2 * i] = __uint_as_float(v.r[i] << 16);
         f[2 * i + 1] = __uint_as_float(v.r[i] & 0xFFFF0000u);
     }
 }
 
-__device__ __forceinline__ void add_widened(const Vec32& v, float* acc)
+template <int VW>
+__device__ __forceinline__ void add_widened(const Vec<VW>& v, float* acc)
 {
 #pragma unroll
-    for (int i = 0; i < 8; ++i) {
+    for (int i = 0; i < VW / 4; ++i) {
         acc[2 * i] = __fadd_rn(acc[2 * i], __uint_as_float(v.r[i] << 16));
         acc[2 * i + 1] = __fadd_rn(acc[2 * i + 1], __uint_as_float(v.r[i] & 0xFFFF0000u));
     }
 }
 
-__device__ __forceinline__ Vec32 narrow_rne16(const float* acc)
+template <int VW>
+__device__ __forceinline__ Vec<VW> narrow_rne(const float* acc)
 {
-    Vec32 o;
+    Vec<VW> o;
 #pragma unroll
-    for (int i = 0; i < 8; ++i) {
+    for (int i = 0; i < VW / 4; ++i) {
         const __nv_bfloat162 b = __floats2bfloat162_rn(acc[2 * i], acc[2 * i + 1]);
         o.r[i] = *reinterpret_cast<const uint32_t*>(&b);
     }
@@ -170,7 +80,7 @@ __global__ void __launch_bounds__(NT) reduce_scatter_wide_kernel(const __grid_co
         const int64_t in_off = int64_t(t) * a.row_bytes;
         char* orow = a.out[s] + int64_t(tl) * a.row_bytes;
         for (int32_t c0 = threadIdx.x; c0 < row_v; c0 += NT * U) {
-            Vec32 x[U][kW];
+            Vec<32> x[U][kW];
 #pragma unroll
             for (int u = 0; u < U; ++u)
 #pragma unroll
@@ -187,11 +97,11 @@ __global__ void __launch_bounds__(NT) reduce_scatter_wide_kernel(const __grid_co
                 for (int b = 1; b < kW; ++b)
                     add_widened(x[u][b], acc);
                 if (a.bias != nullptr) {
-                    Vec32 bv;
+                    Vec<32> bv;
                     ld_cached(bv, a.bias + int64_t(c0 + u * NT) * 32);
                     add_widened(bv, acc);
                 }
-                st_stream(orow + int64_t(c0 + u * NT) * 32, narrow_rne16(acc));
+                st_stream(orow + int64_t(c0 + u * NT) * 32, narrow_rne<32>(acc));
             }
         }
     }
@@ -222,14 +132,14 @@ __global__ void __launch_bounds__(kThreads) reduce_scatter_kernel(const __grid_c
                 live[u] = c0 + u * kThreads < a.row_vecs;
             const int W = kW > 0 ? kW : a.W;
             for (int w0 = 0; w0 < W; w0 += kBatch) {
-                uint4 x[U][kBatch];
+                Vec<16> x[U][kBatch];
 #pragma unroll
                 for (int u = 0; u < U; ++u) {
                     const int64_t off = in_off + int64_t(c0 + u * kThreads) * kVecBytes;
 #pragma unroll
                     for (int b = 0; b < kBatch; ++b)
                         if (live[u] && w0 + b < W)
-                            x[u][b] = ld_stream(a.part[w0 + b] + off);
+                            ld_stream(x[u][b], a.part[w0 + b] + off);
                 }
 #pragma unroll
                 for (int u = 0; u < U; ++u) {
@@ -248,15 +158,18 @@ __global__ void __launch_bounds__(kThreads) reduce_scatter_kernel(const __grid_c
             }
             if (a.bias != nullptr) {
 #pragma unroll
-                for (int u = 0; u < U; ++u)
-                    if (live[u])
-                        add_widened(ld_cached(a.bias + int64_t(c0 + u * kThreads) * kVecBytes),
-                                    acc[u]);
+                for (int u = 0; u < U; ++u) {
+                    if (live[u]) {
+                        Vec<16> bv;
+                        ld_cached(bv, a.bias + int64_t(c0 + u * kThreads) * kVecBytes);
+                        add_widened(bv, acc[u]);
+                    }
+                }
             }
 #pragma unroll
             for (int u = 0; u < U; ++u)
                 if (live[u])
-                    st_stream(orow + int64_t(c0 + u * kThreads) * kVecBytes, narrow_rne(acc[u]));
+                    st_stream(orow + int64_t(c0 + u * kThreads) * kVecBytes, narrow_rne<16>(acc[u]));
         }
     }
 }
@@ -317,15 +230,6 @@ const void* pick_reduce_kernel(int W)
 // x may be the output buffer itself (in place): each element is read by the
 // thread that then writes it, with plain (coherent) loads.
 // ---------------------------------------------------------------------------
-__device__ __forceinline__ uint4 ld_plain(const char* p)
-{
-    uint4 v;
-    asm volatile("ld.global.v4.u32 {%0, %1, %2, %3}, [%4];"
-                 : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
-                 : "l"(p));
-    return v;
-}
-
 template <int kW>
 __global__ void __launch_bounds__(kThreads) reduce_scatter_gated_kernel(const __grid_constant__ GatedArgs g)
 {
@@ -356,11 +260,11 @@ __global__ void __launch_bounds__(kThreads) reduce_scatter_gated_kernel(const __
             float acc[8];
             const int W = kW > 0 ? kW : a.W;
             for (int w0 = 0; w0 < W; w0 += kBatch) {
-                uint4 xv[kBatch];
+                Vec<16> xv[kBatch];
 #pragma unroll
                 for (int b = 0; b < kBatch; ++b)
                     if (w0 + b < W)
-                        xv[b] = ld_stream(a.part[w0 + b] + in_off + off);
+                        ld_stream(xv[b], a.part[w0 + b] + in_off + off);
 #pragma unroll
                 for (int b = 0; b < kBatch; ++b) {
                     if (w0 + b >= W)
@@ -371,26 +275,24 @@ __global__ void __launch_bounds__(kThreads) reduce_scatter_gated_kernel(const __
                         add_widened(xv[b], acc);
                 }
             }
-            if (a.bias != nullptr)
-                add_widened(ld_cached(a.bias + off), acc);
+            if (a.bias != nullptr) {
+                Vec<16> bv;
+                ld_cached(bv, a.bias + off);
+                add_widened(bv, acc);
+            }
             float y[8], gt[8], xr[8];
-            widen(narrow_rne(acc), y);          // the reduce-scatter output, as BF16
-            widen(ld_cached(grow + off), gt);
-            widen(ld_plain(xrow + off), xr);
+            widen(narrow_rne<16>(acc), y);  // the reduce-scatter output, as BF16
+            Vec<16> gv, xv2;
+            ld_cached(gv, grow + off);
+            ld_plain(xv2, xrow + off);
+            widen(gv, gt);
+            widen(xv2, xr);
 #pragma unroll
             for (int e = 0; e < 8; ++e)
                 acc[e] = __fadd_rn(xr[e], __fmul_rn(gt[e], y[e]));
-            st_stream(orow + off, narrow_rne(acc));
+            st_stream(orow + off, narrow_rne<16>(acc));
         }
     }
-}
-
-__device__ __forceinline__ void ld_plain(Vec32& v, const char* p)
-{
-    asm volatile("ld.global.v8.u32 {%0, %1, %2, %3, %4, %5, %6, %7}, [%8];"
-                 : "=r"(v.r[0]), "=r"(v.r[1]), "=r"(v.r[2]), "=r"(v.r[3]), "=r"(v.r[4]),
-                   "=r"(v.r[5]), "=r"(v.r[6]), "=r"(v.r[7])
-                 : "l"(p));
 }
 
 // The gated kernel with 32-byte vectors, U per thread at once (as
@@ -419,7 +321,7 @@ __global__ void __launch_bounds__(NT) reduce_scatter_gated_wide_kernel(const __g
         char* orow = a.out[s] + int64_t(tl) * a.row_bytes;
         const int64_t in_off = int64_t(t) * a.row_bytes;
         for (int32_t c0 = threadIdx.x; c0 < row_v; c0 += NT * U) {
-            Vec32 x[U][kW];
+            Vec<32> x[U][kW];
 #pragma unroll
             for (int u = 0; u < U; ++u)
 #pragma unroll
@@ -437,13 +339,13 @@ __global__ void __launch_bounds__(NT) reduce_scatter_gated_wide_kernel(const __g
                 for (int b = 1; b < kW; ++b)
                     add_widened(x[u][b], acc);
                 if (a.bias != nullptr) {
-                    Vec32 bv;
+                    Vec<32> bv;
                     ld_cached(bv, a.bias + off);
                     add_widened(bv, acc);
                 }
                 float y[16], gt[16], xr[16];
-                widen(narrow_rne16(acc), y);  // the reduce-scatter output, as BF16
-                Vec32 gv, xv;
+                widen(narrow_rne<32>(acc), y);  // the reduce-scatter output, as BF16
+                Vec<32> gv, xv;
                 ld_cached(gv, grow + off);
                 ld_plain(xv, xrow + off);
                 widen(gv, gt);
@@ -451,7 +353,7 @@ __global__ void __launch_bounds__(NT) reduce_scatter_gated_wide_kernel(const __g
 #pragma unroll
                 for (int e = 0; e < 16; ++e)
                     acc[e] = __fadd_rn(xr[e], __fmul_rn(gt[e], y[e]));
-                st_stream(orow + off, narrow_rne16(acc));
+                st_stream(orow + off, narrow_rne<32>(acc));
             }
         }
     }

@@ -21,6 +21,7 @@
 //                                  (a strided copy per rank)
 // seq->head = staged_row<true> then window_block<true>;
 // head->seq = window_block<false> then staged_row<false>.
+#include "device_access.cuh"
 #include "h3rr_internal.h"
 
 namespace h3rr {
@@ -28,44 +29,6 @@ namespace {
 
 constexpr int kThreads = 128;
 constexpr int64_t kMaxGrid = (int64_t(1) << 31) - 1;
-
-__device__ __forceinline__ uint4 ld_stream(const char* p)
-{
-    uint4 v;
-    asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0, %1, %2, %3}, [%4];"
-                 : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
-                 : "l"(p));
-    return v;
-}
-
-// The window is written and read back within one call; plain loads for it
-// (it is not read-only for the duration of the call).
-__device__ __forceinline__ uint4 ld_plain(const char* p)
-{
-    uint4 v;
-    asm volatile("ld.global.v4.u32 {%0, %1, %2, %3}, [%4];"
-                 : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
-                 : "l"(p));
-    return v;
-}
-
-__device__ __forceinline__ void st_plain(char* p, const uint4& v)
-{
-    asm volatile("st.global.v4.u32 [%0], {%1, %2, %3, %4};" ::"l"(p), "r"(v.x), "r"(v.y), "r"(v.z),
-                 "r"(v.w)
-                 : "memory");
-}
-
-__device__ __forceinline__ int32_t split_owner(int32_t x, int32_t q, int32_t m)
-{
-    const int32_t big = m * (q + 1);
-    return x < big ? x / (q + 1) : m + (x - big) / q;
-}
-
-__device__ __forceinline__ int32_t split_start(int32_t i, int32_t q, int32_t m)
-{
-    return i * q + (i < m ? i : m);
-}
 
 // Sequence-side rows t0..t0+n-1 of plane p <-> the chunk's window blocks.
 template <bool kToWindow>
@@ -87,10 +50,15 @@ __global__ void __launch_bounds__(kThreads) staged_row_kernel(const __grid_const
             char* wp = a.window +
                        ((int64_t(a.n) * hs + i * hj + (h - hs)) * a.head_vecs + within) * kVecBytes;
             char* sp = srow + int64_t(c) * kVecBytes;
-            if (kToWindow)
-                st_plain(wp, ld_stream(sp));
-            else
-                st_plain(sp, ld_plain(wp));
+            Vec<16> v;
+            if (kToWindow) {
+                ld_stream(v, sp);
+                st_plain(wp, v);
+            } else {
+                // The window is written and read back within one call: coherent loads.
+                ld_plain(v, wp);
+                st_plain(sp, v);
+            }
         }
     }
 }
@@ -109,10 +77,14 @@ __global__ void __launch_bounds__(kThreads) window_block_kernel(const __grid_con
         char* wrow = a.window + (int64_t(a.n) * hs + i * hj) * a.head_vecs * kVecBytes;
         char* hrow = a.head[j] + ((int64_t(a.t0) + i) * a.P + a.p) * run_vecs * kVecBytes;
         for (int32_t c = threadIdx.x; c < run_vecs; c += kThreads) {
-            if (kToHead)
-                st_plain(hrow + int64_t(c) * kVecBytes, ld_plain(wrow + int64_t(c) * kVecBytes));
-            else
-                st_plain(wrow + int64_t(c) * kVecBytes, ld_stream(hrow + int64_t(c) * kVecBytes));
+            Vec<16> v;
+            if (kToHead) {
+                ld_plain(v, wrow + int64_t(c) * kVecBytes);
+                st_plain(hrow + int64_t(c) * kVecBytes, v);
+            } else {
+                ld_stream(v, hrow + int64_t(c) * kVecBytes);
+                st_plain(wrow + int64_t(c) * kVecBytes, v);
+            }
         }
     }
 }
