@@ -93,9 +93,19 @@ def load_peak():
         return FALLBACK_HBM_GBS, "fallback"
 
 
-def kernel_source_digest() -> str:
+# The sources each measured kernel is compiled from.
+KERNEL_SOURCES = {
+    "seq_to_head": ("relayout.cu", "device_access.cuh", "bulk_copy.cuh", "h3rr_internal.h"),
+    "head_to_seq": ("relayout.cu", "device_access.cuh", "bulk_copy.cuh", "h3rr_internal.h"),
+    "ragged_reduce_scatter": ("reduce_scatter.cu", "device_access.cuh", "h3rr_internal.h"),
+}
+
+
+def kernel_source_digest(kernel: str) -> str:
+    """Digest of the sources `kernel` is compiled from: traffic figures taken
+    with other sources are not reported."""
     h = hashlib.sha256()
-    for name in ("relayout.cu", "reduce_scatter.cu"):
+    for name in KERNEL_SOURCES[kernel]:
         with open(os.path.join(ROOT, "ragged_reduce_b200", "csrc", name), "rb") as f:
             h.update(f.read())
     return h.hexdigest()[:16]
@@ -110,7 +120,7 @@ def load_traffic(kernel: str):
     except (OSError, ValueError):
         return None
     entry = table.get(kernel)
-    if not entry or entry.get("source_digest") != kernel_source_digest():
+    if not entry or kernel not in KERNEL_SOURCES or entry.get("source_digest") != kernel_source_digest(kernel):
         return None
     return entry.get("bytes_per_launch")
 

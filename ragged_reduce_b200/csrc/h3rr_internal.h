@@ -231,6 +231,16 @@ __device__ __forceinline__ void pdl_allow_dependents()
 {
     asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 }
+
+// End of a launch that is independent of the previous one (wait_late): it
+// must not complete before the previous grid has.  One waiting thread is
+// enough for that (a grid completes only when all its threads have exited),
+// so only thread 0 of CTA 0 waits and every other CTA frees its slot at once.
+__device__ __forceinline__ void pdl_wait_at_end(int32_t wait_late)
+{
+    if (wait_late && blockIdx.x == 0 && threadIdx.x == 0)
+        pdl_wait_prerequisites();
+}
 #endif
 
 }  // namespace h3rr

@@ -119,8 +119,7 @@ __global__ void __launch_bounds__(NT) relayout_vec_kernel(const __grid_constant_
             }
         }
     }
-    if (a.wait_late)
-        pdl_wait_prerequisites();
+    pdl_wait_at_end(a.wait_late);
 }
 
 // Any row width: one row per CTA iteration, head-side placement per vector.
@@ -167,8 +166,7 @@ __global__ void __launch_bounds__(kGenericThreads) relayout_generic_kernel(const
             }
         }
     }
-    if (a.wait_late)
-        pdl_wait_prerequisites();
+    pdl_wait_at_end(a.wait_late);
 }
 
 // ---------------------------------------------------------------------------
@@ -331,8 +329,7 @@ __global__ void __launch_bounds__(NT) pull_seq_to_head_kernel(const __grid_const
         }
         __syncthreads();  // the next group overwrites the row table
     }
-    if (a.wait_late)
-        pdl_wait_prerequisites();
+    pdl_wait_at_end(a.wait_late);
 }
 
 // Runs longer than one CTA's slots (NT * MAXV vectors): one run per CTA
@@ -369,8 +366,7 @@ __global__ void __launch_bounds__(NT) pull_seq_to_head_long_kernel(const __grid_
             }
         }
     }
-    if (a.wait_late)
-        pdl_wait_prerequisites();
+    pdl_wait_at_end(a.wait_late);
 }
 
 // ---------------------------------------------------------------------------

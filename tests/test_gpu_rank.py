@@ -18,6 +18,8 @@ DEV = "cuda"
 SHAPES = [  # T, P, H, D, W
     (1024, 3, 56, 128, 2), (1000, 3, 56, 128, 6), (777, 4, 56, 128, 4), (513, 1, 56, 128, 8),
     (300, 2, 30, 64, 7), (97, 3, 9, 8, 3), (200, 2, 56, 128, 1), (129, 1, 64, 256, 5),
+    # head runs longer than a CTA's slots (32 KB and 20 KB): the long-run pull kernel
+    (50, 2, 64, 256, 1), (60, 2, 40, 512, 2),
 ]
 
 
