@@ -777,7 +777,7 @@ def parse_args(argv=None):
     p.add_argument("--steps", type=int, default=1000)
     p.add_argument("--warmup", type=int, default=20)
     p.add_argument("--impl", choices=["native", "reference"], default="native")
-    p.add_argument("--e2e-steps", type=int, default=8)
+    p.add_argument("--e2e-steps", type=int, default=16)
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--profile", choices=["seq_to_head", "head_to_seq", "reduce_scatter"],
                    help="run only this kernel of the step --steps times (ncu captures); no timing")
