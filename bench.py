@@ -779,6 +779,8 @@ def parse_args(argv=None):
     p.add_argument("--impl", choices=["native", "reference"], default="native")
     p.add_argument("--e2e-steps", type=int, default=16)
     p.add_argument("--no-cpu-baseline", action="store_true")
+    p.add_argument("--cpu-budget", type=float, default=12.0,
+                   help="seconds of single-threaded oracle work for cpu_baseline")
     p.add_argument("--profile", choices=["seq_to_head", "head_to_seq", "reduce_scatter"],
                    help="run only this kernel of the step --steps times (ncu captures); no timing")
     p.add_argument("--profile-tokens", type=int, default=STEP_T)
@@ -806,7 +808,8 @@ def main(argv=None):
     if result is not None:
         rank, world, _ = dist_env()
         if world == 1 and not args.no_cpu_baseline:
-            result["cpu_baseline"] = cpu_baseline()
+            result["cpu_baseline"] = cpu_baseline(budget_s=args.cpu_budget,
+                                                  all_cores_s=min(4.0, args.cpu_budget / 3))
         else:
             result["cpu_baseline"] = None
         print(json.dumps(result), flush=True)
