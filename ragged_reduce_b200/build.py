@@ -8,6 +8,7 @@ definition bit for bit.
 from __future__ import annotations
 
 import glob
+import hashlib
 import os
 import subprocess
 import sys
@@ -17,6 +18,7 @@ ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 LIB = os.path.join(PKG, "libh3rr.so")
+DIGEST = LIB + ".sources"  # source_digest() of the build that wrote LIB
 
 NVCC = os.environ.get("NVCC", "nvcc")
 
@@ -35,12 +37,29 @@ def sources() -> list[str]:
     return sorted(glob.glob(os.path.join(CSRC, "*.cu")) + glob.glob(os.path.join(CSRC, "*.cpp")))
 
 
+def dependencies() -> list[str]:
+    """Every file the library is compiled from: sources, internal headers, the
+    public header and this script (its flags)."""
+    headers = glob.glob(os.path.join(CSRC, "*.h")) + glob.glob(os.path.join(CSRC, "*.cuh"))
+    return sources() + sorted(headers) + [os.path.join(INCLUDE, "h3rr.h"), os.path.abspath(__file__)]
+
+
+def source_digest() -> str:
+    """Content digest of dependencies() (file times need not survive a copy)."""
+    h = hashlib.sha256()
+    for path in dependencies():
+        h.update(os.path.relpath(path, ROOT).encode())
+        with open(path, "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()
+
+
 def is_stale() -> bool:
-    if not os.path.exists(LIB):
+    """True if the library is missing or was built from other sources."""
+    if not os.path.exists(LIB) or not os.path.exists(DIGEST):
         return True
-    t = os.path.getmtime(LIB)
-    deps = sources() + glob.glob(os.path.join(CSRC, "*.h")) + [os.path.join(INCLUDE, "h3rr.h")]
-    return any(os.path.getmtime(d) > t for d in deps)
+    with open(DIGEST) as f:
+        return f.read().strip() != source_digest()
 
 
 def build(verbose: bool = False, extra: list[str] | None = None) -> str:
@@ -48,6 +67,9 @@ def build(verbose: bool = False, extra: list[str] | None = None) -> str:
     if verbose:
         print(" ".join(cmd))
     subprocess.run(cmd, check=True)
+    # the digest sits beside the library; extra flags make it a non-default build
+    with open(DIGEST, "w") as f:
+        f.write(source_digest() if not extra else "custom build\n")
     return LIB
 
 
