@@ -85,6 +85,14 @@ __device__ __forceinline__ void st_plain(char* p, const Vec<16>& v)
                  : "memory");
 }
 
+__device__ __forceinline__ void st_plain(char* p, const Vec<32>& v)
+{
+    asm volatile("st.global.v8.u32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};" ::"l"(p),
+                 "r"(v.r[0]), "r"(v.r[1]), "r"(v.r[2]), "r"(v.r[3]), "r"(v.r[4]), "r"(v.r[5]),
+                 "r"(v.r[6]), "r"(v.r[7])
+                 : "memory");
+}
+
 // Owner rank of item x under the quotient/remainder split (q, m) of the
 // partition contract, and the first item of rank i.
 __device__ __forceinline__ int32_t split_owner(int32_t x, int32_t q, int32_t m)
