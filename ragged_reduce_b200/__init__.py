@@ -18,6 +18,7 @@ attention output); D = 128 values per head.
 """
 from __future__ import annotations
 
+import contextlib
 import ctypes as C
 from dataclasses import dataclass
 
@@ -129,21 +130,35 @@ def _as_list(x):
 
 
 def _check_tensors(ts, what: str, itemsize: int = 2):
-    dev = None
+    index = None
     for t in ts:
         if not isinstance(t, torch.Tensor):
             raise TypeError(f"{what}: expected torch tensors")
-        if t.device.type != "cuda":
+        if not t.is_cuda:
             raise ValueError(f"{what}: tensors must be on a CUDA device (got {t.device})")
         if t.element_size() != itemsize:
             raise ValueError(f"{what}: expected {itemsize}-byte elements (got {t.dtype})")
         if not t.is_contiguous():
             raise ValueError(f"{what}: tensors must be contiguous")
-        if dev is None:
-            dev = t.device
-        elif t.device != dev:
+        i = t.get_device()
+        if index is None:
+            index = i
+        elif i != index:
             raise ValueError(f"{what}: all tensors must be on one device")
-    return dev
+    return torch.device("cuda", index) if index is not None else None
+
+
+def _device_guard(dev):
+    """Make `dev` the current device for the call (no-op when it already is)."""
+    if dev is None or dev.index is None or dev.index == torch.cuda.current_device():
+        return contextlib.nullcontext()
+    return torch.cuda.device(dev)
+
+
+def _split_sizes(n: int, w: int) -> list:
+    """Sizes of the quotient/remainder split of n items over w ranks."""
+    q, m = divmod(n, w)
+    return [q + 1 if i < m else q for i in range(w)]
 
 
 def _stream_handle(stream, device) -> int:
@@ -176,13 +191,15 @@ def _relayout_shapes(seq_to_head_dir: bool, send, recv, layout: int = 0):
     else:
         _, P, H, D = seq_side[0].shape
         T = sum(int(t.shape[0]) for t in seq_side)
-    part = partition(T, H, W)
+    if W > T or W > H:
+        partition(T, H, W)  # raises the library's H3_ERR_EMPTY_PARTITION
+    tok, hds = _split_sizes(T, W), _split_sizes(int(H), W)
     for r, t in enumerate(seq_side):
-        want = (P, part.tokens(r), H, D) if seq_pm else (part.tokens(r), P, H, D)
+        want = (P, tok[r], H, D) if seq_pm else (tok[r], P, H, D)
         if tuple(t.shape) != want:
             raise ValueError(f"sequence-side rank {r}: shape {tuple(t.shape)}, expected {want}")
     for j, t in enumerate(head_side):
-        want = (P, T, part.heads(j), D) if head_pm else (T, P, part.heads(j), D)
+        want = (P, T, hds[j], D) if head_pm else (T, P, hds[j], D)
         if tuple(t.shape) != want:
             raise ValueError(f"head-side rank {j}: shape {tuple(t.shape)}, expected {want}")
     return T, int(P), int(H), int(D), W, dev
@@ -196,7 +213,7 @@ def _relayout_layout(seq_to_head_dir: bool, send, recv, layout, window_bytes, st
     info = ExecInfo()
     name = "h3_seq_to_head_layout" if seq_to_head_dir else "h3_head_to_seq_layout"
     cfg = _config(variant, ctas_per_sm, serial)
-    with torch.cuda.device(dev):
+    with _device_guard(dev):
         st = getattr(_abi.lib, name)(
             _abi.pointer_array([t.data_ptr() for t in send]),
             _abi.pointer_array([t.data_ptr() for t in recv]),
@@ -233,7 +250,7 @@ def _relayout_staged(seq_to_head_dir: bool, send, recv, window, stream):
     nbytes = window.numel() * window.element_size()
     info = ExecInfo()
     name = "h3_seq_to_head_staged" if seq_to_head_dir else "h3_head_to_seq_staged"
-    with torch.cuda.device(dev):
+    with _device_guard(dev):
         st = getattr(_abi.lib, name)(
             _abi.pointer_array([t.data_ptr() for t in send]),
             _abi.pointer_array([t.data_ptr() for t in recv]),
@@ -269,25 +286,7 @@ def _relayout(seq_to_head_dir: bool, send, recv, window_bytes, stream, variant, 
               serial=False):
     send = _as_list(send)
     recv = _as_list(recv)
-    W = len(send)
-    if W < 1 or len(recv) != W:
-        raise ValueError("send and recv need one tensor per rank (same count)")
-    dev = _check_tensors(send + recv, "relayout")
-    seq_side = send if seq_to_head_dir else recv
-    head_side = recv if seq_to_head_dir else send
-    if any(t.dim() != 4 for t in send + recv):
-        raise ValueError("relayout buffers are 4-D: [tokens, planes, heads, head_dim]")
-    _, P, H, D = seq_side[0].shape
-    T = sum(int(t.shape[0]) for t in seq_side)
-    part = partition(T, H, W)
-    for r, t in enumerate(seq_side):
-        if tuple(t.shape) != (part.tokens(r), P, H, D):
-            raise ValueError(f"sequence-side rank {r}: shape {tuple(t.shape)}, "
-                             f"expected {(part.tokens(r), P, H, D)}")
-    for j, t in enumerate(head_side):
-        if tuple(t.shape) != (T, P, part.heads(j), D):
-            raise ValueError(f"head-side rank {j}: shape {tuple(t.shape)}, "
-                             f"expected {(T, P, part.heads(j), D)}")
+    T, P, H, D, W, dev = _relayout_shapes(seq_to_head_dir, send, recv)
     info = ExecInfo()
     name = "h3_seq_to_head" if seq_to_head_dir else "h3_head_to_seq"
     cfg = _config(variant, ctas_per_sm, serial)
@@ -295,7 +294,7 @@ def _relayout(seq_to_head_dir: bool, send, recv, window_bytes, stream, variant, 
             _abi.pointer_array([t.data_ptr() for t in recv]),
             T, int(P), int(H), int(D), W, int(window_bytes),
             C.c_void_p(_stream_handle(stream, dev))]
-    with torch.cuda.device(dev):
+    with _device_guard(dev):
         if cfg is None:
             st = getattr(_abi.lib, name)(*args, C.byref(info))
         else:
@@ -346,19 +345,17 @@ def ragged_reduce_scatter(partials, bias, out, *, stream=None, ctas_per_sm: int 
         raise ValueError("all partials must have the same [T, C] shape")
     if bias is not None and tuple(bias.shape) != (Cc,):
         raise ValueError(f"bias must be [C] = [{Cc}]")
-    part = partition(T, W, W) if T >= W else None
-    if part is not None:
-        for r, o in enumerate(out):
-            if tuple(o.shape) != (part.tokens(r), Cc):
-                raise ValueError(f"out rank {r}: shape {tuple(o.shape)}, expected "
-                                 f"{(part.tokens(r), Cc)}")
+    if T >= W:
+        for r, (o, rows) in enumerate(zip(out, _split_sizes(T, W))):
+            if tuple(o.shape) != (rows, Cc):
+                raise ValueError(f"out rank {r}: shape {tuple(o.shape)}, expected {(rows, Cc)}")
     info = ExecInfo()
     cfg = _config(0, ctas_per_sm, serial)
     args = [_abi.pointer_array([p.data_ptr() for p in partials]),
             C.c_void_p(bias.data_ptr() if bias is not None else 0),
             _abi.pointer_array([o.data_ptr() for o in out]),
             int(T), int(Cc), W, C.c_void_p(_stream_handle(stream, dev))]
-    with torch.cuda.device(dev):
+    with _device_guard(dev):
         if cfg is None:
             st = _abi.lib.h3_ragged_reduce_scatter(*args, C.byref(info))
         else:
@@ -373,7 +370,7 @@ def bulk_wait_timeouts(stream=None, reset: bool = False, device=None) -> int:
     bulk launch gave up and its output is incomplete."""
     dev = torch.device("cuda", torch.cuda.current_device()) if device is None else torch.device(device)
     count = C.c_uint32(0)
-    with torch.cuda.device(dev):
+    with _device_guard(dev):
         st = _abi.lib.h3_bulk_wait_timeouts(C.c_void_p(_stream_handle(stream, dev)), C.byref(count),
                                             1 if reset else 0)
     _abi.check(st, "h3_bulk_wait_timeouts")
@@ -386,7 +383,7 @@ def bounded_wait_selftest(polls: int, arrive_first: bool, *, stream=None, device
     expired.  Synchronises the stream."""
     dev = torch.device("cuda", torch.cuda.current_device()) if device is None else torch.device(device)
     expired = C.c_int32(-1)
-    with torch.cuda.device(dev):
+    with _device_guard(dev):
         st = _abi.lib.h3_bounded_wait_selftest(int(polls), 1 if arrive_first else 0,
                                                C.c_void_p(_stream_handle(stream, dev)),
                                                C.byref(expired))
@@ -412,10 +409,9 @@ def ragged_all_gather(blocks, out, *, stream=None, variant: int = 0, ctas_per_sm
     Cc = int(blocks[0].shape[1])
     T = sum(int(b.shape[0]) for b in blocks)
     if T >= W:
-        part = partition(T, W, W)
-        for r, b in enumerate(blocks):
-            if tuple(b.shape) != (part.tokens(r), Cc):
-                raise ValueError(f"block {r}: shape {tuple(b.shape)}, expected {(part.tokens(r), Cc)}")
+        for r, (b, rows) in enumerate(zip(blocks, _split_sizes(T, W))):
+            if tuple(b.shape) != (rows, Cc):
+                raise ValueError(f"block {r}: shape {tuple(b.shape)}, expected {(rows, Cc)}")
     for j, o in enumerate(out):
         if tuple(o.shape) != (T, Cc):
             raise ValueError(f"out {j}: shape {tuple(o.shape)}, expected {(T, Cc)}")
@@ -424,7 +420,7 @@ def ragged_all_gather(blocks, out, *, stream=None, variant: int = 0, ctas_per_sm
             _abi.pointer_array([o.data_ptr() for o in out]),
             T, Cc, W, C.c_void_p(_stream_handle(stream, dev))]
     cfg = _config(variant, ctas_per_sm, serial)
-    with torch.cuda.device(dev):
+    with _device_guard(dev):
         if cfg is None:
             st = _abi.lib.h3_ragged_all_gather(*args, C.byref(info))
         else:
@@ -456,14 +452,13 @@ def ragged_reduce_scatter_gated(partials, bias, gate, seg_bounds, x, out=None, *
     if tuple(gate.shape) != (S, Cc):
         raise ValueError(f"gate must be [S, C] = [{S}, {Cc}]")
     if T >= W:
-        part = partition(T, W, W)
-        for r in range(W):
+        for r, rows in enumerate(_split_sizes(int(T), W)):
             for name, t in (("x", x[r]), ("out", out[r])):
-                if tuple(t.shape) != (part.tokens(r), Cc):
+                if tuple(t.shape) != (rows, Cc):
                     raise ValueError(f"{name} rank {r}: shape {tuple(t.shape)}, expected "
-                                     f"{(part.tokens(r), Cc)}")
+                                     f"{(rows, Cc)}")
     info = ExecInfo()
-    with torch.cuda.device(dev):
+    with _device_guard(dev):
         st = _abi.lib.h3_ragged_reduce_scatter_gated(
             _abi.pointer_array([p.data_ptr() for p in partials]),
             C.c_void_p(bias.data_ptr() if bias is not None else 0), C.c_void_p(gate.data_ptr()),
@@ -518,7 +513,7 @@ def seq_to_head_rank(send, recv, rank: int, *, n_heads: int, window_bytes: int =
         raise ValueError(f"recv has {Hk} heads; rank {rank} of {W} owns "
                          f"{partition(T, n_heads, W).heads(rank)}")
     info = ExecInfo()
-    with torch.cuda.device(dev):
+    with _device_guard(dev):
         st = _abi.lib.h3_seq_to_head_rank(
             _abi.pointer_array(_addresses(send, "send")), C.c_void_p(recv.data_ptr()), T, P,
             int(n_heads), D, W, int(rank), int(window_bytes),
@@ -541,7 +536,7 @@ def head_to_seq_rank(send, recv, rank: int, *, n_tokens: int, window_bytes: int 
         raise ValueError(f"recv has {Tk} tokens; rank {rank} of {W} owns "
                          f"{partition(n_tokens, H, W).tokens(rank)}")
     info = ExecInfo()
-    with torch.cuda.device(dev):
+    with _device_guard(dev):
         st = _abi.lib.h3_head_to_seq_rank(
             _abi.pointer_array(_addresses(send, "send")), C.c_void_p(recv.data_ptr()),
             int(n_tokens), P, H, D, W, int(rank), int(window_bytes),
@@ -565,7 +560,7 @@ def ragged_reduce_scatter_rank(partials, bias, out, rank: int, *, n_tokens: int,
                          f"{partition(n_tokens, W, W).tokens(rank)}")
     b = 0 if bias is None else _addresses([bias], "bias")[0]
     info = ExecInfo()
-    with torch.cuda.device(dev):
+    with _device_guard(dev):
         st = _abi.lib.h3_ragged_reduce_scatter_rank(
             _abi.pointer_array(_addresses(partials, "partials")), C.c_void_p(b),
             C.c_void_p(out.data_ptr()), int(n_tokens), Cc, W, int(rank),
@@ -597,7 +592,7 @@ def ragged_reduce_scatter_gated_rank(partials, bias, gate, seg_bounds, x, rank: 
     bounds = np.ascontiguousarray(np.asarray(seg_bounds, dtype=np.int64))
     b = 0 if bias is None else _addresses([bias], "bias")[0]
     info = ExecInfo()
-    with torch.cuda.device(dev):
+    with _device_guard(dev):
         st = _abi.lib.h3_ragged_reduce_scatter_gated_rank(
             _abi.pointer_array(_addresses(partials, "partials")), C.c_void_p(b),
             C.c_void_p(_addresses([gate], "gate")[0]),
@@ -618,7 +613,7 @@ def ragged_all_gather_rank(blocks, out, rank: int, *, stream=None, ctas_per_sm: 
     dev = _local_output(out, "out", 2)
     T, Cc = (int(v) for v in out.shape)
     info = ExecInfo()
-    with torch.cuda.device(dev):
+    with _device_guard(dev):
         st = _abi.lib.h3_ragged_all_gather_rank(
             _abi.pointer_array(_addresses(blocks, "blocks")), C.c_void_p(out.data_ptr()), T, Cc,
             W, int(rank), C.c_void_p(_stream_handle(stream, dev)),

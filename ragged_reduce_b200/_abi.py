@@ -205,7 +205,4 @@ def check(status: int, call: str) -> None:
 
 
 def pointer_array(ptrs) -> C.Array:
-    arr = (C.c_void_p * len(ptrs))()
-    for i, p in enumerate(ptrs):
-        arr[i] = p
-    return arr
+    return (C.c_void_p * len(ptrs))(*ptrs)
