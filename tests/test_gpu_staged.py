@@ -77,6 +77,31 @@ def test_staged_equals_direct_on_full_qkv_32k():
     assert gu.same_bits(back_full, x)
 
 
+def test_staged_full_250k_qkvg_with_the_pages_window():
+    """The pages' configuration: QKVG [250000, 4, 56, 128] over 4 ranks
+    through an 896,000,000-byte window: staged equals direct in both
+    directions.  The window holds 62,500 full token rows, so each plane
+    takes 4 chunks (16 per direction)."""
+    w = wl.QKVG_250K_W4_CHUNKED
+    x = wl.packed_operand(w, device=DEV)
+    part = rr.partition(w.T, w.H, w.W)
+    send = rr.split_rows(x, part.token_starts)
+    win = torch.empty(w.window_bytes, dtype=torch.uint8, device=DEV)
+    staged = rr.alloc_head_side(w.T, w.P, w.H, w.D, w.W, DEV)
+    info = rr.seq_to_head_staged(send, staged, win)
+    assert info["chunks"] == 16 and info["launches"] == 32
+    assert rr.staged_plan(w.T, w.P, w.H, w.D, w.window_bytes) == (62500, 16)
+    direct = rr.alloc_head_side(w.T, w.P, w.H, w.D, w.W, DEV)
+    rr.seq_to_head(send, direct, window_bytes=w.window_bytes)
+    for j in range(w.W):
+        assert gu.same_bits(staged[j], direct[j]), j
+    del direct
+    torch.cuda.empty_cache()
+    back_full, back = rr.alloc_seq_side(w.T, w.P, w.H, w.D, w.W, DEV)
+    rr.head_to_seq_staged(staged, back, win)
+    assert gu.same_bits(back_full, x)
+
+
 def test_staged_rejects_small_or_overlapping_window():
     T, P, H, D, W = 100, 3, 56, 128, 4
     full = wl.random_bits((T, P, H, D), 3, DEV)
