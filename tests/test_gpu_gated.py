@@ -47,9 +47,11 @@ def test_gated_matches_oracle(oracle_lib, T, C, W, S, in_place):
         assert np.array_equal(gu.bits(out[r]), want[r]), f"rank {r}"
 
 
-def test_gated_equals_reduce_scatter_then_gating_full_size():
-    """The 64k x 7168 x 8 workload, 16 segments: fused == unfused composition
-    (torch binary32 gating on the plain reduce-scatter output)."""
+def test_gated_equals_reduce_scatter_then_gating_full_size(oracle_lib):
+    """The 64k x 7168 x 8 workload, 16 segments: every element against the
+    unfused composition (torch binary32 gating on the plain reduce-scatter
+    output), and sampled rows -- every rank and segment boundary among them --
+    through the oracle."""
     T, C, W, S = 65536, 7168, 8, 16
     partials, bias, gate, bounds, x_full, x = _inputs(T, C, W, S, 4)
     red_full, red = rr.alloc_reduce_outputs(T, C, W, DEV)
@@ -59,6 +61,21 @@ def test_gated_equals_reduce_scatter_then_gating_full_size():
     out_full, out = rr.alloc_reduce_outputs(T, C, W, DEV)
     rr.ragged_reduce_scatter_gated(partials, bias, gate, bounds, x, out)
     assert gu.same_bits(out_full, want)
+    # sampled rows through the oracle: each sampled row becomes a segment of
+    # its own carrying its original gate row, the rows split over W ranks
+    ts = rr.partition(T, W, W).token_starts
+    rng = np.random.default_rng(44)
+    b = np.asarray(bounds)
+    rows = np.unique(np.concatenate([rng.integers(0, T, 160), ts[:-1], ts[1:] - 1, b[:-1], b[1:] - 1]))
+    rows_t = torch.from_numpy(rows).to(DEV)
+    sub_parts = [gu.bits(partials[k].index_select(0, rows_t)) for k in range(W)]
+    sub_gate = gu.bits(gate.index_select(0, seg.index_select(0, rows_t)))
+    sub_bounds = np.arange(len(rows) + 1, dtype=np.int64)
+    sub_x = gu.bits(x_full.index_select(0, rows_t))
+    sts = oracle_lib.partition_range(len(rows), W)
+    got = oracle_lib.reduce_scatter_gated(sub_parts, gu.bits(bias), sub_gate, sub_bounds,
+                                          [sub_x[sts[r]:sts[r + 1]] for r in range(W)], W)
+    assert np.array_equal(np.concatenate(got), gu.bits(out_full.index_select(0, rows_t)))
 
 
 def test_gated_random_bit_patterns(oracle_lib):
