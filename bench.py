@@ -97,7 +97,7 @@ def load_peak():
 KERNEL_SOURCES = {
     "seq_to_head": ("relayout.cu", "device_access.cuh", "bulk_copy.cuh", "h3rr_internal.h"),
     "head_to_seq": ("relayout.cu", "device_access.cuh", "bulk_copy.cuh", "h3rr_internal.h"),
-    "ragged_reduce_scatter": ("reduce_scatter.cu", "device_access.cuh", "h3rr_internal.h"),
+    "ragged_reduce_scatter": ("reduce_scatter.cu", "bf16_sum.cuh", "device_access.cuh", "h3rr_internal.h"),
 }
 
 
