@@ -473,50 +473,62 @@ def host_cores() -> int:
         return os.cpu_count() or 1
 
 
-def oracle_all_cores(seconds: float, sample_tokens: int) -> dict:
-    """The unchanged oracle on every host core at once: one thread per core,
-    each running the step on its own token sample for `seconds` (the C oracle
-    runs without the GIL, so the threads use separate cores)."""
-    from concurrent.futures import ThreadPoolExecutor
-    cores = host_cores()
-    tokens = max(STEP_W, min(1024, sample_tokens // cores))
-    steps = [OracleStep(tokens) for _ in range(cores)]
-    deadline = time.perf_counter() + seconds
+class OracleSteps:
+    """The step through the unchanged oracle on every host core at once: one
+    token sample per thread, run concurrently (the C oracle is called without
+    the GIL, so the threads use separate cores)."""
 
-    def work(s):
-        n = 0
-        while time.perf_counter() < deadline or n == 0:
-            s.run()
-            n += 1
-        return n * s.bytes
+    def __init__(self, tokens_each: int, threads: int):
+        from concurrent.futures import ThreadPoolExecutor
+        self.steps = [OracleStep(tokens_each) for _ in range(threads)]
+        self.tokens_each = tokens_each
+        self.bytes = sum(s.bytes for s in self.steps)
+        self.pool = ThreadPoolExecutor(max_workers=threads)
 
-    t0 = time.perf_counter()
-    with ThreadPoolExecutor(max_workers=cores) as pool:
-        total = sum(pool.map(work, steps))
-    t = time.perf_counter() - t0
-    return {"value": round(total / t / 1e9, 3), "unit": UNIT, "cores": cores, "kind": "oracle",
-            "sample": f"{cores} threads, each the step on {tokens} tokens repeatedly for "
-                      f"{t:.1f} s, C oracle unchanged"}
+    def run(self):
+        list(self.pool.map(lambda s: s.run(), self.steps))
+
+    def close(self):
+        self.pool.shutdown()
 
 
-def cpu_baseline(budget_s: float = 12.0, all_cores_s: float = 4.0) -> dict:
+# tokens of one thread's sample: bounds host memory (about 70 KB per token)
+MAX_TOKENS_PER_THREAD = 2048
+
+
+def cpu_baseline(budget_s: float = 12.0) -> dict:
+    """The oracle on every host core (the reported value) and on one core
+    (`one_core`), each on a bounded token sample of the bench step."""
     per_tok = oracle_seconds_per_token()
-    tokens = int(min(STEP_T, max(STEP_W, budget_s / 2 / per_tok)))
+    # one core: the step on one sample, best of 2
+    tokens = int(min(STEP_T, max(STEP_W, budget_s / 4 / per_tok)))
     s = OracleStep(tokens)
     times = []
     for _ in range(2):
         t0 = time.perf_counter()
         s.run()
         times.append(time.perf_counter() - t0)
-    t = min(times)
-    nbytes = s.bytes
-    del s  # free the sample before the all-cores run allocates its own
-    out = {"value": round(nbytes / t / 1e9, 3), "unit": UNIT, "cores": 1, "kind": "oracle",
+    t1 = min(times)
+    one = {"value": round(s.bytes / t1 / 1e9, 3), "unit": UNIT, "cores": 1, "kind": "oracle",
            "sample": f"the step on {tokens} of {STEP_T} tokens (W={STEP_W}, same shapes otherwise), "
-                     f"best of 2, {t:.2f} s each, single-threaded C oracle"}
-    if all_cores_s > 0 and host_cores() > 1:
-        out["all_cores"] = oracle_all_cores(all_cores_s, tokens)
-    return out
+                     f"best of 2, {t1:.2f} s each, single-threaded C oracle"}
+    del s
+    # every core: one sample per thread, repeated for about budget/2 seconds
+    cores = host_cores()
+    each = int(max(STEP_W, min(MAX_TOKENS_PER_THREAD, budget_s / 8 / per_tok)))
+    steps = OracleSteps(each, cores)
+    steps.run()  # warm
+    n, t0 = 0, time.perf_counter()
+    while n == 0 or time.perf_counter() - t0 < budget_s / 2:
+        steps.run()
+        n += 1
+    t = time.perf_counter() - t0
+    steps.close()
+    return {"value": round(steps.bytes * n / t / 1e9, 3), "unit": UNIT, "cores": cores,
+            "kind": "oracle",
+            "sample": f"{cores} threads, each the step on its own {each} tokens (W={STEP_W}, "
+                      f"same shapes otherwise), {n} rounds in {t:.1f} s, C oracle unchanged",
+            "one_core": one}
 
 
 def run_reference(args):
@@ -526,25 +538,27 @@ def run_reference(args):
     budget = float(args.reference_budget)  # seconds for warm-up + timed steps
     per_tok = oracle_seconds_per_token()
     per_step = budget / max(1, args.steps + args.warmup)
-    tokens = int(min(STEP_T, max(STEP_W, per_step / per_tok)))
-    s = OracleStep(tokens)
+    cores = host_cores()
+    each = int(min(MAX_TOKENS_PER_THREAD, max(STEP_W, per_step / per_tok)))
+    s = OracleSteps(each, cores)
     for _ in range(args.warmup):
         s.run()
     t0 = time.perf_counter()
     for _ in range(args.steps):
         s.run()
     t = time.perf_counter() - t0
+    s.close()
     value = s.bytes * args.steps / t / 1e9
-    sample = (f"each step: the path on {tokens} of {STEP_T} tokens (W={STEP_W}, same shapes "
-              f"otherwise), single-threaded C oracle")
+    sample = (f"each step: {cores} threads, each the path on its own {each} tokens (W={STEP_W}, "
+              f"same shapes otherwise), C oracle unchanged")
     return {
         "impl": "reference", "metric": METRIC, "value": round(value, 3), "unit": UNIT,
         "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": round(t / args.steps * 1e3, 3), "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
         "config": {"workload": "h3_transport_step_T32768_W6", "tokens": STEP_T, "world": STEP_W,
-                   "sample_tokens": tokens},
-        "cpu_baseline": {"value": round(value, 3), "unit": UNIT, "cores": 1, "kind": "oracle",
+                   "sample_tokens": each * cores},
+        "cpu_baseline": {"value": round(value, 3), "unit": UNIT, "cores": cores, "kind": "oracle",
                          "sample": sample},
         "e2e": {"value": round(value, 3), "unit": UNIT, "h2d_bytes_per_step": 0,
                 "d2h_bytes_per_step": 0},
@@ -780,7 +794,7 @@ def parse_args(argv=None):
     p.add_argument("--e2e-steps", type=int, default=16)
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--cpu-budget", type=float, default=12.0,
-                   help="seconds of single-threaded oracle work for cpu_baseline")
+                   help="about how many seconds cpu_baseline spends on the oracle")
     p.add_argument("--profile", choices=["seq_to_head", "head_to_seq", "reduce_scatter"],
                    help="run only this kernel of the step --steps times (ncu captures); no timing")
     p.add_argument("--profile-tokens", type=int, default=STEP_T)
@@ -808,8 +822,7 @@ def main(argv=None):
     if result is not None:
         rank, world, _ = dist_env()
         if world == 1 and not args.no_cpu_baseline:
-            result["cpu_baseline"] = cpu_baseline(budget_s=args.cpu_budget,
-                                                  all_cores_s=min(4.0, args.cpu_budget / 3))
+            result["cpu_baseline"] = cpu_baseline(budget_s=args.cpu_budget)
         else:
             result["cpu_baseline"] = None
         print(json.dumps(result), flush=True)
