@@ -567,23 +567,50 @@ def run_reference(args):
 
 
 def run_profile(args):
-    """Run one kernel of the step --steps times (for ncu captures); no timing."""
+    """Run one kernel of the path --steps times (for ncu captures); no timing.
+    The step's kernels on the bench workload, and the widened rows on the same
+    shapes: gated reduce-scatter (8 segments), all-gather of the reduce
+    outputs, staged seq->head through the 896,000,000-byte window, and rank
+    0's pulled seq->head share."""
     torch.cuda.set_device(0)
     device = torch.device("cuda", 0)
     T = args.profile_tokens
-    relayout = args.profile in ("seq_to_head", "head_to_seq")
+    relayout = args.profile in ("seq_to_head", "head_to_seq", "staged_seq_to_head", "rank_seq_to_head")
     step = Step(device, T=T, relayout=relayout, reduce=not relayout)
     rr = step.rr
     if args.profile == "head_to_seq":
         rr.seq_to_head(step.send, step.heads)
+    extra = {}
+    if args.profile == "gated_reduce_scatter":
+        extra["gate"] = wl.normal_bf16((STEP_SEGS, step.C), STEP_SEED + 2, 1.0, device)
+        extra["x_full"], extra["x"] = rr.alloc_reduce_outputs(T, step.C, step.W, device)
+        extra["x_full"].copy_(wl.normal_bf16((T, step.C), STEP_SEED + 3, 1.0, device))
+    elif args.profile == "all_gather":
+        rr.ragged_reduce_scatter(step.partial_list, step.bias, step.red_out)
+        extra["outs"] = [torch.empty((T, step.C), dtype=torch.bfloat16, device=device)
+                         for _ in range(step.W)]
+    elif args.profile == "staged_seq_to_head":
+        extra["win"] = torch.empty(WINDOW, dtype=torch.uint8, device=device)
+    elif args.profile == "rank_seq_to_head":
+        extra["mine"] = torch.empty_like(step.heads[0])
     launches = 0
     for _ in range(args.steps):
         if args.profile == "seq_to_head":
-            launches += rr.seq_to_head(step.send, step.heads)["launches"]
+            info = rr.seq_to_head(step.send, step.heads)
         elif args.profile == "head_to_seq":
-            launches += rr.head_to_seq(step.heads, step.back, window_bytes=WINDOW)["launches"]
+            info = rr.head_to_seq(step.heads, step.back, window_bytes=WINDOW)
+        elif args.profile == "reduce_scatter":
+            info = rr.ragged_reduce_scatter(step.partial_list, step.bias, step.red_out)
+        elif args.profile == "gated_reduce_scatter":
+            info = rr.ragged_reduce_scatter_gated(step.partial_list, step.bias, extra["gate"],
+                                                  step.bounds, extra["x"], step.red_out)
+        elif args.profile == "all_gather":
+            info = rr.ragged_all_gather(step.red_out, extra["outs"])
+        elif args.profile == "staged_seq_to_head":
+            info = rr.seq_to_head_staged(step.send, step.heads, extra["win"])
         else:
-            launches += rr.ragged_reduce_scatter(step.partial_list, step.bias, step.red_out)["launches"]
+            info = rr.seq_to_head_rank(step.send, extra["mine"], 0, n_heads=step.H)
+        launches += info["launches"]
     torch.cuda.synchronize()
     print(json.dumps({"profile": args.profile, "tokens": T, "launches": launches}), flush=True)
     return 0
@@ -795,7 +822,9 @@ def parse_args(argv=None):
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--cpu-budget", type=float, default=12.0,
                    help="about how many seconds cpu_baseline spends on the oracle")
-    p.add_argument("--profile", choices=["seq_to_head", "head_to_seq", "reduce_scatter"],
+    p.add_argument("--profile", choices=["seq_to_head", "head_to_seq", "reduce_scatter",
+                                         "gated_reduce_scatter", "all_gather",
+                                         "staged_seq_to_head", "rank_seq_to_head"],
                    help="run only this kernel of the step --steps times (ncu captures); no timing")
     p.add_argument("--profile-tokens", type=int, default=STEP_T)
     p.add_argument("--report-workloads", action="store_true",
