@@ -54,3 +54,16 @@ def test_reference_line():
     assert d["impl"] == "reference" and d["unit"] == "GB/s" and d["value"] > 0
     assert d["cpu_baseline"]["kind"] == "oracle" and d["cpu_baseline"]["value"] == d["value"]
     assert d["e2e"]["h2d_bytes_per_step"] == 0 and d["e2e"]["value"] == d["value"]
+
+
+@pytest.mark.parametrize("mode,launches", [
+    ("seq_to_head", 2), ("head_to_seq", 6), ("reduce_scatter", 2), ("gated_reduce_scatter", 2),
+    ("all_gather", 2), ("staged_seq_to_head", 12), ("rank_seq_to_head", 2)])
+def test_profile_modes_run(mode, launches):
+    """Every --profile mode (the commands of the ncu captures) runs its kernel."""
+    out = subprocess.run([sys.executable, "bench.py", "--profile", mode, "--steps", "2",
+                          "--profile-tokens", "4096"], cwd=ROOT, capture_output=True, text=True,
+                         timeout=600)
+    assert out.returncode == 0, out.stdout[-2000:] + out.stderr[-2000:]
+    rec = json.loads([l for l in out.stdout.splitlines() if l.startswith("{")][-1])
+    assert rec["profile"] == mode and rec["tokens"] == 4096 and rec["launches"] == launches
