@@ -110,9 +110,11 @@ typedef struct h3_exec_info {
  * those of plain stream order.  Within one chunked relayout call, the launch
  * of plane p+1 touches memory disjoint from plane p's and runs alongside
  * plane p's tail; it waits for plane p at its end instead, so that the call's
- * completion still implies every plane's.  The bulk (TMA) and staged kernels
- * launch in plain stream order.  A kernel that follows in the stream and was
- * itself launched with programmatic serialization must wait
+ * completion still implies every plane's.  The staged calls' kernels are
+ * launched the same way and always wait at their start (each chunk depends on
+ * the previous launch; only the launch latency is hidden); the bulk (TMA)
+ * kernels launch in plain stream order.  A kernel that follows in the stream
+ * and was itself launched with programmatic serialization must wait
  * (cudaGridDependencySynchronize) before reading these calls' outputs.
  */
 #define H3_LAUNCH_SERIAL 1       /* launch every kernel in plain stream order */

@@ -26,6 +26,13 @@
 // ones; rows or runs too wide for those shapes take the plain per-vector
 // kernels (staged_row_kernel, window_block_kernel).
 // seq->head = row kernel then block kernel; head->seq = block then row.
+//
+// Every launch uses programmatic dependent launch: its CTAs may be scheduled
+// while the previous launch drains, and each waits for that launch to
+// complete (griddepcontrol.wait) before its first memory access.  Each
+// launch reads what the previous one wrote, or overwrites the window it
+// read, so nothing runs early; what is saved is the launch latency between
+// chunks, which bounds small windows.
 #include "device_access.cuh"
 #include "h3rr_internal.h"
 
@@ -39,6 +46,8 @@ constexpr int64_t kMaxGrid = (int64_t(1) << 31) - 1;
 template <bool kToWindow>
 __global__ void __launch_bounds__(kThreads) staged_row_kernel(const __grid_constant__ StagedArgs a)
 {
+    pdl_wait_prerequisites();
+    pdl_allow_dependents();
     const int64_t row_bytes = int64_t(a.row_vecs) * kVecBytes;
     for (int64_t i = blockIdx.x; i < a.n; i += gridDim.x) {
         const int32_t t = a.t0 + int32_t(i);
@@ -72,6 +81,8 @@ __global__ void __launch_bounds__(kThreads) staged_row_kernel(const __grid_const
 template <bool kToHead>
 __global__ void __launch_bounds__(kThreads) window_block_kernel(const __grid_constant__ StagedArgs a)
 {
+    pdl_wait_prerequisites();
+    pdl_allow_dependents();
     const int64_t runs = int64_t(a.W) * a.n;
     for (int64_t r = blockIdx.x; r < runs; r += gridDim.x) {
         const int32_t j = int32_t(r / a.n);
@@ -121,6 +132,8 @@ __global__ void __launch_bounds__(NT) staged_row_vec_kernel(const __grid_constan
         wbase[k] = ((int64_t(a.n) * hs + (h - hs)) * head_v + within) * VW;
         wstride[k] = int64_t(hj) * head_v * VW;
     }
+    pdl_wait_prerequisites();
+    pdl_allow_dependents();
     const int64_t row_bytes = int64_t(row_v) * VW;
     for (int64_t i = blockIdx.x; i < a.n; i += gridDim.x) {
         const int32_t t = a.t0 + int32_t(i);
@@ -171,6 +184,8 @@ __global__ void __launch_bounds__(NT) window_block_vec_kernel(const __grid_const
         slot_row[k] = c / run_v;  // >= ROWS: no vector in this slot
         slot_col[k] = c - slot_row[k] * run_v;
     }
+    pdl_wait_prerequisites();
+    pdl_allow_dependents();
     for (int64_t i0 = int64_t(blockIdx.x) * ROWS; i0 < a.n; i0 += int64_t(gridDim.x) * ROWS) {
         if (threadIdx.x < ROWS) {
             const int64_t i = i0 + threadIdx.x;
@@ -304,8 +319,16 @@ cudaError_t launch_staged(const StagedKernel& k, const StagedArgs& a, cudaStream
         gx = 1;
     *grid_out = int(gx);
     void* params[] = {const_cast<StagedArgs*>(&a)};
-    return cudaLaunchKernel(k.fn, dim3(unsigned(gx), unsigned(k.grid_y)), dim3(k.threads), params, 0,
-                            stream);
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(unsigned(gx), unsigned(k.grid_y));
+    cfg.blockDim = dim3(unsigned(k.threads));
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelExC(&cfg, k.fn, params);
 }
 
 }  // namespace

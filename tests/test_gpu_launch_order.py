@@ -119,3 +119,31 @@ def test_chained_reduce_gather_gated(oracle_lib, serial):
             [gu.bits(v) for v in rr.split_rows(x_src, part.token_starts)], W)
         for r in range(W):
             assert np.array_equal(gu.bits(x[r]), want_g[r]), (round_, r)
+
+
+def test_staged_calls_chain_on_one_stream(oracle_lib):
+    """Staged calls through a 37-row window (330 launches per call, each
+    reading what the previous one wrote or overwriting the window it read),
+    chained with direct relayouts and torch copies on one stream, fresh data
+    every round: the programmatic launches must keep stream order."""
+    T, P, H, D, W = 2000, 3, 56, 128, 6
+    part = rr.partition(T, H, W)
+    full = torch.empty((T, P, H, D), dtype=torch.bfloat16, device=DEV)
+    send = rr.split_rows(full, part.token_starts)
+    heads = rr.alloc_head_side(T, P, H, D, W, DEV)
+    heads2 = rr.alloc_head_side(T, P, H, D, W, DEV)
+    back_full, back = rr.alloc_seq_side(T, P, H, D, W, DEV)
+    win = torch.empty(37 * H * D * 2, dtype=torch.uint8, device=DEV)
+    assert rr.staged_plan(T, P, H, D, win.numel())[1] == 3 * 55
+    for round_ in range(4):
+        src = wl.random_bits((T, P, H, D), 300 + round_, DEV)
+        full.copy_(src)
+        info = rr.seq_to_head_staged(send, heads, win)
+        assert info["launches"] == 330
+        rr.head_to_seq(heads, back)
+        rr.seq_to_head_staged(back, heads2, win)
+        rr.head_to_seq_staged(heads2, back, win)
+        want = oracle_lib.seq_to_head([gu.bits(s) for s in send], T, P, H, D, W)
+        for j in range(W):
+            assert np.array_equal(gu.bits(heads2[j]), want[j]), (round_, j)
+        assert gu.same_bits(back_full, src), round_
