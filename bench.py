@@ -44,6 +44,7 @@ import workloads as wl  # noqa: E402
 METRIC = "relayout + reduce-scatter effective HBM GB/s and % of B200 HBM peak"
 UNIT = "GB/s"
 FALLBACK_HBM_GBS = 6650.0
+NOMINAL_HBM_GBS = 8000.0  # nominal B200 HBM3e bandwidth, for a second percentage only
 STEP_T, STEP_W, STEP_P, STEP_SEGS, STEP_SEED = 32768, 6, 3, 8, 2
 WINDOW = 896_000_000
 
@@ -413,6 +414,9 @@ def run_gpu(args):
                        "l2": "no flush: every kernel's inputs (1.4-2.8 GB) exceed the 126 MB L2",
                        "bytes_per_step": step.bytes_per_step},
             "pct_of_peak": round(100.0 * value / world / peak, 2),
+            "pct_of_nominal_peak": {"value": round(100.0 * value / world / NOMINAL_HBM_GBS, 2),
+                                    "peak_gbs": NOMINAL_HBM_GBS,
+                                    "source": "nominal B200 HBM3e bandwidth, ~8 TB/s"},
             "roofline": roofline,
             "kernels": kernels,
             "gpu_launches": launches_total,

@@ -29,6 +29,8 @@ def test_native_line():
     assert d["dtype"] == "bf16" and d["data"] == "synthetic"
     assert d["config"]["workload"] == "h3_transport_step_T32768_W6"
     assert d["value"] > 1000.0
+    n = d["pct_of_nominal_peak"]
+    assert n["peak_gbs"] == 8000.0 and abs(n["value"] - 100.0 * d["value"] / 8000.0) < 0.01
     r = d["roofline"]
     assert r["bound"] == "hbm" and r["unit"] == "GB/s" and r["peak"] > 0 and r["achieved"] > 0
     assert abs(r["frac"] - r["achieved"] / r["peak"]) < 1e-3
