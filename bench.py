@@ -477,6 +477,18 @@ def host_cores() -> int:
         return os.cpu_count() or 1
 
 
+def host_cpu_model() -> str:
+    """The host CPU's model name (Linux /proc/cpuinfo), or "unknown"."""
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.lower().startswith("model name"):
+                    return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    return "unknown"
+
+
 class OracleSteps:
     """The step through the unchanged oracle on every host core at once: one
     token sample per thread, run concurrently (the C oracle is called without
@@ -532,7 +544,7 @@ def cpu_baseline(budget_s: float = 12.0) -> dict:
             "kind": "oracle",
             "sample": f"{cores} threads, each the step on its own {each} tokens (W={STEP_W}, "
                       f"same shapes otherwise), {n} rounds in {t:.1f} s, C oracle unchanged",
-            "one_core": one}
+            "cpu_model": host_cpu_model(), "one_core": one}
 
 
 def run_reference(args):
@@ -563,7 +575,7 @@ def run_reference(args):
         "config": {"workload": "h3_transport_step_T32768_W6", "tokens": STEP_T, "world": STEP_W,
                    "sample_tokens": each * cores},
         "cpu_baseline": {"value": round(value, 3), "unit": UNIT, "cores": cores, "kind": "oracle",
-                         "sample": sample},
+                         "sample": sample, "cpu_model": host_cpu_model()},
         "e2e": {"value": round(value, 3), "unit": UNIT, "h2d_bytes_per_step": 0,
                 "d2h_bytes_per_step": 0},
         "gpu_launches": 0,

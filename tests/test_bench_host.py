@@ -72,6 +72,7 @@ def test_reference_arm_prints_one_line():
     rec = json.loads(lines[0])
     assert rec["impl"] == "reference" and rec["unit"] == "GB/s" and rec["value"] > 0
     assert rec["e2e"]["h2d_bytes_per_step"] == 0 and rec["cpu_baseline"]["kind"] == "oracle"
+    assert rec["cpu_baseline"]["cpu_model"] == bench.host_cpu_model()
     assert rec["metric"] == bench.METRIC
 
 

@@ -39,6 +39,7 @@ def test_native_line():
     assert c["kind"] == "oracle" and c["cores"] >= 1 and c["value"] > 0 and c["sample"]
     assert c["unit"] == d["unit"]
     assert c["one_core"]["cores"] == 1 and c["one_core"]["value"] > 0
+    assert isinstance(c["cpu_model"], str) and c["cpu_model"]
     e = d["e2e"]
     assert e["unit"] == d["unit"] and 0 < e["value"] < d["value"]
     assert e["h2d_bytes_per_step"] == 4_227_872_768 and e["d2h_bytes_per_step"] == 1_879_048_192
