@@ -309,7 +309,9 @@ H3RR_API h3_status h3_ragged_all_gather_ex(const void* const* in, void* const* o
  * Same as h3_seq_to_head / h3_head_to_seq / h3_ragged_reduce_scatter with
  * explicit launch overrides (cfg may be NULL).  Every variant computes the
  * same bytes; the overrides exist for tuning and for testing each variant.
- * An unknown variant returns H3_ERR_INVALID_ARG.
+ * An unknown variant returns H3_ERR_INVALID_ARG.  H3_VARIANT_BULK relayouts
+ * stage four rows of H*D*2 bytes in shared memory: H3_ERR_UNSUPPORTED if they
+ * do not fit (rows above about 57 KB on B200), or with a non-zero layout.
  */
 H3RR_API h3_status h3_seq_to_head_ex(const void* const* send, void* const* recv,
                             int64_t n_tokens, int32_t planes, int32_t n_heads,

@@ -102,16 +102,30 @@ def test_forced_variant_matches_oracle(oracle_lib, T, P, H, D, W, variant):
     assert rr.bulk_wait_timeouts() == 0
 
 
-def test_bulk_rejects_rows_too_wide_for_its_ring():
-    # D=256: a 28,672-byte row, 14 stages do not fit in shared memory
+def test_bulk_ring_width_limit(oracle_lib):
+    """The bulk ring holds four rows: a 28,672-byte row (D=256) fits and
+    matches the oracle; a 114,688-byte row (D=1024) does not fit in shared
+    memory and is refused, while the default call still runs it."""
     T, P, H, D, W = 33, 3, 56, 256, 4
     full, send, part = _seq_inputs(T, P, H, D, W, seed=1)
+    recv = rr.alloc_head_side(T, P, H, D, W, DEV)
+    info = rr.seq_to_head(send, recv, variant=rr.H3_VARIANT_BULK)
+    assert info["variant"] == rr.H3_VARIANT_BULK
+    want = oracle_lib.seq_to_head([gu.bits(x) for x in send], T, P, H, D, W)
+    for j in range(W):
+        assert np.array_equal(gu.bits(recv[j]), want[j]), j
+
+    T, P, H, D, W = 9, 2, 56, 1024, 4
+    full, send, part = _seq_inputs(T, P, H, D, W, seed=2)
     recv = rr.alloc_head_side(T, P, H, D, W, DEV)
     with pytest.raises(rr.H3Error) as e:
         rr.seq_to_head(send, recv, variant=rr.H3_VARIANT_BULK)
     assert e.value.status == 5  # H3_ERR_UNSUPPORTED
-    info = rr.seq_to_head(send, recv)  # the default falls back to vectors
-    assert info["variant"] == rr.H3_VARIANT_VECTOR
+    info = rr.seq_to_head(send, recv)  # the default takes the register kernels
+    assert info["variant"] != rr.H3_VARIANT_BULK
+    want = oracle_lib.seq_to_head([gu.bits(x) for x in send], T, P, H, D, W)
+    for j in range(W):
+        assert np.array_equal(gu.bits(recv[j]), want[j]), j
 
 
 def test_bulk_ring_sizes_alternate(oracle_lib):
