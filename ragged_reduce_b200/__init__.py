@@ -493,6 +493,14 @@ def _addresses(items, what: str) -> list:
     return out
 
 
+def _require_bf16(items, what: str) -> None:
+    """The reduce arithmetic reads BF16: refuse tensors of any other 2-byte
+    type (device addresses carry no type and are taken as given)."""
+    for x in items:
+        if isinstance(x, torch.Tensor) and x.dtype != torch.bfloat16:
+            raise ValueError(f"{what}: BF16 tensors only (got {x.dtype})")
+
+
 def _local_output(t: torch.Tensor, what: str, dims: int):
     _check_tensors([t], what)
     if t.dim() != dims:
@@ -554,6 +562,7 @@ def ragged_reduce_scatter_rank(partials, bias, out, rank: int, *, n_tokens: int,
     partials = list(partials)
     W = len(partials)
     dev = _local_output(out, "out", 2)
+    _require_bf16(partials + [bias, out], "ragged_reduce_scatter_rank")
     Tk, Cc = (int(v) for v in out.shape)
     if Tk != partition(n_tokens, W, W).tokens(rank):
         raise ValueError(f"out has {Tk} rows; rank {rank} of {W} owns "
@@ -583,6 +592,7 @@ def ragged_reduce_scatter_gated_rank(partials, bias, gate, seg_bounds, x, rank: 
     dev = _local_output(x, "x", 2)
     out = x if out is None else out
     _local_output(out, "out", 2)
+    _require_bf16(partials + [bias, gate, x, out], "ragged_reduce_scatter_gated_rank")
     Tk, Cc = (int(v) for v in x.shape)
     if tuple(out.shape) != (Tk, Cc):
         raise ValueError("out must have x's shape")

@@ -148,3 +148,20 @@ def test_gated_rank_shares(oracle_lib, T, C, W, S):
                                         n_tokens=T, out=out)
     assert gu.guards_intact(buf)
     assert np.array_equal(gu.bits(out), want[k])
+
+
+def test_rank_reduce_calls_refuse_non_bf16_tensors():
+    """float16 (or int16) tensors would be read as BF16 bits: the rank reduce
+    wrappers refuse them before anything is launched, as the one-GPU calls do."""
+    T, C, W = 64, 64, 2
+    partials = [torch.zeros((T, C), dtype=torch.bfloat16, device=DEV) for _ in range(W)]
+    out = torch.empty((32, C), dtype=torch.bfloat16, device=DEV)
+    gate = torch.zeros((1, C), dtype=torch.bfloat16, device=DEV)
+    with pytest.raises(ValueError, match="BF16"):
+        rr.ragged_reduce_scatter_rank(partials, None, out.half(), 0, n_tokens=T)
+    with pytest.raises(ValueError, match="BF16"):
+        rr.ragged_reduce_scatter_rank([p.half() for p in partials], None, out, 0, n_tokens=T)
+    with pytest.raises(ValueError, match="BF16"):
+        rr.ragged_reduce_scatter_gated_rank(partials, None, gate, [0, T], out.half(), 0, n_tokens=T)
+    with pytest.raises(ValueError, match="BF16"):
+        rr.ragged_reduce_scatter_gated_rank(partials, None, gate.half(), [0, T], out, 0, n_tokens=T)

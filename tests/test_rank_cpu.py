@@ -283,3 +283,13 @@ def test_peer_buffers_exchange_with_gloo():
         assert sorted(s for s, _ in opened) == sorted(f"rank{r}" for r in range(world) if r != rank)
         assert sorted(a for a, _ in closed) == sorted(p for r, p in enumerate(pointers) if r != rank)
         assert after == []
+
+
+def test_rank_reduce_wrappers_require_bf16():
+    """The reduce arithmetic reads BF16: a tensor of another 2-byte type is
+    refused by the binding; raw device addresses carry no type."""
+    import ragged_reduce_b200 as rr
+    rr._require_bf16([torch.zeros(4, dtype=torch.bfloat16), 0x10000, None], "ok")
+    for dt in (torch.float16, torch.int16):
+        with pytest.raises(ValueError, match="BF16"):
+            rr._require_bf16([torch.zeros(4, dtype=torch.bfloat16), torch.zeros(4, dtype=dt)], "bad")
