@@ -2,7 +2,7 @@
 
 Each mutant is a textual change to a temporary copy of oracle/h3_oracle.c:
 a dropped term, a wrong index, a transposed layout, a changed order or
-precision.  The copy is compiled with the oracle's own flags and the pins of
+precision, a rounding step skipped.  The copy is compiled with the oracle's own flags and the pins of
 tests/oracle_pins.py run against it in a child process (a mutant that writes
 out of bounds may crash the child; that also counts as caught).
 """
@@ -73,6 +73,24 @@ MUTANTS = [
     ("gated_product_dropped", "float sum = h3o_bf16_to_f32(x[r][tl * C + c]) + prod;",
      "float sum = h3o_bf16_to_f32(x[r][tl * C + c]) + g;"),
     ("widen_drops_sign", "uint32_t u = ((uint32_t)b) << 16;", "uint32_t u = ((uint32_t)(b & 0x7FFFu)) << 16;"),
+    ("gated_gates_unrounded_sum", "float prod = g * h3o_bf16_to_f32(y);",
+     "float yu = h3o_bf16_to_f32(vals[0]);\n"
+     "                for (int32_t w2 = 1; w2 < W; ++w2)\n"
+     "                    yu = yu + h3o_bf16_to_f32(vals[w2]);\n"
+     "                if (bias)\n"
+     "                    yu = yu + h3o_bf16_to_f32(bias[c]);\n"
+     "                (void)y;\n"
+     "                float prod = g * yu;"),
+    ("gated_residual_dropped", "float sum = h3o_bf16_to_f32(x[r][tl * C + c]) + prod;",
+     "float sum = prod;"),
+    ("gated_bias_dropped", "uint16_t y = reduce_one(vals, W, bias ? &bias[c] : NULL);",
+     "uint16_t y = reduce_one(vals, W, NULL);"),
+    ("gated_gate_row_by_token", "float g = h3o_bf16_to_f32(gate[k * C + c]);",
+     "float g = h3o_bf16_to_f32(gate[(t % n_segs) * C + c]);"),
+    ("owner_boundary_inclusive", "        if (x < starts[i + 1])\n            return i;",
+     "        if (x <= starts[i + 1])\n            return i;"),
+    ("reduce_rows_drops_bias", "out[t * C + c] = reduce_one(vals, W, bias ? &bias[c] : NULL);",
+     "out[t * C + c] = reduce_one(vals, W, NULL);"),
 ]
 
 _CHILD = r"""
