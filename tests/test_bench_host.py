@@ -82,3 +82,38 @@ def test_reference_arm_other_ranks_exit_quietly():
                           "--gpus", "2", "--steps", "2", "--warmup", "3"],
                          capture_output=True, text=True, env=env, timeout=120)
     assert out.returncode == 0 and out.stdout.strip() == ""
+
+
+def test_traffic_reported_only_for_the_captured_sources(monkeypatch):
+    """ncu traffic from profiles/dram_traffic.json is reported while the
+    kernel's sources still match the digest recorded with the capture, and
+    is None once they differ or the kernel is unknown."""
+    entries = json.load(open(os.path.join(ROOT, "profiles", "dram_traffic.json")))
+    for kernel in bench.KERNEL_SOURCES:
+        e = entries[kernel]
+        assert e["bytes_per_launch"] == e["read_bytes"] + e["write_bytes"]
+        if e["source_digest"] == bench.kernel_source_digest(kernel):
+            assert bench.load_traffic(kernel) == e["bytes_per_launch"]
+    assert bench.load_traffic("no_such_kernel") is None
+    monkeypatch.setattr(bench, "kernel_source_digest", lambda kernel: "0" * 16)
+    for kernel in bench.KERNEL_SOURCES:
+        assert bench.load_traffic(kernel) is None
+
+
+def test_clock_summary():
+    """The clock record: median SM clock over the samples, the largest max
+    clock, and every throttle reason seen active at least once; malformed
+    lines are skipped and no samples give an empty record."""
+    c = bench.ClockSampler(None)
+    assert c.summary() == {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
+    c.lines = [
+        "0, 1965, 1965, 700.1, 0x0, Not Active, Not Active, Not Active, Not Active",
+        "0, 1710, 1965, 998.0, 0x4, Not Active, Not Active, Not Active, Active",
+        "0, 1800, 1965, 990.5, 0x4, Not Active, Not Active, Not Active, Active",
+        "garbled line",
+        "0, [N/A], 1965, 0, 0x0, Not Active, Not Active, Not Active, Not Active",
+    ]
+    r = c.summary()
+    assert r == {"sm_mhz": 1800.0, "sm_max_mhz": 1965.0, "reasons": ["sw_power_cap"], "samples": 3}
+    c.lines.append("0, 1500, 1965, 1000.0, 0x48, Active, Not Active, Active, Active")
+    assert c.summary()["reasons"] == ["hw_slowdown", "sw_power_cap", "sw_thermal_slowdown"]
