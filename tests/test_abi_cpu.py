@@ -423,3 +423,40 @@ def test_gated_argument_checks():
     assert st(outs=[gate] + outs[1:]) == E.H3_ERR_INVALID_ARG
     assert st(outs=[xs[1]] + outs[1:]) == E.H3_ERR_INVALID_ARG          # another rank's x
     assert st(T=5) == E.H3_ERR_EMPTY_PARTITION
+
+
+@needs_no_gpu
+def test_last_cuda_error_is_kept_per_thread():
+    """With no GPU a call that reaches the CUDA runtime fails with
+    H3_ERR_CUDA; the calling thread's h3_last_cuda_error then holds the CUDA
+    error and its text, another thread's stays 0, and the binding's exception
+    carries the same error."""
+    import threading
+    results = {}
+
+    def run():
+        msg = C.c_char_p()
+        results["fresh"] = _abi.lib.h3_last_cuda_error(C.byref(msg))
+        count = C.c_uint32(0)
+        results["status"] = _abi.lib.h3_bulk_wait_timeouts(None, C.byref(count), 0)
+        results["after"] = _abi.lib.h3_last_cuda_error(C.byref(msg))
+        results["text"] = msg.value.decode()
+        try:
+            _abi.check(results["status"], "h3_bulk_wait_timeouts")
+        except _abi.H3Error as e:
+            results["exc"] = e
+
+    t = threading.Thread(target=run)
+    t.start()
+    t.join(timeout=60)
+    assert results["fresh"] == 0
+    assert results["status"] == _abi.H3_ERR_CUDA
+    assert results["after"] != 0 and results["text"] and results["text"] != "no error"
+    e = results["exc"]
+    assert e.status == _abi.H3_ERR_CUDA and e.cuda_error == results["after"]
+    assert results["text"] in str(e)
+    other = []
+    t2 = threading.Thread(target=lambda: other.append(_abi.lib.h3_last_cuda_error(None)))
+    t2.start()
+    t2.join(timeout=60)
+    assert other == [0]
