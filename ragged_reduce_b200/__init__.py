@@ -62,9 +62,11 @@ class Partition:
         return len(self.token_starts) - 1
 
     def tokens(self, r: int) -> int:
+        """Tokens rank r owns (te_r - ts_r)."""
         return int(self.token_starts[r + 1] - self.token_starts[r])
 
     def heads(self, j: int) -> int:
+        """Heads rank j owns (he_j - hs_j)."""
         return int(self.head_starts[j + 1] - self.head_starts[j])
 
 
@@ -675,6 +677,8 @@ class PreparedRelayout:
         return self._info
 
     def device_stream(self, stream):
+        """The cudaStream_t to launch on: `stream`, or the current stream of
+        the prepared call's device."""
         if stream is None:
             return C.c_void_p(torch.cuda.current_stream(self.device).cuda_stream)
         return C.c_void_p(_stream_handle(stream, self.device))
@@ -732,6 +736,8 @@ class PreparedReduceScatter:
 
 
 def prepare_ragged_reduce_scatter(partials, bias, out, **kw) -> PreparedReduceScatter:
+    """A reduce-scatter over fixed buffers, checked and marshalled once;
+    calling it issues one C call (same arguments as ``ragged_reduce_scatter``)."""
     return PreparedReduceScatter(partials, bias, out, **kw)
 
 

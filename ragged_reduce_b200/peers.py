@@ -26,6 +26,7 @@ class CudaIpc:
     """The library's CUDA IPC calls (``h3_ipc_export`` / ``_open`` / ``_close``)."""
 
     def export(self, tensor: torch.Tensor) -> bytes:
+        """The tensor's h3_ipc_handle record (allocation handle, offset, size) as bytes."""
         h = _abi.IpcHandle()
         with torch.cuda.device(tensor.device):
             _abi.check(_abi.lib.h3_ipc_export(C.c_void_p(tensor.data_ptr()), C.byref(h)),
@@ -41,6 +42,7 @@ class CudaIpc:
         return h
 
     def open(self, record: bytes, device: torch.device) -> int:
+        """Map a peer's exported buffer on `device`; returns its address there."""
         h = self._handle(record)
         ptr = C.c_void_p()
         with torch.cuda.device(device):
@@ -48,6 +50,7 @@ class CudaIpc:
         return int(ptr.value)
 
     def close(self, address: int, record: bytes, device: torch.device) -> None:
+        """Release a mapping made by ``open`` (the last release unmaps it)."""
         h = self._handle(record)
         with torch.cuda.device(device):
             _abi.check(_abi.lib.h3_ipc_close(C.c_void_p(address), C.byref(h)), "h3_ipc_close")
@@ -89,6 +92,7 @@ class PeerBuffers:
         self._local = local  # keep the exported buffer alive with the table
 
     def close(self) -> None:
+        """Unmap every peer buffer this table opened (after the caller's final barrier)."""
         while self._opened:
             p, rec = self._opened.pop()
             self.ipc.close(p, rec, self.device)
