@@ -20,6 +20,7 @@ from __future__ import annotations
 
 import contextlib
 import ctypes as C
+import functools
 from dataclasses import dataclass
 
 import numpy as np
@@ -157,10 +158,14 @@ def _device_guard(dev):
     return torch.cuda.device(dev)
 
 
-def _split_sizes(n: int, w: int) -> list:
-    """Sizes of the quotient/remainder split of n items over w ranks."""
-    q, m = divmod(n, w)
-    return [q + 1 if i < m else q for i in range(w)]
+@functools.lru_cache(maxsize=1024)
+def _rank_sizes(n_tokens: int, n_heads: int, world: int) -> tuple:
+    """(tokens per rank, heads per rank) as ``h3_partition`` assigns them,
+    cached per shape so that repeated calls pay one dictionary lookup.  Raises
+    the library's error (for example an empty partition) like ``partition``."""
+    p = partition(n_tokens, n_heads, world)
+    return (tuple(int(v) for v in np.diff(p.token_starts)),
+            tuple(int(v) for v in np.diff(p.head_starts)))
 
 
 def _stream_handle(stream, device) -> int:
@@ -193,9 +198,7 @@ def _relayout_shapes(seq_to_head_dir: bool, send, recv, layout: int = 0):
     else:
         _, P, H, D = seq_side[0].shape
         T = sum(int(t.shape[0]) for t in seq_side)
-    if W > T or W > H:
-        partition(T, H, W)  # raises the library's H3_ERR_EMPTY_PARTITION
-    tok, hds = _split_sizes(T, W), _split_sizes(int(H), W)
+    tok, hds = _rank_sizes(T, int(H), W)  # raises the library's H3_ERR_EMPTY_PARTITION
     for r, t in enumerate(seq_side):
         want = (P, tok[r], H, D) if seq_pm else (tok[r], P, H, D)
         if tuple(t.shape) != want:
@@ -347,10 +350,9 @@ def ragged_reduce_scatter(partials, bias, out, *, stream=None, ctas_per_sm: int 
         raise ValueError("all partials must have the same [T, C] shape")
     if bias is not None and tuple(bias.shape) != (Cc,):
         raise ValueError(f"bias must be [C] = [{Cc}]")
-    if T >= W:
-        for r, (o, rows) in enumerate(zip(out, _split_sizes(T, W))):
-            if tuple(o.shape) != (rows, Cc):
-                raise ValueError(f"out rank {r}: shape {tuple(o.shape)}, expected {(rows, Cc)}")
+    for r, (o, rows) in enumerate(zip(out, _rank_sizes(int(T), W, W)[0])):
+        if tuple(o.shape) != (rows, Cc):
+            raise ValueError(f"out rank {r}: shape {tuple(o.shape)}, expected {(rows, Cc)}")
     info = ExecInfo()
     cfg = _config(0, ctas_per_sm, serial)
     args = [_abi.pointer_array([p.data_ptr() for p in partials]),
@@ -410,10 +412,9 @@ def ragged_all_gather(blocks, out, *, stream=None, variant: int = 0, ctas_per_sm
         raise ValueError("blocks and outputs are 2-D: [tokens, cols]")
     Cc = int(blocks[0].shape[1])
     T = sum(int(b.shape[0]) for b in blocks)
-    if T >= W:
-        for r, (b, rows) in enumerate(zip(blocks, _split_sizes(T, W))):
-            if tuple(b.shape) != (rows, Cc):
-                raise ValueError(f"block {r}: shape {tuple(b.shape)}, expected {(rows, Cc)}")
+    for r, (b, rows) in enumerate(zip(blocks, _rank_sizes(T, W, W)[0])):
+        if tuple(b.shape) != (rows, Cc):
+            raise ValueError(f"block {r}: shape {tuple(b.shape)}, expected {(rows, Cc)}")
     for j, o in enumerate(out):
         if tuple(o.shape) != (T, Cc):
             raise ValueError(f"out {j}: shape {tuple(o.shape)}, expected {(T, Cc)}")
@@ -453,12 +454,11 @@ def ragged_reduce_scatter_gated(partials, bias, gate, seg_bounds, x, out=None, *
     S = len(b) - 1
     if tuple(gate.shape) != (S, Cc):
         raise ValueError(f"gate must be [S, C] = [{S}, {Cc}]")
-    if T >= W:
-        for r, rows in enumerate(_split_sizes(int(T), W)):
-            for name, t in (("x", x[r]), ("out", out[r])):
-                if tuple(t.shape) != (rows, Cc):
-                    raise ValueError(f"{name} rank {r}: shape {tuple(t.shape)}, expected "
-                                     f"{(rows, Cc)}")
+    for r, rows in enumerate(_rank_sizes(int(T), W, W)[0]):
+        for name, t in (("x", x[r]), ("out", out[r])):
+            if tuple(t.shape) != (rows, Cc):
+                raise ValueError(f"{name} rank {r}: shape {tuple(t.shape)}, expected "
+                                 f"{(rows, Cc)}")
     info = ExecInfo()
     with _device_guard(dev):
         st = _abi.lib.h3_ragged_reduce_scatter_gated(
