@@ -1,9 +1,14 @@
 // h3_seq_to_head_staged_noalloc: the staged sequence->head relayout with its
 // window in a device array owned by the library, for callers that cannot
 // allocate device memory (see include/h3rr.h).  Nothing here allocates or
-// frees device memory.
+// frees device memory; the array itself is reserved when the CUDA runtime
+// loads this file's device module into a context (on the first call in that
+// context, under lazy module loading).
+#include <map>
 #include <mutex>
-#include <unordered_map>
+#include <utility>
+
+#include <cuda.h>
 
 #include "h3rr_internal.h"
 
@@ -16,27 +21,86 @@ static __device__ __align__(256) unsigned char g_static_window[H3RR_STATIC_WINDO
 
 namespace {
 
-// Device address of g_static_window on the current device, looked up once
-// per device (with that device current) and kept.
+using CtxGetCurrentFn = CUresult (*)(CUcontext*);
+using CtxGetIdFn = CUresult (*)(CUcontext, unsigned long long*);
+
+// The driver's cuCtxGetCurrent and cuCtxGetId (CUDA 12.0), fetched through
+// the runtime's entry-point query; null if unavailable.
+struct ContextQuery {
+    CtxGetCurrentFn current = nullptr;
+    CtxGetIdFn id = nullptr;
+};
+
+const ContextQuery& context_query()
+{
+    static std::once_flag once;
+    static ContextQuery q;
+    std::call_once(once, [] {
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult r = cudaDriverEntryPointSymbolNotFound;
+        if (cudaGetDriverEntryPointByVersion("cuCtxGetCurrent", &p, 12000, cudaEnableDefault, &r) ==
+                cudaSuccess &&
+            r == cudaDriverEntryPointSuccess)
+            q.current = reinterpret_cast<CtxGetCurrentFn>(p);
+        p = nullptr;
+        r = cudaDriverEntryPointSymbolNotFound;
+        if (cudaGetDriverEntryPointByVersion("cuCtxGetId", &p, 12000, cudaEnableDefault, &r) ==
+                cudaSuccess &&
+            r == cudaDriverEntryPointSuccess)
+            q.id = reinterpret_cast<CtxGetIdFn>(p);
+    });
+    return q;
+}
+
+// Process-unique id of the calling thread's current context (ids are never
+// reused, unlike context handles); false if there is none or the driver
+// cannot say.
+bool current_context_id(unsigned long long* id)
+{
+    const ContextQuery& q = context_query();
+    if (!q.current || !q.id)
+        return false;
+    CUcontext ctx = nullptr;
+    if (q.current(&ctx) != CUDA_SUCCESS || !ctx)
+        return false;
+    return q.id(ctx, id) == CUDA_SUCCESS;
+}
+
+// Device address of g_static_window in the current context.  Looked up with
+// cudaGetSymbolAddress once per device and context, with that device
+// current, and kept under the context's id: after cudaDeviceReset the
+// device's next context has a new id and may hold the array elsewhere, so
+// the lookup runs again there.  Without a context id the lookup runs on
+// every call.
 cudaError_t static_window_address(void** ptr)
 {
     static std::mutex mu;
-    static std::unordered_map<int, void*> addresses;
+    static std::map<std::pair<int, unsigned long long>, void*> addresses;
     int device = 0;
     cudaError_t err = cudaGetDevice(&device);
     if (err != cudaSuccess)
         return err;
-    std::lock_guard<std::mutex> lock(mu);
-    auto it = addresses.find(device);
-    if (it != addresses.end()) {
-        *ptr = it->second;
-        return cudaSuccess;
+    unsigned long long ctx = 0;
+    bool keyed = current_context_id(&ctx);
+    if (keyed) {
+        std::lock_guard<std::mutex> lock(mu);
+        auto it = addresses.find({device, ctx});
+        if (it != addresses.end()) {
+            *ptr = it->second;
+            return cudaSuccess;
+        }
     }
     void* p = nullptr;
     err = cudaGetSymbolAddress(&p, g_static_window);
     if (err != cudaSuccess)
         return err;
-    addresses.emplace(device, p);
+    // The lookup makes the device's primary context current if nothing was.
+    if (!keyed)
+        keyed = current_context_id(&ctx);
+    if (keyed) {
+        std::lock_guard<std::mutex> lock(mu);
+        addresses[{device, ctx}] = p;
+    }
     *ptr = p;
     return cudaSuccess;
 }

@@ -12,8 +12,11 @@ different inputs and window sizes, and compares each result with the existing
 entry point h3_seq_to_head_staged (given a window this test allocates) bit
 for bit, the tolerance every relayout test uses.  The second call also shows
 that what the first call left in the shared array does not leak into the next
-result.  The file is collected after every other test and passes both alone
-in a fresh process and after the rest of the suite.
+result.  Another test checks the property the entry point exists for: once
+its first call has set it up (that call loads the array), repeated calls leave
+the device's free memory, as cudaMemGetInfo reports it, unchanged.  The file
+is collected after every other test and passes both alone in a fresh process
+and after the rest of the suite.
 """
 import ctypes as C
 
@@ -93,3 +96,44 @@ def test_noalloc_rejects_window_beyond_its_array():
     assert st == _abi.H3_ERR_UNSUPPORTED and info.launches == 0
     st, info = _call_noalloc(send, recv, T, P, H, D, W, 14336 - 16)
     assert st == _abi.H3_ERR_WINDOW and info.launches == 0
+
+
+def test_noalloc_calls_leave_device_memory_unchanged():
+    """The point of the entry point: once set up, calls change no device
+    memory use.  Every buffer is allocated first and one round of calls loads
+    the array and the kernels; after that, two more rounds of both shapes must
+    leave cudaMemGetInfo's free bytes exactly as they were, and still match
+    the staged call."""
+    shapes = [(1000, 3, 56, 128, 6, 7 * 14336 + 100, 21), (777, 4, 56, 128, 8, 0, 22)]
+    cases = []
+    for T, P, H, D, W, window_bytes, seed in shapes:
+        full, send = _case(T, P, H, D, W, seed)
+        got = rr.alloc_head_side(T, P, H, D, W, DEV)
+        want = rr.alloc_head_side(T, P, H, D, W, DEV)
+        window = torch.empty(window_bytes or STATIC_WINDOW_BYTES, dtype=torch.uint8, device=DEV)
+        rr.seq_to_head_staged(send, want, window)
+        cases.append((T, P, H, D, W, window_bytes, full, send, got, want))
+
+    def one_round():
+        for T, P, H, D, W, window_bytes, _, send, got, _ in cases:
+            st, _ = _call_noalloc(send, got, T, P, H, D, W, window_bytes)
+            assert st == _abi.H3_OK, _abi.describe(st)
+
+    def stale_outputs():
+        for case in cases:
+            for g in case[8]:
+                g.view(torch.int16).fill_(0x5A5A)  # must be overwritten
+
+    one_round()  # set-up: the array and the kernels are loaded here
+    stale_outputs()  # and the fill kernel, before the measurement
+    torch.cuda.synchronize()
+    free_before, _ = torch.cuda.mem_get_info()
+    for _ in range(2):
+        stale_outputs()
+        one_round()
+    torch.cuda.synchronize()
+    free_after, _ = torch.cuda.mem_get_info()
+    assert free_after == free_before, (free_before, free_after)
+    for T, P, H, D, W, _, _, _, got, want in cases:
+        for j in range(W):
+            assert gu.same_bits(got[j], want[j]), f"rank {j}"
