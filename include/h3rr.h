@@ -34,9 +34,9 @@
  *     token offsets ts_r; head-side buffers may be views into one tensor.
  *   - Pointer arrays (send[], recv[], partials[], out[]) are HOST arrays of
  *     `world` DEVICE pointers; they are read during the call only.  The
- *     library allocates no device memory (one file-scope 16 MiB window, see
- *     h3_seq_to_head_staged_noalloc, aside) and keeps no caller pointer after
- *     return.
+ *     library allocates no device memory and keeps no caller pointer after
+ *     return.  (One file-scope 16 MiB window aside: the first
+ *     h3_seq_to_head_staged_noalloc call in a context loads it.)
  *   - The caller owns every buffer.  Outputs must not overlap any input or
  *     any other output (outputs keep storage of their own); overlap is
  *     detected and rejected.
@@ -51,9 +51,9 @@
  *     block and kernel variant.
  *   - Thread-safe, and no environment variables are read.  State kept across
  *     calls: per-device caches (SM count, resident CTAs per kernel, the
- *     shared-memory opt-in, the static window's address), each thread's last
- *     CUDA error, the device-side counters of expired bounded waits, and the
- *     peer mappings h3_ipc_open holds until h3_ipc_close.
+ *     shared-memory opt-in, the static window's address per context), each
+ *     thread's last CUDA error, the device-side counters of expired bounded
+ *     waits, and the peer mappings h3_ipc_open holds until h3_ipc_close.
  */
 #ifndef H3RR_H
 #define H3RR_H
@@ -78,7 +78,7 @@ typedef enum h3_status {
     H3_ERR_INVALID_ARG = 1,      /* NULL pointer, negative size, overlapping outputs, bad segments */
     H3_ERR_EMPTY_PARTITION = 2,  /* world > tokens or world > heads: some rank would own nothing */
     H3_ERR_MISALIGNED = 3,       /* a pointer or a contiguous run is not 16-byte aligned */
-    H3_ERR_WINDOW = 4,           /* one plane of one rank does not fit in window_bytes */
+    H3_ERR_WINDOW = 4,           /* window_bytes cannot hold the data of one token */
     H3_ERR_UNSUPPORTED = 5,      /* world > H3RR_MAX_WORLD, or a size beyond the kernels' index range */
     H3_ERR_CUDA = 6              /* the CUDA runtime reported an error while launching */
 } h3_status;
@@ -94,7 +94,7 @@ typedef enum h3_status {
 
 typedef struct h3_exec_info {
     int32_t launches;            /* kernel launches enqueued by the call */
-    int32_t chunks;              /* plane chunks: 1 unchunked, P in chunked mode */
+    int32_t chunks;              /* chunks: 1 unchunked, P * (token chunks per plane) in chunked mode */
     int32_t grid;                /* CTAs per launch */
     int32_t block;               /* threads per CTA */
     int32_t variant;             /* H3_VARIANT_* */
@@ -177,16 +177,36 @@ H3RR_API h3_status h3_partition(int64_t n_tokens, int32_t n_heads, int32_t world
  *   n_tokens T, planes P (3 = QKV, 4 = QKVG, 1 = a single operand),
  *   n_heads H, head_dim D, world W.
  *   window_bytes : 0 = one launch over all planes.  > 0 = chunked mode (FastVideo
- *                  PR #1807, "Problem and behavior"): one launch per plane p,
- *                  and both the largest per-rank send slice of one plane
- *                  (max_r T_r*H*D*2) and the largest per-rank receive slice
- *                  (max_j T*H_j*D*2) must be <= window_bytes, else
- *                  H3_ERR_WINDOW.  The result is identical either way.
+ *                  PR #1807, "Problem and behavior"): one batch plane p per
+ *                  launch, as long as the largest per-rank send slice of one
+ *                  plane (max_r T_r*H*D*2) and the largest per-rank receive
+ *                  slice (max_j T*H_j*D*2) are <= window_bytes.  A plane larger
+ *                  than that is split by tokens: k launches per plane, launch
+ *                  c moving local tokens [c*L, c*L + L) of every rank's range
+ *                  (fewer in the last), with k the fewest chunks and L the
+ *                  equal length for which L*H*D*2 <= window_bytes and
+ *                  W*L*max_j(H_j)*D*2 <= window_bytes (h3_relayout_chunk_plan
+ *                  reports k and L).  H3_ERR_WINDOW only if not even L = 1
+ *                  fits.  The result is identical either way.
  */
 H3RR_API h3_status h3_seq_to_head(const void* const* send, void* const* recv,
                          int64_t n_tokens, int32_t planes, int32_t n_heads,
                          int32_t head_dim, int32_t world, int64_t window_bytes,
                          void* stream, h3_exec_info* info);
+
+/*
+ * h3_relayout_chunk_plan - host only: how the chunked relayouts (and the
+ * h3_*_rank relayouts) cut their work under window_bytes.
+ *   tokens_per_chunk : out, L: tokens of each rank per launch (max_r T_r when
+ *                      a whole plane fits the window or window_bytes == 0).
+ *   chunks           : out, launches of a one-GPU call: 1 if window_bytes == 0,
+ *                      else planes * k (k token chunks per plane).
+ * Errors as h3_seq_to_head's argument checks (H3_ERR_EMPTY_PARTITION,
+ * H3_ERR_WINDOW, H3_ERR_INVALID_ARG on NULL outputs or non-positive sizes).
+ */
+H3RR_API h3_status h3_relayout_chunk_plan(int64_t n_tokens, int32_t planes, int32_t n_heads,
+                                          int32_t head_dim, int32_t world, int64_t window_bytes,
+                                          int64_t* tokens_per_chunk, int64_t* chunks);
 
 /*
  * h3_head_to_seq - inverse head->sequence relayout ("Distributed H3
@@ -359,7 +379,8 @@ H3RR_API h3_status h3_head_to_seq_staged(const void* const* send, void* const* r
 
 /*
  * h3_seq_to_head_staged_noalloc - h3_seq_to_head_staged with a window that
- * lives inside the library, so the call allocates no device memory at all.
+ * lives inside the library, so that, once set up (below), a call allocates
+ * no device memory at all.
  * The pages have no counterpart to this entry point; it exists for callers
  * that cannot allocate device memory themselves: for example a plugin that
  * only receives tensors from a host framework whose caching allocator owns
@@ -368,9 +389,8 @@ H3RR_API h3_status h3_head_to_seq_staged(const void* const* send, void* const* r
  * inputs and outputs; only the staging window is provided here.
  *
  * The window is a file-scope device array of H3RR_STATIC_WINDOW_BYTES
- * (16 MiB).  Every GPU that loads the library holds that array until the
- * process exits.  The call neither allocates nor frees device memory, and
- * calls no allocating library routine.
+ * (16 MiB).  The call never calls cudaMalloc or cudaFree, nor any allocating
+ * library routine.
  *
  *   window_bytes : how much of the array to use, 0 = all of it.  Values
  *                  above H3RR_STATIC_WINDOW_BYTES (or negative) are rejected
@@ -379,9 +399,18 @@ H3RR_API h3_status h3_head_to_seq_staged(const void* const* send, void* const* r
  *                  H3_ERR_WINDOW.
  *   Other arguments, layouts, results and errors as h3_seq_to_head_staged.
  *
- * The first call on a device looks up the array's device address (one
- * cudaGetSymbolAddress with that device current, kept for later calls); make
- * that first call before any stream capture.  Every call on a device shares
+ * The first call on a device (more exactly, in each CUDA context: again after
+ * cudaDeviceReset) sets the entry point up: it looks up the array's device
+ * address with cudaGetSymbolAddress, with that device current, and keeps it
+ * for later calls in that context.  Under CUDA's default lazy module loading
+ * that lookup is also when the runtime loads the array onto the device, and
+ * the load reserves the 16 MiB there: the first call can therefore fail with
+ * H3_ERR_CUDA (h3_last_cuda_error: cudaErrorMemoryAllocation) when the
+ * device is full, and it may synchronise.  Only later calls allocate
+ * nothing.  So make the first call early: before a caching allocator reserves
+ * its whole budget, and before any stream capture.  From then on the device
+ * holds the array until the process exits (with eager module loading, every
+ * device the process uses holds it from the start).  Every call on a device shares
  * the one array and leaves its last chunk in it: nothing in it needs to
  * start at zero, because each chunk is written in full before it is read.
  * Calls that overlap on the GPU (for example on two streams without ordering
@@ -457,7 +486,8 @@ H3RR_API h3_status h3_bounded_wait_selftest(uint32_t polls, int32_t arrive_first
 /* Rank k's head-side buffer: recv [T, P, H_k, D] (this GPU) gets
  * recv[t, p, h, d] = send[r(t)][t - ts_{r(t)}, p, hs_k + h, d]
  * from send[world], the sequence-side buffers [T_r, P, H, D] of all ranks.
- * window_bytes as h3_seq_to_head (same check over all ranks' slices). */
+ * window_bytes as h3_seq_to_head: the same chunk plan over all ranks' slices,
+ * so that all ranks chunk alike. */
 H3RR_API h3_status h3_seq_to_head_rank(const void* const* send, void* recv, int64_t n_tokens,
                                        int32_t planes, int32_t n_heads, int32_t head_dim,
                                        int32_t world, int32_t rank, int64_t window_bytes,

@@ -37,7 +37,7 @@ __all__ = [
     "ragged_reduce_scatter", "alloc_head_side", "alloc_seq_side", "split_rows",
     "H3_VARIANT_VECTOR", "H3_VARIANT_BULK", "H3_VARIANT_REDUCE", "MAX_WORLD", "library_path",
     "bulk_wait_timeouts", "alloc_reduce_outputs", "seq_to_head_staged", "head_to_seq_staged",
-    "staged_plan", "H3_VARIANT_STAGED", "ragged_all_gather", "H3_VARIANT_GATHER",
+    "staged_plan", "relayout_chunk_plan", "H3_VARIANT_STAGED", "ragged_all_gather", "H3_VARIANT_GATHER",
     "seq_to_head_layout", "head_to_seq_layout", "H3_LAYOUT_SEQ_PLANE_MAJOR",
     "H3_LAYOUT_HEAD_PLANE_MAJOR", "ragged_reduce_scatter_gated", "PreparedRelayout", "H3_LAUNCH_SERIAL",
     "PreparedReduceScatter", "prepare_seq_to_head", "prepare_head_to_seq",
@@ -284,6 +284,19 @@ def staged_plan(n_tokens: int, planes: int, n_heads: int, head_dim: int, window_
     st = _abi.lib.h3_staged_plan(int(n_tokens), int(planes), int(n_heads), int(head_dim),
                                  int(window_bytes), C.byref(n), C.byref(k))
     _abi.check(st, "h3_staged_plan")
+    return int(n.value), int(k.value)
+
+
+def relayout_chunk_plan(n_tokens: int, planes: int, n_heads: int, head_dim: int, world: int,
+                        window_bytes: int):
+    """(tokens of each rank per launch, launches) of a chunked relayout
+    (``h3_relayout_chunk_plan``, host only): one batch plane per launch, a
+    plane larger than the window split into equal token chunks."""
+    n = C.c_int64(0)
+    k = C.c_int64(0)
+    st = _abi.lib.h3_relayout_chunk_plan(int(n_tokens), int(planes), int(n_heads), int(head_dim),
+                                         int(world), int(window_bytes), C.byref(n), C.byref(k))
+    _abi.check(st, "h3_relayout_chunk_plan")
     return int(n.value), int(k.value)
 
 

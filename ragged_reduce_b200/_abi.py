@@ -154,6 +154,9 @@ def _load() -> C.CDLL:
     lib.h3_staged_plan.restype = C.c_int
     lib.h3_staged_plan.argtypes = [C.c_int64, C.c_int32, C.c_int32, C.c_int32, C.c_int64,
                                    _i64p, _i64p]
+    lib.h3_relayout_chunk_plan.restype = C.c_int
+    lib.h3_relayout_chunk_plan.argtypes = [C.c_int64, C.c_int32, C.c_int32, C.c_int32, C.c_int32,
+                                           C.c_int64, _i64p, _i64p]
     lib.h3_last_cuda_error.restype = C.c_int32
     lib.h3_last_cuda_error.argtypes = [C.POINTER(C.c_char_p)]
     lib.h3_bulk_wait_timeouts.restype = C.c_int

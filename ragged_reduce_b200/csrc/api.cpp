@@ -146,14 +146,15 @@ h3_status relayout(bool seq_to_head, const void* const* send, void* const* recv,
     const uint64_t head_bytes = uint64_t(head_dim) * 2;
 
     // Chunked mode (FastVideo PR #1807, "Problem and behavior"): one batch
-    // plane per launch; one plane's per-rank send and receive slices must
-    // both fit in the window.
+    // plane per launch, each rank's send and receive slices within the
+    // window; a plane too large for the window is split by tokens.
     const bool chunked = window_bytes > 0;
+    RelayoutChunks ch;
+    ch.tokens = ts.largest();
     if (chunked) {
-        const uint64_t seq_plane = uint64_t(ts.largest()) * row_bytes;
-        const uint64_t head_plane = uint64_t(n_tokens) * uint64_t(hs.largest()) * head_bytes;
-        if (seq_plane > uint64_t(window_bytes) || head_plane > uint64_t(window_bytes))
-            return H3_ERR_WINDOW;
+        st = plan_relayout_chunks(ts, hs, n_tokens, row_bytes, head_bytes, window_bytes, &ch);
+        if (st != H3_OK)
+            return st;
     }
 
     RelayoutArgs a;
@@ -186,29 +187,38 @@ h3_status relayout(bool seq_to_head, const void* const* send, void* const* recv,
         if (!relayout_bulk_fits(a, device))
             return H3_ERR_UNSUPPORTED;  // a row does not fit the shared-memory ring
     }
-    const int chunks = chunked ? planes : 1;
+    const int plane_groups = chunked ? planes : 1;
     const int per_launch = chunked ? 1 : planes;
+    const int chunks = int(plane_groups * ch.per_plane);
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     LaunchShape shape;
     int launched = 0;
     const bool programmatic = programmatic_launch(cfg);
-    for (int c = 0; c < chunks; ++c) {
-        a.plane0 = c * per_launch;
-        a.nplanes = per_launch;
-        a.rows = int32_t(n_tokens * per_launch);
-        // Planes are disjoint: a later plane's launch depends on nothing the
-        // previous one does and only has to finish after it.
-        a.wait_late = c > 0 ? 1 : 0;
-        const cudaError_t err = launch_relayout(seq_to_head, a, variant, ctas_per_sm, s, &shape,
-                                                layout != 0, programmatic);
-        if (err != cudaSuccess) {
-            if (info) {
-                info->launches = launched;
-                info->chunks = chunks;
+    for (int g = 0; g < plane_groups; ++g) {
+        for (int64_t c = 0; c < ch.per_plane; ++c) {
+            int64_t cq = 0, cm = 0, t0 = 0;
+            chunk_split(ts, ch, c, &cq, &cm, &t0);
+            a.cq = int32_t(cq);
+            a.cm = int32_t(cm);
+            a.t0 = int32_t(t0);
+            a.plane0 = g * per_launch;
+            a.nplanes = per_launch;
+            a.rows = int32_t((cq * world + cm) * per_launch);
+            // Chunks are disjoint rows of every buffer: a later chunk's launch
+            // depends on nothing the previous one does and only has to
+            // finish after it.
+            a.wait_late = launched > 0 ? 1 : 0;
+            const cudaError_t err = launch_relayout(seq_to_head, a, variant, ctas_per_sm, s,
+                                                    &shape, layout != 0, programmatic);
+            if (err != cudaSuccess) {
+                if (info) {
+                    info->launches = launched;
+                    info->chunks = chunks;
+                }
+                return cuda_failure(err);
             }
-            return cuda_failure(err);
+            ++launched;
         }
-        ++launched;
     }
     if (info) {
         info->launches = launched;
@@ -357,6 +367,30 @@ h3_status h3_staged_plan(int64_t n_tokens, int32_t planes, int32_t n_heads, int3
 }
 
 
+h3_status h3_relayout_chunk_plan(int64_t n_tokens, int32_t planes, int32_t n_heads,
+                                 int32_t head_dim, int32_t world, int64_t window_bytes,
+                                 int64_t* tokens_per_chunk, int64_t* chunks)
+{
+    if (!tokens_per_chunk || !chunks || planes < 1 || head_dim < 1 || window_bytes < 0)
+        return H3_ERR_INVALID_ARG;
+    const h3_status st = check_world(n_tokens, n_heads, world);
+    if (st != H3_OK)
+        return st;
+    const Split ts = make_split(n_tokens, world);
+    const Split hs = make_split(n_heads, world);
+    RelayoutChunks ch;
+    ch.tokens = ts.largest();
+    if (window_bytes > 0) {
+        const h3_status pst = plan_relayout_chunks(ts, hs, n_tokens, uint64_t(n_heads) * head_dim * 2,
+                                                   uint64_t(head_dim) * 2, window_bytes, &ch);
+        if (pst != H3_OK)
+            return pst;
+    }
+    *tokens_per_chunk = ch.tokens;
+    *chunks = window_bytes > 0 ? int64_t(planes) * ch.per_plane : 1;
+    return H3_OK;
+}
+
 int32_t h3_abi_version(void) { return H3RR_ABI_VERSION; }
 
 int32_t h3_last_cuda_error(const char** message)
@@ -373,7 +407,7 @@ const char* h3_status_string(h3_status status)
         case H3_ERR_INVALID_ARG: return "invalid argument";
         case H3_ERR_EMPTY_PARTITION: return "empty token or head partition";
         case H3_ERR_MISALIGNED: return "pointer or run not 16-byte aligned";
-        case H3_ERR_WINDOW: return "the data of one launch does not fit in the byte window";
+        case H3_ERR_WINDOW: return "the byte window cannot hold the data of one token";
         case H3_ERR_UNSUPPORTED: return "unsupported size or world";
         case H3_ERR_CUDA: return "CUDA launch error";
     }

@@ -106,4 +106,22 @@ __device__ __forceinline__ int32_t split_start(int32_t i, int32_t q, int32_t m)
     return i * q + (i < m ? i : m);
 }
 
+// Token unit v of a launch that covers, for every rank r, the local tokens
+// [t0, t0 + cq + (r < cm)) of r's range (a chunk of the token split (tq, tm);
+// cq = tq, cm = tm, t0 = 0 for all tokens): the owning rank s, its local
+// token tl and the global token t.
+struct ChunkToken {
+    int32_t s, tl, t;
+};
+
+__device__ __forceinline__ ChunkToken chunk_token(int32_t v, int32_t cq, int32_t cm, int32_t t0,
+                                                  int32_t tq, int32_t tm)
+{
+    ChunkToken k;
+    k.s = split_owner(v, cq, cm);
+    k.tl = t0 + v - split_start(k.s, cq, cm);
+    k.t = split_start(k.s, tq, tm) + k.tl;
+    return k;
+}
+
 }  // namespace h3rr

@@ -48,6 +48,32 @@ struct Split {
 
 Split make_split(int64_t n, int32_t w);
 
+// Token chunks of a chunked relayout (FastVideo PR #1807, "Problem and
+// behavior": one batch plane at a time through a byte window).  Each plane is
+// moved in `per_plane` launches; launch c covers local tokens
+// [c*tokens, c*tokens + tokens) of every rank (fewer in the last one), so
+// every launch is still one all-to-all over all ranks.  per_plane is 1 when a
+// whole plane fits the window.
+struct RelayoutChunks {
+    int64_t per_plane = 1;
+    int64_t tokens = 0;
+};
+
+// The chunking of a relayout over `window_bytes` (> 0): one plane per chunk
+// if every rank's send slice of a plane (T_r*row_bytes) and receive slice
+// (T*H_j*head_bytes) fit; otherwise the fewest equal token chunks whose
+// per-rank send slice (L*row_bytes) and receive slice (W*L*H_j*head_bytes)
+// fit.  H3_ERR_WINDOW if not even one token of every rank fits.
+h3_status plan_relayout_chunks(const Split& ts, const Split& hs, int64_t n_tokens,
+                               uint64_t row_bytes, uint64_t head_bytes, int64_t window_bytes,
+                               RelayoutChunks* out);
+
+// Token split of chunk c: rank r holds cq + (r < cm) tokens of the chunk,
+// local tokens t0 .. of its range.  Full chunks are (tokens, 0); the last
+// chunk is what remains of the quotient/remainder split, (q - t0, m).
+void chunk_split(const Split& ts, const RelayoutChunks& ch, int64_t c, int64_t* cq, int64_t* cm,
+                 int64_t* t0);
+
 // Clip packed segments to [ts, te) and rebase; returns the piece count.
 int32_t clip_segments(const int64_t* bounds, int32_t n_segs, int64_t ts, int64_t te,
                       int64_t* local_bounds, int32_t* seg_ids);
@@ -70,8 +96,9 @@ struct RelayoutArgs {
     int32_t W;
     int32_t plane0;
     int32_t nplanes;
-    int32_t rows;            // T * nplanes
+    int32_t rows;            // tokens of the launch * nplanes
     int32_t tq, tm;          // token split
+    int32_t cq, cm, t0;      // the launch's tokens: cq + (r < cm) of rank r from local token t0
     int32_t hq, hm;          // head split
     int32_t row_vecs;        // H * D * 2 / 16
     int32_t head_vecs;       // D * 2 / 16
@@ -132,8 +159,9 @@ struct PullArgs {
     int32_t P;
     int32_t plane0;
     int32_t nplanes;
-    int32_t rows;                // T * nplanes
+    int32_t rows;                // tokens of the launch * nplanes
     int32_t tq, tm;              // token split
+    int32_t cq, cm, t0;          // the launch's tokens, as RelayoutArgs
     int32_t row_vecs;            // H * D * 2 / 16
     int32_t run_vecs;            // H_k * D * 2 / 16
     int32_t col0_vecs;           // hs * D * 2 / 16

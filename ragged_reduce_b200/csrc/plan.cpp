@@ -22,6 +22,46 @@ Split make_split(int64_t n, int32_t w)
     return s;
 }
 
+h3_status plan_relayout_chunks(const Split& ts, const Split& hs, int64_t n_tokens,
+                               uint64_t row_bytes, uint64_t head_bytes, int64_t window_bytes,
+                               RelayoutChunks* out)
+{
+    const uint64_t window = uint64_t(window_bytes);
+    const int64_t tmax = ts.largest();
+    const uint64_t head_run = uint64_t(hs.largest()) * head_bytes;  // one token of the widest head rank
+    if (uint64_t(tmax) * row_bytes <= window && uint64_t(n_tokens) * head_run <= window) {
+        out->per_plane = 1;
+        out->tokens = tmax;
+        return H3_OK;
+    }
+    // A full chunk sends L rows from every rank and gives every head rank L
+    // tokens from each of the W ranks.
+    const uint64_t by_send = window / row_bytes;
+    const uint64_t by_recv = window / (uint64_t(ts.w) * head_run);
+    const uint64_t most = by_send < by_recv ? by_send : by_recv;
+    if (most < 1)
+        return H3_ERR_WINDOW;
+    // Fewest chunks, then equal lengths: ceil(tmax / L) is again k, so every
+    // chunk but the last is full and the last is not empty.
+    const int64_t k = (tmax + int64_t(most) - 1) / int64_t(most);
+    out->per_plane = k;
+    out->tokens = (tmax + k - 1) / k;
+    return H3_OK;
+}
+
+void chunk_split(const Split& ts, const RelayoutChunks& ch, int64_t c, int64_t* cq, int64_t* cm,
+                 int64_t* t0)
+{
+    *t0 = c * ch.tokens;
+    if (c + 1 < ch.per_plane) {
+        *cq = ch.tokens;
+        *cm = 0;
+    } else {
+        *cq = ts.q - *t0;
+        *cm = ts.m;
+    }
+}
+
 int32_t clip_segments(const int64_t* bounds, int32_t n_segs, int64_t ts, int64_t te,
                       int64_t* local_bounds, int32_t* seg_ids)
 {

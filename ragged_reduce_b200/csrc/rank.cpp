@@ -47,11 +47,11 @@ void fill_info(h3_exec_info* info, int launches, int chunks, const LaunchShape& 
 }
 
 // Checks of a relayout rank call; on success *chunked tells whether the
-// window asks for one plane per launch.
+// window asks for one plane per launch and *ch how each plane is split.
 h3_status check_relayout_rank(bool seq_to_head, const void* const* send, const void* recv,
                               int64_t n_tokens, int32_t planes, int32_t n_heads, int32_t head_dim,
                               int32_t world, int32_t rank, int64_t window_bytes,
-                              const h3_launch_config* cfg, bool* chunked)
+                              const h3_launch_config* cfg, bool* chunked, RelayoutChunks* ch)
 {
     if (window_bytes < 0)
         return H3_ERR_INVALID_ARG;
@@ -93,15 +93,13 @@ h3_status check_relayout_rank(bool seq_to_head, const void* const* send, const v
     st = check_no_overlap(send, in_bytes, world, out, &out_bytes, 1);
     if (st != H3_OK)
         return st;
-    // The window bounds every rank's per-plane slices, exactly as in the
-    // one-GPU call, so that all ranks chunk alike.
+    // The window bounds every rank's slices, exactly as in the one-GPU call,
+    // so that all ranks chunk alike.
     *chunked = window_bytes > 0;
-    if (*chunked) {
-        const uint64_t seq_plane = uint64_t(ts.largest()) * row_bytes;
-        const uint64_t head_plane = uint64_t(n_tokens) * uint64_t(hs.largest()) * head_bytes;
-        if (seq_plane > uint64_t(window_bytes) || head_plane > uint64_t(window_bytes))
-            return H3_ERR_WINDOW;
-    }
+    ch->per_plane = 1;
+    ch->tokens = ts.largest();
+    if (*chunked)
+        return plan_relayout_chunks(ts, hs, n_tokens, row_bytes, head_bytes, window_bytes, ch);
     return H3_OK;
 }
 
@@ -168,8 +166,9 @@ h3_status h3_seq_to_head_rank(const void* const* send, void* recv, int64_t n_tok
 {
     clear_info(info);
     bool chunked = false;
+    RelayoutChunks ch;
     h3_status st = check_relayout_rank(true, send, recv, n_tokens, planes, n_heads, head_dim, world,
-                                       rank, window_bytes, cfg, &chunked);
+                                       rank, window_bytes, cfg, &chunked, &ch);
     if (st != H3_OK)
         return st;
     const Split ts = make_split(n_tokens, world);
@@ -188,24 +187,34 @@ h3_status h3_seq_to_head_rank(const void* const* send, void* recv, int64_t n_tok
     a.row_vecs = int32_t(int64_t(n_heads) * head_vecs);
     a.run_vecs = int32_t(hs.size(rank) * head_vecs);
     a.col0_vecs = int32_t(hs.start(rank) * head_vecs);
-    const int chunks = chunked ? planes : 1;
+    const int plane_groups = chunked ? planes : 1;
     const int per_launch = chunked ? 1 : planes;
+    const int chunks = int(plane_groups * ch.per_plane);
     const bool programmatic = programmatic_launch(cfg);
     LaunchShape shape;
-    for (int c = 0; c < chunks; ++c) {
-        a.plane0 = c * per_launch;
-        a.nplanes = per_launch;
-        a.rows = int32_t(n_tokens * per_launch);
-        a.wait_late = c > 0 ? 1 : 0;  // planes are disjoint (see h3_launch_config)
-        const cudaError_t err = launch_pull_seq_to_head(a, cfg ? cfg->ctas_per_sm : 0,
-                                                        static_cast<cudaStream_t>(stream), &shape,
-                                                        programmatic);
-        if (err != cudaSuccess) {
-            fill_info(info, c, chunks, shape, per_launch);
-            return fail(err);
+    int launched = 0;
+    for (int g = 0; g < plane_groups; ++g) {
+        for (int64_t c = 0; c < ch.per_plane; ++c) {
+            int64_t cq = 0, cm = 0, t0 = 0;
+            chunk_split(ts, ch, c, &cq, &cm, &t0);
+            a.cq = int32_t(cq);
+            a.cm = int32_t(cm);
+            a.t0 = int32_t(t0);
+            a.plane0 = g * per_launch;
+            a.nplanes = per_launch;
+            a.rows = int32_t((cq * world + cm) * per_launch);
+            a.wait_late = launched > 0 ? 1 : 0;  // chunks are disjoint (see h3_launch_config)
+            const cudaError_t err = launch_pull_seq_to_head(a, cfg ? cfg->ctas_per_sm : 0,
+                                                            static_cast<cudaStream_t>(stream),
+                                                            &shape, programmatic);
+            if (err != cudaSuccess) {
+                fill_info(info, launched, chunks, shape, per_launch);
+                return fail(err);
+            }
+            ++launched;
         }
     }
-    fill_info(info, chunks, chunks, shape, per_launch);
+    fill_info(info, launched, chunks, shape, per_launch);
     return H3_OK;
 }
 
@@ -216,8 +225,9 @@ h3_status h3_head_to_seq_rank(const void* const* send, void* recv, int64_t n_tok
 {
     clear_info(info);
     bool chunked = false;
+    RelayoutChunks ch;
     h3_status st = check_relayout_rank(false, send, recv, n_tokens, planes, n_heads, head_dim,
-                                       world, rank, window_bytes, cfg, &chunked);
+                                       world, rank, window_bytes, cfg, &chunked, &ch);
     if (st != H3_OK)
         return st;
     const Split ts = make_split(n_tokens, world);
@@ -243,25 +253,41 @@ h3_status h3_head_to_seq_rank(const void* const* send, void* recv, int64_t n_tok
     a.hm = int32_t(hs.m);
     a.row_vecs = int32_t(int64_t(n_heads) * head_bytes / kVecBytes);
     a.head_vecs = int32_t(head_bytes / kVecBytes);
-    const int chunks = chunked ? planes : 1;
+    const int plane_groups = chunked ? planes : 1;
     const int per_launch = chunked ? 1 : planes;
+    const int chunks = int(plane_groups * ch.per_plane);
     const bool programmatic = programmatic_launch(cfg);
     const int variant = cfg ? cfg->variant : 0;
     LaunchShape shape;
-    for (int c = 0; c < chunks; ++c) {
-        a.plane0 = c * per_launch;
-        a.nplanes = per_launch;
-        a.rows = int32_t(t_rows * per_launch);
-        a.wait_late = c > 0 ? 1 : 0;
-        const cudaError_t err =
-            launch_relayout(false, a, variant, cfg ? cfg->ctas_per_sm : 0,
-                            static_cast<cudaStream_t>(stream), &shape, false, programmatic);
-        if (err != cudaSuccess) {
-            fill_info(info, c, chunks, shape, per_launch);
-            return fail(err);
+    int launched = 0;
+    for (int g = 0; g < plane_groups; ++g) {
+        for (int64_t c = 0; c < ch.per_plane; ++c) {
+            // This rank's tokens of chunk c of the plan all ranks share; the
+            // last chunk may hold none of them.
+            const int64_t t0 = c * ch.tokens;
+            int64_t n = t_rows - t0;
+            if (n > ch.tokens)
+                n = ch.tokens;
+            if (n <= 0)
+                continue;
+            a.cq = int32_t(n);
+            a.cm = 0;
+            a.t0 = int32_t(t0);
+            a.plane0 = g * per_launch;
+            a.nplanes = per_launch;
+            a.rows = int32_t(n * per_launch);
+            a.wait_late = launched > 0 ? 1 : 0;
+            const cudaError_t err =
+                launch_relayout(false, a, variant, cfg ? cfg->ctas_per_sm : 0,
+                                static_cast<cudaStream_t>(stream), &shape, false, programmatic);
+            if (err != cudaSuccess) {
+                fill_info(info, launched, chunks, shape, per_launch);
+                return fail(err);
+            }
+            ++launched;
         }
     }
-    fill_info(info, chunks, chunks, shape, per_launch);
+    fill_info(info, launched, chunks, shape, per_launch);
     return H3_OK;
 }
 

@@ -82,10 +82,10 @@ __global__ void __launch_bounds__(NT) relayout_vec_kernel(const __grid_constant_
         for (int r = 0; r < ROWS; ++r) {
             rv[r] = i0 + r < a.rows;
             const int32_t ii = int32_t(rv[r] ? i0 + r : i0);
-            const int32_t t = ii / a.nplanes;
-            const int32_t p = a.plane0 + (ii - t * a.nplanes);
-            const int32_t s = split_owner(t, a.tq, a.tm);
-            const int32_t tl = t - split_start(s, a.tq, a.tm);
+            const int32_t u = ii / a.nplanes;  // token unit of the launch
+            const int32_t p = a.plane0 + (ii - u * a.nplanes);
+            const ChunkToken k = chunk_token(u, a.cq, a.cm, a.t0, a.tq, a.tm);
+            const int32_t s = k.s, tl = k.tl, t = k.t;
             if constexpr (kLayout) {
                 // plane-major sides: plane p is a contiguous block of T (or T_s) rows
                 const int32_t ts_len = a.tq + (s < a.tm ? 1 : 0);
@@ -134,10 +134,10 @@ __global__ void __launch_bounds__(kGenericThreads) relayout_generic_kernel(const
     pdl_allow_dependents();
     for (int64_t i64 = blockIdx.x; i64 < a.rows; i64 += gridDim.x) {
         const int32_t i = int32_t(i64);
-        const int32_t t = i / a.nplanes;
-        const int32_t p = a.plane0 + (i - t * a.nplanes);
-        const int32_t s = split_owner(t, a.tq, a.tm);
-        const int32_t tl = t - split_start(s, a.tq, a.tm);
+        const int32_t u = i / a.nplanes;  // token unit of the launch
+        const int32_t p = a.plane0 + (i - u * a.nplanes);
+        const ChunkToken k = chunk_token(u, a.cq, a.cm, a.t0, a.tq, a.tm);
+        const int32_t s = k.s, tl = k.tl, t = k.t;
         int64_t g = int64_t(t) * a.P + p;
         int64_t srow_index = int64_t(tl) * a.P + p;
         if constexpr (kLayout) {
@@ -202,12 +202,11 @@ __global__ void __launch_bounds__(32) relayout_bulk_kernel(const __grid_constant
     // Row n of this CTA -> (sequence-side row address, head-side row index g).
     auto locate = [&](int64_t n, char** seq_row, int64_t* g) {
         const int32_t i = int32_t(blockIdx.x + n * gridDim.x);
-        const int32_t t = i / a.nplanes;
-        const int32_t p = a.plane0 + (i - t * a.nplanes);
-        const int32_t s = split_owner(t, a.tq, a.tm);
-        const int32_t tl = t - split_start(s, a.tq, a.tm);
-        *seq_row = a.seq[s] + (int64_t(tl) * a.P + p) * row_bytes;
-        *g = int64_t(t) * a.P + p;
+        const int32_t u = i / a.nplanes;  // token unit of the launch
+        const int32_t p = a.plane0 + (i - u * a.nplanes);
+        const ChunkToken k = chunk_token(u, a.cq, a.cm, a.t0, a.tq, a.tm);
+        *seq_row = a.seq[k.s] + (int64_t(k.tl) * a.P + p) * row_bytes;
+        *g = int64_t(k.t) * a.P + p;
     };
     auto issue_load = [&](int64_t n) {
         char* seq_row;
@@ -303,12 +302,11 @@ __global__ void __launch_bounds__(NT) pull_seq_to_head_kernel(const __grid_const
             char* dst = nullptr;
             if (i64 < a.rows) {
                 const int32_t i = int32_t(i64);
-                const int32_t t = i / a.nplanes;
-                const int32_t p = a.plane0 + (i - t * a.nplanes);
-                const int32_t s = split_owner(t, a.tq, a.tm);
-                const int32_t tl = t - split_start(s, a.tq, a.tm);
-                src = a.src[s] + ((int64_t(tl) * a.P + p) * a.row_vecs + a.col0_vecs) * kVecBytes;
-                dst = a.dst + (int64_t(t) * a.P + p) * a.run_vecs * kVecBytes;
+                const int32_t u = i / a.nplanes;  // token unit of the launch
+                const int32_t p = a.plane0 + (i - u * a.nplanes);
+                const ChunkToken k = chunk_token(u, a.cq, a.cm, a.t0, a.tq, a.tm);
+                src = a.src[k.s] + ((int64_t(k.tl) * a.P + p) * a.row_vecs + a.col0_vecs) * kVecBytes;
+                dst = a.dst + (int64_t(k.t) * a.P + p) * a.run_vecs * kVecBytes;
             }
             s_src[threadIdx.x] = src;
             s_dst[threadIdx.x] = dst;
@@ -348,12 +346,11 @@ __global__ void __launch_bounds__(NT) pull_seq_to_head_long_kernel(const __grid_
     pdl_allow_dependents();
     for (int64_t i64 = blockIdx.x; i64 < a.rows; i64 += gridDim.x) {
         const int32_t i = int32_t(i64);
-        const int32_t t = i / a.nplanes;
-        const int32_t p = a.plane0 + (i - t * a.nplanes);
-        const int32_t s = split_owner(t, a.tq, a.tm);
-        const int32_t tl = t - split_start(s, a.tq, a.tm);
-        const char* src = a.src[s] + ((int64_t(tl) * a.P + p) * a.row_vecs + a.col0_vecs) * kVecBytes;
-        char* dst = a.dst + (int64_t(t) * a.P + p) * a.run_vecs * kVecBytes;
+        const int32_t u = i / a.nplanes;  // token unit of the launch
+        const int32_t p = a.plane0 + (i - u * a.nplanes);
+        const ChunkToken k = chunk_token(u, a.cq, a.cm, a.t0, a.tq, a.tm);
+        const char* src = a.src[k.s] + ((int64_t(k.tl) * a.P + p) * a.row_vecs + a.col0_vecs) * kVecBytes;
+        char* dst = a.dst + (int64_t(k.t) * a.P + p) * a.run_vecs * kVecBytes;
         for (int32_t c0 = 0; c0 < run_v; c0 += MAXV * NT) {
             Vec<VW> v[MAXV];
 #pragma unroll

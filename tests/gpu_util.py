@@ -104,3 +104,17 @@ def nan_aware_equal(got: np.ndarray, want: np.ndarray) -> np.ndarray:
     def is_nan(x):
         return ((x & 0x7F80) == 0x7F80) & ((x & 0x7F) != 0)
     return (got == want) | (is_nan(got) & is_nan(want))
+
+
+def chunk_window(kind, T, H, D, W):
+    """Window bytes for a chunked-mode test: 0 (unchunked), "plane" (exactly
+    one plane of the largest rank, one launch per plane), "sub" (half of that,
+    so every plane is split into token chunks) or "min" (one token of every
+    rank: one-token chunks)."""
+    if not kind:
+        return 0
+    tmax, hmax = -(-T // W), -(-H // W)
+    row, head = H * D * 2, D * 2
+    smallest = max(row, W * hmax * head)
+    plane = max(tmax * row, T * hmax * head)
+    return {"plane": plane, "sub": max(smallest, plane // 2), "min": smallest}[kind]

@@ -179,8 +179,9 @@ def test_relayout_argument_checks(fn):
     bad = list(recv)
     bad[2] = recv[1] + 512
     assert _relayout_status(send, bad, T, P, H, D, W, fn=fn)[0] == E.H3_ERR_INVALID_ARG
-    # window smaller than one plane of one rank (largest slice: 167 tokens x 14,336 B)
-    assert _relayout_status(send, recv, T, P, H, D, W, window=167 * 14336 - 1, fn=fn)[0] == E.H3_ERR_WINDOW
+    # a window that cannot hold one token of every rank: each head rank
+    # receives one token from each of the 6 ranks, 6 x 10 heads x 256 B
+    assert _relayout_status(send, recv, T, P, H, D, W, window=6 * 10 * 256 - 1, fn=fn)[0] == E.H3_ERR_WINDOW
     # sizes beyond the kernels' 32-bit row index
     assert _relayout_status(send, recv, 2**31, P, H, D, W, fn=fn)[0] == E.H3_ERR_UNSUPPORTED
     # a NULL pointer array
@@ -239,13 +240,69 @@ def test_bulk_timeout_query_needs_count():
 
 @needs_no_gpu
 def test_relayout_window_check_long_workload():
-    # 250k tokens over 4 ranks: one plane of one rank is exactly 896,000,000 bytes
+    # 250k tokens over 4 ranks: one plane of one rank is exactly 896,000,000
+    # bytes, so the pages' window moves one plane per launch; 16 bytes less
+    # splits every plane into two token chunks; a window below one token of
+    # every rank is refused before anything is launched.
     T, P, H, D, W = 250000, 4, 56, 128, 4
     send, recv = _layout(T, P, H, D, W)
     assert 62500 * 56 * 128 * 2 == 896_000_000
     assert 250000 * 14 * 128 * 2 == 896_000_000
-    st, info = _relayout_status(send, recv, T, P, H, D, W, window=896_000_000 - 16)
+    assert rr.relayout_chunk_plan(T, P, H, D, W, 896_000_000) == (62500, 4)
+    assert rr.relayout_chunk_plan(T, P, H, D, W, 896_000_000 - 16) == (31250, 8)
+    st, info = _relayout_status(send, recv, T, P, H, D, W, window=H * D * 2 - 16)
     assert st == _abi.H3_ERR_WINDOW and info.launches == 0
+
+
+def _expected_plan(T, P, H, D, W, window):
+    """The chunk plan restated from its definition: one plane per chunk if a
+    whole plane of every rank fits; else the fewest token chunks k, and the
+    equal length L = ceil(T_max / k), whose full chunks fit."""
+    tmax = -(-T // W)
+    hmax = -(-H // W)
+    row, head = H * D * 2, D * 2
+    if tmax * row <= window and T * hmax * head <= window:
+        return tmax, P
+    for k in range(2, tmax + 1):
+        L = -(-tmax // k)
+        if L * row <= window and W * L * hmax * head <= window:
+            return L, P * k
+    return None
+
+
+def test_relayout_chunk_plan_properties():
+    """Against the plan's definition over a grid of shapes and windows, and
+    the properties the kernels rely on: full chunks within the window, the
+    chunks cover every rank's tokens once, and the last chunk is not empty."""
+    rng = np.random.default_rng(5)
+    cases = [(250000, 4, 56, 128, 4), (250000, 4, 56, 128, 2), (32768, 3, 56, 128, 6),
+             (1000, 3, 56, 128, 8), (777, 1, 7, 64, 3), (64, 2, 56, 128, 56)]
+    for _ in range(60):
+        W = int(rng.integers(1, 9))
+        cases.append((int(rng.integers(W, 5000)), int(rng.integers(1, 5)),
+                      int(rng.integers(W, 80)), 8 * int(rng.integers(1, 40)), W))
+    for T, P, H, D, W in cases:
+        tmax, hmax = -(-T // W), -(-H // W)
+        row, head = H * D * 2, D * 2
+        smallest = max(row, W * hmax * head)
+        windows = {smallest, smallest + 16, T * row, tmax * row, tmax * row - 16,
+                   int(rng.integers(smallest, 4 * tmax * row + 1))}
+        for win in sorted(windows):
+            want = _expected_plan(T, P, H, D, W, win)
+            assert want is not None, (T, P, H, D, W, win)
+            L, chunks = rr.relayout_chunk_plan(T, P, H, D, W, win)
+            assert (L, chunks) == want, (T, P, H, D, W, win)
+            k = chunks // P
+            if k > 1:
+                assert L * row <= win and W * L * hmax * head <= win
+                assert (k - 1) * L < tmax <= k * L       # exact cover, last chunk not empty
+                # the plan is also the fewest chunks: one fewer would not fit
+                Lfew = -(-tmax // (k - 1))
+                assert Lfew * row > win or W * Lfew * hmax * head > win
+        assert rr.relayout_chunk_plan(T, P, H, D, W, 0) == (tmax, 1)
+        with pytest.raises(rr.H3Error) as e:
+            rr.relayout_chunk_plan(T, P, H, D, W, smallest - 1)
+        assert e.value.status == _abi.H3_ERR_WINDOW
 
 
 @needs_no_gpu

@@ -31,14 +31,14 @@ def _head_buffers(T, P, H, D, W, head_pm, part):
                                        (130, 2, 7, 64, 3), (50, 3, 5, 8, 5), (20, 2, 300, 128, 7),
                                        (33, 3, 56, 256, 4), (64, 3, 56, 128, 1)])
 @pytest.mark.parametrize("layout", [0, SPM, HPM, SPM | HPM])
-@pytest.mark.parametrize("chunked", [False, True])
+@pytest.mark.parametrize("chunked", [None, "plane", "sub"])
 def test_layout_matches_oracle(oracle_lib, T, P, H, D, W, layout, chunked):
     spm, hpm = bool(layout & SPM), bool(layout & HPM)
     send, part = _seq_buffers(T, P, H, D, W, spm, seed=T + W + layout)
     heads = _head_buffers(T, P, H, D, W, hpm, part)
-    window = max(part.tokens(0) * H * D * 2, T * part.heads(0) * D * 2) if chunked else 0
+    window = gu.chunk_window(chunked, T, H, D, W)
     info = rr.seq_to_head_layout(send, heads, layout, window_bytes=window)
-    assert info["launches"] == (P if chunked else 1)
+    assert info["launches"] == rr.relayout_chunk_plan(T, P, H, D, W, window)[1]
     want = oracle_lib.relayout_layout([gu.bits(s) for s in send], T, P, H, D, W, True, spm, hpm)
     for j in range(W):
         assert np.array_equal(gu.bits(heads[j]), want[j]), f"seq->head rank {j}"

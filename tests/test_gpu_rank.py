@@ -24,25 +24,30 @@ SHAPES = [  # T, P, H, D, W
 
 
 @pytest.mark.parametrize("T,P,H,D,W", SHAPES)
-@pytest.mark.parametrize("chunked", [False, True])
+@pytest.mark.parametrize("chunked", [None, "plane", "sub"])
 def test_relayout_rank_shares(oracle_lib, T, P, H, D, W, chunked):
     part = rr.partition(T, H, W)
     x = wl.random_bits((T, P, H, D), T + W, DEV)
     send = rr.split_rows(x, part.token_starts)
     addrs = [int(s.data_ptr()) for s in send]
-    window = max(part.tokens(0) * H * D * 2, T * part.heads(0) * D * 2) if chunked else 0
+    window = gu.chunk_window(chunked, T, H, D, W)
+    L, chunks = rr.relayout_chunk_plan(T, P, H, D, W, window)
     heads = [torch.empty((T, P, part.heads(k), D), dtype=torch.bfloat16, device=DEV)
              for k in range(W)]
     for k in range(W):
         info = rr.seq_to_head_rank(addrs, heads[k], k, n_heads=H, window_bytes=window)
-        assert info["launches"] == (P if chunked else 1)
+        assert info["chunks"] == chunks and info["launches"] == chunks
     want = oracle_lib.seq_to_head([gu.bits(s) for s in send], T, P, H, D, W)
     for k in range(W):
         assert np.array_equal(gu.bits(heads[k]), want[k]), (T, P, H, D, W, k)
     back_full, back = rr.alloc_seq_side(T, P, H, D, W, DEV)
     head_addrs = [int(h.data_ptr()) for h in heads]
     for k in range(W):
-        rr.head_to_seq_rank(head_addrs, back[k], k, n_tokens=T, window_bytes=window)
+        info = rr.head_to_seq_rank(head_addrs, back[k], k, n_tokens=T, window_bytes=window)
+        # launches: the chunks that hold tokens of rank k
+        per_plane = chunks // P if window else 1
+        held = sum(1 for c in range(per_plane) if c * L < part.tokens(k))
+        assert info["chunks"] == chunks and info["launches"] == (held * P if window else 1)
     assert gu.same_bits(back_full, x)
 
 

@@ -229,21 +229,88 @@ def test_separate_send_buffers_and_side_stream(oracle_lib):
 
 
 def test_chunked_plan_actually_ran():
-    """The chunked plan reports one launch per plane; an unchunked control
-    reports one launch and fails the chunked assertion."""
+    """The chunked plan reports one launch per plane; a window 16 bytes short
+    of a plane splits every plane into two token chunks; an unchunked control
+    reports one launch and fails the chunked assertion; a window that cannot
+    hold one token of every rank is refused."""
     T, P, H, D, W = 1000, 4, 56, 128, 4
     full, send, part = _seq_inputs(T, P, H, D, W, seed=3)
     plane = max(part.tokens(0) * H * D * 2, T * part.heads(0) * D * 2)
     recv = rr.alloc_head_side(T, P, H, D, W, DEV)
     info = rr.seq_to_head(send, recv, window_bytes=plane)
     assert info["chunks"] == P and info["launches"] == P and info["planes_per_launch"] == 1
+    info = rr.seq_to_head(send, recv, window_bytes=plane - 16)
+    assert info["chunks"] == 2 * P and info["launches"] == 2 * P and info["planes_per_launch"] == 1
+    assert rr.relayout_chunk_plan(T, P, H, D, W, plane - 16) == (125, 2 * P)
     control = rr.seq_to_head(send, recv, window_bytes=0)
     assert control["chunks"] == 1 and control["launches"] == 1
     with pytest.raises(AssertionError):
         assert control["launches"] == P
     with pytest.raises(rr.H3Error) as e:
-        rr.seq_to_head(send, recv, window_bytes=plane - 16)
+        rr.seq_to_head(send, recv, window_bytes=H * D * 2 - 16)
     assert e.value.status == 4  # H3_ERR_WINDOW
+
+
+# Planes larger than the window are split into token chunks (FastVideo PR
+# #1807, "Problem and behavior": transfers bounded by the window): half a
+# plane, and one token of every rank per launch; ragged tokens and heads,
+# a head rank receiving more than a token row (W x H_max > H), one token per
+# rank, narrow rows.
+SUB_PLANE = [
+    (1000, 3, 56, 128, 4),
+    (1000, 3, 56, 128, 6),
+    (777, 4, 56, 128, 8),
+    (301, 2, 16, 64, 5),
+    (130, 2, 7, 64, 3),
+    (19, 3, 56, 128, 9),
+]
+
+
+@pytest.mark.parametrize("T,P,H,D,W", SUB_PLANE)
+@pytest.mark.parametrize("kind", ["sub", "min"])
+@pytest.mark.parametrize("variant", [0, rr.H3_VARIANT_BULK])
+def test_sub_plane_chunks_match_oracle(oracle_lib, T, P, H, D, W, kind, variant):
+    full, send, part = _seq_inputs(T, P, H, D, W, seed=T * 13 + W + len(kind))
+    window = gu.chunk_window(kind, T, H, D, W)
+    L, chunks = rr.relayout_chunk_plan(T, P, H, D, W, window)
+    assert chunks > P  # every plane is split
+    recv = rr.alloc_head_side(T, P, H, D, W, DEV)
+    rr.bulk_wait_timeouts(reset=True)
+    info = rr.seq_to_head(send, recv, window_bytes=window, variant=variant)
+    assert info["chunks"] == chunks and info["launches"] == chunks
+    want = oracle_lib.seq_to_head([gu.bits(s) for s in send], T, P, H, D, W)
+    for j in range(W):
+        assert np.array_equal(gu.bits(recv[j]), want[j]), f"seq->head rank {j}"
+    back_full, back = rr.alloc_seq_side(T, P, H, D, W, DEV)
+    info = rr.head_to_seq(recv, back, window_bytes=window, variant=variant)
+    assert info["chunks"] == chunks and info["launches"] == chunks
+    want_back = oracle_lib.head_to_seq(want, T, P, H, D, W)
+    for r in range(W):
+        assert np.array_equal(gu.bits(back[r]), want_back[r]), f"head->seq rank {r}"
+    assert gu.same_bits(back_full, full)
+    assert rr.bulk_wait_timeouts() == 0
+
+
+def test_sub_plane_chunks_guard_bands():
+    """One-token chunks write nothing outside the outputs."""
+    T, P, H, D, W = 257, 3, 56, 128, 6
+    full, send, part = _seq_inputs(T, P, H, D, W, seed=41)
+    window = gu.chunk_window("min", T, H, D, W)
+    bufs, recv = [], []
+    for j in range(W):
+        b, o = gu.guarded((T, P, part.heads(j), D), DEV)
+        bufs.append(b)
+        recv.append(o)
+    rr.seq_to_head(send, recv, window_bytes=window)
+    assert all(gu.guards_intact(b) for b in bufs)
+    sbufs, back = [], []
+    for r in range(W):
+        b, o = gu.guarded((part.tokens(r), P, H, D), DEV)
+        sbufs.append(b)
+        back.append(o)
+    rr.head_to_seq(recv, back, window_bytes=window)
+    assert all(gu.guards_intact(b) for b in sbufs)
+    assert gu.same_bits(torch.cat(back), full)
 
 
 def test_overlapping_output_rejected_on_device():
@@ -330,6 +397,19 @@ def test_full_qkvg_250k_w4_chunked(oracle_lib):
     info, info_back = _full_size_round_trip(oracle_lib, w, window=w.window_bytes)
     for i in (info, info_back):
         assert i["chunks"] == 4 and i["launches"] == 4 and i["planes_per_launch"] == 1
+    torch.cuda.empty_cache()
+
+
+def test_full_qkvg_250k_w2_sub_plane(oracle_lib):
+    """The long-sequence operand over 2 ranks: one plane of one rank is
+    1,792,000,000 bytes, twice the 896,000,000-byte window, so every plane
+    moves in two token chunks."""
+    w = wl.RelayoutWorkload("qkvg_T250000_W2_chunked", T=250000, P=4, W=2, seed=6,
+                            window_bytes=896_000_000)
+    assert rr.relayout_chunk_plan(w.T, w.P, w.H, w.D, w.W, w.window_bytes) == (62500, 8)
+    info, info_back = _full_size_round_trip(oracle_lib, w, window=w.window_bytes)
+    for i in (info, info_back):
+        assert i["chunks"] == 8 and i["launches"] == 8 and i["planes_per_launch"] == 1
     torch.cuda.empty_cache()
 
 

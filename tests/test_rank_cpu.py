@@ -72,10 +72,8 @@ def test_relayout_rank_argument_checks():
         # the output overlapping any input, the rank's own or a peer's
         for k in range(W):
             assert _call_relayout(fn, send, send[k] + 4096 * 4, T, P, H, D, W, k) == E.H3_ERR_INVALID_ARG
-        # window too small for one plane of the largest rank
-        row = H * D * 2
-        plane = max((_split(T, W)[1]) * row, T * 10 * D * 2)
-        assert _call_relayout(fn, send, free, T, P, H, D, W, 0, window=plane - 16) == E.H3_ERR_WINDOW
+        # a window that cannot hold one token of every rank (6 ranks x 10 heads)
+        assert _call_relayout(fn, send, free, T, P, H, D, W, 0, window=6 * 10 * D * 2 - 16) == E.H3_ERR_WINDOW
         assert _call_relayout(fn, send, free, T, P, H, D, W, 0, window=-1) == E.H3_ERR_INVALID_ARG
         # bulk is not offered; unknown variants and flags are rejected
         bulk = C.byref(_abi.LaunchConfig(E.H3_VARIANT_BULK, 0, 0, 0))
