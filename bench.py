@@ -1,22 +1,26 @@
 #!/usr/bin/env python
 """Benchmark of the H3 transport hot path on B200: effective HBM GB/s.
 
-One step is one pass of the whole path on the ragged 32k-token workload
-(T = 32768 packed tokens, W = 6 virtual ranks, heads 10,10,9,9,9,9, 8 packed
-segments):
+One step is one pass of the whole path over the two largest workloads of the
+path:
 
-  1. h3_partition            token/head ranges, segments clipped and rebased (host)
-  2. h3_seq_to_head          packed QKV [32768, 3, 56, 128] -> 6 x [32768, 3, H_j, 128]
-  3. h3_head_to_seq          back to [32768, 3, 56, 128], chunked one plane per
-                             launch under the 896,000,000-byte window
-  4. h3_ragged_reduce_scatter 6 BF16 partials [32768, 7168] + bias -> 6 x [T_r, 7168]
+  1. h3_partition             token/head ranges, packed segments clipped and rebased (host)
+  2. h3_seq_to_head           packed QKVG [250000, 4, 56, 128] over W = 4 ranks (heads
+                              14 each) -> 4 x [250000, 4, 14, 128], one batch plane
+                              per launch under the 896,000,000-byte window (4 launches)
+  3. h3_head_to_seq           back to [250000, 4, 56, 128], chunked the same way
+  4. h3_ragged_reduce_scatter 8 BF16 partials [65536, 7168] + bias -> 8 x [8192, 7168]
 
 value = algorithmic bytes of all steps (each input read once + each output
-written once) / device time, summed over GPUs.  Every kernel's inputs are
-1.4-2.8 GB, far larger than the 126 MB L2, so no flush is needed between
-steps.  With --gpus N (torchrun) every GPU runs an independent replica of the
-step: the path has no exchange between GPUs when all virtual ranks share one
-GPU's memory.
+written once) / device time.  Every kernel's inputs are 7.2-15 GB, far larger
+than the 126 MB L2, so no flush is needed between steps.
+
+With --gpus N > 1 (torchrun, one process per GPU) the same two problems run
+with one rank per GPU (W = N): every GPU holds its rank's buffers only and
+computes its rank's share with the h3_*_rank calls, pulling what it needs
+from the peers' buffers (mapped with CUDA IPC) over NVLink; a one-element
+NCCL all-reduce on the compute stream orders the ranks between the calls.
+The total problem is fixed as N grows (strong scaling).
 
 --impl reference times the plain CPU oracle (oracle/) on the host cores on a
 bounded sample of the same workload; it is the slow reference, not a target.
@@ -45,8 +49,12 @@ METRIC = "relayout + reduce-scatter effective HBM GB/s and % of B200 HBM peak"
 UNIT = "GB/s"
 FALLBACK_HBM_GBS = 6650.0
 NOMINAL_HBM_GBS = 8000.0  # nominal B200 HBM3e bandwidth, for a second percentage only
-STEP_T, STEP_W, STEP_P, STEP_SEGS, STEP_SEED = 32768, 6, 3, 8, 2
-WINDOW = 896_000_000
+# The step's two problems: the long-sequence QKVG round trip, one batch plane
+# per launch under the 896,000,000-byte window, and the 8-way reduce-scatter.
+RELAYOUT = wl.QKVG_250K_W4_CHUNKED
+REDUCE = wl.RS_64K_W8
+WINDOW = RELAYOUT.window_bytes
+WORKLOAD = f"{RELAYOUT.name}+{REDUCE.name}"
 
 
 # ---------------------------------------------------------------------------
@@ -79,6 +87,16 @@ def sum_over_ranks(x: float, device) -> float:
     return float(t.item())
 
 
+def min_over_ranks(x: float, device) -> float:
+    """Smallest value of x over all ranks (x itself without a process group)."""
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return float(x)
+    t = torch.tensor([float(x)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MIN)
+    return float(t.item())
+
+
 def throughput_gbs(bytes_per_step_per_gpu: float, steps: int, n_gpus: int, seconds: float) -> float:
     """Whole-job GB/s: every GPU's bytes over the slowest GPU's time."""
     return bytes_per_step_per_gpu * steps * n_gpus / seconds / 1e9
@@ -94,7 +112,8 @@ def load_peak():
         return FALLBACK_HBM_GBS, "fallback"
 
 
-# The sources each measured kernel is compiled from.
+# The sources each measured kernel is compiled from (the rank calls' pull
+# kernel lives in relayout.cu too).
 KERNEL_SOURCES = {
     "seq_to_head": ("relayout.cu", "device_access.cuh", "bulk_copy.cuh", "h3rr_internal.h"),
     "head_to_seq": ("relayout.cu", "device_access.cuh", "bulk_copy.cuh", "h3rr_internal.h"),
@@ -112,9 +131,10 @@ def kernel_source_digest(kernel: str) -> str:
     return h.hexdigest()[:16]
 
 
-def load_traffic(kernel: str):
-    """DRAM bytes per launch from the committed ncu summary, or None when the
-    kernels changed since it was taken."""
+def load_traffic(kernel: str, instance: str | None = None):
+    """DRAM bytes per launch of `kernel` on the launches `instance` names,
+    from the committed ncu summary; None when no capture covers that
+    instance or the kernel's sources changed since it was taken."""
     try:
         with open(os.path.join(ROOT, "profiles", "dram_traffic.json")) as f:
             table = json.load(f)
@@ -122,6 +142,8 @@ def load_traffic(kernel: str):
         return None
     entry = table.get(kernel)
     if not entry or kernel not in KERNEL_SOURCES or entry.get("source_digest") != kernel_source_digest(kernel):
+        return None
+    if instance is not None and entry.get("instance") != instance:
         return None
     return entry.get("bytes_per_launch")
 
@@ -188,78 +210,242 @@ class ClockSampler:
 # the step on the GPU
 # ---------------------------------------------------------------------------
 
-class Step:
-    """Device buffers and calls of one step of the path (inputs resident)."""
+KERNELS = ("seq_to_head", "head_to_seq", "ragged_reduce_scatter")
 
-    def __init__(self, device, T=STEP_T, W=STEP_W, P=STEP_P, n_segs=STEP_SEGS, seed=STEP_SEED,
-                 relayout=True, reduce=True):
+
+def relayout_bytes(T: int, P: int, H: int, D: int) -> int:
+    """Algorithmic bytes of one relayout direction: every element read once
+    and written once."""
+    return 2 * T * P * H * D * 2
+
+
+def reduce_bytes(T: int, C: int, W: int) -> int:
+    """Algorithmic bytes of the reduce-scatter: W partials read, the [T, C]
+    output written, the bias read once."""
+    return (W + 1) * T * C * 2 + C * 2
+
+
+class Step:
+    """Device buffers and calls of one step of the path on one GPU, with all
+    W virtual ranks in its memory (inputs resident).  tokens / rows shrink the
+    two problems (ncu captures of small cases); relayout / reduce leave one out."""
+
+    def __init__(self, device, *, tokens=None, rows=None, relayout=True, reduce=True):
         import ragged_reduce_b200 as rr
         self.rr = rr
         self.device = device
-        self.T, self.W, self.P, self.H, self.D = T, W, P, wl.H3_HEADS, wl.H3_HEAD_DIM
-        self.C = wl.H3_HIDDEN
-        self.bounds = wl.segment_bounds(T, n_segs, seed)
-        self.part = rr.partition(T, self.H, W, self.bounds)
+        rw, red = RELAYOUT, REDUCE
+        self.T, self.P, self.W, self.H, self.D = tokens or rw.T, rw.P, rw.W, rw.H, rw.D
+        self.window = rw.window_bytes
+        self.Tr, self.C, self.Wr = rows or red.T, red.C, red.W
+        self.bounds = wl.segment_bounds(self.T, rw.n_segs, rw.seed)
+        self.kernel_bytes = {}
+        self.has_relayout, self.has_reduce = relayout, reduce
         if relayout:
-            self.qkv = wl.normal_bf16((T, P, self.H, self.D), seed, 1.0, device)
+            self.part = rr.partition(self.T, self.H, self.W, self.bounds)
+            self.qkv = wl.normal_bf16((self.T, self.P, self.H, self.D), rw.seed, 1.0, device)
             self.send = rr.split_rows(self.qkv, self.part.token_starts)
-            self.heads = rr.alloc_head_side(T, P, self.H, self.D, W, device)
-            self.back_full, self.back = rr.alloc_seq_side(T, P, self.H, self.D, W, device)
+            self.heads = rr.alloc_head_side(self.T, self.P, self.H, self.D, self.W, device)
+            self.back_full, self.back = rr.alloc_seq_side(self.T, self.P, self.H, self.D, self.W, device)
+            b = relayout_bytes(self.T, self.P, self.H, self.D)
+            self.kernel_bytes["seq_to_head"] = b
+            self.kernel_bytes["head_to_seq"] = b
         if reduce:
-            rw = wl.ReduceWorkload("step", T=T, C=self.C, W=W, seed=seed + 100)
-            self.partials, self.bias = wl.partials_and_bias(rw, device)
+            w = wl.ReduceWorkload(red.name, T=self.Tr, C=self.C, W=self.Wr, seed=red.seed)
+            self.partials, self.bias = wl.partials_and_bias(w, device)
             self.partial_list = list(self.partials.unbind(0))
-            self.red_full, self.red_out = rr.alloc_reduce_outputs(T, self.C, W, device)
-        relayout_bytes = T * P * self.H * self.D * 2 * 2
-        reduce_bytes = (W + 1) * T * self.C * 2 + self.C * 2
-        self.kernel_bytes = {"seq_to_head": relayout_bytes, "head_to_seq": relayout_bytes,
-                             "ragged_reduce_scatter": reduce_bytes}
+            self.red_full, self.red_out = rr.alloc_reduce_outputs(self.Tr, self.C, self.Wr, device)
+            self.kernel_bytes["ragged_reduce_scatter"] = reduce_bytes(self.Tr, self.C, self.Wr)
         self.bytes_per_step = sum(self.kernel_bytes.values())
         self.launches = {}
 
+    def instance(self, kernel: str) -> str:
+        """The launches `kernel` makes in this step, as ncu summaries name them."""
+        if kernel == "ragged_reduce_scatter":
+            return f"reduce_scatter T={self.Tr} C={self.C} W={self.Wr}"
+        return (f"{kernel} T={self.T} P={self.P} W={self.W} one plane per launch "
+                f"(window {self.window})")
+
     def run(self, events=None, stream=None):
+        """Enqueue one step; events[0..3] (optional) bracket the three calls."""
         rr = self.rr
-        if events is not None:
-            events[0].record(stream)
-        rr.partition(self.T, self.H, self.W, self.bounds)
-        i1 = rr.seq_to_head(self.send, self.heads, stream=stream)
-        if events is not None:
-            events[1].record(stream)
-        i2 = rr.head_to_seq(self.heads, self.back, window_bytes=WINDOW, stream=stream)
-        if events is not None:
-            events[2].record(stream)
-        i3 = rr.ragged_reduce_scatter(self.partial_list, self.bias, self.red_out, stream=stream)
-        if events is not None:
-            events[3].record(stream)
-        self.launches = {"seq_to_head": i1["launches"], "head_to_seq": i2["launches"],
-                         "ragged_reduce_scatter": i3["launches"]}
-        return i1["launches"] + i2["launches"] + i3["launches"]
+
+        def mark(i):
+            if events is not None:
+                events[i].record(stream)
+
+        mark(0)
+        infos = {}
+        if self.has_relayout:
+            rr.partition(self.T, self.H, self.W, self.bounds)
+            infos["seq_to_head"] = rr.seq_to_head(self.send, self.heads, window_bytes=self.window,
+                                                  stream=stream)
+        mark(1)
+        if self.has_relayout:
+            infos["head_to_seq"] = rr.head_to_seq(self.heads, self.back, window_bytes=self.window,
+                                                  stream=stream)
+        mark(2)
+        if self.has_reduce:
+            infos["ragged_reduce_scatter"] = rr.ragged_reduce_scatter(self.partial_list, self.bias,
+                                                                      self.red_out, stream=stream)
+        mark(3)
+        self.launches = {k: v["launches"] for k, v in infos.items()}
+        return sum(self.launches.values())
 
     def verify(self) -> bool:
-        """Round trip and reduce spot check (not timed)."""
-        ok = torch.equal(self.back_full.view(torch.int16), self.qkv.view(torch.int16))
-        acc = self.partials[0].float()
-        for k in range(1, self.W):
-            acc += self.partials[k].float()
-        acc += self.bias.float()
-        ok = ok and torch.equal(self.red_full.view(torch.int16), acc.to(torch.bfloat16).view(torch.int16))
+        """Round trip and reduce check on the device with torch (not timed)."""
+        ok = True
+        if self.has_relayout:
+            ok = torch.equal(self.back_full.view(torch.int16), self.qkv.view(torch.int16))
+        if self.has_reduce:
+            acc = self.partials[0].float()
+            for k in range(1, self.Wr):
+                acc += self.partials[k].float()
+            acc += self.bias.float()
+            ok = ok and torch.equal(self.red_full.view(torch.int16),
+                                    acc.to(torch.bfloat16).view(torch.int16))
+            del acc
         return bool(ok)
 
-    def host_io(self):
-        """Pinned host copies of the step's inputs and room for its results."""
-        return {
-            "qkv": self.qkv.cpu().pin_memory(),
-            "partials": self.partials.cpu().pin_memory(),
-            "bias": self.bias.cpu().pin_memory(),
-            "back": torch.empty(self.back_full.shape, dtype=torch.bfloat16).pin_memory(),
-            "red": torch.empty(self.red_full.shape, dtype=torch.bfloat16).pin_memory(),
-        }
+    def inputs(self) -> dict:
+        """Device tensors a caller fills from the host every step."""
+        return {"qkv": self.qkv, "partials": self.partials, "bias": self.bias}
 
-    @staticmethod
-    def io_bytes(io):
-        h2d = sum(io[k].numel() * 2 for k in ("qkv", "partials", "bias"))
-        d2h = sum(io[k].numel() * 2 for k in ("back", "red"))
-        return h2d, d2h
+    def outputs(self) -> dict:
+        """Device tensors a caller reads back every step."""
+        return {"back": self.back_full, "red": self.red_full}
+
+    def nvlink(self, per_kernel_s: dict, steps: int):
+        return None
+
+
+class ShardedStep:
+    """One rank's share of the step with one rank per GPU (W = world).
+
+    Each process holds its rank's buffers only: the sequence-side rows
+    [T_k, P, H, D], the head-side buffer [T, P, H_k, D], the rows it gets back,
+    its partial [T, C], the bias and its reduce-scatter rows [T_k, C].  The
+    rank calls pull what rank k needs from every rank's buffer through the
+    peer tables.  Between the calls `fence(stream)` orders all ranks (a
+    one-element all-reduce enqueued on the compute stream): head->seq reads
+    the peers' head-side buffers that seq->head has just written, and the next
+    step's seq->head must not overwrite a head-side buffer a peer still reads.
+
+    Injectable for host-side tests: `rr` (the binding's partition and rank
+    calls), `peer_table` (tensor -> object with .pointers and .close()),
+    `fence`, and `empty(shape, dtype)`, which allocates the three buffers the
+    peers read (sequence-side rows, head-side buffer, partial)."""
+
+    def __init__(self, device, rank: int, world: int, *, rr, peer_table, fence,
+                 tokens=None, rows=None, empty=None):
+        if empty is None:
+            def empty(shape, dtype):
+                return torch.empty(shape, dtype=dtype, device=device)
+        self.rr, self.fence = rr, fence
+        self.device, self.rank, self.W = device, rank, world
+        rw, red = RELAYOUT, REDUCE
+        self.T, self.P, self.H, self.D = tokens or rw.T, rw.P, rw.H, rw.D
+        self.window = rw.window_bytes
+        self.Tr, self.C = rows or red.T, red.C
+        self.bounds = wl.segment_bounds(self.T, rw.n_segs, rw.seed)
+        part = rr.partition(self.T, self.H, world, self.bounds)
+        self.ts = (int(part.token_starts[rank]), int(part.token_starts[rank + 1]))
+        self.hk = part.heads(rank)
+        # the whole operand is drawn from the same seed as the one-GPU step;
+        # this rank keeps its token rows
+        x = wl.normal_bf16((self.T, self.P, self.H, self.D), rw.seed, 1.0, device)
+        self.send = empty((self.ts[1] - self.ts[0], self.P, self.H, self.D), torch.bfloat16)
+        self.send.copy_(x[self.ts[0]:self.ts[1]])
+        del x
+        self.heads = empty((self.T, self.P, self.hk, self.D), torch.bfloat16)
+        self.back = torch.empty_like(self.send)
+        w = wl.ReduceWorkload(red.name, T=self.Tr, C=self.C, W=world, seed=red.seed)
+        partials, self.bias = wl.partials_and_bias(w, device)
+        rp = rr.partition(self.Tr, world, world)
+        self.rows = (int(rp.token_starts[rank]), int(rp.token_starts[rank + 1]))
+        self.partial = empty((self.Tr, self.C), torch.bfloat16)
+        self.partial.copy_(partials[rank])
+        # every rank's rows of this rank's output, kept for verify()
+        self.check_rows = partials[:, self.rows[0]:self.rows[1]].clone()
+        del partials
+        self.red_out = torch.empty((self.rows[1] - self.rows[0], self.C), dtype=torch.bfloat16,
+                                   device=device)
+        # collective: every rank builds the tables in the same order
+        self.seq_tab = peer_table(self.send)
+        self.head_tab = peer_table(self.heads)
+        self.part_tab = peer_table(self.partial)
+        # whole-job algorithmic bytes (every element read and written once;
+        # each rank reads the bias once)
+        rb = relayout_bytes(self.T, self.P, self.H, self.D)
+        self.kernel_bytes = {"seq_to_head": rb, "head_to_seq": rb,
+                             "ragged_reduce_scatter": reduce_bytes(self.Tr, self.C, world)
+                             + (world - 1) * self.C * 2}
+        self.bytes_per_step = sum(self.kernel_bytes.values())
+        self.launches = {}
+
+    def instance(self, kernel: str) -> str:
+        return f"{kernel} rank share, one rank per GPU, W={self.W}"
+
+    def run(self, events=None, stream=None):
+        """Enqueue this rank's share of one step; events[0..4] (optional)
+        bracket the calls, the fence after seq->head excluded."""
+        rr, k = self.rr, self.rank
+
+        def mark(i):
+            if events is not None:
+                events[i].record(stream)
+
+        mark(0)
+        rr.partition(self.T, self.H, self.W, self.bounds)
+        i1 = rr.seq_to_head_rank(self.seq_tab.pointers, self.heads, k, n_heads=self.H,
+                                 window_bytes=self.window, stream=stream)
+        mark(1)
+        self.fence(stream)  # every head-side buffer is complete before anyone reads it
+        mark(2)
+        i2 = rr.head_to_seq_rank(self.head_tab.pointers, self.back, k, n_tokens=self.T,
+                                 window_bytes=self.window, stream=stream)
+        mark(3)
+        i3 = rr.ragged_reduce_scatter_rank(self.part_tab.pointers, self.bias, self.red_out, k,
+                                           n_tokens=self.Tr, stream=stream)
+        mark(4)
+        self.fence(stream)  # no head-side buffer is overwritten while a peer reads it
+        self.launches = {"seq_to_head": i1["launches"], "head_to_seq": i2["launches"],
+                         "ragged_reduce_scatter": i3["launches"]}
+        return sum(self.launches.values())
+
+    def verify(self) -> bool:
+        """This rank's round trip and its reduce rows, checked with torch."""
+        ok = torch.equal(self.back.view(torch.int16), self.send.view(torch.int16))
+        acc = self.check_rows[0].float()
+        for r in range(1, self.W):
+            acc += self.check_rows[r].float()
+        acc += self.bias.float()
+        return bool(ok and torch.equal(self.red_out.view(torch.int16),
+                                       acc.to(torch.bfloat16).view(torch.int16)))
+
+    def inputs(self) -> dict:
+        return {"send": self.send, "partial": self.partial, "bias": self.bias}
+
+    def outputs(self) -> dict:
+        return {"back": self.back, "red": self.red_out}
+
+    def pulled_bytes(self) -> dict:
+        """Bytes this rank's calls read from other ranks' memory per step."""
+        row = self.H * self.D * 2
+        tk = self.ts[1] - self.ts[0]
+        return {"seq_to_head": (self.T - tk) * self.P * self.hk * self.D * 2,
+                "head_to_seq": tk * self.P * (row - self.hk * self.D * 2),
+                "ragged_reduce_scatter": (self.W - 1) * (self.rows[1] - self.rows[0]) * self.C * 2}
+
+    def nvlink(self, per_kernel_s: dict, steps: int):
+        pulled = self.pulled_bytes()
+        return {k: {"bytes_per_step": int(v),
+                    "gbs": round(v * steps / per_kernel_s[k] / 1e9, 1) if per_kernel_s[k] > 0 else None}
+                for k, v in pulled.items()}
+
+    def close(self):
+        for t in (self.seq_tab, self.head_tab, self.part_tab):
+            t.close()
 
 
 def gpu_uuid(device) -> str | None:
@@ -270,11 +456,183 @@ def gpu_uuid(device) -> str | None:
         return None
 
 
-def barrier(local):
+class CudaTimer:
+    """Device timestamps: CUDA events recorded on the launching stream."""
+
+    def event(self):
+        return torch.cuda.Event(enable_timing=True)
+
+    @staticmethod
+    def seconds(a, b) -> float:
+        return a.elapsed_time(b) / 1e3
+
+    @staticmethod
+    def synchronize():
+        torch.cuda.synchronize()
+
+
+class _HostEvent:
+    def __init__(self):
+        self.t = None
+
+    def record(self, stream=None):
+        self.t = time.perf_counter()
+
+
+class HostTimer:
+    """Host timestamps for runs without a GPU (host-side tests)."""
+
+    def event(self):
+        return _HostEvent()
+
+    @staticmethod
+    def seconds(a, b) -> float:
+        return b.t - a.t
+
+    @staticmethod
+    def synchronize():
+        pass
+
+
+def barrier(local, timer=None):
     import torch.distributed as dist
     if dist.is_available() and dist.is_initialized():
-        dist.barrier(device_ids=[local])
+        if dist.get_backend() == "nccl":
+            dist.barrier(device_ids=[local])
+        else:
+            dist.barrier()
+    (timer or CudaTimer()).synchronize()
+
+
+def nccl_fence(device):
+    """A stream-ordered barrier of all ranks: a one-element all-reduce
+    enqueued on `stream` completes on a rank only after every rank's stream
+    has reached it, so whatever each rank enqueued before it has finished."""
+    import torch.distributed as dist
+    token = torch.zeros(1, dtype=torch.int32, device=device)
+
+    def fence(stream=None):
+        if stream is None:
+            dist.all_reduce(token)
+        else:
+            with torch.cuda.stream(stream):
+                dist.all_reduce(token)
+    return fence
+
+
+def time_steps(step, K: int, timer, stream, local, device, n_events: int):
+    """Run K steps between barriers; (seconds, launches, per-kernel seconds)."""
+    evs = [[timer.event() for _ in range(n_events)] for _ in range(K)]
+    start, end = timer.event(), timer.event()
+    launches = 0
+    barrier(local, timer)
+    start.record(stream)
+    for k in range(K):
+        launches += step.run(events=evs[k], stream=stream)
+    end.record(stream)
+    barrier(local, timer)
+    per_kernel_s = {name: 0.0 for name in KERNELS}
+    # the events bracketing each call (the sharded step has a fence between
+    # its first two calls, which no kernel's time includes)
+    spans = ({"seq_to_head": (0, 1), "head_to_seq": (1, 2), "ragged_reduce_scatter": (2, 3)}
+             if n_events == 4 else
+             {"seq_to_head": (0, 1), "head_to_seq": (2, 3), "ragged_reduce_scatter": (3, 4)})
+    for e in evs:
+        for name, (a, b) in spans.items():
+            per_kernel_s[name] += timer.seconds(e[a], e[b])
+    return timer.seconds(start, end), launches, per_kernel_s
+
+
+def kernel_table(step, per_kernel_s: dict, K: int) -> dict:
+    kernels = {}
+    total = sum(per_kernel_s.values())
+    for name, secs in per_kernel_s.items():
+        n = step.launches.get(name, 0)
+        if n == 0 or secs <= 0:
+            continue
+        per_launch_s = secs / (n * K)
+        bytes_per_launch = step.kernel_bytes[name] / n
+        kernels[name] = {"gbs": round(bytes_per_launch / per_launch_s / 1e9, 1),
+                         "us_per_launch": round(per_launch_s * 1e6, 2),
+                         "launches_per_step": n,
+                         "bytes_per_launch": int(bytes_per_launch),
+                         "share": round(secs / total, 3),
+                         "instance": step.instance(name)}
+    return kernels
+
+
+def run_e2e(make_step, first, n_steps: int, local, device, world: int, timer):
+    """End to end through the public API with pinned host buffers: every step
+    copies its inputs in and its results out.  Two device buffer sets and
+    three streams (host->device, compute, device->host) ordered by events let
+    step k's result copy and step k+1's input copy overlap the kernels."""
+    ins = {k: torch.empty(v.shape, dtype=v.dtype, pin_memory=True) for k, v in first.inputs().items()}
+    for k, v in first.inputs().items():
+        ins[k].copy_(v)
+    outs = {k: torch.empty(v.shape, dtype=v.dtype, pin_memory=True) for k, v in first.outputs().items()}
+    h2d = sum(v.numel() * v.element_size() for v in ins.values())
+    d2h = sum(v.numel() * v.element_size() for v in outs.values())
+    bufs = [first, make_step()]
+    s_in, s_run, s_out = torch.cuda.Stream(device), torch.cuda.Stream(device), torch.cuda.Stream(device)
+    loaded = [torch.cuda.Event() for _ in bufs]
+    computed = [torch.cuda.Event() for _ in bufs]
+    unloaded = [torch.cuda.Event() for _ in bufs]
+
+    def e2e_step(k):
+        b = k % 2
+        st = bufs[b]
+        if k >= 2:
+            s_in.wait_event(computed[b])      # step k-2 is done reading this buffer set
+        with torch.cuda.stream(s_in):
+            for name, dst in st.inputs().items():
+                dst.copy_(ins[name], non_blocking=True)
+            loaded[b].record(s_in)
+        s_run.wait_event(loaded[b])
+        if k >= 2:
+            s_run.wait_event(unloaded[b])     # step k-2's results have left this buffer set
+        n = st.run(stream=s_run)
+        computed[b].record(s_run)
+        s_out.wait_event(computed[b])
+        with torch.cuda.stream(s_out):
+            for name, src in st.outputs().items():
+                outs[name].copy_(src, non_blocking=True)
+            unloaded[b].record(s_out)
+        return n
+
+    for k in range(2):                        # warm both buffer sets
+        e2e_step(k)
     torch.cuda.synchronize()
+    barrier(local, timer)
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(s_in)
+    s_run.wait_stream(s_in)
+    s_out.wait_stream(s_in)
+    for k in range(n_steps):
+        e2e_step(k + 2)
+    s_in.wait_stream(s_run)
+    s_in.wait_stream(s_out)
+    e1.record(s_in)
+    barrier(local, timer)
+    t_e2e = max_over_ranks(e0.elapsed_time(e1) / 1e3, device)
+    # the round trip comes back unchanged
+    key_in, key_out = ("qkv", "back") if "qkv" in ins else ("send", "back")
+    ok = torch.equal(outs[key_out].view(torch.int16), ins[key_in].view(torch.int16))
+    ok = bool(min_over_ranks(1.0 if ok else 0.0, device) > 0)
+    second = bufs[1]
+    if hasattr(second, "close"):
+        torch.cuda.synchronize()
+        barrier(local, timer)
+        second.close()
+    del bufs
+    return {"value": round(throughput_gbs(first.bytes_per_step, n_steps, 1, t_e2e), 2),
+            "unit": UNIT,
+            "h2d_bytes_per_step": int(sum_over_ranks(h2d, device)),
+            "d2h_bytes_per_step": int(sum_over_ranks(d2h, device)),
+            "steps": n_steps, "ms_per_step": round(t_e2e / n_steps * 1e3, 3),
+            "mode": "pinned host buffers; copies in, kernels and copies out on three streams, "
+                    "two device buffer sets" + (f", {world} GPUs" if world > 1 else ""),
+            "round_trip_ok": ok}
 
 
 def run_gpu(args):
@@ -284,134 +642,91 @@ def run_gpu(args):
         raise SystemExit(f"--gpus {args.gpus} but WORLD_SIZE={world}")
     torch.cuda.set_device(local)
     device = torch.device("cuda", local)
+    timer = CudaTimer()
     if world > 1:
         import datetime
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
                                 device_id=device)
-    step = Step(device)
-    stream = torch.cuda.current_stream(device)
+    import ragged_reduce_b200 as rr
+    if world > 1:
+        from ragged_reduce_b200 import peers
 
+        def make_step():
+            return ShardedStep(device, rank, world, rr=rr, peer_table=peers.PeerBuffers,
+                               fence=nccl_fence(device))
+        n_events = 5
+    else:
+        def make_step():
+            return Step(device)
+        n_events = 4
+    result = measure(args, make_step, rank, world, local, device, timer, n_events)
+    torch.cuda.empty_cache()
+    if world > 1:
+        dist.barrier(device_ids=[local])
+        dist.destroy_process_group()
+    return result
+
+
+def measure(args, make_step, rank, world, local, device, timer, n_events):
+    """Warm-up, correctness check, K timed steps, e2e; rank 0's JSON record."""
+    step = make_step()
+    stream = torch.cuda.current_stream(device) if isinstance(timer, CudaTimer) else None
     # warm-up (untimed) and a correctness check of the buffers the bench times
     for _ in range(args.warmup):
         step.run(stream=stream)
-    torch.cuda.synchronize()
-    if not step.verify():
+    timer.synchronize()
+    ok = step.verify()
+    if min_over_ranks(1.0 if ok else 0.0, device) <= 0:
         raise SystemExit("bench step produced wrong results")
 
     K = args.steps
-    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(K)]
-    start = torch.cuda.Event(enable_timing=True)
-    end = torch.cuda.Event(enable_timing=True)
-    launches = 0
-    with ClockSampler(gpu_uuid(device)) as clocks:
-        barrier(local)
-        start.record(stream)
-        for k in range(K):
-            launches += step.run(events=evs[k], stream=stream)
-        end.record(stream)
-        barrier(local)
-    elapsed = start.elapsed_time(end) / 1e3
-    per_kernel_s = {"seq_to_head": 0.0, "head_to_seq": 0.0, "ragged_reduce_scatter": 0.0}
-    for e in evs:
-        per_kernel_s["seq_to_head"] += e[0].elapsed_time(e[1]) / 1e3
-        per_kernel_s["head_to_seq"] += e[1].elapsed_time(e[2]) / 1e3
-        per_kernel_s["ragged_reduce_scatter"] += e[2].elapsed_time(e[3]) / 1e3
+    with ClockSampler(gpu_uuid(device) if isinstance(timer, CudaTimer) else None) as clocks:
+        elapsed, launches, per_kernel_s = time_steps(step, K, timer, stream, local, device, n_events)
     t_max = max_over_ranks(elapsed, device)
     launches_total = int(sum_over_ranks(launches, device))
-    value = throughput_gbs(step.bytes_per_step, K, world, t_max)
+    value = throughput_gbs(step.bytes_per_step, K, 1, t_max)
     peak, peak_kind = load_peak()
-
-    kernels = {}
-    for name, secs in per_kernel_s.items():
-        n_launch = step.launches[name] * K
-        per_launch_s = secs / n_launch
-        bytes_per_launch = step.kernel_bytes[name] / step.launches[name]
-        kernels[name] = {"gbs": round(bytes_per_launch / per_launch_s / 1e9, 1),
-                         "us_per_launch": round(per_launch_s * 1e6, 2),
-                         "launches_per_step": step.launches[name],
-                         "bytes_per_launch": int(bytes_per_launch),
-                         "share": round(secs / sum(per_kernel_s.values()), 3)}
+    kernels = kernel_table(step, per_kernel_s, K)
     dom = max(kernels, key=lambda k: kernels[k]["share"])
-    achieved = kernels[dom]["gbs"]
-    roofline = {"bound": "hbm", "kernel": dom, "achieved": achieved, "peak": peak,
+    achieved = kernels[dom]["gbs"] / world  # per GPU: each GPU moves 1/W of the bytes
+    roofline = {"bound": "hbm", "kernel": dom, "instance": kernels[dom]["instance"],
+                "achieved": round(achieved, 1), "peak": peak,
                 "unit": "GB/s", "frac": round(achieved / peak, 4),
                 "peak_source": f"{peak_kind}: MEASURED_PEAKS.json hbm_gbs" if peak_kind == "measured"
                 else "fallback 6650 GB/s",
-                "traffic": load_traffic(dom), "algorithmic_bytes_per_launch": kernels[dom]["bytes_per_launch"]}
+                "traffic": load_traffic(dom, kernels[dom]["instance"]) if world == 1 else None,
+                "algorithmic_bytes_per_launch": kernels[dom]["bytes_per_launch"] // world}
+    nvlink = step.nvlink(per_kernel_s, K)
 
-    # end to end through the public API with pinned host buffers: every step
-    # copies its inputs in and its results out.  Two device buffer sets and
-    # three streams (host->device, compute, device->host) ordered by events
-    # let step k's result copy and step k+1's input copy overlap the kernels.
     e2e = None
-    if args.e2e_steps > 0:
-        io = step.host_io()
-        h2d, d2h = Step.io_bytes(io)
-        bufs = [step, Step(device)]
-        s_in, s_run, s_out = torch.cuda.Stream(), torch.cuda.Stream(), torch.cuda.Stream()
-        loaded = [torch.cuda.Event() for _ in bufs]
-        computed = [torch.cuda.Event() for _ in bufs]
-        unloaded = [torch.cuda.Event() for _ in bufs]
-
-        def e2e_step(k):
-            b = k % 2
-            st = bufs[b]
-            if k >= 2:
-                s_in.wait_event(computed[b])      # step k-2 is done reading this buffer set
-            with torch.cuda.stream(s_in):
-                st.qkv.copy_(io["qkv"], non_blocking=True)
-                st.partials.copy_(io["partials"], non_blocking=True)
-                st.bias.copy_(io["bias"], non_blocking=True)
-                loaded[b].record(s_in)
-            s_run.wait_event(loaded[b])
-            if k >= 2:
-                s_run.wait_event(unloaded[b])     # step k-2's results have left this buffer set
-            n = st.run(stream=s_run)
-            computed[b].record(s_run)
-            s_out.wait_event(computed[b])
-            with torch.cuda.stream(s_out):
-                io["back"].copy_(st.back_full, non_blocking=True)
-                io["red"].copy_(st.red_full, non_blocking=True)
-                unloaded[b].record(s_out)
-            return n
-
-        for k in range(2):                        # warm both buffer sets
-            e2e_step(k)
-        torch.cuda.synchronize()
-        barrier(local)
-        e0 = torch.cuda.Event(enable_timing=True)
-        e1 = torch.cuda.Event(enable_timing=True)
-        e0.record(s_in)
-        s_run.wait_stream(s_in)
-        s_out.wait_stream(s_in)
-        for k in range(args.e2e_steps):
-            e2e_step(k + 2)
-        s_in.wait_stream(s_run)
-        s_in.wait_stream(s_out)
-        e1.record(s_in)
-        barrier(local)
-        t_e2e = max_over_ranks(e0.elapsed_time(e1) / 1e3, device)
-        ok = torch.equal(io["back"].view(torch.int16), io["qkv"].view(torch.int16))
-        e2e = {"value": round(throughput_gbs(step.bytes_per_step, args.e2e_steps, world, t_e2e), 2),
-               "unit": UNIT, "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
-               "steps": args.e2e_steps, "ms_per_step": round(t_e2e / args.e2e_steps * 1e3, 3),
-               "mode": "pinned host buffers; copies in, kernels and copies out on three streams, "
-                       "two device buffer sets",
-               "round_trip_ok": bool(ok)}
-        del io, bufs
+    if args.e2e_steps > 0 and isinstance(timer, CudaTimer):
+        e2e = run_e2e(make_step, step, args.e2e_steps, local, device, world, timer)
 
     result = None
     if rank == 0:
+        if world > 1:
+            parallelism = (f"one rank per GPU: W={world} ranks, tokens and heads split "
+                           f"by quotient/remainder, shares pulled over NVLink")
+        else:
+            parallelism = (f"one GPU: W={RELAYOUT.W} virtual ranks (relayout), "
+                           f"W={REDUCE.W} (reduce-scatter)")
         result = {
             "metric": METRIC, "value": round(value, 1), "unit": UNIT, "n_gpus": world,
             "steps": K, "warmup": args.warmup, "ms_per_step": round(t_max / K * 1e3, 4),
-            "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
-            "dtype": "bf16", "data": "synthetic",
-            "config": {"workload": "h3_transport_step_T32768_W6", "tokens": STEP_T,
-                       "planes": STEP_P, "heads": wl.H3_HEADS, "head_dim": wl.H3_HEAD_DIM,
-                       "world": STEP_W, "segments": STEP_SEGS, "reduce_cols": wl.H3_HIDDEN,
-                       "window_bytes": WINDOW, "parallelism": f"replicas x{world}",
-                       "l2": "no flush: every kernel's inputs (1.4-2.8 GB) exceed the 126 MB L2",
+            "higher_is_better": True, "scaling": "strong" if world > 1 else "weak",
+            "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "config": {"workload": WORKLOAD,
+                       "relayout": {"tokens": RELAYOUT.T, "planes": RELAYOUT.P,
+                                    "heads": RELAYOUT.H, "head_dim": RELAYOUT.D,
+                                    "world": world if world > 1 else RELAYOUT.W,
+                                    "segments": RELAYOUT.n_segs, "window_bytes": WINDOW,
+                                    "chunking": "one batch plane per launch"},
+                       "reduce_scatter": {"tokens": REDUCE.T, "cols": REDUCE.C,
+                                          "world": world if world > 1 else REDUCE.W,
+                                          "partial_std": REDUCE.partial_std,
+                                          "bias_std": REDUCE.bias_std},
+                       "parallelism": parallelism,
+                       "l2": "no flush: every kernel's inputs (7.2-15 GB) exceed the 126 MB L2",
                        "bytes_per_step": step.bytes_per_step},
             "pct_of_peak": round(100.0 * value / world / peak, 2),
             "pct_of_nominal_peak": {"value": round(100.0 * value / world / NOMINAL_HBM_GBS, 2),
@@ -422,13 +737,16 @@ def run_gpu(args):
             "gpu_launches": launches_total,
             "clocks": clocks.summary(),
             "e2e": e2e,
-            "library": os.path.relpath(step.rr.library_path, ROOT),
+            "library": os.path.relpath(step.rr.library_path, ROOT)
+            if hasattr(step.rr, "library_path") else None,
         }
+        if nvlink is not None:
+            result["nvlink_rank0"] = nvlink
+    if hasattr(step, "close"):
+        timer.synchronize()
+        barrier(local, timer)
+        step.close()
     del step
-    torch.cuda.empty_cache()
-    if world > 1:
-        dist.barrier(device_ids=[local])
-        dist.destroy_process_group()
     return result
 
 
@@ -437,21 +755,26 @@ def run_gpu(args):
 # ---------------------------------------------------------------------------
 
 class OracleStep:
-    """The same step through the CPU oracle on a token sample of the workload."""
+    """The step through the CPU oracle on a sample of the workload: `tokens`
+    tokens of the relayout problem (same planes, heads and W) and `rows` rows
+    of the reduce-scatter (same C and W)."""
 
-    def __init__(self, tokens: int, W=STEP_W, P=STEP_P, seed=STEP_SEED):
+    def __init__(self, tokens: int, rows: int):
         import oracle
         self.o = oracle.load()
-        self.T, self.W, self.P, self.H, self.D, self.C = tokens, W, P, wl.H3_HEADS, wl.H3_HEAD_DIM, wl.H3_HIDDEN
-        self.bounds = wl.segment_bounds(tokens, min(STEP_SEGS, tokens), seed)
-        full = wl.bf16_bits(wl.normal_bf16((tokens, P, self.H, self.D), seed))
-        ts = self.o.partition_range(tokens, W)
-        self.send = [full[ts[r]:ts[r + 1]] for r in range(W)]
-        rw = wl.ReduceWorkload("sample", T=tokens, C=self.C, W=W, seed=seed + 100)
-        partials, bias = wl.partials_and_bias(rw, "cpu")
+        rw, red = RELAYOUT, REDUCE
+        self.T, self.W, self.P, self.H, self.D = tokens, rw.W, rw.P, rw.H, rw.D
+        self.Tr, self.Wr, self.C = rows, red.W, red.C
+        self.bounds = wl.segment_bounds(tokens, min(rw.n_segs, tokens), rw.seed)
+        full = wl.bf16_bits(wl.normal_bf16((tokens, self.P, self.H, self.D), rw.seed))
+        ts = self.o.partition_range(tokens, self.W)
+        self.send = [full[ts[r]:ts[r + 1]] for r in range(self.W)]
+        w = wl.ReduceWorkload("sample", T=rows, C=self.C, W=self.Wr, seed=red.seed)
+        partials, bias = wl.partials_and_bias(w, "cpu")
         self.partials = [wl.bf16_bits(p) for p in partials.unbind(0)]
         self.bias = wl.bf16_bits(bias)
-        self.bytes = tokens * P * self.H * self.D * 2 * 2 * 2 + (W + 1) * tokens * self.C * 2 + self.C * 2
+        self.bytes = (2 * relayout_bytes(tokens, self.P, self.H, self.D)
+                      + reduce_bytes(rows, self.C, self.Wr))
 
     def run(self):
         o = self.o
@@ -460,11 +783,23 @@ class OracleStep:
             o.clip_segments(self.bounds, int(ts[r]), int(ts[r + 1]))
         heads = o.seq_to_head(self.send, self.T, self.P, self.H, self.D, self.W)
         o.head_to_seq(heads, self.T, self.P, self.H, self.D, self.W)
-        o.ragged_reduce_scatter(self.partials, self.bias, self.W)
+        o.ragged_reduce_scatter(self.partials, self.bias, self.Wr)
+
+
+def sample_rows(tokens: int) -> int:
+    """Reduce-scatter rows that go with `tokens` relayout tokens in a sample,
+    so that the sample keeps the step's mix of the two problems."""
+    return max(REDUCE.W, round(tokens * REDUCE.T / RELAYOUT.T))
+
+
+def sample_text(tokens: int) -> str:
+    return (f"{tokens} of {RELAYOUT.T} tokens of the QKVG round trip (W={RELAYOUT.W}) and "
+            f"{sample_rows(tokens)} of {REDUCE.T} rows of the reduce-scatter (W={REDUCE.W}), "
+            f"shapes otherwise the step's")
 
 
 def oracle_seconds_per_token() -> float:
-    s = OracleStep(256)
+    s = OracleStep(256, sample_rows(256))
     t0 = time.perf_counter()
     s.run()
     return (time.perf_counter() - t0) / 256
@@ -491,12 +826,12 @@ def host_cpu_model() -> str:
 
 class OracleSteps:
     """The step through the unchanged oracle on every host core at once: one
-    token sample per thread, run concurrently (the C oracle is called without
-    the GIL, so the threads use separate cores)."""
+    sample per thread, run concurrently (the C oracle is called without the
+    GIL, so the threads use separate cores)."""
 
     def __init__(self, tokens_each: int, threads: int):
         from concurrent.futures import ThreadPoolExecutor
-        self.steps = [OracleStep(tokens_each) for _ in range(threads)]
+        self.steps = [OracleStep(tokens_each, sample_rows(tokens_each)) for _ in range(threads)]
         self.tokens_each = tokens_each
         self.bytes = sum(s.bytes for s in self.steps)
         self.pool = ThreadPoolExecutor(max_workers=threads)
@@ -508,17 +843,17 @@ class OracleSteps:
         self.pool.shutdown()
 
 
-# tokens of one thread's sample: bounds host memory (about 70 KB per token)
-MAX_TOKENS_PER_THREAD = 2048
+# tokens of one thread's sample: bounds host memory (about 210 KB per token)
+MAX_TOKENS_PER_THREAD = 1024
 
 
 def cpu_baseline(budget_s: float = 12.0) -> dict:
     """The oracle on every host core (the reported value) and on one core
-    (`one_core`), each on a bounded token sample of the bench step."""
+    (`one_core`), each on a bounded sample of the bench step."""
     per_tok = oracle_seconds_per_token()
     # one core: the step on one sample, best of 2
-    tokens = int(min(STEP_T, max(STEP_W, budget_s / 4 / per_tok)))
-    s = OracleStep(tokens)
+    tokens = int(min(RELAYOUT.T, max(RELAYOUT.W, budget_s / 4 / per_tok)))
+    s = OracleStep(tokens, sample_rows(tokens))
     times = []
     for _ in range(2):
         t0 = time.perf_counter()
@@ -526,12 +861,12 @@ def cpu_baseline(budget_s: float = 12.0) -> dict:
         times.append(time.perf_counter() - t0)
     t1 = min(times)
     one = {"value": round(s.bytes / t1 / 1e9, 3), "unit": UNIT, "cores": 1, "kind": "oracle",
-           "sample": f"the step on {tokens} of {STEP_T} tokens (W={STEP_W}, same shapes otherwise), "
-                     f"best of 2, {t1:.2f} s each, single-threaded C oracle"}
+           "sample": f"the step on {sample_text(tokens)}, best of 2, {t1:.2f} s each, "
+                     f"single-threaded C oracle"}
     del s
     # every core: one sample per thread, repeated for about budget/2 seconds
     cores = host_cores()
-    each = int(max(STEP_W, min(MAX_TOKENS_PER_THREAD, budget_s / 8 / per_tok)))
+    each = int(max(RELAYOUT.W, min(MAX_TOKENS_PER_THREAD, budget_s / 8 / per_tok)))
     steps = OracleSteps(each, cores)
     steps.run()  # warm
     n, t0 = 0, time.perf_counter()
@@ -542,8 +877,8 @@ def cpu_baseline(budget_s: float = 12.0) -> dict:
     steps.close()
     return {"value": round(steps.bytes * n / t / 1e9, 3), "unit": UNIT, "cores": cores,
             "kind": "oracle",
-            "sample": f"{cores} threads, each the step on its own {each} tokens (W={STEP_W}, "
-                      f"same shapes otherwise), {n} rounds in {t:.1f} s, C oracle unchanged",
+            "sample": f"{cores} threads, each the step on its own {sample_text(each)}; "
+                      f"{n} rounds in {t:.1f} s, C oracle unchanged",
             "cpu_model": host_cpu_model(), "one_core": one}
 
 
@@ -555,7 +890,7 @@ def run_reference(args):
     per_tok = oracle_seconds_per_token()
     per_step = budget / max(1, args.steps + args.warmup)
     cores = host_cores()
-    each = int(min(MAX_TOKENS_PER_THREAD, max(STEP_W, per_step / per_tok)))
+    each = int(min(MAX_TOKENS_PER_THREAD, max(RELAYOUT.W, per_step / per_tok)))
     s = OracleSteps(each, cores)
     for _ in range(args.warmup):
         s.run()
@@ -565,15 +900,14 @@ def run_reference(args):
     t = time.perf_counter() - t0
     s.close()
     value = s.bytes * args.steps / t / 1e9
-    sample = (f"each step: {cores} threads, each the path on its own {each} tokens (W={STEP_W}, "
-              f"same shapes otherwise), C oracle unchanged")
+    sample = f"each step: {cores} threads, each the path on its own {sample_text(each)}; C oracle unchanged"
     return {
         "impl": "reference", "metric": METRIC, "value": round(value, 3), "unit": UNIT,
         "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": round(t / args.steps * 1e3, 3), "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-        "config": {"workload": "h3_transport_step_T32768_W6", "tokens": STEP_T, "world": STEP_W,
-                   "sample_tokens": each * cores},
+        "config": {"workload": WORKLOAD, "relayout_tokens": RELAYOUT.T, "reduce_rows": REDUCE.T,
+                   "sample_tokens": each * cores, "sample_rows": sample_rows(each) * cores},
         "cpu_baseline": {"value": round(value, 3), "unit": UNIT, "cores": cores, "kind": "oracle",
                          "sample": sample, "cpu_model": host_cpu_model()},
         "e2e": {"value": round(value, 3), "unit": UNIT, "h2d_bytes_per_step": 0,
@@ -584,51 +918,67 @@ def run_reference(args):
 
 def run_profile(args):
     """Run one kernel of the path --steps times (for ncu captures); no timing.
-    The step's kernels on the bench workload, and the widened rows on the same
-    shapes: gated reduce-scatter (8 segments), all-gather of the reduce
+    The step's kernels (--profile-tokens shrinks the relayout problem,
+    --profile-rows the reduce-scatter), and the widened rows on the same
+    shapes: gated reduce-scatter (16 segments), all-gather of the reduce
     outputs, staged seq->head through the 896,000,000-byte window, and rank
     0's pulled seq->head share."""
     torch.cuda.set_device(0)
     device = torch.device("cuda", 0)
-    T = args.profile_tokens
     relayout = args.profile in ("seq_to_head", "head_to_seq", "staged_seq_to_head", "rank_seq_to_head")
-    step = Step(device, T=T, relayout=relayout, reduce=not relayout)
+    step = Step(device, tokens=args.profile_tokens, rows=args.profile_rows, relayout=relayout,
+                reduce=not relayout)
     rr = step.rr
     if args.profile == "head_to_seq":
         rr.seq_to_head(step.send, step.heads)
     extra = {}
     if args.profile == "gated_reduce_scatter":
-        extra["gate"] = wl.normal_bf16((STEP_SEGS, step.C), STEP_SEED + 2, 1.0, device)
-        extra["x_full"], extra["x"] = rr.alloc_reduce_outputs(T, step.C, step.W, device)
-        extra["x_full"].copy_(wl.normal_bf16((T, step.C), STEP_SEED + 3, 1.0, device))
+        extra["bounds"] = wl.segment_bounds(step.Tr, 16, REDUCE.seed)
+        extra["gate"] = wl.normal_bf16((16, step.C), REDUCE.seed + 2, 1.0, device)
+        extra["x_full"], extra["x"] = rr.alloc_reduce_outputs(step.Tr, step.C, step.Wr, device)
+        extra["x_full"].copy_(wl.normal_bf16((step.Tr, step.C), REDUCE.seed + 3, 1.0, device))
     elif args.profile == "all_gather":
         rr.ragged_reduce_scatter(step.partial_list, step.bias, step.red_out)
-        extra["outs"] = [torch.empty((T, step.C), dtype=torch.bfloat16, device=device)
-                         for _ in range(step.W)]
+        extra["outs"] = [torch.empty((step.Tr, step.C), dtype=torch.bfloat16, device=device)
+                         for _ in range(step.Wr)]
     elif args.profile == "staged_seq_to_head":
         extra["win"] = torch.empty(WINDOW, dtype=torch.uint8, device=device)
     elif args.profile == "rank_seq_to_head":
         extra["mine"] = torch.empty_like(step.heads[0])
+    layout = args.profile_layout
+    if layout and args.profile in ("seq_to_head", "head_to_seq"):
+        # the same bytes with plane-major buffers on the sides `layout` names
+        part = rr.partition(step.T, step.H, step.W)
+        if layout & rr.H3_LAYOUT_SEQ_PLANE_MAJOR:
+            step.send = [x.permute(1, 0, 2, 3).contiguous() for x in step.send]
+            step.back = [torch.empty_like(x) for x in step.send]
+        if layout & rr.H3_LAYOUT_HEAD_PLANE_MAJOR:
+            step.heads = [torch.empty((step.P, step.T, part.heads(j), step.D), dtype=torch.bfloat16,
+                                      device=device) for j in range(step.W)]
+        if args.profile == "head_to_seq":
+            rr.seq_to_head_layout(step.send, step.heads, layout)
     launches = 0
     for _ in range(args.steps):
         if args.profile == "seq_to_head":
-            info = rr.seq_to_head(step.send, step.heads)
+            info = rr.seq_to_head_layout(step.send, step.heads, layout, window_bytes=step.window)
         elif args.profile == "head_to_seq":
-            info = rr.head_to_seq(step.heads, step.back, window_bytes=WINDOW)
+            info = rr.head_to_seq_layout(step.heads, step.back, layout, window_bytes=step.window)
         elif args.profile == "reduce_scatter":
             info = rr.ragged_reduce_scatter(step.partial_list, step.bias, step.red_out)
         elif args.profile == "gated_reduce_scatter":
             info = rr.ragged_reduce_scatter_gated(step.partial_list, step.bias, extra["gate"],
-                                                  step.bounds, extra["x"], step.red_out)
+                                                  extra["bounds"], extra["x"], step.red_out)
         elif args.profile == "all_gather":
             info = rr.ragged_all_gather(step.red_out, extra["outs"])
         elif args.profile == "staged_seq_to_head":
             info = rr.seq_to_head_staged(step.send, step.heads, extra["win"])
         else:
-            info = rr.seq_to_head_rank(step.send, extra["mine"], 0, n_heads=step.H)
+            info = rr.seq_to_head_rank(step.send, extra["mine"], 0, n_heads=step.H,
+                                       window_bytes=step.window)
         launches += info["launches"]
     torch.cuda.synchronize()
-    print(json.dumps({"profile": args.profile, "tokens": T, "launches": launches}), flush=True)
+    print(json.dumps({"profile": args.profile, "tokens": step.T, "rows": step.Tr,
+                      "layout": layout, "launches": launches}), flush=True)
     return 0
 
 
@@ -685,6 +1035,34 @@ def run_workload_report(args):
             emit(w.name, "head_to_seq", vname, nbytes, secs, info)
             if not torch.equal(back_full.view(torch.int16), x.view(torch.int16)):
                 raise SystemExit(f"{w.name} {vname}: round trip differs")
+        if w.T in (32768, 250000):
+            # one plane per launch against one launch, with token-major and
+            # plane-major buffers (layout bits: 1 sequence side, 2 head side):
+            # the cost of one-plane launches on token-major buffers is the
+            # interleaving of the planes in memory
+            seq_pm = [t.permute(1, 0, 2, 3).contiguous() for t in send]
+            heads_pm = [torch.empty((w.P, w.T, part.heads(j), w.D), dtype=torch.bfloat16, device=dev)
+                        for j in range(w.W)]
+            back_pm = [torch.empty_like(t) for t in seq_pm]
+            for layout in (0, 1, 2, 3):
+                lsend = seq_pm if layout & 1 else send
+                lback = back_pm if layout & 1 else back
+                lheads = heads_pm if layout & 2 else heads
+                for wb in (0, WINDOW):
+                    tag = f"layout{layout}_{'chunked' if wb else 'unchunked'}"
+                    info = rr.seq_to_head_layout(lsend, lheads, layout, window_bytes=wb)
+                    secs = _time_calls(lambda: rr.seq_to_head_layout(lsend, lheads, layout,
+                                                                     window_bytes=wb), iters)
+                    emit(w.name, "seq_to_head", tag, nbytes, secs, info)
+                    info = rr.head_to_seq_layout(lheads, lback, layout, window_bytes=wb)
+                    secs = _time_calls(lambda: rr.head_to_seq_layout(lheads, lback, layout,
+                                                                     window_bytes=wb), iters)
+                    emit(w.name, "head_to_seq", tag, nbytes, secs, info)
+                    if not all(torch.equal(a.view(torch.int16), b.view(torch.int16))
+                               for a, b in zip(lback, lsend)):
+                        raise SystemExit(f"{w.name} {tag}: round trip differs")
+            del seq_pm, heads_pm, back_pm
+            torch.cuda.empty_cache()
         if w.T in (32768, 131072):
             # one rank per GPU, all W ranks' shares on this GPU back to back
             # (the same bytes as the one-GPU call)
@@ -756,6 +1134,26 @@ def run_workload_report(args):
             del heads, back_full, back
         del x, send
         torch.cuda.empty_cache()
+    # a plane larger than the window: the long sequence over 2 ranks, where one
+    # plane of one rank is 1.79 GB, moves in two token chunks per plane
+    w = wl.QKVG_250K_W2_CHUNKED
+    x = wl.packed_operand(w, device=dev)
+    part = rr.partition(w.T, w.H, w.W)
+    send = rr.split_rows(x, part.token_starts)
+    heads = rr.alloc_head_side(w.T, w.P, w.H, w.D, w.W, dev)
+    back_full, back = rr.alloc_seq_side(w.T, w.P, w.H, w.D, w.W, dev)
+    nbytes = 2 * x.numel() * 2
+    for wb, tag in ((w.window_bytes, "token_chunks"), (0, "unchunked")):
+        info = rr.seq_to_head(send, heads, window_bytes=wb)
+        secs = _time_calls(lambda: rr.seq_to_head(send, heads, window_bytes=wb), iters)
+        emit(w.name, "seq_to_head", tag, nbytes, secs, info)
+        info = rr.head_to_seq(heads, back, window_bytes=wb)
+        secs = _time_calls(lambda: rr.head_to_seq(heads, back, window_bytes=wb), iters)
+        emit(w.name, "head_to_seq", tag, nbytes, secs, info)
+        if not torch.equal(back_full.view(torch.int16), x.view(torch.int16)):
+            raise SystemExit(f"{w.name} {tag}: round trip differs")
+    del x, send, heads, back_full, back
+    torch.cuda.empty_cache()
     for rw in (wl.RS_64K_W8, wl.ReduceWorkload("reduce_scatter_T32768_C7168_W6", T=32768,
                                                C=wl.H3_HIDDEN, W=6, seed=102)):
         partials, bias = wl.partials_and_bias(rw, dev)
@@ -831,10 +1229,10 @@ def run_workload_report(args):
 def parse_args(argv=None):
     p = argparse.ArgumentParser(description=__doc__.split("\n")[0])
     p.add_argument("--gpus", type=int, default=1)
-    p.add_argument("--steps", type=int, default=1000)
-    p.add_argument("--warmup", type=int, default=20)
+    p.add_argument("--steps", type=int, default=200)
+    p.add_argument("--warmup", type=int, default=10)
     p.add_argument("--impl", choices=["native", "reference"], default="native")
-    p.add_argument("--e2e-steps", type=int, default=16)
+    p.add_argument("--e2e-steps", type=int, default=4)
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--cpu-budget", type=float, default=12.0,
                    help="about how many seconds cpu_baseline spends on the oracle")
@@ -842,7 +1240,11 @@ def parse_args(argv=None):
                                          "gated_reduce_scatter", "all_gather",
                                          "staged_seq_to_head", "rank_seq_to_head"],
                    help="run only this kernel of the step --steps times (ncu captures); no timing")
-    p.add_argument("--profile-tokens", type=int, default=STEP_T)
+    p.add_argument("--profile-tokens", type=int, default=RELAYOUT.T)
+    p.add_argument("--profile-rows", type=int, default=REDUCE.T)
+    p.add_argument("--profile-layout", type=int, default=0,
+                   help="relayout buffers for --profile: bit 1 sequence side plane-major, "
+                        "bit 2 head side plane-major (h3_*_layout)")
     p.add_argument("--report-workloads", action="store_true",
                    help="time every kernel and variant on every workload (one JSON line each)")
     p.add_argument("--reference-budget", type=float, default=90.0,

@@ -10,6 +10,8 @@ import pytest
 pytestmark = pytest.mark.gpu
 
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+sys.path.insert(0, ROOT)
+import bench  # noqa: E402
 
 
 def _run(args):
@@ -27,7 +29,10 @@ def test_native_line():
     assert d["steps"] == 100 and d["warmup"] == 3 and d["ms_per_step"] > 0
     assert d["higher_is_better"] is True and d["scaling"] == "weak" and d["vs_baseline"] is None
     assert d["dtype"] == "bf16" and d["data"] == "synthetic"
-    assert d["config"]["workload"] == "h3_transport_step_T32768_W6"
+    assert d["config"]["workload"] == bench.WORKLOAD == \
+        "qkvg_T250000_W4_chunked+reduce_scatter_T65536_C7168_W8"
+    assert d["config"]["relayout"]["window_bytes"] == 896_000_000
+    assert d["config"]["bytes_per_step"] == 2 * 2 * 14_336_000_000 + 8_455_731_200
     assert d["value"] > 1000.0
     n = d["pct_of_nominal_peak"]
     assert n["peak_gbs"] == 8000.0 and abs(n["value"] - 100.0 * d["value"] / 8000.0) < 0.01
@@ -42,9 +47,14 @@ def test_native_line():
     assert isinstance(c["cpu_model"], str) and c["cpu_model"]
     e = d["e2e"]
     assert e["unit"] == d["unit"] and 0 < e["value"] < d["value"]
-    assert e["h2d_bytes_per_step"] == 4_227_872_768 and e["d2h_bytes_per_step"] == 1_879_048_192
+    # in: QKVG, 8 partials, bias; out: the QKVG round trip and the reduce rows
+    assert e["h2d_bytes_per_step"] == 14_336_000_000 + 7_516_192_768 + 14_336
+    assert e["d2h_bytes_per_step"] == 14_336_000_000 + 939_524_096
     assert e["round_trip_ok"] is True
-    assert d["gpu_launches"] == 5 * d["steps"]
+    # one batch plane per launch each way (4 + 4) and one reduce-scatter launch
+    assert d["gpu_launches"] == 9 * d["steps"]
+    assert {k: v["launches_per_step"] for k, v in d["kernels"].items()} == \
+        {"seq_to_head": 4, "head_to_seq": 4, "ragged_reduce_scatter": 1}
     k = d["clocks"]
     assert k["samples"] > 0 and k["sm_mhz"] > 0 and k["sm_max_mhz"] >= k["sm_mhz"]
     assert isinstance(k["reasons"], list)
@@ -59,14 +69,18 @@ def test_reference_line():
     assert d["e2e"]["h2d_bytes_per_step"] == 0 and d["e2e"]["value"] == d["value"]
 
 
-@pytest.mark.parametrize("mode,launches", [
-    ("seq_to_head", 2), ("head_to_seq", 6), ("reduce_scatter", 2), ("gated_reduce_scatter", 2),
-    ("all_gather", 2), ("staged_seq_to_head", 12), ("rank_seq_to_head", 2)])
-def test_profile_modes_run(mode, launches):
-    """Every --profile mode (the commands of the ncu captures) runs its kernel."""
+@pytest.mark.parametrize("mode,layout,launches", [
+    ("seq_to_head", 0, 8), ("head_to_seq", 0, 8), ("seq_to_head", 3, 8), ("head_to_seq", 2, 8),
+    ("reduce_scatter", 0, 2), ("gated_reduce_scatter", 0, 2), ("all_gather", 0, 2),
+    ("staged_seq_to_head", 0, 16), ("rank_seq_to_head", 0, 8)])
+def test_profile_modes_run(mode, layout, launches):
+    """Every --profile mode (the commands of the ncu captures) runs its kernel:
+    the relayouts one batch plane per launch (4 planes, 2 calls)."""
     out = subprocess.run([sys.executable, "bench.py", "--profile", mode, "--steps", "2",
-                          "--profile-tokens", "4096"], cwd=ROOT, capture_output=True, text=True,
-                         timeout=600)
+                          "--profile-tokens", "4096", "--profile-rows", "4096",
+                          "--profile-layout", str(layout)], cwd=ROOT, capture_output=True,
+                         text=True, timeout=600)
     assert out.returncode == 0, out.stdout[-2000:] + out.stderr[-2000:]
     rec = json.loads([l for l in out.stdout.splitlines() if l.startswith("{")][-1])
-    assert rec["profile"] == mode and rec["tokens"] == 4096 and rec["launches"] == launches
+    assert rec["profile"] == mode and rec["launches"] == launches
+    assert rec["tokens" if "reduce" not in mode and mode != "all_gather" else "rows"] == 4096

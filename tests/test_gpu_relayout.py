@@ -404,8 +404,7 @@ def test_full_qkvg_250k_w2_sub_plane(oracle_lib):
     """The long-sequence operand over 2 ranks: one plane of one rank is
     1,792,000,000 bytes, twice the 896,000,000-byte window, so every plane
     moves in two token chunks."""
-    w = wl.RelayoutWorkload("qkvg_T250000_W2_chunked", T=250000, P=4, W=2, seed=6,
-                            window_bytes=896_000_000)
+    w = wl.QKVG_250K_W2_CHUNKED
     assert rr.relayout_chunk_plan(w.T, w.P, w.H, w.D, w.W, w.window_bytes) == (62500, 8)
     info, info_back = _full_size_round_trip(oracle_lib, w, window=w.window_bytes)
     for i in (info, info_back):

@@ -79,8 +79,14 @@ QKVG_250K_W4_CHUNKED = RelayoutWorkload(
     "qkvg_T250000_W4_chunked", T=250000, P=4, W=4, seed=5, n_segs=1, window_bytes=896_000_000,
     description="packed QKVG BF16 [250000,4,56,128], one plane per launch under an 896,000,000-byte window; both directions")
 
+# The long sequence over two ranks: one plane of one rank (1,792,000,000 bytes)
+# is twice the window, so each plane moves in token chunks.
+QKVG_250K_W2_CHUNKED = RelayoutWorkload(
+    "qkvg_T250000_W2_chunked", T=250000, P=4, W=2, seed=6, n_segs=1, window_bytes=896_000_000,
+    description="packed QKVG BF16 [250000,4,56,128] over 2 ranks; planes larger than the window, two token chunks each")
+
 WORKLOADS = {w.name: w for w in (TINY_QKV_W2, QKV_32K_W6, QKVG_128K_W4, RS_64K_W8,
-                                 QKVG_250K_W4_CHUNKED)}
+                                 QKVG_250K_W4_CHUNKED, QKVG_250K_W2_CHUNKED)}
 
 
 def _generator(seed: int, device) -> torch.Generator:
