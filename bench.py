@@ -68,33 +68,33 @@ def dist_env():
     return rank, world, local
 
 
-def max_over_ranks(x: float, device) -> float:
-    """Largest value of x over all ranks (x itself without a process group)."""
+def _reduce_over_ranks(x: float, device, op) -> float:
+    """x reduced over all ranks with `op` (x itself without a process group);
+    gloo reduces a host tensor, NCCL one on `device`."""
     import torch.distributed as dist
     if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
         return float(x)
-    t = torch.tensor([float(x)], dtype=torch.float64, device=device)
-    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    dev = device if dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([float(x)], dtype=torch.float64, device=dev)
+    dist.all_reduce(t, op=op)
     return float(t.item())
+
+
+def max_over_ranks(x: float, device) -> float:
+    """Largest value of x over all ranks (x itself without a process group)."""
+    import torch.distributed as dist
+    return _reduce_over_ranks(x, device, dist.ReduceOp.MAX)
 
 
 def sum_over_ranks(x: float, device) -> float:
     import torch.distributed as dist
-    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
-        return float(x)
-    t = torch.tensor([float(x)], dtype=torch.float64, device=device)
-    dist.all_reduce(t, op=dist.ReduceOp.SUM)
-    return float(t.item())
+    return _reduce_over_ranks(x, device, dist.ReduceOp.SUM)
 
 
 def min_over_ranks(x: float, device) -> float:
     """Smallest value of x over all ranks (x itself without a process group)."""
     import torch.distributed as dist
-    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
-        return float(x)
-    t = torch.tensor([float(x)], dtype=torch.float64, device=device)
-    dist.all_reduce(t, op=dist.ReduceOp.MIN)
-    return float(t.item())
+    return _reduce_over_ranks(x, device, dist.ReduceOp.MIN)
 
 
 def throughput_gbs(bytes_per_step_per_gpu: float, steps: int, n_gpus: int, seconds: float) -> float:
@@ -960,9 +960,11 @@ def run_profile(args):
     launches = 0
     for _ in range(args.steps):
         if args.profile == "seq_to_head":
-            info = rr.seq_to_head_layout(step.send, step.heads, layout, window_bytes=step.window)
+            info = rr.seq_to_head_layout(step.send, step.heads, layout, window_bytes=step.window,
+                                         variant=args.profile_variant)
         elif args.profile == "head_to_seq":
-            info = rr.head_to_seq_layout(step.heads, step.back, layout, window_bytes=step.window)
+            info = rr.head_to_seq_layout(step.heads, step.back, layout, window_bytes=step.window,
+                                         variant=args.profile_variant)
         elif args.profile == "reduce_scatter":
             info = rr.ragged_reduce_scatter(step.partial_list, step.bias, step.red_out)
         elif args.profile == "gated_reduce_scatter":
@@ -1085,6 +1087,37 @@ def run_workload_report(args):
                 emit(w.name, call, "rank_shares", nbytes, secs, info)
             if not torch.equal(back_full.view(torch.int16), x.view(torch.int16)):
                 raise SystemExit(f"{w.name} rank shares: round trip differs")
+            # the same W shares at once, one stream each: every source row is
+            # read by all W pulls at about the same time, as when W GPUs pull
+            # from one GPU's memory (no share waits on another)
+            side = [torch.cuda.Stream(dev) for _ in range(w.W)]
+
+            def concurrently(share):
+                def fn():
+                    cur = torch.cuda.current_stream(dev)
+                    for st in side:
+                        st.wait_stream(cur)
+                    for k in range(w.W):
+                        last = share(k, side[k])
+                    for st in side:
+                        cur.wait_stream(st)
+                    return last
+                return fn
+
+            back_full.zero_()
+            for call, fn in (
+                    ("seq_to_head", concurrently(lambda k, st: rr.seq_to_head_rank(
+                        send, heads[k], k, n_heads=w.H, window_bytes=w.window_bytes, stream=st))),
+                    ("head_to_seq", concurrently(lambda k, st: rr.head_to_seq_rank(
+                        heads, back[k], k, n_tokens=w.T, window_bytes=w.window_bytes, stream=st)))):
+                info = dict(fn())
+                info["launches"] *= w.W
+                secs = _time_calls(fn, iters)
+                emit(w.name, call, "rank_shares_concurrent", nbytes, secs, info)
+            torch.cuda.synchronize()
+            if not torch.equal(back_full.view(torch.int16), x.view(torch.int16)):
+                raise SystemExit(f"{w.name} concurrent rank shares: round trip differs")
+            del side
         if w.T < 32768:
             # small case: host overhead per call dominates; a prepared call
             # (checks and marshalling done once) and CUDA-graph replay
@@ -1232,7 +1265,7 @@ def parse_args(argv=None):
     p.add_argument("--steps", type=int, default=200)
     p.add_argument("--warmup", type=int, default=10)
     p.add_argument("--impl", choices=["native", "reference"], default="native")
-    p.add_argument("--e2e-steps", type=int, default=4)
+    p.add_argument("--e2e-steps", type=int, default=10)
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--cpu-budget", type=float, default=12.0,
                    help="about how many seconds cpu_baseline spends on the oracle")
@@ -1242,6 +1275,8 @@ def parse_args(argv=None):
                    help="run only this kernel of the step --steps times (ncu captures); no timing")
     p.add_argument("--profile-tokens", type=int, default=RELAYOUT.T)
     p.add_argument("--profile-rows", type=int, default=REDUCE.T)
+    p.add_argument("--profile-variant", type=int, default=0,
+                   help="relayout kernel family for --profile: 0 default, 1 vector, 2 bulk (TMA ring)")
     p.add_argument("--profile-layout", type=int, default=0,
                    help="relayout buffers for --profile: bit 1 sequence side plane-major, "
                         "bit 2 head side plane-major (h3_*_layout)")
