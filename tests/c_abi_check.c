@@ -47,6 +47,14 @@ int main(void)
 
     expect(h3_staged_plan(250000, 4, 56, 128, 896000000, &chunk_tokens, &chunks) == H3_OK &&
            chunk_tokens == 62500 && chunks == 16, "staged plan");
+    /* the long sequence over 4 ranks: one plane per launch at the pages'
+     * window; over 2 ranks each plane moves in two token chunks */
+    expect(h3_relayout_chunk_plan(250000, 4, 56, 128, 4, 896000000, &chunk_tokens, &chunks) ==
+           H3_OK && chunk_tokens == 62500 && chunks == 4, "chunk plan, 4 ranks");
+    expect(h3_relayout_chunk_plan(250000, 4, 56, 128, 2, 896000000, &chunk_tokens, &chunks) ==
+           H3_OK && chunk_tokens == 62500 && chunks == 8, "chunk plan, 2 ranks");
+    expect(h3_relayout_chunk_plan(250000, 4, 56, 128, 4, 14335, &chunk_tokens, &chunks) ==
+           H3_ERR_WINDOW, "window below one token");
 
     /* argument checks fail before anything is launched */
     expect(h3_seq_to_head(NULL, NULL, 1000, 3, 56, 128, 6, 0, NULL, &info) == H3_ERR_INVALID_ARG &&

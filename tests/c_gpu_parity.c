@@ -4,9 +4,10 @@
  * (oracle/h3_oracle.c, linked as test infrastructure).  Built and run by
  * tests/test_gpu_c_program.py.
  *
- * Cases: both Ulysses relayouts ("Distributed H3 Execution", intro), whole
- * and one batch plane per launch (FastVideo PR #1807, "Problem and
- * behavior"); the ragged reduce-scatter and the ragged all-gather
+ * Cases: both Ulysses relayouts ("Distributed H3 Execution", intro), whole,
+ * one batch plane per launch and in token chunks of a plane (FastVideo PR
+ * #1807, "Problem and behavior"); the ragged reduce-scatter and the ragged
+ * all-gather
  * ("Distributed H3 Execution", "Partition Contract"). */
 #include <stdint.h>
 #include <stdio.h>
@@ -140,9 +141,14 @@ static void relayout_case(int64_t T, int32_t P, int32_t H, int32_t D, int32_t W,
     expect(h3o_head_to_seq((const uint16_t* const*)want, back_want, T, P, H, D, W) == 0,
            "oracle h2s");
 
-    expect(h3_seq_to_head((const void* const*)d_send, d_heads, T, P, H, D, W, window, stream,
-                          &info) == H3_OK, "h3_seq_to_head status");
-    expect(info.launches == (window > 0 ? P : 1), "seq->head launches");
+    {
+        int64_t tokens = 0, chunks = 0;
+        expect(h3_relayout_chunk_plan(T, P, H, D, W, window, &tokens, &chunks) == H3_OK,
+               "chunk plan");
+        expect(h3_seq_to_head((const void* const*)d_send, d_heads, T, P, H, D, W, window, stream,
+                              &info) == H3_OK, "h3_seq_to_head status");
+        expect(info.launches == chunks && info.chunks == chunks, "seq->head launches");
+    }
     expect(h3_head_to_seq((const void* const*)d_heads, d_back, T, P, H, D, W, window, stream,
                           &info) == H3_OK, "h3_head_to_seq status");
     cuda_ok(cudaStreamSynchronize(stream), "relayout sync");
@@ -242,6 +248,9 @@ int main(void)
     /* one plane per launch: the window holds the largest plane slice (rank
      * 0's 167 tokens x 56 heads and 1000 tokens x 10 heads, both x 256 B) */
     relayout_case(1000, 3, 56, 128, 6, 1000 * 10 * 256, stream);
+    /* a window of a third of a plane: every plane in token chunks (at most 55
+     * tokens of every rank fit, so 4 chunks of 42 per plane) */
+    relayout_case(1000, 3, 56, 128, 6, 1000 * 10 * 256 / 3, stream);
     relayout_case(777, 4, 56, 128, 8, 0, stream);
     relayout_case(97, 2, 9, 8, 3, 0, stream);
     reduce_gather_case(777, 7168, 8, stream);
