@@ -520,7 +520,7 @@ def nccl_fence(device):
     return fence
 
 
-def time_steps(step, K: int, timer, stream, local, device, n_events: int):
+def time_steps(step, K: int, timer, stream, local, n_events: int):
     """Run K steps between barriers; (seconds, launches, per-kernel seconds)."""
     evs = [[timer.event() for _ in range(n_events)] for _ in range(K)]
     start, end = timer.event(), timer.event()
@@ -681,7 +681,7 @@ def measure(args, make_step, rank, world, local, device, timer, n_events):
 
     K = args.steps
     with ClockSampler(gpu_uuid(device) if isinstance(timer, CudaTimer) else None) as clocks:
-        elapsed, launches, per_kernel_s = time_steps(step, K, timer, stream, local, device, n_events)
+        elapsed, launches, per_kernel_s = time_steps(step, K, timer, stream, local, n_events)
     t_max = max_over_ranks(elapsed, device)
     launches_total = int(sum_over_ranks(launches, device))
     value = throughput_gbs(step.bytes_per_step, K, 1, t_max)
