@@ -17,6 +17,7 @@ scaling, whole-job bytes, every kernel timed, launches summed over ranks),
 the order of the calls and fences in every step, the peer tables' exchange
 order, and that the per-rank check of the results catches a wrong share.
 """
+import json
 import os
 import socket
 import sys
@@ -66,10 +67,10 @@ class ShmIpc:
 
     def export(self, tensor):
         path, shape, dtype = self.files[tensor.data_ptr()]
-        return repr((path, shape, dtype)).encode()
+        return json.dumps([path, list(shape), dtype]).encode()
 
     def open(self, record, device):
-        path, shape, dtype = eval(record.decode())  # our own repr() of plain tuples
+        path, shape, dtype = json.loads(record.decode())
         dt = getattr(torch, dtype.split(".")[1])
         t = torch.from_file(path, shared=True, size=int(np.prod(shape)), dtype=dt).view(shape)
         self.by_address[t.data_ptr()] = t
