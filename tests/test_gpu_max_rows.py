@@ -87,6 +87,36 @@ def test_relayouts_at_the_row_limit(oracle_lib):
     del send, heads, flat_in, flat_out
 
 
+def test_token_chunked_relayouts_at_the_row_limit(oracle_lib):
+    """A window of a third of the plane: the plane of 2^31 - 1 rows moves in
+    three token chunks, the last starting above row 2^30 (chunk offsets and
+    rows stay in the kernels' 32-bit range; byte offsets above 2^35)."""
+    T, P, H, D, W = MAX_ROWS, 1, 1, 8, 1
+    nbytes = T * P * H * D * 2
+    _need(2 * nbytes)
+    window = nbytes // 3 + 16
+    L, chunks = rr.relayout_chunk_plan(T, P, H, D, W, window)
+    assert chunks == 3 and 2 * L < T <= 3 * L
+    send = wl.normal_bf16((T, P, H, D), 2034, 1.0, DEV)
+    heads = [torch.empty((T, P, H, D), dtype=torch.bfloat16, device=DEV)]
+    info = rr.seq_to_head([send], heads, window_bytes=window)
+    assert info["launches"] == 3 and info["chunks"] == 3
+    torch.cuda.synchronize()
+    assert _same_in_chunks(heads[0], send)
+    elems = _sample_elems(T * P * H * D, 3)
+    flat_in = send.view(-1).view(torch.int16)
+    keep = flat_in.index_select(0, torch.from_numpy(elems).to(DEV)).cpu().numpy()
+    src_rank, src_elem = oracle_lib.head_to_seq_locate(T, P, H, D, W, 0, elems)
+    assert np.all(src_rank == 0) and np.array_equal(np.asarray(src_elem), elems)
+    send.view(torch.int16).fill_(0x7fc1)
+    info = rr.head_to_seq(heads, [send], window_bytes=window)
+    assert info["launches"] == 3
+    torch.cuda.synchronize()
+    assert _same_in_chunks(send, heads[0])
+    assert np.array_equal(flat_in.index_select(0, torch.from_numpy(elems).to(DEV)).cpu().numpy(), keep)
+    del send, heads, flat_in
+
+
 def test_reduce_scatter_and_all_gather_at_the_row_limit(oracle_lib):
     T, C, W = MAX_ROWS, 8, 2
     row_bytes = C * 2
