@@ -615,7 +615,27 @@ def run_e2e(make_step, first, n_steps: int, local, device, world: int, timer):
     e1.record(s_in)
     barrier(local, timer)
     t_e2e = max_over_ranks(e0.elapsed_time(e1) / 1e3, device)
-    # the round trip comes back unchanged
+    # the link's own bound: the same copies, both directions at once, no kernels
+    torch.cuda.synchronize()
+    barrier(local, timer)
+    c0 = torch.cuda.Event(enable_timing=True)
+    c1 = torch.cuda.Event(enable_timing=True)
+    c0.record(s_in)
+    s_out.wait_stream(s_in)
+    link_steps = 2
+    for _ in range(link_steps):
+        with torch.cuda.stream(s_in):
+            for name, dst in bufs[0].inputs().items():
+                dst.copy_(ins[name], non_blocking=True)
+        with torch.cuda.stream(s_out):
+            for name, src in bufs[1].outputs().items():
+                outs[name].copy_(src, non_blocking=True)
+    s_in.wait_stream(s_out)
+    c1.record(s_in)
+    barrier(local, timer)
+    t_link = max_over_ranks(c0.elapsed_time(c1) / 1e3 / link_steps, device)
+    # the round trip comes back unchanged (the last step's results, copied
+    # again above from the same buffers)
     key_in, key_out = ("qkv", "back") if "qkv" in ins else ("send", "back")
     ok = torch.equal(outs[key_out].view(torch.int16), ins[key_in].view(torch.int16))
     ok = bool(min_over_ranks(1.0 if ok else 0.0, device) > 0)
@@ -630,6 +650,8 @@ def run_e2e(make_step, first, n_steps: int, local, device, world: int, timer):
             "h2d_bytes_per_step": int(sum_over_ranks(h2d, device)),
             "d2h_bytes_per_step": int(sum_over_ranks(d2h, device)),
             "steps": n_steps, "ms_per_step": round(t_e2e / n_steps * 1e3, 3),
+            "link_bound_ms_per_step": round(t_link * 1e3, 3),
+            "frac_of_link_bound": round(t_link / (t_e2e / n_steps), 3),
             "mode": "pinned host buffers; copies in, kernels and copies out on three streams, "
                     "two device buffer sets" + (f", {world} GPUs" if world > 1 else ""),
             "round_trip_ok": ok}

@@ -51,6 +51,8 @@ def test_native_line():
     assert e["h2d_bytes_per_step"] == 14_336_000_000 + 7_516_192_768 + 14_336
     assert e["d2h_bytes_per_step"] == 14_336_000_000 + 939_524_096
     assert e["round_trip_ok"] is True
+    # the same copies alone bound the end-to-end step from below
+    assert 0 < e["link_bound_ms_per_step"] and 0 < e["frac_of_link_bound"] <= 1.05
     # one batch plane per launch each way (4 + 4) and one reduce-scatter launch
     assert d["gpu_launches"] == 9 * d["steps"]
     assert {k: v["launches_per_step"] for k, v in d["kernels"].items()} == \
