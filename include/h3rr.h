@@ -496,7 +496,10 @@ H3RR_API h3_status h3_seq_to_head_rank(const void* const* send, void* recv, int6
 
 /* Rank k's sequence-side buffer: recv [T_k, P, H, D] (this GPU) gets
  * recv[t', p, hs_j + h, d] = send[j][ts_k + t', p, h, d] from send[world],
- * the head-side buffers [T, P, H_j, D] of all ranks. */
+ * the head-side buffers [T, P, H_j, D] of all ranks.  Under a window that
+ * splits planes into token chunks, info->chunks is the plan's count and
+ * info->launches counts only the chunks that hold tokens of rank k (the
+ * last chunk of a plane may hold none of a smaller rank's tokens). */
 H3RR_API h3_status h3_head_to_seq_rank(const void* const* send, void* recv, int64_t n_tokens,
                                        int32_t planes, int32_t n_heads, int32_t head_dim,
                                        int32_t world, int32_t rank, int64_t window_bytes,
