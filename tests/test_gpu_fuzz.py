@@ -42,10 +42,12 @@ def test_fuzz_relayout(oracle_lib, case):
     shape = (lambda j: (P, T, part.heads(j), D)) if hpm else (lambda j: (T, P, part.heads(j), D))
     heads = [torch.empty(shape(j), dtype=torch.bfloat16, device=DEV) for j in range(W)]
     plane = max(part.tokens(0) * H * D * 2, T * part.heads(0) * D * 2)
-    window = int(rng.choice([0, plane, plane * P]))
+    smallest = max(H * D * 2, W * part.heads(0) * D * 2)  # one token of every rank
+    # no window, a whole plane, more than a plane, or less than a plane (token chunks)
+    window = int(rng.choice([0, plane, plane * P, int(rng.integers(smallest, plane + 1))]))
     variant = int(rng.choice([0, rr.H3_VARIANT_VECTOR]))
     info = rr.seq_to_head_layout(send, heads, layout, window_bytes=window, variant=variant)
-    assert info["launches"] == (P if window else 1)
+    assert info["launches"] == rr.relayout_chunk_plan(T, P, H, D, W, window)[1]
     want = oracle_lib.relayout_layout([gu.bits(s) for s in send], T, P, H, D, W, True, spm, hpm)
     for j in range(W):
         assert np.array_equal(gu.bits(heads[j]), want[j]), (T, P, H, D, W, layout, j)
@@ -58,6 +60,15 @@ def test_fuzz_relayout(oracle_lib, case):
         rr.seq_to_head(send, bulk, window_bytes=window, variant=rr.H3_VARIANT_BULK)
         for j in range(W):
             assert gu.same_bits(bulk[j], heads[j])
+    if layout == 0:
+        # one rank's shares (one rank per GPU) under the same window
+        k = int(rng.integers(0, W))
+        mine = torch.empty_like(heads[k])
+        rr.seq_to_head_rank(send, mine, k, n_heads=H, window_bytes=window)
+        assert gu.same_bits(mine, heads[k]), (T, P, H, D, W, window, k)
+        rows = torch.empty_like(send[k])
+        rr.head_to_seq_rank(heads, rows, k, n_tokens=T, window_bytes=window)
+        assert gu.same_bits(rows, send[k]), (T, P, H, D, W, window, k)
 
 
 @pytest.mark.parametrize("case", range(N_CASES // 2))

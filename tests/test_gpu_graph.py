@@ -2,10 +2,10 @@
 
 Every call enqueues its kernels on the caller's stream and does nothing that
 breaks stream capture once a first, eager call has run (per-device caches,
-shared-memory opt-in).  A whole step -- seq->head, chunked head->seq,
-reduce-scatter, all-gather, gated reduce-scatter -- is captured once, the
-inputs are overwritten in place, and each replay must give the oracle's
-results for the new inputs."""
+shared-memory opt-in).  A whole step -- seq->head in token chunks, head->seq
+one plane per launch, reduce-scatter, all-gather, gated reduce-scatter -- is
+captured once, the inputs are overwritten in place, and each replay must give
+the oracle's results for the new inputs."""
 import numpy as np
 import pytest
 import torch
@@ -37,8 +37,12 @@ def test_step_replays_from_a_cuda_graph(oracle_lib):
     resid_full = resid_src.clone()
     resid = rr.split_rows(resid_full, rr.partition(T, W, W).token_starts)
 
+    # seq->head with every plane in token chunks, head->seq one plane per launch
+    sub = gu.chunk_window("sub", T, H, D, W)
+    assert rr.relayout_chunk_plan(T, P, H, D, W, sub)[1] > P
+
     def step():
-        rr.seq_to_head(send, heads)
+        rr.seq_to_head(send, heads, window_bytes=sub)
         rr.head_to_seq(heads, back, window_bytes=window)
         rr.ragged_reduce_scatter(partials, bias, red)
         rr.ragged_all_gather(red, gath)

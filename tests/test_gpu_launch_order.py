@@ -19,18 +19,18 @@ pytestmark = pytest.mark.gpu
 DEV = "cuda"
 
 
-@pytest.mark.parametrize("chunked", [False, True])
+@pytest.mark.parametrize("chunked", [None, "plane", "sub"])
 def test_serial_and_programmatic_launches_agree(oracle_lib, chunked):
     T, P, H, D, W = 1000, 4, 56, 128, 6
     part = rr.partition(T, H, W)
     x = wl.random_bits((T, P, H, D), 71, DEV)
     send = rr.split_rows(x, part.token_starts)
-    window = max(part.tokens(0) * H * D * 2, T * part.heads(0) * D * 2) if chunked else 0
+    window = gu.chunk_window(chunked, T, H, D, W)
     outs = {}
     for serial in (False, True):
         heads = rr.alloc_head_side(T, P, H, D, W, DEV)
         info = rr.seq_to_head(send, heads, window_bytes=window, serial=serial)
-        assert info["launches"] == (P if chunked else 1)
+        assert info["launches"] == rr.relayout_chunk_plan(T, P, H, D, W, window)[1]
         back_full, back = rr.alloc_seq_side(T, P, H, D, W, DEV)
         rr.head_to_seq(heads, back, window_bytes=window, serial=serial)
         outs[serial] = (heads, back_full)
@@ -42,9 +42,11 @@ def test_serial_and_programmatic_launches_agree(oracle_lib, chunked):
 
 
 @pytest.mark.parametrize("serial", [False, True])
-def test_chained_dependent_calls(oracle_lib, serial):
-    """x -> heads -> back -> heads2 -> back2, all chunked, on one stream, with
-    a fresh x written by a PyTorch kernel before every round."""
+@pytest.mark.parametrize("chunked", ["plane", "sub"])
+def test_chained_dependent_calls(oracle_lib, serial, chunked):
+    """x -> heads -> back -> heads2 -> back2, all chunked (one plane per
+    launch, or every plane in token chunks), on one stream, with a fresh x
+    written by a PyTorch kernel before every round."""
     T, P, H, D, W = 4096, 4, 56, 128, 6
     part = rr.partition(T, H, W)
     x = torch.empty((T, P, H, D), dtype=torch.bfloat16, device=DEV)
@@ -53,7 +55,10 @@ def test_chained_dependent_calls(oracle_lib, serial):
     heads2 = rr.alloc_head_side(T, P, H, D, W, DEV)
     back_full, back = rr.alloc_seq_side(T, P, H, D, W, DEV)
     back2_full, back2 = rr.alloc_seq_side(T, P, H, D, W, DEV)
-    window = max(part.tokens(0) * H * D * 2, T * part.heads(0) * D * 2)
+    window = gu.chunk_window(chunked, T, H, D, W)
+    if chunked == "sub":
+        window //= 3  # about six token chunks per plane: long chains of launches
+        assert rr.relayout_chunk_plan(T, P, H, D, W, window)[1] >= 5 * P
     for round_ in range(8):
         x.copy_(wl.random_bits((T, P, H, D), 500 + round_, DEV))
         rr.seq_to_head(send, heads, window_bytes=window, serial=serial)

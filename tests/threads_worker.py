@@ -134,7 +134,7 @@ def main():
     o = oracle.load()
     jobs = [
         Relayout(o, 401, 1000, 3, 56, 128, 6),
-        Relayout(o, 402, 777, 4, 56, 128, 8, window=2_000_000),
+        Relayout(o, 402, 777, 4, 56, 128, 8, window=700_000),  # 3 token chunks per plane
         Relayout(o, 403, 513, 1, 56, 128, 4, variant=rr.H3_VARIANT_BULK),
         Relayout(o, 404, 1000, 3, 56, 128, 6, variant=rr.H3_VARIANT_BULK),
         Staged(o, 405, 600, 3, 56, 128, 5, window_rows=41),
