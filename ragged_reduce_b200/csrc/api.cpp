@@ -75,6 +75,8 @@ h3_status check_no_overlap(const void* const* in, const uint64_t* in_bytes, int 
 
 namespace {
 
+// Shared checks of the relayout calls: world, shapes, pointers, alignment,
+// overlap.  `extra_out` (nullable) is one more output range (the window).
 h3_status check_relayout_args(bool seq_to_head, const void* const* send, void* const* recv,
                               int64_t n_tokens, int32_t planes, int32_t n_heads, int32_t head_dim,
                               int32_t world, void* extra_out, uint64_t extra_bytes)
@@ -231,8 +233,8 @@ h3_status relayout(bool seq_to_head, const void* const* send, void* const* recv,
     return H3_OK;
 }
 
-// Shared checks of the relayout calls: world, shapes, pointers, alignment,
-// overlap.  `extra_out` (nullable) is one more output range (the window).
+// Tokens per chunk of a staged call: as many whole token rows (H*D*2 bytes)
+// as the window holds, at most T; H3_ERR_WINDOW below one row.
 h3_status staged_plan(int64_t n_tokens, int32_t n_heads, int32_t head_dim, int64_t window_bytes,
                       int64_t* chunk_tokens)
 {
