@@ -50,10 +50,12 @@
  *   - `info` (nullable) receives what actually ran: launches, chunks, grid,
  *     block and kernel variant.
  *   - Thread-safe, and no environment variables are read.  State kept across
- *     calls: per-device caches (SM count, resident CTAs per kernel, the
- *     shared-memory opt-in, the static window's address per context), each
- *     thread's last CUDA error, the device-side counters of expired bounded
- *     waits, and the peer mappings h3_ipc_open holds until h3_ipc_close.
+ *     calls: per-device caches (SM count, resident CTAs per kernel),
+ *     per-context state (the bulk kernels' shared-memory opt-in, the static
+ *     window's address, the peer mappings h3_ipc_open holds until
+ *     h3_ipc_close; after cudaDeviceReset the device's next context sets them
+ *     up again), each thread's last CUDA error, and the device-side counters
+ *     of expired bounded waits.
  */
 #ifndef H3RR_H
 #define H3RR_H

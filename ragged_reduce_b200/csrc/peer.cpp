@@ -14,10 +14,12 @@
 #include <cstring>
 #include <map>
 #include <mutex>
+#include <tuple>
 #include <utility>
 
 #include <cuda.h>
 
+#include "context.h"
 #include "h3rr_internal.h"
 
 using namespace h3rr;
@@ -49,17 +51,23 @@ struct Mapping {
     int64_t refs = 0;
 };
 
-using MappingKey = std::pair<int, std::array<unsigned char, H3_IPC_HANDLE_BYTES>>;
+// Mappings belong to a context: after cudaDeviceReset the device's next
+// context holds none of them, so the key carries the context's id (0 when
+// the driver cannot say).
+using MappingKey =
+    std::tuple<int, unsigned long long, std::array<unsigned char, H3_IPC_HANDLE_BYTES>>;
 
 std::mutex g_map_mutex;
 std::map<MappingKey, Mapping> g_mappings;
 
 MappingKey key_of(int device, const h3_ipc_handle* handle)
 {
-    MappingKey k;
-    k.first = device;
-    std::memcpy(k.second.data(), handle->handle, H3_IPC_HANDLE_BYTES);
-    return k;
+    unsigned long long ctx = 0;
+    if (!current_context_id(&ctx))
+        ctx = 0;
+    std::array<unsigned char, H3_IPC_HANDLE_BYTES> bytes;
+    std::memcpy(bytes.data(), handle->handle, H3_IPC_HANDLE_BYTES);
+    return MappingKey(device, ctx, bytes);
 }
 
 }  // namespace

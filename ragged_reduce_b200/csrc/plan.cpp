@@ -9,6 +9,9 @@
 #include <mutex>
 #include <unordered_map>
 
+#include <cuda.h>
+
+#include "context.h"
 #include "h3rr_internal.h"
 
 namespace h3rr {
@@ -88,6 +91,53 @@ bool ranges_overlap(uintptr_t a, uint64_t na, uintptr_t b, uint64_t nb)
     return a < b + nb && b < a + na;
 }
 
+namespace {
+
+using CtxGetCurrentFn = CUresult (*)(CUcontext*);
+using CtxGetIdFn = CUresult (*)(CUcontext, unsigned long long*);
+
+// The driver's cuCtxGetCurrent and cuCtxGetId (CUDA 12.0), fetched through
+// the runtime's entry-point query (no link against libcuda); null if
+// unavailable.
+struct ContextQuery {
+    CtxGetCurrentFn current = nullptr;
+    CtxGetIdFn id = nullptr;
+};
+
+const ContextQuery& context_query()
+{
+    static std::once_flag once;
+    static ContextQuery q;
+    std::call_once(once, [] {
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult r = cudaDriverEntryPointSymbolNotFound;
+        if (cudaGetDriverEntryPointByVersion("cuCtxGetCurrent", &p, 12000, cudaEnableDefault, &r) ==
+                cudaSuccess &&
+            r == cudaDriverEntryPointSuccess)
+            q.current = reinterpret_cast<CtxGetCurrentFn>(p);
+        p = nullptr;
+        r = cudaDriverEntryPointSymbolNotFound;
+        if (cudaGetDriverEntryPointByVersion("cuCtxGetId", &p, 12000, cudaEnableDefault, &r) ==
+                cudaSuccess &&
+            r == cudaDriverEntryPointSuccess)
+            q.id = reinterpret_cast<CtxGetIdFn>(p);
+    });
+    return q;
+}
+
+}  // namespace
+
+bool current_context_id(unsigned long long* id)
+{
+    const ContextQuery& q = context_query();
+    if (!q.current || !q.id)
+        return false;
+    CUcontext ctx = nullptr;
+    if (q.current(&ctx) != CUDA_SUCCESS || !ctx)
+        return false;
+    return q.id(ctx, id) == CUDA_SUCCESS;
+}
+
 int current_sm_count(int* device)
 {
     static std::mutex mu;
@@ -149,26 +199,37 @@ int resident_ctas(const void* kernel, int block, size_t smem, int device)
 cudaError_t allow_dynamic_smem(const void* kernel, size_t smem, int device)
 {
     // The opt-in is one value per kernel, so it is raised once per kernel and
-    // device to the device's whole opt-in limit; any later launch with a
+    // context to the device's whole opt-in limit; any later launch with a
     // smaller ring then stays within it.  (Setting it to each launch's own
-    // size would lower it under a later, larger launch.)
+    // size would lower it under a later, larger launch.)  It belongs to the
+    // context: after cudaDeviceReset the next context starts from the
+    // default, so the cache is keyed by the context's id; without an id the
+    // opt-in is set on every call.
     if (smem <= 48 * 1024)
         return cudaSuccess;
     struct Key {
         const void* k;
         int dev;
-        bool operator==(const Key& o) const { return k == o.k && dev == o.dev; }
+        unsigned long long ctx;
+        bool operator==(const Key& o) const { return k == o.k && dev == o.dev && ctx == o.ctx; }
     };
     struct Hash {
-        size_t operator()(const Key& x) const { return std::hash<const void*>()(x.k) ^ size_t(x.dev); }
+        size_t operator()(const Key& x) const
+        {
+            return std::hash<const void*>()(x.k) ^ size_t(x.dev) ^ std::hash<unsigned long long>()(x.ctx);
+        }
     };
     static std::mutex mu;
     static std::unordered_map<Key, int, Hash> limit;
+    unsigned long long ctx = 0;
+    const bool keyed = current_context_id(&ctx);
     std::lock_guard<std::mutex> lock(mu);
-    const Key key{kernel, device};
-    auto it = limit.find(key);
-    if (it != limit.end())
-        return smem <= size_t(it->second) ? cudaSuccess : cudaErrorInvalidValue;
+    const Key key{kernel, device, ctx};
+    if (keyed) {
+        auto it = limit.find(key);
+        if (it != limit.end())
+            return smem <= size_t(it->second) ? cudaSuccess : cudaErrorInvalidValue;
+    }
     int optin = 0;
     cudaError_t err = cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, device);
     if (err != cudaSuccess)
@@ -176,7 +237,7 @@ cudaError_t allow_dynamic_smem(const void* kernel, size_t smem, int device)
     if (smem > size_t(optin))
         return cudaErrorInvalidValue;
     err = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, optin);
-    if (err == cudaSuccess)
+    if (err == cudaSuccess && keyed)
         limit.emplace(key, optin);
     return err;
 }

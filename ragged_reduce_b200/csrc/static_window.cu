@@ -8,8 +8,7 @@
 #include <mutex>
 #include <utility>
 
-#include <cuda.h>
-
+#include "context.h"
 #include "h3rr_internal.h"
 
 namespace h3rr {
@@ -20,51 +19,6 @@ namespace h3rr {
 static __device__ __align__(256) unsigned char g_static_window[H3RR_STATIC_WINDOW_BYTES];
 
 namespace {
-
-using CtxGetCurrentFn = CUresult (*)(CUcontext*);
-using CtxGetIdFn = CUresult (*)(CUcontext, unsigned long long*);
-
-// The driver's cuCtxGetCurrent and cuCtxGetId (CUDA 12.0), fetched through
-// the runtime's entry-point query; null if unavailable.
-struct ContextQuery {
-    CtxGetCurrentFn current = nullptr;
-    CtxGetIdFn id = nullptr;
-};
-
-const ContextQuery& context_query()
-{
-    static std::once_flag once;
-    static ContextQuery q;
-    std::call_once(once, [] {
-        void* p = nullptr;
-        cudaDriverEntryPointQueryResult r = cudaDriverEntryPointSymbolNotFound;
-        if (cudaGetDriverEntryPointByVersion("cuCtxGetCurrent", &p, 12000, cudaEnableDefault, &r) ==
-                cudaSuccess &&
-            r == cudaDriverEntryPointSuccess)
-            q.current = reinterpret_cast<CtxGetCurrentFn>(p);
-        p = nullptr;
-        r = cudaDriverEntryPointSymbolNotFound;
-        if (cudaGetDriverEntryPointByVersion("cuCtxGetId", &p, 12000, cudaEnableDefault, &r) ==
-                cudaSuccess &&
-            r == cudaDriverEntryPointSuccess)
-            q.id = reinterpret_cast<CtxGetIdFn>(p);
-    });
-    return q;
-}
-
-// Process-unique id of the calling thread's current context (ids are never
-// reused, unlike context handles); false if there is none or the driver
-// cannot say.
-bool current_context_id(unsigned long long* id)
-{
-    const ContextQuery& q = context_query();
-    if (!q.current || !q.id)
-        return false;
-    CUcontext ctx = nullptr;
-    if (q.current(&ctx) != CUDA_SUCCESS || !ctx)
-        return false;
-    return q.id(ctx, id) == CUDA_SUCCESS;
-}
 
 // Device address of g_static_window in the current context.  Looked up with
 // cudaGetSymbolAddress once per device and context, with that device
