@@ -950,6 +950,8 @@ def run_profile(args):
     relayout = args.profile in ("seq_to_head", "head_to_seq", "staged_seq_to_head", "rank_seq_to_head")
     step = Step(device, tokens=args.profile_tokens, rows=args.profile_rows, relayout=relayout,
                 reduce=not relayout)
+    if args.profile_window >= 0:
+        step.window = args.profile_window
     rr = step.rr
     if args.profile == "head_to_seq":
         rr.seq_to_head(step.send, step.heads)
@@ -1002,7 +1004,7 @@ def run_profile(args):
         launches += info["launches"]
     torch.cuda.synchronize()
     print(json.dumps({"profile": args.profile, "tokens": step.T, "rows": step.Tr,
-                      "layout": layout, "launches": launches}), flush=True)
+                      "layout": layout, "window": step.window, "launches": launches}), flush=True)
     return 0
 
 
@@ -1297,6 +1299,9 @@ def parse_args(argv=None):
                    help="run only this kernel of the step --steps times (ncu captures); no timing")
     p.add_argument("--profile-tokens", type=int, default=RELAYOUT.T)
     p.add_argument("--profile-rows", type=int, default=REDUCE.T)
+    p.add_argument("--profile-window", type=int, default=-1,
+                   help="window bytes of the relayouts for --profile (-1: the bench's 896,000,000; "
+                        "0: one launch over all planes)")
     p.add_argument("--profile-variant", type=int, default=0,
                    help="relayout kernel family for --profile: 0 default, 1 vector, 2 bulk (TMA ring)")
     p.add_argument("--profile-layout", type=int, default=0,

@@ -71,17 +71,19 @@ def test_reference_line():
     assert d["e2e"]["h2d_bytes_per_step"] == 0 and d["e2e"]["value"] == d["value"]
 
 
-@pytest.mark.parametrize("mode,layout,launches", [
-    ("seq_to_head", 0, 8), ("head_to_seq", 0, 8), ("seq_to_head", 3, 8), ("head_to_seq", 2, 8),
-    ("reduce_scatter", 0, 2), ("gated_reduce_scatter", 0, 2), ("all_gather", 0, 2),
-    ("staged_seq_to_head", 0, 16), ("rank_seq_to_head", 0, 8)])
-def test_profile_modes_run(mode, layout, launches):
+@pytest.mark.parametrize("mode,layout,window,launches", [
+    ("seq_to_head", 0, -1, 8), ("head_to_seq", 0, -1, 8), ("seq_to_head", 3, -1, 8),
+    ("head_to_seq", 2, -1, 8), ("seq_to_head", 0, 0, 2), ("reduce_scatter", 0, -1, 2),
+    ("gated_reduce_scatter", 0, -1, 2), ("all_gather", 0, -1, 2),
+    ("staged_seq_to_head", 0, -1, 16), ("rank_seq_to_head", 0, -1, 8)])
+def test_profile_modes_run(mode, layout, window, launches):
     """Every --profile mode (the commands of the ncu captures) runs its kernel:
-    the relayouts one batch plane per launch (4 planes, 2 calls)."""
+    the relayouts one batch plane per launch (4 planes, 2 calls), or in one
+    launch with no window."""
     out = subprocess.run([sys.executable, "bench.py", "--profile", mode, "--steps", "2",
                           "--profile-tokens", "4096", "--profile-rows", "4096",
-                          "--profile-layout", str(layout)], cwd=ROOT, capture_output=True,
-                         text=True, timeout=600)
+                          "--profile-layout", str(layout), "--profile-window", str(window)],
+                         cwd=ROOT, capture_output=True, text=True, timeout=600)
     assert out.returncode == 0, out.stdout[-2000:] + out.stderr[-2000:]
     rec = json.loads([l for l in out.stdout.splitlines() if l.startswith("{")][-1])
     assert rec["profile"] == mode and rec["launches"] == launches
