@@ -517,3 +517,53 @@ def test_last_cuda_error_is_kept_per_thread():
     t2.start()
     t2.join(timeout=60)
     assert other == [0]
+
+
+def test_token_chunks_cover_every_token_once():
+    """The token chunks a chunked relayout launches, as the header defines
+    them: chunk c of a plane holds local tokens [c*L, c*L + L) of every rank
+    (fewer in the last chunk, possibly none for a smaller rank).  Over many
+    random shapes and windows, mapping each launch's token units to (rank,
+    local token) by the chunk's quotient/remainder split covers every token
+    of every rank exactly once, and every launch's per-rank slices fit the
+    window."""
+    rng = np.random.default_rng(11)
+    checked_empty_rank = False
+    for _ in range(400):
+        W = int(rng.integers(1, 17))
+        T = int(rng.integers(W, 3000))
+        H = int(rng.integers(W, 90))
+        D = 8 * int(rng.integers(1, 33))
+        P = int(rng.integers(1, 5))
+        row, head = H * D * 2, D * 2
+        part = rr.partition(T, H, W)
+        tq, tm = divmod(T, W)
+        hmax = max(part.heads(j) for j in range(W))
+        smallest = max(row, W * hmax * head)
+        window = int(rng.integers(smallest, (tq + 1) * row * 2 + 1))
+        L, chunks = rr.relayout_chunk_plan(T, P, H, D, W, window)
+        k = chunks // P
+        assert chunks == k * P and k >= 1
+        seen = {}
+        for c in range(k):
+            t0 = c * L
+            cq, cm = (L, 0) if c + 1 < k else (tq - t0, tm)
+            assert cq >= 0 and cq * W + cm > 0           # no empty launch
+            if cq == 0:
+                checked_empty_rank = True
+            counts = [0] * W
+            for v in range(cq * W + cm):
+                big = cm * (cq + 1)                      # owner under the chunk's split
+                s = v // (cq + 1) if v < big else cm + (v - big) // cq
+                start = s * cq + min(s, cm)
+                tl = t0 + v - start
+                assert 0 <= tl < part.tokens(s)
+                assert (s, tl) not in seen
+                seen[(s, tl)] = c
+                counts[s] += 1
+            # this launch's slices: each rank sends its tokens, each head rank
+            # receives every rank's tokens of its heads
+            assert max(counts) * row <= window
+            assert sum(counts) * hmax * head <= window
+        assert len(seen) == T
+    assert checked_empty_rank  # some last chunk left a smaller rank without tokens
