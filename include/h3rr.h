@@ -104,20 +104,21 @@ typedef struct h3_exec_info {
 } h3_exec_info;
 
 /*
- * Launch order.  By default the register kernels (relayouts, reduce-scatter,
- * gated reduce-scatter, all-gather) use programmatic dependent launch (sm_90
- * and later): a kernel may be scheduled while the previous kernel in the
- * stream is draining, and it waits for that kernel to complete
+ * Launch order.  By default every kernel the library launches (both
+ * relayout and all-gather variants, the reduce-scatters, the staged and rank
+ * calls' kernels) uses programmatic dependent launch (sm_90 and later): a
+ * kernel may be scheduled while the previous kernel in the stream is
+ * draining, and it waits for that kernel to complete
  * (griddepcontrol.wait) before its first global-memory access, so results are
  * those of plain stream order.  Within one chunked relayout call, the launch
  * of plane p+1 touches memory disjoint from plane p's and runs alongside
  * plane p's tail; it waits for plane p at its end instead, so that the call's
  * completion still implies every plane's.  The staged calls' kernels are
  * launched the same way and always wait at their start (each chunk depends on
- * the previous launch; only the launch latency is hidden); the bulk (TMA)
- * kernels launch in plain stream order.  A kernel that follows in the stream
- * and was itself launched with programmatic serialization must wait
- * (cudaGridDependencySynchronize) before reading these calls' outputs.
+ * the previous launch; only the launch latency is hidden).  A kernel that
+ * follows in the stream and was itself launched with programmatic
+ * serialization must wait (cudaGridDependencySynchronize) before reading
+ * these calls' outputs.
  */
 #define H3_LAUNCH_SERIAL 1       /* launch every kernel in plain stream order */
 
@@ -321,7 +322,8 @@ H3RR_API h3_status h3_ragged_all_gather(const void* const* in, void* const* out,
                                         void* stream, h3_exec_info* info);
 /* With launch overrides: variant 0 / H3_VARIANT_VECTOR (registers) or
  * H3_VARIANT_BULK (bulk copies through shared memory; H3_ERR_UNSUPPORTED if
- * 12 rows of C*2 bytes do not fit in shared memory), and ctas_per_sm. */
+ * four rows of C*2 bytes do not fit in shared memory, rows above about 57 KB
+ * on B200), and ctas_per_sm. */
 H3RR_API h3_status h3_ragged_all_gather_ex(const void* const* in, void* const* out,
                                            int64_t n_tokens, int64_t cols, int32_t world,
                                            void* stream, const h3_launch_config* cfg,

@@ -84,57 +84,54 @@ __global__ void __launch_bounds__(kGenericThreads) all_gather_generic_kernel(con
 }
 
 // ---------------------------------------------------------------------------
-// bulk variant: one thread per CTA; each row is bulk-loaded once into a ring
-// of shared-memory stages and bulk-stored to the W outputs (the copy engine
-// does the fan-out).  No multicast.  Waits are bounded; expiries are counted
-// in g_gather_wait_timeouts and reported with the relayout's count.
+// bulk variant: a CTA is one warp and gathers kBulkRows consecutive token
+// rows; lane r bulk-loads row r once into its own shared-memory stage, waits
+// on its own mbarrier and bulk-stores the stage to each of the W outputs (the
+// copy engine does the fan-out).  One CTA per row group, scheduled by the
+// hardware (not persistent); no multicast, no L2 cache hint.  Waits are
+// bounded; expiries are counted in g_gather_wait_timeouts and reported with
+// the relayout's count.
 // ---------------------------------------------------------------------------
-constexpr int kBulkStages = 12;
-constexpr int kBulkLookahead = 8;
-constexpr int kBulkBarrierBytes = 128;
+constexpr int kBulkRows = 4;
+constexpr int kBulkBarrierBytes = 128;  // the lanes' mbarriers, padded to keep stages aligned
 
-template <int S, int L>
 __global__ void __launch_bounds__(32) all_gather_bulk_kernel(const __grid_constant__ GatherArgs a)
 {
-    static_assert(S <= kBulkBarrierBytes / 8 && L >= 1 && L < S, "bulk ring shape");
+    static_assert(kBulkRows <= 32 && kBulkRows * 8 <= kBulkBarrierBytes, "bulk CTA shape");
     extern __shared__ __align__(128) unsigned char smem[];
-    uint64_t* bars = reinterpret_cast<uint64_t*>(smem);
-    unsigned char* ring = smem + kBulkBarrierBytes;
-    if (threadIdx.x != 0)
-        return;
+    const int lane = int(threadIdx.x);
+    const bool driver = lane < kBulkRows;
     const uint32_t row_bytes = uint32_t(a.row_bytes);
-    const uint64_t pol = evict_first_policy();
-    for (int s = 0; s < S; ++s)
-        mbar_init(&bars[s], 1);
-    mbar_fence_init();
-    const int64_t n_rows = a.T > int32_t(blockIdx.x) ? (int64_t(a.T) - blockIdx.x + gridDim.x - 1) / gridDim.x : 0;
-    auto issue_load = [&](int64_t n) {
-        const int32_t t = int32_t(blockIdx.x + n * gridDim.x);
+    uint64_t* bar = reinterpret_cast<uint64_t*>(smem) + (driver ? lane : 0);
+    unsigned char* stage = smem + kBulkBarrierBytes + size_t(driver ? lane : 0) * row_bytes;
+    if (driver) {
+        mbar_init(bar, 1);
+        mbar_fence_init();
+    }
+    // Programmatic launch: the previous kernel in the stream completes before
+    // the first global access.
+    pdl_wait_prerequisites();
+    pdl_allow_dependents();
+    if (!driver)
+        return;
+    const int64_t stride = int64_t(gridDim.x) * kBulkRows;
+    uint32_t parity = 0;
+    for (int64_t t64 = int64_t(blockIdx.x) * kBulkRows + lane; t64 < a.T; t64 += stride) {
+        if (t64 >= stride)
+            bulk_wait_read<0>();  // a later row: the stage's previous stores have read it
+        const int32_t t = int32_t(t64);
         const int32_t s = split_owner(t, a.tq, a.tm);
         const int32_t tl = t - split_start(s, a.tq, a.tm);
-        uint64_t* bar = &bars[n % S];
         mbar_arrive_expect_tx(bar, row_bytes);
-        bulk_load(ring + size_t(n % S) * row_bytes, a.in[s] + int64_t(tl) * row_bytes, row_bytes, bar,
-                  pol);
-    };
-    const int64_t prologue = n_rows < L ? n_rows : L;
-    for (int64_t n = 0; n < prologue; ++n)
-        issue_load(n);
-    for (int64_t n = 0; n < n_rows; ++n) {
-        if (n + L < n_rows) {
-            bulk_wait_read<S - L - 1>();
-            issue_load(n + L);
-        }
-        if (!mbar_wait(&bars[n % S], uint32_t((n / S) & 1))) {
+        bulk_load(stage, a.in[s] + int64_t(tl) * row_bytes, row_bytes, bar);
+        if (!mbar_wait(bar, parity)) {
             atomicAdd(&g_gather_wait_timeouts, 1u);
-            for (int64_t m = n + 1; m < n_rows && m <= n + L; ++m)
-                mbar_wait(&bars[m % S], uint32_t((m / S) & 1));
+            mbar_wait(bar, parity);  // give the copy in flight one more bounded wait
             break;
         }
-        const int32_t t = int32_t(blockIdx.x + n * gridDim.x);
-        const unsigned char* stage = ring + size_t(n % S) * row_bytes;
+        parity ^= 1u;
         for (int j = 0; j < a.W; ++j)
-            bulk_store(a.out[j] + int64_t(t) * row_bytes, stage, row_bytes, pol);
+            bulk_store(a.out[j] + int64_t(t) * row_bytes, stage, row_bytes);
         bulk_commit();
     }
     bulk_wait_all();
@@ -185,7 +182,7 @@ bool all_gather_bulk_fits(const GatherArgs& a, int device)
     int max_smem = 0;
     if (cudaDeviceGetAttribute(&max_smem, cudaDevAttrMaxSharedMemoryPerBlockOptin, device) != cudaSuccess)
         return false;
-    return size_t(kBulkBarrierBytes) + size_t(kBulkStages) * size_t(a.row_bytes) <= size_t(max_smem);
+    return size_t(kBulkBarrierBytes) + size_t(kBulkRows) * size_t(a.row_bytes) <= size_t(max_smem);
 }
 
 cudaError_t launch_all_gather(const GatherArgs& a, int variant, int ctas_per_sm, cudaStream_t stream,
@@ -199,9 +196,9 @@ cudaError_t launch_all_gather(const GatherArgs& a, int variant, int ctas_per_sm,
     if (variant == H3_VARIANT_BULK) {
         if (!all_gather_bulk_fits(a, device))
             return cudaErrorInvalidConfiguration;
-        gc.fn = (const void*)all_gather_bulk_kernel<kBulkStages, kBulkLookahead>;
+        gc.fn = (const void*)all_gather_bulk_kernel;
         gc.threads = 32;
-        gc.smem = size_t(kBulkBarrierBytes) + size_t(kBulkStages) * size_t(a.row_bytes);
+        gc.smem = size_t(kBulkBarrierBytes) + size_t(kBulkRows) * size_t(a.row_bytes);
         gc.variant = H3_VARIANT_BULK;
         const cudaError_t err = allow_dynamic_smem(gc.fn, gc.smem, device);
         if (err != cudaSuccess)
@@ -217,17 +214,17 @@ cudaError_t launch_all_gather(const GatherArgs& a, int variant, int ctas_per_sm,
             gc.threads = kGenericThreads;
         }
     }
-    // The vector kernel launches one CTA per token row by default, scheduled
-    // by the hardware: on B200 that measured 6.6-6.8 TB/s against 5.6-6.0 TB/s
-    // for persistent grid-stride launches.  The bulk kernel runs one CTA per
-    // SM (its ring fills the SM).  ctas_per_sm > 0 caps the grid.
-    int64_t grid = int64_t(a.T);
+    // One CTA per token row (per kBulkRows rows for the bulk kernel) by
+    // default, scheduled by the hardware: on B200 that measured 6.6-6.8 TB/s
+    // against 5.6-6.0 TB/s for persistent grid-stride launches.
+    // ctas_per_sm > 0 caps the grid (grid-stride).
+    const int64_t needed = gc.variant == H3_VARIANT_BULK ? (int64_t(a.T) + kBulkRows - 1) / kBulkRows
+                                                          : int64_t(a.T);
+    int64_t grid = needed;
     if (ctas_per_sm > 0)
         grid = int64_t(sms) * ctas_per_sm;
-    else if (gc.variant == H3_VARIANT_BULK)
-        grid = int64_t(sms) * resident_ctas(gc.fn, gc.threads, gc.smem, device);
-    if (grid > a.T)
-        grid = a.T;
+    if (grid > needed)
+        grid = needed;
     if (grid < 1)
         grid = 1;
     if (shape) {
@@ -235,11 +232,9 @@ cudaError_t launch_all_gather(const GatherArgs& a, int variant, int ctas_per_sm,
         shape->block = gc.threads;
         shape->variant = gc.variant;
     }
-    // The register kernels follow the griddepcontrol protocol; the bulk
-    // kernel launches in plain stream order.
+    // Every all-gather kernel follows the griddepcontrol protocol.
     void* params[] = {const_cast<GatherArgs*>(&a)};
-    return launch_kernel(gc.fn, grid, gc.threads, gc.smem, stream, params,
-                         programmatic && gc.variant != H3_VARIANT_BULK);
+    return launch_kernel(gc.fn, grid, gc.threads, gc.smem, stream, params, programmatic);
 }
 
 cudaError_t read_gather_wait_timeouts(unsigned int* count, bool reset, cudaStream_t stream)

@@ -130,7 +130,7 @@ h3_status relayout(bool seq_to_head, const void* const* send, void* const* recv,
     if (layout & ~(H3_LAYOUT_SEQ_PLANE_MAJOR | H3_LAYOUT_HEAD_PLANE_MAJOR))
         return H3_ERR_INVALID_ARG;
     if (layout != 0 && cfg && cfg->variant == H3_VARIANT_BULK)
-        return H3_ERR_UNSUPPORTED;  // the bulk ring moves token-major rows only
+        return H3_ERR_UNSUPPORTED;  // the bulk kernel moves token-major rows only
     if (window_bytes < 0)
         return H3_ERR_INVALID_ARG;
     if (cfg && cfg->variant != 0 && cfg->variant != H3_VARIANT_VECTOR && cfg->variant != H3_VARIANT_BULK)
@@ -187,7 +187,7 @@ h3_status relayout(bool seq_to_head, const void* const* send, void* const* recv,
         if (err != cudaSuccess)
             return cuda_failure(err);
         if (!relayout_bulk_fits(a, device))
-            return H3_ERR_UNSUPPORTED;  // a row does not fit the shared-memory ring
+            return H3_ERR_UNSUPPORTED;  // the bulk kernel's row stages do not fit in shared memory
     }
     const int plane_groups = chunked ? planes : 1;
     const int per_launch = chunked ? 1 : planes;
@@ -653,7 +653,7 @@ h3_status h3_ragged_all_gather_ex(const void* const* in, void* const* out, int64
         if (derr != cudaSuccess)
             return cuda_failure(derr);
         if (!all_gather_bulk_fits(a, device))
-            return H3_ERR_UNSUPPORTED;  // a row does not fit the shared-memory ring
+            return H3_ERR_UNSUPPORTED;  // the bulk kernel's row stages do not fit in shared memory
     }
     LaunchShape shape;
     const cudaError_t err = launch_all_gather(a, variant, cfg ? cfg->ctas_per_sm : 0,

@@ -190,7 +190,7 @@ cudaError_t launch_relayout(bool seq_to_head, const RelayoutArgs& a, int variant
                             int ctas_per_sm, cudaStream_t stream, LaunchShape* shape,
                             bool layout = false, bool programmatic = false);
 
-// Whether the bulk kernel's shared-memory ring fits one row of these args.
+// Whether the bulk kernel's shared-memory stages fit the rows of these args.
 bool relayout_bulk_fits(const RelayoutArgs& a, int device);
 
 // Copy (and optionally clear) the per-device count of expired bulk waits.
@@ -229,10 +229,6 @@ cudaError_t launch_reduce_scatter(const ReduceArgs& a, int ctas_per_sm, cudaStre
 
 // SM count of the current device (cached per device).
 int current_sm_count(int* device);
-
-// Resident CTAs per SM of a kernel at the given block size and dynamic shared
-// memory (cached per kernel and device).
-int resident_ctas(const void* kernel, int block, size_t smem, int device);
 
 // Opt a kernel in to `smem` bytes of dynamic shared memory on the current
 // device (once per kernel, device and size).

@@ -158,44 +158,6 @@ int current_sm_count(int* device)
     return n;
 }
 
-int resident_ctas(const void* kernel, int block, size_t smem, int device)
-{
-    struct Key {
-        const void* k;
-        int block;
-        size_t smem;
-        int dev;
-        bool operator==(const Key& o) const
-        {
-            return k == o.k && block == o.block && smem == o.smem && dev == o.dev;
-        }
-    };
-    struct Hash {
-        size_t operator()(const Key& x) const
-        {
-            return std::hash<const void*>()(x.k) ^ (size_t(x.block) << 20) ^ (x.smem << 3) ^
-                   size_t(x.dev);
-        }
-    };
-    static std::mutex mu;
-    static std::unordered_map<Key, int, Hash> cache;
-    const Key key{kernel, block, smem, device};
-    {
-        std::lock_guard<std::mutex> lock(mu);
-        auto it = cache.find(key);
-        if (it != cache.end())
-            return it->second;
-    }
-    int n = 0;
-    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, kernel, block, smem) != cudaSuccess)
-        n = 1;
-    if (n < 1)
-        n = 1;
-    std::lock_guard<std::mutex> lock(mu);
-    cache.emplace(key, n);
-    return n;
-}
-
 cudaError_t allow_dynamic_smem(const void* kernel, size_t smem, int device)
 {
     // The opt-in is one value per kernel, so it is raised once per kernel and

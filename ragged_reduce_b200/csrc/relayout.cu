@@ -22,13 +22,13 @@
 //   streaming loads (inputs never overlap outputs; the host checks this),
 //   outputs streaming stores.
 //
-// * Bulk kernel: one thread per CTA drives the tensor memory accelerator's
-//   1-D bulk copies through a ring of S shared-memory stages, one row per
-//   stage.  Loads run L rows ahead of stores; an mbarrier per stage tracks
-//   load completion and bulk-group waits keep a stage from being refilled
-//   before its stores have read it.  No multicast is used.  Every mbarrier
-//   wait is bounded: on expiry the kernel counts the event in a device word
-//   (read with h3_bulk_wait_timeouts), drains what it issued and returns.
+// * Bulk kernel: the tensor memory accelerator's 1-D bulk copies move each
+//   row through shared memory.  A CTA is one warp; each of its first few
+//   lanes owns one row, one shared-memory stage and one mbarrier that counts
+//   the row's load bytes, and stores the stage once the load has landed.  No
+//   multicast is used.  Every mbarrier wait is bounded: on expiry the kernel
+//   counts the event in a device word (read with h3_bulk_wait_timeouts),
+//   waits once more for what it issued and returns.
 #include "bulk_copy.cuh"
 #include "device_access.cuh"
 #include "h3rr_internal.h"
@@ -172,98 +172,84 @@ __global__ void __launch_bounds__(kGenericThreads) relayout_generic_kernel(const
 // ---------------------------------------------------------------------------
 // bulk kernel (tensor memory accelerator, 1-D bulk copies, no multicast)
 // ---------------------------------------------------------------------------
-// A 4-stage ring (57,472 B for a 14,336-byte H3 row) lets three CTAs share an
-// SM; on B200 that ran 0.3-8 % faster in the worst cases than one CTA per
-// SM with 14 stages, 2-3 % slower in the best, and it fits rows up to a
-// quarter of the shared memory.
-constexpr int kBulkStages = 4;
-constexpr int kBulkLookahead = 3;
-constexpr int kBulkBarrierBytes = 128;          // room for 16 mbarriers
+// A CTA is one warp and moves kBulkRows consecutive rows; lane r drives row
+// r on its own: bulk loads into its shared-memory stage (the whole sequence-
+// side row, or the row's W head-side runs), a wait on its own mbarrier, bulk
+// stores out of the stage.  CTAs are not persistent: one per kBulkRows rows,
+// handed out by the block scheduler as SMs free up.  On B200 a persistent
+// ring (one thread per CTA streaming rows through 4-14 stages, grid = the
+// SM count times the CTAs that fit) ran 9-13 % slower on every full-size
+// workload, the same lockstep effect that made the vector kernels one CTA
+// per row; 1-8 rows per CTA measured within 1.5 % of each other, 4 best.
+// The copies carry no L2 cache hint: evict-first loads cost 1-2 %.
+constexpr int kBulkRows = 4;
+constexpr int kBulkBarrierBytes = 128;  // the lanes' mbarriers, padded to keep stages aligned
 
-template <bool kSeqToHead, int S, int L>
+template <bool kSeqToHead>
 __global__ void __launch_bounds__(32) relayout_bulk_kernel(const __grid_constant__ RelayoutArgs a)
 {
-    static_assert(S <= kBulkBarrierBytes / 8 && L >= 1 && L < S, "bulk ring shape");
+    static_assert(kBulkRows <= 32 && kBulkRows * 8 <= kBulkBarrierBytes, "bulk CTA shape");
     extern __shared__ __align__(128) unsigned char smem[];
-    uint64_t* bars = reinterpret_cast<uint64_t*>(smem);
-    unsigned char* ring = smem + kBulkBarrierBytes;
-    if (threadIdx.x != 0)
-        return;
+    const int lane = int(threadIdx.x);
+    const bool driver = lane < kBulkRows;
     const uint32_t row_bytes = uint32_t(a.row_vecs) * kVecBytes;
     const uint32_t head_bytes = uint32_t(a.head_vecs) * kVecBytes;
-    const uint64_t pol = evict_first_policy();
-    for (int s = 0; s < S; ++s)
-        mbar_init(&bars[s], 1);
-    mbar_fence_init();
-
-    const int64_t n_rows =
-        a.rows > int32_t(blockIdx.x) ? (int64_t(a.rows) - blockIdx.x + gridDim.x - 1) / gridDim.x : 0;
-
-    // Row n of this CTA -> (sequence-side row address, head-side row index g).
-    auto locate = [&](int64_t n, char** seq_row, int64_t* g) {
-        const int32_t i = int32_t(blockIdx.x + n * gridDim.x);
-        const int32_t u = i / a.nplanes;  // token unit of the launch
-        const int32_t p = a.plane0 + (i - u * a.nplanes);
-        const ChunkToken k = chunk_token(u, a.cq, a.cm, a.t0, a.tq, a.tm);
-        *seq_row = a.seq[k.s] + (int64_t(k.tl) * a.P + p) * row_bytes;
-        *g = int64_t(k.t) * a.P + p;
-    };
-    auto issue_load = [&](int64_t n) {
-        char* seq_row;
-        int64_t g;
-        locate(n, &seq_row, &g);
-        unsigned char* stage = ring + size_t(n % S) * row_bytes;
-        uint64_t* bar = &bars[n % S];
-        mbar_arrive_expect_tx(bar, row_bytes);
-        if (kSeqToHead) {
-            bulk_load(stage, seq_row, row_bytes, bar, pol);
-        } else {
-            uint32_t off = 0;
-            for (int j = 0; j < a.W; ++j) {
-                const uint32_t run = uint32_t(a.hq + (j < a.hm ? 1 : 0)) * head_bytes;
-                bulk_load(stage + off, a.head[j] + g * run, run, bar, pol);
-                off += run;
-            }
-        }
-    };
-    auto issue_store = [&](int64_t n) {
-        char* seq_row;
-        int64_t g;
-        locate(n, &seq_row, &g);
-        const unsigned char* stage = ring + size_t(n % S) * row_bytes;
-        if (kSeqToHead) {
-            uint32_t off = 0;
-            for (int j = 0; j < a.W; ++j) {
-                const uint32_t run = uint32_t(a.hq + (j < a.hm ? 1 : 0)) * head_bytes;
-                bulk_store(a.head[j] + g * run, stage + off, run, pol);
-                off += run;
-            }
-        } else {
-            bulk_store(seq_row, stage, row_bytes, pol);
-        }
-        bulk_commit();
-    };
-
-    const int64_t prologue = n_rows < L ? n_rows : L;
-    for (int64_t n = 0; n < prologue; ++n)
-        issue_load(n);
-    for (int64_t n = 0; n < n_rows; ++n) {
-        if (n + L < n_rows) {
-            // Stage (n+L)%S last served row n+L-S, whose store group must have
-            // finished reading it: at most S-L-1 newer groups may be pending.
-            bulk_wait_read<S - L - 1>();
-            issue_load(n + L);
-        }
-        if (!mbar_wait(&bars[n % S], uint32_t((n / S) & 1))) {
-            atomicAdd(&g_bulk_wait_timeouts, 1u);
-            // Drain the loads already in flight (bounded) before leaving.
-            for (int64_t m = n + 1; m < n_rows && m <= n + L; ++m)
-                mbar_wait(&bars[m % S], uint32_t((m / S) & 1));
-            break;
-        }
-        issue_store(n);
+    uint64_t* bar = reinterpret_cast<uint64_t*>(smem) + (driver ? lane : 0);
+    unsigned char* stage = smem + kBulkBarrierBytes + size_t(driver ? lane : 0) * row_bytes;
+    if (driver) {
+        mbar_init(bar, 1);
+        mbar_fence_init();
     }
-    bulk_wait_all();
+    // Programmatic launch, as in the vector kernels: wait for the previous
+    // kernel before the first global access unless this launch is a later,
+    // independent plane of a chunked call, which waits at its end instead.
+    if (!a.wait_late)
+        pdl_wait_prerequisites();
+    pdl_allow_dependents();
+
+    if (driver) {
+        const int64_t stride = int64_t(gridDim.x) * kBulkRows;
+        uint32_t parity = 0;
+        for (int64_t i = int64_t(blockIdx.x) * kBulkRows + lane; i < a.rows; i += stride) {
+            if (i >= stride)
+                bulk_wait_read<0>();  // a later row: the stage's previous stores have read it
+            const int32_t u = int32_t(i / a.nplanes);  // token unit of the launch
+            const int32_t p = a.plane0 + int32_t(i - int64_t(u) * a.nplanes);
+            const ChunkToken k = chunk_token(u, a.cq, a.cm, a.t0, a.tq, a.tm);
+            char* seq_row = a.seq[k.s] + (int64_t(k.tl) * a.P + p) * row_bytes;
+            const int64_t g = int64_t(k.t) * a.P + p;  // head-side row
+            mbar_arrive_expect_tx(bar, row_bytes);
+            if (kSeqToHead) {
+                bulk_load(stage, seq_row, row_bytes, bar);
+            } else {
+                uint32_t off = 0;
+                for (int j = 0; j < a.W; ++j) {
+                    const uint32_t run = uint32_t(a.hq + (j < a.hm ? 1 : 0)) * head_bytes;
+                    bulk_load(stage + off, a.head[j] + g * run, run, bar);
+                    off += run;
+                }
+            }
+            if (!mbar_wait(bar, parity)) {
+                atomicAdd(&g_bulk_wait_timeouts, 1u);
+                mbar_wait(bar, parity);  // give the copies in flight one more bounded wait
+                break;
+            }
+            parity ^= 1u;
+            if (kSeqToHead) {
+                uint32_t off = 0;
+                for (int j = 0; j < a.W; ++j) {
+                    const uint32_t run = uint32_t(a.hq + (j < a.hm ? 1 : 0)) * head_bytes;
+                    bulk_store(a.head[j] + g * run, stage + off, run);
+                    off += run;
+                }
+            } else {
+                bulk_store(seq_row, stage, row_bytes);
+            }
+            bulk_commit();
+        }
+        bulk_wait_all();
+    }
+    pdl_wait_at_end(a.wait_late);
 }
 
 // ---------------------------------------------------------------------------
@@ -434,16 +420,15 @@ void choose_vec(const RelayoutArgs& a, bool wide_ok, KernelChoice* kc)
 bool choose_bulk(bool s2h, const RelayoutArgs& a, int device, KernelChoice* kc)
 {
     const size_t row_bytes = size_t(a.row_vecs) * kVecBytes;
-    const size_t smem = kBulkBarrierBytes + kBulkStages * row_bytes;
+    const size_t smem = kBulkBarrierBytes + kBulkRows * row_bytes;
     int max_smem = 0;
     if (cudaDeviceGetAttribute(&max_smem, cudaDevAttrMaxSharedMemoryPerBlockOptin, device) != cudaSuccess)
         return false;
     if (smem > size_t(max_smem))
         return false;
-    kc->fn = s2h ? (const void*)relayout_bulk_kernel<true, kBulkStages, kBulkLookahead>
-                 : (const void*)relayout_bulk_kernel<false, kBulkStages, kBulkLookahead>;
+    kc->fn = s2h ? (const void*)relayout_bulk_kernel<true> : (const void*)relayout_bulk_kernel<false>;
     kc->threads = 32;
-    kc->rows_per_cta_iter = 1;
+    kc->rows_per_cta_iter = kBulkRows;
     kc->smem = smem;
     kc->variant = H3_VARIANT_BULK;
     return true;
@@ -483,7 +468,7 @@ cudaError_t launch_relayout(bool seq_to_head, const RelayoutArgs& a, int variant
     if (variant == H3_VARIANT_BULK && !bulk)
         return cudaErrorInvalidConfiguration;
     if (bulk && layout)
-        return cudaErrorInvalidConfiguration;  // the bulk ring moves token-major rows only
+        return cudaErrorInvalidConfiguration;  // the bulk kernel moves token-major rows only
     if (!bulk) {
         if (layout) {
             if (seq_to_head)
@@ -500,19 +485,16 @@ cudaError_t launch_relayout(bool seq_to_head, const RelayoutArgs& a, int variant
         if (err != cudaSuccess)
             return err;
     }
-    // Grid: the vector kernels launch one CTA per row (or row pair) by
-    // default and let the hardware schedule them.  On B200 that measured
-    // 2-8 % faster than any persistent grid-stride launch (a multiple of the
+    // Grid: every kernel launches one CTA per row, row pair or row group by
+    // default and lets the hardware schedule them.  On B200 that measured
+    // 2-13 % faster than any persistent grid-stride launch (a multiple of the
     // SM count): CTAs marching through the rows in lockstep resonated with the
-    // DRAM mapping at some grid sizes.  The bulk kernel is persistent: as many
-    // CTAs per SM as its shared-memory ring allows.  ctas_per_sm > 0 caps the
-    // grid at that many CTAs per SM (grid-stride).
+    // DRAM mapping at some grid sizes.  ctas_per_sm > 0 caps the grid at that
+    // many CTAs per SM (grid-stride).
     const int64_t needed = (int64_t(a.rows) + kc.rows_per_cta_iter - 1) / kc.rows_per_cta_iter;
     int64_t grid = needed;
     if (ctas_per_sm > 0)
         grid = int64_t(sms) * ctas_per_sm;
-    else if (kc.variant == H3_VARIANT_BULK)
-        grid = int64_t(sms) * resident_ctas(kc.fn, kc.threads, kc.smem, device);
     if (grid > needed)
         grid = needed;
     if (grid < 1)
@@ -522,11 +504,9 @@ cudaError_t launch_relayout(bool seq_to_head, const RelayoutArgs& a, int variant
         shape->block = kc.threads;
         shape->variant = kc.variant;
     }
-    // The vector and generic kernels follow the griddepcontrol protocol; the
-    // bulk kernel launches in plain stream order.
+    // Every relayout kernel follows the griddepcontrol protocol.
     void* params[] = {const_cast<RelayoutArgs*>(&a)};
-    return launch_kernel(kc.fn, grid, kc.threads, kc.smem, stream, params,
-                         programmatic && kc.variant != H3_VARIANT_BULK);
+    return launch_kernel(kc.fn, grid, kc.threads, kc.smem, stream, params, programmatic);
 }
 
 namespace {

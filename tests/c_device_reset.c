@@ -79,7 +79,7 @@ static void round_trip(int round)
     }
     expect(h3o_seq_to_head((const uint16_t* const*)send, want, T, P, H, D, W) == 0, "oracle");
 
-    /* the bulk kernel: its ring needs more than the default 48 KB of shared memory */
+    /* the bulk kernel: its four row stages need more than the default 48 KB of shared memory */
     memset(&cfg, 0, sizeof(cfg));
     cfg.variant = H3_VARIANT_BULK;
     expect(h3_seq_to_head_ex((const void* const*)d_send, d_heads, T, P, H, D, W, 0, stream, &cfg,

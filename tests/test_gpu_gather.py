@@ -49,8 +49,28 @@ def test_all_gather_forced_variant(oracle_lib, T, C, W, variant):
     assert rr.bulk_wait_timeouts() == 0
 
 
+@pytest.mark.parametrize("ctas_per_sm", [0, 1])
+def test_all_gather_bulk_row_groups_and_capped_grid(oracle_lib, ctas_per_sm):
+    """The bulk all-gather launches one warp per four rows; capped at one CTA
+    per SM every CTA walks several row groups and refills its stages.  Rows
+    of 36,000 bytes: four stages fit in shared memory."""
+    for T, C, W in [(3001, 7168, 8), (301, 18000, 3)]:
+        full, blocks = _blocks(T, C, W, 11 * T + W + ctas_per_sm)
+        outs = [torch.empty((T, C), dtype=torch.bfloat16, device=DEV) for _ in range(W)]
+        rr.bulk_wait_timeouts(reset=True)
+        info = rr.ragged_all_gather(blocks, outs, variant=rr.H3_VARIANT_BULK, ctas_per_sm=ctas_per_sm)
+        sms = torch.cuda.get_device_properties(0).multi_processor_count
+        groups = (T + 3) // 4
+        assert info["variant"] == rr.H3_VARIANT_BULK and info["block"] == 32
+        assert info["grid"] == (groups if not ctas_per_sm else min(groups, ctas_per_sm * sms))
+        want = oracle_lib.ragged_all_gather([gu.bits(b) for b in blocks], W)
+        for j in range(W):
+            assert np.array_equal(gu.bits(outs[j]), want[j]), f"rank {j}"
+        assert rr.bulk_wait_timeouts() == 0
+
+
 def test_all_gather_bulk_rejects_wide_rows():
-    T, C, W = 16, 18000, 2  # 36,000-byte rows: 12 stages do not fit
+    T, C, W = 16, 30000, 2  # 60,000-byte rows: four stages do not fit
     full, blocks = _blocks(T, C, W, 1)
     outs = [torch.empty((T, C), dtype=torch.bfloat16, device=DEV) for _ in range(W)]
     with pytest.raises(rr.H3Error) as e:

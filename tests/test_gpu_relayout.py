@@ -102,8 +102,8 @@ def test_forced_variant_matches_oracle(oracle_lib, T, P, H, D, W, variant):
     assert rr.bulk_wait_timeouts() == 0
 
 
-def test_bulk_ring_width_limit(oracle_lib):
-    """The bulk ring holds four rows: a 28,672-byte row (D=256) fits and
+def test_bulk_row_width_limit(oracle_lib):
+    """A bulk CTA stages four rows: a 28,672-byte row (D=256) fits and
     matches the oracle; a 114,688-byte row (D=1024) does not fit in shared
     memory and is refused, while the default call still runs it."""
     T, P, H, D, W = 33, 3, 56, 256, 4
@@ -128,9 +128,9 @@ def test_bulk_ring_width_limit(oracle_lib):
         assert np.array_equal(gu.bits(recv[j]), want[j]), j
 
 
-def test_bulk_ring_sizes_alternate(oracle_lib):
-    """Bulk launches whose shared-memory rings differ in size, in both orders
-    (a smaller ring must not shrink what a later, larger one may use)."""
+def test_bulk_stage_sizes_alternate(oracle_lib):
+    """Bulk launches whose shared-memory stages differ in size, in both orders
+    (a smaller launch must not shrink what a later, larger one may use)."""
     for T, P, H, D, W in [(40, 3, 24, 128, 3), (64, 3, 56, 128, 2), (40, 3, 24, 128, 3),
                           (64, 3, 56, 128, 4), (130, 2, 7, 64, 3), (64, 3, 56, 128, 2)]:
         full, send, part = _seq_inputs(T, P, H, D, W, seed=T + H + W)
@@ -144,9 +144,40 @@ def test_bulk_ring_sizes_alternate(oracle_lib):
             assert np.array_equal(gu.bits(recv[j]), want[j])
 
 
+@pytest.mark.parametrize("ctas_per_sm", [0, 1, 3])
+def test_bulk_row_groups_and_capped_grid(oracle_lib, ctas_per_sm):
+    """The bulk kernel launches one warp per four rows.  A capped grid makes
+    every CTA walk several row groups, so each lane refills its stage and
+    reuses its barrier (the stage only after its stores have read it); both
+    directions, one plane per launch on the way back."""
+    T, P, H, D, W = 2003, 3, 56, 128, 6
+    full, send, part = _seq_inputs(T, P, H, D, W, seed=97 + ctas_per_sm)
+    sms = torch.cuda.get_device_properties(0).multi_processor_count
+
+    def grid(rows):
+        groups = (rows + 3) // 4
+        return groups if not ctas_per_sm else min(groups, ctas_per_sm * sms)
+
+    recv = rr.alloc_head_side(T, P, H, D, W, DEV)
+    rr.bulk_wait_timeouts(reset=True)
+    info = rr.seq_to_head(send, recv, variant=rr.H3_VARIANT_BULK, ctas_per_sm=ctas_per_sm)
+    assert info["variant"] == rr.H3_VARIANT_BULK and info["block"] == 32
+    assert info["grid"] == grid(T * P)
+    want = oracle_lib.seq_to_head([gu.bits(s) for s in send], T, P, H, D, W)
+    for j in range(W):
+        assert np.array_equal(gu.bits(recv[j]), want[j]), f"seq->head rank {j}"
+    back_full, back = rr.alloc_seq_side(T, P, H, D, W, DEV)
+    plane = max(part.tokens(0) * H * D * 2, T * part.heads(0) * D * 2)
+    info = rr.head_to_seq(recv, back, variant=rr.H3_VARIANT_BULK, ctas_per_sm=ctas_per_sm,
+                          window_bytes=plane)
+    assert info["launches"] == P and info["grid"] == grid(T)
+    assert gu.same_bits(back_full, full)
+    assert rr.bulk_wait_timeouts() == 0
+
+
 def test_default_variants():
     """Defaults: the vector kernels in both directions, one CTA per row pair
-    (seq->head) or row (head->seq); the bulk ring only when asked for."""
+    (seq->head) or row (head->seq); the bulk kernel only when asked for."""
     for W, want_back in [(2, rr.H3_VARIANT_VECTOR), (4, rr.H3_VARIANT_VECTOR), (6, rr.H3_VARIANT_VECTOR)]:
         T, P, H, D = 300, 3, 56, 128
         full, send, part = _seq_inputs(T, P, H, D, W, seed=W)
