@@ -1264,6 +1264,13 @@ def run_workload_report(args):
             raise SystemExit("all-gather output differs")
         for o in outs:
             o.zero_()
+        info = rr.ragged_all_gather(blocks, outs, variant=rr.H3_VARIANT_BULK)
+        secs = _time_calls(lambda: rr.ragged_all_gather(blocks, outs, variant=rr.H3_VARIANT_BULK), iters)
+        emit(f"all_gather_T{T}_C{C_}_W{W}", "ragged_all_gather", "bulk", nbytes, secs, info)
+        if not all(torch.equal(o.view(torch.int16), full.view(torch.int16)) for o in outs):
+            raise SystemExit("bulk all-gather output differs")
+        for o in outs:
+            o.zero_()
 
         def ag_ranks():
             for k in range(W):
