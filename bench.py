@@ -318,6 +318,36 @@ class Step:
     def nvlink(self, per_kernel_s: dict, steps: int):
         return None
 
+    def token_range_rates(self, iters: int, stream) -> dict:
+        """The step's two relayouts under the same window cut into token
+        ranges of every plane (H3_LAUNCH_CHUNK_TOKENS) instead of one batch
+        plane per launch: GB/s per direction by CUDA events over `iters`
+        calls after two warm-up calls, and the round trip checked.  Not part
+        of the bench's value."""
+        rr = self.rr
+        out = {}
+        kw = dict(window_bytes=self.window, stream=stream, token_chunks=True)
+        for name, call in (("seq_to_head", lambda: rr.seq_to_head(self.send, self.heads, **kw)),
+                           ("head_to_seq", lambda: rr.head_to_seq(self.heads, self.back, **kw))):
+            for _ in range(2):
+                info = call()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            for _ in range(iters):
+                call()
+            e1.record(stream)
+            e1.synchronize()
+            secs = e0.elapsed_time(e1) / 1e3 / iters
+            out[name] = {"gbs": round(self.kernel_bytes[name] / secs / 1e9, 1),
+                         "us_per_call": round(secs * 1e6, 1), "launches_per_call": info["launches"],
+                         "planes_per_launch": info["planes_per_launch"]}
+        tokens, _ = rr.relayout_chunk_plan(self.T, self.P, self.H, self.D, self.W, self.window,
+                                           token_chunks=True)
+        out["tokens_per_launch"] = tokens
+        out["round_trip_ok"] = bool(torch.equal(self.back_full.view(torch.int16),
+                                                self.qkv.view(torch.int16)))
+        return out
+
 
 class ShardedStep:
     """One rank's share of the step with one rank per GPU (W = world).
@@ -724,6 +754,14 @@ def measure(args, make_step, rank, world, local, device, timer, n_events):
     if args.e2e_steps > 0 and isinstance(timer, CudaTimer):
         e2e = run_e2e(make_step, step, args.e2e_steps, local, device, world, timer)
 
+    # Beside the line, not in its value: the same window cut into token
+    # ranges of every plane instead of one batch plane per launch.
+    ranges = None
+    if world == 1 and isinstance(timer, CudaTimer) and getattr(step, "has_relayout", False):
+        ranges = step.token_range_rates(max(3, min(20, K)), stream)
+        if not ranges["round_trip_ok"]:
+            raise SystemExit("token-range relayouts produced wrong results")
+
     result = None
     if rank == 0:
         if world > 1:
@@ -764,6 +802,15 @@ def measure(args, make_step, rank, world, local, device, timer, n_events):
         }
         if nvlink is not None:
             result["nvlink_rank0"] = nvlink
+        if ranges is not None:
+            result["chunk_shapes"] = {
+                "window_bytes": WINDOW,
+                "one_plane_per_launch": {k: {"gbs": kernels[k]["gbs"],
+                                             "launches_per_call": kernels[k]["launches_per_step"]}
+                                         for k in ("seq_to_head", "head_to_seq")},
+                "token_ranges_all_planes": ranges,
+                "note": "not part of value: the step's relayouts under the same window cut into "
+                        "token ranges of every plane (H3_LAUNCH_CHUNK_TOKENS)"}
     if hasattr(step, "close"):
         timer.synchronize()
         barrier(local, timer)
@@ -1074,15 +1121,20 @@ def run_workload_report(args):
                 lsend = seq_pm if layout & 1 else send
                 lback = back_pm if layout & 1 else back
                 lheads = heads_pm if layout & 2 else heads
-                for wb in (0, WINDOW):
-                    tag = f"layout{layout}_{'chunked' if wb else 'unchunked'}"
-                    info = rr.seq_to_head_layout(lsend, lheads, layout, window_bytes=wb)
-                    secs = _time_calls(lambda: rr.seq_to_head_layout(lsend, lheads, layout,
-                                                                     window_bytes=wb), iters)
+                # the same window cut into token ranges of every plane
+                # (H3_LAUNCH_CHUNK_TOKENS), on token-major buffers
+                shapes = [(0, False, "unchunked"), (WINDOW, False, "chunked")]
+                if layout == 0:
+                    shapes.append((WINDOW, True, "token_ranges"))
+                for wb, tok, kind in shapes:
+                    tag = f"layout{layout}_{kind}"
+                    info = rr.seq_to_head_layout(lsend, lheads, layout, window_bytes=wb, token_chunks=tok)
+                    secs = _time_calls(lambda: rr.seq_to_head_layout(
+                        lsend, lheads, layout, window_bytes=wb, token_chunks=tok), iters)
                     emit(w.name, "seq_to_head", tag, nbytes, secs, info)
-                    info = rr.head_to_seq_layout(lheads, lback, layout, window_bytes=wb)
-                    secs = _time_calls(lambda: rr.head_to_seq_layout(lheads, lback, layout,
-                                                                     window_bytes=wb), iters)
+                    info = rr.head_to_seq_layout(lheads, lback, layout, window_bytes=wb, token_chunks=tok)
+                    secs = _time_calls(lambda: rr.head_to_seq_layout(
+                        lheads, lback, layout, window_bytes=wb, token_chunks=tok), iters)
                     emit(w.name, "head_to_seq", tag, nbytes, secs, info)
                     if not all(torch.equal(a.view(torch.int16), b.view(torch.int16))
                                for a, b in zip(lback, lsend)):
@@ -1200,12 +1252,13 @@ def run_workload_report(args):
     heads = rr.alloc_head_side(w.T, w.P, w.H, w.D, w.W, dev)
     back_full, back = rr.alloc_seq_side(w.T, w.P, w.H, w.D, w.W, dev)
     nbytes = 2 * x.numel() * 2
-    for wb, tag in ((w.window_bytes, "token_chunks"), (0, "unchunked")):
-        info = rr.seq_to_head(send, heads, window_bytes=wb)
-        secs = _time_calls(lambda: rr.seq_to_head(send, heads, window_bytes=wb), iters)
+    for wb, tok, tag in ((w.window_bytes, False, "token_chunks"), (w.window_bytes, True, "token_ranges"),
+                         (0, False, "unchunked")):
+        info = rr.seq_to_head(send, heads, window_bytes=wb, token_chunks=tok)
+        secs = _time_calls(lambda: rr.seq_to_head(send, heads, window_bytes=wb, token_chunks=tok), iters)
         emit(w.name, "seq_to_head", tag, nbytes, secs, info)
-        info = rr.head_to_seq(heads, back, window_bytes=wb)
-        secs = _time_calls(lambda: rr.head_to_seq(heads, back, window_bytes=wb), iters)
+        info = rr.head_to_seq(heads, back, window_bytes=wb, token_chunks=tok)
+        secs = _time_calls(lambda: rr.head_to_seq(heads, back, window_bytes=wb, token_chunks=tok), iters)
         emit(w.name, "head_to_seq", tag, nbytes, secs, info)
         if not torch.equal(back_full.view(torch.int16), x.view(torch.int16)):
             raise SystemExit(f"{w.name} {tag}: round trip differs")

@@ -72,7 +72,7 @@ extern "C" {
 #define H3RR_API
 #endif
 
-#define H3RR_ABI_VERSION 2
+#define H3RR_ABI_VERSION 3
 #define H3RR_MAX_WORLD 64
 
 typedef enum h3_status {
@@ -121,6 +121,22 @@ typedef struct h3_exec_info {
  * these calls' outputs.
  */
 #define H3_LAUNCH_SERIAL 1       /* launch every kernel in plain stream order */
+/*
+ * H3_LAUNCH_CHUNK_TOKENS (relayout calls only; H3_ERR_INVALID_ARG elsewhere):
+ * a chunked relayout (window_bytes > 0) cuts its work into token ranges that
+ * cover every plane instead of one batch plane per launch.  Launch c moves
+ * local tokens [c*L, c*L + L) of every rank's range (fewer in the last), all
+ * P planes of them, with k the fewest launches and L the equal length for
+ * which each rank's send slice (L*P*H*D*2) and receive slice
+ * (W*L*P*max_j(H_j)*D*2) fit in window_bytes; one launch if everything fits.
+ * The window bounds the same bytes per launch as in one-plane mode and the
+ * result is identical, but every launch touches whole token rows of both
+ * sides: on token-major buffers that is the unchunked rate, where one plane
+ * per launch leaves the other planes' bytes between each row it touches and
+ * runs 3-5 % slower on B200.  H3_ERR_WINDOW if the window cannot hold one
+ * token of every plane.
+ */
+#define H3_LAUNCH_CHUNK_TOKENS 2
 
 /* Optional launch overrides for h3_*_ex; zero fields mean "library default". */
 typedef struct h3_launch_config {
@@ -191,6 +207,8 @@ H3RR_API h3_status h3_partition(int64_t n_tokens, int32_t n_heads, int32_t world
  *                  W*L*max_j(H_j)*D*2 <= window_bytes (h3_relayout_chunk_plan
  *                  reports k and L).  H3_ERR_WINDOW only if not even L = 1
  *                  fits.  The result is identical either way.
+ *                  (h3_seq_to_head_ex with H3_LAUNCH_CHUNK_TOKENS cuts the
+ *                  same window into token ranges of all planes instead.)
  */
 H3RR_API h3_status h3_seq_to_head(const void* const* send, void* const* recv,
                          int64_t n_tokens, int32_t planes, int32_t n_heads,
@@ -210,6 +228,20 @@ H3RR_API h3_status h3_seq_to_head(const void* const* send, void* const* recv,
 H3RR_API h3_status h3_relayout_chunk_plan(int64_t n_tokens, int32_t planes, int32_t n_heads,
                                           int32_t head_dim, int32_t world, int64_t window_bytes,
                                           int64_t* tokens_per_chunk, int64_t* chunks);
+
+/*
+ * h3_relayout_chunk_plan_ex - as h3_relayout_chunk_plan for the chunk shape
+ * that `flags` selects (0, or H3_LAUNCH_CHUNK_TOKENS: token ranges over all
+ * planes; H3_LAUNCH_SERIAL is accepted and changes nothing).
+ *   chunks            : out, launches of a one-GPU call (1 if window_bytes == 0;
+ *                       planes * k one plane per launch; k token ranges with
+ *                       H3_LAUNCH_CHUNK_TOKENS).
+ *   planes_per_launch : out (may be NULL), 1 one plane per launch, else P.
+ */
+H3RR_API h3_status h3_relayout_chunk_plan_ex(int64_t n_tokens, int32_t planes, int32_t n_heads,
+                                             int32_t head_dim, int32_t world, int64_t window_bytes,
+                                             int32_t flags, int64_t* tokens_per_chunk,
+                                             int64_t* chunks, int32_t* planes_per_launch);
 
 /*
  * h3_head_to_seq - inverse head->sequence relayout ("Distributed H3

@@ -30,7 +30,7 @@ from . import _abi
 from ._abi import (ExecInfo, H3Error, LaunchConfig, H3_LAYOUT_HEAD_PLANE_MAJOR,
                    H3_LAYOUT_SEQ_PLANE_MAJOR, H3_VARIANT_BULK, H3_VARIANT_GATHER,
                    H3_VARIANT_REDUCE, H3_VARIANT_STAGED, H3_VARIANT_VECTOR, H3_LAUNCH_SERIAL,
-                   MAX_WORLD)
+                   H3_LAUNCH_CHUNK_TOKENS, MAX_WORLD)
 
 __all__ = [
     "H3Error", "Partition", "partition", "seq_to_head", "head_to_seq",
@@ -40,6 +40,7 @@ __all__ = [
     "staged_plan", "relayout_chunk_plan", "H3_VARIANT_STAGED", "ragged_all_gather", "H3_VARIANT_GATHER",
     "seq_to_head_layout", "head_to_seq_layout", "H3_LAYOUT_SEQ_PLANE_MAJOR",
     "H3_LAYOUT_HEAD_PLANE_MAJOR", "ragged_reduce_scatter_gated", "PreparedRelayout", "H3_LAUNCH_SERIAL",
+    "H3_LAUNCH_CHUNK_TOKENS",
     "PreparedReduceScatter", "prepare_seq_to_head", "prepare_head_to_seq",
     "seq_to_head_rank", "head_to_seq_rank", "ragged_reduce_scatter_rank", "ragged_all_gather_rank",
     "ragged_reduce_scatter_gated_rank", "bounded_wait_selftest",
@@ -174,10 +175,14 @@ def _stream_handle(stream, device) -> int:
     return int(stream.cuda_stream) if hasattr(stream, "cuda_stream") else int(stream)
 
 
-def _config(variant: int, ctas_per_sm: int, serial: bool = False):
-    if not variant and not ctas_per_sm and not serial:
+def _flags(serial: bool = False, token_chunks: bool = False) -> int:
+    return (H3_LAUNCH_SERIAL if serial else 0) | (H3_LAUNCH_CHUNK_TOKENS if token_chunks else 0)
+
+
+def _config(variant: int, ctas_per_sm: int, serial: bool = False, token_chunks: bool = False):
+    if not variant and not ctas_per_sm and not serial and not token_chunks:
         return None
-    return C.byref(LaunchConfig(int(variant), int(ctas_per_sm), H3_LAUNCH_SERIAL if serial else 0, 0))
+    return C.byref(LaunchConfig(int(variant), int(ctas_per_sm), _flags(serial, token_chunks), 0))
 
 
 def _relayout_shapes(seq_to_head_dir: bool, send, recv, layout: int = 0):
@@ -211,13 +216,13 @@ def _relayout_shapes(seq_to_head_dir: bool, send, recv, layout: int = 0):
 
 
 def _relayout_layout(seq_to_head_dir: bool, send, recv, layout, window_bytes, stream, variant,
-                     ctas_per_sm, serial=False):
+                     ctas_per_sm, serial=False, token_chunks=False):
     send = _as_list(send)
     recv = _as_list(recv)
     T, P, H, D, W, dev = _relayout_shapes(seq_to_head_dir, send, recv, layout)
     info = ExecInfo()
     name = "h3_seq_to_head_layout" if seq_to_head_dir else "h3_head_to_seq_layout"
-    cfg = _config(variant, ctas_per_sm, serial)
+    cfg = _config(variant, ctas_per_sm, serial, token_chunks)
     with _device_guard(dev):
         st = getattr(_abi.lib, name)(
             _abi.pointer_array([t.data_ptr() for t in send]),
@@ -229,20 +234,22 @@ def _relayout_layout(seq_to_head_dir: bool, send, recv, layout, window_bytes, st
 
 
 def seq_to_head_layout(send, recv, layout: int, *, window_bytes: int = 0, stream=None,
-                       variant: int = 0, ctas_per_sm: int = 0, serial: bool = False) -> dict:
+                       variant: int = 0, ctas_per_sm: int = 0, serial: bool = False,
+                       token_chunks: bool = False) -> dict:
     """seq->head with plane-major buffers (``layout``: bit set of
     H3_LAYOUT_SEQ_PLANE_MAJOR / H3_LAYOUT_HEAD_PLANE_MAJOR).  Plane-major
     sequence side: W tensors [P, T_r, H, D]; plane-major head side: W tensors
     [P, T, H_j, D] (out[j][0], [1], [2] are that rank's Q, K, V)."""
     return _relayout_layout(True, send, recv, layout, window_bytes, stream, variant, ctas_per_sm,
-                            serial)
+                            serial, token_chunks)
 
 
 def head_to_seq_layout(send, recv, layout: int, *, window_bytes: int = 0, stream=None,
-                       variant: int = 0, ctas_per_sm: int = 0, serial: bool = False) -> dict:
+                       variant: int = 0, ctas_per_sm: int = 0, serial: bool = False,
+                       token_chunks: bool = False) -> dict:
     """head->seq with plane-major buffers (see ``seq_to_head_layout``)."""
     return _relayout_layout(False, send, recv, layout, window_bytes, stream, variant, ctas_per_sm,
-                            serial)
+                            serial, token_chunks)
 
 
 def _relayout_staged(seq_to_head_dir: bool, send, recv, window, stream):
@@ -288,26 +295,28 @@ def staged_plan(n_tokens: int, planes: int, n_heads: int, head_dim: int, window_
 
 
 def relayout_chunk_plan(n_tokens: int, planes: int, n_heads: int, head_dim: int, world: int,
-                        window_bytes: int):
+                        window_bytes: int, *, token_chunks: bool = False):
     """(tokens of each rank per launch, launches) of a chunked relayout
-    (``h3_relayout_chunk_plan``, host only): one batch plane per launch, a
-    plane larger than the window split into equal token chunks."""
+    (``h3_relayout_chunk_plan_ex``, host only): one batch plane per launch, a
+    plane larger than the window split into equal token chunks; with
+    token_chunks=True, equal token ranges of every plane instead."""
     n = C.c_int64(0)
     k = C.c_int64(0)
-    st = _abi.lib.h3_relayout_chunk_plan(int(n_tokens), int(planes), int(n_heads), int(head_dim),
-                                         int(world), int(window_bytes), C.byref(n), C.byref(k))
-    _abi.check(st, "h3_relayout_chunk_plan")
+    st = _abi.lib.h3_relayout_chunk_plan_ex(int(n_tokens), int(planes), int(n_heads), int(head_dim),
+                                            int(world), int(window_bytes), _flags(False, token_chunks),
+                                            C.byref(n), C.byref(k), None)
+    _abi.check(st, "h3_relayout_chunk_plan_ex")
     return int(n.value), int(k.value)
 
 
 def _relayout(seq_to_head_dir: bool, send, recv, window_bytes, stream, variant, ctas_per_sm,
-              serial=False):
+              serial=False, token_chunks=False):
     send = _as_list(send)
     recv = _as_list(recv)
     T, P, H, D, W, dev = _relayout_shapes(seq_to_head_dir, send, recv)
     info = ExecInfo()
     name = "h3_seq_to_head" if seq_to_head_dir else "h3_head_to_seq"
-    cfg = _config(variant, ctas_per_sm, serial)
+    cfg = _config(variant, ctas_per_sm, serial, token_chunks)
     args = [_abi.pointer_array([t.data_ptr() for t in send]),
             _abi.pointer_array([t.data_ptr() for t in recv]),
             T, int(P), int(H), int(D), W, int(window_bytes),
@@ -322,22 +331,27 @@ def _relayout(seq_to_head_dir: bool, send, recv, window_bytes, stream, variant, 
 
 
 def seq_to_head(send, recv, *, window_bytes: int = 0, stream=None, variant: int = 0,
-                ctas_per_sm: int = 0, serial: bool = False) -> dict:
+                ctas_per_sm: int = 0, serial: bool = False, token_chunks: bool = False) -> dict:
     """Ulysses sequence->head relayout.
 
     send: W tensors [T_r, P, H, D] (or views of one [T, P, H, D] tensor, see
     ``split_rows``); recv: W tensors [T, P, H_j, D], written.  window_bytes > 0
-    moves one plane per launch under that byte bound.  serial=True launches
-    in plain stream order (H3_LAUNCH_SERIAL) instead of programmatic dependent
-    launch.  Returns what ran (launches, chunks, grid, block, variant)."""
-    return _relayout(True, send, recv, window_bytes, stream, variant, ctas_per_sm, serial)
+    moves one plane per launch under that byte bound; with token_chunks=True
+    (H3_LAUNCH_CHUNK_TOKENS) the window is cut into token ranges of every
+    plane instead, which keeps whole rows together.  serial=True launches in
+    plain stream order (H3_LAUNCH_SERIAL) instead of programmatic dependent
+    launch.  Returns what ran (launches, chunks, grid, block, variant,
+    planes_per_launch)."""
+    return _relayout(True, send, recv, window_bytes, stream, variant, ctas_per_sm, serial,
+                     token_chunks)
 
 
 def head_to_seq(send, recv, *, window_bytes: int = 0, stream=None, variant: int = 0,
-                ctas_per_sm: int = 0, serial: bool = False) -> dict:
+                ctas_per_sm: int = 0, serial: bool = False, token_chunks: bool = False) -> dict:
     """Inverse head->sequence relayout: send W tensors [T, P, H_j, D] -> recv W
-    tensors [T_r, P, H, D]."""
-    return _relayout(False, send, recv, window_bytes, stream, variant, ctas_per_sm, serial)
+    tensors [T_r, P, H, D].  Options as ``seq_to_head``."""
+    return _relayout(False, send, recv, window_bytes, stream, variant, ctas_per_sm, serial,
+                     token_chunks)
 
 
 def ragged_reduce_scatter(partials, bias, out, *, stream=None, ctas_per_sm: int = 0,
@@ -524,7 +538,8 @@ def _local_output(t: torch.Tensor, what: str, dims: int):
 
 
 def seq_to_head_rank(send, recv, rank: int, *, n_heads: int, window_bytes: int = 0, stream=None,
-                     variant: int = 0, ctas_per_sm: int = 0, serial: bool = False) -> dict:
+                     variant: int = 0, ctas_per_sm: int = 0, serial: bool = False,
+                     token_chunks: bool = False) -> dict:
     """Rank ``rank``'s head-side buffer with one rank per GPU
     (``h3_seq_to_head_rank``): send = the W ranks' sequence-side buffers
     [T_r, P, H, D]; recv = this rank's [T, P, H_k, D]."""
@@ -540,14 +555,15 @@ def seq_to_head_rank(send, recv, rank: int, *, n_heads: int, window_bytes: int =
         st = _abi.lib.h3_seq_to_head_rank(
             _abi.pointer_array(_addresses(send, "send")), C.c_void_p(recv.data_ptr()), T, P,
             int(n_heads), D, W, int(rank), int(window_bytes),
-            C.c_void_p(_stream_handle(stream, dev)), _config(variant, ctas_per_sm, serial),
-            C.byref(info))
+            C.c_void_p(_stream_handle(stream, dev)),
+            _config(variant, ctas_per_sm, serial, token_chunks), C.byref(info))
     _abi.check(st, "h3_seq_to_head_rank")
     return info.as_dict()
 
 
 def head_to_seq_rank(send, recv, rank: int, *, n_tokens: int, window_bytes: int = 0, stream=None,
-                     variant: int = 0, ctas_per_sm: int = 0, serial: bool = False) -> dict:
+                     variant: int = 0, ctas_per_sm: int = 0, serial: bool = False,
+                     token_chunks: bool = False) -> dict:
     """Rank ``rank``'s sequence-side rows with one rank per GPU
     (``h3_head_to_seq_rank``): send = the W ranks' head-side buffers
     [T, P, H_j, D]; recv = this rank's [T_k, P, H, D]."""
@@ -563,8 +579,8 @@ def head_to_seq_rank(send, recv, rank: int, *, n_tokens: int, window_bytes: int 
         st = _abi.lib.h3_head_to_seq_rank(
             _abi.pointer_array(_addresses(send, "send")), C.c_void_p(recv.data_ptr()),
             int(n_tokens), P, H, D, W, int(rank), int(window_bytes),
-            C.c_void_p(_stream_handle(stream, dev)), _config(variant, ctas_per_sm, serial),
-            C.byref(info))
+            C.c_void_p(_stream_handle(stream, dev)),
+            _config(variant, ctas_per_sm, serial, token_chunks), C.byref(info))
     _abi.check(st, "h3_head_to_seq_rank")
     return info.as_dict()
 
@@ -659,7 +675,7 @@ class PreparedRelayout:
 
     def __init__(self, seq_to_head_dir: bool, send, recv, *, layout: int = 0,
                  window_bytes: int = 0, variant: int = 0, ctas_per_sm: int = 0,
-                 serial: bool = False):
+                 serial: bool = False, token_chunks: bool = False):
         send = _as_list(send)
         recv = _as_list(recv)
         T, P, H, D, W, dev = _relayout_shapes(seq_to_head_dir, send, recv, layout)
@@ -671,12 +687,13 @@ class PreparedRelayout:
         self.variant = int(variant)
         self.ctas_per_sm = int(ctas_per_sm)
         self.serial = bool(serial)
+        self.token_chunks = bool(token_chunks)
         self._keep = (send, recv)  # keep the tensors alive while the call holds their addresses
         name = "h3_seq_to_head_layout" if seq_to_head_dir else "h3_head_to_seq_layout"
         self._fn = getattr(_abi.lib, name)
         self._name = name
         self._cfg = LaunchConfig(self.variant, self.ctas_per_sm,
-                                 H3_LAUNCH_SERIAL if self.serial else 0, 0)
+                                 _flags(self.serial, self.token_chunks), 0)
         self._info = ExecInfo()
         self._head = (_abi.pointer_array([t.data_ptr() for t in send]),
                       _abi.pointer_array([t.data_ptr() for t in recv]),
@@ -701,7 +718,8 @@ class PreparedRelayout:
         options; send/recv are that direction's buffers."""
         return PreparedRelayout(not self.seq_to_head_dir, send, recv, layout=self.layout,
                                 window_bytes=self.window_bytes, variant=self.variant,
-                                ctas_per_sm=self.ctas_per_sm, serial=self.serial)
+                                ctas_per_sm=self.ctas_per_sm, serial=self.serial,
+                                token_chunks=self.token_chunks)
 
 
 def prepare_seq_to_head(send, recv, **kw) -> PreparedRelayout:

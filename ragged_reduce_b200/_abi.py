@@ -44,8 +44,9 @@ MAX_WORLD = 64
 H3_LAYOUT_SEQ_PLANE_MAJOR = 1
 H3_LAYOUT_HEAD_PLANE_MAJOR = 2
 H3_LAUNCH_SERIAL = 1
+H3_LAUNCH_CHUNK_TOKENS = 2
 H3_IPC_HANDLE_BYTES = 64
-ABI_VERSION = 2
+ABI_VERSION = 3
 
 
 class ExecInfo(C.Structure):
@@ -157,6 +158,10 @@ def _load() -> C.CDLL:
     lib.h3_relayout_chunk_plan.restype = C.c_int
     lib.h3_relayout_chunk_plan.argtypes = [C.c_int64, C.c_int32, C.c_int32, C.c_int32, C.c_int32,
                                            C.c_int64, _i64p, _i64p]
+    lib.h3_relayout_chunk_plan_ex.restype = C.c_int
+    lib.h3_relayout_chunk_plan_ex.argtypes = [C.c_int64, C.c_int32, C.c_int32, C.c_int32, C.c_int32,
+                                              C.c_int64, C.c_int32, _i64p, _i64p,
+                                              C.POINTER(C.c_int32)]
     lib.h3_last_cuda_error.restype = C.c_int32
     lib.h3_last_cuda_error.argtypes = [C.POINTER(C.c_char_p)]
     lib.h3_bulk_wait_timeouts.restype = C.c_int

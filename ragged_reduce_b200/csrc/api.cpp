@@ -33,10 +33,12 @@ void clear_info(h3_exec_info* info)
 }
 
 // Launch-config fields every entry point checks the same way.
-bool config_ok(const h3_launch_config* cfg)
+bool config_ok(const h3_launch_config* cfg, int32_t allowed)
 {
-    return !cfg || (cfg->ctas_per_sm >= 0 && (cfg->flags & ~H3_LAUNCH_SERIAL) == 0 && cfg->reserved1 == 0);
+    return !cfg || (cfg->ctas_per_sm >= 0 && (cfg->flags & ~allowed) == 0 && cfg->reserved1 == 0);
 }
+
+bool token_range_chunks(const h3_launch_config* cfg) { return cfg && (cfg->flags & H3_LAUNCH_CHUNK_TOKENS); }
 
 bool programmatic_launch(const h3_launch_config* cfg) { return !(cfg && (cfg->flags & H3_LAUNCH_SERIAL)); }
 
@@ -135,7 +137,7 @@ h3_status relayout(bool seq_to_head, const void* const* send, void* const* recv,
         return H3_ERR_INVALID_ARG;
     if (cfg && cfg->variant != 0 && cfg->variant != H3_VARIANT_VECTOR && cfg->variant != H3_VARIANT_BULK)
         return H3_ERR_INVALID_ARG;
-    if (!config_ok(cfg))
+    if (!config_ok(cfg, H3_LAUNCH_SERIAL | H3_LAUNCH_CHUNK_TOKENS))
         return H3_ERR_INVALID_ARG;
     h3_status st = check_relayout_args(seq_to_head, send, recv, n_tokens, planes, n_heads, head_dim,
                                        world, nullptr, 0);
@@ -149,15 +151,14 @@ h3_status relayout(bool seq_to_head, const void* const* send, void* const* recv,
 
     // Chunked mode (FastVideo PR #1807, "Problem and behavior"): one batch
     // plane per launch, each rank's send and receive slices within the
-    // window; a plane too large for the window is split by tokens.
-    const bool chunked = window_bytes > 0;
+    // window; a plane too large for the window is split by tokens.  With
+    // H3_LAUNCH_CHUNK_TOKENS the same window is cut into token ranges of
+    // every plane instead.
     RelayoutChunks ch;
-    ch.tokens = ts.largest();
-    if (chunked) {
-        st = plan_relayout_chunks(ts, hs, n_tokens, row_bytes, head_bytes, window_bytes, &ch);
-        if (st != H3_OK)
-            return st;
-    }
+    st = plan_relayout(ts, hs, n_tokens, planes, row_bytes, head_bytes, window_bytes,
+                       token_range_chunks(cfg), &ch);
+    if (st != H3_OK)
+        return st;
 
     RelayoutArgs a;
     std::memset(&a, 0, sizeof(a));
@@ -189,15 +190,15 @@ h3_status relayout(bool seq_to_head, const void* const* send, void* const* recv,
         if (!relayout_bulk_fits(a, device))
             return H3_ERR_UNSUPPORTED;  // the bulk kernel's row stages do not fit in shared memory
     }
-    const int plane_groups = chunked ? planes : 1;
-    const int per_launch = chunked ? 1 : planes;
-    const int chunks = int(plane_groups * ch.per_plane);
+    const int plane_groups = ch.plane_groups;
+    const int per_launch = ch.per_launch;
+    const int chunks = int(plane_groups * ch.per_group);
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     LaunchShape shape;
     int launched = 0;
     const bool programmatic = programmatic_launch(cfg);
     for (int g = 0; g < plane_groups; ++g) {
-        for (int64_t c = 0; c < ch.per_plane; ++c) {
+        for (int64_t c = 0; c < ch.per_group; ++c) {
             int64_t cq = 0, cm = 0, t0 = 0;
             chunk_split(ts, ch, c, &cq, &cm, &t0);
             a.cq = int32_t(cq);
@@ -369,11 +370,13 @@ h3_status h3_staged_plan(int64_t n_tokens, int32_t planes, int32_t n_heads, int3
 }
 
 
-h3_status h3_relayout_chunk_plan(int64_t n_tokens, int32_t planes, int32_t n_heads,
-                                 int32_t head_dim, int32_t world, int64_t window_bytes,
-                                 int64_t* tokens_per_chunk, int64_t* chunks)
+h3_status h3_relayout_chunk_plan_ex(int64_t n_tokens, int32_t planes, int32_t n_heads,
+                                    int32_t head_dim, int32_t world, int64_t window_bytes,
+                                    int32_t flags, int64_t* tokens_per_chunk, int64_t* chunks,
+                                    int32_t* planes_per_launch)
 {
-    if (!tokens_per_chunk || !chunks || planes < 1 || head_dim < 1 || window_bytes < 0)
+    if (!tokens_per_chunk || !chunks || planes < 1 || head_dim < 1 || window_bytes < 0 ||
+        (flags & ~(H3_LAUNCH_SERIAL | H3_LAUNCH_CHUNK_TOKENS)) != 0)
         return H3_ERR_INVALID_ARG;
     const h3_status st = check_world(n_tokens, n_heads, world);
     if (st != H3_OK)
@@ -381,16 +384,24 @@ h3_status h3_relayout_chunk_plan(int64_t n_tokens, int32_t planes, int32_t n_hea
     const Split ts = make_split(n_tokens, world);
     const Split hs = make_split(n_heads, world);
     RelayoutChunks ch;
-    ch.tokens = ts.largest();
-    if (window_bytes > 0) {
-        const h3_status pst = plan_relayout_chunks(ts, hs, n_tokens, uint64_t(n_heads) * head_dim * 2,
-                                                   uint64_t(head_dim) * 2, window_bytes, &ch);
-        if (pst != H3_OK)
-            return pst;
-    }
+    const h3_status pst = plan_relayout(ts, hs, n_tokens, planes, uint64_t(n_heads) * head_dim * 2,
+                                        uint64_t(head_dim) * 2, window_bytes,
+                                        (flags & H3_LAUNCH_CHUNK_TOKENS) != 0, &ch);
+    if (pst != H3_OK)
+        return pst;
     *tokens_per_chunk = ch.tokens;
-    *chunks = window_bytes > 0 ? int64_t(planes) * ch.per_plane : 1;
+    *chunks = int64_t(ch.plane_groups) * ch.per_group;
+    if (planes_per_launch)
+        *planes_per_launch = ch.per_launch;
     return H3_OK;
+}
+
+h3_status h3_relayout_chunk_plan(int64_t n_tokens, int32_t planes, int32_t n_heads,
+                                 int32_t head_dim, int32_t world, int64_t window_bytes,
+                                 int64_t* tokens_per_chunk, int64_t* chunks)
+{
+    return h3_relayout_chunk_plan_ex(n_tokens, planes, n_heads, head_dim, world, window_bytes, 0,
+                                     tokens_per_chunk, chunks, nullptr);
 }
 
 int32_t h3_abi_version(void) { return H3RR_ABI_VERSION; }

@@ -21,8 +21,11 @@ constexpr int64_t kMaxRowVecs = int64_t(1) << 30;
 // ---------------------------------------------------------------------------
 bool aligned16(const void* p);
 void clear_info(h3_exec_info* info);
-// Launch-config fields every entry point checks the same way.
-bool config_ok(const h3_launch_config* cfg);
+// Launch-config fields every entry point checks the same way; `flags` may
+// hold only the bits in `allowed` (H3_LAUNCH_SERIAL everywhere, plus
+// H3_LAUNCH_CHUNK_TOKENS for the relayouts).
+bool config_ok(const h3_launch_config* cfg, int32_t allowed = H3_LAUNCH_SERIAL);
+bool token_range_chunks(const h3_launch_config* cfg);
 bool programmatic_launch(const h3_launch_config* cfg);
 // Partition checks ("Distributed H3 Execution", intro: empty token or head
 // partitions are rejected).
@@ -48,29 +51,38 @@ struct Split {
 
 Split make_split(int64_t n, int32_t w);
 
-// Token chunks of a chunked relayout (FastVideo PR #1807, "Problem and
-// behavior": one batch plane at a time through a byte window).  Each plane is
-// moved in `per_plane` launches; launch c covers local tokens
-// [c*tokens, c*tokens + tokens) of every rank (fewer in the last one), so
-// every launch is still one all-to-all over all ranks.  per_plane is 1 when a
-// whole plane fits the window.
+// The launches of a relayout call: plane_groups x per_group launches, each
+// moving per_launch planes of a range of local tokens of every rank:
+// range c of a group covers [c*tokens, c*tokens + tokens) (fewer in the
+// last one), so that every launch is one all-to-all over all ranks.
+//   unchunked (window 0):   1 group of all P planes, one range;
+//   one plane per launch:   P groups of one plane (FastVideo PR #1807,
+//                           "Problem and behavior": one batch plane at a
+//                           time through a byte window), split by tokens
+//                           when a plane does not fit;
+//   token ranges (H3_LAUNCH_CHUNK_TOKENS): 1 group of all P planes, split
+//                           by tokens so that every launch fits the window.
 struct RelayoutChunks {
-    int64_t per_plane = 1;
-    int64_t tokens = 0;
+    int64_t per_group = 1;  // token ranges per plane group
+    int64_t tokens = 0;     // local tokens of each rank per full range
+    int32_t plane_groups = 1;
+    int32_t per_launch = 1;  // planes per launch
 };
 
-// The chunking of a relayout over `window_bytes` (> 0): one plane per chunk
-// if every rank's send slice of a plane (T_r*row_bytes) and receive slice
-// (T*H_j*head_bytes) fit; otherwise the fewest equal token chunks whose
-// per-rank send slice (L*row_bytes) and receive slice (W*L*H_j*head_bytes)
-// fit.  H3_ERR_WINDOW if not even one token of every rank fits.
-h3_status plan_relayout_chunks(const Split& ts, const Split& hs, int64_t n_tokens,
-                               uint64_t row_bytes, uint64_t head_bytes, int64_t window_bytes,
-                               RelayoutChunks* out);
+// The plan of a relayout of `planes` planes over `window_bytes` (0 = one
+// launch).  A window must hold each rank's send slice (L tokens of
+// row_bytes per plane moved) and receive slice (L tokens of W ranks, of the
+// widest head rank, per plane moved); the fewest ranges of equal length L
+// that fit are used, or one per plane group when its whole slices fit.
+// H3_ERR_WINDOW if not even one token fits.
+h3_status plan_relayout(const Split& ts, const Split& hs, int64_t n_tokens, int32_t planes,
+                        uint64_t row_bytes, uint64_t head_bytes, int64_t window_bytes,
+                        bool token_ranges, RelayoutChunks* out);
 
-// Token split of chunk c: rank r holds cq + (r < cm) tokens of the chunk,
-// local tokens t0 .. of its range.  Full chunks are (tokens, 0); the last
-// chunk is what remains of the quotient/remainder split, (q - t0, m).
+// Token split of range c of a plane group: rank r holds cq + (r < cm) tokens
+// of the range, local tokens t0 .. of its own range.  Full ranges are
+// (tokens, 0); the last is what remains of the quotient/remainder split,
+// (q - t0, m).
 void chunk_split(const Split& ts, const RelayoutChunks& ch, int64_t c, int64_t* cq, int64_t* cm,
                  int64_t* t0);
 

@@ -25,38 +25,60 @@ Split make_split(int64_t n, int32_t w)
     return s;
 }
 
-h3_status plan_relayout_chunks(const Split& ts, const Split& hs, int64_t n_tokens,
-                               uint64_t row_bytes, uint64_t head_bytes, int64_t window_bytes,
-                               RelayoutChunks* out)
+namespace {
+
+// Token ranges of one plane group moving `planes` planes per launch.
+h3_status plan_ranges(const Split& ts, const Split& hs, int64_t n_tokens, int64_t planes,
+                      uint64_t row_bytes, uint64_t head_bytes, uint64_t window,
+                      int64_t* per_group, int64_t* tokens)
 {
-    const uint64_t window = uint64_t(window_bytes);
     const int64_t tmax = ts.largest();
-    const uint64_t head_run = uint64_t(hs.largest()) * head_bytes;  // one token of the widest head rank
-    if (uint64_t(tmax) * row_bytes <= window && uint64_t(n_tokens) * head_run <= window) {
-        out->per_plane = 1;
-        out->tokens = tmax;
+    const uint64_t send_token = uint64_t(planes) * row_bytes;  // one token of a rank, every plane moved
+    const uint64_t recv_token = uint64_t(planes) * uint64_t(hs.largest()) * head_bytes;
+    if (uint64_t(tmax) * send_token <= window && uint64_t(n_tokens) * recv_token <= window) {
+        *per_group = 1;
+        *tokens = tmax;
         return H3_OK;
     }
-    // A full chunk sends L rows from every rank and gives every head rank L
+    // A full range sends L tokens from every rank and gives every head rank L
     // tokens from each of the W ranks.
-    const uint64_t by_send = window / row_bytes;
-    const uint64_t by_recv = window / (uint64_t(ts.w) * head_run);
+    const uint64_t by_send = window / send_token;
+    const uint64_t by_recv = window / (uint64_t(ts.w) * recv_token);
     const uint64_t most = by_send < by_recv ? by_send : by_recv;
     if (most < 1)
         return H3_ERR_WINDOW;
-    // Fewest chunks, then equal lengths: ceil(tmax / L) is again k, so every
-    // chunk but the last is full and the last is not empty.
+    // Fewest ranges, then equal lengths: ceil(tmax / L) is again k, so every
+    // range but the last is full and the last is not empty.
     const int64_t k = (tmax + int64_t(most) - 1) / int64_t(most);
-    out->per_plane = k;
-    out->tokens = (tmax + k - 1) / k;
+    *per_group = k;
+    *tokens = (tmax + k - 1) / k;
     return H3_OK;
+}
+
+}  // namespace
+
+h3_status plan_relayout(const Split& ts, const Split& hs, int64_t n_tokens, int32_t planes,
+                        uint64_t row_bytes, uint64_t head_bytes, int64_t window_bytes,
+                        bool token_ranges, RelayoutChunks* out)
+{
+    if (window_bytes <= 0) {
+        out->plane_groups = 1;
+        out->per_launch = planes;
+        out->per_group = 1;
+        out->tokens = ts.largest();
+        return H3_OK;
+    }
+    out->plane_groups = token_ranges ? 1 : planes;
+    out->per_launch = token_ranges ? planes : 1;
+    return plan_ranges(ts, hs, n_tokens, out->per_launch, row_bytes, head_bytes, uint64_t(window_bytes),
+                       &out->per_group, &out->tokens);
 }
 
 void chunk_split(const Split& ts, const RelayoutChunks& ch, int64_t c, int64_t* cq, int64_t* cm,
                  int64_t* t0)
 {
     *t0 = c * ch.tokens;
-    if (c + 1 < ch.per_plane) {
+    if (c + 1 < ch.per_group) {
         *cq = ch.tokens;
         *cm = 0;
     } else {

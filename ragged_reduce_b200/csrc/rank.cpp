@@ -46,12 +46,11 @@ void fill_info(h3_exec_info* info, int launches, int chunks, const LaunchShape& 
     info->planes_per_launch = planes_per_launch;
 }
 
-// Checks of a relayout rank call; on success *chunked tells whether the
-// window asks for one plane per launch and *ch how each plane is split.
+// Checks of a relayout rank call; on success *ch is the call's launch plan.
 h3_status check_relayout_rank(bool seq_to_head, const void* const* send, const void* recv,
                               int64_t n_tokens, int32_t planes, int32_t n_heads, int32_t head_dim,
                               int32_t world, int32_t rank, int64_t window_bytes,
-                              const h3_launch_config* cfg, bool* chunked, RelayoutChunks* ch)
+                              const h3_launch_config* cfg, RelayoutChunks* ch)
 {
     if (window_bytes < 0)
         return H3_ERR_INVALID_ARG;
@@ -59,7 +58,7 @@ h3_status check_relayout_rank(bool seq_to_head, const void* const* send, const v
         return H3_ERR_UNSUPPORTED;
     if (cfg && cfg->variant != 0 && cfg->variant != H3_VARIANT_VECTOR)
         return H3_ERR_INVALID_ARG;
-    if (!config_ok(cfg))
+    if (!config_ok(cfg, H3_LAUNCH_SERIAL | H3_LAUNCH_CHUNK_TOKENS))
         return H3_ERR_INVALID_ARG;
     h3_status st = check_world(n_tokens, n_heads, world);
     if (st != H3_OK)
@@ -95,12 +94,8 @@ h3_status check_relayout_rank(bool seq_to_head, const void* const* send, const v
         return st;
     // The window bounds every rank's slices, exactly as in the one-GPU call,
     // so that all ranks chunk alike.
-    *chunked = window_bytes > 0;
-    ch->per_plane = 1;
-    ch->tokens = ts.largest();
-    if (*chunked)
-        return plan_relayout_chunks(ts, hs, n_tokens, row_bytes, head_bytes, window_bytes, ch);
-    return H3_OK;
+    return plan_relayout(ts, hs, n_tokens, planes, row_bytes, head_bytes, window_bytes,
+                         token_range_chunks(cfg), ch);
 }
 
 // Inputs one rank call may check: W partials, the gate rows, the residual
@@ -165,10 +160,9 @@ h3_status h3_seq_to_head_rank(const void* const* send, void* recv, int64_t n_tok
                               const h3_launch_config* cfg, h3_exec_info* info)
 {
     clear_info(info);
-    bool chunked = false;
     RelayoutChunks ch;
     h3_status st = check_relayout_rank(true, send, recv, n_tokens, planes, n_heads, head_dim, world,
-                                       rank, window_bytes, cfg, &chunked, &ch);
+                                       rank, window_bytes, cfg, &ch);
     if (st != H3_OK)
         return st;
     const Split ts = make_split(n_tokens, world);
@@ -187,14 +181,14 @@ h3_status h3_seq_to_head_rank(const void* const* send, void* recv, int64_t n_tok
     a.row_vecs = int32_t(int64_t(n_heads) * head_vecs);
     a.run_vecs = int32_t(hs.size(rank) * head_vecs);
     a.col0_vecs = int32_t(hs.start(rank) * head_vecs);
-    const int plane_groups = chunked ? planes : 1;
-    const int per_launch = chunked ? 1 : planes;
-    const int chunks = int(plane_groups * ch.per_plane);
+    const int plane_groups = ch.plane_groups;
+    const int per_launch = ch.per_launch;
+    const int chunks = int(plane_groups * ch.per_group);
     const bool programmatic = programmatic_launch(cfg);
     LaunchShape shape;
     int launched = 0;
     for (int g = 0; g < plane_groups; ++g) {
-        for (int64_t c = 0; c < ch.per_plane; ++c) {
+        for (int64_t c = 0; c < ch.per_group; ++c) {
             int64_t cq = 0, cm = 0, t0 = 0;
             chunk_split(ts, ch, c, &cq, &cm, &t0);
             a.cq = int32_t(cq);
@@ -224,10 +218,9 @@ h3_status h3_head_to_seq_rank(const void* const* send, void* recv, int64_t n_tok
                               const h3_launch_config* cfg, h3_exec_info* info)
 {
     clear_info(info);
-    bool chunked = false;
     RelayoutChunks ch;
     h3_status st = check_relayout_rank(false, send, recv, n_tokens, planes, n_heads, head_dim,
-                                       world, rank, window_bytes, cfg, &chunked, &ch);
+                                       world, rank, window_bytes, cfg, &ch);
     if (st != H3_OK)
         return st;
     const Split ts = make_split(n_tokens, world);
@@ -253,15 +246,15 @@ h3_status h3_head_to_seq_rank(const void* const* send, void* recv, int64_t n_tok
     a.hm = int32_t(hs.m);
     a.row_vecs = int32_t(int64_t(n_heads) * head_bytes / kVecBytes);
     a.head_vecs = int32_t(head_bytes / kVecBytes);
-    const int plane_groups = chunked ? planes : 1;
-    const int per_launch = chunked ? 1 : planes;
-    const int chunks = int(plane_groups * ch.per_plane);
+    const int plane_groups = ch.plane_groups;
+    const int per_launch = ch.per_launch;
+    const int chunks = int(plane_groups * ch.per_group);
     const bool programmatic = programmatic_launch(cfg);
     const int variant = cfg ? cfg->variant : 0;
     LaunchShape shape;
     int launched = 0;
     for (int g = 0; g < plane_groups; ++g) {
-        for (int64_t c = 0; c < ch.per_plane; ++c) {
+        for (int64_t c = 0; c < ch.per_group; ++c) {
             // This rank's tokens of chunk c of the plan all ranks share; the
             // last chunk may hold none of them.
             const int64_t t0 = c * ch.tokens;

@@ -55,6 +55,22 @@ int main(void)
            H3_OK && chunk_tokens == 62500 && chunks == 8, "chunk plan, 2 ranks");
     expect(h3_relayout_chunk_plan(250000, 4, 56, 128, 4, 14335, &chunk_tokens, &chunks) ==
            H3_ERR_WINDOW, "window below one token");
+    /* token ranges over all planes: the same window holds 15,625 tokens of
+     * all four planes of every rank, again 4 launches */
+    {
+        int32_t per_launch = 0;
+        expect(h3_relayout_chunk_plan_ex(250000, 4, 56, 128, 4, 896000000, H3_LAUNCH_CHUNK_TOKENS,
+                                         &chunk_tokens, &chunks, &per_launch) == H3_OK &&
+                   chunk_tokens == 15625 && chunks == 4 && per_launch == 4,
+               "token-range plan, 4 ranks");
+        expect(h3_relayout_chunk_plan_ex(250000, 4, 56, 128, 4, 896000000, 0, &chunk_tokens, &chunks,
+                                         &per_launch) == H3_OK &&
+                   chunk_tokens == 62500 && chunks == 4 && per_launch == 1,
+               "one-plane plan through _ex");
+        expect(h3_relayout_chunk_plan_ex(250000, 4, 56, 128, 4, 4 * 14336 - 16, H3_LAUNCH_CHUNK_TOKENS,
+                                         &chunk_tokens, &chunks, NULL) == H3_ERR_WINDOW,
+               "window below one token of every plane");
+    }
 
     /* argument checks fail before anything is launched */
     expect(h3_seq_to_head(NULL, NULL, 1000, 3, 56, 128, 6, 0, NULL, &info) == H3_ERR_INVALID_ARG &&

@@ -118,3 +118,15 @@ def chunk_window(kind, T, H, D, W):
     smallest = max(row, W * hmax * head)
     plane = max(tmax * row, T * hmax * head)
     return {"plane": plane, "sub": max(smallest, plane // 2), "min": smallest}[kind]
+
+
+def range_window(kind, T, P, H, D, W):
+    """Window bytes for token ranges over all planes (H3_LAUNCH_CHUNK_TOKENS):
+    "plane" (one plane of the largest rank: about P ranges), "half" (half of
+    that) or "min" (one token of every plane of every rank: one-token
+    ranges)."""
+    tmax, hmax = -(-T // W), -(-H // W)
+    row, head = H * D * 2, D * 2
+    smallest = P * max(row, W * hmax * head)
+    plane = max(tmax * row, T * hmax * head)
+    return {"plane": max(smallest, plane), "half": max(smallest, plane // 2), "min": smallest}[kind]

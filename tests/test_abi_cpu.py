@@ -208,14 +208,24 @@ def test_relayout_rejects_unknown_variant():
 
 @needs_no_gpu
 def test_launch_config_rejects_unknown_flags_and_reserved():
-    """Only H3_LAUNCH_SERIAL is a flag; reserved1 must be 0 (every _ex call)."""
+    """H3_LAUNCH_SERIAL is a flag of every _ex call, H3_LAUNCH_CHUNK_TOKENS of
+    the relayouts only; reserved1 must be 0."""
     T, P, H, D, W = 100, 3, 56, 128, 2
     send, recv = _layout(T, P, H, D, W)
     Cc = 64
     blocks = [BASE + r * (1 << 20) for r in range(W)]
     full = [BASE + (8 << 20) + r * (1 << 20) for r in range(W)]
-    for flags, reserved in ((2, 0), (4, 0), (-1, 0), (_abi.H3_LAUNCH_SERIAL | 8, 0), (0, 1),
-                            (_abi.H3_LAUNCH_SERIAL, -1)):
+    tok = _abi.H3_LAUNCH_CHUNK_TOKENS
+    for flags, reserved in ((tok, 0), (tok | _abi.H3_LAUNCH_SERIAL, 0)):
+        cfg = C.byref(_abi.LaunchConfig(0, 0, flags, reserved))
+        st = _abi.lib.h3_ragged_reduce_scatter_ex(_ptrs(full), None, _ptrs(blocks), T, Cc, W, None,
+                                                  cfg, C.byref(_abi.ExecInfo()))
+        assert st == _abi.H3_ERR_INVALID_ARG, flags
+        st = _abi.lib.h3_ragged_all_gather_ex(_ptrs(blocks), _ptrs(full), T, Cc, W, None, cfg,
+                                              C.byref(_abi.ExecInfo()))
+        assert st == _abi.H3_ERR_INVALID_ARG, flags
+    for flags, reserved in ((4, 0), (-1, 0), (_abi.H3_LAUNCH_SERIAL | 8, 0), (tok | 16, 0), (0, 1),
+                            (_abi.H3_LAUNCH_SERIAL, -1), (tok, 1)):
         cfg = C.byref(_abi.LaunchConfig(0, 0, flags, reserved))
         for fn in ("h3_seq_to_head_ex", "h3_head_to_seq_ex"):
             info = _abi.ExecInfo()
@@ -517,6 +527,111 @@ def test_last_cuda_error_is_kept_per_thread():
     t2.start()
     t2.join(timeout=60)
     assert other == [0]
+
+
+def _expected_range_plan(T, P, H, D, W, window):
+    """Token ranges over all planes, restated from the header's definition:
+    one launch if every rank's whole send and receive slices fit; else the
+    fewest ranges k and the equal length L = ceil(T_max / k) whose full
+    ranges fit (L tokens of P rows sent per rank, W*L tokens of P runs of the
+    widest head rank received)."""
+    tmax = -(-T // W)
+    hmax = -(-H // W)
+    send, recv = P * H * D * 2, P * hmax * D * 2
+    if tmax * send <= window and T * recv <= window:
+        return tmax, 1
+    for k in range(2, tmax + 1):
+        L = -(-tmax // k)
+        if L * send <= window and W * L * recv <= window:
+            return L, k
+    return None
+
+
+def test_relayout_range_plan_properties():
+    """h3_relayout_chunk_plan_ex with H3_LAUNCH_CHUNK_TOKENS against the
+    definition, over a grid of shapes and windows; the windows a one-plane
+    plan accepts but that cannot hold one token of every plane are refused;
+    without the flag _ex is h3_relayout_chunk_plan; planes per launch."""
+    rng = np.random.default_rng(17)
+    cases = [(250000, 4, 56, 128, 4), (250000, 4, 56, 128, 2), (32768, 3, 56, 128, 6),
+             (131072, 4, 56, 128, 4), (65536, 4, 56, 128, 8), (777, 1, 7, 64, 3)]
+    for _ in range(60):
+        W = int(rng.integers(1, 9))
+        cases.append((int(rng.integers(W, 5000)), int(rng.integers(1, 5)),
+                      int(rng.integers(W, 80)), 8 * int(rng.integers(1, 40)), W))
+    tok = _abi.H3_LAUNCH_CHUNK_TOKENS
+    for T, P, H, D, W in cases:
+        tmax, hmax = -(-T // W), -(-H // W)
+        row, head = H * D * 2, D * 2
+        smallest = P * max(row, W * hmax * head)
+        windows = {smallest, smallest + 16, T * P * row, tmax * P * row, tmax * P * row - 16,
+                   tmax * row, int(rng.integers(smallest, 4 * tmax * P * row + 1))}
+        for win in sorted(windows):
+            n, k, per = C.c_int64(0), C.c_int64(0), C.c_int32(0)
+            st = _abi.lib.h3_relayout_chunk_plan_ex(T, P, H, D, W, win, tok, C.byref(n), C.byref(k),
+                                                    C.byref(per))
+            want = _expected_range_plan(T, P, H, D, W, win)
+            if win < smallest:
+                assert st == _abi.H3_ERR_WINDOW and want is None
+                continue
+            assert st == _abi.H3_OK and (n.value, k.value) == want, (T, P, H, D, W, win)
+            assert per.value == P
+            assert rr.relayout_chunk_plan(T, P, H, D, W, win, token_chunks=True) == want
+            L, chunks = want
+            assert (chunks - 1) * L < tmax <= chunks * L    # exact cover, last range not empty
+            if chunks > 1:
+                assert L * P * row <= win and W * L * P * hmax * head <= win
+        # one token of one plane fits, one token of every plane does not
+        if P > 1:
+            st = _abi.lib.h3_relayout_chunk_plan_ex(T, P, H, D, W, smallest - 16, tok, C.byref(n),
+                                                    C.byref(k), None)
+            assert st == _abi.H3_ERR_WINDOW
+            assert rr.relayout_chunk_plan(T, P, H, D, W, smallest - 16)[1] >= P
+        # flags 0: the one-plane plan; window 0: one launch of all planes either way
+        for flags in (0, _abi.H3_LAUNCH_SERIAL):
+            win = tmax * row
+            st = _abi.lib.h3_relayout_chunk_plan_ex(T, P, H, D, W, win, flags, C.byref(n), C.byref(k),
+                                                    C.byref(per))
+            assert st == _abi.H3_OK and (n.value, k.value) == rr.relayout_chunk_plan(T, P, H, D, W, win)
+            assert per.value == 1
+        for flags in (0, tok):
+            st = _abi.lib.h3_relayout_chunk_plan_ex(T, P, H, D, W, 0, flags, C.byref(n), C.byref(k),
+                                                    C.byref(per))
+            assert st == _abi.H3_OK and (n.value, k.value, per.value) == (tmax, 1, P)
+
+
+def test_relayout_range_plan_rejects_bad_arguments():
+    n, k = C.c_int64(0), C.c_int64(0)
+    f = _abi.lib.h3_relayout_chunk_plan_ex
+    for flags in (4, -1, _abi.H3_LAUNCH_CHUNK_TOKENS | 8):
+        assert f(1000, 3, 56, 128, 4, 10 ** 9, flags, C.byref(n), C.byref(k), None) == _abi.H3_ERR_INVALID_ARG
+    assert f(1000, 3, 56, 128, 4, 10 ** 9, 2, None, C.byref(k), None) == _abi.H3_ERR_INVALID_ARG
+    assert f(1000, 3, 56, 128, 4, 10 ** 9, 2, C.byref(n), None, None) == _abi.H3_ERR_INVALID_ARG
+    assert f(1000, 0, 56, 128, 4, 10 ** 9, 2, C.byref(n), C.byref(k), None) == _abi.H3_ERR_INVALID_ARG
+    assert f(1000, 3, 56, 128, 4, -1, 2, C.byref(n), C.byref(k), None) == _abi.H3_ERR_INVALID_ARG
+    assert f(3, 3, 56, 128, 4, 10 ** 9, 2, C.byref(n), C.byref(k), None) == _abi.H3_ERR_EMPTY_PARTITION
+
+
+@needs_no_gpu
+def test_relayout_range_window_check_long_workload():
+    """250k QKVG over 4 ranks: the pages' window holds one plane of one rank
+    and equally 15,625 tokens of all four planes, so both shapes take 4
+    launches; a window below one token of every plane is refused by the
+    range shape before anything is launched, though one plane per launch
+    still fits it."""
+    T, P, H, D, W = 250000, 4, 56, 128, 4
+    send, recv = _layout(T, P, H, D, W)
+    assert 15625 * 4 * 56 * 128 * 2 == 896_000_000
+    assert rr.relayout_chunk_plan(T, P, H, D, W, 896_000_000, token_chunks=True) == (15625, 4)
+    assert rr.relayout_chunk_plan(T, P, H, D, W, 896_000_000 - 16, token_chunks=True) == (12500, 5)
+    small = P * H * D * 2 - 16
+    cfg = C.byref(_abi.LaunchConfig(0, 0, _abi.H3_LAUNCH_CHUNK_TOKENS, 0))
+    for fn in ("h3_seq_to_head_ex", "h3_head_to_seq_ex"):
+        info = _abi.ExecInfo()
+        st = getattr(_abi.lib, fn)(_ptrs(send), _ptrs(recv), T, P, H, D, W, small, None, cfg,
+                                   C.byref(info))
+        assert st == _abi.H3_ERR_WINDOW and info.launches == 0, fn
+    assert rr.relayout_chunk_plan(T, P, H, D, W, small)[1] > P
 
 
 def test_token_chunks_cover_every_token_once():

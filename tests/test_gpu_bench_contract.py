@@ -62,6 +62,14 @@ def test_native_line():
     assert isinstance(k["reasons"], list)
     shares = sum(v["share"] for v in d["kernels"].values())
     assert abs(shares - 1.0) < 0.01
+    # beside the line: the same window cut into token ranges of all planes
+    c = d["chunk_shapes"]
+    assert c["window_bytes"] == 896_000_000
+    r = c["token_ranges_all_planes"]
+    assert r["round_trip_ok"] is True and r["tokens_per_launch"] == 15625
+    for k in ("seq_to_head", "head_to_seq"):
+        assert r[k]["launches_per_call"] == 4 and r[k]["planes_per_launch"] == 4 and r[k]["gbs"] > 1000
+        assert c["one_plane_per_launch"][k]["launches_per_call"] == 4
 
 
 def test_reference_line():

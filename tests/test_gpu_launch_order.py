@@ -42,11 +42,12 @@ def test_serial_and_programmatic_launches_agree(oracle_lib, chunked):
 
 
 @pytest.mark.parametrize("serial", [False, True])
-@pytest.mark.parametrize("chunked", ["plane", "sub"])
+@pytest.mark.parametrize("chunked", ["plane", "sub", "ranges"])
 def test_chained_dependent_calls(oracle_lib, serial, chunked):
     """x -> heads -> back -> heads2 -> back2, all chunked (one plane per
-    launch, or every plane in token chunks), on one stream, with a fresh x
-    written by a PyTorch kernel before every round."""
+    launch, every plane in token chunks, or token ranges of all planes), on
+    one stream, with a fresh x written by a PyTorch kernel before every
+    round."""
     T, P, H, D, W = 4096, 4, 56, 128, 6
     part = rr.partition(T, H, W)
     x = torch.empty((T, P, H, D), dtype=torch.bfloat16, device=DEV)
@@ -55,16 +56,22 @@ def test_chained_dependent_calls(oracle_lib, serial, chunked):
     heads2 = rr.alloc_head_side(T, P, H, D, W, DEV)
     back_full, back = rr.alloc_seq_side(T, P, H, D, W, DEV)
     back2_full, back2 = rr.alloc_seq_side(T, P, H, D, W, DEV)
-    window = gu.chunk_window(chunked, T, H, D, W)
+    ranges = chunked == "ranges"
+    if ranges:
+        window = gu.range_window("plane", T, P, H, D, W) // 3  # about twelve ranges
+        assert rr.relayout_chunk_plan(T, P, H, D, W, window, token_chunks=True)[1] >= 10
+    else:
+        window = gu.chunk_window(chunked, T, H, D, W)
     if chunked == "sub":
         window //= 3  # about six token chunks per plane: long chains of launches
         assert rr.relayout_chunk_plan(T, P, H, D, W, window)[1] >= 5 * P
+    kw = dict(window_bytes=window, serial=serial, token_chunks=ranges)
     for round_ in range(8):
         x.copy_(wl.random_bits((T, P, H, D), 500 + round_, DEV))
-        rr.seq_to_head(send, heads, window_bytes=window, serial=serial)
-        rr.head_to_seq(heads, back, window_bytes=window, serial=serial)
-        rr.seq_to_head(back, heads2, window_bytes=window, serial=serial)
-        rr.head_to_seq(heads2, back2, window_bytes=window, serial=serial)
+        rr.seq_to_head(send, heads, **kw)
+        rr.head_to_seq(heads, back, **kw)
+        rr.seq_to_head(back, heads2, **kw)
+        rr.head_to_seq(heads2, back2, **kw)
         assert gu.same_bits(back_full, x), round_
         assert gu.same_bits(back2_full, x), round_
         for j in range(W):

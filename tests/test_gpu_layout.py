@@ -31,19 +31,20 @@ def _head_buffers(T, P, H, D, W, head_pm, part):
                                        (130, 2, 7, 64, 3), (50, 3, 5, 8, 5), (20, 2, 300, 128, 7),
                                        (33, 3, 56, 256, 4), (64, 3, 56, 128, 1)])
 @pytest.mark.parametrize("layout", [0, SPM, HPM, SPM | HPM])
-@pytest.mark.parametrize("chunked", [None, "plane", "sub"])
+@pytest.mark.parametrize("chunked", [None, "plane", "sub", "ranges"])
 def test_layout_matches_oracle(oracle_lib, T, P, H, D, W, layout, chunked):
     spm, hpm = bool(layout & SPM), bool(layout & HPM)
     send, part = _seq_buffers(T, P, H, D, W, spm, seed=T + W + layout)
     heads = _head_buffers(T, P, H, D, W, hpm, part)
-    window = gu.chunk_window(chunked, T, H, D, W)
-    info = rr.seq_to_head_layout(send, heads, layout, window_bytes=window)
-    assert info["launches"] == rr.relayout_chunk_plan(T, P, H, D, W, window)[1]
+    ranges = chunked == "ranges"  # token ranges of every plane (H3_LAUNCH_CHUNK_TOKENS)
+    window = gu.range_window("half", T, P, H, D, W) if ranges else gu.chunk_window(chunked, T, H, D, W)
+    info = rr.seq_to_head_layout(send, heads, layout, window_bytes=window, token_chunks=ranges)
+    assert info["launches"] == rr.relayout_chunk_plan(T, P, H, D, W, window, token_chunks=ranges)[1]
     want = oracle_lib.relayout_layout([gu.bits(s) for s in send], T, P, H, D, W, True, spm, hpm)
     for j in range(W):
         assert np.array_equal(gu.bits(heads[j]), want[j]), f"seq->head rank {j}"
     back = [torch.empty_like(s) for s in send]
-    rr.head_to_seq_layout(heads, back, layout, window_bytes=window)
+    rr.head_to_seq_layout(heads, back, layout, window_bytes=window, token_chunks=ranges)
     for r in range(W):
         assert gu.same_bits(back[r], send[r]), f"round trip rank {r}"
 

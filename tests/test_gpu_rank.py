@@ -24,18 +24,20 @@ SHAPES = [  # T, P, H, D, W
 
 
 @pytest.mark.parametrize("T,P,H,D,W", SHAPES)
-@pytest.mark.parametrize("chunked", [None, "plane", "sub"])
+@pytest.mark.parametrize("chunked", [None, "plane", "sub", "ranges"])
 def test_relayout_rank_shares(oracle_lib, T, P, H, D, W, chunked):
     part = rr.partition(T, H, W)
     x = wl.random_bits((T, P, H, D), T + W, DEV)
     send = rr.split_rows(x, part.token_starts)
     addrs = [int(s.data_ptr()) for s in send]
-    window = gu.chunk_window(chunked, T, H, D, W)
-    L, chunks = rr.relayout_chunk_plan(T, P, H, D, W, window)
+    ranges = chunked == "ranges"  # token ranges of every plane (H3_LAUNCH_CHUNK_TOKENS)
+    window = gu.range_window("half", T, P, H, D, W) if ranges else gu.chunk_window(chunked, T, H, D, W)
+    L, chunks = rr.relayout_chunk_plan(T, P, H, D, W, window, token_chunks=ranges)
     heads = [torch.empty((T, P, part.heads(k), D), dtype=torch.bfloat16, device=DEV)
              for k in range(W)]
     for k in range(W):
-        info = rr.seq_to_head_rank(addrs, heads[k], k, n_heads=H, window_bytes=window)
+        info = rr.seq_to_head_rank(addrs, heads[k], k, n_heads=H, window_bytes=window,
+                                   token_chunks=ranges)
         assert info["chunks"] == chunks and info["launches"] == chunks
     want = oracle_lib.seq_to_head([gu.bits(s) for s in send], T, P, H, D, W)
     for k in range(W):
@@ -43,11 +45,13 @@ def test_relayout_rank_shares(oracle_lib, T, P, H, D, W, chunked):
     back_full, back = rr.alloc_seq_side(T, P, H, D, W, DEV)
     head_addrs = [int(h.data_ptr()) for h in heads]
     for k in range(W):
-        info = rr.head_to_seq_rank(head_addrs, back[k], k, n_tokens=T, window_bytes=window)
+        info = rr.head_to_seq_rank(head_addrs, back[k], k, n_tokens=T, window_bytes=window,
+                                   token_chunks=ranges)
         # launches: the chunks that hold tokens of rank k
-        per_plane = chunks // P if window else 1
-        held = sum(1 for c in range(per_plane) if c * L < part.tokens(k))
-        assert info["chunks"] == chunks and info["launches"] == (held * P if window else 1)
+        groups = P if window and not ranges else 1
+        per_group = chunks // groups
+        held = sum(1 for c in range(per_group) if c * L < part.tokens(k))
+        assert info["chunks"] == chunks and info["launches"] == held * groups
     assert gu.same_bits(back_full, x)
 
 

@@ -322,6 +322,58 @@ def test_sub_plane_chunks_match_oracle(oracle_lib, T, P, H, D, W, kind, variant)
     assert rr.bulk_wait_timeouts() == 0
 
 
+@pytest.mark.parametrize("T,P,H,D,W", SUB_PLANE)
+@pytest.mark.parametrize("kind", ["plane", "half", "min"])
+@pytest.mark.parametrize("variant", [0, rr.H3_VARIANT_BULK])
+def test_token_range_chunks_match_oracle(oracle_lib, T, P, H, D, W, kind, variant):
+    """H3_LAUNCH_CHUNK_TOKENS: the window cut into token ranges of every
+    plane; launches, chunks and planes per launch as the plan says, results
+    equal to the oracle's in both directions."""
+    full, send, part = _seq_inputs(T, P, H, D, W, seed=T * 17 + W + len(kind))
+    window = gu.range_window(kind, T, P, H, D, W)
+    L, chunks = rr.relayout_chunk_plan(T, P, H, D, W, window, token_chunks=True)
+    recv = rr.alloc_head_side(T, P, H, D, W, DEV)
+    rr.bulk_wait_timeouts(reset=True)
+    info = rr.seq_to_head(send, recv, window_bytes=window, variant=variant, token_chunks=True)
+    assert info["chunks"] == chunks and info["launches"] == chunks and info["planes_per_launch"] == P
+    want = oracle_lib.seq_to_head([gu.bits(s) for s in send], T, P, H, D, W)
+    for j in range(W):
+        assert np.array_equal(gu.bits(recv[j]), want[j]), f"seq->head rank {j}"
+    back_full, back = rr.alloc_seq_side(T, P, H, D, W, DEV)
+    info = rr.head_to_seq(recv, back, window_bytes=window, variant=variant, token_chunks=True)
+    assert info["chunks"] == chunks and info["launches"] == chunks and info["planes_per_launch"] == P
+    want_back = oracle_lib.head_to_seq(want, T, P, H, D, W)
+    for r in range(W):
+        assert np.array_equal(gu.bits(back[r]), want_back[r]), f"head->seq rank {r}"
+    assert gu.same_bits(back_full, full)
+    assert rr.bulk_wait_timeouts() == 0
+
+
+def test_token_range_chunks_guard_bands():
+    """One-token ranges of every plane write nothing outside the outputs."""
+    T, P, H, D, W = 257, 3, 56, 128, 6
+    full, send, part = _seq_inputs(T, P, H, D, W, seed=43)
+    window = gu.range_window("min", T, P, H, D, W)
+    bufs, recv = [], []
+    for j in range(W):
+        b, r = gu.guarded((T, P, part.heads(j), D), DEV)
+        bufs.append(b)
+        recv.append(r)
+    info = rr.seq_to_head(send, recv, window_bytes=window, token_chunks=True)
+    assert info["launches"] == -(-T // W)
+    assert all(gu.guards_intact(b) for b in bufs)
+    back_bufs, back = [], []
+    for r in range(W):
+        b, o = gu.guarded((part.tokens(r), P, H, D), DEV)
+        back_bufs.append(b)
+        back.append(o)
+    rr.head_to_seq(recv, back, window_bytes=window, token_chunks=True)
+    assert all(gu.guards_intact(b) for b in back_bufs)
+    for r in range(W):
+        ts, te = int(part.token_starts[r]), int(part.token_starts[r + 1])
+        assert gu.same_bits(back[r], full[ts:te])
+
+
 def test_sub_plane_chunks_guard_bands():
     """One-token chunks write nothing outside the outputs."""
     T, P, H, D, W = 257, 3, 56, 128, 6
@@ -378,21 +430,21 @@ def test_stress_alternating(oracle_lib):
 # full-size workloads: sampled oracle elements + properties at any size
 # ---------------------------------------------------------------------------
 
-def _full_size_round_trip(o, w, planes=None, window=0, seed_offset=0):
+def _full_size_round_trip(o, w, planes=None, window=0, seed_offset=0, token_chunks=False):
     P = w.P if planes is None else planes
     full = wl.packed_operand(w, planes=P, device=DEV, seed_offset=seed_offset)
     bounds = wl.segment_bounds(w.T, w.n_segs, w.seed, w.seg_lengths)
     part = rr.partition(w.T, w.H, w.W, bounds)
     send = rr.split_rows(full, part.token_starts)
     recv = rr.alloc_head_side(w.T, P, w.H, w.D, w.W, DEV)
-    info = rr.seq_to_head(send, recv, window_bytes=window)
+    info = rr.seq_to_head(send, recv, window_bytes=window, token_chunks=token_chunks)
     # torch slicing as a third opinion on every element
     for j in range(w.W):
         hs, he = int(part.head_starts[j]), int(part.head_starts[j + 1])
         assert gu.same_bits(recv[j], full[:, :, hs:he, :]), f"rank {j} differs from slicing"
     gu.sampled_check_seq_to_head(o, send, recv, w.T, P, w.H, w.D, w.W, seed=w.seed)
     back_full, back = rr.alloc_seq_side(w.T, P, w.H, w.D, w.W, DEV)
-    info_back = rr.head_to_seq(recv, back, window_bytes=window)
+    info_back = rr.head_to_seq(recv, back, window_bytes=window, token_chunks=token_chunks)
     gu.sampled_check_head_to_seq(o, recv, back, w.T, P, w.H, w.D, w.W, seed=w.seed + 1)
     assert gu.same_bits(back_full, full)
     return info, info_back
@@ -431,6 +483,20 @@ def test_full_qkvg_250k_w4_chunked(oracle_lib):
     torch.cuda.empty_cache()
 
 
+def test_full_qkvg_250k_w4_token_ranges(oracle_lib):
+    """The long-sequence operand under the pages' window cut into token
+    ranges of all four planes: 15,625 tokens of every rank per launch
+    (896,000,000 bytes each way per rank, as one plane of one rank), 4
+    launches per direction; every element against torch slicing, sampled
+    elements against the oracle, the round trip exact."""
+    w = wl.QKVG_250K_W4_CHUNKED
+    assert rr.relayout_chunk_plan(w.T, w.P, w.H, w.D, w.W, w.window_bytes, token_chunks=True) == (15625, 4)
+    info, info_back = _full_size_round_trip(oracle_lib, w, window=w.window_bytes, token_chunks=True)
+    for i in (info, info_back):
+        assert i["chunks"] == 4 and i["launches"] == 4 and i["planes_per_launch"] == 4
+    torch.cuda.empty_cache()
+
+
 def test_full_qkvg_250k_w2_sub_plane(oracle_lib):
     """The long-sequence operand over 2 ranks: one plane of one rank is
     1,792,000,000 bytes, twice the 896,000,000-byte window, so every plane
@@ -463,5 +529,18 @@ def test_prepared_calls_and_inverse(oracle_lib):
         for j in range(W):
             assert np.array_equal(gu.bits(heads[j]), want[j])
         assert gu.same_bits(back_full, full)
+    # prepared token-range chunks, and their inverse, keep the option
+    window = gu.range_window("half", T, P, H, D, W)
+    chunks = rr.relayout_chunk_plan(T, P, H, D, W, window, token_chunks=True)[1]
+    fwd = rr.prepare_seq_to_head(send, heads, window_bytes=window, token_chunks=True)
+    bwd = fwd.inverse(heads, back)
+    assert bwd.token_chunks
+    full.copy_(wl.random_bits((T, P, H, D), 40, DEV))
+    assert fwd().launches == chunks and bwd().launches == chunks
+    torch.cuda.synchronize()
+    want = oracle_lib.seq_to_head([gu.bits(s) for s in send], T, P, H, D, W)
+    for j in range(W):
+        assert np.array_equal(gu.bits(heads[j]), want[j])
+    assert gu.same_bits(back_full, full)
     with pytest.raises(ValueError):
         rr.prepare_seq_to_head(send, heads[:-1])

@@ -79,8 +79,13 @@ def test_relayout_rank_argument_checks():
         bulk = C.byref(_abi.LaunchConfig(E.H3_VARIANT_BULK, 0, 0, 0))
         assert _call_relayout(fn, send, free, T, P, H, D, W, 0, cfg=bulk) == E.H3_ERR_UNSUPPORTED
         for cfg in (_abi.LaunchConfig(7, 0, 0, 0), _abi.LaunchConfig(0, -1, 0, 0),
-                    _abi.LaunchConfig(0, 0, 2, 0), _abi.LaunchConfig(0, 0, 0, 1)):
+                    _abi.LaunchConfig(0, 0, 4, 0), _abi.LaunchConfig(0, 0, 0, 1)):
             assert _call_relayout(fn, send, free, T, P, H, D, W, 0, cfg=C.byref(cfg)) == E.H3_ERR_INVALID_ARG
+        # token-range chunks are a relayout option: the window check applies to
+        # one token of every plane (P = 3 planes here)
+        tok = C.byref(_abi.LaunchConfig(0, 0, _abi.H3_LAUNCH_CHUNK_TOKENS, 0))
+        assert _call_relayout(fn, send, free, T, P, H, D, W, 0, cfg=tok,
+                              window=P * 6 * 10 * D * 2 - 16) == E.H3_ERR_WINDOW
 
 
 @needs_no_gpu
@@ -124,6 +129,8 @@ def test_rows_rank_argument_checks():
         assert f(o=0) == E.H3_ERR_INVALID_ARG
         assert f(o=ins[2] + 4096) == E.H3_ERR_INVALID_ARG      # output inside an input
         assert f(cfg=C.byref(_abi.LaunchConfig(0, 0, 4, 0))) == E.H3_ERR_INVALID_ARG
+        # token-range chunks only mean something to the relayouts
+        assert f(cfg=C.byref(_abi.LaunchConfig(0, 0, _abi.H3_LAUNCH_CHUNK_TOKENS, 0))) == E.H3_ERR_INVALID_ARG
         if f is rs:
             assert f(parts=full[:-1] + [full[-1] + 8]) == E.H3_ERR_MISALIGNED
         else:
