@@ -115,9 +115,9 @@ def load_peak():
 # The sources each measured kernel is compiled from (the rank calls' pull
 # kernel lives in relayout.cu too).
 KERNEL_SOURCES = {
-    "seq_to_head": ("relayout.cu", "device_access.cuh", "bulk_copy.cuh", "h3rr_internal.h"),
-    "head_to_seq": ("relayout.cu", "device_access.cuh", "bulk_copy.cuh", "h3rr_internal.h"),
-    "ragged_reduce_scatter": ("reduce_scatter.cu", "bf16_sum.cuh", "device_access.cuh", "h3rr_internal.h"),
+    "seq_to_head": ("relayout.cu", "device_access.cuh", "bulk_copy.cuh", "kernel_args.h"),
+    "head_to_seq": ("relayout.cu", "device_access.cuh", "bulk_copy.cuh", "kernel_args.h"),
+    "ragged_reduce_scatter": ("reduce_scatter.cu", "bf16_sum.cuh", "device_access.cuh", "kernel_args.h"),
 }
 
 

@@ -13,7 +13,7 @@
 #include <cuda_bf16.h>
 
 #include "device_access.cuh"
-#include "h3rr_internal.h"
+#include "kernel_args.h"
 
 namespace h3rr {
 

@@ -18,6 +18,7 @@
 // 16-byte vectors with 128 threads; W > 8 loads the partials in batches of 8.
 // The gated variant is in reduce_scatter_gated.cu.
 #include "bf16_sum.cuh"
+#include "h3rr_internal.h"
 
 namespace h3rr {
 namespace {

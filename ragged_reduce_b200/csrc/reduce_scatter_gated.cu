@@ -10,6 +10,7 @@
 // x may be the output buffer itself (in place): each element is read by the
 // thread that then writes it, with plain (coherent) loads.
 #include "bf16_sum.cuh"
+#include "h3rr_internal.h"
 
 namespace h3rr {
 namespace {

@@ -6,7 +6,8 @@
  *
  * Cases: both Ulysses relayouts ("Distributed H3 Execution", intro), whole,
  * one batch plane per launch and in token chunks of a plane (FastVideo PR
- * #1807, "Problem and behavior"); the ragged reduce-scatter and the ragged
+ * #1807, "Problem and behavior"), and in token ranges of every plane
+ * (H3_LAUNCH_CHUNK_TOKENS); the ragged reduce-scatter and the ragged
  * all-gather
  * ("Distributed H3 Execution", "Partition Contract"). */
 #include <stdint.h>
@@ -113,7 +114,7 @@ static int same_as_dev(const void* d, const uint16_t* want, int64_t elems)
 
 /* seq->head then head->seq of a [T, P, H, D] operand over W ranks. */
 static void relayout_case(int64_t T, int32_t P, int32_t H, int32_t D, int32_t W, int64_t window,
-                          cudaStream_t stream)
+                          int32_t flags, cudaStream_t stream)
 {
     int64_t ts[MAXW + 1], hs[MAXW + 1];
     uint16_t *send[MAXW], *want[MAXW], *back_want[MAXW];
@@ -143,14 +144,21 @@ static void relayout_case(int64_t T, int32_t P, int32_t H, int32_t D, int32_t W,
 
     {
         int64_t tokens = 0, chunks = 0;
-        expect(h3_relayout_chunk_plan(T, P, H, D, W, window, &tokens, &chunks) == H3_OK,
+        int32_t per_launch = 0;
+        h3_launch_config cfg;
+        memset(&cfg, 0, sizeof(cfg));
+        cfg.flags = flags;
+        expect(h3_relayout_chunk_plan_ex(T, P, H, D, W, window, flags, &tokens, &chunks,
+                                         &per_launch) == H3_OK,
                "chunk plan");
-        expect(h3_seq_to_head((const void* const*)d_send, d_heads, T, P, H, D, W, window, stream,
-                              &info) == H3_OK, "h3_seq_to_head status");
-        expect(info.launches == chunks && info.chunks == chunks, "seq->head launches");
+        expect(h3_seq_to_head_ex((const void* const*)d_send, d_heads, T, P, H, D, W, window, stream,
+                                 &cfg, &info) == H3_OK, "h3_seq_to_head status");
+        expect(info.launches == chunks && info.chunks == chunks && info.planes_per_launch == per_launch,
+               "seq->head launches");
+        expect(h3_head_to_seq_ex((const void* const*)d_heads, d_back, T, P, H, D, W, window, stream,
+                                 &cfg, &info) == H3_OK, "h3_head_to_seq status");
+        expect(info.launches == chunks && info.planes_per_launch == per_launch, "head->seq launches");
     }
-    expect(h3_head_to_seq((const void* const*)d_heads, d_back, T, P, H, D, W, window, stream,
-                          &info) == H3_OK, "h3_head_to_seq status");
     cuda_ok(cudaStreamSynchronize(stream), "relayout sync");
     for (r = 0; r < W; ++r) {
         snprintf(what, sizeof what, "seq->head T=%lld P=%d W=%d window=%lld rank %d", (long long)T,
@@ -244,15 +252,18 @@ int main(void)
         return 2;
     expect(h3_abi_version() == H3RR_ABI_VERSION, "abi version");
 
-    relayout_case(1000, 3, 56, 128, 6, 0, stream);
+    relayout_case(1000, 3, 56, 128, 6, 0, 0, stream);
     /* one plane per launch: the window holds the largest plane slice (rank
      * 0's 167 tokens x 56 heads and 1000 tokens x 10 heads, both x 256 B) */
-    relayout_case(1000, 3, 56, 128, 6, 1000 * 10 * 256, stream);
+    relayout_case(1000, 3, 56, 128, 6, 1000 * 10 * 256, 0, stream);
     /* a window of a third of a plane: every plane in token chunks (at most 55
      * tokens of every rank fit, so 4 chunks of 42 per plane) */
-    relayout_case(1000, 3, 56, 128, 6, 1000 * 10 * 256 / 3, stream);
-    relayout_case(777, 4, 56, 128, 8, 0, stream);
-    relayout_case(97, 2, 9, 8, 3, 0, stream);
+    relayout_case(1000, 3, 56, 128, 6, 1000 * 10 * 256 / 3, 0, stream);
+    /* the same window cut into token ranges of all three planes: at most 18
+     * tokens of every rank fit, so 10 launches of 17 */
+    relayout_case(1000, 3, 56, 128, 6, 1000 * 10 * 256 / 3, H3_LAUNCH_CHUNK_TOKENS, stream);
+    relayout_case(777, 4, 56, 128, 8, 0, 0, stream);
+    relayout_case(97, 2, 9, 8, 3, 0, 0, stream);
     reduce_gather_case(777, 7168, 8, stream);
     reduce_gather_case(1000, 2048, 6, stream);
     reduce_gather_case(33, 24, 1, stream);
