@@ -1032,10 +1032,12 @@ def run_profile(args):
     for _ in range(args.steps):
         if args.profile == "seq_to_head":
             info = rr.seq_to_head_layout(step.send, step.heads, layout, window_bytes=step.window,
-                                         variant=args.profile_variant)
+                                         variant=args.profile_variant,
+                                         token_chunks=args.profile_token_chunks)
         elif args.profile == "head_to_seq":
             info = rr.head_to_seq_layout(step.heads, step.back, layout, window_bytes=step.window,
-                                         variant=args.profile_variant)
+                                         variant=args.profile_variant,
+                                         token_chunks=args.profile_token_chunks)
         elif args.profile == "reduce_scatter":
             info = rr.ragged_reduce_scatter(step.partial_list, step.bias, step.red_out)
         elif args.profile == "gated_reduce_scatter":
@@ -1051,7 +1053,8 @@ def run_profile(args):
         launches += info["launches"]
     torch.cuda.synchronize()
     print(json.dumps({"profile": args.profile, "tokens": step.T, "rows": step.Tr,
-                      "layout": layout, "window": step.window, "launches": launches}), flush=True)
+                      "layout": layout, "window": step.window, "launches": launches,
+                      "token_chunks": bool(args.profile_token_chunks)}), flush=True)
     return 0
 
 
@@ -1363,7 +1366,10 @@ def parse_args(argv=None):
                    help="window bytes of the relayouts for --profile (-1: the bench's 896,000,000; "
                         "0: one launch over all planes)")
     p.add_argument("--profile-variant", type=int, default=0,
-                   help="relayout kernel family for --profile: 0 default, 1 vector, 2 bulk (TMA ring)")
+                   help="relayout kernel family for --profile: 0 default, 1 vector, 2 bulk (TMA)")
+    p.add_argument("--profile-token-chunks", action="store_true",
+                   help="relayouts for --profile cut the window into token ranges of every plane "
+                        "(H3_LAUNCH_CHUNK_TOKENS) instead of one plane per launch")
     p.add_argument("--profile-layout", type=int, default=0,
                    help="relayout buffers for --profile: bit 1 sequence side plane-major, "
                         "bit 2 head side plane-major (h3_*_layout)")

@@ -83,16 +83,22 @@ def test_reference_line():
     ("seq_to_head", 0, -1, 8), ("head_to_seq", 0, -1, 8), ("seq_to_head", 3, -1, 8),
     ("head_to_seq", 2, -1, 8), ("seq_to_head", 0, 0, 2), ("reduce_scatter", 0, -1, 2),
     ("gated_reduce_scatter", 0, -1, 2), ("all_gather", 0, -1, 2),
-    ("staged_seq_to_head", 0, -1, 16), ("rank_seq_to_head", 0, -1, 8)])
+    ("staged_seq_to_head", 0, -1, 16), ("rank_seq_to_head", 0, -1, 8),
+    ("seq_to_head", 0, 14_680_064, 8), ("head_to_seq", 0, 14_680_064, 8)])
 def test_profile_modes_run(mode, layout, window, launches):
     """Every --profile mode (the commands of the ncu captures) runs its kernel:
     the relayouts one batch plane per launch (4 planes, 2 calls), or in one
     launch with no window."""
+    # a window of one plane of one rank of the 4096-token operand (1,024 tokens
+    # x 56 x 128 x 2 B = 14,680,064 B) cut into token ranges of all four
+    # planes: 256 tokens a launch, four per call (the token-range captures)
+    tok = ["--profile-token-chunks"] if window == 14_680_064 else []
     out = subprocess.run([sys.executable, "bench.py", "--profile", mode, "--steps", "2",
                           "--profile-tokens", "4096", "--profile-rows", "4096",
-                          "--profile-layout", str(layout), "--profile-window", str(window)],
+                          "--profile-layout", str(layout), "--profile-window", str(window), *tok],
                          cwd=ROOT, capture_output=True, text=True, timeout=600)
     assert out.returncode == 0, out.stdout[-2000:] + out.stderr[-2000:]
     rec = json.loads([l for l in out.stdout.splitlines() if l.startswith("{")][-1])
     assert rec["profile"] == mode and rec["launches"] == launches
+    assert rec["token_chunks"] == bool(tok)
     assert rec["tokens" if "reduce" not in mode and mode != "all_gather" else "rows"] == 4096
