@@ -45,30 +45,36 @@ def test_fuzz_relayout(oracle_lib, case):
     smallest = max(H * D * 2, W * part.heads(0) * D * 2)  # one token of every rank
     # no window, a whole plane, more than a plane, or less than a plane (token chunks)
     window = int(rng.choice([0, plane, plane * P, int(rng.integers(smallest, plane + 1))]))
+    # half the windowed cases cut the window into token ranges of every plane,
+    # which needs room for one token of every plane
+    tok = window > 0 and bool(rng.integers(0, 2))
+    if tok:
+        window = max(window, P * smallest)
     variant = int(rng.choice([0, rr.H3_VARIANT_VECTOR]))
-    info = rr.seq_to_head_layout(send, heads, layout, window_bytes=window, variant=variant)
-    assert info["launches"] == rr.relayout_chunk_plan(T, P, H, D, W, window)[1]
+    kw = dict(window_bytes=window, token_chunks=tok)
+    info = rr.seq_to_head_layout(send, heads, layout, variant=variant, **kw)
+    assert info["launches"] == rr.relayout_chunk_plan(T, P, H, D, W, window, token_chunks=tok)[1]
     want = oracle_lib.relayout_layout([gu.bits(s) for s in send], T, P, H, D, W, True, spm, hpm)
     for j in range(W):
-        assert np.array_equal(gu.bits(heads[j]), want[j]), (T, P, H, D, W, layout, j)
+        assert np.array_equal(gu.bits(heads[j]), want[j]), (T, P, H, D, W, layout, tok, j)
     back = [torch.empty_like(s) for s in send]
-    rr.head_to_seq_layout(heads, back, layout, window_bytes=window, variant=variant)
+    rr.head_to_seq_layout(heads, back, layout, variant=variant, **kw)
     for r in range(W):
-        assert gu.same_bits(back[r], send[r]), (T, P, H, D, W, layout, r)
-    if layout == 0 and H * D * 2 * 14 + 128 <= 227 * 1024:
+        assert gu.same_bits(back[r], send[r]), (T, P, H, D, W, layout, tok, r)
+    if layout == 0 and H * D * 2 * 4 + 128 <= 227 * 1024:  # four row stages fit
         bulk = [torch.empty_like(h) for h in heads]
-        rr.seq_to_head(send, bulk, window_bytes=window, variant=rr.H3_VARIANT_BULK)
+        rr.seq_to_head(send, bulk, variant=rr.H3_VARIANT_BULK, **kw)
         for j in range(W):
             assert gu.same_bits(bulk[j], heads[j])
     if layout == 0:
         # one rank's shares (one rank per GPU) under the same window
         k = int(rng.integers(0, W))
         mine = torch.empty_like(heads[k])
-        rr.seq_to_head_rank(send, mine, k, n_heads=H, window_bytes=window)
-        assert gu.same_bits(mine, heads[k]), (T, P, H, D, W, window, k)
+        rr.seq_to_head_rank(send, mine, k, n_heads=H, **kw)
+        assert gu.same_bits(mine, heads[k]), (T, P, H, D, W, window, tok, k)
         rows = torch.empty_like(send[k])
-        rr.head_to_seq_rank(heads, rows, k, n_tokens=T, window_bytes=window)
-        assert gu.same_bits(rows, send[k]), (T, P, H, D, W, window, k)
+        rr.head_to_seq_rank(heads, rows, k, n_tokens=T, **kw)
+        assert gu.same_bits(rows, send[k]), (T, P, H, D, W, window, tok, k)
 
 
 @pytest.mark.parametrize("case", range(N_CASES // 2))
