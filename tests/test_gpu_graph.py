@@ -37,13 +37,19 @@ def test_step_replays_from_a_cuda_graph(oracle_lib):
     resid_full = resid_src.clone()
     resid = rr.split_rows(resid_full, rr.partition(T, W, W).token_starts)
 
-    # seq->head with every plane in token chunks, head->seq one plane per launch
+    # seq->head with every plane in token chunks, head->seq one plane per
+    # launch, then seq->head again in token ranges of every plane into a
+    # second set of buffers
     sub = gu.chunk_window("sub", T, H, D, W)
     assert rr.relayout_chunk_plan(T, P, H, D, W, sub)[1] > P
+    ranges_window = gu.range_window("half", T, P, H, D, W)
+    assert rr.relayout_chunk_plan(T, P, H, D, W, ranges_window, token_chunks=True)[1] > 1
+    heads2 = rr.alloc_head_side(T, P, H, D, W, DEV)
 
     def step():
         rr.seq_to_head(send, heads, window_bytes=sub)
         rr.head_to_seq(heads, back, window_bytes=window)
+        rr.seq_to_head(send, heads2, window_bytes=ranges_window, token_chunks=True)
         rr.ragged_reduce_scatter(partials, bias, red)
         rr.ragged_all_gather(red, gath)
         resid_full.copy_(resid_src)
@@ -66,6 +72,7 @@ def test_step_replays_from_a_cuda_graph(oracle_lib):
         want = oracle_lib.seq_to_head([gu.bits(s) for s in send], T, P, H, D, W)
         for j in range(W):
             assert np.array_equal(gu.bits(heads[j]), want[j]), (round_, j)
+            assert gu.same_bits(heads2[j], heads[j]), (round_, j)
         assert gu.same_bits(back_full, x)
         want_red = oracle_lib.ragged_reduce_scatter([gu.bits(p) for p in partials.unbind(0)],
                                                     gu.bits(bias), W)

@@ -56,9 +56,10 @@ class Job:
 
 
 class Relayout(Job):
-    def __init__(self, o, seed, T, P, H, D, W, window=0, variant=0):
-        self.name = f"relayout T={T} P={P} W={W} window={window} variant={variant}"
-        self.window, self.variant = window, variant
+    def __init__(self, o, seed, T, P, H, D, W, window=0, variant=0, token_chunks=False):
+        self.name = (f"relayout T={T} P={P} W={W} window={window} variant={variant}"
+                     f"{' token ranges' if token_chunks else ''}")
+        self.window, self.variant, self.token_chunks = window, variant, token_chunks
         full = wl.random_bits((T, P, H, D), seed, DEV)
         part = rr.partition(T, H, W)
         self.send = rr.split_rows(full, part.token_starts)
@@ -72,9 +73,9 @@ class Relayout(Job):
 
     def calls(self, stream):
         rr.seq_to_head(self.send, self.heads, window_bytes=self.window, variant=self.variant,
-                       stream=stream)
+                       stream=stream, token_chunks=self.token_chunks)
         rr.head_to_seq(self.heads, self.back, window_bytes=self.window, variant=self.variant,
-                       stream=stream)
+                       stream=stream, token_chunks=self.token_chunks)
 
 
 class Staged(Relayout):
@@ -136,7 +137,9 @@ def main():
         Relayout(o, 401, 1000, 3, 56, 128, 6),
         Relayout(o, 402, 777, 4, 56, 128, 8, window=700_000),  # 3 token chunks per plane
         Relayout(o, 403, 513, 1, 56, 128, 4, variant=rr.H3_VARIANT_BULK),
-        Relayout(o, 404, 1000, 3, 56, 128, 6, variant=rr.H3_VARIANT_BULK),
+        # bulk kernels over token ranges of all three planes (5 ranges)
+        Relayout(o, 404, 1000, 3, 56, 128, 6, window=1_700_000, variant=rr.H3_VARIANT_BULK,
+                 token_chunks=True),
         Staged(o, 405, 600, 3, 56, 128, 5, window_rows=41),
         ReduceGather(o, 406, 1000, 7168, 6),
         ReduceGather(o, 407, 333, 7168, 3, ctas_per_sm=2, gather_variant=rr.H3_VARIANT_BULK),
