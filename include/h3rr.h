@@ -49,8 +49,11 @@
  *     nothing is launched and the returned status says why.
  *   - `info` (nullable) receives what actually ran: launches, chunks, grid,
  *     block and kernel variant.
+ *   - Sizes: a relayout's T and T*P below 2^31, a row (H*D*2 bytes) of at
+ *     most 2^30 16-byte vectors and each side (T*P*H*D*2 bytes) at most 2^56
+ *     bytes; beyond them H3_ERR_UNSUPPORTED.
  *   - Thread-safe, and no environment variables are read.  State kept across
- *     calls: per-device caches (SM count, resident CTAs per kernel),
+ *     calls: per-device caches (SM count),
  *     per-context state (the bulk kernels' shared-memory opt-in, the static
  *     window's address, the peer mappings h3_ipc_open holds until
  *     h3_ipc_close; after cudaDeviceReset the device's next context sets them

@@ -40,6 +40,23 @@ bool config_ok(const h3_launch_config* cfg, int32_t allowed)
 
 bool token_range_chunks(const h3_launch_config* cfg) { return cfg && (cfg->flags & H3_LAUNCH_CHUNK_TOKENS); }
 
+h3_status check_relayout_sizes(int64_t n_tokens, int32_t planes, int32_t n_heads, int32_t head_dim)
+{
+    if (planes < 1 || head_dim < 1 || n_heads < 1 || n_tokens < 1)
+        return H3_ERR_INVALID_ARG;
+    if ((int64_t(head_dim) * 2) % kVecBytes != 0)
+        return H3_ERR_MISALIGNED;
+    const int64_t row_bytes = int64_t(n_heads) * head_dim * 2;
+    if (n_tokens > kMaxInt32 || n_tokens * planes > kMaxInt32 || row_bytes / kVecBytes > kMaxRowVecs)
+        return H3_ERR_UNSUPPORTED;
+    // Every side of the relayout is T*P rows of row_bytes; bounding it keeps
+    // every byte count of the checks and the launch plan within 64 bits
+    // (the plan multiplies it by at most the rank count).
+    if (n_tokens * planes > int64_t(kMaxSideBytes / uint64_t(row_bytes)))
+        return H3_ERR_UNSUPPORTED;
+    return H3_OK;
+}
+
 bool programmatic_launch(const h3_launch_config* cfg) { return !(cfg && (cfg->flags & H3_LAUNCH_SERIAL)); }
 
 // Partition checks shared by the relayouts and the reduce-scatter
@@ -86,13 +103,11 @@ h3_status check_relayout_args(bool seq_to_head, const void* const* send, void* c
     h3_status st = check_world(n_tokens, n_heads, world);
     if (st != H3_OK)
         return st;
-    if (planes < 1 || head_dim < 1 || !send || !recv)
+    if (!send || !recv)
         return H3_ERR_INVALID_ARG;
-    if ((int64_t(head_dim) * 2) % kVecBytes != 0)
-        return H3_ERR_MISALIGNED;
-    if (n_tokens > kMaxInt32 || n_tokens * planes > kMaxInt32 ||
-        int64_t(n_heads) * head_dim * 2 / kVecBytes > kMaxRowVecs)
-        return H3_ERR_UNSUPPORTED;
+    st = check_relayout_sizes(n_tokens, planes, n_heads, head_dim);
+    if (st != H3_OK)
+        return st;
     const Split ts = make_split(n_tokens, world);
     const Split hs = make_split(n_heads, world);
     const uint64_t row_bytes = uint64_t(n_heads) * head_dim * 2;
@@ -378,7 +393,10 @@ h3_status h3_relayout_chunk_plan_ex(int64_t n_tokens, int32_t planes, int32_t n_
     if (!tokens_per_chunk || !chunks || planes < 1 || head_dim < 1 || window_bytes < 0 ||
         (flags & ~(H3_LAUNCH_SERIAL | H3_LAUNCH_CHUNK_TOKENS)) != 0)
         return H3_ERR_INVALID_ARG;
-    const h3_status st = check_world(n_tokens, n_heads, world);
+    h3_status st = check_world(n_tokens, n_heads, world);
+    if (st != H3_OK)
+        return st;
+    st = check_relayout_sizes(n_tokens, planes, n_heads, head_dim);
     if (st != H3_OK)
         return st;
     const Split ts = make_split(n_tokens, world);

@@ -21,6 +21,15 @@ void clear_info(h3_exec_info* info);
 // H3_LAUNCH_CHUNK_TOKENS for the relayouts).
 bool config_ok(const h3_launch_config* cfg, int32_t allowed = H3_LAUNCH_SERIAL);
 bool token_range_chunks(const h3_launch_config* cfg);
+// Largest side of a relayout in bytes (64 PiB: far above any device), so
+// that byte counts times the rank count stay within 64 bits.
+constexpr uint64_t kMaxSideBytes = uint64_t(1) << 56;
+// Sizes of a relayout (all entry points and the plan queries): positive
+// sizes (H3_ERR_INVALID_ARG), head rows of whole 16-byte vectors
+// (H3_ERR_MISALIGNED), T*P rows within int32, a row within kMaxRowVecs
+// vectors and each side's T*P*H*D*2 bytes within kMaxSideBytes
+// (H3_ERR_UNSUPPORTED).
+h3_status check_relayout_sizes(int64_t n_tokens, int32_t planes, int32_t n_heads, int32_t head_dim);
 bool programmatic_launch(const h3_launch_config* cfg);
 // Partition checks ("Distributed H3 Execution", intro: empty token or head
 // partitions are rejected).

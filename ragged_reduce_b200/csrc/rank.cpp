@@ -63,13 +63,11 @@ h3_status check_relayout_rank(bool seq_to_head, const void* const* send, const v
     h3_status st = check_world(n_tokens, n_heads, world);
     if (st != H3_OK)
         return st;
-    if (rank < 0 || rank >= world || planes < 1 || head_dim < 1 || !send || !recv)
+    if (rank < 0 || rank >= world || !send || !recv)
         return H3_ERR_INVALID_ARG;
-    if ((int64_t(head_dim) * 2) % kVecBytes != 0)
-        return H3_ERR_MISALIGNED;
-    if (n_tokens > kMaxInt32 || n_tokens * planes > kMaxInt32 ||
-        int64_t(n_heads) * head_dim * 2 / kVecBytes > kMaxRowVecs)
-        return H3_ERR_UNSUPPORTED;
+    st = check_relayout_sizes(n_tokens, planes, n_heads, head_dim);
+    if (st != H3_OK)
+        return st;
     const Split ts = make_split(n_tokens, world);
     const Split hs = make_split(n_heads, world);
     const uint64_t row_bytes = uint64_t(n_heads) * head_dim * 2;

@@ -682,3 +682,34 @@ def test_token_chunks_cover_every_token_once():
             assert sum(counts) * hmax * head <= window
         assert len(seen) == T
     assert checked_empty_rank  # some last chunk left a smaller rank without tokens
+
+
+@needs_no_gpu
+def test_relayout_sides_beyond_the_byte_limit_are_refused():
+    """A relayout side of T*P*H*D*2 bytes above 2^56 (rows and row width each
+    within their own limits) is refused with H3_ERR_UNSUPPORTED by every
+    relayout entry point and the plan queries, before any byte count could
+    leave 64 bits; just below the limit the plan query answers."""
+    W = 2
+    send = [BASE + r * (1 << 50) for r in range(W)]   # made-up, never dereferenced
+    recv = [BASE + (4 + r) * (1 << 50) for r in range(W)]
+    n, k = C.c_int64(0), C.c_int64(0)
+    plan = _abi.lib.h3_relayout_chunk_plan_ex
+    for T, P, H, D in ((1 << 30, 1, 1 << 16, 1 << 14), (1 << 28, 4, 1 << 16, 1 << 14),
+                       ((1 << 31) - 1, 1, 1 << 15, 1 << 14)):
+        assert T * P * H * D * 2 > 1 << 56 and T * P < 2 ** 31 and H * D * 2 // 16 <= 1 << 30
+        for flags in (0, _abi.H3_LAUNCH_CHUNK_TOKENS):
+            assert plan(T, P, H, D, W, 10 ** 9, flags, C.byref(n), C.byref(k), None) == _abi.H3_ERR_UNSUPPORTED
+        assert _abi.lib.h3_relayout_chunk_plan(T, P, H, D, W, 0, C.byref(n), C.byref(k)) == _abi.H3_ERR_UNSUPPORTED
+        for fn in ("h3_seq_to_head", "h3_head_to_seq"):
+            st, info = _relayout_status(send, recv, T, P, H, D, W, fn=fn)
+            assert st == _abi.H3_ERR_UNSUPPORTED and info.launches == 0, (fn, T, P)
+        for fn in ("h3_seq_to_head_rank", "h3_head_to_seq_rank"):
+            info = _abi.ExecInfo()
+            st = getattr(_abi.lib, fn)(_ptrs(send), C.c_void_p(recv[0]), T, P, H, D, W, 0, 0, None,
+                                       None, C.byref(info))
+            assert st == _abi.H3_ERR_UNSUPPORTED and info.launches == 0, (fn, T, P)
+    # 2^55 bytes a side: within the limit
+    assert plan(1 << 30, 1, 1 << 10, 1 << 14, W, 10 ** 9, 0, C.byref(n), C.byref(k), None) == _abi.H3_OK
+    # a head row that is not whole 16-byte vectors, through the plan query too
+    assert plan(1000, 3, 56, 4, W, 10 ** 9, 0, C.byref(n), C.byref(k), None) == _abi.H3_ERR_MISALIGNED
