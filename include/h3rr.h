@@ -51,7 +51,8 @@
  *     block and kernel variant.
  *   - Sizes: a relayout's T and T*P below 2^31, a row (H*D*2 bytes) of at
  *     most 2^30 16-byte vectors and each side (T*P*H*D*2 bytes) at most 2^56
- *     bytes; beyond them H3_ERR_UNSUPPORTED.
+ *     bytes; the row calls' T below 2^31, C/8 at most 2^30 and T*C*2 at most
+ *     2^56 bytes; beyond them H3_ERR_UNSUPPORTED.
  *   - Thread-safe, and no environment variables are read.  State kept across
  *     calls: per-device caches (SM count),
  *     per-context state (the bulk kernels' shared-memory opt-in, the static

@@ -40,6 +40,12 @@ bool config_ok(const h3_launch_config* cfg, int32_t allowed)
 
 bool token_range_chunks(const h3_launch_config* cfg) { return cfg && (cfg->flags & H3_LAUNCH_CHUNK_TOKENS); }
 
+bool rows_beyond_limits(int64_t n_tokens, int64_t cols)
+{
+    return n_tokens > kMaxInt32 || cols / 8 > kMaxRowVecs ||
+           n_tokens > int64_t(kMaxSideBytes / uint64_t(cols * 2));
+}
+
 h3_status check_relayout_sizes(int64_t n_tokens, int32_t planes, int32_t n_heads, int32_t head_dim)
 {
     if (planes < 1 || head_dim < 1 || n_heads < 1 || n_tokens < 1)
@@ -551,7 +557,7 @@ h3_status h3_ragged_reduce_scatter_ex(const void* const* partials, const void* b
         return H3_ERR_INVALID_ARG;
     if (cols % 8 != 0)
         return H3_ERR_MISALIGNED;
-    if (n_tokens > kMaxInt32 || cols / 8 > kMaxRowVecs)
+    if (rows_beyond_limits(n_tokens, cols))
         return H3_ERR_UNSUPPORTED;
     const Split ts = make_split(n_tokens, world);
     const uint64_t row_bytes = uint64_t(cols) * 2;
@@ -645,7 +651,7 @@ h3_status h3_ragged_all_gather_ex(const void* const* in, void* const* out, int64
         return H3_ERR_INVALID_ARG;
     if (cols % 8 != 0)
         return H3_ERR_MISALIGNED;
-    if (n_tokens > kMaxInt32 || cols / 8 > kMaxRowVecs)
+    if (rows_beyond_limits(n_tokens, cols))
         return H3_ERR_UNSUPPORTED;
     const Split ts = make_split(n_tokens, world);
     const uint64_t row_bytes = uint64_t(cols) * 2;
@@ -722,7 +728,7 @@ h3_status h3_ragged_reduce_scatter_gated(const void* const* partials, const void
             return H3_ERR_INVALID_ARG;
     if (cols % 8 != 0)
         return H3_ERR_MISALIGNED;
-    if (n_tokens > kMaxInt32 || cols / 8 > kMaxRowVecs)
+    if (rows_beyond_limits(n_tokens, cols))
         return H3_ERR_UNSUPPORTED;
     if (!aligned16(gate) || (bias && !aligned16(bias)))
         return H3_ERR_MISALIGNED;

@@ -30,6 +30,10 @@ constexpr uint64_t kMaxSideBytes = uint64_t(1) << 56;
 // vectors and each side's T*P*H*D*2 bytes within kMaxSideBytes
 // (H3_ERR_UNSUPPORTED).
 h3_status check_relayout_sizes(int64_t n_tokens, int32_t planes, int32_t n_heads, int32_t head_dim);
+// Row-based calls (reduce-scatters, all-gather) on [T, C] BF16 rows (C >= 1):
+// true if T is beyond int32, a row beyond kMaxRowVecs vectors or T*C*2
+// beyond kMaxSideBytes.
+bool rows_beyond_limits(int64_t n_tokens, int64_t cols);
 bool programmatic_launch(const h3_launch_config* cfg);
 // Partition checks ("Distributed H3 Execution", intro: empty token or head
 // partitions are rejected).

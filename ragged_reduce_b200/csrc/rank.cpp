@@ -143,7 +143,7 @@ h3_status check_cols(int64_t n_tokens, int64_t cols, int32_t world, int32_t rank
         return H3_ERR_INVALID_ARG;
     if (cols % 8 != 0)
         return H3_ERR_MISALIGNED;
-    if (n_tokens > kMaxInt32 || cols / 8 > kMaxRowVecs)
+    if (rows_beyond_limits(n_tokens, cols))
         return H3_ERR_UNSUPPORTED;
     return H3_OK;
 }

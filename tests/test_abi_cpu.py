@@ -713,3 +713,24 @@ def test_relayout_sides_beyond_the_byte_limit_are_refused():
     assert plan(1 << 30, 1, 1 << 10, 1 << 14, W, 10 ** 9, 0, C.byref(n), C.byref(k), None) == _abi.H3_OK
     # a head row that is not whole 16-byte vectors, through the plan query too
     assert plan(1000, 3, 56, 4, W, 10 ** 9, 0, C.byref(n), C.byref(k), None) == _abi.H3_ERR_MISALIGNED
+
+
+@needs_no_gpu
+def test_row_calls_beyond_the_byte_limit_are_refused():
+    """Reduce-scatter, gated reduce-scatter, all-gather and their rank calls
+    refuse T*C*2 above 2^56 bytes (T and C/8 each within their own limits)
+    with H3_ERR_UNSUPPORTED before anything is launched."""
+    W, T, Cc = 2, (1 << 31) - 1, 1 << 28
+    assert T * Cc * 2 > 1 << 56 and Cc // 8 <= 1 << 30
+    full = [BASE + r * (1 << 52) for r in range(W)]   # made-up, never dereferenced
+    blocks = [BASE + (4 + r) * (1 << 52) for r in range(W)]
+    info = _abi.ExecInfo()
+    assert _abi.lib.h3_ragged_reduce_scatter(_ptrs(full), None, _ptrs(blocks), T, Cc, W, None,
+                                             C.byref(info)) == _abi.H3_ERR_UNSUPPORTED
+    assert _abi.lib.h3_ragged_all_gather(_ptrs(blocks), _ptrs(full), T, Cc, W, None,
+                                         C.byref(info)) == _abi.H3_ERR_UNSUPPORTED
+    assert _abi.lib.h3_ragged_reduce_scatter_rank(_ptrs(full), None, C.c_void_p(blocks[0]), T, Cc, W, 0,
+                                                  None, None, C.byref(info)) == _abi.H3_ERR_UNSUPPORTED
+    assert _abi.lib.h3_ragged_all_gather_rank(_ptrs(blocks), C.c_void_p(full[0]), T, Cc, W, 0, None,
+                                              None, C.byref(info)) == _abi.H3_ERR_UNSUPPORTED
+    assert info.launches == 0
