@@ -774,7 +774,7 @@ def measure(args, make_step, rank, world, local, device, timer, n_events):
             "metric": METRIC, "value": round(value, 1), "unit": UNIT, "n_gpus": world,
             "steps": K, "warmup": args.warmup, "ms_per_step": round(t_max / K * 1e3, 4),
             "higher_is_better": True, "scaling": "strong" if world > 1 else "weak",
-            "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "vs_baseline": None, "dtype": "bf16", "accumulate_dtype": "f32", "data": "synthetic",
             "config": {"workload": WORKLOAD,
                        "relayout": {"tokens": RELAYOUT.T, "planes": RELAYOUT.P,
                                     "heads": RELAYOUT.H, "head_dim": RELAYOUT.D,
@@ -974,7 +974,8 @@ def run_reference(args):
         "impl": "reference", "metric": METRIC, "value": round(value, 3), "unit": UNIT,
         "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": round(t / args.steps * 1e3, 3), "higher_is_better": True,
-        "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "accumulate_dtype": "f32",
+        "data": "synthetic",
         "config": {"workload": WORKLOAD, "relayout_tokens": RELAYOUT.T, "reduce_rows": REDUCE.T,
                    "sample_tokens": each * cores, "sample_rows": sample_rows(each) * cores},
         "cpu_baseline": {"value": round(value, 3), "unit": UNIT, "cores": cores, "kind": "oracle",

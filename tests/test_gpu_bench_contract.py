@@ -28,7 +28,7 @@ def test_native_line():
     assert d["metric"] and d["unit"] == "GB/s" and d["n_gpus"] == 1
     assert d["steps"] == 100 and d["warmup"] == 3 and d["ms_per_step"] > 0
     assert d["higher_is_better"] is True and d["scaling"] == "weak" and d["vs_baseline"] is None
-    assert d["dtype"] == "bf16" and d["data"] == "synthetic"
+    assert d["dtype"] == "bf16" and d["accumulate_dtype"] == "f32" and d["data"] == "synthetic"
     assert d["config"]["workload"] == bench.WORKLOAD == \
         "qkvg_T250000_W4_chunked+reduce_scatter_T65536_C7168_W8"
     assert d["config"]["relayout"]["window_bytes"] == 896_000_000
