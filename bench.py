@@ -757,7 +757,8 @@ def measure(args, make_step, rank, world, local, device, timer, n_events):
     # Beside the line, not in its value: the same window cut into token
     # ranges of every plane instead of one batch plane per launch.
     ranges = None
-    if world == 1 and isinstance(timer, CudaTimer) and getattr(step, "has_relayout", False):
+    if (world == 1 and isinstance(timer, CudaTimer) and getattr(step, "has_relayout", False)
+            and not getattr(args, "no_chunk_shapes", False)):
         ranges = step.token_range_rates(max(3, min(20, K)), stream)
         if not ranges["round_trip_ok"]:
             raise SystemExit("token-range relayouts produced wrong results")
@@ -1355,6 +1356,9 @@ def parse_args(argv=None):
     p.add_argument("--impl", choices=["native", "reference"], default="native")
     p.add_argument("--e2e-steps", type=int, default=10)
     p.add_argument("--no-cpu-baseline", action="store_true")
+    p.add_argument("--no-chunk-shapes", action="store_true",
+                   help="skip the token-range relayouts timed beside the line (chunk_shapes), "
+                        "e.g. for a launch list of the step's own kernels")
     p.add_argument("--cpu-budget", type=float, default=12.0,
                    help="about how many seconds cpu_baseline spends on the oracle")
     p.add_argument("--profile", choices=["seq_to_head", "head_to_seq", "reduce_scatter",
