@@ -37,7 +37,8 @@ __all__ = [
     "ragged_reduce_scatter", "alloc_head_side", "alloc_seq_side", "split_rows",
     "H3_VARIANT_VECTOR", "H3_VARIANT_BULK", "H3_VARIANT_REDUCE", "MAX_WORLD", "library_path",
     "bulk_wait_timeouts", "alloc_reduce_outputs", "seq_to_head_staged", "head_to_seq_staged",
-    "staged_plan", "relayout_chunk_plan", "H3_VARIANT_STAGED", "ragged_all_gather", "H3_VARIANT_GATHER",
+    "staged_plan", "relayout_chunk_plan", "relayout_launch_plan", "H3_VARIANT_STAGED",
+    "ragged_all_gather", "H3_VARIANT_GATHER",
     "seq_to_head_layout", "head_to_seq_layout", "H3_LAYOUT_SEQ_PLANE_MAJOR",
     "H3_LAYOUT_HEAD_PLANE_MAJOR", "ragged_reduce_scatter_gated", "PreparedRelayout", "H3_LAUNCH_SERIAL",
     "H3_LAUNCH_CHUNK_TOKENS",
@@ -307,6 +308,23 @@ def relayout_chunk_plan(n_tokens: int, planes: int, n_heads: int, head_dim: int,
                                             C.byref(n), C.byref(k), None)
     _abi.check(st, "h3_relayout_chunk_plan_ex")
     return int(n.value), int(k.value)
+
+
+def relayout_launch_plan(n_tokens: int, planes: int, n_heads: int, head_dim: int, world: int,
+                         window_bytes: int, *, token_chunks: bool = False) -> dict:
+    """The launches a relayout call will make (``h3_relayout_chunk_plan_ex``,
+    host only): {"tokens_per_launch": L (tokens of each rank, the last launch
+    of a plane group may hold fewer), "launches": count, "planes_per_launch":
+    1 one plane per launch or P}."""
+    n = C.c_int64(0)
+    k = C.c_int64(0)
+    per = C.c_int32(0)
+    st = _abi.lib.h3_relayout_chunk_plan_ex(int(n_tokens), int(planes), int(n_heads), int(head_dim),
+                                            int(world), int(window_bytes), _flags(False, token_chunks),
+                                            C.byref(n), C.byref(k), C.byref(per))
+    _abi.check(st, "h3_relayout_chunk_plan_ex")
+    return {"tokens_per_launch": int(n.value), "launches": int(k.value),
+            "planes_per_launch": int(per.value)}
 
 
 def _relayout(seq_to_head_dir: bool, send, recv, window_bytes, stream, variant, ctas_per_sm,

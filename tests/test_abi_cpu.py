@@ -734,3 +734,17 @@ def test_row_calls_beyond_the_byte_limit_are_refused():
     assert _abi.lib.h3_ragged_all_gather_rank(_ptrs(blocks), C.c_void_p(full[0]), T, Cc, W, 0, None,
                                               None, C.byref(info)) == _abi.H3_ERR_UNSUPPORTED
     assert info.launches == 0
+
+
+def test_relayout_launch_plan_dict():
+    """The binding's full plan query: tokens per launch, launches and planes
+    per launch for the three cuts of the 250k QKVG operand over 4 ranks."""
+    T, P, H, D, W = 250000, 4, 56, 128, 4
+    assert rr.relayout_launch_plan(T, P, H, D, W, 0) == \
+        {"tokens_per_launch": 62500, "launches": 1, "planes_per_launch": 4}
+    assert rr.relayout_launch_plan(T, P, H, D, W, 896_000_000) == \
+        {"tokens_per_launch": 62500, "launches": 4, "planes_per_launch": 1}
+    assert rr.relayout_launch_plan(T, P, H, D, W, 896_000_000, token_chunks=True) == \
+        {"tokens_per_launch": 15625, "launches": 4, "planes_per_launch": 4}
+    with pytest.raises(rr.H3Error):
+        rr.relayout_launch_plan(T, P, H, D, W, P * H * D * 2 - 16, token_chunks=True)
