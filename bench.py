@@ -102,6 +102,40 @@ def throughput_gbs(bytes_per_step_per_gpu: float, steps: int, n_gpus: int, secon
     return bytes_per_step_per_gpu * steps * n_gpus / seconds / 1e9
 
 
+def step_bytes(world: int) -> int:
+    """Whole-job algorithmic bytes of one step: the QKVG round trip (every
+    element read and written once each way) and the reduce-scatter; with one
+    rank per GPU every rank also reads the bias."""
+    rb = relayout_bytes(RELAYOUT.T, RELAYOUT.P, RELAYOUT.H, RELAYOUT.D)
+    if world > 1:
+        return 2 * rb + reduce_bytes(REDUCE.T, REDUCE.C, world) + (world - 1) * REDUCE.C * 2
+    return 2 * rb + reduce_bytes(REDUCE.T, REDUCE.C, REDUCE.W)
+
+
+def step_config(world: int) -> dict:
+    """The line's `config`: the workload the step runs at `world` GPUs, the
+    same for the native and the reference arm."""
+    if world > 1:
+        parallelism = (f"one rank per GPU: W={world} ranks, tokens and heads split "
+                       f"by quotient/remainder, shares pulled over NVLink")
+    else:
+        parallelism = (f"one GPU: W={RELAYOUT.W} virtual ranks (relayout), "
+                       f"W={REDUCE.W} (reduce-scatter)")
+    return {"workload": WORKLOAD,
+            "relayout": {"tokens": RELAYOUT.T, "planes": RELAYOUT.P,
+                         "heads": RELAYOUT.H, "head_dim": RELAYOUT.D,
+                         "world": world if world > 1 else RELAYOUT.W,
+                         "segments": RELAYOUT.n_segs, "window_bytes": WINDOW,
+                         "chunking": "one batch plane per launch"},
+            "reduce_scatter": {"tokens": REDUCE.T, "cols": REDUCE.C,
+                               "world": world if world > 1 else REDUCE.W,
+                               "partial_std": REDUCE.partial_std,
+                               "bias_std": REDUCE.bias_std},
+            "parallelism": parallelism,
+            "l2": "no flush: every kernel's inputs (7.2-15 GB) exceed the 126 MB L2",
+            "bytes_per_step": step_bytes(world)}
+
+
 def load_peak():
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     try:
@@ -765,30 +799,14 @@ def measure(args, make_step, rank, world, local, device, timer, n_events):
 
     result = None
     if rank == 0:
-        if world > 1:
-            parallelism = (f"one rank per GPU: W={world} ranks, tokens and heads split "
-                           f"by quotient/remainder, shares pulled over NVLink")
-        else:
-            parallelism = (f"one GPU: W={RELAYOUT.W} virtual ranks (relayout), "
-                           f"W={REDUCE.W} (reduce-scatter)")
+        config = step_config(world)
+        config["bytes_per_step"] = step.bytes_per_step  # the workload's, unless a test shrank it
         result = {
             "metric": METRIC, "value": round(value, 1), "unit": UNIT, "n_gpus": world,
             "steps": K, "warmup": args.warmup, "ms_per_step": round(t_max / K * 1e3, 4),
             "higher_is_better": True, "scaling": "strong" if world > 1 else "weak",
             "vs_baseline": None, "dtype": "bf16", "accumulate_dtype": "f32", "data": "synthetic",
-            "config": {"workload": WORKLOAD,
-                       "relayout": {"tokens": RELAYOUT.T, "planes": RELAYOUT.P,
-                                    "heads": RELAYOUT.H, "head_dim": RELAYOUT.D,
-                                    "world": world if world > 1 else RELAYOUT.W,
-                                    "segments": RELAYOUT.n_segs, "window_bytes": WINDOW,
-                                    "chunking": "one batch plane per launch"},
-                       "reduce_scatter": {"tokens": REDUCE.T, "cols": REDUCE.C,
-                                          "world": world if world > 1 else REDUCE.W,
-                                          "partial_std": REDUCE.partial_std,
-                                          "bias_std": REDUCE.bias_std},
-                       "parallelism": parallelism,
-                       "l2": "no flush: every kernel's inputs (7.2-15 GB) exceed the 126 MB L2",
-                       "bytes_per_step": step.bytes_per_step},
+            "config": config,
             "pct_of_peak": round(100.0 * value / world / peak, 2),
             "pct_of_nominal_peak": {"value": round(100.0 * value / world / NOMINAL_HBM_GBS, 2),
                                     "peak_gbs": NOMINAL_HBM_GBS,
@@ -977,10 +995,10 @@ def run_reference(args):
         "ms_per_step": round(t / args.steps * 1e3, 3), "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "accumulate_dtype": "f32",
         "data": "synthetic",
-        "config": {"workload": WORKLOAD, "relayout_tokens": RELAYOUT.T, "reduce_rows": REDUCE.T,
-                   "sample_tokens": each * cores, "sample_rows": sample_rows(each) * cores},
+        "config": step_config(world),
         "cpu_baseline": {"value": round(value, 3), "unit": UNIT, "cores": cores, "kind": "oracle",
-                         "sample": sample, "cpu_model": host_cpu_model()},
+                         "sample": sample, "cpu_model": host_cpu_model(),
+                         "sample_tokens": each * cores, "sample_rows": sample_rows(each) * cores},
         "e2e": {"value": round(value, 3), "unit": UNIT, "h2d_bytes_per_step": 0,
                 "d2h_bytes_per_step": 0},
         "gpu_launches": 0,

@@ -74,6 +74,23 @@ def test_reference_arm_prints_one_line():
     assert rec["e2e"]["h2d_bytes_per_step"] == 0 and rec["cpu_baseline"]["kind"] == "oracle"
     assert rec["cpu_baseline"]["cpu_model"] == bench.host_cpu_model()
     assert rec["metric"] == bench.METRIC
+    # the native arm's config, so that the two lines describe the same workload
+    assert rec["config"] == bench.step_config(1)
+    assert rec["config"]["bytes_per_step"] == 2 * 2 * 14_336_000_000 + 8_455_731_200
+
+
+def test_step_config_per_world():
+    """The config both arms print: one GPU with 4 (relayout) and 8
+    (reduce-scatter) virtual ranks, or N ranks, one per GPU, whose bytes count
+    every rank's read of the bias."""
+    one = bench.step_config(1)
+    assert one["relayout"]["world"] == 4 and one["reduce_scatter"]["world"] == 8
+    assert one["relayout"]["chunking"] == "one batch plane per launch"
+    for n in (2, 4, 8):
+        c = bench.step_config(n)
+        assert c["relayout"]["world"] == n and c["reduce_scatter"]["world"] == n
+        assert c["bytes_per_step"] == (2 * 2 * 14_336_000_000 + (n + 1) * 65536 * 7168 * 2
+                                       + n * 7168 * 2)
 
 
 def test_reference_arm_other_ranks_exit_quietly():

@@ -31,6 +31,7 @@ def test_native_line():
     assert d["dtype"] == "bf16" and d["accumulate_dtype"] == "f32" and d["data"] == "synthetic"
     assert d["config"]["workload"] == bench.WORKLOAD == \
         "qkvg_T250000_W4_chunked+reduce_scatter_T65536_C7168_W8"
+    assert d["config"] == bench.step_config(1)  # the reference arm's config too
     assert d["config"]["relayout"]["window_bytes"] == 896_000_000
     assert d["config"]["bytes_per_step"] == 2 * 2 * 14_336_000_000 + 8_455_731_200
     assert d["value"] > 1000.0
@@ -75,6 +76,9 @@ def test_native_line():
 def test_reference_line():
     d = _run(["--impl", "reference", "--steps", "2", "--warmup", "3", "--reference-budget", "4"])
     assert d["impl"] == "reference" and d["unit"] == "GB/s" and d["value"] > 0
+    assert d["config"] == bench.step_config(1)  # the native arm's config
+    assert d["metric"] == bench.METRIC and d["higher_is_better"] is True
+    assert d["cpu_baseline"]["sample_tokens"] > 0 and d["cpu_baseline"]["sample_rows"] > 0
     assert d["cpu_baseline"]["kind"] == "oracle" and d["cpu_baseline"]["value"] == d["value"]
     assert d["e2e"]["h2d_bytes_per_step"] == 0 and d["e2e"]["value"] == d["value"]
 
