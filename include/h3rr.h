@@ -100,7 +100,8 @@ typedef enum h3_status {
 
 typedef struct h3_exec_info {
     int32_t launches;            /* kernel launches enqueued by the call */
-    int32_t chunks;              /* chunks: 1 unchunked, P * (token chunks per plane) in chunked mode */
+    int32_t chunks;              /* chunks of the plan: 1 unchunked, P * (token chunks per plane) one
+                                    plane per launch, the token ranges with H3_LAUNCH_CHUNK_TOKENS */
     int32_t grid;                /* CTAs per launch */
     int32_t block;               /* threads per CTA */
     int32_t variant;             /* H3_VARIANT_* */
