@@ -497,6 +497,37 @@ def test_full_qkvg_250k_w4_token_ranges(oracle_lib):
     torch.cuda.empty_cache()
 
 
+def test_full_qkvg_250k_w4_bulk_kernels_and_both_cuts():
+    """At the long-sequence size, the TMA bulk kernels give the vector
+    kernels' bytes under both cuts of the pages' window (one plane per launch
+    and token ranges of every plane), in both directions; the vector result
+    is itself checked against the oracle in the tests above."""
+    w = wl.QKVG_250K_W4_CHUNKED
+    full = wl.packed_operand(w, device=DEV)
+    part = rr.partition(w.T, w.H, w.W)
+    send = rr.split_rows(full, part.token_starts)
+    ref = rr.alloc_head_side(w.T, w.P, w.H, w.D, w.W, DEV)
+    rr.seq_to_head(send, ref, window_bytes=w.window_bytes)
+    got = rr.alloc_head_side(w.T, w.P, w.H, w.D, w.W, DEV)
+    back_full, back = rr.alloc_seq_side(w.T, w.P, w.H, w.D, w.W, DEV)
+    rr.bulk_wait_timeouts(reset=True)
+    for tok in (False, True):
+        for h in got:
+            h.zero_()
+        info = rr.seq_to_head(send, got, window_bytes=w.window_bytes, variant=rr.H3_VARIANT_BULK,
+                              token_chunks=tok)
+        assert info["variant"] == rr.H3_VARIANT_BULK and info["launches"] == 4
+        for j in range(w.W):
+            assert gu.same_bits(got[j], ref[j]), (tok, j)
+        back_full.zero_()
+        rr.head_to_seq(ref, back, window_bytes=w.window_bytes, variant=rr.H3_VARIANT_BULK,
+                       token_chunks=tok)
+        assert gu.same_bits(back_full, full), tok
+    assert rr.bulk_wait_timeouts() == 0
+    del full, send, ref, got, back_full, back
+    torch.cuda.empty_cache()
+
+
 def test_full_qkvg_250k_w2_sub_plane(oracle_lib):
     """The long-sequence operand over 2 ranks: one plane of one rank is
     1,792,000,000 bytes, twice the 896,000,000-byte window, so every plane
