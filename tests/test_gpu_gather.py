@@ -117,9 +117,16 @@ def test_reduce_scatter_then_all_gather_is_unsharded_gemm():
 
 
 def test_full_all_gather_64k_w8():
+    """Every output equals the full [65536, 7168] rows, with the register
+    kernel and with the bulk (TMA) kernel."""
     T, C, W = 65536, 7168, 8
     full, blocks = _blocks(T, C, W, 4)
     outs = [torch.empty((T, C), dtype=torch.bfloat16, device=DEV) for _ in range(W)]
-    rr.ragged_all_gather(blocks, outs)
-    for o in outs:
-        assert gu.same_bits(o, full)
+    rr.bulk_wait_timeouts(reset=True)
+    for variant in (0, rr.H3_VARIANT_BULK):
+        for o in outs:
+            o.zero_()
+        rr.ragged_all_gather(blocks, outs, variant=variant)
+        for o in outs:
+            assert gu.same_bits(o, full), variant
+    assert rr.bulk_wait_timeouts() == 0
