@@ -31,8 +31,11 @@ def _inputs(T, C, W, S, seed, bits=False):
                                      (97, 2048, 8, 5), (64, 64, 64, 1), (90, 512, 9, 7),
                                      (300, 1024, 5, 256)])
 @pytest.mark.parametrize("in_place", [False, True])
-def test_gated_matches_oracle(oracle_lib, T, C, W, S, in_place):
+@pytest.mark.parametrize("with_bias", [True, False])
+def test_gated_matches_oracle(oracle_lib, T, C, W, S, in_place, with_bias):
     partials, bias, gate, bounds, x_full, x = _inputs(T, C, W, S, T + W + S)
+    if not with_bias:
+        bias = None  # the bias is optional, as in the plain reduce-scatter
     x_bits = [gu.bits(v) for v in x]
     if in_place:
         out = x
@@ -41,7 +44,8 @@ def test_gated_matches_oracle(oracle_lib, T, C, W, S, in_place):
         out_full, out = rr.alloc_reduce_outputs(T, C, W, DEV)
         info = rr.ragged_reduce_scatter_gated(partials, bias, gate, bounds, x, out)
     assert info["launches"] == 1
-    want = oracle_lib.reduce_scatter_gated([gu.bits(p) for p in partials], gu.bits(bias),
+    want = oracle_lib.reduce_scatter_gated([gu.bits(p) for p in partials],
+                                           gu.bits(bias) if with_bias else None,
                                            gu.bits(gate), bounds, x_bits, W)
     for r in range(W):
         assert np.array_equal(gu.bits(out[r]), want[r]), f"rank {r}"
