@@ -89,3 +89,32 @@ def test_row_calls_with_16_byte_aligned_buffers(oracle_lib):
         want_a = oracle_lib.ragged_all_gather([gu.bits(v) for v in out], W)
         for j in range(W):
             assert np.array_equal(gu.bits(outs[j]), want_a[j]), (variant, j)
+
+
+def test_rank_calls_with_16_byte_aligned_peer_buffers():
+    """One rank per GPU: a peer's buffer (here a local one standing in for it)
+    at 16 modulo 32 bytes; each rank's share equals the one-GPU call's."""
+    T, P, H, D, W = 300, 3, 56, 128, 4
+    part = rr.partition(T, H, W)
+    full = wl.random_bits((T, P, H, D), 91, DEV)
+    send = [t.clone() for t in rr.split_rows(full, part.token_starts)]
+    send[2] = _off16(send[2])
+    ref = rr.alloc_head_side(T, P, H, D, W, DEV)
+    rr.seq_to_head(send, ref)
+    ref[1] = _off16(ref[1])
+    for k in range(W):
+        mine = torch.empty_like(ref[k])
+        rr.seq_to_head_rank(send, mine, k, n_heads=H)
+        assert gu.same_bits(mine, ref[k]), k
+        rows = torch.empty_like(send[k])
+        rr.head_to_seq_rank(ref, rows, k, n_tokens=T)
+        assert gu.same_bits(rows, send[k]), k
+    C = 2048
+    parts = [wl.normal_bf16((T, C), 92 + r, 0.5, DEV) for r in range(W)]
+    parts[3] = _off16(parts[3])
+    red = rr.alloc_reduce_outputs(T, C, W, DEV)[1]
+    rr.ragged_reduce_scatter(parts, None, red)
+    for k in range(W):
+        mine = torch.empty_like(red[k])
+        rr.ragged_reduce_scatter_rank(parts, None, mine, k, n_tokens=T)
+        assert gu.same_bits(mine, red[k]), k
