@@ -118,3 +118,21 @@ def test_rank_calls_with_16_byte_aligned_peer_buffers():
         mine = torch.empty_like(red[k])
         rr.ragged_reduce_scatter_rank(parts, None, mine, k, n_tokens=T)
         assert gu.same_bits(mine, red[k]), k
+
+
+def test_staged_relayouts_with_a_16_byte_aligned_window(oracle_lib):
+    """The staged calls through a window buffer at 16 modulo 32 bytes (its
+    kernels fall back to 16-byte vectors) equal the oracle."""
+    T, P, H, D, W = 300, 3, 56, 128, 4
+    part = rr.partition(T, H, W)
+    full = wl.random_bits((T, P, H, D), 95, DEV)
+    send = rr.split_rows(full, part.token_starts)
+    window = _off16(torch.zeros(37 * H * D * 2, dtype=torch.uint8, device=DEV))
+    heads = rr.alloc_head_side(T, P, H, D, W, DEV)
+    rr.seq_to_head_staged(send, heads, window)
+    want = oracle_lib.seq_to_head([gu.bits(s) for s in send], T, P, H, D, W)
+    for j in range(W):
+        assert np.array_equal(gu.bits(heads[j]), want[j]), j
+    back_full, back = rr.alloc_seq_side(T, P, H, D, W, DEV)
+    rr.head_to_seq_staged(heads, back, window)
+    assert gu.same_bits(back_full, full)
