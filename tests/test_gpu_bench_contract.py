@@ -63,6 +63,10 @@ def test_native_line():
     assert isinstance(k["reasons"], list)
     shares = sum(v["share"] for v in d["kernels"].values())
     assert abs(shares - 1.0) < 0.01
+    # the bar every kernel of the step must clear: 70 % of B200's ~8 TB/s,
+    # by algorithmic bytes over CUDA-event time at full size
+    for name, k in d["kernels"].items():
+        assert k["gbs"] >= 0.70 * 8000.0, (name, k["gbs"])
     # beside the line: the same window cut into token ranges of all planes
     c = d["chunk_shapes"]
     assert c["window_bytes"] == 896_000_000
