@@ -73,7 +73,8 @@ def test_native_line():
     r = c["token_ranges_all_planes"]
     assert r["round_trip_ok"] is True and r["tokens_per_launch"] == 15625
     for k in ("seq_to_head", "head_to_seq"):
-        assert r[k]["launches_per_call"] == 4 and r[k]["planes_per_launch"] == 4 and r[k]["gbs"] > 1000
+        assert r[k]["launches_per_call"] == 4 and r[k]["planes_per_launch"] == 4
+        assert r[k]["gbs"] >= 0.70 * 8000.0, (k, r[k]["gbs"])
         assert c["one_plane_per_launch"][k]["launches_per_call"] == 4
 
 
